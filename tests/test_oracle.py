@@ -1,0 +1,355 @@
+"""Pins for the float64 oracle against what the pages and the mathematics fix (CPU only).
+
+Each pin checks the oracle against something other than itself: a pure-Python loop version
+written from the definitions, a library routine (torch float64), a closed form, an exact
+integer computation, or an invariant stated on the pages:
+  GLM invariant and two-group form, masked linear, FM equation, closure equation
+  ("ROCS：面向请求的大规模推荐计算共享" review, §2.1); grouped cross-attention (§2.2);
+  Y_i^C = Z_{m_i} + W_CC X_i^C (§2.4); amortised cost (§2.3).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import rocs_oracle as O
+from oracle import tiny
+
+pytestmark = pytest.mark.filterwarnings("ignore::DeprecationWarning")
+
+
+# ---------------------------------------------------------------------------------------------
+# a0 segment bookkeeping
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("counts", [[3, 0, 5, 1], [64] * 4, [0, 0, 0], [1], [0, 7, 0]])
+def test_segments_definition(counts):
+    counts = np.asarray(counts, np.int32)
+    offsets, m = O.segments(counts)
+    assert offsets[0] == 0 and offsets[-1] == counts.sum() == len(m)
+    # brute force: request r owns exactly the candidate slots between its offsets
+    for r in range(len(counts)):
+        owned = [c for c in range(len(m)) if m[c] == r]
+        assert owned == list(range(offsets[r], offsets[r + 1]))
+        assert len(owned) == counts[r]
+    assert np.all(np.diff(m) >= 0)
+
+
+def test_segments_config_counts():
+    c3 = synth.model_cfg3().counts
+    assert c3.min() >= 100 and c3.max() <= 1000 and len(c3) == 64
+    c5 = synth.model_cfg5().counts
+    assert c5.min() >= 16 and c5.max() <= 2000 and len(c5) == 512
+    assert 200 <= np.median(c5) <= 400
+    off, m = O.segments(c5)
+    assert off[-1] == c5.sum() and np.bincount(m, minlength=512).tolist() == c5.tolist()
+
+
+# ---------------------------------------------------------------------------------------------
+# A3 GLM linear
+# ---------------------------------------------------------------------------------------------
+def _tiny_linear_case(seed=3, B_R=3, counts=(2, 0, 3), dRi=5, dCi=4, dRo=3, dCo=6, integer=None):
+    rng = np.random.default_rng(seed)
+    def a(*s):
+        if integer:
+            return rng.integers(-integer, integer + 1, size=s).astype(np.float64)
+        return rng.standard_normal(s)
+    counts = np.asarray(counts)
+    _, m = O.segments(counts)
+    return dict(X_R=a(B_R, dRi), X_C=a(len(m), dCi), m=m, W_RR=a(dRo, dRi), W_CR=a(dCo, dRi),
+                W_CC=a(dCo, dCi), b_R=a(dRo), b_C=a(dCo))
+
+
+def test_linear_matches_loop_version():
+    p = _tiny_linear_case()
+    YR, YC = O.glm_linear(p["X_R"], p["X_C"], p["m"], p["W_RR"], p["W_CR"], p["W_CC"], p["b_R"], p["b_C"])
+    tR, tC = tiny.linear_two_group(p["X_R"].tolist(), p["X_C"].tolist(), p["m"].tolist(), p["W_RR"].tolist(),
+                                   p["W_CR"].tolist(), p["W_CC"].tolist(), p["b_R"].tolist(), p["b_C"].tolist())
+    np.testing.assert_allclose(YR, np.array(tR), rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(YC, np.array(tC), rtol=1e-13, atol=1e-13)
+
+
+def test_linear_integer_inputs_exact_three_ways():
+    """Small integers: dense masked, IKBO-decomposed and the loop version agree bit for bit."""
+    p = _tiny_linear_case(seed=5, B_R=4, counts=(3, 1, 0, 4), dRi=16, dCi=8, dRo=8, dCo=12, integer=7)
+    args = (p["X_R"], p["X_C"], p["m"], p["W_RR"], p["W_CR"], p["W_CC"], p["b_R"], p["b_C"])
+    YR, YC = O.glm_linear(*args)
+    dR, dC = O.glm_linear_decomposed(*args)
+    tR, tC = tiny.linear_two_group(*[np.asarray(x).tolist() for x in args])
+    assert np.array_equal(YR, dR) and np.array_equal(YC, dC)
+    assert np.array_equal(YR, np.array(tR)) and np.array_equal(YC, np.array(tC))
+
+
+def test_linear_dense_equals_ikbo_closed_form_cfg1():
+    case = synth.linear_cfg1()
+    x = synth.linear_inputs(case)
+    _, m = O.segments(case.counts)
+    args = (x["X_R"], x["X_C"], m, x["W_RR"], x["W_CR"], x["W_CC"], x["b_R"], x["b_C"])
+    YR, YC = O.glm_linear(*args)
+    dR, dC = O.glm_linear_decomposed(*args)
+    np.testing.assert_allclose(YR, dR, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(YC, dC, rtol=1e-13, atol=1e-13)
+    # the closed form of each output also matches torch float64 linear on the concatenation
+    Xd = torch.tensor(np.concatenate([x["X_R"][m], x["X_C"]], 1), dtype=torch.float64)
+    Wd = torch.tensor(np.concatenate([x["W_CR"], x["W_CC"]], 1), dtype=torch.float64)
+    ref = torch.nn.functional.linear(Xd, Wd, torch.tensor(x["b_C"], dtype=torch.float64)).numpy()
+    np.testing.assert_allclose(YC, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_linear_glm_invariant():
+    """Perturbing every candidate input leaves every request output value-equal ([REV] §2.1)."""
+    p = _tiny_linear_case(seed=9, B_R=3, counts=(4, 2, 5), dRi=32, dCi=16, dRo=24, dCo=8)
+    YR, YC = O.glm_linear(p["X_R"], p["X_C"], p["m"], p["W_RR"], p["W_CR"], p["W_CC"], p["b_R"], p["b_C"], "relu")
+    XC2 = p["X_C"] + np.random.default_rng(1).standard_normal(p["X_C"].shape) * 10
+    YR2, YC2 = O.glm_linear(p["X_R"], XC2, p["m"], p["W_RR"], p["W_CR"], p["W_CC"], p["b_R"], p["b_C"], "relu")
+    assert np.array_equal(YR, YR2)
+    assert not np.allclose(YC, YC2)
+
+
+def test_linear_row_independence():
+    p = _tiny_linear_case(seed=11, B_R=2, counts=(4, 3), dRi=8, dCi=8, dRo=4, dCo=4)
+    args = [p["X_R"], p["X_C"].copy(), p["m"], p["W_RR"], p["W_CR"], p["W_CC"], p["b_R"], p["b_C"]]
+    _, YC = O.glm_linear(*args)
+    args[1][2] += 5.0
+    _, YC2 = O.glm_linear(*args)
+    keep = np.arange(len(YC)) != 2
+    assert np.array_equal(YC[keep], YC2[keep]) and not np.allclose(YC[2], YC2[2])
+
+
+def test_linear_special_cases():
+    """W_CC = 0, b^C = 0: each candidate output is its request's W_CR X^R (the broadcast);
+    W_CR = 0: candidate outputs ignore the request (plain per-candidate linear)."""
+    p = _tiny_linear_case(seed=13)
+    zc = np.zeros_like(p["W_CC"])
+    _, YC = O.glm_linear(p["X_R"], p["X_C"], p["m"], p["W_RR"], p["W_CR"], zc, p["b_R"], 0 * p["b_C"])
+    np.testing.assert_allclose(YC, (p["X_R"] @ p["W_CR"].T)[p["m"]], rtol=1e-14, atol=1e-14)
+    _, YC = O.glm_linear(p["X_R"], p["X_C"], p["m"], p["W_RR"], 0 * p["W_CR"], p["W_CC"], p["b_R"], p["b_C"])
+    np.testing.assert_allclose(YC, p["X_C"] @ p["W_CC"].T + p["b_C"], rtol=1e-14, atol=1e-14)
+
+
+def test_masked_weight_has_zero_upper_right_block():
+    W = O.masked_weight(np.ones((2, 3)), 2 * np.ones((4, 3)), 3 * np.ones((4, 5)))
+    assert W.shape == (6, 8)
+    assert np.all(W[:2, 3:] == 0) and np.all(W[:2, :3] == 1) and np.all(W[2:, :3] == 2) and np.all(W[2:, 3:] == 3)
+
+
+# ---------------------------------------------------------------------------------------------
+# activations / LayerNorm (library routines as the reference)
+# ---------------------------------------------------------------------------------------------
+def test_activations_match_torch():
+    x = np.linspace(-8, 8, 1001)
+    t = torch.tensor(x, dtype=torch.float64)
+    np.testing.assert_allclose(O.activation(x, "gelu"), torch.nn.functional.gelu(t).numpy(), rtol=1e-14, atol=1e-15)
+    np.testing.assert_allclose(O.activation(x, "sigmoid"), torch.sigmoid(t).numpy(), rtol=1e-14, atol=1e-16)
+    np.testing.assert_array_equal(O.activation(x, "relu"), torch.relu(t).numpy())
+
+
+def test_layernorm_pins():
+    rng = np.random.default_rng(0)
+    X = rng.standard_normal((5, 4096)) * 3 + 1
+    g = 1 + rng.uniform(-0.1, 0.1, 4096)
+    b = rng.uniform(-0.1, 0.1, 4096)
+    Y = O.group_layernorm(X, g, b)
+    ref = torch.nn.functional.layer_norm(torch.tensor(X), (4096,), torch.tensor(g), torch.tensor(b), 1e-5).numpy()
+    np.testing.assert_allclose(Y, ref, rtol=1e-12, atol=1e-12)
+    # constant row -> exactly the shift
+    Yc = O.group_layernorm(np.full((2, 64), 3.25), np.ones(64) * 2, b[:64])
+    assert np.array_equal(Yc, np.broadcast_to(b[:64], (2, 64)))
+    # without affine: zero mean and unit variance (up to eps)
+    Yn = O.group_layernorm(X, np.ones(4096), np.zeros(4096))
+    np.testing.assert_allclose(Yn.mean(-1), 0, atol=1e-12)
+    np.testing.assert_allclose(Yn.var(-1), X.var(-1) / (X.var(-1) + 1e-5), rtol=1e-12)
+    # the loop version
+    t = tiny.layernorm_row(X[0, :50].tolist(), g[:50].tolist(), b[:50].tolist())
+    np.testing.assert_allclose(O.group_layernorm(X[:1, :50], g[:50], b[:50])[0], t, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------------
+# A5 masked FM, token LCB
+# ---------------------------------------------------------------------------------------------
+def test_fm_matches_loops_and_masks():
+    rng = np.random.default_rng(2)
+    counts = np.array([2, 0, 3])
+    _, m = O.segments(counts)
+    ER = rng.standard_normal((3, 4, 6))
+    EC = rng.standard_normal((5, 2, 6))
+    FR, FC = O.fm_masked(ER, EC, m)
+    tR, tC = tiny.fm_masked(ER.tolist(), EC.tolist(), m.tolist())
+    np.testing.assert_allclose(FR, np.array(tR), rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(FC, np.array(tC), rtol=1e-13, atol=1e-13)
+    # request block symmetric, candidate-input columns of request rows zero in the dense gram
+    G = O.fm_gram_rows(ER[m], EC)
+    assert np.all(G[:, :4, 4:] == 0)
+    FRm = FR.reshape(3, 4, 4)
+    np.testing.assert_array_equal(FRm, FRm.transpose(0, 2, 1))
+    # candidate x request block is E^C E^R[m]^T (torch bmm reference)
+    ref = torch.bmm(torch.tensor(EC), torch.tensor(ER[m]).transpose(1, 2)).numpy()
+    np.testing.assert_allclose(FC.reshape(5, 2, 6)[:, :, :4], ref, rtol=1e-13, atol=1e-13)
+
+
+def test_fm_glm_invariant():
+    rng = np.random.default_rng(4)
+    _, m = O.segments(np.array([3, 2]))
+    ER = rng.standard_normal((2, 32, 16))
+    EC = rng.standard_normal((5, 16, 16))
+    FR, _ = O.fm_masked(ER, EC, m)
+    FR2, _ = O.fm_masked(ER, EC * 7 + 1, m)
+    assert np.array_equal(FR, FR2)
+
+
+def test_token_lcb_matches_loops():
+    rng = np.random.default_rng(6)
+    _, m = O.segments(np.array([1, 2]))
+    ER = rng.standard_normal((2, 3, 5))
+    EC = rng.standard_normal((3, 2, 5))
+    P_RR, P_CR, P_CC = rng.standard_normal((2, 3)), rng.standard_normal((4, 3)), rng.standard_normal((4, 2))
+    db = O.DenseBatch(m, 2)
+    LR, LC = O.token_lcb_rows(db.broadcast(ER), db.with_probe(EC), P_RR, P_CR, P_CC)
+    tR, tC = tiny.token_lcb(ER.tolist(), EC.tolist(), m.tolist(), P_RR.tolist(), P_CR.tolist(), P_CC.tolist())
+    np.testing.assert_allclose(db.request_out(LR), np.array(tR), rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(db.cand_out(LC), np.array(tC), rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------------------------
+# attention
+# ---------------------------------------------------------------------------------------------
+def test_attention_brute_force_and_library():
+    rng = np.random.default_rng(8)
+    B_R, L, d, H = 2, 5, 8, 2
+    K = rng.standard_normal((B_R, L, d))
+    V = rng.standard_normal((B_R, L, d))
+    owner = np.array([0, 1, 1])
+    Q = rng.standard_normal((3, d))
+    out = O.cross_attn(Q, K, V, owner, H)
+    for c in range(3):
+        t = tiny.attention_one_query(Q[c].tolist(), K[owner[c]].tolist(), V[owner[c]].tolist(), H)
+        np.testing.assert_allclose(out[c], t, rtol=1e-13, atol=1e-13)
+    # torch SDPA in float64 as a library reference
+    q = torch.tensor(Q).reshape(3, 1, H, d // H).transpose(1, 2)
+    k = torch.tensor(K[owner]).reshape(3, L, H, d // H).transpose(1, 2)
+    v = torch.tensor(V[owner]).reshape(3, L, H, d // H).transpose(1, 2)
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v).transpose(1, 2).reshape(3, d).numpy()
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_attention_special_cases():
+    rng = np.random.default_rng(10)
+    d, H = 8, 2
+    V = rng.standard_normal((1, 1, d))
+    K = rng.standard_normal((1, 1, d))
+    Q = rng.standard_normal((4, d))
+    out = O.cross_attn(Q, K, V, np.zeros(4, np.int64), H)
+    np.testing.assert_array_equal(out, np.broadcast_to(V[0, 0], (4, d)))   # L = 1
+    Ke = np.broadcast_to(rng.standard_normal(d), (1, 7, d)).copy()
+    V7 = rng.standard_normal((1, 7, d))
+    out = O.cross_attn(Q, Ke, V7, np.zeros(4, np.int64), H)                 # equal keys -> mean
+    np.testing.assert_allclose(out, np.broadcast_to(V7[0].mean(0), (4, d)), rtol=1e-13, atol=1e-13)
+    K3 = np.zeros((1, 3, d)); K3[0, 1] = 40.0
+    q = np.ones((1, d))
+    out = O.cross_attn(q, K3, V7[:, :3], np.zeros(1, np.int64), H)          # one dominant logit
+    np.testing.assert_allclose(out[0], V7[0, 1], rtol=1e-12, atol=1e-12)
+
+
+def test_encoder_layer_matches_torch_mha():
+    rng = np.random.default_rng(12)
+    B, L, d, H = 2, 7, 16, 4
+    S = rng.standard_normal((B, L, d))
+    Wq, Wk, Wv, Wo = (rng.standard_normal((d, d)) / 4 for _ in range(4))
+    g, b = 1 + rng.uniform(-0.1, 0.1, d), rng.uniform(-0.1, 0.1, d)
+    out = O.encoder_layer(S, Wq, Wk, Wv, Wo, g, b, H)
+    mha = torch.nn.MultiheadAttention(d, H, bias=False, batch_first=True, dtype=torch.float64)
+    with torch.no_grad():
+        mha.in_proj_weight.copy_(torch.tensor(np.concatenate([Wq, Wk, Wv], 0)))
+        mha.out_proj.weight.copy_(torch.tensor(Wo))
+        St = torch.tensor(S)
+        a, _ = mha(St, St, St, need_weights=False)
+        ref = torch.nn.functional.layer_norm(St + a, (d,), torch.tensor(g), torch.tensor(b), 1e-5).numpy()
+    np.testing.assert_allclose(out, ref, rtol=1e-11, atol=1e-11)
+
+
+# ---------------------------------------------------------------------------------------------
+# composition closure and invariants on the model configs (reduced sizes)
+# ---------------------------------------------------------------------------------------------
+def _small_cfg3():
+    case = synth.model_cfg3(B_R=3, counts=[4, 0, 3])
+    return case, synth.model_weights(case), synth.model_inputs(case)
+
+
+def test_glm_stack_closure_and_invariant():
+    case, W, x = _small_cfg3()
+    _, m = O.segments(case.counts)
+    out = O.forward_cfg3(case, x, W, m)            # asserts request copies agree per layer
+    x2 = dict(x)
+    x2["E_C"] = x["E_C"] + np.random.default_rng(0).standard_normal(x["E_C"].shape).astype(np.float32)
+    out2 = O.forward_cfg3(case, x2, W, m)
+    for (r1, _), (r2, _) in zip(out["layers"], out2["layers"]):
+        assert np.array_equal(r1, r2)
+    assert not np.allclose(out["E_C"], out2["E_C"])
+    # row independence through 3 layers
+    x3 = dict(x)
+    x3["E_C"] = x["E_C"].copy()
+    x3["E_C"][1] += 1.0
+    out3 = O.forward_cfg3(case, x3, W, m)
+    keep = np.arange(case.B_C) != 1
+    assert np.array_equal(out["E_C"][keep], out3["E_C"][keep])
+
+
+def test_glm_stack_sampled_equals_full():
+    """Evaluating a subset of candidates gives the same rows as the full evaluation."""
+    case, W, x = _small_cfg3()
+    _, m = O.segments(case.counts)
+    full = O.forward_cfg3(case, x, W, m)
+    rows = np.array([0, 3, 6])
+    xs = dict(x)
+    xs["E_C"] = synth.model_inputs(case, cand_rows=rows)["E_C"]
+    sub = O.forward_cfg3(case, xs, W, m[rows])
+    np.testing.assert_array_equal(xs["E_C"], x["E_C"][rows])
+    np.testing.assert_allclose(sub["E_C"], full["E_C"][rows], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(sub["E_R"], full["E_R"], rtol=1e-12, atol=1e-12)
+
+
+def test_dca_cfg4_invariants_small():
+    case = synth.model_cfg4(B_R=2, counts=[3, 2])
+    case.dca.L = 12
+    W = synth.model_weights(case)
+    x = synth.model_inputs(case)
+    _, m = O.segments(case.counts)
+    out = O.forward_cfg4(case, x, W, m)
+    x2 = dict(x)
+    x2["Y_C"] = x["Y_C"] * -3 + 1
+    out2 = O.forward_cfg4(case, x2, W, m)
+    for a, b in zip(out["A_R"], out2["A_R"]):
+        assert np.array_equal(a, b)
+    for a, b in zip(out["S"], out2["S"]):
+        assert np.array_equal(a, b)
+    assert not np.allclose(out["A_C"][1], out2["A_C"][1])
+
+
+def test_cfg5_small_runs_and_is_glm():
+    case = synth.model_cfg5(B_R=2, counts=[2, 3], L=8)
+    W = synth.model_weights(case)
+    x = synth.model_inputs(case)
+    _, m = O.segments(case.counts)
+    out = O.forward_cfg5(case, x, W, m)
+    assert out["score"].shape == (5,) and np.all((out["score"] > 0) & (out["score"] < 1))
+    x2 = dict(x)
+    x2["E_C"] = x["E_C"] * 0.5
+    out2 = O.forward_cfg5(case, x2, W, m)
+    for a, b in zip(out["A_R"], out2["A_R"]):
+        assert np.array_equal(a, b)
+    assert np.array_equal(out["E_R"], out2["E_R"])
+
+
+def test_amortised_cost():
+    assert O.amortised_cost(2.0, 100.0, 100) == 3.0
+    assert O.amortised_cost(2.0, 100.0, 1) == 102.0
+
+
+def test_bf16_rounding_of_inputs():
+    x = np.array([1.0, 1.00390625, 1.005859375, -2.0e-3, 3.0e38], np.float32)
+    r = synth.bf16_round(x)
+    t = torch.tensor(x).to(torch.bfloat16).to(torch.float32).numpy()
+    np.testing.assert_array_equal(r, t)
+    big = np.random.default_rng(0).standard_normal(100000).astype(np.float32)
+    np.testing.assert_array_equal(synth.bf16_round(big), torch.tensor(big).to(torch.bfloat16).float().numpy())
