@@ -104,7 +104,7 @@ class DenseBatch:
     def check_request_copies(self, R_rows: np.ndarray, what: str, rtol: float = 0.0) -> None:
         """Closure property ([REV] §2.1): every candidate's copy of the request outputs equals
         the request's own output F^R(X^R).  rtol=0 demands value equality."""
-        if self.n == 0:
+        if self.n == 0 or R_rows.size == 0:
             return
         cand = R_rows[:self.n]
         ref = R_rows[self.n:][self.m]
