@@ -1,0 +1,497 @@
+#!/usr/bin/env python
+"""Throughput of the ROCS forward hot path on B200 (librocs), one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl librocs|reference]
+
+A step is one rocs_forward over one batch of synthetic requests (default workload: the
+end-to-end ranking forward -- Wukong-style GLM stack, DCA with L=1024 histories, scoring head --
+over 512 requests with lognormal candidate counts).  `value` is candidates scored per second
+with inputs resident in HBM (device-timed with CUDA events, max over ranks); `e2e` repeats the
+measurement through the same C-ABI call with the inputs copied from pinned host memory and the
+scores copied back inside the timed region.  With N > 1 (torchrun) every rank runs its own shard
+of requests (weak scaling, no collective on the data path).
+
+--impl reference times the float64 oracle (the reference arm of this build) on bounded samples
+of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "candidates/sec per B200 for ROCS forward; % of HBM or bf16 tensor roofline"
+FP32_KEYS = ("b_R", "b_C", ".b", "gamma", "beta")
+
+
+# ---------------------------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------------------------
+WORKLOADS = {
+    "rocs_forward_e2e": "end-to-end ranking forward: GLM stack (3 layers, 32|16 embeddings of 128) + DCA "
+                        "(L=1024, d=256, 8 heads, 3 depths) + scoring MLP 512-256-1; 512 requests, "
+                        "candidates ~ clipped lognormal (median 300, 16..2000), seed 1",
+    "glm_stack": "Wukong-style GLM stack, 3 layers; 64 requests, candidates ~ U[100,1000], seed 0",
+    "dca": "DCA path: L=200, d=256, 4 heads, 2 layers; 32 requests x 500 candidates, seed 0",
+}
+
+
+def make_case(name: str, rank: int):
+    seed_shift = 1000 * rank
+    if name == "rocs_forward_e2e":
+        return synth.model_cfg5(seed=1 + seed_shift)
+    if name == "glm_stack":
+        return synth.model_cfg3(seed=0 + seed_shift)
+    if name == "dca":
+        return synth.model_cfg4(seed=0 + seed_shift)
+    raise SystemExit(f"unknown workload {name}")
+
+
+# ---------------------------------------------------------------------------------------------
+# algorithmic work per launch (for the roofline of the dominant kernel)
+# ---------------------------------------------------------------------------------------------
+def algo_work(case, label: str):
+    """(bound, amount per launch, unit) for a timing-report label "<site>:<kernel>", or None.
+    GEMMs: mathematical flops 2*M*N*K (a split hi/lo operand counts once).  Bandwidth-bound
+    kernels: compulsory bytes of the tensors they read and write, in their stored precision.
+    Attention: exp2 evaluations (one per score), the MUFU-bound quantity."""
+    B_R, B_C = case.B_R, case.B_C
+    g, a = case.glm, case.dca
+    site, _, kern = label.partition(":")
+    if g is not None:
+        fR, fC = g.n_R * g.n_R, g.n_C * (g.n_R + g.n_C)
+        wr, wc = g.n_R * g.D, g.n_C * g.D
+        oRw, oCw = g.fm_out_R * g.D, g.fm_out_C * g.D
+        lRw, lCw = g.lcb_out_R * g.D, g.lcb_out_C * g.D
+        table = {
+            "glm.mlp1.cand:gemm_tc": ("tensor", 2.0 * B_C * g.hidden * fC),
+            "glm.mlp1.req:gemm_tc": ("tensor", 2.0 * B_R * g.hidden * fR * 2),
+            "glm.mlp2.cand:gemm_tc": ("tensor", 2.0 * B_C * oCw * g.hidden),
+            "glm.mlp2.req:gemm_tc": ("tensor", 2.0 * B_R * (oRw + oCw) * g.hidden),
+            "glm.fm:fm_cand": ("hbm", B_C * (wc * 4 + fC * 4)),
+            "glm.lcb:lcb_cand": ("hbm", B_C * (wc * 4 + lCw * 4)),
+            "glm.lnC:layernorm": ("hbm", B_C * (oCw * 4 + lCw * 4 + wc * 4 + wc * 4)),
+        }
+        if label in table:
+            return table[label]
+    if a is not None:
+        L, d, H = a.L, a.d, a.H
+        table = {
+            "enc.attn:attn": ("alu", float(B_R) * H * L * L),
+            "xattn.cand:attn": ("alu", float(B_C) * H * L),
+            "enc.qkv:gemm_tc": ("tensor", 2.0 * B_R * L * d * d * 3),
+            "enc.kv:gemm_tc": ("tensor", 2.0 * B_R * L * d * d * 4),
+            "enc.wo:gemm_tc": ("tensor", 2.0 * B_R * L * d * d),
+            "enc.ln:layernorm": ("hbm", B_R * L * d * 2 * 3.0),
+        }
+        if label in table:
+            return table[label]
+    if case.scoring is not None:
+        h1, h2 = case.scoring
+        xc = g.n_C * g.D + a.layers * a.d
+        table = {"score.l1.cand:gemm_tc": ("tensor", 2.0 * B_C * h1 * xc),
+                 "score.l2:gemm_tc": ("tensor", 2.0 * B_C * h2 * h1)}
+        if label in table:
+            return table[label]
+    return None
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return dict(hbm=float(j["hbm_gbs"]), tensor=float(j["bf16_tflops"]),
+                    tensor_sustained=float(j["bf16_tflops_sustained"]), sm_mhz=float(j.get("sm_max_mhz", 1965.0)),
+                    source="measured")
+    return dict(hbm=6650.0, tensor=1590.0, tensor_sustained=1400.0, sm_mhz=1965.0, source="fallback")
+
+
+def roofline_entry(case, label, launches, total_ms, peaks, sustained: bool):
+    w = algo_work(case, label)
+    if w is None or launches == 0:
+        return None
+    bound, amount = w
+    per_launch_s = total_ms / launches / 1e3
+    if bound == "tensor":
+        achieved = amount / per_launch_s / 1e12
+        peak = peaks["tensor_sustained"] if sustained else peaks["tensor"]
+        unit = "TFLOP/s"
+    elif bound == "hbm":
+        achieved = amount / per_launch_s / 1e9
+        peak = peaks["hbm"]
+        unit = "GB/s"
+    else:
+        # MUFU ex2: 16 per clock per SM (4 per SM sub-partition) x 148 SMs at the max SM clock
+        achieved = amount / per_launch_s / 1e9
+        peak = 16 * 148 * peaks["sm_mhz"] * 1e6 / 1e9
+        unit = "Gexp2/s"
+    return {"kernel": label, "bound": bound, "achieved": round(achieved, 3), "peak": round(peak, 1), "unit": unit,
+            "frac": round(achieved / peak, 4), "per_launch_ms": round(total_ms / launches, 4), "launches": launches,
+            "peak_source": f"{peaks['source']}{' sustained' if sustained and bound == 'tensor' else ''}"}
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = float(rows[0][2]) if rows[0][2].strip().replace(".", "").isdigit() else None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 5 + i and "Active" in r[5 + i]
+                          and "Not" not in r[5 + i]})
+        under = sorted(sm)[len(sm) // 2:] if sm else []
+        return {"sm_mhz": statistics.median(under) if under else None, "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------------------------
+# oracle timing (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------------------------
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_requests(case, req_ids):
+    """Runs the oracle on whole requests `req_ids` of the workload; returns candidates processed."""
+    from oracle import rocs_oracle as O
+    counts = np.asarray(case.counts)
+    offsets = np.concatenate([[0], np.cumsum(counts)])
+    req_ids = np.asarray(req_ids, np.int64)
+    cand_rows = np.concatenate([np.arange(offsets[r], offsets[r + 1]) for r in req_ids]) if len(req_ids) else \
+        np.zeros(0, np.int64)
+    sub = dataclasses.replace(case, counts=counts[req_ids])
+    x = synth.model_inputs(case, cand_rows=cand_rows, req_rows=req_ids)
+    W = synth.model_weights(case)
+    _, m = O.segments(sub.counts)
+    if case.scoring is not None:
+        O.forward_cfg5(sub, x, W, m)
+    elif case.dca is not None:
+        O.forward_cfg4(sub, x, W, m)
+    else:
+        O.forward_cfg3(sub, x, W, m)
+    return int(counts[req_ids].sum())
+
+
+def oracle_rate(case, seconds: float, start_req: int = 0):
+    """Oracle candidates/s over whole requests taken in order until `seconds` of CPU time."""
+    t0 = time.perf_counter()
+    n = 0
+    r = start_req
+    reqs = 0
+    while time.perf_counter() - t0 < seconds and reqs < case.B_R:
+        n += oracle_requests(case, [r % case.B_R])
+        r += 1
+        reqs += 1
+    dt = time.perf_counter() - t0
+    return n / dt, n, reqs, dt
+
+
+# ---------------------------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------------------------
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    return rank, world, local
+
+
+def allreduce(x: float, op: str, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------------------------
+# librocs arm
+# ---------------------------------------------------------------------------------------------
+def run_librocs(args, rank, world, local):
+    import torch
+
+    from request_candidate_sharing_b200 import rocs
+    torch.cuda.set_device(local)
+    case = make_case(args.workload, rank)
+    dev = torch.device("cuda", local)
+    t_gen = time.perf_counter()
+    W = synth.model_weights(case)
+    x = synth.model_inputs(case)
+    gen_s = time.perf_counter() - t_gen
+
+    def to_dev(v, dt):
+        return torch.from_numpy(np.ascontiguousarray(v, np.float32)).to(dev).to(dt)
+
+    Wd = {k: to_dev(v, torch.float32 if k.endswith(FP32_KEYS) else torch.bfloat16) for k, v in W.items()}
+    xd = {k: to_dev(v, torch.bfloat16) for k, v in x.items()}
+    counts_d = torch.from_numpy(case.counts).to(dev)
+    g, a = case.glm, case.dca
+    R = rocs.Rocs(local)
+    md = rocs.model_desc(case)
+    mw = rocs.model_weights(Wd, g.layers if g else 0, a.layers if a else 0, case.scoring is not None)
+    B_C = case.B_C
+    score = torch.empty(max(B_C, 1), dtype=torch.float32, device=dev)
+    outE = None
+    if case.scoring is None:   # without a scoring head the final activations are the result
+        if g is not None:
+            outE = (torch.empty((case.B_R, g.n_R, g.D), dtype=torch.float32, device=dev),
+                    torch.empty((max(B_C, 1), g.n_C, g.D), dtype=torch.float32, device=dev))
+        else:
+            outE = (torch.empty((a.layers, case.B_R, a.d), dtype=torch.float32, device=dev),
+                    torch.empty((a.layers, max(B_C, 1), a.d), dtype=torch.float32, device=dev))
+    nb = R.rocs_forward_workspace(md)
+    ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+
+    def outputs():
+        if case.scoring is not None:
+            return rocs.Outputs(None, None, None, None, None, None, None, score.data_ptr())
+        if g is not None:
+            return rocs.Outputs(None, None, outE[0].data_ptr(), outE[1].data_ptr(), None, None, None, None)
+        return rocs.Outputs(None, None, None, None, None, outE[0].data_ptr(), outE[1].data_ptr(), None)
+
+    inp = rocs.Inputs(counts_d.data_ptr(), rocs.ptr(xd.get("E_R")), rocs.ptr(xd.get("E_C")), rocs.ptr(xd.get("H")),
+                      rocs.ptr(xd.get("Y_R")), rocs.ptr(xd.get("Y_C")))
+    out = outputs()
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+
+    def step():
+        R.rocs_forward(md, mw, inp, out, ws, nb, sh)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st = R.rocs_get_device_status(sh)
+    if st != 0:
+        raise RuntimeError(f"device status {rocs.STATUS_NAMES.get(st, st)} after warm-up")
+
+    # ---- device-timed region: inputs resident in HBM ----
+    uuid = str(getattr(torch.cuda.get_device_properties(dev), "uuid", "") or "")
+    clocks = ClockSampler(("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else (uuid or str(local)))
+    clocks.start()
+    time.sleep(0.3)
+    R.rocs_timing_start(200 * args.steps + 64)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = e0.elapsed_time(e1)
+    report = R.rocs_timing_stop()
+    clk = clocks.stop()
+    st = R.rocs_get_device_status(sh)
+    if st != 0:
+        raise RuntimeError(f"device status {rocs.STATUS_NAMES.get(st, st)} in the timed region")
+    ms_max = allreduce(ms, "max", world)
+    cands = allreduce(float(B_C) * args.steps, "sum", world)
+    value = cands / (ms_max / 1e3)
+
+    # ---- end-to-end through the same call with host buffers ----
+    host = {k: v.cpu().pin_memory() for k, v in xd.items()}
+    counts_h = counts_d.cpu().pin_memory()
+    score_h = torch.empty_like(score, device="cpu").pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values()) + counts_h.numel() * 4
+    res = score if case.scoring is not None else outE[1]
+    res_h = torch.empty_like(res, device="cpu").pin_memory()
+    d2h = res.numel() * res.element_size()
+
+    def e2e_step():
+        for k, v in host.items():
+            xd[k].copy_(v, non_blocking=True)
+        counts_d.copy_(counts_h, non_blocking=True)
+        step()
+        res_h.copy_(res, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e2e_ms = allreduce(f0.elapsed_time(f1), "max", world)
+    e2e_value = cands / (e2e_ms / 1e3)
+
+    # ---- per-kernel breakdown and the dominant kernel's roofline ----
+    peaks = load_peaks()
+    kernels = sorted(report.items(), key=lambda kv: -kv[1][1])
+    launches = sum(n for name, (n, _) in report.items() if name != "dropped")
+    total_k = sum(t for _, (_, t) in report.items())
+    rooflines = []
+    for name, (n, t) in kernels:
+        e = roofline_entry(case, name, n, t, peaks, sustained=True)
+        if e is not None:
+            e["share"] = round(t / total_k, 4) if total_k else None
+            rooflines.append(e)
+    top = rooflines[0] if rooflines else None
+    if top is not None:
+        traffic = None
+        tp = os.path.join(ROOT, "profiles", "traffic.json")
+        if os.path.exists(tp):
+            tj = json.load(open(tp)).get(args.workload, {}).get(top["kernel"])
+            if tj is not None:
+                traffic = tj
+        top = {"bound": top["bound"], "achieved": top["achieved"], "peak": top["peak"], "unit": top["unit"],
+               "frac": top["frac"], "traffic": traffic, "kernel": top["kernel"],
+               "per_launch_ms": top["per_launch_ms"], "peak_source": top["peak_source"] + " (of measured)"
+               if top["peak_source"].startswith("measured") else top["peak_source"]}
+
+    line = {"metric": METRIC, "value": round(value, 1), "unit": "candidates/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) inputs, N(0,1/fan_in) bf16 weights)",
+            "config": {"workload": args.workload, "description": WORKLOADS[args.workload], "B_R": case.B_R,
+                       "B_C_per_rank": B_C, "l2": "inputs larger than L2 (E_C alone is "
+                       f"{(xd['E_C'].numel() * 2 / 1e9) if 'E_C' in xd else 0:.2f} GB)",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": top,
+            "e2e": {"value": round(e2e_value, 1), "unit": "candidates/s", "h2d_bytes_per_step": int(h2d),
+                    "d2h_bytes_per_step": int(d2h)},
+            "gpu_launches": int(launches),
+            "clocks": clk,
+            "kernels": [{k: v for k, v in e.items() if k in ("kernel", "bound", "achieved", "unit", "frac", "share",
+                                                             "per_launch_ms", "launches")} for e in rooflines[:8]],
+            "kernel_ms": {name: round(t / args.steps, 4) for name, (n, t) in kernels[:16]},
+            "input_generation_s": round(gen_s, 1)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, n, reqs, dt = oracle_rate(case, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": round(rate, 2), "unit": "candidates/s", "cores": blas_threads(),
+                                "kind": "oracle",
+                                "sample": f"{reqs} whole requests ({n} candidates) of the same workload, "
+                                          f"{dt:.1f} s of float64 numpy on the host"}
+    R.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------------------------
+# reference arm: the float64 oracle on the host
+# ---------------------------------------------------------------------------------------------
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    case = make_case(args.workload, 0)
+    per_step = max(1.0, args.ref_step_seconds)
+    for i in range(args.warmup):
+        oracle_rate(case, per_step, start_req=i)
+    t = 0.0
+    n = 0
+    for i in range(args.steps):
+        rate, c, reqs, dt = oracle_rate(case, per_step, start_req=args.warmup + i)
+        t += dt
+        n += c
+    value = n / t
+    line = {"metric": METRIC, "value": round(value, 2), "unit": "candidates/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * t / args.steps, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": args.workload, "description": WORKLOADS[args.workload]},
+            "cpu_baseline": {"value": round(value, 2), "unit": "candidates/s", "cores": blas_threads(),
+                             "kind": "oracle",
+                             "sample": f"each step: whole requests of the workload for ~{per_step:.0f} s"},
+            "e2e": {"value": round(value, 2), "unit": "candidates/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="rocs_forward_e2e", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="librocs", choices=["librocs", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=4.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "librocs":
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        run_reference(args, rank, world)
+        return
+    rank, world, local = dist_setup(args.gpus)
+    run_librocs(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,361 @@
+// a4: block-masked factorization machine and token-axis linear compression (LCB).
+//
+// FM ([REV] §2.1 FM equation, Figure 2(c)): output group i interacts only with input groups
+// j <= i, so
+//   request:   F^R_r = E^R_r E^R_r^T                        (n_R x n_R, once per request)
+//   candidate: F^C_c = E^C_c [E^R_{m_c} ; E^C_c]^T          (n_C x (n_R + n_C))
+// The candidate kernel reads the request embeddings through the map m (no broadcast tensor):
+// one warp per candidate stages T = [E^R_{m_c} ; E^C_c] in shared memory (re-staging E^R only
+// when m changes along its run of consecutive candidates) and computes the products with
+// m16n8k16 tensor-core fragments.
+//
+// Token LCB ([REV] §2.1 masked linear along the embedding-count axis; IKBO split of §2.4):
+//   L^R_r = P_RR E^R_r,   Z^L_r = P_CR E^R_r   (request batch, fp32 Z^L in the workspace)
+//   L^C_c = Z^L_{m_c} + P_CC E^C_c              (candidate batch)
+#include "common.cuh"
+#include "internal.h"
+#include "mma_frag.cuh"
+
+namespace rocs {
+namespace {
+
+constexpr int FM_WARPS = 4;
+constexpr int FM_RUN = 8;   // consecutive candidates per warp
+
+__device__ __forceinline__ uint4 load8_as_bf16(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
+__device__ __forceinline__ uint4 load8_as_bf16(const float* p) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  return make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+}
+
+// rows x D (contiguous source rows, bf16 or fp32) -> bf16 shared rows of `pitch` bytes.
+template <typename TIN>
+__device__ __forceinline__ void stage_rows(uint8_t* dst, int pitch, const TIN* src, int rows, int D) {
+  const int lane = threadIdx.x & 31;
+  const int vpr = D / 8;
+  for (int i = lane; i < rows * vpr; i += 32) {
+    const int r = i / vpr, v = i - r * vpr;
+    *reinterpret_cast<uint4*>(dst + r * pitch + v * 16) = load8_as_bf16(src + (long long)r * D + v * 8);
+  }
+}
+
+__device__ __forceinline__ void zero_rows(uint8_t* dst, int pitch, int rows, int D) {
+  const int lane = threadIdx.x & 31;
+  const int vpr = D / 8;
+  for (int i = lane; i < rows * vpr; i += 32) {
+    const int r = i / vpr, v = i - r * vpr;
+    *reinterpret_cast<uint4*>(dst + r * pitch + v * 16) = make_uint4(0, 0, 0, 0);
+  }
+}
+
+__device__ __forceinline__ void store_bf16_pair(__nv_bfloat16* p, long long o, float a, float b, bool two) {
+  if (two && (o & 1) == 0) {
+    *reinterpret_cast<uint32_t*>(p) = pack_bf16x2(a, b);
+  } else {
+    p[0] = __float2bfloat16_rn(a);
+    if (two) p[1] = __float2bfloat16_rn(b);
+  }
+}
+
+// Writes one 16x8 fp32 C fragment (rows r0.., cols c0..) of a [rows_valid x cols_valid] output
+// with row stride ld.  out_mode 0: fp32; 1: bf16; 2: bf16 hi at offset o and bf16 lo = value - hi
+// at offset o + lo_off (fp32-precise activation for a following tensor-core GEMM).
+__device__ __forceinline__ void store_c_frag(void* out, int out_mode, long long base, int ld, int r0, int c0,
+                                             int rows_valid, int cols_valid, const float (&c)[4],
+                                             long long lo_off = 0) {
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int r = r0 + g + 8 * h;
+    const int col = c0 + 2 * t;
+    if (r >= rows_valid || col >= cols_valid) continue;
+    const long long o = base + (long long)r * ld + col;
+    const bool two = col + 1 < cols_valid;
+    if (out_mode == 1) {
+      store_bf16_pair(reinterpret_cast<__nv_bfloat16*>(out) + o, o, c[2 * h], c[2 * h + 1], two);
+    } else if (out_mode == 2) {
+      const float h0 = __bfloat162float(__float2bfloat16_rn(c[2 * h]));
+      const float h1 = __bfloat162float(__float2bfloat16_rn(c[2 * h + 1]));
+      __nv_bfloat16* p = reinterpret_cast<__nv_bfloat16*>(out);
+      store_bf16_pair(p + o, o, h0, h1, two);
+      store_bf16_pair(p + o + lo_off, o + lo_off, c[2 * h] - h0, c[2 * h + 1] - h1, two);
+    } else {
+      float* p = reinterpret_cast<float*>(out) + o;
+      if (col < cols_valid) p[0] = c[2 * h];
+      if (col + 1 < cols_valid) p[1] = c[2 * h + 1];
+    }
+  }
+}
+
+// Gram products of one staged tile: out[i][j] = sum_k T[a0 + i][k] T[j][k] for i < mrows,
+// j < ncols (ncols <= 64, multiple of 8 after padding; rows beyond the valid ones are zero).
+__device__ __forceinline__ void gram_tile(uint32_t sbase, int pitch, int a0, int mrows, int ncols, int D, void* out,
+                                          int out_mode, long long obase, int ld, long long lo_off) {
+  const int mt = (mrows + 15) / 16;
+  const int nt2 = (ncols + 15) / 16;   // pairs of 8-wide n-tiles
+  for (int mi = 0; mi < mt; ++mi) {
+    float acc[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    for (int k0 = 0; k0 < D; k0 += 16) {
+      uint32_t a[4];
+      load_a_frag(sbase, pitch, a0 + mi * 16, k0, a);
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        if (p < nt2) {
+          uint32_t b[4];
+          load_b_frag_nmajor_x2(sbase, pitch, p * 16, k0, b);
+          mma_bf16_16816(acc[2 * p], a, b[0], b[1]);
+          mma_bf16_16816(acc[2 * p + 1], a, b[2], b[3]);
+        }
+      }
+    }
+#pragma unroll
+    for (int p = 0; p < 8; ++p)
+      if (p * 8 < ncols) store_c_frag(out, out_mode, obase, ld, mi * 16, p * 8, mrows, ncols, acc[p], lo_off);
+  }
+}
+
+// Shared tile rows: n_R request rows, then n_C candidate rows, padded with zeros up to TROWS.
+// TROWS >= max(n_R + roundup16(n_C), roundup16(n_R + n_C), roundup16(n_R)).
+template <typename TIN>
+__global__ void __launch_bounds__(FM_WARPS * 32) fm_cand_kernel(const TIN* __restrict__ E_R, const TIN* __restrict__ E_C,
+                                                               const int32_t* __restrict__ req_idx, int B_R,
+                                                               long long B_C, int n_R, int n_C, int D, int trows,
+                                                               int pitch, void* F_C, int out_mode, int* status) {
+  extern __shared__ __align__(16) uint8_t fm_smem[];
+  const int warp = threadIdx.x >> 5;
+  uint8_t* T = fm_smem + warp * trows * pitch;
+  const uint32_t sbase = smem_u32(T);
+  const long long c_begin = ((long long)blockIdx.x * FM_WARPS + warp) * FM_RUN;
+  const int ncols = n_R + n_C;
+  int staged = -1;
+  // zero the padding rows once
+  zero_rows(T + (n_R + n_C) * pitch, pitch, trows - (n_R + n_C), D);
+  for (int i = 0; i < FM_RUN; ++i) {
+    const long long c = c_begin + i;
+    if (c >= B_C) break;
+    const int r = req_idx[c];
+    if (r < 0 || r >= B_R) {
+      if ((threadIdx.x & 31) == 0) set_status(status, ROCS_ERR_INDEX);
+      continue;
+    }
+    __syncwarp();
+    if (r != staged) {
+      stage_rows(T, pitch, E_R + (long long)r * n_R * D, n_R, D);
+      staged = r;
+    }
+    stage_rows(T + n_R * pitch, pitch, E_C + c * n_C * D, n_C, D);
+    __syncwarp();
+    const long long fsz = (long long)n_C * ncols;   // one candidate's F^C; split rows hold [hi | lo]
+    gram_tile(sbase, pitch, n_R, n_C, ncols, D, F_C, out_mode, c * fsz * (out_mode == 2 ? 2 : 1), ncols, fsz);
+  }
+}
+
+template <typename TIN>
+__global__ void __launch_bounds__(FM_WARPS * 32) fm_req_kernel(const TIN* __restrict__ E_R, int B_R, int n_R, int D,
+                                                              int trows, int pitch, void* F_R, int out_mode) {
+  extern __shared__ __align__(16) uint8_t fm_smem[];
+  const int warp = threadIdx.x >> 5;
+  const int r = blockIdx.x * FM_WARPS + warp;
+  if (r >= B_R) return;
+  uint8_t* T = fm_smem + warp * trows * pitch;
+  zero_rows(T + n_R * pitch, pitch, trows - n_R, D);
+  stage_rows(T, pitch, E_R + (long long)r * n_R * D, n_R, D);
+  __syncwarp();
+  const long long fsz = (long long)n_R * n_R;
+  gram_tile(smem_u32(T), pitch, 0, n_R, n_R, D, F_R, out_mode, r * fsz * (out_mode == 2 ? 2 : 1), n_R, fsz);
+}
+
+// ---------------------------------------------------------------------------------------------
+// token LCB (SIMT; P is tiny).  Inputs bf16 or fp32; out_mode 0 fp32, 1 bf16, 2 bf16 hi/lo pair
+// (the low half at +lo_off elements within the row).
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ float ld_f(const float* p) { return __ldg(p); }
+__device__ __forceinline__ float ld_f(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+
+__device__ __forceinline__ void store_val(void* out, long long off, float v, int out_mode, long long lo_off) {
+  if (out_mode == 0) {
+    reinterpret_cast<float*>(out)[off] = v;
+  } else {
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    reinterpret_cast<__nv_bfloat16*>(out)[off] = h;
+    if (out_mode == 2) reinterpret_cast<__nv_bfloat16*>(out)[off + lo_off] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
+}
+
+// Request side: one block per request, thread per (o, d).
+template <typename TIN>
+__global__ void lcb_req_kernel(const TIN* __restrict__ E_R, long long ld_ER, int n_R, int D,
+                               const __nv_bfloat16* __restrict__ P_RR, const __nv_bfloat16* __restrict__ P_CR,
+                               int o_R, int o_C, void* L_R, long long ld_LR, int out_mode, long long lo_off,
+                               float* __restrict__ ZL) {
+  const int r = blockIdx.x;
+  const TIN* e = E_R + (long long)r * ld_ER;
+  for (int i = threadIdx.x; i < (o_R + o_C) * D; i += blockDim.x) {
+    const int o = i / D, d = i - o * D;
+    const bool req = o < o_R;
+    const __nv_bfloat16* p = req ? P_RR + (long long)o * n_R : P_CR + (long long)(o - o_R) * n_R;
+    float acc = 0.f;
+    for (int t = 0; t < n_R; ++t) acc = fmaf(__bfloat162float(p[t]), ld_f(e + t * D + d), acc);
+    if (req) store_val(L_R, (long long)r * ld_LR + (long long)o * D + d, acc, out_mode, lo_off);
+    else ZL[((long long)r * o_C + (o - o_R)) * D + d] = acc;
+  }
+}
+
+// Candidate side: one warp per candidate; lane owns features d = lane + 32 j (j < DPL).
+constexpr int LCB_OMAX = 8;
+
+template <typename TIN, int DPL>
+__global__ void lcb_cand_kernel(const TIN* __restrict__ E_C, long long ld_EC, const int32_t* __restrict__ req_idx,
+                                int B_R, long long B_C, int n_C, int D, const __nv_bfloat16* __restrict__ P_CC, int o_C,
+                                const float* __restrict__ ZL, void* L_C, long long ld_LC, int out_mode,
+                                long long lo_off, int* status) {
+  __shared__ float sP[LCB_OMAX * 64];
+  for (int i = threadIdx.x; i < o_C * n_C; i += blockDim.x) sP[i] = __bfloat162float(P_CC[i]);
+  __syncthreads();
+  const long long c = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (c >= B_C) return;
+  const int r = req_idx[c];
+  if (r < 0 || r >= B_R) {
+    if (lane == 0) set_status(status, ROCS_ERR_INDEX);
+    return;
+  }
+  float acc[LCB_OMAX][DPL];
+#pragma unroll
+  for (int o = 0; o < LCB_OMAX; ++o)
+#pragma unroll
+    for (int j = 0; j < DPL; ++j) {
+      const int d = lane + 32 * j;
+      acc[o][j] = (o < o_C && d < D) ? ZL[((long long)r * o_C + o) * D + d] : 0.f;
+    }
+  const TIN* ec = E_C + c * ld_EC;
+  for (int t = 0; t < n_C; ++t) {
+    float e[DPL];
+#pragma unroll
+    for (int j = 0; j < DPL; ++j) {
+      const int d = lane + 32 * j;
+      e[j] = d < D ? ld_f(ec + t * D + d) : 0.f;
+    }
+#pragma unroll
+    for (int o = 0; o < LCB_OMAX; ++o) {
+      if (o < o_C) {
+        const float p = sP[o * n_C + t];
+#pragma unroll
+        for (int j = 0; j < DPL; ++j) acc[o][j] = fmaf(p, e[j], acc[o][j]);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 0; o < LCB_OMAX; ++o) {
+    if (o >= o_C) continue;
+#pragma unroll
+    for (int j = 0; j < DPL; ++j) {
+      const int d = lane + 32 * j;
+      if (d < D) store_val(L_C, c * ld_LC + (long long)o * D + d, acc[o][j], out_mode, lo_off);
+    }
+  }
+}
+
+int fm_trows(int n_R, int n_C) {
+  auto r16 = [](int x) { return (x + 15) / 16 * 16; };
+  int t = n_R + r16(n_C);
+  t = t > r16(n_R + n_C) ? t : r16(n_R + n_C);
+  t = t > r16(n_R) ? t : r16(n_R);
+  return t;
+}
+
+template <typename TIN>
+rocs_status fm_launch(rocs_context* ctx, const TIN* E_R, const TIN* E_C, const int32_t* req_idx, int B_R, long long B_C,
+                      int n_R, int n_C, int D, void* F_R, void* F_C, int out_mode, cudaStream_t s) {
+  const int pitch = D * 2 + 16;
+  const int trows = fm_trows(n_R, n_C);
+  const int smem = FM_WARPS * trows * pitch;
+  static bool attr[64] = {false};
+  if (ctx->device < 64 && !attr[ctx->device]) {
+    rocs_status st = cuda_check(cudaFuncSetAttribute(fm_cand_kernel<TIN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     227 * 1024),
+                                "cudaFuncSetAttribute(fm_cand)");
+    if (st != ROCS_OK) return st;
+    st = cuda_check(cudaFuncSetAttribute(fm_req_kernel<TIN>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024),
+                    "cudaFuncSetAttribute(fm_req)");
+    if (st != ROCS_OK) return st;
+    attr[ctx->device] = true;
+  }
+  if (F_R != nullptr && B_R > 0) {
+    LaunchTimer lt_("fm_req", s);
+    fm_req_kernel<TIN><<<(B_R + FM_WARPS - 1) / FM_WARPS, FM_WARPS * 32, smem, s>>>(E_R, B_R, n_R, D, trows, pitch, F_R,
+                                                                                  out_mode);
+    rocs_status st = cuda_check(cudaGetLastError(), "fm_req_kernel");
+    if (st != ROCS_OK) return st;
+  }
+  if (B_C > 0) {
+    const long long per_block = (long long)FM_WARPS * FM_RUN;
+    const long long blocks = (B_C + per_block - 1) / per_block;
+    LaunchTimer lt_("fm_cand", s);
+    fm_cand_kernel<TIN><<<(unsigned)blocks, FM_WARPS * 32, smem, s>>>(E_R, E_C, req_idx, B_R, B_C, n_R, n_C, D, trows,
+                                                                     pitch, F_C, out_mode, ctx->d_status);
+    return cuda_check(cudaGetLastError(), "fm_cand_kernel");
+  }
+  return ROCS_OK;
+}
+
+template <typename TIN>
+rocs_status lcb_launch(rocs_context* ctx, const TIN* E_R, long long ld_ER, const TIN* E_C, long long ld_EC,
+                       const int32_t* req_idx, int B_R, long long B_C, int n_R, int n_C, int D, const void* P_RR,
+                       const void* P_CR, const void* P_CC, int o_R, int o_C, void* L_R, long long ld_LR, void* L_C,
+                       long long ld_LC, int out_mode, long long lo_R, long long lo_C, float* ws_Z, cudaStream_t s) {
+  if (B_R > 0 && (o_R + o_C) > 0) {
+    LaunchTimer lt_("lcb_req", s);
+    lcb_req_kernel<TIN><<<B_R, 256, 0, s>>>(E_R, ld_ER, n_R, D, (const __nv_bfloat16*)P_RR,
+                                            (const __nv_bfloat16*)P_CR, o_R, o_C, L_R, ld_LR, out_mode, lo_R, ws_Z);
+    rocs_status st = cuda_check(cudaGetLastError(), "lcb_req_kernel");
+    if (st != ROCS_OK) return st;
+  }
+  if (B_C > 0 && o_C > 0) {
+    const long long threads = B_C * 32;
+    const unsigned blocks = (unsigned)((threads + 255) / 256);
+    const int dpl = (D + 31) / 32;
+    LaunchTimer lt_("lcb_cand", s);
+    if (dpl <= 4)
+      lcb_cand_kernel<TIN, 4><<<blocks, 256, 0, s>>>(E_C, ld_EC, req_idx, B_R, B_C, n_C, D, (const __nv_bfloat16*)P_CC,
+                                                     o_C, ws_Z, L_C, ld_LC, out_mode, lo_C, ctx->d_status);
+    else
+      lcb_cand_kernel<TIN, 8><<<blocks, 256, 0, s>>>(E_C, ld_EC, req_idx, B_R, B_C, n_C, D, (const __nv_bfloat16*)P_CC,
+                                                     o_C, ws_Z, L_C, ld_LC, out_mode, lo_C, ctx->d_status);
+    return cuda_check(cudaGetLastError(), "lcb_cand_kernel");
+  }
+  return ROCS_OK;
+}
+
+}  // namespace
+
+rocs_status launch_fm(rocs_context* ctx, const void* E_R, const void* E_C, const int32_t* req_idx, int B_R,
+                      long long B_C, int n_R, int n_C, int D, void* F_R, void* F_C, int in_f32, int out_mode,
+                      cudaStream_t s) {
+  if (in_f32)
+    return fm_launch<float>(ctx, (const float*)E_R, (const float*)E_C, req_idx, B_R, B_C, n_R, n_C, D, F_R, F_C,
+                            out_mode, s);
+  return fm_launch<__nv_bfloat16>(ctx, (const __nv_bfloat16*)E_R, (const __nv_bfloat16*)E_C, req_idx, B_R, B_C, n_R,
+                                  n_C, D, F_R, F_C, out_mode, s);
+}
+
+rocs_status launch_token_lcb(rocs_context* ctx, const void* E_R, long long ld_ER, const void* E_C, long long ld_EC,
+                             const int32_t* req_idx, int B_R, long long B_C, int n_R, int n_C, int D,
+                             const void* P_RR, const void* P_CR, const void* P_CC, int o_R, int o_C, void* L_R,
+                             long long ld_LR, void* L_C, long long ld_LC, int in_f32, int out_mode, long long lo_R,
+                             long long lo_C, float* ws_Z, cudaStream_t s) {
+  if (in_f32)
+    return lcb_launch<float>(ctx, (const float*)E_R, ld_ER, (const float*)E_C, ld_EC, req_idx, B_R, B_C, n_R, n_C, D,
+                             P_RR, P_CR, P_CC, o_R, o_C, L_R, ld_LR, L_C, ld_LC, out_mode, lo_R, lo_C, ws_Z, s);
+  return lcb_launch<__nv_bfloat16>(ctx, (const __nv_bfloat16*)E_R, ld_ER, (const __nv_bfloat16*)E_C, ld_EC, req_idx,
+                                   B_R, B_C, n_R, n_C, D, P_RR, P_CR, P_CC, o_R, o_C, L_R, ld_LR, L_C, ld_LC, out_mode,
+                                   lo_R, lo_C, ws_Z, s);
+}
+
+}  // namespace rocs

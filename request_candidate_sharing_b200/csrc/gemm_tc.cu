@@ -1,0 +1,416 @@
+// Persistent grouped GEMM on the 5th-generation tensor cores (tcgen05 + TMEM + TMA), with the
+// IKBO epilogue: bias, the request-map gather Z[m_i] and the activation are applied to the
+// accumulator tile in registers and only the final output is written
+// ([REV] §2.4: "the candidate GEMM's epilogue looks up m_i, loads the request contribution
+// and adds it in registers").
+//
+// Design (B200, one CTA per SM, 192 threads):
+//   warp 0      TMA producer: A tile 128x64 and B tile BNx64 (bf16, 128-B swizzle) per stage,
+//               4-stage ring of mbarriers (full: TMA -> MMA, empty: MMA -> TMA).
+//   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators); lane 0 issues
+//               tcgen05.mma (M=128, N=BN, K=16) and commits to the ring / accumulator barriers.
+//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time (each thread owns one output row),
+//               + bias + Z[gidx[row]] + act, bf16/fp32 stores.  The second accumulator lets the
+//               epilogue of tile i overlap the main loop of tile i+1 (the Blackwell form of the
+//               pages' producer / ping-pong consumer warp specialisation).
+// Tiles of all problems form one static round-robin schedule over the persistent CTAs; when
+// every problem has the same M, tiles are interleaved per 128-row block so the problems that
+// share the A operand read it from L2 rather than HBM.
+// No cluster launch, no multicast: each CTA loads its own operand tiles.
+#include <algorithm>
+#include <cstring>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace rocs {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int BN_MAX = 256;
+constexpr int STAGES = 4;
+constexpr int A_STAGE = BM * BK * 2;       // 16 KiB
+constexpr int B_STAGE = BN_MAX * BK * 2;   // 32 KiB
+constexpr int THREADS = 192;
+constexpr int TMEM_COLS = 512;
+constexpr int SMEM_BYTES = 1024 + STAGES * (A_STAGE + B_STAGE) + 256;
+
+struct Problem {
+  CUtensorMap tmA;
+  CUtensorMap tmB;
+  const float* bias;
+  const float* Z;
+  const int32_t* gidx;
+  void* out;
+  long long ldo, ldz;
+  int M, N, K, BN;
+  int out_mode, act, gidx_bound, vec_ok;
+  int m_tiles, n_tiles, k_blocks, b_kblocks, tile_start, n_start;
+  long long lo_off;   // out_mode 2: column offset of the low half
+};
+
+struct Params {
+  Problem p[kMaxGemmProblems];
+  int nprob;
+  int total_tiles;
+  int interleave;     // 1: tile order (m block, problem, n block); 0: problem-major
+  int n_per_m;        // sum of n_tiles over problems (interleave mode)
+  int* status;
+};
+
+__device__ __forceinline__ void decode_tile(const Params& P, int t, int& pi, int& mb, int& nb) {
+  if (P.interleave) {
+    mb = t / P.n_per_m;
+    int r = t - mb * P.n_per_m;
+    pi = 0;
+    while (pi + 1 < P.nprob && r >= P.p[pi + 1].n_start) ++pi;
+    nb = r - P.p[pi].n_start;
+  } else {
+    pi = 0;
+    while (pi + 1 < P.nprob && t >= P.p[pi + 1].tile_start) ++pi;
+    int local = t - P.p[pi].tile_start;
+    mb = local / P.p[pi].n_tiles;
+    nb = local - mb * P.p[pi].n_tiles;
+  }
+}
+
+__device__ __forceinline__ void store_bf16_32(__nv_bfloat16* o, int ncol, bool vec, const float (&v)[32]) {
+  if (ncol == 32 && vec) {
+    uint4* o4 = reinterpret_cast<uint4*>(o);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint4 w;
+      w.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+      w.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+      w.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+      w.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+      o4[j] = w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < ncol) o[j] = __float2bfloat16_rn(v[j]);
+  }
+}
+
+// out_mode 0: fp32; 1: bf16; 2: bf16 pair -- hi = bf16(v) at column c, lo = bf16(v - hi) at
+// column c + lo_off (activations carried as hi + lo keep ~16 mantissa bits for the next GEMM).
+__device__ __forceinline__ void store_chunk(const Problem& pr, long long grow, int col0, float (&v)[32]) {
+  const int ncol = min(32, pr.N - col0);
+  if (pr.out_mode == 1) {
+    store_bf16_32(reinterpret_cast<__nv_bfloat16*>(pr.out) + grow * pr.ldo + col0, ncol, pr.vec_ok, v);
+  } else if (pr.out_mode == 2) {
+    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(pr.out) + grow * pr.ldo + col0;
+    float lo[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float h = __bfloat162float(__float2bfloat16_rn(v[j]));
+      lo[j] = v[j] - h;
+      v[j] = h;
+    }
+    store_bf16_32(o, ncol, pr.vec_ok, v);
+    store_bf16_32(o + pr.lo_off, ncol, pr.vec_ok, lo);
+  } else {
+    float* o = reinterpret_cast<float*>(pr.out) + grow * pr.ldo + col0;
+    if (ncol == 32 && pr.vec_ok) {
+      float4* o4 = reinterpret_cast<float4*>(o);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o4[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (j < ncol) o[j] = v[j];
+    }
+  }
+}
+
+__global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_constant__ Params P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = base;
+  uint8_t* sB = base + STAGES * A_STAGE;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      for (int i = 0; i < P.nprob; ++i) {
+        prefetch_tensormap(&P.p[i].tmA);
+        prefetch_tensormap(&P.p[i].tmB);
+      }
+      int stage = 0;
+      uint32_t phase = 0;
+      long long issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < P.total_tiles && ok; t += gridDim.x) {
+        int pi, mb, nb;
+        decode_tile(P, t, pi, mb, nb);
+        const Problem& pr = P.p[pi];
+        for (int kb = 0; kb < pr.k_blocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, P.status, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[stage], A_STAGE + pr.BN * BK * 2);
+          tma_load_2d(sA + stage * A_STAGE, &pr.tmA, &full[stage], kb * BK, mb * BM);
+          // split operands: A rows are [hi | lo], B's k blocks repeat for the low half
+          const int kbB = kb < pr.b_kblocks ? kb : kb - pr.b_kblocks;
+          tma_load_2d(sB + stage * B_STAGE, &pr.tmB, &full[stage], kbB * BK, nb * pr.BN);
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      // Make sure no copy issued by this CTA is still landing in shared memory at exit.
+      for (int i = 0; i < STAGES && i < issued; ++i) {
+        if (--stage < 0) { stage = STAGES - 1; phase ^= 1; }
+        mbar_wait(&full[stage], phase, P.status, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < P.total_tiles && ok; t += gridDim.x) {
+        int pi, mb, nb;
+        decode_tile(P, t, pi, mb, nb);
+        const Problem& pr = P.p[pi];
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1, P.status, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN_MAX);
+        const uint32_t idesc = idesc_bf16_f32(BM, pr.BN);
+        for (int kb = 0; kb < pr.k_blocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, P.status, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * A_STAGE);
+          const uint32_t b0 = smem_u32(sB + stage * B_STAGE);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            tc_mma_bf16(d_tmem, smem_desc_sw128(a0 + k * 32), smem_desc_sw128(b0 + k * 32), idesc,
+                        (kb | k) != 0 ? 1u : 0u);
+          tc_commit(&empty[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        tc_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+      // Drain: every MMA this thread issued has completed before TMEM is released.
+      tc_commit(drain);
+      mbar_wait(drain, 0, P.status, nullptr);
+    }
+  } else {
+    // ---------------- epilogue warps ----------------
+    const int q = warp & 3;            // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < P.total_tiles; t += gridDim.x) {
+      int pi, mb, nb;
+      decode_tile(P, t, pi, mb, nb);
+      const Problem& pr = P.p[pi];
+      if (!mbar_wait(&tfull[acc], acc_phase, P.status, abort_flag)) break;
+      tc_fence_after();
+      const long long grow = (long long)mb * BM + row;
+      bool rvalid = grow < pr.M;
+      const float* zrow = nullptr;
+      if (rvalid && pr.Z != nullptr) {
+        const int zi = pr.gidx[grow];
+        if (zi < 0 || zi >= pr.gidx_bound) {
+          set_status(P.status, ROCS_ERR_INDEX);
+          rvalid = false;
+        } else {
+          zrow = pr.Z + (long long)zi * pr.ldz;
+        }
+      }
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MAX);
+      const int nchunks = pr.BN / 32;
+      for (int c = 0; c < nchunks; ++c) {
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(tbase + (uint32_t)(c * 32), r);
+        tmem_ld_wait();
+        if (c == nchunks - 1) {
+          tc_fence_before();
+          mbar_arrive(&tempty[acc]);
+        }
+        const int col0 = nb * pr.BN + c * 32;
+        if (rvalid && col0 < pr.N) {
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        const bool full32 = (col0 + 32 <= pr.N) && pr.vec_ok;
+        if (pr.bias != nullptr) {
+          if (full32) {
+            const float4* b4 = reinterpret_cast<const float4*>(pr.bias + col0);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              float4 b = __ldg(b4 + j);
+              v[4 * j] += b.x; v[4 * j + 1] += b.y; v[4 * j + 2] += b.z; v[4 * j + 3] += b.w;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (col0 + j < pr.N) v[j] += pr.bias[col0 + j];
+          }
+        }
+        if (zrow != nullptr) {
+          if (full32) {
+            const float4* z4 = reinterpret_cast<const float4*>(zrow + col0);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              float4 z = __ldg(z4 + j);
+              v[4 * j] += z.x; v[4 * j + 1] += z.y; v[4 * j + 2] += z.z; v[4 * j + 3] += z.w;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (col0 + j < pr.N) v[j] += zrow[col0 + j];
+          }
+        }
+        if (pr.act != ROCS_ACT_NONE) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = act_apply(v[j], pr.act);
+        }
+        store_chunk(pr, grow, col0, v);
+        }
+      }
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+bool encode_bf16_kmajor(rocs_context* ctx, CUtensorMap* map, const void* ptr, long long rows, int K, long long ld,
+                        int box_rows) {
+  EncodeTiledFn fn = reinterpret_cast<EncodeTiledFn>(ctx->encode_fn);
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+rocs_status launch_gemm_bf16(rocs_context* ctx, const GemmDesc* probs, int nprob, cudaStream_t s) {
+  if (nprob < 1 || nprob > kMaxGemmProblems) {
+    set_error("gemm: %d problems (1..%d supported)", nprob, kMaxGemmProblems);
+    return ROCS_ERR_INVALID_ARG;
+  }
+  static bool attr_set[64] = {false};
+  if (ctx->device < 64 && !attr_set[ctx->device]) {
+    rocs_status st = cuda_check(
+        cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES),
+        "cudaFuncSetAttribute(gemm)");
+    if (st != ROCS_OK) return st;
+    attr_set[ctx->device] = true;
+  }
+  Params P;
+  memset(&P, 0, sizeof(P));
+  P.nprob = nprob;
+  P.status = ctx->d_status;
+  int tiles = 0;
+  bool same_m = true;
+  int nstart = 0;
+  for (int i = 0; i < nprob; ++i) {
+    const GemmDesc& g = probs[i];
+    const int kA = g.split_a ? 2 * g.K : g.K;   // A columns read
+    if (g.M < 1 || g.N < 1 || g.K < 1 || g.K % 8 || g.lda % 8 || g.ldb % 8 || g.lda < kA || g.ldb < g.K ||
+        (g.split_a && g.K % BK) || ((uintptr_t)g.A & 15) || ((uintptr_t)g.B & 15) || g.out == nullptr ||
+        (g.Z && !g.gidx) || g.ldo < (g.out_mode == 2 ? 2LL * g.N : g.N)) {
+      set_error("gemm problem %d: unsupported shape/alignment (M=%d N=%d K=%d lda=%lld ldb=%lld)", i, g.M, g.N, g.K,
+                g.lda, g.ldb);
+      return ROCS_ERR_INVALID_ARG;
+    }
+    Problem& p = P.p[i];
+    p.BN = g.N >= BN_MAX ? BN_MAX : ((g.N + 31) / 32) * 32;
+    if (!encode_bf16_kmajor(ctx, &p.tmA, g.A, g.M, kA, g.lda, BM) ||
+        !encode_bf16_kmajor(ctx, &p.tmB, g.B, g.N, g.K, g.ldb, p.BN)) {
+      set_error("gemm problem %d: cuTensorMapEncodeTiled failed", i);
+      return ROCS_ERR_CUDA;
+    }
+    p.bias = g.bias;
+    p.Z = g.Z;
+    p.gidx = g.gidx;
+    p.gidx_bound = g.gidx_bound;
+    p.out = g.out;
+    p.ldo = g.ldo;
+    p.ldz = g.ldz;
+    p.M = g.M;
+    p.N = g.N;
+    p.K = g.K;
+    p.out_mode = g.out_mode;
+    p.act = g.act;
+    p.lo_off = g.N;
+    const int ve = g.out_mode == 0 ? 4 : 8;
+    p.vec_ok = (g.ldo % ve == 0) && (((uintptr_t)g.out & 15) == 0) && (!g.bias || ((uintptr_t)g.bias & 15) == 0) &&
+               (!g.Z || (((uintptr_t)g.Z & 15) == 0 && g.ldz % 4 == 0)) && (g.out_mode != 2 || g.N % 8 == 0);
+    p.m_tiles = (g.M + BM - 1) / BM;
+    p.n_tiles = (g.N + p.BN - 1) / p.BN;
+    p.b_kblocks = (g.K + BK - 1) / BK;
+    p.k_blocks = g.split_a ? 2 * p.b_kblocks : p.b_kblocks;
+    p.tile_start = tiles;
+    p.n_start = nstart;
+    tiles += p.m_tiles * p.n_tiles;
+    nstart += p.n_tiles;
+    if (g.M != probs[0].M) same_m = false;
+  }
+  P.total_tiles = tiles;
+  P.interleave = same_m ? 1 : 0;
+  P.n_per_m = nstart;
+  const int grid = std::min(tiles, ctx->num_sms);
+  LaunchTimer lt_("gemm_tc", s);
+  gemm_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(P);
+  return cuda_check(cudaGetLastError(), "gemm_tc_kernel launch");
+}
+
+}  // namespace rocs

@@ -1,0 +1,133 @@
+// Host-side internal interfaces of librocs (not part of the C ABI).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "../../include/rocs.h"
+
+// Per-launch CUDA-event timing (see rocs_timing_start / rocs_timing_stop).
+struct RocsTimer {
+  bool enabled = false;
+  std::vector<cudaEvent_t> pool;   // 2 events per recorded launch
+  size_t next = 0;
+  std::vector<std::string> labels; // label of launch i uses pool[2i], pool[2i+1]
+  long long dropped = 0;           // launches beyond the pool size
+};
+
+struct rocs_context {
+  int device = 0;
+  int num_sms = 148;
+  int* d_status = nullptr;   // sticky device status word
+  void* encode_fn = nullptr; // cuTensorMapEncodeTiled
+  RocsTimer timer;
+};
+
+namespace rocs {
+
+// The handle whose API call is running on this thread, and the call-site label that prefixes
+// kernel names in the timing report; set by the entry points in api.cpp.
+extern thread_local rocs_context* g_ctx;
+extern thread_local const char* g_site;
+
+struct SiteLabel {
+  const char* prev;
+  explicit SiteLabel(const char* site) : prev(g_site) { g_site = site; }
+  ~SiteLabel() { g_site = prev; }
+};
+
+// Records start/stop events around one kernel launch on `s` when timing is enabled.
+struct LaunchTimer {
+  rocs_context* ctx;
+  cudaStream_t s;
+  long long idx = -1;
+  LaunchTimer(const char* kernel, cudaStream_t stream) : ctx(g_ctx), s(stream) {
+    if (!ctx || !ctx->timer.enabled) return;
+    RocsTimer& t = ctx->timer;
+    if (2 * (t.next + 1) > t.pool.size()) {
+      ++t.dropped;
+      return;
+    }
+    idx = (long long)t.next++;
+    t.labels.push_back(std::string(g_site ? g_site : "api") + ":" + kernel);
+    cudaEventRecord(t.pool[2 * idx], s);
+  }
+  ~LaunchTimer() {
+    if (idx >= 0) cudaEventRecord(ctx->timer.pool[2 * idx + 1], s);
+  }
+};
+
+void set_error(const char* fmt, ...);
+rocs_status cuda_check(cudaError_t e, const char* what);
+
+// One GEMM problem for the tcgen05 kernel:
+//   out[r, c] = act( sum_k A[r, k] * B[c, k] + bias[c] + Z[gidx[r], c] )
+// A [M, K] bf16 (row stride lda), B [N, K] bf16 (row stride ldb); bias, Z, gidx optional.
+// split_a: A rows hold a hi/lo pair [hi (K) | lo (K)] of one fp32-precise activation
+//   (K % 64 == 0); the kernel accumulates hi*B + lo*B.
+// out_mode: 0 fp32, 1 bf16, 2 bf16 hi/lo pair (row [hi (N) | lo (N)], ldo >= 2N).
+struct GemmDesc {
+  const void* A = nullptr; long long lda = 0; int M = 0; int K = 0; int split_a = 0;
+  const void* B = nullptr; long long ldb = 0; int N = 0;
+  const float* bias = nullptr;
+  const float* Z = nullptr; long long ldz = 0; const int32_t* gidx = nullptr; int gidx_bound = 0;
+  void* out = nullptr; long long ldo = 0; int out_mode = 1; int act = ROCS_ACT_NONE;
+};
+
+constexpr int kMaxGemmProblems = 4;
+
+// Launches one persistent grouped GEMM over `nprob` problems (<= kMaxGemmProblems).
+// Requirements (checked): K % 8 == 0, lda/ldb % 8 == 0, A/B 16-byte aligned, M, N, K >= 1.
+rocs_status launch_gemm_bf16(rocs_context* ctx, const GemmDesc* probs, int nprob, cudaStream_t s);
+
+// fp32 SIMT GEMM with the same epilogue (exact-order FFMA, used by the fp32 IKBO path).
+rocs_status launch_gemm_f32(rocs_context* ctx, const float* A, long long lda, int M, int K, const float* B,
+                            long long ldb, int N, const float* bias, const float* Z, long long ldz,
+                            const int32_t* gidx, int gidx_bound, float* out, long long ldo, int act,
+                            cudaStream_t s);
+
+rocs_status launch_segments(rocs_context* ctx, const int32_t* counts, int B_R, int32_t* offsets,
+                            int32_t* req_idx, long long B_C, cudaStream_t s);
+
+rocs_status launch_iota(int32_t* out, int n, int step, cudaStream_t s);
+
+// Copies a [rows, cols] matrix (row stride ld_src elements, 2 or 4 bytes each) into a
+// zero-padded [rows, ld_dst] buffer.
+rocs_status launch_pad_rows(const void* src, long long ld_src, void* dst, long long ld_dst, long long rows,
+                            int cols, int elem_bytes, cudaStream_t s);
+
+// in_f32: X1, X2, residual are fp32 (else bf16).  Y is fp32 or bf16 (y_bf16); Y2 (optional) gets a
+// second, bf16 copy of the output with row stride ldy2.
+rocs_status launch_layernorm(rocs_context* ctx, const void* X1, int w1, long long ld1, const void* X2, int w2,
+                             long long ld2, const void* res, long long ldr, long long rows, const float* gamma,
+                             const float* beta, float eps, void* Y, long long ldy, int in_f32, int y_bf16, void* Y2,
+                             long long ldy2, cudaStream_t s);
+
+rocs_status launch_convert_bf16_f32(const void* src, long long ld_src, float* dst, long long ld_dst, long long rows,
+                                    int cols, cudaStream_t s);
+
+// Output modes shared by the FM / token-LCB / LN kernels: 0 fp32, 1 bf16, 2 bf16 hi/lo pair.
+rocs_status launch_fm(rocs_context* ctx, const void* E_R, const void* E_C, const int32_t* req_idx, int B_R,
+                      long long B_C, int n_R, int n_C, int D, void* F_R, void* F_C, int in_f32, int out_mode,
+                      cudaStream_t s);
+
+rocs_status launch_token_lcb(rocs_context* ctx, const void* E_R, long long ld_ER, const void* E_C,
+                             long long ld_EC, const int32_t* req_idx, int B_R, long long B_C, int n_R, int n_C,
+                             int D, const void* P_RR, const void* P_CR, const void* P_CC, int o_R, int o_C,
+                             void* L_R, long long ld_LR, void* L_C, long long ld_LC, int in_f32, int out_mode,
+                             long long lo_R, long long lo_C, float* ws_Z, cudaStream_t s);
+
+// q_split: Q rows hold [hi (H*d_h) | lo (H*d_h)] (ldq covers both).  O in fp32 or bf16 (out_bf16);
+// O2 (optional) receives a bf16 copy with row stride ldo2.
+rocs_status launch_attention(rocs_context* ctx, const void* Q, long long ldq, int q_split, const void* K,
+                             const void* V, long long ldkv, long long kv_req_stride, const int32_t* offsets, int B_R,
+                             long long rows, int L, int H, int d_h, float scale, void* O, long long ldo,
+                             int out_bf16, void* O2, long long ldo2, cudaStream_t s);
+
+rocs_status launch_score_head(const void* X, long long ldx, long long rows, int K, const void* w,
+                              const float* b, float* out, cudaStream_t s);
+
+}  // namespace rocs

@@ -1,0 +1,109 @@
+"""GPU parity of the whole ROCS forward (rocs_forward) against the float64 dense early-broadcast
+oracle: GLM stack (Wukong-style), DCA with own queries, and the end-to-end ranking forward with
+the scoring head.  Reduced batch sizes so the oracle finishes in seconds; the model dims are the
+configs' own.  Bounds: relative L2 5e-3, max abs 2e-2 + half a bf16 ulp (bf16 outputs)."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import rocs_oracle as O
+from tests.gpu_util import check_bf16, dev, dev_i32, host, stream
+
+pytestmark = pytest.mark.gpu
+
+FP32_KEYS = ("b_R", "b_C", ".b", "gamma", "beta")
+
+
+@pytest.fixture(scope="module")
+def R():
+    from request_candidate_sharing_b200 import rocs
+    h = rocs.Rocs(0)
+    yield h
+    h.close()
+
+
+def run_forward(R, case, x, W):
+    from request_candidate_sharing_b200 import rocs
+    md = rocs.model_desc(case)
+    Wd = {k: dev(v, torch.float32 if k.endswith(FP32_KEYS) else torch.bfloat16) for k, v in W.items()}
+    g, a = case.glm, case.dca
+    mw = rocs.model_weights(Wd, g.layers if g else 0, a.layers if a else 0, case.scoring is not None)
+    keep = dict(W=Wd)
+    xin = {k: dev(v) for k, v in x.items()}
+    keep["x"] = xin
+    counts = dev_i32(case.counts)
+    inp = rocs.Inputs(counts.data_ptr(), rocs.ptr(xin.get("E_R")), rocs.ptr(xin.get("E_C")),
+                      rocs.ptr(xin.get("H")), rocs.ptr(xin.get("Y_R")), rocs.ptr(xin.get("Y_C")))
+    B_R, B_C = case.B_R, case.B_C
+    out = {"offsets": torch.empty(B_R + 1, dtype=torch.int32, device="cuda"),
+           "req_idx": torch.empty(max(B_C, 1), dtype=torch.int32, device="cuda")}
+    if g is not None:
+        out["E_R"] = torch.empty((B_R, g.n_R, g.D), dtype=torch.float32, device="cuda")
+        out["E_C"] = torch.empty((max(B_C, 1), g.n_C, g.D), dtype=torch.float32, device="cuda")
+    if a is not None:
+        out["S"] = torch.empty((a.layers, B_R, a.L, a.d), dtype=torch.bfloat16, device="cuda")
+        out["A_R"] = torch.empty((a.layers, B_R, a.d), dtype=torch.float32, device="cuda")
+        out["A_C"] = torch.empty((a.layers, B_C, a.d), dtype=torch.float32, device="cuda")
+    if case.scoring is not None:
+        out["score"] = torch.empty(max(B_C, 1), dtype=torch.float32, device="cuda")
+    o = rocs.Outputs(*[rocs.ptr(out.get(k)) for k in ("offsets", "req_idx", "E_R", "E_C", "S", "A_R", "A_C", "score")])
+    nb = R.rocs_forward_workspace(md)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    R.rocs_forward(md, mw, inp, o, ws, nb, stream())
+    assert R.rocs_get_device_status(stream()) == 0
+    return out
+
+
+def test_forward_glm_stack(R):
+    case = synth.model_cfg3(B_R=3, counts=[5, 0, 37])
+    x, W = synth.model_inputs(case), synth.model_weights(case)
+    out = run_forward(R, case, x, W)
+    off, m = O.segments(case.counts)
+    assert np.array_equal(out["offsets"].cpu().numpy(), off)
+    assert np.array_equal(out["req_idx"][:case.B_C].cpu().numpy(), m)
+    ref = O.forward_cfg3(case, x, W, m)
+    check_bf16(host(out["E_R"]), ref["E_R"], what="E_R")
+    check_bf16(host(out["E_C"][:case.B_C]), ref["E_C"], what="E_C")
+
+
+def test_forward_glm_invariant_on_gpu(R):
+    case = synth.model_cfg3(B_R=2, counts=[9, 4])
+    x, W = synth.model_inputs(case), synth.model_weights(case)
+    o1 = run_forward(R, case, x, W)
+    x2 = dict(x)
+    x2["E_C"] = synth.bf16_round(x["E_C"] * 0.5 - 1.0)
+    o2 = run_forward(R, case, x2, W)
+    assert torch.equal(o1["E_R"], o2["E_R"])
+    x3 = dict(x)
+    x3["E_C"] = x["E_C"].copy()
+    x3["E_C"][2] = synth.bf16_round(x3["E_C"][2] + 1.0)
+    o3 = run_forward(R, case, x3, W)
+    keep = [i for i in range(case.B_C) if i != 2]
+    assert torch.equal(o1["E_C"][keep], o3["E_C"][keep])
+
+
+def test_forward_dca_own_queries(R):
+    case = synth.model_cfg4(B_R=2, counts=[7, 3])
+    x, W = synth.model_inputs(case), synth.model_weights(case)
+    out = run_forward(R, case, x, W)
+    _, m = O.segments(case.counts)
+    ref = O.forward_cfg4(case, x, W, m)
+    for l in range(case.dca.layers):
+        check_bf16(host(out["S"][l]), ref["S"][l], out_bf16=True, what=f"S_{l}")
+        check_bf16(host(out["A_R"][l]), ref["A_R"][l], what=f"A_R_{l}")
+        check_bf16(host(out["A_C"][l]), ref["A_C"][l], what=f"A_C_{l}")
+
+
+def test_forward_end_to_end_scoring(R):
+    case = synth.model_cfg5(B_R=3, counts=[4, 1, 20], L=256)
+    x, W = synth.model_inputs(case), synth.model_weights(case)
+    out = run_forward(R, case, x, W)
+    _, m = O.segments(case.counts)
+    ref = O.forward_cfg5(case, x, W, m)
+    check_bf16(host(out["score"][:case.B_C]), ref["score"], what="score")
+    check_bf16(host(out["E_R"]), ref["E_R"], what="E_R")
+    check_bf16(host(out["E_C"][:case.B_C]), ref["E_C"], what="E_C")
+    for l in range(case.dca.layers):
+        check_bf16(host(out["A_R"][l]), ref["A_R"][l], what=f"A_R_{l}")
+        check_bf16(host(out["A_C"][l]), ref["A_C"][l], what=f"A_C_{l}")

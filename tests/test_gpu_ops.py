@@ -1,0 +1,316 @@
+"""GPU parity of each librocs entry point against the float64 oracle, through the C ABI.
+
+Sizes span several tiles and ragged tails; edge cases: empty requests, one-candidate requests,
+rows not multiple of 16 bytes (alignment fix), partial N tiles.  Bounds: bit-exact for the
+segment bookkeeping and for small-integer inputs (every summation order exact); fp32 path max
+relative error 1e-4; bf16 path relative L2 5e-3 and max abs 2e-2 (+ half an output ulp when
+the output itself is bf16).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import rocs_oracle as O
+from tests.gpu_util import (check_bf16, check_fp32, dev, dev_i32, host, sample_candidates, stream)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def R():
+    from request_candidate_sharing_b200 import rocs
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    h = rocs.Rocs(0)
+    yield h
+    h.close()
+
+
+def _status_ok(R):
+    assert R.rocs_get_device_status(stream()) == 0
+
+
+# ---------------------------------------------------------------------------------------------
+# a0
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("counts", [[3, 0, 5, 1], [64] * 4, [0], [1],
+                                    synth.model_cfg3().counts.tolist(), synth.model_cfg5().counts.tolist(),
+                                    [7] * 3000])
+def test_segments_bit_exact(R, counts):
+    from request_candidate_sharing_b200 import rocs
+    counts = np.asarray(counts, np.int32)
+    off_ref, m_ref = O.segments(counts)
+    B_C = int(counts.sum())
+    off = torch.full((len(counts) + 1,), -7, dtype=torch.int32, device="cuda")
+    m = torch.full((max(B_C, 1),), -7, dtype=torch.int32, device="cuda")
+    R.rocs_segments_from_counts(dev_i32(counts), len(counts), off, m, B_C, stream())
+    _status_ok(R)
+    assert np.array_equal(off.cpu().numpy(), off_ref)
+    if B_C:
+        assert np.array_equal(m.cpu().numpy(), m_ref)
+
+
+def test_segments_count_mismatch_sets_status(R):
+    from request_candidate_sharing_b200 import rocs
+    counts = np.array([3, 4], np.int32)
+    off = torch.zeros(3, dtype=torch.int32, device="cuda")
+    m = torch.full((5,), -1, dtype=torch.int32, device="cuda")
+    R.rocs_segments_from_counts(dev_i32(counts), 2, off, m, 5, stream())
+    assert R.rocs_get_device_status(stream()) == rocs.ROCS_ERR_COUNTS
+    assert np.all(m.cpu().numpy()[:3] == 0)      # only slots inside [0, B_C) written
+    assert R.rocs_get_device_status(stream()) == 0   # status cleared
+
+
+# ---------------------------------------------------------------------------------------------
+# a1-a3 IKBO linear
+# ---------------------------------------------------------------------------------------------
+def _run_linear(R, case, x, m, dtype_in, dtype_out):
+    from request_candidate_sharing_b200 import rocs
+    tdt = torch.bfloat16 if dtype_in == rocs.ROCS_BF16 else torch.float32
+    odt = torch.bfloat16 if dtype_out == rocs.ROCS_BF16 else torch.float32
+    d = rocs.IkboDesc(case.B_R, case.B_C, case.d_R_in, case.d_C_in, case.d_R_out, case.d_C_out, dtype_in,
+                      dtype_out, rocs.ACT[case.act])
+    ws_bytes = R.rocs_linear_ikbo_workspace(d)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
+    t = {k: dev(v, tdt) for k, v in x.items() if k.startswith(("X", "W"))}
+    bR, bC = dev(x["b_R"], torch.float32), dev(x["b_C"], torch.float32)
+    YR = torch.full((case.B_R, case.d_R_out), float("nan"), dtype=odt, device="cuda")
+    YC = torch.full((max(case.B_C, 1), case.d_C_out), float("nan"), dtype=odt, device="cuda")
+    R.rocs_linear_ikbo(d, t["X_R"], t["X_C"], dev_i32(m), t["W_RR"], t["W_CR"], t["W_CC"], bR, bC, YR, YC, ws,
+                       ws_bytes, stream())
+    _status_ok(R)
+    return YR, YC[:case.B_C]
+
+
+def test_linear_fp32_cfg1(R):
+    from request_candidate_sharing_b200 import rocs
+    case = synth.linear_cfg1()
+    x = synth.linear_inputs(case)
+    _, m = O.segments(case.counts)
+    YR, YC = _run_linear(R, case, x, m, rocs.ROCS_F32, rocs.ROCS_F32)
+    rR, rC = O.glm_linear(x["X_R"], x["X_C"], m, x["W_RR"], x["W_CR"], x["W_CC"], x["b_R"], x["b_C"], case.act)
+    check_fp32(host(YR), rR, what="Y_R")
+    check_fp32(host(YC), rC, what="Y_C")
+
+
+@pytest.mark.parametrize("dtype_in", [0, 1])
+@pytest.mark.parametrize("shape", [
+    # (counts, d_R_in, d_C_in, d_R_out, d_C_out): tails in M, N and K; empty request
+    ([70, 0, 190], 192, 320, 136, 264),
+    ([1, 2, 3], 64, 64, 32, 32),
+    ([129], 100, 36, 40, 300),        # K not a multiple of 8 -> alignment fix on the bf16 path
+    ([5, 300], 512, 512, 0, 512),     # no request output (scoring-head form)
+])
+def test_linear_integer_inputs_bit_exact(R, dtype_in, shape):
+    """Small integers: every product and partial sum is exact in fp32, so GPU == oracle bit for bit."""
+    from request_candidate_sharing_b200 import rocs
+    counts, dRi, dCi, dRo, dCo = shape
+    case = synth.LinearCase("int", np.asarray(counts, np.int32), dRi, dCi, dRo, dCo, "relu", dtype_in == 1, 7)
+    x = synth.linear_inputs(case, integer=3)
+    _, m = O.segments(case.counts)
+    YR, YC = _run_linear(R, case, x, m, dtype_in, rocs.ROCS_F32)
+    rR, rC = O.glm_linear(x["X_R"], x["X_C"], m, x["W_RR"] if dRo else None, x["W_CR"], x["W_CC"],
+                          x["b_R"] if dRo else None, x["b_C"], "relu")
+    if dRo:
+        assert np.array_equal(host(YR), rR)
+    assert np.array_equal(host(YC), rC)
+
+
+@pytest.mark.parametrize("out_dtype", [0, 1])
+@pytest.mark.parametrize("N,d", [(64, 512), (17, 1024), (3, 256)])
+def test_linear_bf16_random(R, out_dtype, N, d):
+    from request_candidate_sharing_b200 import rocs
+    case = synth.linear_cfg2(N, d, B_R=9)
+    x = synth.linear_inputs(case)
+    _, m = O.segments(case.counts)
+    YR, YC = _run_linear(R, case, x, m, rocs.ROCS_BF16, out_dtype)
+    rR, rC = O.glm_linear(x["X_R"], x["X_C"], m, x["W_RR"], x["W_CR"], x["W_CC"], x["b_R"], x["b_C"], "relu")
+    check_bf16(host(YR), rR, out_bf16=out_dtype == 1, what="Y_R")
+    check_bf16(host(YC), rC, out_bf16=out_dtype == 1, what="Y_C")
+    if out_dtype == 0:   # fp32 outputs: only accumulation-order error remains
+        check_fp32(host(YC), rC, rel=1e-4, what="Y_C fp32")
+
+
+def test_linear_glm_invariant_and_row_independence_gpu(R):
+    from request_candidate_sharing_b200 import rocs
+    case = synth.linear_cfg2(64, 512, B_R=6)
+    x = synth.linear_inputs(case)
+    _, m = O.segments(case.counts)
+    YR1, YC1 = _run_linear(R, case, x, m, rocs.ROCS_BF16, rocs.ROCS_BF16)
+    x2 = dict(x)
+    x2["X_C"] = synth.bf16_round(x["X_C"] * -2.0 + 0.5)
+    YR2, _ = _run_linear(R, case, x2, m, rocs.ROCS_BF16, rocs.ROCS_BF16)
+    assert torch.equal(YR1, YR2)
+    x3 = dict(x)
+    x3["X_C"] = x["X_C"].copy()
+    x3["X_C"][100] = synth.bf16_round(x3["X_C"][100] + 1.0)
+    _, YC3 = _run_linear(R, case, x3, m, rocs.ROCS_BF16, rocs.ROCS_BF16)
+    keep = torch.ones(case.B_C, dtype=torch.bool, device="cuda")
+    keep[100] = False
+    assert torch.equal(YC1[keep], YC3[keep]) and not torch.equal(YC1[100], YC3[100])
+
+
+def test_linear_bad_request_index_sets_status(R):
+    from request_candidate_sharing_b200 import rocs
+    case = synth.linear_cfg2(64, 512, B_R=2)
+    x = synth.linear_inputs(case)
+    _, m = O.segments(case.counts)
+    m = m.copy()
+    m[5] = 99
+    d = rocs.IkboDesc(case.B_R, case.B_C, 512, 512, 512, 512, rocs.ROCS_BF16, rocs.ROCS_F32, 1)
+    nb = R.rocs_linear_ikbo_workspace(d)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    t = {k: dev(v) for k, v in x.items() if k.startswith(("X", "W"))}
+    YR = torch.zeros(2, 512, device="cuda")
+    YC = torch.full((case.B_C, 512), -5.0, device="cuda")
+    R.rocs_linear_ikbo(d, t["X_R"], t["X_C"], dev_i32(m), t["W_RR"], t["W_CR"], t["W_CC"],
+                       dev(x["b_R"], torch.float32), dev(x["b_C"], torch.float32), YR, YC, ws, nb, stream())
+    assert R.rocs_get_device_status(stream()) == rocs.ROCS_ERR_INDEX
+    assert torch.all(YC[5] == -5.0)       # the bad row is skipped, not written
+    assert not torch.all(YC[4] == -5.0)
+
+
+def test_linear_cfg2_sampled_full_size(R):
+    """IKBO sweep point N=256, d=1024 at full size (65536 candidates); oracle on a sample."""
+    from request_candidate_sharing_b200 import rocs
+    case = synth.linear_cfg2(256, 1024)
+    x = synth.linear_inputs(case)
+    _, m = O.segments(case.counts)
+    YR, YC = _run_linear(R, case, x, m, rocs.ROCS_BF16, rocs.ROCS_BF16)
+    rows = sample_candidates(case.counts, 4)
+    rR, rC = O.glm_linear(x["X_R"], x["X_C"][rows], m[rows], x["W_RR"], x["W_CR"], x["W_CC"], x["b_R"], x["b_C"],
+                          "relu")
+    check_bf16(host(YR), rR, out_bf16=True, what="Y_R")
+    check_bf16(host(YC[torch.from_numpy(rows).cuda()]), rC, out_bf16=True, what="Y_C sample")
+
+
+# ---------------------------------------------------------------------------------------------
+# a6 group LayerNorm
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("io", [0, 1])
+@pytest.mark.parametrize("w1,w2,res,rows", [(2048, 2048, True, 37), (1024, 1024, True, 300), (256, 0, True, 1000),
+                                            (100, 28, False, 9), (4096, 0, False, 3)])
+def test_group_layernorm(R, io, w1, w2, res, rows):
+    g = np.random.default_rng(w1 + w2 + rows)
+    tdt = torch.bfloat16 if io == 1 else torch.float32
+    rnd = (lambda a: synth.bf16_round(a)) if io == 1 else (lambda a: a)
+    X1 = rnd((g.standard_normal((rows, w1)) * 2 + 0.3).astype(np.float32))
+    X2 = rnd(g.standard_normal((rows, w2)).astype(np.float32))
+    Rr = rnd(g.standard_normal((rows, w1 + w2)).astype(np.float32)) if res else None
+    gam = (1 + g.uniform(-0.1, 0.1, w1 + w2)).astype(np.float32)
+    bet = g.uniform(-0.1, 0.1, w1 + w2).astype(np.float32)
+    Y = torch.empty((rows, w1 + w2), dtype=tdt, device="cuda")
+    R.rocs_group_layernorm(dev(X1, tdt), w1, dev(X2, tdt) if w2 else None, w2, dev(Rr, tdt) if res else None, rows,
+                           dev(gam, torch.float32), dev(bet, torch.float32), 1e-5, Y, io, stream())
+    _status_ok(R)
+    x = np.concatenate([X1, X2], 1).astype(np.float64) + (Rr if res else 0)
+    ref = O.group_layernorm(x, gam, bet)
+    if io == 0:
+        check_fp32(host(Y), ref, what="LN fp32")
+    else:
+        check_bf16(host(Y), ref, out_bf16=True, what="LN bf16")
+
+
+# ---------------------------------------------------------------------------------------------
+# a4 masked FM and token LCB
+# ---------------------------------------------------------------------------------------------
+def _glm_small(counts, seed=3):
+    case = synth.model_cfg3(B_R=len(counts), counts=counts, seed=seed)
+    return case, synth.model_inputs(case), synth.model_weights(case)
+
+
+@pytest.mark.parametrize("counts", [[3, 0, 17, 1, 40], [130, 64]])
+def test_fm_masked(R, counts):
+    case, x, W = _glm_small(counts)
+    g = case.glm
+    _, m = O.segments(case.counts)
+    FR = torch.empty((case.B_R, g.n_R * g.n_R), device="cuda")
+    FC = torch.empty((case.B_C, g.n_C * (g.n_R + g.n_C)), device="cuda")
+    R.rocs_fm_masked(dev(x["E_R"]), dev(x["E_C"]), dev_i32(m), case.B_R, case.B_C, g.n_R, g.n_C, g.D, FR, FC, 0,
+                     stream())
+    _status_ok(R)
+    rR, rC = O.fm_masked(x["E_R"], x["E_C"], m)
+    check_fp32(host(FR), rR, what="F_R")
+    check_fp32(host(FC), rC, what="F_C")
+
+
+def test_fm_integer_exact(R):
+    counts = np.array([2, 5], np.int32)
+    _, m = O.segments(counts)
+    ER = synth.small_ints(1, "ER", (2, 32, 128), 2)
+    EC = synth.small_ints(1, "EC", (7, 16, 128), 2)
+    FR = torch.empty((2, 1024), device="cuda")
+    FC = torch.empty((7, 768), device="cuda")
+    R.rocs_fm_masked(dev(ER), dev(EC), dev_i32(m), 2, 7, 32, 16, 128, FR, FC, 0, stream())
+    rR, rC = O.fm_masked(ER, EC, m)
+    assert np.array_equal(host(FR), rR) and np.array_equal(host(FC), rC)
+
+
+@pytest.mark.parametrize("o_R,o_C", [(16, 8), (1, 1)])
+def test_token_lcb(R, o_R, o_C):
+    case, x, W = _glm_small([4, 0, 33])
+    g = case.glm
+    _, m = O.segments(case.counts)
+    rng = np.random.default_rng(5)
+    P_RR = synth.bf16_round(rng.standard_normal((o_R, g.n_R)).astype(np.float32) / 5)
+    P_CR = synth.bf16_round(rng.standard_normal((o_C, g.n_R)).astype(np.float32) / 5)
+    P_CC = synth.bf16_round(rng.standard_normal((o_C, g.n_C)).astype(np.float32) / 4)
+    nb = R.rocs_token_lcb_workspace(case.B_R, o_C, g.D)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    LR = torch.empty((case.B_R, o_R * g.D + 64), device="cuda")   # wider rows: strided output
+    LC = torch.empty((case.B_C, o_C * g.D), device="cuda")
+    R.rocs_token_lcb(dev(x["E_R"]), dev(x["E_C"]), dev_i32(m), case.B_R, case.B_C, g.n_R, g.n_C, g.D, dev(P_RR),
+                     dev(P_CR), dev(P_CC), o_R, o_C, LR, o_R * g.D + 64, LC, o_C * g.D, 0, ws, nb, stream())
+    _status_ok(R)
+    db = O.DenseBatch(m, case.B_R)
+    rR, rC = O.token_lcb_rows(db.broadcast(x["E_R"]), db.with_probe(x["E_C"]), P_RR, P_CR, P_CC)
+    check_fp32(host(LR[:, :o_R * g.D]), db.request_out(rR).reshape(case.B_R, -1), what="L_R")
+    check_fp32(host(LC), db.cand_out(rC).reshape(case.B_C, -1), what="L_C")
+
+
+# ---------------------------------------------------------------------------------------------
+# a9 cross-attention
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("L,H,dh,counts", [(200, 4, 64, [3, 0, 40, 17]), (1024, 8, 32, [33, 1]),
+                                           (5, 2, 32, [16, 2, 0]), (512, 1, 64, [70])])
+def test_cross_attention(R, L, H, dh, counts):
+    counts = np.asarray(counts, np.int32)
+    off, m = O.segments(counts)
+    B_R, n, d = len(counts), int(counts.sum()), H * dh
+    g = np.random.default_rng(L + n)
+    K = synth.bf16_round(g.standard_normal((B_R, L, d)).astype(np.float32))
+    V = synth.bf16_round(g.standard_normal((B_R, L, d)).astype(np.float32))
+    Q = synth.bf16_round(g.standard_normal((n, d)).astype(np.float32))
+    Ot = torch.full((max(n, 1), d), float("nan"), device="cuda")
+    R.rocs_dca_cross_attn(dev(Q), dev(K), dev(V), dev_i32(off), B_R, n, L, H, dh, 1.0 / math.sqrt(dh), Ot, d, 0,
+                          stream())
+    _status_ok(R)
+    ref = O.cross_attn(Q, K, V, m, H)
+    check_bf16(host(Ot[:n]), ref, what="cross-attention")
+
+
+# ---------------------------------------------------------------------------------------------
+# a7 DCA encoder
+# ---------------------------------------------------------------------------------------------
+def test_dca_encode(R):
+    from request_candidate_sharing_b200 import rocs
+    case = synth.model_cfg4(B_R=3, counts=[1, 1, 1])
+    a = case.dca
+    W = synth.model_weights(case)
+    x = synth.model_inputs(case)
+    Wd = {k: dev(v, torch.float32 if ("ln." in k) else torch.bfloat16) for k, v in W.items()}
+    desc = rocs.DcaDesc(case.B_R, a.L, a.d, a.H, a.layers)
+    nb = R.rocs_dca_encode_workspace(desc)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    S = torch.empty((a.layers, case.B_R, a.L, a.d), dtype=torch.bfloat16, device="cuda")
+    KV = torch.empty((a.layers, 4, case.B_R, a.L, a.d), dtype=torch.bfloat16, device="cuda")
+    R.rocs_dca_encode(desc, dev(x["H"]), [rocs.dca_layer_weights(Wd, l) for l in range(a.layers)], S, KV, ws, nb,
+                      stream())
+    _status_ok(R)
+    Ss, KVs = O.dca_encode(x["H"], W, a.layers, a.H)
+    for l in range(a.layers):
+        check_bf16(host(S[l]), Ss[l], out_bf16=True, what=f"S_{l}")
+        for i in range(4):
+            check_bf16(host(KV[l, i]), KVs[l][i], out_bf16=True, what=f"KV_{l}_{i}")
