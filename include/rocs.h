@@ -124,6 +124,31 @@ rocs_status rocs_linear_ikbo(rocs_handle_t handle, const rocs_ikbo_desc* desc,
                              void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------------
+ * rocs_linear_ikbo_noalloc: the same operation as rocs_linear_ikbo for callers that cannot
+ * allocate device memory at all, not even a workspace to hand over -- for example plugin hosts
+ * and serving loops that plan every device buffer up front and forbid allocation while
+ * requests are in flight.  The paper has no counterpart; this is a deployment variant.
+ *   - Scratch: Z = W_CR X^R + b^C lives in one built-in device array of 1,048,576 fp32 values
+ *     (4 MiB) that every GPU loading the library keeps until the process exits.  Requests with
+ *     B_R * d_C_out above that limit, or bf16 rows that would need the alignment fix
+ *     (d_R_in or d_C_in not a multiple of 8), return ROCS_ERR_UNSUPPORTED with a message
+ *     pointing to rocs_linear_ikbo.  The call never allocates or frees device memory.
+ *   - Set-up: the first call on each device (with that device current, as for every call on
+ *     the handle) looks up the array's device address once and caches it; make that first call
+ *     before any stream capture.
+ *   - Sharing: all calls on a device use the same array, and it keeps the last call's Z.
+ *     Z is fully rewritten before it is read, so nothing has to be cleared, but calls whose
+ *     work overlaps on the GPU (different streams, or different host threads) race on it:
+ *     order them on one stream or with events.
+ *   - Arguments, layouts, dtypes and results are those of rocs_linear_ikbo.
+ * ---------------------------------------------------------------------------------------- */
+rocs_status rocs_linear_ikbo_noalloc(rocs_handle_t handle, const rocs_ikbo_desc* desc,
+                                     const void* X_R, const void* X_C, const int32_t* req_idx,
+                                     const void* W_RR, const void* W_CR, const void* W_CC,
+                                     const float* b_R, const float* b_C, void* Y_R, void* Y_C,
+                                     void* stream);
+
+/* ------------------------------------------------------------------------------------------
  * a6. Concat + residual + group-local LayerNorm ([SUM]: normalisation statistics per group,
  * never over the concatenation; [REV] §2.1 Figure 2(b)).  For each of `rows` rows:
  *   x = concat(X1[row, 0:w1], X2[row, 0:w2]) (+ residual[row, 0:w1+w2] if non-NULL)

@@ -122,10 +122,11 @@ _lib_fwd_ws = _proto("rocs_forward_workspace", P, C.POINTER(ModelDesc), C.POINTE
 _lib_fwd = _proto("rocs_forward", P, C.POINTER(ModelDesc), C.POINTER(ModelWeights), C.POINTER(Inputs),
                   C.POINTER(Outputs), P, C.c_size_t, P)
 
+_lib_ikbo_na = _proto("rocs_linear_ikbo_noalloc", P, C.POINTER(IkboDesc), P, P, P, P, P, P, P, P, P, P, P)
 _lib_tstart = _proto("rocs_timing_start", P, I32)
 _lib_tstop = _proto("rocs_timing_stop", P, C.c_char_p, C.c_size_t)
 
-EXPORTED = ["rocs_timing_start", "rocs_timing_stop", "rocs_create", "rocs_destroy", "rocs_last_error", "rocs_get_device_status", "rocs_num_sms",
+EXPORTED = ["rocs_linear_ikbo_noalloc", "rocs_timing_start", "rocs_timing_stop", "rocs_create", "rocs_destroy", "rocs_last_error", "rocs_get_device_status", "rocs_num_sms",
             "rocs_segments_from_counts", "rocs_linear_ikbo_workspace", "rocs_linear_ikbo", "rocs_group_layernorm",
             "rocs_fm_masked", "rocs_token_lcb_workspace", "rocs_token_lcb", "rocs_dca_cross_attn",
             "rocs_dca_encode_workspace", "rocs_dca_encode", "rocs_forward_workspace", "rocs_forward"]
@@ -202,6 +203,12 @@ class Rocs:
                          workspace, workspace_bytes: int, stream=None):
         _check(_lib_ikbo(self.h, C.byref(desc), ptr(X_R), ptr(X_C), ptr(req_idx), ptr(W_RR), ptr(W_CR), ptr(W_CC),
                          ptr(b_R), ptr(b_C), ptr(Y_R), ptr(Y_C), ptr(workspace), int(workspace_bytes), stream))
+
+    def rocs_linear_ikbo_noalloc(self, desc: IkboDesc, X_R, X_C, req_idx, W_RR, W_CR, W_CC, b_R, b_C, Y_R, Y_C,
+                                 stream=None):
+        """rocs_linear_ikbo without a workspace: for callers that may not allocate device memory."""
+        _check(_lib_ikbo_na(self.h, C.byref(desc), ptr(X_R), ptr(X_C), ptr(req_idx), ptr(W_RR), ptr(W_CR),
+                            ptr(W_CC), ptr(b_R), ptr(b_C), ptr(Y_R), ptr(Y_C), stream))
 
     # -- a6 --
     def rocs_group_layernorm(self, X1, w1, X2, w2, residual, rows, gamma, beta, eps, Y, io, stream=None):
