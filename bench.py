@@ -83,8 +83,10 @@ def algo_work(case, label: str):
             "glm.mlp1.req:gemm_tc": ("tensor", 2.0 * B_R * g.hidden * fR * 2),
             "glm.mlp2.cand:gemm_tc": ("tensor", 2.0 * B_C * oCw * g.hidden),
             "glm.mlp2.req:gemm_tc": ("tensor", 2.0 * B_R * (oRw + oCw) * g.hidden),
-            "glm.fm:fm_cand": ("hbm", B_C * (wc * 4 + fC * 4)),
-            "glm.lcb:lcb_cand": ("hbm", B_C * (wc * 4 + lCw * 4)),
+            # fused candidate pass: reads E^C (bf16 at layer 0, fp32 after), writes F^C (hi/lo),
+            # L^C (fp32) and, when DCA queries come from the GLM stack, t^C (hi/lo)
+            "glm.fm:glm_cand_fused": ("hbm", B_C * (wc * (2 + 4 * (g.layers - 1)) / g.layers + fC * 4 + lCw * 4
+                                                   + (4 * a.q_dim if (a is not None and a.source == "glm") else 0))),
             "glm.lnC:layernorm": ("hbm", B_C * (oCw * 4 + lCw * 4 + wc * 4 + wc * 4)),
         }
         if label in table:

@@ -344,7 +344,7 @@ extern "C" rocs_status rocs_group_layernorm(rocs_handle_t h, const void* X1, int
   ROCS_REQUIRE(eps > 0.f, "rocs_group_layernorm: eps must be > 0");
   const int f32 = io == ROCS_F32;
   return launch_layernorm(h, X1, w1, w1, w2 ? X2 : nullptr, w2, w2, residual, w1 + w2, rows, gamma, beta, eps, Y,
-                          w1 + w2, f32, !f32, nullptr, 0, (cudaStream_t)stream);
+                          w1 + w2, f32, f32, !f32, nullptr, 0, (cudaStream_t)stream);
 }
 
 // =============================================================================================
@@ -461,8 +461,8 @@ rocs_status encoder_layer(rocs_context* ctx, const EncScratch& e, int B_R, int L
   SiteLabel sl2("enc.wo");
   ROCS_TRY(linear_bf16(ctx, e.att, d, M, d, w.Wo, d, nullptr, e.tmp, d, 1, ROCS_ACT_NONE, s));
   SiteLabel sl3("enc.ln");
-  ROCS_TRY(launch_layernorm(ctx, e.tmp, d, d, nullptr, 0, 0, S_in, d, M, w.ln_gamma, w.ln_beta, 1e-5f, S_out, d, 0, 1,
-                            nullptr, 0, s));
+  ROCS_TRY(launch_layernorm(ctx, e.tmp, d, d, nullptr, 0, 0, S_in, d, M, w.ln_gamma, w.ln_beta, 1e-5f, S_out, d, 0, 0,
+                            1, nullptr, 0, s));
   SiteLabel sl4("enc.kv");
   const void* Wk[4] = {w.WK_R, w.WV_R, w.WK_C, w.WV_C};
   void* kv[4] = {KR, VR, KC, VC};
@@ -737,19 +737,15 @@ extern "C" rocs_status rocs_forward(rocs_handle_t h, const rocs_model_desc* m, c
   const long long wr = (long long)m->n_R * m->D, wc = (long long)m->n_C * m->D;
   const long long xr = m->score_h1 > 0 ? wr + (long long)m->dca_layers * m->d : 0;
   const long long xc = m->score_h1 > 0 ? wc + (long long)m->dca_layers * m->d : 0;
-  // GLM residual stream (fp32): layer l reads E_l, writes E_{l+1}
-  const float* ER = nullptr;
-  const float* EC = nullptr;
-  if (m->glm_layers > 0) {
-    ROCS_TRY(launch_convert_bf16_f32(in->E_R, wr, p.ER[0], wr, BR, (int)wr, s));
-    ROCS_TRY(launch_convert_bf16_f32(in->E_C, wc, p.EC[0], wc, BC, (int)wc, s));
-    ER = p.ER[0];
-    EC = p.EC[0];
-  }
+  // GLM residual stream: layer 0 reads the bf16 inputs, later layers the fp32 stream
+  const void* ER = in->E_R;
+  const void* EC = in->E_C;
+  int e_f32 = 0;
   // own-query token streams (fp32): the inputs fill the first q_n tokens
   const long long yr_ld = (long long)(m->q_n_R + m->dca_layers) * m->q_dim;
   const long long yc_ld = (long long)(m->q_n_C + m->dca_layers) * m->q_dim;
   if (m->dca_layers > 0 && m->dca_query_source == 0) {
+    SiteLabel sl("fwd.ytokens");
     ROCS_TRY(launch_convert_bf16_f32(in->Y_R, (long long)m->q_n_R * m->q_dim, p.YR, yr_ld, BR, m->q_n_R * m->q_dim, s));
     ROCS_TRY(launch_convert_bf16_f32(in->Y_C, (long long)m->q_n_C * m->q_dim, p.YC, yc_ld, BC, m->q_n_C * m->q_dim, s));
   }
@@ -759,27 +755,60 @@ extern "C" rocs_status rocs_forward(rocs_handle_t h, const rocs_model_desc* m, c
   const void* S_prev = in->Hist;
   const int steps = m->glm_layers > m->dca_layers ? m->glm_layers : m->dca_layers;
   const long long d2 = 2LL * m->d, q2 = 2LL * m->q_dim;
+  const bool fused_ok = m->D == 128 && m->lcb_out_C <= 8 && m->n_C <= 64;
 
   for (int l = 0; l < steps; ++l) {
+    const bool glm_l = l < m->glm_layers;
+    const bool dca_l = l < m->dca_layers;
+    const bool q_from_glm = dca_l && m->dca_query_source == 1;
+    const int fR = m->n_R * m->n_R, fC = m->n_C * (m->n_R + m->n_C);
+    const int lRw = m->lcb_out_R * m->D, lCw = m->lcb_out_C * m->D;
+    bool t_done = false;
+    // ---------------- a4: one pass over this layer's embeddings ----------------
+    if (glm_l) {
+      const rocs_glm_layer_weights& gw = W->glm[l];
+      const rocs_qgen_weights* qw = q_from_glm ? &W->qgen[l] : nullptr;
+      SiteLabel s_fm("glm.fm");
+      // request side: F^R (hi/lo), L^R and Z^L, and the query generator's token for depth l
+      ROCS_TRY(launch_fm(h, ER, EC, req_idx, BR, 0, m->n_R, m->n_C, m->D, p.FR, nullptr, e_f32, 2, s));
+      ROCS_TRY(launch_token_lcb(h, ER, wr, EC, wc, req_idx, BR, 0, m->n_R, m->n_C, m->D, gw.P_RR, gw.P_CR, gw.P_CC,
+                                m->lcb_out_R, m->lcb_out_C, p.LR, lRw, p.LC, lCw, e_f32, 0, 0, 0, p.ZL, s));
+      if (qw)
+        ROCS_TRY(launch_token_lcb(h, ER, wr, EC, wc, req_idx, BR, 0, m->n_R, m->n_C, m->D, qw->p_RR, qw->p_CR,
+                                  qw->p_CC, 1, 1, p.tR, q2, p.tC, q2, e_f32, 2, m->q_dim, m->q_dim, p.ZqL, s));
+      if (fused_ok) {
+        // candidate side in one kernel: F^C (hi/lo), L^C and the depth-l query token t^C
+        ROCS_TRY(launch_glm_cand_fused(h, ER, EC, req_idx, BR, BC, m->n_R, m->n_C, e_f32, p.FC, gw.P_CC, m->lcb_out_C,
+                                       p.ZL, p.LC, qw ? qw->p_CC : nullptr, p.ZqL, qw ? p.tC : nullptr, s));
+        t_done = qw != nullptr;
+      } else {
+        ROCS_TRY(launch_fm(h, ER, EC, req_idx, BR, BC, m->n_R, m->n_C, m->D, nullptr, p.FC, e_f32, 2, s));
+        SiteLabel s_lcb("glm.lcb");
+        ROCS_TRY(launch_token_lcb(h, ER, wr, EC, wc, req_idx, BR, BC, m->n_R, m->n_C, m->D, gw.P_RR, gw.P_CR,
+                                  gw.P_CC, m->lcb_out_R, m->lcb_out_C, p.LR, lRw, p.LC, lCw, e_f32, 0, 0, 0, p.ZL, s));
+      }
+    }
     // ---------------- DCA depth l ----------------
-    if (l < m->dca_layers) {
+    if (dca_l) {
       const rocs_dca_layer_weights& dw = W->dca[l];
       void* S_l = out->S ? (void*)((char*)out->S + S_plane * l) : p.S[l & 1];
       ROCS_TRY(encoder_layer(h, p.enc, BR, m->L, m->d, m->H, dw, S_prev, S_l, p.KR, p.VR, p.KC, p.VC, s));
       S_prev = S_l;
       // query generator: token LCB to one token per group (hi/lo), then the GLM-MLP
       const rocs_qgen_weights& qw = W->qgen[l];
-      const float *qER, *qEC;
-      long long qldR, qldC;
-      int qnR, qnC;
-      if (m->dca_query_source == 0) {
-        qER = p.YR; qEC = p.YC; qldR = yr_ld; qldC = yc_ld; qnR = m->q_n_R + l; qnC = m->q_n_C + l;
-      } else {
-        qER = ER; qEC = EC; qldR = wr; qldC = wc; qnR = m->n_R; qnC = m->n_C;
+      if (!t_done) {
+        const void *qER, *qEC;
+        long long qldR, qldC;
+        int qnR, qnC, qf32;
+        if (m->dca_query_source == 0) {
+          qER = p.YR; qEC = p.YC; qldR = yr_ld; qldC = yc_ld; qnR = m->q_n_R + l; qnC = m->q_n_C + l; qf32 = 1;
+        } else {
+          qER = ER; qEC = EC; qldR = wr; qldC = wc; qnR = m->n_R; qnC = m->n_C; qf32 = e_f32;
+        }
+        SiteLabel s_qlcb("qgen.lcb");
+        ROCS_TRY(launch_token_lcb(h, qER, qldR, qEC, qldC, req_idx, BR, BC, qnR, qnC, m->q_dim, qw.p_RR, qw.p_CR,
+                                  qw.p_CC, 1, 1, p.tR, q2, p.tC, q2, qf32, 2, m->q_dim, m->q_dim, p.ZqL, s));
       }
-      SiteLabel s_qlcb("qgen.lcb");
-      ROCS_TRY(launch_token_lcb(h, qER, qldR, qEC, qldC, req_idx, BR, BC, qnR, qnC, m->q_dim, qw.p_RR, qw.p_CR,
-                                qw.p_CC, 1, 1, p.tR, q2, p.tC, q2, 1, 2, m->q_dim, m->q_dim, p.ZqL, s));
       IkboArgs a1;
       a1.B_R = BR; a1.B_C = BC; a1.dRi = m->q_dim; a1.dCi = m->q_dim; a1.dRo = m->d; a1.dCo = m->d;
       a1.X_R = p.tR; a1.ldxr = q2; a1.X_C = p.tC; a1.ldxc = q2; a1.req_idx = req_idx; a1.split_in = 1;
@@ -815,12 +844,16 @@ extern "C" rocs_status rocs_forward(rocs_handle_t h, const rocs_model_desc* m, c
       const int dh = m->d / m->H;
       const float scale = 1.0f / std::sqrt((float)dh);
       const long long kvs = (long long)m->L * m->d;
-      SiteLabel s_xa("xattn.req");
-      ROCS_TRY(launch_attention(h, p.QR, d2, 1, p.KR, p.VR, m->d, kvs, p.iota1, BR, BR, m->L, m->H, dh, scale, dR, ldR,
-                                0, xR2, xr, s));
-      SiteLabel s_xc("xattn.cand");
-      ROCS_TRY(launch_attention(h, p.QC, d2, 1, p.KC, p.VC, m->d, kvs, offsets, BR, BC, m->L, m->H, dh, scale, dC, ldC,
-                                0, xC2, xc, s));
+      {
+        SiteLabel s_xa("xattn.req");
+        ROCS_TRY(launch_attention(h, p.QR, d2, 1, p.KR, p.VR, m->d, kvs, p.iota1, BR, BR, m->L, m->H, dh, scale, dR,
+                                  ldR, 0, xR2, xr, s));
+      }
+      {
+        SiteLabel s_xc("xattn.cand");
+        ROCS_TRY(launch_attention(h, p.QC, d2, 1, p.KC, p.VC, m->d, kvs, offsets, BR, BC, m->L, m->H, dh, scale, dC,
+                                  ldC, 0, xC2, xc, s));
+      }
       if (m->dca_query_source == 0) {
         if (out->A_R)
           ROCS_TRY(cuda_check(cudaMemcpy2DAsync((float*)out->A_R + (size_t)BR * m->d * l, (size_t)m->d * 4, dR, ldR * 4,
@@ -832,13 +865,9 @@ extern "C" rocs_status rocs_forward(rocs_handle_t h, const rocs_model_desc* m, c
                               "copy A_C"));
       }
     }
-    // ---------------- GLM layer l ----------------
-    if (l < m->glm_layers) {
+    // ---------------- GLM layer l: MLP and LayerNorm ----------------
+    if (glm_l) {
       const rocs_glm_layer_weights& gw = W->glm[l];
-      const int fR = m->n_R * m->n_R, fC = m->n_C * (m->n_R + m->n_C);
-      // a4: masked FM on the fp32 stream (bf16 operands, fp32 accumulate), F as hi/lo pairs
-      SiteLabel s_fm("glm.fm");
-      ROCS_TRY(launch_fm(h, ER, EC, req_idx, BR, BC, m->n_R, m->n_C, m->D, p.FR, p.FC, 1, 2, s));
       // a5: GLM-MLP as two IKBO linears; h as hi/lo pairs, o in fp32
       IkboArgs a;
       a.B_R = BR; a.B_C = BC; a.dRi = fR; a.dCi = fC; a.dRo = m->hidden; a.dCo = m->hidden;
@@ -860,26 +889,25 @@ extern "C" rocs_status rocs_forward(rocs_handle_t h, const rocs_model_desc* m, c
         SiteLabel sl("glm.mlp2");
         ROCS_TRY(ikbo_bf16(h, b, s));
       }
-      // token LCB on the fp32 stream, fp32 output
-      const int lRw = m->lcb_out_R * m->D, lCw = m->lcb_out_C * m->D;
-      SiteLabel s_lcb("glm.lcb");
-      ROCS_TRY(launch_token_lcb(h, ER, wr, EC, wc, req_idx, BR, BC, m->n_R, m->n_C, m->D, gw.P_RR, gw.P_CR, gw.P_CC,
-                                m->lcb_out_R, m->lcb_out_C, p.LR, lRw, p.LC, lCw, 1, 0, 0, 0, p.ZL, s));
       // a6: concat + residual + group-local LN -> next fp32 stream (plus the scoring input copy)
       const bool last = (l == m->glm_layers - 1);
       float* dR = (last && out->E_R) ? (float*)out->E_R : p.ER[(l + 1) & 1];
       float* dC = (last && out->E_C) ? (float*)out->E_C : p.EC[(l + 1) & 1];
       void* xR2 = (last && m->score_h1 > 0) ? p.xR : nullptr;
       void* xC2 = (last && m->score_h1 > 0) ? p.xC : nullptr;
-      SiteLabel s_ln("glm.lnR");
-      ROCS_TRY(launch_layernorm(h, p.oR, oRw, oRw, p.LR, lRw, lRw, ER, wr, BR, gw.lnR_gamma, gw.lnR_beta, 1e-5f, dR,
-                                wr, 1, 0, xR2, xr, s));
-      SiteLabel s_lnc("glm.lnC");
-      if (BC > 0)
+      {
+        SiteLabel s_ln("glm.lnR");
+        ROCS_TRY(launch_layernorm(h, p.oR, oRw, oRw, p.LR, lRw, lRw, ER, wr, BR, gw.lnR_gamma, gw.lnR_beta, 1e-5f, dR,
+                                  wr, 1, e_f32, 0, xR2, xr, s));
+      }
+      if (BC > 0) {
+        SiteLabel s_lnc("glm.lnC");
         ROCS_TRY(launch_layernorm(h, p.oC, oCw, oCw, p.LC, lCw, lCw, EC, wc, BC, gw.lnC_gamma, gw.lnC_beta, 1e-5f, dC,
-                                  wc, 1, 0, xC2, xc, s));
+                                  wc, 1, e_f32, 0, xC2, xc, s));
+      }
       ER = dR;
       EC = dC;
+      e_f32 = 1;
     }
   }
 

@@ -166,6 +166,38 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
 // ------------------------------------------------------------------------------------------
 // small math helpers
 // ------------------------------------------------------------------------------------------
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// GELU, exact (erf) form x * Phi(x) = x/2 * (1 + erf(x / sqrt 2)), with erf from Abramowitz &
+// Stegun, Handbook of Mathematical Functions, formula 7.1.26 (|error| <= 1.5e-7):
+//   erf(z) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2),  t = 1 / (1 + p z), z >= 0.
+// For x < 0 the factor 1 + erf(x/sqrt 2) equals the tail term itself, so no cancellation.
+__device__ __forceinline__ float gelu_erf(float x) {
+  const float z = fabsf(x) * 0.70710678118654752f;
+  const float t = rcp_approx(fmaf(0.3275911f, z, 1.0f));
+  float poly = fmaf(1.061405429f, t, -1.453152027f);
+  poly = fmaf(poly, t, 1.421413741f);
+  poly = fmaf(poly, t, -0.284496736f);
+  poly = fmaf(poly, t, 0.254829592f);
+  poly *= t;
+  const float tail = poly * ex2_approx(-z * z * 1.4426950408889634f);   // 1 - erf(z)
+  const float s = x >= 0.f ? 2.0f - tail : tail;                           // 1 + erf(x / sqrt 2)
+  return 0.5f * x * s;
+}
+
+__device__ __forceinline__ float sigmoid_fast(float x) {
+  return rcp_approx(1.0f + ex2_approx(-x * 1.4426950408889634f));
+}
+
 __device__ __forceinline__ float act_apply(float x, int act) {
   switch (act) {
     case ROCS_ACT_RELU: return fmaxf(x, 0.0f);

@@ -21,6 +21,7 @@ namespace {
 
 constexpr int FM_WARPS = 4;
 constexpr int FM_RUN = 8;   // consecutive candidates per warp
+constexpr int LCB_OMAX_F = 8;
 
 __device__ __forceinline__ uint4 load8_as_bf16(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
 __device__ __forceinline__ uint4 load8_as_bf16(const float* p) {
@@ -117,6 +118,116 @@ __device__ __forceinline__ void gram_tile(uint32_t sbase, int pitch, int a0, int
 #pragma unroll
     for (int p = 0; p < 8; ++p)
       if (p * 8 < ncols) store_c_frag(out, out_mode, obase, ld, mi * 16, p * 8, mrows, ncols, acc[p], lo_off);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Fused candidate pass of one GLM layer: reads each candidate's embeddings E^C_c ONCE and emits
+//   F^C_c  = E^C_c [E^R_{m_c} ; E^C_c]^T             (masked FM, bf16 hi/lo pairs)
+//   L^C_c  = Z^L_{m_c} + P_CC E^C_c                  (token LCB, fp32; Z^L = P_CR E^R per request)
+//   t^C_c  = Z^Q_{m_c} + p_CC E^C_c                  (optional: the DCA query generator's one-token
+//                                                      LCB of the same embeddings, bf16 hi/lo pairs)
+// Lane j owns features [DPL*j, DPL*j + DPL); the LCB sums use the full-precision embeddings, the
+// FM products their bf16 rounding (tensor-core operands).
+// ---------------------------------------------------------------------------------------------
+template <typename TIN, int DPL>
+__device__ __forceinline__ void load_feats(const TIN* p, float (&e)[DPL]);
+template <>
+__device__ __forceinline__ void load_feats<float, 4>(const float* p, float (&e)[4]) {
+  const float4 v = __ldg(reinterpret_cast<const float4*>(p));
+  e[0] = v.x; e[1] = v.y; e[2] = v.z; e[3] = v.w;
+}
+template <>
+__device__ __forceinline__ void load_feats<__nv_bfloat16, 4>(const __nv_bfloat16* p, float (&e)[4]) {
+  const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+  e[0] = bf16_lo(v.x); e[1] = bf16_hi(v.x); e[2] = bf16_lo(v.y); e[3] = bf16_hi(v.y);
+}
+
+template <typename TIN>
+__global__ void __launch_bounds__(FM_WARPS * 32) glm_cand_fused_kernel(
+    const TIN* __restrict__ E_R, const TIN* __restrict__ E_C, const int32_t* __restrict__ req_idx, int B_R,
+    long long B_C, int n_R, int n_C, int trows, int pitch, __nv_bfloat16* __restrict__ F_C,
+    const __nv_bfloat16* __restrict__ P_CC, int o_C, const float* __restrict__ ZL, float* __restrict__ L_C,
+    const __nv_bfloat16* __restrict__ q_pCC, const float* __restrict__ ZQ, __nv_bfloat16* __restrict__ tC,
+    int* status) {
+  constexpr int D = 128, DPL = 4;
+  extern __shared__ __align__(16) uint8_t fm_smem[];
+  __shared__ float sP[LCB_OMAX_F * 64];
+  __shared__ float sQ[64];
+  for (int i = threadIdx.x; i < o_C * n_C; i += blockDim.x) sP[i] = __bfloat162float(P_CC[i]);
+  for (int i = threadIdx.x; i < n_C; i += blockDim.x) sQ[i] = q_pCC ? __bfloat162float(q_pCC[i]) : 0.f;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* T = fm_smem + warp * trows * pitch;
+  const uint32_t sbase = smem_u32(T);
+  const long long c_begin = ((long long)blockIdx.x * FM_WARPS + warp) * FM_RUN;
+  const int ncols = n_R + n_C;
+  const long long fsz = (long long)n_C * ncols;
+  int staged = -1;
+  zero_rows(T + (n_R + n_C) * pitch, pitch, trows - (n_R + n_C), D);
+  for (int i = 0; i < FM_RUN; ++i) {
+    const long long c = c_begin + i;
+    if (c >= B_C) break;
+    const int r = req_idx[c];
+    if (r < 0 || r >= B_R) {
+      if (lane == 0) set_status(status, ROCS_ERR_INDEX);
+      continue;
+    }
+    __syncwarp();
+    if (r != staged) {
+      stage_rows(T, pitch, E_R + (long long)r * n_R * D, n_R, D);
+      staged = r;
+    }
+    float acc[LCB_OMAX_F][DPL];
+    float qa[DPL];
+#pragma unroll
+    for (int j = 0; j < DPL; ++j) qa[j] = 0.f;
+#pragma unroll
+    for (int o = 0; o < LCB_OMAX_F; ++o)
+#pragma unroll
+      for (int j = 0; j < DPL; ++j) acc[o][j] = 0.f;
+    const TIN* ec = E_C + c * (long long)n_C * D;
+    for (int t = 0; t < n_C; ++t) {
+      float e[DPL];
+      load_feats<TIN, DPL>(ec + t * D + DPL * lane, e);
+      *reinterpret_cast<uint2*>(T + (n_R + t) * pitch + DPL * lane * 2) =
+          make_uint2(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]));
+#pragma unroll
+      for (int o = 0; o < LCB_OMAX_F; ++o) {
+        if (o < o_C) {
+          const float p = sP[o * n_C + t];
+#pragma unroll
+          for (int j = 0; j < DPL; ++j) acc[o][j] = fmaf(p, e[j], acc[o][j]);
+        }
+      }
+      const float q = sQ[t];
+#pragma unroll
+      for (int j = 0; j < DPL; ++j) qa[j] = fmaf(q, e[j], qa[j]);
+    }
+    // LCB output (fp32, float4 per token)
+#pragma unroll
+    for (int o = 0; o < LCB_OMAX_F; ++o) {
+      if (o < o_C) {
+        const float4 z = __ldg(reinterpret_cast<const float4*>(ZL + ((long long)r * o_C + o) * D + DPL * lane));
+        reinterpret_cast<float4*>(L_C + c * (long long)o_C * D + (long long)o * D)[lane] =
+            make_float4(acc[o][0] + z.x, acc[o][1] + z.y, acc[o][2] + z.z, acc[o][3] + z.w);
+      }
+    }
+    if (tC != nullptr) {
+      const float4 z = __ldg(reinterpret_cast<const float4*>(ZQ + (long long)r * D + DPL * lane));
+      const float v[4] = {qa[0] + z.x, qa[1] + z.y, qa[2] + z.z, qa[3] + z.w};
+      float hi[4], lo[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        hi[j] = __bfloat162float(__float2bfloat16_rn(v[j]));
+        lo[j] = v[j] - hi[j];
+      }
+      __nv_bfloat16* tp = tC + c * 2LL * D + DPL * lane;
+      *reinterpret_cast<uint2*>(tp) = make_uint2(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]));
+      *reinterpret_cast<uint2*>(tp + D) = make_uint2(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]));
+    }
+    __syncwarp();
+    gram_tile(sbase, pitch, n_R, n_C, ncols, D, F_C, 2, c * fsz * 2, ncols, fsz);
   }
 }
 
@@ -333,7 +444,44 @@ rocs_status lcb_launch(rocs_context* ctx, const TIN* E_R, long long ld_ER, const
   return ROCS_OK;
 }
 
+template <typename TIN>
+rocs_status fused_launch(rocs_context* ctx, const TIN* E_R, const TIN* E_C, const int32_t* req_idx, int B_R,
+                         long long B_C, int n_R, int n_C, void* F_C, const void* P_CC, int o_C, const float* ZL,
+                         float* L_C, const void* q_pCC, const float* ZQ, void* tC, cudaStream_t s) {
+  const int D = 128;
+  const int pitch = D * 2 + 16;
+  const int trows = fm_trows(n_R, n_C);
+  const int smem = FM_WARPS * trows * pitch;
+  static bool attr[64] = {false};
+  if (ctx->device < 64 && !attr[ctx->device]) {
+    rocs_status st = cuda_check(cudaFuncSetAttribute(glm_cand_fused_kernel<TIN>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024),
+                                "cudaFuncSetAttribute(glm_cand_fused)");
+    if (st != ROCS_OK) return st;
+    attr[ctx->device] = true;
+  }
+  if (B_C == 0) return ROCS_OK;
+  const long long per_block = (long long)FM_WARPS * FM_RUN;
+  const long long blocks = (B_C + per_block - 1) / per_block;
+  LaunchTimer lt_("glm_cand_fused", s);
+  glm_cand_fused_kernel<TIN><<<(unsigned)blocks, FM_WARPS * 32, smem, s>>>(
+      E_R, E_C, req_idx, B_R, B_C, n_R, n_C, trows, pitch, (__nv_bfloat16*)F_C, (const __nv_bfloat16*)P_CC, o_C,
+      ZL, L_C, (const __nv_bfloat16*)q_pCC, ZQ, (__nv_bfloat16*)tC, ctx->d_status);
+  return cuda_check(cudaGetLastError(), "glm_cand_fused_kernel");
+}
+
 }  // namespace
+
+rocs_status launch_glm_cand_fused(rocs_context* ctx, const void* E_R, const void* E_C, const int32_t* req_idx,
+                                  int B_R, long long B_C, int n_R, int n_C, int in_f32, void* F_C, const void* P_CC,
+                                  int o_C, const float* ZL, float* L_C, const void* q_pCC, const float* ZQ, void* tC,
+                                  cudaStream_t s) {
+  if (in_f32)
+    return fused_launch<float>(ctx, (const float*)E_R, (const float*)E_C, req_idx, B_R, B_C, n_R, n_C, F_C, P_CC, o_C,
+                               ZL, L_C, q_pCC, ZQ, tC, s);
+  return fused_launch<__nv_bfloat16>(ctx, (const __nv_bfloat16*)E_R, (const __nv_bfloat16*)E_C, req_idx, B_R, B_C,
+                                     n_R, n_C, F_C, P_CC, o_C, ZL, L_C, q_pCC, ZQ, tC, s);
+}
 
 rocs_status launch_fm(rocs_context* ctx, const void* E_R, const void* E_C, const int32_t* req_idx, int B_R,
                       long long B_C, int n_R, int n_C, int D, void* F_R, void* F_C, int in_f32, int out_mode,

@@ -9,10 +9,11 @@
 //               4-stage ring of mbarriers (full: TMA -> MMA, empty: MMA -> TMA).
 //   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators); lane 0 issues
 //               tcgen05.mma (M=128, N=BN, K=16) and commits to the ring / accumulator barriers.
-//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time (each thread owns one output row),
-//               + bias + Z[gidx[row]] + act, bf16/fp32 stores.  The second accumulator lets the
-//               epilogue of tile i overlap the main loop of tile i+1 (the Blackwell form of the
-//               pages' producer / ping-pong consumer warp specialisation).
+//   warps 2..9  epilogue: two warps per TMEM lane quarter, splitting the tile's 32-column
+//               chunks between them; tcgen05.ld 32 columns at a time (each thread owns one
+//               output row), + bias + Z[gidx[row]] + act, bf16/fp32 stores.  The second
+//               accumulator lets the epilogue of tile i overlap the main loop of tile i+1 (the
+//               Blackwell form of the pages' producer / ping-pong consumer warp specialisation).
 // Tiles of all problems form one static round-robin schedule over the persistent CTAs; when
 // every problem has the same M, tiles are interleaved per 128-row block so the problems that
 // share the A operand read it from L2 rather than HBM.
@@ -32,7 +33,8 @@ constexpr int BN_MAX = 256;
 constexpr int STAGES = 4;
 constexpr int A_STAGE = BM * BK * 2;       // 16 KiB
 constexpr int B_STAGE = BN_MAX * BK * 2;   // 32 KiB
-constexpr int THREADS = 192;
+constexpr int THREADS = 320;
+constexpr int EPI_THREADS = 256;
 constexpr int TMEM_COLS = 512;
 constexpr int SMEM_BYTES = 1024 + STAGES * (A_STAGE + B_STAGE) + 256;
 
@@ -149,7 +151,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 128);
+      mbar_init(&tempty[b], EPI_THREADS);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -236,6 +238,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
   } else {
     // ---------------- epilogue warps ----------------
     const int q = warp & 3;            // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;  // which of the two warps on this quarter
     const int row = q * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -259,54 +262,71 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
       }
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MAX);
       const int nchunks = pr.BN / 32;
-      for (int c = 0; c < nchunks; ++c) {
+      // this warp takes chunks half, half + 2, ...; it releases the accumulator after its last load
+      const int last = nchunks - 1 - ((nchunks - 1 - half) & 1);
+      if (last < 0) {
+        mbar_arrive(&tempty[acc]);
+      }
+      for (int c = half; c < nchunks; c += 2) {
         uint32_t r[32];
         __syncwarp();
         tmem_ld_32x32b_x32(tbase + (uint32_t)(c * 32), r);
         tmem_ld_wait();
-        if (c == nchunks - 1) {
+        if (c == last) {
           tc_fence_before();
           mbar_arrive(&tempty[acc]);
         }
         const int col0 = nb * pr.BN + c * 32;
         if (rvalid && col0 < pr.N) {
-        float v[32];
+          float v[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-        const bool full32 = (col0 + 32 <= pr.N) && pr.vec_ok;
-        if (pr.bias != nullptr) {
-          if (full32) {
-            const float4* b4 = reinterpret_cast<const float4*>(pr.bias + col0);
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          const bool full32 = (col0 + 32 <= pr.N) && pr.vec_ok;
+          if (pr.bias != nullptr) {
+            if (full32) {
+              const float4* b4 = reinterpret_cast<const float4*>(pr.bias + col0);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              float4 b = __ldg(b4 + j);
-              v[4 * j] += b.x; v[4 * j + 1] += b.y; v[4 * j + 2] += b.z; v[4 * j + 3] += b.w;
+              for (int j = 0; j < 8; ++j) {
+                float4 b = __ldg(b4 + j);
+                v[4 * j] += b.x; v[4 * j + 1] += b.y; v[4 * j + 2] += b.z; v[4 * j + 3] += b.w;
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col0 + j < pr.N) v[j] += pr.bias[col0 + j];
             }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (col0 + j < pr.N) v[j] += pr.bias[col0 + j];
           }
-        }
-        if (zrow != nullptr) {
-          if (full32) {
-            const float4* z4 = reinterpret_cast<const float4*>(zrow + col0);
+          if (zrow != nullptr) {
+            if (full32) {
+              const float4* z4 = reinterpret_cast<const float4*>(zrow + col0);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              float4 z = __ldg(z4 + j);
-              v[4 * j] += z.x; v[4 * j + 1] += z.y; v[4 * j + 2] += z.z; v[4 * j + 3] += z.w;
+              for (int j = 0; j < 8; ++j) {
+                float4 z = __ldg(z4 + j);
+                v[4 * j] += z.x; v[4 * j + 1] += z.y; v[4 * j + 2] += z.z; v[4 * j + 3] += z.w;
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col0 + j < pr.N) v[j] += zrow[col0 + j];
             }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (col0 + j < pr.N) v[j] += zrow[col0 + j];
           }
-        }
-        if (pr.act != ROCS_ACT_NONE) {
+          switch (pr.act) {
+            case ROCS_ACT_RELU:
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = act_apply(v[j], pr.act);
-        }
-        store_chunk(pr, grow, col0, v);
+              for (int j = 0; j < 32; ++j) v[j] = fmaxf(v[j], 0.f);
+              break;
+            case ROCS_ACT_GELU:
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
+              break;
+            case ROCS_ACT_SIGMOID:
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = sigmoid_fast(v[j]);
+              break;
+            default:
+              break;
+          }
+          store_chunk(pr, grow, col0, v);
         }
       }
       acc ^= 1;

@@ -99,12 +99,12 @@ rocs_status launch_iota(int32_t* out, int n, int step, cudaStream_t s);
 rocs_status launch_pad_rows(const void* src, long long ld_src, void* dst, long long ld_dst, long long rows,
                             int cols, int elem_bytes, cudaStream_t s);
 
-// in_f32: X1, X2, residual are fp32 (else bf16).  Y is fp32 or bf16 (y_bf16); Y2 (optional) gets a
-// second, bf16 copy of the output with row stride ldy2.
+// in_f32: X1, X2 are fp32 (else bf16); res_f32: the residual is fp32 (else bf16).  Y is fp32 or
+// bf16 (y_bf16); Y2 (optional) gets a second, bf16 copy of the output with row stride ldy2.
 rocs_status launch_layernorm(rocs_context* ctx, const void* X1, int w1, long long ld1, const void* X2, int w2,
                              long long ld2, const void* res, long long ldr, long long rows, const float* gamma,
-                             const float* beta, float eps, void* Y, long long ldy, int in_f32, int y_bf16, void* Y2,
-                             long long ldy2, cudaStream_t s);
+                             const float* beta, float eps, void* Y, long long ldy, int in_f32, int res_f32,
+                             int y_bf16, void* Y2, long long ldy2, cudaStream_t s);
 
 rocs_status launch_convert_bf16_f32(const void* src, long long ld_src, float* dst, long long ld_dst, long long rows,
                                     int cols, cudaStream_t s);
@@ -113,6 +113,14 @@ rocs_status launch_convert_bf16_f32(const void* src, long long ld_src, float* ds
 rocs_status launch_fm(rocs_context* ctx, const void* E_R, const void* E_C, const int32_t* req_idx, int B_R,
                       long long B_C, int n_R, int n_C, int D, void* F_R, void* F_C, int in_f32, int out_mode,
                       cudaStream_t s);
+
+// One pass over the candidates' embeddings (D = 128): masked-FM products as bf16 hi/lo pairs, the
+// token LCB output L_C (fp32, o_C tokens, Z^L from the request side) and, if tC is non-NULL, the
+// one-token query-generator LCB (hi/lo pairs, Z^Q from the request side).
+rocs_status launch_glm_cand_fused(rocs_context* ctx, const void* E_R, const void* E_C, const int32_t* req_idx,
+                                  int B_R, long long B_C, int n_R, int n_C, int in_f32, void* F_C, const void* P_CC,
+                                  int o_C, const float* ZL, float* L_C, const void* q_pCC, const float* ZQ, void* tC,
+                                  cudaStream_t s);
 
 rocs_status launch_token_lcb(rocs_context* ctx, const void* E_R, long long ld_ER, const void* E_C,
                              long long ld_EC, const int32_t* req_idx, int B_R, long long B_C, int n_R, int n_C,

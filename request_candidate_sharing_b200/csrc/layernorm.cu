@@ -79,10 +79,10 @@ __device__ __forceinline__ float row_sum(float x, float* red) {
   return t;
 }
 
-template <typename TIN, typename TOUT, int VEC, int NV, int TPR>
+template <typename TIN, typename TRES, typename TOUT, int VEC, int NV, int TPR>
 __global__ void __launch_bounds__(TPR == 32 ? 256 : TPR) layernorm_kernel(
     const TIN* __restrict__ X1, int w1, long long ld1, const TIN* __restrict__ X2, long long ld2,
-    const TIN* __restrict__ R, long long ldr, long long rows, int width, const float* __restrict__ gamma,
+    const TRES* __restrict__ R, long long ldr, long long rows, int width, const float* __restrict__ gamma,
     const float* __restrict__ beta, float eps, TOUT* __restrict__ Y, long long ldy, __nv_bfloat16* __restrict__ Y2,
     long long ldy2) {
   __shared__ float red[32];
@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(TPR == 32 ? 256 : TPR) layernorm_kernel(
       else load_vec<TIN, VEC>(X2 + row * ld2 + (c - w1), v[i]);
       if (R != nullptr) {
         float r[VEC];
-        load_vec<TIN, VEC>(R + row * ldr + c, r);
+        load_vec<TRES, VEC>(R + row * ldr + c, r);
 #pragma unroll
         for (int j = 0; j < VEC; ++j) v[i][j] += r[j];
       }
@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(TPR == 32 ? 256 : TPR) layernorm_kernel(
   }
 }
 
-template <typename TIN, typename TOUT, int VEC, int NV, int TPR>
+template <typename TIN, typename TRES, typename TOUT, int VEC, int NV, int TPR>
 rocs_status run(const void* X1, int w1, long long ld1, const void* X2, long long ld2, const void* R, long long ldr,
                 long long rows, int width, const float* g, const float* b, float eps, void* Y, long long ldy, void* Y2,
                 long long ldy2, cudaStream_t s) {
@@ -165,22 +165,24 @@ rocs_status run(const void* X1, int w1, long long ld1, const void* X2, long long
     return ROCS_ERR_UNSUPPORTED;
   }
   LaunchTimer lt_("layernorm", s);
-  layernorm_kernel<TIN, TOUT, VEC, NV, TPR><<<(unsigned)blocks, threads, 0, s>>>(
-      (const TIN*)X1, w1, ld1, (const TIN*)X2, ld2, (const TIN*)R, ldr, rows, width, g, b, eps, (TOUT*)Y, ldy,
+  layernorm_kernel<TIN, TRES, TOUT, VEC, NV, TPR><<<(unsigned)blocks, threads, 0, s>>>(
+      (const TIN*)X1, w1, ld1, (const TIN*)X2, ld2, (const TRES*)R, ldr, rows, width, g, b, eps, (TOUT*)Y, ldy,
       (__nv_bfloat16*)Y2, ldy2);
   return cuda_check(cudaGetLastError(), "layernorm_kernel");
 }
 
-template <typename TIN, typename TOUT>
+template <typename TIN, typename TRES, typename TOUT>
 rocs_status dispatch(const void* X1, int w1, long long ld1, const void* X2, long long ld2, const void* R,
                      long long ldr, long long rows, int width, const float* g, const float* b, float eps, void* Y,
                      long long ldy, void* Y2, long long ldy2, bool vec, cudaStream_t s) {
 #define ROCS_LN(VEC, NV, TPR) \
-  return run<TIN, TOUT, VEC, NV, TPR>(X1, w1, ld1, X2, ld2, R, ldr, rows, width, g, b, eps, Y, ldy, Y2, ldy2, s)
+  return run<TIN, TRES, TOUT, VEC, NV, TPR>(X1, w1, ld1, X2, ld2, R, ldr, rows, width, g, b, eps, Y, ldy, Y2, ldy2, s)
   if (vec) {
+    // one warp per row (registers only, no block barrier) up to 2048 values, a block beyond
     if (width <= 256) ROCS_LN(8, 1, 32);
-    if (width <= 1024) ROCS_LN(8, 1, 128);
-    if (width <= 2048) ROCS_LN(8, 2, 128);
+    if (width <= 512) ROCS_LN(8, 2, 32);
+    if (width <= 1024) ROCS_LN(8, 4, 32);
+    if (width <= 2048) ROCS_LN(8, 8, 32);
     if (width <= 4096) ROCS_LN(8, 4, 128);
     ROCS_LN(8, 8, 128);
   }
@@ -205,8 +207,8 @@ __global__ void convert_kernel(const __nv_bfloat16* __restrict__ src, long long 
 
 rocs_status launch_layernorm(rocs_context* ctx, const void* X1, int w1, long long ld1, const void* X2, int w2,
                              long long ld2, const void* res, long long ldr, long long rows, const float* gamma,
-                             const float* beta, float eps, void* Y, long long ldy, int in_f32, int y_bf16, void* Y2,
-                             long long ldy2, cudaStream_t s) {
+                             const float* beta, float eps, void* Y, long long ldy, int in_f32, int res_f32,
+                             int y_bf16, void* Y2, long long ldy2, cudaStream_t s) {
   (void)ctx;
   if (rows == 0) return ROCS_OK;
   const int width = w1 + w2;
@@ -214,17 +216,23 @@ rocs_status launch_layernorm(rocs_context* ctx, const void* X1, int w1, long lon
   const bool vec = (w1 % 8 == 0) && (width % 8 == 0) && ld1 % 8 == 0 && (X2 == nullptr || ld2 % 8 == 0) &&
                    (res == nullptr || ldr % 8 == 0) && ldy % 8 == 0 && (Y2 == nullptr || ldy2 % 8 == 0) && al(X1) &&
                    al(X2) && al(res) && al(Y) && al(Y2);
-  if (in_f32) {
-    if (y_bf16) return dispatch<float, __nv_bfloat16>(X1, w1, ld1, X2, ld2, res, ldr, rows, width, gamma, beta, eps, Y,
-                                                      ldy, Y2, ldy2, vec, s);
-    return dispatch<float, float>(X1, w1, ld1, X2, ld2, res, ldr, rows, width, gamma, beta, eps, Y, ldy, Y2, ldy2, vec,
-                                  s);
+  if (in_f32 && y_bf16) {
+    set_error("layernorm: fp32 inputs with a bf16 primary output are not instantiated");
+    return ROCS_ERR_UNSUPPORTED;
   }
-  if (y_bf16)
-    return dispatch<__nv_bfloat16, __nv_bfloat16>(X1, w1, ld1, X2, ld2, res, ldr, rows, width, gamma, beta, eps, Y, ldy,
-                                                  Y2, ldy2, vec, s);
-  return dispatch<__nv_bfloat16, float>(X1, w1, ld1, X2, ld2, res, ldr, rows, width, gamma, beta, eps, Y, ldy, Y2,
-                                        ldy2, vec, s);
+  if (in_f32) {
+    if (res_f32 || res == nullptr)
+      return dispatch<float, float, float>(X1, w1, ld1, X2, ld2, res, ldr, rows, width, gamma, beta, eps, Y, ldy, Y2,
+                                           ldy2, vec, s);
+    return dispatch<float, __nv_bfloat16, float>(X1, w1, ld1, X2, ld2, res, ldr, rows, width, gamma, beta, eps, Y, ldy,
+                                                 Y2, ldy2, vec, s);
+  }
+  if (!y_bf16 || (res != nullptr && res_f32)) {
+    set_error("layernorm: bf16 inputs need a bf16 residual and output");
+    return ROCS_ERR_UNSUPPORTED;
+  }
+  return dispatch<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(X1, w1, ld1, X2, ld2, res, ldr, rows, width, gamma,
+                                                               beta, eps, Y, ldy, Y2, ldy2, vec, s);
 }
 
 rocs_status launch_convert_bf16_f32(const void* src, long long ld_src, float* dst, long long ld_dst, long long rows,
