@@ -51,15 +51,20 @@ WORKLOADS = {
 }
 
 
-def make_case(name: str, rank: int):
+def make_case(name: str, rank: int, requests: int = 0):
+    """The workload's case; `requests` > 0 keeps only the first requests (smaller profiling runs)."""
     seed_shift = 1000 * rank
     if name == "rocs_forward_e2e":
-        return synth.model_cfg5(seed=1 + seed_shift)
-    if name == "glm_stack":
-        return synth.model_cfg3(seed=0 + seed_shift)
-    if name == "dca":
-        return synth.model_cfg4(seed=0 + seed_shift)
-    raise SystemExit(f"unknown workload {name}")
+        case = synth.model_cfg5(seed=1 + seed_shift)
+    elif name == "glm_stack":
+        case = synth.model_cfg3(seed=0 + seed_shift)
+    elif name == "dca":
+        case = synth.model_cfg4(seed=0 + seed_shift)
+    else:
+        raise SystemExit(f"unknown workload {name}")
+    if requests and requests < case.B_R:
+        case = dataclasses.replace(case, counts=case.counts[:requests].copy())
+    return case
 
 
 # ---------------------------------------------------------------------------------------------
@@ -95,7 +100,7 @@ def algo_work(case, label: str):
         L, d, H = a.L, a.d, a.H
         table = {
             "enc.attn:attn": ("alu", float(B_R) * H * L * L),
-            "xattn.cand:attn": ("alu", float(B_C) * H * L),
+            "xattn.cand:attn_stream": ("alu", float(B_C) * H * L),
             "enc.qkv:gemm_tc": ("tensor", 2.0 * B_R * L * d * d * 3),
             "enc.kv:gemm_tc": ("tensor", 2.0 * B_R * L * d * d * 4),
             "enc.wo:gemm_tc": ("tensor", 2.0 * B_R * L * d * d),
@@ -281,7 +286,7 @@ def run_librocs(args, rank, world, local):
 
     from request_candidate_sharing_b200 import rocs
     torch.cuda.set_device(local)
-    case = make_case(args.workload, rank)
+    case = make_case(args.workload, rank, args.requests)
     dev = torch.device("cuda", local)
     t_gen = time.perf_counter()
     W = synth.model_weights(case)
@@ -416,7 +421,8 @@ def run_librocs(args, rank, world, local):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) inputs, N(0,1/fan_in) bf16 weights)",
-            "config": {"workload": args.workload, "description": WORKLOADS[args.workload], "B_R": case.B_R,
+            "config": {"workload": args.workload + (f"[first {case.B_R} requests]" if args.requests else ""),
+                       "description": WORKLOADS[args.workload], "B_R": case.B_R,
                        "B_C_per_rank": B_C, "l2": "inputs larger than L2 (E_C alone is "
                        f"{(xd['E_C'].numel() * 2 / 1e9) if 'E_C' in xd else 0:.2f} GB)",
                        "parallelism": f"replicas x{world}"},
@@ -450,7 +456,7 @@ def run_librocs(args, rank, world, local):
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    case = make_case(args.workload, 0)
+    case = make_case(args.workload, 0, args.requests)
     per_step = max(1.0, args.ref_step_seconds)
     for i in range(args.warmup):
         oracle_rate(case, per_step, start_req=i)
@@ -483,6 +489,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--requests", type=int, default=0, help="keep only the first N requests (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "librocs":
         raise SystemExit("--warmup must be >= 3")

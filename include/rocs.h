@@ -201,8 +201,9 @@ rocs_status rocs_token_lcb(rocs_handle_t handle, const void* E_R, const void* E_
  *   K, V [B_R, L, H*d_h] bf16 (each request's K/V stored once).
  *   O [rows, ld_O] in `out` dtype (bf16 or fp32), head h at columns [h*d_h, (h+1)*d_h).
  *   O_q = softmax(q k^T * scale) v per head, no masking; fp32 softmax statistics.
- *   Limits: d_h in {32, 64}; L * d_h <= 32768 (each (request, head) K/V staged in shared
- *   memory once and reused by all of that request's queries).
+ *   Each (request, head)'s K/V is streamed through shared memory once per 128 queries of that
+ *   request and shared by those queries (no per-candidate copy of K/V exists).
+ *   Limits: d_h in {32, 64}; L * d_h <= 32768.
  * ---------------------------------------------------------------------------------------- */
 rocs_status rocs_dca_cross_attn(rocs_handle_t handle, const void* Q, const void* K, const void* V,
                                 const int32_t* offsets, int32_t B_R, int64_t rows, int32_t L,

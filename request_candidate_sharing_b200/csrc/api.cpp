@@ -412,8 +412,8 @@ extern "C" rocs_status rocs_dca_cross_attn(rocs_handle_t h, const void* Q, const
   ROCS_REQUIRE(out == ROCS_F32 || out == ROCS_BF16, "rocs_dca_cross_attn: bad dtype");
   ROCS_REQUIRE(std::isfinite(scale), "rocs_dca_cross_attn: scale not finite");
   const long long dm = (long long)H * d_h;
-  return launch_attention(h, Q, dm, 0, K, V, dm, (long long)L * dm, offsets, B_R, rows, L, H, d_h, scale, O, ld_O,
-                          out == ROCS_BF16, nullptr, 0, (cudaStream_t)stream);
+  return launch_attention_stream(h, Q, dm, 0, K, V, dm, (long long)L * dm, offsets, B_R, rows, L, H, d_h, scale, O,
+                                 ld_O, out == ROCS_BF16, nullptr, 0, (cudaStream_t)stream);
 }
 
 // =============================================================================================
@@ -755,7 +755,7 @@ extern "C" rocs_status rocs_forward(rocs_handle_t h, const rocs_model_desc* m, c
   const void* S_prev = in->Hist;
   const int steps = m->glm_layers > m->dca_layers ? m->glm_layers : m->dca_layers;
   const long long d2 = 2LL * m->d, q2 = 2LL * m->q_dim;
-  const bool fused_ok = m->D == 128 && m->lcb_out_C <= 8 && m->n_C <= 64;
+  const bool fused_ok = m->D == 128 && m->lcb_out_C <= 8 && m->n_C <= 16;
 
   for (int l = 0; l < steps; ++l) {
     const bool glm_l = l < m->glm_layers;
@@ -846,13 +846,13 @@ extern "C" rocs_status rocs_forward(rocs_handle_t h, const rocs_model_desc* m, c
       const long long kvs = (long long)m->L * m->d;
       {
         SiteLabel s_xa("xattn.req");
-        ROCS_TRY(launch_attention(h, p.QR, d2, 1, p.KR, p.VR, m->d, kvs, p.iota1, BR, BR, m->L, m->H, dh, scale, dR,
-                                  ldR, 0, xR2, xr, s));
+        ROCS_TRY(launch_attention_single(h, p.QR, d2, 1, p.KR, p.VR, m->d, kvs, p.iota1, BR, BR, m->L, m->H, dh,
+                                         scale, dR, ldR, 0, xR2, xr, s));
       }
       {
         SiteLabel s_xc("xattn.cand");
-        ROCS_TRY(launch_attention(h, p.QC, d2, 1, p.KC, p.VC, m->d, kvs, offsets, BR, BC, m->L, m->H, dh, scale, dC,
-                                  ldC, 0, xC2, xc, s));
+        ROCS_TRY(launch_attention_stream(h, p.QC, d2, 1, p.KC, p.VC, m->d, kvs, offsets, BR, BC, m->L, m->H, dh,
+                                         scale, dC, ldC, 0, xC2, xc, s));
       }
       if (m->dca_query_source == 0) {
         if (out->A_R)

@@ -22,6 +22,7 @@ namespace {
 constexpr int FM_WARPS = 4;
 constexpr int FM_RUN = 8;   // consecutive candidates per warp
 constexpr int LCB_OMAX_F = 8;
+constexpr int NC_MAX = 16;   // candidate embeddings per candidate handled by the fused pass
 
 __device__ __forceinline__ uint4 load8_as_bf16(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
 __device__ __forceinline__ uint4 load8_as_bf16(const float* p) {
@@ -144,7 +145,7 @@ __device__ __forceinline__ void load_feats<__nv_bfloat16, 4>(const __nv_bfloat16
 }
 
 template <typename TIN>
-__global__ void __launch_bounds__(FM_WARPS * 32) glm_cand_fused_kernel(
+__global__ void __launch_bounds__(FM_WARPS * 32, 4) glm_cand_fused_kernel(
     const TIN* __restrict__ E_R, const TIN* __restrict__ E_C, const int32_t* __restrict__ req_idx, int B_R,
     long long B_C, int n_R, int n_C, int trows, int pitch, __nv_bfloat16* __restrict__ F_C,
     const __nv_bfloat16* __restrict__ P_CC, int o_C, const float* __restrict__ ZL, float* __restrict__ L_C,
@@ -187,22 +188,28 @@ __global__ void __launch_bounds__(FM_WARPS * 32) glm_cand_fused_kernel(
 #pragma unroll
       for (int j = 0; j < DPL; ++j) acc[o][j] = 0.f;
     const TIN* ec = E_C + c * (long long)n_C * D;
-    for (int t = 0; t < n_C; ++t) {
-      float e[DPL];
-      load_feats<TIN, DPL>(ec + t * D + DPL * lane, e);
-      *reinterpret_cast<uint2*>(T + (n_R + t) * pitch + DPL * lane * 2) =
-          make_uint2(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]));
+    // issue every row load of this candidate before using any (n_C <= NC_MAX)
+    float e[NC_MAX][DPL];
 #pragma unroll
-      for (int o = 0; o < LCB_OMAX_F; ++o) {
-        if (o < o_C) {
-          const float p = sP[o * n_C + t];
+    for (int t = 0; t < NC_MAX; ++t)
+      if (t < n_C) load_feats<TIN, DPL>(ec + t * D + DPL * lane, e[t]);
 #pragma unroll
-          for (int j = 0; j < DPL; ++j) acc[o][j] = fmaf(p, e[j], acc[o][j]);
+    for (int t = 0; t < NC_MAX; ++t) {
+      if (t < n_C) {
+        *reinterpret_cast<uint2*>(T + (n_R + t) * pitch + DPL * lane * 2) =
+            make_uint2(pack_bf16x2(e[t][0], e[t][1]), pack_bf16x2(e[t][2], e[t][3]));
+#pragma unroll
+        for (int o = 0; o < LCB_OMAX_F; ++o) {
+          if (o < o_C) {
+            const float p = sP[o * n_C + t];
+#pragma unroll
+            for (int j = 0; j < DPL; ++j) acc[o][j] = fmaf(p, e[t][j], acc[o][j]);
+          }
         }
-      }
-      const float q = sQ[t];
+        const float q = sQ[t];
 #pragma unroll
-      for (int j = 0; j < DPL; ++j) qa[j] = fmaf(q, e[j], qa[j]);
+        for (int j = 0; j < DPL; ++j) qa[j] = fmaf(q, e[t][j], qa[j]);
+      }
     }
     // LCB output (fp32, float4 per token)
 #pragma unroll

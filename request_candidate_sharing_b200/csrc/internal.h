@@ -135,6 +135,18 @@ rocs_status launch_attention(rocs_context* ctx, const void* Q, long long ldq, in
                              long long rows, int L, int H, int d_h, float scale, void* O, long long ldo,
                              int out_bf16, void* O2, long long ldo2, cudaStream_t s);
 
+// Same contract as launch_attention.  _stream: K/V streamed through a small shared-memory ring
+// (any number of query rows per request); _single: one query row per request (a few at most),
+// K/V read straight from HBM (L <= 1024).
+rocs_status launch_attention_stream(rocs_context* ctx, const void* Q, long long ldq, int q_split, const void* K,
+                                    const void* V, long long ldkv, long long kv_req_stride, const int32_t* offsets,
+                                    int B_R, long long rows, int L, int H, int d_h, float scale, void* O,
+                                    long long ldo, int out_bf16, void* O2, long long ldo2, cudaStream_t s);
+rocs_status launch_attention_single(rocs_context* ctx, const void* Q, long long ldq, int q_split, const void* K,
+                                    const void* V, long long ldkv, long long kv_req_stride, const int32_t* offsets,
+                                    int B_R, long long rows, int L, int H, int d_h, float scale, void* O,
+                                    long long ldo, int out_bf16, void* O2, long long ldo2, cudaStream_t s);
+
 rocs_status launch_score_head(const void* X, long long ldx, long long rows, int K, const void* w,
                               const float* b, float* out, cudaStream_t s);
 

@@ -274,7 +274,8 @@ def test_token_lcb(R, o_R, o_C):
 # a9 cross-attention
 # ---------------------------------------------------------------------------------------------
 @pytest.mark.parametrize("L,H,dh,counts", [(200, 4, 64, [3, 0, 40, 17]), (1024, 8, 32, [33, 1]),
-                                           (5, 2, 32, [16, 2, 0]), (512, 1, 64, [70])])
+                                           (5, 2, 32, [16, 2, 0]), (512, 1, 64, [70]),
+                                           (1024, 8, 32, [300, 129, 0, 1000]), (200, 4, 64, [517, 2])])
 def test_cross_attention(R, L, H, dh, counts):
     counts = np.asarray(counts, np.int32)
     off, m = O.segments(counts)
