@@ -263,13 +263,24 @@ def dist_setup(n_gpus):
 
 
 def allreduce(x: float, op: str, world: int) -> float:
+    """Max or sum of a scalar over ranks (the measurement's only collective)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    device = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def shard_totals(workload: str, rank: int, world: int, requests: int, local_ms: float):
+    """Weak-scaling bookkeeping of one rank: its own request shard, the job-wide candidate total
+    and the max-over-ranks time that the throughput divides by."""
+    case = make_case(workload, rank, requests)
+    total = allreduce(float(case.B_C), "sum", world)
+    ms_max = allreduce(local_ms, "max", world)
+    return case.B_C, total, ms_max
 
 
 def barrier(world):
@@ -360,8 +371,8 @@ def run_librocs(args, rank, world, local):
     st = R.rocs_get_device_status(sh)
     if st != 0:
         raise RuntimeError(f"device status {rocs.STATUS_NAMES.get(st, st)} in the timed region")
-    ms_max = allreduce(ms, "max", world)
-    cands = allreduce(float(B_C) * args.steps, "sum", world)
+    _, total_c, ms_max = shard_totals(args.workload, rank, world, args.requests, ms)
+    cands = total_c * args.steps
     value = cands / (ms_max / 1e3)
 
     # ---- end-to-end through the same call with host buffers ----
