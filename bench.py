@@ -100,7 +100,9 @@ def algo_work(case, label: str):
         L, d, H = a.L, a.d, a.H
         table = {
             "enc.attn:attn": ("alu", float(B_R) * H * L * L),
+            "enc.attn:attn_tc": ("alu", float(B_R) * H * L * L),
             "xattn.cand:attn_stream": ("alu", float(B_C) * H * L),
+            "xattn.cand:attn_tc": ("alu", float(B_C) * H * L),
             "enc.qkv:gemm_tc": ("tensor", 2.0 * B_R * L * d * d * 3),
             "enc.kv:gemm_tc": ("tensor", 2.0 * B_R * L * d * d * 4),
             "enc.wo:gemm_tc": ("tensor", 2.0 * B_R * L * d * d),

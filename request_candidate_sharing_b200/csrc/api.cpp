@@ -132,6 +132,22 @@ rocs_status linear_bf16(rocs_context* ctx, const void* X, long long ldx, long lo
   return launch_gemm_bf16(ctx, &g, 1, s);
 }
 
+// Attention against per-request K/V: the tcgen05 kernel where its shared memory holds the
+// request's K/V, else the streaming (cross) or resident (self) mma.sync kernels.
+rocs_status attention_best(rocs_context* ctx, bool streaming_fallback, const void* Q, long long ldq, int q_split,
+                           const void* K, const void* V, long long ldkv, const int32_t* offsets, int B_R,
+                           long long rows, int L, int H, int d_h, float scale, void* O, long long ldo, int out_bf16,
+                           void* O2, long long ldo2, cudaStream_t s) {
+  rocs_status st = launch_attention_tc(ctx, Q, ldq, q_split, K, V, ldkv, (long long)B_R * L, offsets, B_R, rows, L, H,
+                                       d_h, scale, O, ldo, out_bf16, O2, ldo2, s);
+  if (st != ROCS_ERR_UNSUPPORTED) return st;
+  if (streaming_fallback)
+    return launch_attention_stream(ctx, Q, ldq, q_split, K, V, ldkv, (long long)L * ldkv, offsets, B_R, rows, L, H,
+                                   d_h, scale, O, ldo, out_bf16, O2, ldo2, s);
+  return launch_attention(ctx, Q, ldq, q_split, K, V, ldkv, (long long)L * ldkv, offsets, B_R, rows, L, H, d_h, scale,
+                          O, ldo, out_bf16, O2, ldo2, s);
+}
+
 // Workspace of rocs_linear_ikbo: Z, then (only if a row is not 16-B aligned) padded operands.
 struct IkboPlan {
   float* Z = nullptr;
@@ -412,8 +428,8 @@ extern "C" rocs_status rocs_dca_cross_attn(rocs_handle_t h, const void* Q, const
   ROCS_REQUIRE(out == ROCS_F32 || out == ROCS_BF16, "rocs_dca_cross_attn: bad dtype");
   ROCS_REQUIRE(std::isfinite(scale), "rocs_dca_cross_attn: scale not finite");
   const long long dm = (long long)H * d_h;
-  return launch_attention_stream(h, Q, dm, 0, K, V, dm, (long long)L * dm, offsets, B_R, rows, L, H, d_h, scale, O,
-                                 ld_O, out == ROCS_BF16, nullptr, 0, (cudaStream_t)stream);
+  return attention_best(h, true, Q, dm, 0, K, V, dm, offsets, B_R, rows, L, H, d_h, scale, O, ld_O, out == ROCS_BF16,
+                        nullptr, 0, (cudaStream_t)stream);
 }
 
 // =============================================================================================
@@ -456,8 +472,8 @@ rocs_status encoder_layer(rocs_context* ctx, const EncScratch& e, int B_R, int L
   SiteLabel sl0("enc.qkv");
   ROCS_TRY(launch_gemm_bf16(ctx, g, 3, s));
   SiteLabel sl1("enc.attn");
-  ROCS_TRY(launch_attention(ctx, e.q, d, 0, e.k, e.v, d, (long long)L * d, e.self_off, B_R, M, L, H, d / H,
-                            1.0f / std::sqrt((float)(d / H)), e.att, d, 1, nullptr, 0, s));
+  ROCS_TRY(attention_best(ctx, false, e.q, d, 0, e.k, e.v, d, e.self_off, B_R, M, L, H, d / H,
+                          1.0f / std::sqrt((float)(d / H)), e.att, d, 1, nullptr, 0, s));
   SiteLabel sl2("enc.wo");
   ROCS_TRY(linear_bf16(ctx, e.att, d, M, d, w.Wo, d, nullptr, e.tmp, d, 1, ROCS_ACT_NONE, s));
   SiteLabel sl3("enc.ln");
@@ -851,8 +867,8 @@ extern "C" rocs_status rocs_forward(rocs_handle_t h, const rocs_model_desc* m, c
       }
       {
         SiteLabel s_xc("xattn.cand");
-        ROCS_TRY(launch_attention_stream(h, p.QC, d2, 1, p.KC, p.VC, m->d, kvs, offsets, BR, BC, m->L, m->H, dh,
-                                         scale, dC, ldC, 0, xC2, xc, s));
+        ROCS_TRY(attention_best(h, true, p.QC, d2, 1, p.KC, p.VC, m->d, offsets, BR, BC, m->L, m->H, dh, scale, dC,
+                                ldC, 0, xC2, xc, s));
       }
       if (m->dca_query_source == 0) {
         if (out->A_R)

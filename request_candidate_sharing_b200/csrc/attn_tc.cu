@@ -1,0 +1,493 @@
+// a7/a9: attention against per-request shared K/V on the 5th-generation tensor cores.
+//
+// [REV] §2.2: S_i and its K/V are computed once per request and every query of that request
+// (the request's own history positions for the encoder, its candidates for the grouped
+// cross-attention) reads the same K/V; [REV] §2.4 (IKBO-DCA): the kernel consumes request-batch
+// K/V directly, never a per-candidate copy.
+//
+// One CTA per (request, head), three warpgroups (384 threads):
+//   warp 0      TMA: the head's K and V (L x d_h bf16) into shared memory ONCE, in 128-key blocks
+//               with one mbarrier each (compute starts when block 0 lands); 128-row query tiles
+//               (bf16, or a hi/lo pair), one per softmax warpgroup.
+//   warp 1      allocates TMEM; one thread issues, for both query tiles in flight and each
+//               128-key block j,
+//                 S_j = Q K_j^T       (tcgen05.mma M=128, N=128, K=d_h; one S buffer per tile)
+//                 O  += P_j V_j       (M=128, N=d_h, K=128; V read as an MN-major operand; O
+//                                      accumulates in TMEM across the key blocks)
+//               issuing both tiles' S blocks before it waits on either tile's P, so one tile's
+//               exponentials overlap the other tile's tensor-core work.
+//   warps 4..11 two softmax warpgroups, one thread per query row (TMEM lane): the S row is read
+//               from TMEM in one batch, its maximum and exp2 taken in registers (no shuffles), P_j
+//               written as bf16 to shared memory (128-byte swizzle, K-major).  The row's reference
+//               maximum moves only when a block exceeds it by more than 2^8 (then the warp rescales
+//               its O rows in TMEM); at the end O is read once and divided by the row sum.
+//   setmaxnreg moves registers from the producer warpgroup (40) to the softmax warpgroups (224).
+// All waits are bounded; a wait that runs out sets ROCS_ERR_DEVICE_TIMEOUT and the CTA unwinds
+// (in-flight copies and MMAs drained, TMEM released) instead of spinning.
+#include "common.cuh"
+#include "internal.h"
+
+namespace rocs {
+namespace {
+
+constexpr int TQ = 128;    // query rows per tile (MMA M)
+constexpr int TK = 128;    // keys per block
+constexpr int AT_TMEM_COLS = 512;
+constexpr int AT_MAX_KB = 8;   // L <= 1024
+
+struct AttnTcParams {
+  CUtensorMap tmQ;   // queries [rows, cols] bf16: box {d_h, 128}
+  CUtensorMap tmK;   // keys    [B_R * L, H * d_h]: box {d_h, 128}
+  CUtensorMap tmV;   // values  same layout
+  const int32_t* offsets;
+  long long rows;
+  int B_R, H, L, nkb;
+  long long q_lo_col;   // column of the low half in a query row (hi/lo queries)
+  float scale_log2;
+  void* O;
+  long long ldo;
+  int out_bf16;
+  __nv_bfloat16* O2;
+  long long ldo2;
+  int* status;
+};
+
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (b_mn_major ? (1u << 16) : 0u) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+// Shared-memory matrix descriptor: swizzle `layout` (2 = 128 B, 4 = 64 B), stride between 8-row
+// groups `sbo` bytes.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t sbo, uint32_t layout) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(sbo >> 4) << 32) | ((uint64_t)1 << 46) |
+         ((uint64_t)layout << 61);
+}
+
+__device__ __forceinline__ void fence_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// A row's running maximum is only moved when a block's maximum exceeds it by more than this
+// (log2 units): exponentials stay <= 2^8, and the O accumulator in TMEM is rescaled rarely.
+constexpr float kLazyRescaleLog2 = 8.0f;
+
+// GROUPS query tiles are in flight per CTA (two softmax warpgroups for d_h = 32), each with its
+// own S and O accumulators in TMEM and its own P tile in shared memory; the MMA thread issues
+// both groups' S blocks before it waits on either group's P, so one group's exponentials overlap
+// the other's tensor-core work.
+template <int DH, bool SPLIT, int GROUPS>
+__global__ void __launch_bounds__(128 + 128 * GROUPS, 1) attn_tc_kernel(const __grid_constant__ AttnTcParams P) {
+  constexpr int ROWB = DH * 2;                        // bytes per K/V/Q row
+  constexpr uint32_t SW = DH == 32 ? 4u : 2u;         // 64-B or 128-B swizzle for K/V/Q
+  constexpr uint32_t SBO = 8 * ROWB;                  // 8-row group stride
+  constexpr int KV_BLOCK = TK * ROWB;                 // bytes of one 128-key block
+  constexpr int Q_TILE = TQ * ROWB;
+  constexpr int NQ = SPLIT ? 2 : 1;
+  constexpr int P_TILE = TQ * TK * 2;                 // 32 KiB, two 64-key sub-tiles of 16 KiB
+  constexpr uint32_t IDESC_S = idesc_bf16(TQ, TK, false);
+  constexpr uint32_t IDESC_O = idesc_bf16(TQ, DH, true);
+  constexpr uint32_t O_COL0 = GROUPS * TK;            // S of group G at G*TK, O at O_COL0 + G*DH
+
+  const int r = blockIdx.x / P.H;
+  const int h = blockIdx.x - r * P.H;
+  const long long q0 = P.offsets[r], q1 = P.offsets[r + 1];
+  if (q0 < 0 || q1 < q0 || q1 > P.rows) {
+    if (threadIdx.x == 0) set_status(P.status, ROCS_ERR_INDEX);
+    return;
+  }
+  const int ntiles = (int)((q1 - q0 + TQ - 1) / TQ);
+  if (ntiles == 0) return;
+  const int nkb = P.nkb;
+
+  extern __shared__ uint8_t at_smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(at_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = base;
+  uint8_t* sV = sK + nkb * KV_BLOCK;
+  uint8_t* sQ = sV + nkb * KV_BLOCK;                  // [GROUPS][NQ][Q_TILE]
+  uint8_t* sP = sQ + GROUPS * NQ * Q_TILE;            // [GROUPS][P_TILE]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + GROUPS * P_TILE);
+  uint64_t* kv_full = bars;                           // [AT_MAX_KB]
+  uint64_t* q_full = kv_full + AT_MAX_KB;             // [GROUPS] each
+  uint64_t* q_free = q_full + GROUPS;
+  uint64_t* s_full = q_free + GROUPS;
+  uint64_t* s_free = s_full + GROUPS;
+  uint64_t* p_full = s_free + GROUPS;
+  uint64_t* o_full = p_full + GROUPS;
+  uint64_t* drain = o_full + GROUPS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < AT_MAX_KB; ++i) mbar_init(&kv_full[i], 1);
+    for (int g = 0; g < GROUPS; ++g) {
+      mbar_init(&q_full[g], 1);
+      mbar_init(&q_free[g], 1);
+      mbar_init(&s_full[g], 1);
+      mbar_init(&s_free[g], TQ);
+      mbar_init(&p_full[g], TQ);
+      mbar_init(&o_full[g], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, AT_TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  // group G takes tiles G, G + GROUPS, ...; its sequence has tiles_g(G) * nkb key blocks
+  auto tiles_g = [&](int g) { return ntiles > g ? (ntiles - g + GROUPS - 1) / GROUPS : 0; };
+
+  // registers move from the producer/MMA warpgroup to the softmax warpgroups:
+  // 128 x 40 + 128 * GROUPS x 224 <= (128 + 128 * GROUPS) x 168, the block's launch allocation
+  static_assert(128 * 40 + 128 * GROUPS * 224 <= (128 + 128 * GROUPS) * 168, "register split");
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
+    if (warp == 0 && lane == 0) {
+      // ---------------- TMA producer ----------------
+      prefetch_tensormap(&P.tmQ);
+      prefetch_tensormap(&P.tmK);
+      prefetch_tensormap(&P.tmV);
+      const int kv_row0 = r * P.L;
+      for (int j = 0; j < nkb; ++j) {
+        mbar_arrive_expect_tx(&kv_full[j], 2 * KV_BLOCK);
+        tma_load_2d(sK + j * KV_BLOCK, &P.tmK, &kv_full[j], h * DH, kv_row0 + j * TK);
+        tma_load_2d(sV + j * KV_BLOCK, &P.tmV, &kv_full[j], h * DH, kv_row0 + j * TK);
+      }
+      int last_k[GROUPS];
+      for (int g = 0; g < GROUPS; ++g) last_k[g] = -1;
+      bool ok = true;
+      for (int t = 0; t < ntiles && ok; ++t) {
+        const int g = t % GROUPS, k = t / GROUPS;
+        if (k > 0 && !mbar_wait(&q_free[g], (k - 1) & 1, P.status, abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(&q_full[g], NQ * Q_TILE);
+        const int qrow = (int)(q0 + (long long)t * TQ);
+        tma_load_2d(sQ + (g * NQ) * Q_TILE, &P.tmQ, &q_full[g], h * DH, qrow);
+        if (SPLIT) tma_load_2d(sQ + (g * NQ + 1) * Q_TILE, &P.tmQ, &q_full[g], (int)P.q_lo_col + h * DH, qrow);
+        last_k[g] = k;
+      }
+      // no copy of this CTA may still be landing when it exits
+      for (int j = 0; j < nkb; ++j) mbar_wait(&kv_full[j], 0, P.status, nullptr);
+      for (int g = 0; g < GROUPS; ++g)
+        if (last_k[g] >= 0) mbar_wait(&q_full[g], last_k[g] & 1, P.status, nullptr);
+    } else if (warp == 1 && lane == 0) {
+      // ---------------- MMA issuer ----------------
+      int T[GROUPS];
+      int Tmax = 0;
+      for (int g = 0; g < GROUPS; ++g) {
+        T[g] = tiles_g(g) * nkb;
+        Tmax = T[g] > Tmax ? T[g] : Tmax;
+      }
+      bool ok = true;
+      for (int i = 0; i <= Tmax && ok; ++i) {
+        // S_i of every group first ...
+        for (int g = 0; g < GROUPS && ok; ++g) {
+          if (i >= T[g]) continue;
+          const int k = i / nkb, j = i - k * nkb;
+          if (j == 0 && !mbar_wait(&q_full[g], k & 1, P.status, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&kv_full[j], 0, P.status, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&s_free[g], (i & 1) ^ 1, P.status, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t qa = smem_u32(sQ + (g * NQ) * Q_TILE);
+          const uint32_t ka = smem_u32(sK + j * KV_BLOCK);
+#pragma unroll
+          for (int ks = 0; ks < DH / 16; ++ks) {
+            tc_mma_ss(tmem_base + g * TK, sdesc(qa + ks * 32, SBO, SW), sdesc(ka + ks * 32, SBO, SW), IDESC_S,
+                      ks > 0 ? 1u : 0u);
+            if (SPLIT)
+              tc_mma_ss(tmem_base + g * TK, sdesc(qa + Q_TILE + ks * 32, SBO, SW), sdesc(ka + ks * 32, SBO, SW),
+                        IDESC_S, 1u);
+          }
+          tc_commit(&s_full[g]);
+          if (j == nkb - 1) tc_commit(&q_free[g]);   // this tile's queries are no longer read
+        }
+        // ... then P_{i-1} V_{i-1} of every group
+        for (int g = 0; g < GROUPS && ok; ++g) {
+          if (i < 1 || i > T[g]) continue;
+          const int jb = (i - 1) % nkb;
+          if (!mbar_wait(&p_full[g], (i - 1) & 1, P.status, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t pa = smem_u32(sP + g * P_TILE);
+          const uint32_t va = smem_u32(sV + jb * KV_BLOCK);
+#pragma unroll
+          for (int ks = 0; ks < TK / 16; ++ks) {
+            const uint64_t adesc = sdesc(pa + (ks >> 2) * (TQ * 128) + (ks & 3) * 32, 1024, 2);
+            const uint64_t bdesc = sdesc(va + ks * 16 * ROWB, SBO, SW);
+            tc_mma_ss(tmem_base + O_COL0 + g * DH, adesc, bdesc, IDESC_O, (ks > 0 || jb > 0) ? 1u : 0u);
+          }
+          tc_commit(&o_full[g]);
+        }
+      }
+      tc_commit(drain);
+      mbar_wait(drain, 0, P.status, nullptr);
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 224;");
+    // ---------------- softmax warpgroups: thread = query row = TMEM lane ----------------
+    const int g = (warp - 4) >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t saddr = lane_addr + g * TK;
+    const uint32_t oaddr = lane_addr + O_COL0 + g * DH;
+    uint8_t* prow = sP + g * P_TILE + row * 128;
+    const int Tg = tiles_g(g) * nkb;
+    float m_cur = -INFINITY, l_sum = 0.f;
+
+    // O accumulator of the finished tile k_tile, divided by its row sum, to global memory
+    auto emit_row = [&](int k_tile, float l_final) {
+      float out[DH];
+#pragma unroll
+      for (int c = 0; c < DH / 32; ++c) {
+        uint32_t w[32];
+        tmem_ld_32x32b_x32(oaddr + c * 32, w);
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) out[c * 32 + k] = __uint_as_float(w[k]);
+      }
+      const long long qrow = q0 + (long long)(g + GROUPS * k_tile) * TQ + row;
+      if (qrow >= q1) return;
+      const float inv = 1.0f / l_final;
+#pragma unroll
+      for (int e = 0; e < DH; ++e) out[e] *= inv;
+      if (P.out_bf16) {
+        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(P.O) + qrow * P.ldo + h * DH;
+#pragma unroll
+        for (int e = 0; e < DH; e += 8)
+          *reinterpret_cast<uint4*>(o + e) = make_uint4(pack_bf16x2(out[e], out[e + 1]), pack_bf16x2(out[e + 2], out[e + 3]),
+                                                       pack_bf16x2(out[e + 4], out[e + 5]), pack_bf16x2(out[e + 6], out[e + 7]));
+      } else {
+        float* o = reinterpret_cast<float*>(P.O) + qrow * P.ldo + h * DH;
+#pragma unroll
+        for (int e = 0; e < DH; e += 4) *reinterpret_cast<float4*>(o + e) = make_float4(out[e], out[e + 1], out[e + 2], out[e + 3]);
+      }
+      if (P.O2 != nullptr) {
+        __nv_bfloat16* o = P.O2 + qrow * P.ldo2 + h * DH;
+#pragma unroll
+        for (int e = 0; e < DH; e += 8)
+          *reinterpret_cast<uint4*>(o + e) = make_uint4(pack_bf16x2(out[e], out[e + 1]), pack_bf16x2(out[e + 2], out[e + 3]),
+                                                       pack_bf16x2(out[e + 4], out[e + 5]), pack_bf16x2(out[e + 6], out[e + 7]));
+      }
+    };
+
+    bool ok = true;
+    for (int i = 0; i < Tg; ++i) {
+      const int k_tile = i / nkb, j = i - k_tile * nkb;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[g], i & 1, P.status, abort_flag))) { ok = false; break; }
+      tc_fence_after();
+      // the whole S row into registers with one wait, then the S accumulator is released
+      uint32_t v[TK / 32][32];
+      __syncwarp();
+#pragma unroll
+      for (int c = 0; c < TK / 32; ++c) tmem_ld_32x32b_x32(saddr + c * 32, v[c]);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&s_free[g]);
+      if ((j + 1) * TK > P.L) {
+#pragma unroll
+        for (int c = 0; c < TK / 32; ++c)
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            if (j * TK + c * 32 + k >= P.L) v[c][k] = __float_as_uint(-INFINITY);
+      }
+      // row maximum as a tree (eight independent chains)
+      float mt[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) mt[t] = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < TK / 32; ++c)
+#pragma unroll
+        for (int k = 0; k < 32; ++k) mt[k & 7] = fmaxf(mt[k & 7], __uint_as_float(v[c][k]));
+      const float mx = fmaxf(fmaxf(fmaxf(mt[0], mt[1]), fmaxf(mt[2], mt[3])), fmaxf(fmaxf(mt[4], mt[5]), fmaxf(mt[6], mt[7]))) *
+                       P.scale_log2;
+      // the first block sets the row's reference maximum; later blocks move it only when some
+      // row of the warp would otherwise produce exponentials above 2^8 (warp-uniform, since the
+      // O rescale below is a warp-wide TMEM access)
+      float m_new = m_cur, corr = 1.0f;
+      bool rescale = false;
+      if (j == 0) {
+        m_new = mx;
+      } else if (__any_sync(0xffffffffu, mx > m_cur + kLazyRescaleLog2)) {
+        m_new = fmaxf(m_cur, mx);
+        corr = ex2_approx(m_cur - m_new);
+        rescale = true;
+      }
+      float rs[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[TK / 2];
+#pragma unroll
+      for (int c = 0; c < TK / 32; ++c)
+#pragma unroll
+        for (int k = 0; k < 32; k += 2) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(v[c][k]), P.scale_log2, -m_new));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(v[c][k + 1]), P.scale_log2, -m_new));
+          rs[(k >> 1) & 3] += p0 + p1;
+          pk[(c * 32 + k) >> 1] = pack_bf16x2(p0, p1);
+        }
+      const float rsum = (rs[0] + rs[1]) + (rs[2] + rs[3]);
+      // the previous block's P V has completed: the P tile may be overwritten and the O
+      // accumulator read (finished tile) or rescaled
+      if (i > 0) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&o_full[g], (i - 1) & 1, P.status, abort_flag))) { ok = false; break; }
+        tc_fence_after();
+        if (j == 0) {
+          emit_row(k_tile - 1, l_sum);
+        } else if (rescale) {
+#pragma unroll
+          for (int c = 0; c < DH / 32; ++c) {
+            uint32_t w[32];
+            tmem_ld_32x32b_x32(oaddr + c * 32, w);
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) w[k] = __float_as_uint(__uint_as_float(w[k]) * corr);
+            tmem_st_32x32b_x32(oaddr + c * 32, w);
+          }
+          tmem_st_wait();
+        }
+      }
+      // P_i as bf16, K-major with a 128-byte swizzle (two 64-key sub-tiles)
+#pragma unroll
+      for (int q = 0; q < TK / 8; ++q) {
+        const int chunk = q & 7;
+        *reinterpret_cast<uint4*>(prow + (q >> 3) * (TQ * 128) + ((chunk ^ (row & 7)) << 4)) =
+            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+      }
+      fence_async_shared();
+      tc_fence_before();
+      mbar_arrive(&p_full[g]);
+      l_sum = j == 0 ? rsum : fmaf(l_sum, corr, rsum);
+      m_cur = m_new;
+    }
+    if (ok && Tg > 0 && __all_sync(0xffffffffu, mbar_wait(&o_full[g], (Tg - 1) & 1, P.status, abort_flag))) {
+      tc_fence_after();
+      emit_row(Tg / nkb - 1, l_sum);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, AT_TMEM_COLS);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+bool encode_rows(rocs_context* ctx, CUtensorMap* map, const void* ptr, long long rows, long long cols, long long ld,
+                 int dh) {
+  EncodeTiledFn fn = reinterpret_cast<EncodeTiledFn>(ctx->encode_fn);
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)dh, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, dh == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int DH, bool SPLIT, int GROUPS>
+size_t at_smem_bytes(int nkb) {
+  return 1024 + (size_t)2 * nkb * TK * DH * 2 + (size_t)GROUPS * (SPLIT ? 2 : 1) * TQ * DH * 2 +
+         (size_t)GROUPS * TQ * TK * 2 + (AT_MAX_KB + 6 * GROUPS + 1) * 8 + 16;
+}
+
+template <int DH, bool SPLIT, int GROUPS>
+rocs_status at_launch(rocs_context* ctx, AttnTcParams& P, int B_R, int H, cudaStream_t s) {
+  const size_t smem = at_smem_bytes<DH, SPLIT, GROUPS>(P.nkb);
+  if (smem > 232448) {
+    set_error("tcgen05 attention: L=%d needs %zu B of shared memory", P.L, smem);
+    return ROCS_ERR_UNSUPPORTED;
+  }
+  static bool attr[64] = {false};
+  if (ctx->device < 64 && !attr[ctx->device]) {
+    rocs_status st = cuda_check(
+        cudaFuncSetAttribute(attn_tc_kernel<DH, SPLIT, GROUPS>, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448),
+        "cudaFuncSetAttribute(attn_tc)");
+    if (st != ROCS_OK) return st;
+    // the softmax warpgroups raise their register limit out of the block's launch allocation;
+    // refuse to launch if the compiled kernel was given fewer registers than that split needs
+    cudaFuncAttributes fa;
+    st = cuda_check(cudaFuncGetAttributes(&fa, attn_tc_kernel<DH, SPLIT, GROUPS>), "cudaFuncGetAttributes(attn_tc)");
+    if (st != ROCS_OK) return st;
+    if ((long long)fa.numRegs * (128 + 128 * GROUPS) < 128LL * 40 + 128LL * GROUPS * 224) {
+      set_error("tcgen05 attention: kernel compiled with %d registers per thread, below the warpgroup split",
+                fa.numRegs);
+      return ROCS_ERR_UNSUPPORTED;
+    }
+    attr[ctx->device] = true;
+  }
+  attn_tc_kernel<DH, SPLIT, GROUPS><<<(unsigned)((long long)B_R * H), 128 + 128 * GROUPS, smem, s>>>(P);
+  return cuda_check(cudaGetLastError(), "attn_tc_kernel");
+}
+
+}  // namespace
+
+rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq, int q_split, const void* K,
+                                const void* V, long long ldkv, long long kv_rows, const int32_t* offsets, int B_R,
+                                long long rows, int L, int H, int d_h, float scale, void* O, long long ldo,
+                                int out_bf16, void* O2, long long ldo2, cudaStream_t s) {
+  if (B_R == 0 || rows == 0) return ROCS_OK;
+  if ((d_h != 32 && d_h != 64) || L < 1 || (long long)L * d_h > 32768 || (L + TK - 1) / TK > AT_MAX_KB ||
+      ((uintptr_t)Q & 15) || ((uintptr_t)K & 15) || ((uintptr_t)V & 15) || ldq % 8 || ldkv % 8 ||
+      (q_split && (ldq < 2LL * H * d_h)) || ldkv < (long long)H * d_h || ((uintptr_t)O & 15) ||
+      (O2 && ((uintptr_t)O2 & 15)) || ldo % 8 || (O2 && ldo2 % 8)) {
+    set_error("tcgen05 attention: unsupported shape or alignment (d_h=%d L=%d)", d_h, L);
+    return ROCS_ERR_UNSUPPORTED;
+  }
+  AttnTcParams P;
+  memset(&P, 0, sizeof(P));
+  const long long qcols = q_split ? 2LL * H * d_h : (long long)H * d_h;
+  if (!encode_rows(ctx, &P.tmQ, Q, rows, qcols, ldq, d_h) || !encode_rows(ctx, &P.tmK, K, kv_rows, (long long)H * d_h, ldkv, d_h) ||
+      !encode_rows(ctx, &P.tmV, V, kv_rows, (long long)H * d_h, ldkv, d_h)) {
+    set_error("tcgen05 attention: cuTensorMapEncodeTiled failed");
+    return ROCS_ERR_CUDA;
+  }
+  P.offsets = offsets;
+  P.rows = rows;
+  P.B_R = B_R;
+  P.H = H;
+  P.L = L;
+  P.nkb = (L + TK - 1) / TK;
+  P.q_lo_col = (long long)H * d_h;
+  P.scale_log2 = scale * 1.4426950408889634f;
+  P.O = O;
+  P.ldo = ldo;
+  P.out_bf16 = out_bf16;
+  P.O2 = (__nv_bfloat16*)O2;
+  P.ldo2 = ldo2;
+  P.status = ctx->d_status;
+  LaunchTimer lt_("attn_tc", s);
+  if (d_h == 32)
+    return q_split ? at_launch<32, true, 2>(ctx, P, B_R, H, s) : at_launch<32, false, 2>(ctx, P, B_R, H, s);
+  return q_split ? at_launch<64, true, 2>(ctx, P, B_R, H, s) : at_launch<64, false, 2>(ctx, P, B_R, H, s);
+}
+
+}  // namespace rocs

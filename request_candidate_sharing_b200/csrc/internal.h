@@ -147,6 +147,14 @@ rocs_status launch_attention_single(rocs_context* ctx, const void* Q, long long 
                                     int B_R, long long rows, int L, int H, int d_h, float scale, void* O,
                                     long long ldo, int out_bf16, void* O2, long long ldo2, cudaStream_t s);
 
+// tcgen05/TMEM attention (one CTA per (request, head), K/V resident in shared memory): d_h 32
+// (L <= 1024) or 64 (L <= 256 with hi/lo queries, 512 without).  kv_rows = rows of K/V (B_R * L).
+// Returns ROCS_ERR_UNSUPPORTED, launching nothing, for shapes outside that range.
+rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq, int q_split, const void* K,
+                                const void* V, long long ldkv, long long kv_rows, const int32_t* offsets, int B_R,
+                                long long rows, int L, int H, int d_h, float scale, void* O, long long ldo,
+                                int out_bf16, void* O2, long long ldo2, cudaStream_t s);
+
 rocs_status launch_score_head(const void* X, long long ldx, long long rows, int K, const void* w,
                               const float* b, float* out, cudaStream_t s);
 
