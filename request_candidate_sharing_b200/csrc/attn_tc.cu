@@ -64,7 +64,6 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t sbo, uint32_t
          ((uint64_t)layout << 61);
 }
 
-__device__ __forceinline__ void fence_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 __device__ __forceinline__ void tc_mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
@@ -87,26 +86,111 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]: the A operand (M rows in TMEM lanes, two bf16 of K per column)
+// is read from tensor memory.
+__device__ __forceinline__ void tc_mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_32x32b_x1(uint32_t taddr, uint32_t& r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st_32x32b_x1(uint32_t taddr, uint32_t r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(r) : "memory");
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// (a0, a1) * (b, b) + (c, c) on the packed fp32x2 FMA path.
+__device__ __forceinline__ void ffma2(float a0, float a1, float b, float c, float& d0, float& d1) {
+  uint64_t av, bv, cv, dv;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(av) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(bv) : "f"(b));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(cv) : "f"(c));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(dv) : "l"(av), "l"(bv), "l"(cv));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d0), "=f"(d1) : "l"(dv));
+}
+
+__device__ __forceinline__ uint64_t dup2(float c) {
+  uint64_t v;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(v) : "f"(c));
+  return v;
+}
+
+// 2^x0, 2^x1 on the FMA pipe: x = n + f with n = round(x) by the 1.5 * 2^23 shifter, 2^f by a
+// degree-3 minimax polynomial on [-1/2, 1/2] (max relative error 7.5e-5, coefficients from
+// gen_exp2_poly.py), 2^n added into the exponent field.  Arguments are clamped to [-126, 126].
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+  x0 = fminf(fmaxf(x0, -126.0f), 126.0f);
+  x1 = fminf(fmaxf(x1, -126.0f), 126.0f);
+  uint64_t xv, tv, nv, fv, pv;
+  const uint64_t shifter = dup2(12582912.0f);   // 1.5 * 2^23 in both halves
+  asm("mov.b64 %0, {%1, %2};" : "=l"(xv) : "f"(x0), "f"(x1));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(tv) : "l"(xv), "l"(shifter));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(nv) : "l"(tv), "l"(shifter));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(fv) : "l"(xv), "l"(nv));
+  const uint64_t c3 = dup2(0.0551716685f), c2 = dup2(0.242611125f), c1 = dup2(0.693260968f), c0 = dup2(0.999928057f);
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(pv) : "l"(c3), "l"(fv), "l"(c2));
+  asm("fma.rn.f32x2 %0, %0, %1, %2;" : "+l"(pv) : "l"(fv), "l"(c1));
+  asm("fma.rn.f32x2 %0, %0, %1, %2;" : "+l"(pv) : "l"(fv), "l"(c0));
+  uint32_t t0, t1, p0, p1;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(t0), "=r"(t1) : "l"(tv));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(p0), "=r"(p1) : "l"(pv));
+  // the shifter's low 9 bits are zero, so (bits(t) << 23) is exactly n << 23
+  y0 = __uint_as_float(p0 + (t0 << 23));
+  y1 = __uint_as_float(p1 + (t1 << 23));
+}
+
 // A row's running maximum is only moved when a block's maximum exceeds it by more than this
 // (log2 units): exponentials stay <= 2^8, and the O accumulator in TMEM is rescaled rarely.
 constexpr float kLazyRescaleLog2 = 8.0f;
 
-// GROUPS query tiles are in flight per CTA (two softmax warpgroups for d_h = 32), each with its
-// own S and O accumulators in TMEM and its own P tile in shared memory; the MMA thread issues
-// both groups' S blocks before it waits on either group's P, so one group's exponentials overlap
-// the other's tensor-core work.
-template <int DH, bool SPLIT, int GROUPS>
-__global__ void __launch_bounds__(128 + 128 * GROUPS, 1) attn_tc_kernel(const __grid_constant__ AttnTcParams P) {
+template <int DH>
+struct AtCfg {
+  static constexpr int GROUPS = 2;                   // query tiles in flight
+  static constexpr bool SUM_MMA = DH == 32;          // row sums by an MMA of P against ones
+  static constexpr int THREADS = 128 + 128 * GROUPS;
+  static constexpr int REG_LAUNCH = 168;
+  static constexpr int REG_CTRL = 72;                // producer / MMA warpgroup after setmaxnreg.dec
+  static constexpr int REG_SOFTMAX = 216;
+  static_assert(128 * REG_CTRL + 128 * GROUPS * REG_SOFTMAX <= THREADS * REG_LAUNCH, "register split");
+  // tensor memory: S (128 fp32 columns) | P (64 columns of bf16 pairs) | O (DH) | row sum (16)
+  static constexpr int S_COL = 0, P_COL = GROUPS * 128, O_COL = P_COL + GROUPS * 64,
+                       L_COL = O_COL + GROUPS * DH;
+  static_assert(L_COL + (SUM_MMA ? GROUPS * 16 : 0) <= 512, "tensor memory columns");
+};
+
+template <int DH, bool SPLIT>
+__global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __grid_constant__ AttnTcParams P) {
+  using C = AtCfg<DH>;
+  constexpr int GROUPS = C::GROUPS;
   constexpr int ROWB = DH * 2;                        // bytes per K/V/Q row
   constexpr uint32_t SW = DH == 32 ? 4u : 2u;         // 64-B or 128-B swizzle for K/V/Q
   constexpr uint32_t SBO = 8 * ROWB;                  // 8-row group stride
   constexpr int KV_BLOCK = TK * ROWB;                 // bytes of one 128-key block
   constexpr int Q_TILE = TQ * ROWB;
   constexpr int NQ = SPLIT ? 2 : 1;
-  constexpr int P_TILE = TQ * TK * 2;                 // 32 KiB, two 64-key sub-tiles of 16 KiB
+  constexpr int ONES_BYTES = 2048;                    // 16 rows x 64 bf16 ones (128-byte rows)
   constexpr uint32_t IDESC_S = idesc_bf16(TQ, TK, false);
   constexpr uint32_t IDESC_O = idesc_bf16(TQ, DH, true);
-  constexpr uint32_t O_COL0 = GROUPS * TK;            // S of group G at G*TK, O at O_COL0 + G*DH
+  constexpr uint32_t IDESC_L = idesc_bf16(TQ, 16, false);
 
   const int r = blockIdx.x / P.H;
   const int h = blockIdx.x - r * P.H;
@@ -124,17 +208,17 @@ __global__ void __launch_bounds__(128 + 128 * GROUPS, 1) attn_tc_kernel(const __
   uint8_t* sK = base;
   uint8_t* sV = sK + nkb * KV_BLOCK;
   uint8_t* sQ = sV + nkb * KV_BLOCK;                  // [GROUPS][NQ][Q_TILE]
-  uint8_t* sP = sQ + GROUPS * NQ * Q_TILE;            // [GROUPS][P_TILE]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + GROUPS * P_TILE);
+  uint8_t* sOnes = sQ + GROUPS * NQ * Q_TILE;         // 1024-B aligned (Q tiles are 8 KiB multiples)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOnes + ONES_BYTES);
   uint64_t* kv_full = bars;                           // [AT_MAX_KB]
   uint64_t* q_full = kv_full + AT_MAX_KB;             // [GROUPS] each
   uint64_t* q_free = q_full + GROUPS;
   uint64_t* s_full = q_free + GROUPS;
   uint64_t* s_free = s_full + GROUPS;
-  uint64_t* p_full = s_free + GROUPS;
-  uint64_t* o_full = p_full + GROUPS;
-  uint64_t* drain = o_full + GROUPS;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* p_full = s_free + GROUPS;                 // [GROUPS][2]: P half h of the block written
+  uint64_t* o_full = p_full + 2 * GROUPS;             // [GROUPS][2]: P half h times V consumed
+  uint64_t* drain = o_full + 2 * GROUPS;              // [GROUPS]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + GROUPS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -145,12 +229,18 @@ __global__ void __launch_bounds__(128 + 128 * GROUPS, 1) attn_tc_kernel(const __
       mbar_init(&q_free[g], 1);
       mbar_init(&s_full[g], 1);
       mbar_init(&s_free[g], TQ);
-      mbar_init(&p_full[g], TQ);
-      mbar_init(&o_full[g], 1);
+      for (int hh = 0; hh < 2; ++hh) {
+        mbar_init(&p_full[2 * g + hh], TQ);
+        mbar_init(&o_full[2 * g + hh], 1);
+      }
+      mbar_init(&drain[g], 1);
     }
-    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
+  }
+  if (C::SUM_MMA && threadIdx.x < ONES_BYTES / 16) {
+    reinterpret_cast<uint4*>(sOnes)[threadIdx.x] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, AT_TMEM_COLS);
@@ -163,11 +253,8 @@ __global__ void __launch_bounds__(128 + 128 * GROUPS, 1) attn_tc_kernel(const __
   // group G takes tiles G, G + GROUPS, ...; its sequence has tiles_g(G) * nkb key blocks
   auto tiles_g = [&](int g) { return ntiles > g ? (ntiles - g + GROUPS - 1) / GROUPS : 0; };
 
-  // registers move from the producer/MMA warpgroup to the softmax warpgroups:
-  // 128 x 40 + 128 * GROUPS x 224 <= (128 + 128 * GROUPS) x 168, the block's launch allocation
-  static_assert(128 * 40 + 128 * GROUPS * 224 <= (128 + 128 * GROUPS) * 168, "register split");
   if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REG_CTRL));
     if (warp == 0 && lane == 0) {
       // ---------------- TMA producer ----------------
       prefetch_tensormap(&P.tmQ);
@@ -179,88 +266,87 @@ __global__ void __launch_bounds__(128 + 128 * GROUPS, 1) attn_tc_kernel(const __
         tma_load_2d(sK + j * KV_BLOCK, &P.tmK, &kv_full[j], h * DH, kv_row0 + j * TK);
         tma_load_2d(sV + j * KV_BLOCK, &P.tmV, &kv_full[j], h * DH, kv_row0 + j * TK);
       }
-      int last_k[GROUPS];
-      for (int g = 0; g < GROUPS; ++g) last_k[g] = -1;
-      bool ok = true;
-      for (int t = 0; t < ntiles && ok; ++t) {
+      int last_t = -1;
+      for (int t = 0; t < ntiles; ++t) {
         const int g = t % GROUPS, k = t / GROUPS;
-        if (k > 0 && !mbar_wait(&q_free[g], (k - 1) & 1, P.status, abort_flag)) { ok = false; break; }
+        if (k > 0 && !mbar_wait(&q_free[g], (k - 1) & 1, P.status, abort_flag)) break;
         mbar_arrive_expect_tx(&q_full[g], NQ * Q_TILE);
         const int qrow = (int)(q0 + (long long)t * TQ);
         tma_load_2d(sQ + (g * NQ) * Q_TILE, &P.tmQ, &q_full[g], h * DH, qrow);
         if (SPLIT) tma_load_2d(sQ + (g * NQ + 1) * Q_TILE, &P.tmQ, &q_full[g], (int)P.q_lo_col + h * DH, qrow);
-        last_k[g] = k;
+        last_t = t;
       }
       // no copy of this CTA may still be landing when it exits
       for (int j = 0; j < nkb; ++j) mbar_wait(&kv_full[j], 0, P.status, nullptr);
-      for (int g = 0; g < GROUPS; ++g)
-        if (last_k[g] >= 0) mbar_wait(&q_full[g], last_k[g] & 1, P.status, nullptr);
-    } else if (warp == 1 && lane == 0) {
-      // ---------------- MMA issuer ----------------
-      int T[GROUPS];
-      int Tmax = 0;
-      for (int g = 0; g < GROUPS; ++g) {
-        T[g] = tiles_g(g) * nkb;
-        Tmax = T[g] > Tmax ? T[g] : Tmax;
-      }
+      for (int t = last_t - GROUPS + 1 < 0 ? 0 : last_t - GROUPS + 1; t <= last_t; ++t)
+        mbar_wait(&q_full[t % GROUPS], (t / GROUPS) & 1, P.status, nullptr);
+    } else if (warp >= 1 && warp <= GROUPS && lane == 0) {
+      // ---------------- MMA issuer of query-tile group g = warp - 1 ----------------
+      // Per key block i:  S_i = Q K_j^T once the softmax has read S_{i-1} (s_free); then, for the
+      // previous block, O += P V_j and l += P 1 in two 64-key halves, each once the softmax has
+      // written that half of P (p_full).  Each group's MMAs touch only its own TMEM columns.
+      const int g = warp - 1;
+      const int T = tiles_g(g) * nkb;
+      auto issue_pv = [&](int ib, int hh) -> bool {
+        if (!mbar_wait(&p_full[2 * g + hh], ib & 1, P.status, abort_flag)) return false;
+        tc_fence_after();
+        const int j = ib % nkb;
+        const uint32_t va = smem_u32(sV + j * KV_BLOCK);
+#pragma unroll
+        for (int kq = 0; kq < TK / 32; ++kq) {
+          const int ks = hh * (TK / 32) + kq;
+          const uint32_t pa = tmem_base + C::P_COL + g * 64 + ks * 8;
+          tc_mma_ts(tmem_base + C::O_COL + g * DH, pa, sdesc(va + ks * 16 * ROWB, SBO, SW), IDESC_O,
+                    (ks > 0 || j > 0) ? 1u : 0u);
+          if (C::SUM_MMA)
+            tc_mma_ts(tmem_base + C::L_COL + g * 16, pa, sdesc(smem_u32(sOnes), 1024, 2), IDESC_L,
+                      (ks > 0 || j > 0) ? 1u : 0u);
+        }
+        tc_commit(&o_full[2 * g + hh]);
+        return true;
+      };
       bool ok = true;
-      for (int i = 0; i <= Tmax && ok; ++i) {
-        // S_i of every group first ...
-        for (int g = 0; g < GROUPS && ok; ++g) {
-          if (i >= T[g]) continue;
-          const int k = i / nkb, j = i - k * nkb;
-          if (j == 0 && !mbar_wait(&q_full[g], k & 1, P.status, abort_flag)) { ok = false; break; }
-          if (!mbar_wait(&kv_full[j], 0, P.status, abort_flag)) { ok = false; break; }
-          if (!mbar_wait(&s_free[g], (i & 1) ^ 1, P.status, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t qa = smem_u32(sQ + (g * NQ) * Q_TILE);
-          const uint32_t ka = smem_u32(sK + j * KV_BLOCK);
+      for (int i = 0; i < T && ok; ++i) {
+        const int k = i / nkb, j = i - k * nkb;
+        if (j == 0 && !mbar_wait(&q_full[g], k & 1, P.status, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&kv_full[j], 0, P.status, abort_flag)) { ok = false; break; }
+        if (i > 0 && !mbar_wait(&s_free[g], (i - 1) & 1, P.status, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t qa = smem_u32(sQ + (g * NQ) * Q_TILE);
+        const uint32_t ka = smem_u32(sK + j * KV_BLOCK);
 #pragma unroll
-          for (int ks = 0; ks < DH / 16; ++ks) {
-            tc_mma_ss(tmem_base + g * TK, sdesc(qa + ks * 32, SBO, SW), sdesc(ka + ks * 32, SBO, SW), IDESC_S,
-                      ks > 0 ? 1u : 0u);
-            if (SPLIT)
-              tc_mma_ss(tmem_base + g * TK, sdesc(qa + Q_TILE + ks * 32, SBO, SW), sdesc(ka + ks * 32, SBO, SW),
-                        IDESC_S, 1u);
-          }
-          tc_commit(&s_full[g]);
-          if (j == nkb - 1) tc_commit(&q_free[g]);   // this tile's queries are no longer read
+        for (int ks = 0; ks < DH / 16; ++ks) {
+          tc_mma_ss(tmem_base + C::S_COL + g * TK, sdesc(qa + ks * 32, SBO, SW), sdesc(ka + ks * 32, SBO, SW),
+                    IDESC_S, ks > 0 ? 1u : 0u);
+          if (SPLIT)
+            tc_mma_ss(tmem_base + C::S_COL + g * TK, sdesc(qa + Q_TILE + ks * 32, SBO, SW),
+                      sdesc(ka + ks * 32, SBO, SW), IDESC_S, 1u);
         }
-        // ... then P_{i-1} V_{i-1} of every group
-        for (int g = 0; g < GROUPS && ok; ++g) {
-          if (i < 1 || i > T[g]) continue;
-          const int jb = (i - 1) % nkb;
-          if (!mbar_wait(&p_full[g], (i - 1) & 1, P.status, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t pa = smem_u32(sP + g * P_TILE);
-          const uint32_t va = smem_u32(sV + jb * KV_BLOCK);
-#pragma unroll
-          for (int ks = 0; ks < TK / 16; ++ks) {
-            const uint64_t adesc = sdesc(pa + (ks >> 2) * (TQ * 128) + (ks & 3) * 32, 1024, 2);
-            const uint64_t bdesc = sdesc(va + ks * 16 * ROWB, SBO, SW);
-            tc_mma_ss(tmem_base + O_COL0 + g * DH, adesc, bdesc, IDESC_O, (ks > 0 || jb > 0) ? 1u : 0u);
-          }
-          tc_commit(&o_full[g]);
-        }
+        tc_commit(&s_full[g]);
+        if (j == nkb - 1) tc_commit(&q_free[g]);   // this tile's queries are no longer read
+        if (i > 0) ok = issue_pv(i - 1, 0) && issue_pv(i - 1, 1);
       }
-      tc_commit(drain);
-      mbar_wait(drain, 0, P.status, nullptr);
+      if (ok && T > 0) ok = issue_pv(T - 1, 0) && issue_pv(T - 1, 1);
+      tc_commit(&drain[g]);
+      mbar_wait(&drain[g], 0, P.status, nullptr);
     }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 224;");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REG_SOFTMAX));
     // ---------------- softmax warpgroups: thread = query row = TMEM lane ----------------
     const int g = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t saddr = lane_addr + g * TK;
-    const uint32_t oaddr = lane_addr + O_COL0 + g * DH;
-    uint8_t* prow = sP + g * P_TILE + row * 128;
+    const uint32_t saddr = lane_addr + C::S_COL + g * TK;
+    const uint32_t paddr = lane_addr + C::P_COL + g * 64;
+    const uint32_t oaddr = lane_addr + C::O_COL + g * DH;
+    const uint32_t laddr = lane_addr + C::L_COL + g * 16;
     const int Tg = tiles_g(g) * nkb;
-    float m_cur = -INFINITY, l_sum = 0.f;
+    const float sl2 = P.scale_log2;
+    float m_cur = -INFINITY, l_reg = 0.f;
 
-    // O accumulator of the finished tile k_tile, divided by its row sum, to global memory
-    auto emit_row = [&](int k_tile, float l_final) {
+    // O of the finished tile k_tile, divided by its row sum, to global memory
+    auto emit_row = [&](int k_tile) {
       float out[DH];
 #pragma unroll
       for (int c = 0; c < DH / 32; ++c) {
@@ -269,6 +355,13 @@ __global__ void __launch_bounds__(128 + 128 * GROUPS, 1) attn_tc_kernel(const __
         tmem_ld_wait();
 #pragma unroll
         for (int k = 0; k < 32; ++k) out[c * 32 + k] = __uint_as_float(w[k]);
+      }
+      float l_final = l_reg;
+      if (C::SUM_MMA) {
+        uint32_t lw;
+        tmem_ld_32x32b_x1(laddr, lw);
+        tmem_ld_wait();
+        l_final = __uint_as_float(lw);
       }
       const long long qrow = q0 + (long long)(g + GROUPS * k_tile) * TQ + row;
       if (qrow >= q1) return;
@@ -302,60 +395,53 @@ __global__ void __launch_bounds__(128 + 128 * GROUPS, 1) attn_tc_kernel(const __
       tc_fence_after();
       // the whole S row into registers with one wait, then the S accumulator is released
       uint32_t v[TK / 32][32];
-      __syncwarp();
 #pragma unroll
       for (int c = 0; c < TK / 32; ++c) tmem_ld_32x32b_x32(saddr + c * 32, v[c]);
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&s_free[g]);
-      if ((j + 1) * TK > P.L) {
+      const int valid = P.L - j * TK;   // keys of this block that exist (>= 1)
+      if (valid < TK) {
 #pragma unroll
         for (int c = 0; c < TK / 32; ++c)
 #pragma unroll
           for (int k = 0; k < 32; ++k)
-            if (j * TK + c * 32 + k >= P.L) v[c][k] = __float_as_uint(-INFINITY);
+            if (c * 32 + k >= valid) v[c][k] = __float_as_uint(-INFINITY);
       }
-      // row maximum as a tree (eight independent chains)
+      // row maximum: eight chains of three-input max
       float mt[8];
 #pragma unroll
-      for (int t = 0; t < 8; ++t) mt[t] = -INFINITY;
+      for (int t = 0; t < 8; ++t) mt[t] = fmaxf(__uint_as_float(v[0][t]), __uint_as_float(v[0][t + 8]));
 #pragma unroll
-      for (int c = 0; c < TK / 32; ++c)
+      for (int e = 16; e < TK; e += 16)
 #pragma unroll
-        for (int k = 0; k < 32; ++k) mt[k & 7] = fmaxf(mt[k & 7], __uint_as_float(v[c][k]));
-      const float mx = fmaxf(fmaxf(fmaxf(mt[0], mt[1]), fmaxf(mt[2], mt[3])), fmaxf(fmaxf(mt[4], mt[5]), fmaxf(mt[6], mt[7]))) *
-                       P.scale_log2;
+        for (int t = 0; t < 8; ++t)
+          mt[t] = fmax3(mt[t], __uint_as_float(v[(e + t) >> 5][(e + t) & 31]),
+                        __uint_as_float(v[(e + 8 + t) >> 5][(e + 8 + t) & 31]));
+      const float mx = fmax3(fmax3(mt[0], mt[1], mt[2]), fmax3(mt[3], mt[4], mt[5]), fmaxf(mt[6], mt[7])) * sl2;
       // the first block sets the row's reference maximum; later blocks move it only when some
       // row of the warp would otherwise produce exponentials above 2^8 (warp-uniform, since the
-      // O rescale below is a warp-wide TMEM access)
+      // rescale is a warp-wide TMEM access)
       float m_new = m_cur, corr = 1.0f;
-      bool rescale = false;
+      const bool rescale = j != 0 && __any_sync(0xffffffffu, mx > m_cur + kLazyRescaleLog2);
       if (j == 0) {
         m_new = mx;
-      } else if (__any_sync(0xffffffffu, mx > m_cur + kLazyRescaleLog2)) {
+      } else if (rescale) {
         m_new = fmaxf(m_cur, mx);
         corr = ex2_approx(m_cur - m_new);
-        rescale = true;
       }
-      float rs[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[TK / 2];
-#pragma unroll
-      for (int c = 0; c < TK / 32; ++c)
-#pragma unroll
-        for (int k = 0; k < 32; k += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(v[c][k]), P.scale_log2, -m_new));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(v[c][k + 1]), P.scale_log2, -m_new));
-          rs[(k >> 1) & 3] += p0 + p1;
-          pk[(c * 32 + k) >> 1] = pack_bf16x2(p0, p1);
-        }
-      const float rsum = (rs[0] + rs[1]) + (rs[2] + rs[3]);
-      // the previous block's P V has completed: the P tile may be overwritten and the O
-      // accumulator read (finished tile) or rescaled
+      // the previous block's P V, first half, has completed: that half of P may be overwritten;
+      // O is read (finished tile) or rescaled only once both halves have completed
+      const bool need_o = i > 0 && (j == 0 || rescale);
       if (i > 0) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&o_full[g], (i - 1) & 1, P.status, abort_flag))) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(&o_full[2 * g], (i - 1) & 1, P.status, abort_flag) &&
+                                         (!need_o || mbar_wait(&o_full[2 * g + 1], (i - 1) & 1, P.status, abort_flag)))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         if (j == 0) {
-          emit_row(k_tile - 1, l_sum);
+          emit_row(k_tile - 1);
         } else if (rescale) {
 #pragma unroll
           for (int c = 0; c < DH / 32; ++c) {
@@ -366,25 +452,64 @@ __global__ void __launch_bounds__(128 + 128 * GROUPS, 1) attn_tc_kernel(const __
             for (int k = 0; k < 32; ++k) w[k] = __float_as_uint(__uint_as_float(w[k]) * corr);
             tmem_st_32x32b_x32(oaddr + c * 32, w);
           }
-          tmem_st_wait();
+          if (C::SUM_MMA) {
+            uint32_t lw;
+            tmem_ld_32x32b_x1(laddr, lw);
+            tmem_ld_wait();
+            tmem_st_32x32b_x1(laddr, __float_as_uint(__uint_as_float(lw) * corr));
+          }
         }
       }
-      // P_i as bf16, K-major with a 128-byte swizzle (two 64-key sub-tiles)
+      // exponentials: one pair in four on the FMA pipe (polynomial), the rest on MUFU; P_i as
+      // bf16 pairs into TMEM, 32 keys per store
+      const float neg_m = -m_new;
+      float rs = 0.f;
 #pragma unroll
-      for (int q = 0; q < TK / 8; ++q) {
-        const int chunk = q & 7;
-        *reinterpret_cast<uint4*>(prow + (q >> 3) * (TQ * 128) + ((chunk ^ (row & 7)) << 4)) =
-            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+      for (int c = 0; c < TK / 32; ++c) {
+        if (c == TK / 64) {
+          // first half of P_i is written: hand it to the tensor core, then wait for the
+          // previous block's second-half P V before overwriting that half
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&p_full[2 * g]);
+          if (i > 0 && !need_o &&
+              !__all_sync(0xffffffffu, mbar_wait(&o_full[2 * g + 1], (i - 1) & 1, P.status, abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 32; k += 2) {
+          float x0, x1, p0, p1;
+          ffma2(__uint_as_float(v[c][k]), __uint_as_float(v[c][k + 1]), sl2, neg_m, x0, x1);
+          if ((k & 6) == 6) {
+            exp2_poly2(x0, x1, p0, p1);
+            if (valid < TK) {   // masked keys (x = -inf) must give exactly zero
+              p0 = x0 == -INFINITY ? 0.f : p0;
+              p1 = x1 == -INFINITY ? 0.f : p1;
+            }
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          if (!C::SUM_MMA) rs += p0 + p1;
+          pk[k >> 1] = pack_bf16x2(p0, p1);
+        }
+        tmem_st_32x32b_x16(paddr + c * 16, pk);
       }
-      fence_async_shared();
+      if (!ok) break;
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&p_full[g]);
-      l_sum = j == 0 ? rsum : fmaf(l_sum, corr, rsum);
+      mbar_arrive(&p_full[2 * g + 1]);
+      if (!C::SUM_MMA) l_reg = j == 0 ? rs : fmaf(l_reg, corr, rs);
       m_cur = m_new;
     }
-    if (ok && Tg > 0 && __all_sync(0xffffffffu, mbar_wait(&o_full[g], (Tg - 1) & 1, P.status, abort_flag))) {
+    if (ok && Tg > 0 && __all_sync(0xffffffffu, mbar_wait(&o_full[2 * g], (Tg - 1) & 1, P.status, abort_flag) &&
+                                               mbar_wait(&o_full[2 * g + 1], (Tg - 1) & 1, P.status, abort_flag))) {
       tc_fence_after();
-      emit_row(Tg / nkb - 1, l_sum);
+      emit_row(Tg / nkb - 1);
     }
   }
 
@@ -395,6 +520,13 @@ __global__ void __launch_bounds__(128 + 128 * GROUPS, 1) attn_tc_kernel(const __
     tc_fence_after();
     tmem_dealloc(tmem_base, AT_TMEM_COLS);
   }
+}
+
+template <int DH, bool SPLIT>
+size_t at_smem_bytes(int nkb) {
+  constexpr int G = AtCfg<DH>::GROUPS;
+  return 1024 + (size_t)2 * nkb * TK * DH * 2 + (size_t)G * (SPLIT ? 2 : 1) * TQ * DH * 2 + 2048 +
+         (AT_MAX_KB + 9 * G) * 8 + 16;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -413,15 +545,9 @@ bool encode_rows(rocs_context* ctx, CUtensorMap* map, const void* ptr, long long
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int DH, bool SPLIT, int GROUPS>
-size_t at_smem_bytes(int nkb) {
-  return 1024 + (size_t)2 * nkb * TK * DH * 2 + (size_t)GROUPS * (SPLIT ? 2 : 1) * TQ * DH * 2 +
-         (size_t)GROUPS * TQ * TK * 2 + (AT_MAX_KB + 6 * GROUPS + 1) * 8 + 16;
-}
-
-template <int DH, bool SPLIT, int GROUPS>
+template <int DH, bool SPLIT>
 rocs_status at_launch(rocs_context* ctx, AttnTcParams& P, int B_R, int H, cudaStream_t s) {
-  const size_t smem = at_smem_bytes<DH, SPLIT, GROUPS>(P.nkb);
+  const size_t smem = at_smem_bytes<DH, SPLIT>(P.nkb);
   if (smem > 232448) {
     set_error("tcgen05 attention: L=%d needs %zu B of shared memory", P.L, smem);
     return ROCS_ERR_UNSUPPORTED;
@@ -429,22 +555,23 @@ rocs_status at_launch(rocs_context* ctx, AttnTcParams& P, int B_R, int H, cudaSt
   static bool attr[64] = {false};
   if (ctx->device < 64 && !attr[ctx->device]) {
     rocs_status st = cuda_check(
-        cudaFuncSetAttribute(attn_tc_kernel<DH, SPLIT, GROUPS>, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448),
+        cudaFuncSetAttribute(attn_tc_kernel<DH, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448),
         "cudaFuncSetAttribute(attn_tc)");
     if (st != ROCS_OK) return st;
     // the softmax warpgroups raise their register limit out of the block's launch allocation;
     // refuse to launch if the compiled kernel was given fewer registers than that split needs
     cudaFuncAttributes fa;
-    st = cuda_check(cudaFuncGetAttributes(&fa, attn_tc_kernel<DH, SPLIT, GROUPS>), "cudaFuncGetAttributes(attn_tc)");
+    st = cuda_check(cudaFuncGetAttributes(&fa, attn_tc_kernel<DH, SPLIT>), "cudaFuncGetAttributes(attn_tc)");
     if (st != ROCS_OK) return st;
-    if ((long long)fa.numRegs * (128 + 128 * GROUPS) < 128LL * 40 + 128LL * GROUPS * 224) {
+    using C = AtCfg<DH>;
+    if (fa.numRegs < C::REG_LAUNCH) {
       set_error("tcgen05 attention: kernel compiled with %d registers per thread, below the warpgroup split",
                 fa.numRegs);
       return ROCS_ERR_UNSUPPORTED;
     }
     attr[ctx->device] = true;
   }
-  attn_tc_kernel<DH, SPLIT, GROUPS><<<(unsigned)((long long)B_R * H), 128 + 128 * GROUPS, smem, s>>>(P);
+  attn_tc_kernel<DH, SPLIT><<<(unsigned)((long long)B_R * H), AtCfg<DH>::THREADS, smem, s>>>(P);
   return cuda_check(cudaGetLastError(), "attn_tc_kernel");
 }
 
@@ -485,9 +612,8 @@ rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq,
   P.ldo2 = ldo2;
   P.status = ctx->d_status;
   LaunchTimer lt_("attn_tc", s);
-  if (d_h == 32)
-    return q_split ? at_launch<32, true, 2>(ctx, P, B_R, H, s) : at_launch<32, false, 2>(ctx, P, B_R, H, s);
-  return q_split ? at_launch<64, true, 2>(ctx, P, B_R, H, s) : at_launch<64, false, 2>(ctx, P, B_R, H, s);
+  if (d_h == 32) return q_split ? at_launch<32, true>(ctx, P, B_R, H, s) : at_launch<32, false>(ctx, P, B_R, H, s);
+  return q_split ? at_launch<64, true>(ctx, P, B_R, H, s) : at_launch<64, false>(ctx, P, B_R, H, s);
 }
 
 }  // namespace rocs
