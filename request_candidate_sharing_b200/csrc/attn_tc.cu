@@ -136,10 +136,11 @@ __device__ __forceinline__ uint64_t dup2(float c) {
 
 // 2^x0, 2^x1 on the FMA pipe: x = n + f with n = round(x) by the 1.5 * 2^23 shifter, 2^f by a
 // degree-3 minimax polynomial on [-1/2, 1/2] (max relative error 7.5e-5, coefficients from
-// gen_exp2_poly.py), 2^n added into the exponent field.  Arguments are clamped to [-126, 126].
+// gen_exp2_poly.py), 2^n added into the exponent field.  Valid for x < 128 (the softmax keeps
+// x <= 8); arguments below -126 are raised to -126.
 __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
-  x0 = fminf(fmaxf(x0, -126.0f), 126.0f);
-  x1 = fminf(fmaxf(x1, -126.0f), 126.0f);
+  x0 = fmaxf(x0, -126.0f);
+  x1 = fmaxf(x1, -126.0f);
   uint64_t xv, tv, nv, fv, pv;
   const uint64_t shifter = dup2(12582912.0f);   // 1.5 * 2^23 in both halves
   asm("mov.b64 %0, {%1, %2};" : "=l"(xv) : "f"(x0), "f"(x1));
@@ -153,9 +154,12 @@ __device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float&
   uint32_t t0, t1, p0, p1;
   asm("mov.b64 {%0, %1}, %2;" : "=r"(t0), "=r"(t1) : "l"(tv));
   asm("mov.b64 {%0, %1}, %2;" : "=r"(p0), "=r"(p1) : "l"(pv));
-  // the shifter's low 9 bits are zero, so (bits(t) << 23) is exactly n << 23
-  y0 = __uint_as_float(p0 + (t0 << 23));
-  y1 = __uint_as_float(p1 + (t1 << 23));
+  // the shifter's low 9 bits are zero, so bits(t) * 2^23 is exactly n << 23 (mod 2^32)
+  uint32_t r0, r1;
+  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(r0) : "r"(t0), "r"(p0));
+  asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(r1) : "r"(t1), "r"(p1));
+  y0 = __uint_as_float(r0);
+  y1 = __uint_as_float(r1);
 }
 
 // A row's running maximum is only moved when a block's maximum exceeds it by more than this
@@ -460,8 +464,8 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
           }
         }
       }
-      // exponentials: one pair in four on the FMA pipe (polynomial), the rest on MUFU; P_i as
-      // bf16 pairs into TMEM, 32 keys per store
+      // exponentials: three pairs in eight on the FMA pipe (polynomial), the rest on MUFU; P_i
+      // as bf16 pairs into TMEM, 32 keys per store
       const float neg_m = -m_new;
       float rs = 0.f;
 #pragma unroll
@@ -484,7 +488,7 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
         for (int k = 0; k < 32; k += 2) {
           float x0, x1, p0, p1;
           ffma2(__uint_as_float(v[c][k]), __uint_as_float(v[c][k + 1]), sl2, neg_m, x0, x1);
-          if ((k & 6) == 6) {
+          if (((k >> 1) & 7) >= 5) {
             exp2_poly2(x0, x1, p0, p1);
             if (valid < TK) {   // masked keys (x = -inf) must give exactly zero
               p0 = x0 == -INFINITY ? 0.f : p0;

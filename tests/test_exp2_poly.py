@@ -32,7 +32,7 @@ def _fma32(a, b, c):
 
 def _exp2_poly(x, coeffs):
     c0, c1, c2, c3 = coeffs
-    x = np.clip(x.astype(np.float32), np.float32(-126), np.float32(126))
+    x = np.maximum(x.astype(np.float32), np.float32(-126))
     shifter = np.float32(12582912.0)
     t = (x + shifter).astype(np.float32)
     n = (t - shifter).astype(np.float32)
