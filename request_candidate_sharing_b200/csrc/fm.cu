@@ -131,52 +131,126 @@ __device__ __forceinline__ void gram_tile(uint32_t sbase, int pitch, int a0, int
 // Lane j owns features [DPL*j, DPL*j + DPL); the LCB sums use the full-precision embeddings, the
 // FM products their bf16 rounding (tensor-core operands).
 // ---------------------------------------------------------------------------------------------
-template <typename TIN, int DPL>
-__device__ __forceinline__ void load_feats(const TIN* p, float (&e)[DPL]);
-template <>
-__device__ __forceinline__ void load_feats<float, 4>(const float* p, float (&e)[4]) {
-  const float4 v = __ldg(reinterpret_cast<const float4*>(p));
-  e[0] = v.x; e[1] = v.y; e[2] = v.z; e[3] = v.w;
-}
-template <>
-__device__ __forceinline__ void load_feats<__nv_bfloat16, 4>(const __nv_bfloat16* p, float (&e)[4]) {
-  const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
-  e[0] = bf16_lo(v.x); e[1] = bf16_hi(v.x); e[2] = bf16_lo(v.y); e[3] = bf16_hi(v.y);
-}
+// One CTA per SM walks a contiguous range of candidates.  Warp 0 streams each candidate's E^C rows
+// (contiguous, n_C x D) into a ring of shared-memory stages with bulk async copies, FC_STAGES
+// candidates ahead; consumer warp w takes the candidates w, w + FC_CONSUMERS, ... of the range, so
+// its loads are already in flight while it computes.
+constexpr int FC_CONSUMERS = 7;   // 8 warps in all: the whole register file (255 per thread) is available
+constexpr int FC_STAGES = 12;
 
 template <typename TIN>
-__global__ void __launch_bounds__(FM_WARPS * 32, 4) glm_cand_fused_kernel(
+__global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_kernel(
     const TIN* __restrict__ E_R, const TIN* __restrict__ E_C, const int32_t* __restrict__ req_idx, int B_R,
-    long long B_C, int n_R, int n_C, int trows, int pitch, __nv_bfloat16* __restrict__ F_C,
+    long long B_C, long long per_block, int n_R, int n_C, int trows, int pitch, __nv_bfloat16* __restrict__ F_C,
     const __nv_bfloat16* __restrict__ P_CC, int o_C, const float* __restrict__ ZL, float* __restrict__ L_C,
     const __nv_bfloat16* __restrict__ q_pCC, const float* __restrict__ ZQ, __nv_bfloat16* __restrict__ tC,
     int* status) {
   constexpr int D = 128, DPL = 4;
-  extern __shared__ __align__(16) uint8_t fm_smem[];
+  extern __shared__ __align__(128) uint8_t fc_smem[];
   __shared__ float sP[LCB_OMAX_F * 64];
   __shared__ float sQ[64];
+  __shared__ __align__(8) uint64_t full[FC_STAGES], empty[FC_STAGES];
+  __shared__ int stage_r[FC_STAGES];   // request index of the candidate in each stage
+  __shared__ int abort_flag_s;
+  volatile int* abort_flag = &abort_flag_s;
+
+  const long long c0 = (long long)blockIdx.x * per_block;
+  const long long c1 = c0 + per_block < B_C ? c0 + per_block : B_C;
+  if (c0 >= c1) return;
+  const int n = (int)(c1 - c0);
+  const uint32_t stage_bytes = (uint32_t)(n_C * D * sizeof(TIN));
+  uint8_t* ring = fc_smem;
+  uint8_t* tiles = fc_smem + FC_STAGES * NC_MAX * D * sizeof(TIN);
+
   for (int i = threadIdx.x; i < o_C * n_C; i += blockDim.x) sP[i] = __bfloat162float(P_CC[i]);
   for (int i = threadIdx.x; i < n_C; i += blockDim.x) sQ[i] = q_pCC ? __bfloat162float(q_pCC[i]) : 0.f;
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < FC_STAGES; ++k) {
+      mbar_init(&full[k], 1);
+      mbar_init(&empty[k], 32);
+    }
+    abort_flag_s = 0;
+    fence_barrier_init();
+  }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint8_t* T = fm_smem + warp * trows * pitch;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- producer ----------------
+      int issued = 0;
+      for (int i = 0; i < n; ++i) {
+        const int st = i % FC_STAGES, use = i / FC_STAGES;
+        const int r = req_idx[c0 + i];   // loaded ahead of the consumers
+        if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1, status, abort_flag)) break;
+        stage_r[st] = r;
+        mbar_arrive_expect_tx(&full[st], stage_bytes);
+        bulk_load(ring + st * NC_MAX * D * sizeof(TIN), E_C + (c0 + i) * (long long)n_C * D, stage_bytes, &full[st]);
+        issued = i + 1;
+      }
+      // no copy of this CTA may still be landing when it exits
+      for (int i = issued - FC_STAGES < 0 ? 0 : issued - FC_STAGES; i < issued; ++i)
+        mbar_wait(&full[i % FC_STAGES], (i / FC_STAGES) & 1, status, nullptr);
+    }
+    return;
+  }
+
+  // ---------------- consumers ----------------
+  const int cw = warp - 1;
+  uint8_t* T = tiles + cw * trows * pitch;
   const uint32_t sbase = smem_u32(T);
-  const long long c_begin = ((long long)blockIdx.x * FM_WARPS + warp) * FM_RUN;
   const int ncols = n_R + n_C;
   const long long fsz = (long long)n_C * ncols;
   int staged = -1;
+  float zl[LCB_OMAX_F][DPL], zq[DPL];
+#pragma unroll
+  for (int o = 0; o < LCB_OMAX_F; ++o)
+#pragma unroll
+    for (int j = 0; j < DPL; ++j) zl[o][j] = 0.f;
+#pragma unroll
+  for (int j = 0; j < DPL; ++j) zq[j] = 0.f;
   zero_rows(T + (n_R + n_C) * pitch, pitch, trows - (n_R + n_C), D);
-  for (int i = 0; i < FM_RUN; ++i) {
-    const long long c = c_begin + i;
-    if (c >= B_C) break;
-    const int r = req_idx[c];
+  for (int i = cw; i < n; i += FC_CONSUMERS) {
+    const int st = i % FC_STAGES;
+    if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (i / FC_STAGES) & 1, status, abort_flag))) break;
+    const long long c = c0 + i;
+    // this candidate's rows from the stage into registers (lane j owns features 4j..4j+3), then
+    // the stage goes back to the producer
+    const TIN* ec = reinterpret_cast<const TIN*>(ring + st * NC_MAX * D * sizeof(TIN));
+    float e[NC_MAX][DPL];
+#pragma unroll
+    for (int t = 0; t < NC_MAX; ++t) {
+      if (t < n_C) {
+        if constexpr (sizeof(TIN) == 4) {
+          const float4 v = reinterpret_cast<const float4*>(ec + t * D)[lane];
+          e[t][0] = v.x; e[t][1] = v.y; e[t][2] = v.z; e[t][3] = v.w;
+        } else {
+          const uint2 v = reinterpret_cast<const uint2*>(ec + t * D)[lane];
+          e[t][0] = bf16_lo(v.x); e[t][1] = bf16_hi(v.x); e[t][2] = bf16_lo(v.y); e[t][3] = bf16_hi(v.y);
+        }
+      }
+    }
+    const int r = stage_r[st];
+    mbar_arrive(&empty[st]);
     if (r < 0 || r >= B_R) {
       if (lane == 0) set_status(status, ROCS_ERR_INDEX);
       continue;
     }
     __syncwarp();
     if (r != staged) {
+      // a new request run: its rows into the tile, its Z^L and Z^Q rows into registers
       stage_rows(T, pitch, E_R + (long long)r * n_R * D, n_R, D);
+#pragma unroll
+      for (int o = 0; o < LCB_OMAX_F; ++o) {
+        if (o < o_C) {
+          const float4 z = __ldg(reinterpret_cast<const float4*>(ZL + ((long long)r * o_C + o) * D + DPL * lane));
+          zl[o][0] = z.x; zl[o][1] = z.y; zl[o][2] = z.z; zl[o][3] = z.w;
+        }
+      }
+      if (tC != nullptr) {
+        const float4 z = __ldg(reinterpret_cast<const float4*>(ZQ + (long long)r * D + DPL * lane));
+        zq[0] = z.x; zq[1] = z.y; zq[2] = z.z; zq[3] = z.w;
+      }
       staged = r;
     }
     float acc[LCB_OMAX_F][DPL];
@@ -187,12 +261,6 @@ __global__ void __launch_bounds__(FM_WARPS * 32, 4) glm_cand_fused_kernel(
     for (int o = 0; o < LCB_OMAX_F; ++o)
 #pragma unroll
       for (int j = 0; j < DPL; ++j) acc[o][j] = 0.f;
-    const TIN* ec = E_C + c * (long long)n_C * D;
-    // issue every row load of this candidate before using any (n_C <= NC_MAX)
-    float e[NC_MAX][DPL];
-#pragma unroll
-    for (int t = 0; t < NC_MAX; ++t)
-      if (t < n_C) load_feats<TIN, DPL>(ec + t * D + DPL * lane, e[t]);
 #pragma unroll
     for (int t = 0; t < NC_MAX; ++t) {
       if (t < n_C) {
@@ -214,15 +282,12 @@ __global__ void __launch_bounds__(FM_WARPS * 32, 4) glm_cand_fused_kernel(
     // LCB output (fp32, float4 per token)
 #pragma unroll
     for (int o = 0; o < LCB_OMAX_F; ++o) {
-      if (o < o_C) {
-        const float4 z = __ldg(reinterpret_cast<const float4*>(ZL + ((long long)r * o_C + o) * D + DPL * lane));
+      if (o < o_C)
         reinterpret_cast<float4*>(L_C + c * (long long)o_C * D + (long long)o * D)[lane] =
-            make_float4(acc[o][0] + z.x, acc[o][1] + z.y, acc[o][2] + z.z, acc[o][3] + z.w);
-      }
+            make_float4(acc[o][0] + zl[o][0], acc[o][1] + zl[o][1], acc[o][2] + zl[o][2], acc[o][3] + zl[o][3]);
     }
     if (tC != nullptr) {
-      const float4 z = __ldg(reinterpret_cast<const float4*>(ZQ + (long long)r * D + DPL * lane));
-      const float v[4] = {qa[0] + z.x, qa[1] + z.y, qa[2] + z.z, qa[3] + z.w};
+      const float v[4] = {qa[0] + zq[0], qa[1] + zq[1], qa[2] + zq[2], qa[3] + zq[3]};
       float hi[4], lo[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -237,6 +302,7 @@ __global__ void __launch_bounds__(FM_WARPS * 32, 4) glm_cand_fused_kernel(
     gram_tile(sbase, pitch, n_R, n_C, ncols, D, F_C, 2, c * fsz * 2, ncols, fsz);
   }
 }
+
 
 // Shared tile rows: n_R request rows, then n_C candidate rows, padded with zeros up to TROWS.
 // TROWS >= max(n_R + roundup16(n_C), roundup16(n_R + n_C), roundup16(n_R)).
@@ -458,22 +524,27 @@ rocs_status fused_launch(rocs_context* ctx, const TIN* E_R, const TIN* E_C, cons
   const int D = 128;
   const int pitch = D * 2 + 16;
   const int trows = fm_trows(n_R, n_C);
-  const int smem = FM_WARPS * trows * pitch;
+  const size_t smem = (size_t)FC_STAGES * NC_MAX * D * sizeof(TIN) + (size_t)FC_CONSUMERS * trows * pitch;
+  if (n_C > NC_MAX || o_C > LCB_OMAX_F || smem > 220 * 1024) {
+    set_error("fused candidate pass: unsupported n_C=%d o_C=%d", n_C, o_C);
+    return ROCS_ERR_UNSUPPORTED;
+  }
   static bool attr[64] = {false};
   if (ctx->device < 64 && !attr[ctx->device]) {
     rocs_status st = cuda_check(cudaFuncSetAttribute(glm_cand_fused_kernel<TIN>,
-                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024),
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024),
                                 "cudaFuncSetAttribute(glm_cand_fused)");
     if (st != ROCS_OK) return st;
     attr[ctx->device] = true;
   }
   if (B_C == 0) return ROCS_OK;
-  const long long per_block = (long long)FM_WARPS * FM_RUN;
-  const long long blocks = (B_C + per_block - 1) / per_block;
+  // one CTA per SM, each over a contiguous candidate range (runs of a request stay together)
+  const long long blocks = B_C < ctx->num_sms ? B_C : ctx->num_sms;
+  const long long per_block = (B_C + blocks - 1) / blocks;
   LaunchTimer lt_("glm_cand_fused", s);
-  glm_cand_fused_kernel<TIN><<<(unsigned)blocks, FM_WARPS * 32, smem, s>>>(
-      E_R, E_C, req_idx, B_R, B_C, n_R, n_C, trows, pitch, (__nv_bfloat16*)F_C, (const __nv_bfloat16*)P_CC, o_C,
-      ZL, L_C, (const __nv_bfloat16*)q_pCC, ZQ, (__nv_bfloat16*)tC, ctx->d_status);
+  glm_cand_fused_kernel<TIN><<<(unsigned)blocks, 32 * (1 + FC_CONSUMERS), smem, s>>>(
+      E_R, E_C, req_idx, B_R, B_C, per_block, n_R, n_C, trows, pitch, (__nv_bfloat16*)F_C,
+      (const __nv_bfloat16*)P_CC, o_C, ZL, L_C, (const __nv_bfloat16*)q_pCC, ZQ, (__nv_bfloat16*)tC, ctx->d_status);
   return cuda_check(cudaGetLastError(), "glm_cand_fused_kernel");
 }
 

@@ -31,6 +31,16 @@ __device__ __forceinline__ void load_vec<float, 8>(const float* p, float (&v)[8]
   v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 template <>
+__device__ __forceinline__ void load_vec<float, 4>(const float* p, float (&v)[4]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+}
+template <>
+__device__ __forceinline__ void load_vec<__nv_bfloat16, 4>(const __nv_bfloat16* p, float (&v)[4]) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
+}
+template <>
 __device__ __forceinline__ void load_vec<__nv_bfloat16, 1>(const __nv_bfloat16* p, float (&v)[1]) {
   v[0] = __bfloat162float(*p);
 }
@@ -53,6 +63,14 @@ template <>
 __device__ __forceinline__ void store_vec<float, 8>(float* p, const float (&v)[8]) {
   reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
   reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+template <>
+__device__ __forceinline__ void store_vec<float, 4>(float* p, const float (&v)[4]) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+template <>
+__device__ __forceinline__ void store_vec<__nv_bfloat16, 4>(__nv_bfloat16* p, const float (&v)[4]) {
+  *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
 }
 template <>
 __device__ __forceinline__ void store_vec<__nv_bfloat16, 1>(__nv_bfloat16* p, const float (&v)[1]) {
@@ -177,8 +195,19 @@ rocs_status dispatch(const void* X1, int w1, long long ld1, const void* X2, long
                      long long ldy, void* Y2, long long ldy2, bool vec, cudaStream_t s) {
 #define ROCS_LN(VEC, NV, TPR) \
   return run<TIN, TRES, TOUT, VEC, NV, TPR>(X1, w1, ld1, X2, ld2, R, ldr, rows, width, g, b, eps, Y, ldy, Y2, ldy2, s)
-  if (vec) {
+  if (vec && sizeof(TIN) == 4) {
+    // fp32 rows: one float4 per lane per vector, so each warp-wide load is 512 contiguous bytes;
     // one warp per row (registers only, no block barrier) up to 2048 values, a block beyond
+    if (width <= 128) ROCS_LN(4, 1, 32);
+    if (width <= 256) ROCS_LN(4, 2, 32);
+    if (width <= 512) ROCS_LN(4, 4, 32);
+    if (width <= 1024) ROCS_LN(4, 8, 32);
+    if (width <= 2048) ROCS_LN(4, 16, 32);
+    if (width <= 4096) ROCS_LN(4, 8, 128);
+    ROCS_LN(4, 16, 128);
+  }
+  if (vec) {
+    // bf16 rows: 16 bytes (8 values) per lane per vector
     if (width <= 256) ROCS_LN(8, 1, 32);
     if (width <= 512) ROCS_LN(8, 2, 32);
     if (width <= 1024) ROCS_LN(8, 4, 32);
