@@ -145,7 +145,7 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
     const __nv_bfloat16* __restrict__ P_CC, int o_C, const float* __restrict__ ZL, float* __restrict__ L_C,
     const __nv_bfloat16* __restrict__ q_pCC, const float* __restrict__ ZQ, __nv_bfloat16* __restrict__ tC,
     int* status) {
-  constexpr int D = 128, DPL = 4;
+  constexpr int D = 128;
   extern __shared__ __align__(128) uint8_t fc_smem[];
   __shared__ float sP[LCB_OMAX_F * 64];
   __shared__ float sQ[64];
@@ -197,36 +197,55 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
 
   // ---------------- consumers ----------------
   const int cw = warp - 1;
-  uint8_t* T = tiles + cw * trows * pitch;
+  uint8_t* T = tiles + cw * (trows + NC_MAX) * pitch;   // [E^R rows ; E^C hi rows ; 0 pad] then E^C lo rows
+  uint8_t* TL = T + trows * pitch;
   const uint32_t sbase = smem_u32(T);
   const int ncols = n_R + n_C;
   const long long fsz = (long long)n_C * ncols;
+  const int g8 = lane >> 2, t4 = lane & 3;
+  // A operand of the token LCB (16 x 16 tokens): rows 0..o_C-1 hold P_CC, row 8 the query
+  // generator's one-token weights, every other entry zero.  Constant for the whole kernel.
+  uint32_t pa[4];
+  {
+    auto A = [&](int row, int k) -> float {
+      if (k >= n_C) return 0.f;
+      if (row < o_C && row < 8) return sP[row * n_C + k];
+      if (row == 8) return sQ[k];
+      return 0.f;
+    };
+    pa[0] = pack_bf16x2(A(g8, 2 * t4), A(g8, 2 * t4 + 1));
+    pa[1] = pack_bf16x2(A(g8 + 8, 2 * t4), A(g8 + 8, 2 * t4 + 1));
+    pa[2] = pack_bf16x2(A(g8, 2 * t4 + 8), A(g8, 2 * t4 + 9));
+    pa[3] = pack_bf16x2(A(g8 + 8, 2 * t4 + 8), A(g8 + 8, 2 * t4 + 9));
+  }
+  // Z^L row g8 and Z^Q (lanes with g8 == 0) of the current request, in the C-fragment layout:
+  // n-tile nt, columns nt*8 + 2*t4 and +1
+  float zl[D / 8][2], zq[D / 8][2];
+#pragma unroll
+  for (int nt = 0; nt < D / 8; ++nt) zl[nt][0] = zl[nt][1] = zq[nt][0] = zq[nt][1] = 0.f;
   int staged = -1;
-  float zl[LCB_OMAX_F][DPL], zq[DPL];
-#pragma unroll
-  for (int o = 0; o < LCB_OMAX_F; ++o)
-#pragma unroll
-    for (int j = 0; j < DPL; ++j) zl[o][j] = 0.f;
-#pragma unroll
-  for (int j = 0; j < DPL; ++j) zq[j] = 0.f;
   zero_rows(T + (n_R + n_C) * pitch, pitch, trows - (n_R + n_C), D);
+  zero_rows(TL + n_C * pitch, pitch, NC_MAX - n_C, D);
   for (int i = cw; i < n; i += FC_CONSUMERS) {
     const int st = i % FC_STAGES;
     if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (i / FC_STAGES) & 1, status, abort_flag))) break;
     const long long c = c0 + i;
-    // this candidate's rows from the stage into registers (lane j owns features 4j..4j+3), then
-    // the stage goes back to the producer
+    // this candidate's rows from the stage into the tile as bf16 (hi, and lo = E - hi for fp32
+    // inputs); lane j converts features 4j..4j+3, then the stage goes back to the producer
     const TIN* ec = reinterpret_cast<const TIN*>(ring + st * NC_MAX * D * sizeof(TIN));
-    float e[NC_MAX][DPL];
+    __syncwarp();   // the previous candidate's tile reads are done
 #pragma unroll
     for (int t = 0; t < NC_MAX; ++t) {
       if (t < n_C) {
         if constexpr (sizeof(TIN) == 4) {
           const float4 v = reinterpret_cast<const float4*>(ec + t * D)[lane];
-          e[t][0] = v.x; e[t][1] = v.y; e[t][2] = v.z; e[t][3] = v.w;
+          const uint32_t h01 = pack_bf16x2(v.x, v.y), h23 = pack_bf16x2(v.z, v.w);
+          *reinterpret_cast<uint2*>(T + (n_R + t) * pitch + lane * 8) = make_uint2(h01, h23);
+          *reinterpret_cast<uint2*>(TL + t * pitch + lane * 8) =
+              make_uint2(pack_bf16x2(v.x - bf16_lo(h01), v.y - bf16_hi(h01)),
+                         pack_bf16x2(v.z - bf16_lo(h23), v.w - bf16_hi(h23)));
         } else {
-          const uint2 v = reinterpret_cast<const uint2*>(ec + t * D)[lane];
-          e[t][0] = bf16_lo(v.x); e[t][1] = bf16_hi(v.x); e[t][2] = bf16_lo(v.y); e[t][3] = bf16_hi(v.y);
+          *reinterpret_cast<uint2*>(T + (n_R + t) * pitch + lane * 8) = reinterpret_cast<const uint2*>(ec + t * D)[lane];
         }
       }
     }
@@ -236,69 +255,61 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
       if (lane == 0) set_status(status, ROCS_ERR_INDEX);
       continue;
     }
-    __syncwarp();
     if (r != staged) {
       // a new request run: its rows into the tile, its Z^L and Z^Q rows into registers
+      __syncwarp();
       stage_rows(T, pitch, E_R + (long long)r * n_R * D, n_R, D);
 #pragma unroll
-      for (int o = 0; o < LCB_OMAX_F; ++o) {
-        if (o < o_C) {
-          const float4 z = __ldg(reinterpret_cast<const float4*>(ZL + ((long long)r * o_C + o) * D + DPL * lane));
-          zl[o][0] = z.x; zl[o][1] = z.y; zl[o][2] = z.z; zl[o][3] = z.w;
+      for (int nt = 0; nt < D / 8; ++nt) {
+        if (g8 < o_C) {
+          const float2 z = __ldg(reinterpret_cast<const float2*>(ZL + ((long long)r * o_C + g8) * D + nt * 8 + 2 * t4));
+          zl[nt][0] = z.x;
+          zl[nt][1] = z.y;
         }
-      }
-      if (tC != nullptr) {
-        const float4 z = __ldg(reinterpret_cast<const float4*>(ZQ + (long long)r * D + DPL * lane));
-        zq[0] = z.x; zq[1] = z.y; zq[2] = z.z; zq[3] = z.w;
+        if (tC != nullptr && g8 == 0) {
+          const float2 z = __ldg(reinterpret_cast<const float2*>(ZQ + (long long)r * D + nt * 8 + 2 * t4));
+          zq[nt][0] = z.x;
+          zq[nt][1] = z.y;
+        }
       }
       staged = r;
     }
-    float acc[LCB_OMAX_F][DPL];
-    float qa[DPL];
-#pragma unroll
-    for (int j = 0; j < DPL; ++j) qa[j] = 0.f;
-#pragma unroll
-    for (int o = 0; o < LCB_OMAX_F; ++o)
-#pragma unroll
-      for (int j = 0; j < DPL; ++j) acc[o][j] = 0.f;
-#pragma unroll
-    for (int t = 0; t < NC_MAX; ++t) {
-      if (t < n_C) {
-        *reinterpret_cast<uint2*>(T + (n_R + t) * pitch + DPL * lane * 2) =
-            make_uint2(pack_bf16x2(e[t][0], e[t][1]), pack_bf16x2(e[t][2], e[t][3]));
-#pragma unroll
-        for (int o = 0; o < LCB_OMAX_F; ++o) {
-          if (o < o_C) {
-            const float p = sP[o * n_C + t];
-#pragma unroll
-            for (int j = 0; j < DPL; ++j) acc[o][j] = fmaf(p, e[t][j], acc[o][j]);
-          }
-        }
-        const float q = sQ[t];
-#pragma unroll
-        for (int j = 0; j < DPL; ++j) qa[j] = fmaf(q, e[t][j], qa[j]);
-      }
-    }
-    // LCB output (fp32, float4 per token)
-#pragma unroll
-    for (int o = 0; o < LCB_OMAX_F; ++o) {
-      if (o < o_C)
-        reinterpret_cast<float4*>(L_C + c * (long long)o_C * D + (long long)o * D)[lane] =
-            make_float4(acc[o][0] + zl[o][0], acc[o][1] + zl[o][1], acc[o][2] + zl[o][2], acc[o][3] + zl[o][3]);
-    }
-    if (tC != nullptr) {
-      const float v[4] = {qa[0] + zq[0], qa[1] + zq[1], qa[2] + zq[2], qa[3] + zq[3]};
-      float hi[4], lo[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        hi[j] = __bfloat162float(__float2bfloat16_rn(v[j]));
-        lo[j] = v[j] - hi[j];
-      }
-      __nv_bfloat16* tp = tC + c * 2LL * D + DPL * lane;
-      *reinterpret_cast<uint2*>(tp) = make_uint2(pack_bf16x2(hi[0], hi[1]), pack_bf16x2(hi[2], hi[3]));
-      *reinterpret_cast<uint2*>(tp + D) = make_uint2(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]));
-    }
     __syncwarp();
+    // token LCB on the tensor cores: [P_CC ; p_CC] (16 x 16) times E^C (16 tokens x 128), the
+    // fp32 embeddings as hi + lo bf16 parts
+    float acc[D / 8][4];
+#pragma unroll
+    for (int nt = 0; nt < D / 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+    for (int p = 0; p < D / 16; ++p) {
+      uint32_t b[4];
+      load_b_frag_kmajor_x2(sbase, pitch, n_R, p * 16, b);
+      mma_bf16_16816(acc[2 * p], pa, b[0], b[1]);
+      mma_bf16_16816(acc[2 * p + 1], pa, b[2], b[3]);
+      if constexpr (sizeof(TIN) == 4) {
+        load_b_frag_kmajor_x2(smem_u32(TL), pitch, 0, p * 16, b);
+        mma_bf16_16816(acc[2 * p], pa, b[0], b[1]);
+        mma_bf16_16816(acc[2 * p + 1], pa, b[2], b[3]);
+      }
+    }
+    // L^C = Z^L + P_CC E^C (fp32), row g8 of every n-tile
+    if (g8 < o_C) {
+      float* lp = L_C + (c * o_C + g8) * (long long)D + 2 * t4;
+#pragma unroll
+      for (int nt = 0; nt < D / 8; ++nt)
+        *reinterpret_cast<float2*>(lp + nt * 8) = make_float2(acc[nt][0] + zl[nt][0], acc[nt][1] + zl[nt][1]);
+    }
+    // t^C = Z^Q + p_CC E^C as a bf16 hi/lo pair (row 8 of the fragment: lanes with g8 == 0)
+    if (tC != nullptr && g8 == 0) {
+      __nv_bfloat16* tp = tC + c * 2LL * D + 2 * t4;
+#pragma unroll
+      for (int nt = 0; nt < D / 8; ++nt) {
+        const float v0 = acc[nt][2] + zq[nt][0], v1 = acc[nt][3] + zq[nt][1];
+        const uint32_t h = pack_bf16x2(v0, v1);
+        *reinterpret_cast<uint32_t*>(tp + nt * 8) = h;
+        *reinterpret_cast<uint32_t*>(tp + D + nt * 8) = pack_bf16x2(v0 - bf16_lo(h), v1 - bf16_hi(h));
+      }
+    }
     gram_tile(sbase, pitch, n_R, n_C, ncols, D, F_C, 2, c * fsz * 2, ncols, fsz);
   }
 }
@@ -524,7 +535,7 @@ rocs_status fused_launch(rocs_context* ctx, const TIN* E_R, const TIN* E_C, cons
   const int D = 128;
   const int pitch = D * 2 + 16;
   const int trows = fm_trows(n_R, n_C);
-  const size_t smem = (size_t)FC_STAGES * NC_MAX * D * sizeof(TIN) + (size_t)FC_CONSUMERS * trows * pitch;
+  const size_t smem = (size_t)FC_STAGES * NC_MAX * D * sizeof(TIN) + (size_t)FC_CONSUMERS * (trows + NC_MAX) * pitch;
   if (n_C > NC_MAX || o_C > LCB_OMAX_F || smem > 220 * 1024) {
     set_error("fused candidate pass: unsupported n_C=%d o_C=%d", n_C, o_C);
     return ROCS_ERR_UNSUPPORTED;
