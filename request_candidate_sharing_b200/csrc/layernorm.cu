@@ -221,6 +221,183 @@ rocs_status dispatch(const void* X1, int w1, long long ld1, const void* X2, long
 #undef ROCS_LN
 }
 
+// ---------------------------------------------------------------------------------------------
+// Streaming variant for long row counts with contiguous rows (ld == width of every operand):
+// one CTA per SM walks a contiguous row range; one thread bulk-copies blocks of RB rows of the two
+// segments and the residual into a ring of shared-memory stages, LN_CONSUMERS warps normalise
+// them (one row at a time per warp, lane j holding the float4 groups j, j + 32, ...) and write the
+// outputs straight from registers.  gamma/beta live in shared memory.
+// ---------------------------------------------------------------------------------------------
+constexpr int LN_CONSUMERS = 8;
+constexpr int LN_STAGES = 8;
+constexpr int LN_STAGE_BYTES = 16384;
+
+template <typename T>
+__device__ __forceinline__ void ld4(const T* p, float (&v)[4]);
+template <>
+__device__ __forceinline__ void ld4<float>(const float* p, float (&v)[4]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+}
+template <>
+__device__ __forceinline__ void ld4<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[4]) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
+}
+
+template <typename TIN, typename TRES, typename TOUT, int NV>
+__global__ void __launch_bounds__(32 * (1 + LN_CONSUMERS), 1) layernorm_ring_kernel(
+    const TIN* __restrict__ X1, int w1, const TIN* __restrict__ X2, const TRES* __restrict__ R, long long rows,
+    long long rows_per_block, int RB, const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
+    TOUT* __restrict__ Y, __nv_bfloat16* __restrict__ Y2, long long ldy2, int* status) {
+  constexpr int width = NV * 128;
+  const int w2 = width - w1;
+  extern __shared__ __align__(128) uint8_t ln_smem[];
+  float* s_gamma = reinterpret_cast<float*>(ln_smem);
+  float* s_beta = s_gamma + width;
+  uint8_t* ring = ln_smem + 2 * width * sizeof(float);
+  __shared__ __align__(8) uint64_t full[LN_STAGES], empty[LN_STAGES];
+  __shared__ int abort_flag_s;
+  volatile int* abort_flag = &abort_flag_s;
+
+  const long long r0 = (long long)blockIdx.x * rows_per_block;
+  const long long r1 = r0 + rows_per_block < rows ? r0 + rows_per_block : rows;
+  if (r0 >= r1) return;
+  const int nblk = (int)((r1 - r0 + RB - 1) / RB);
+  // stage layout: RB rows of X1 | RB rows of X2 | RB rows of R
+  const int off2 = RB * w1 * (int)sizeof(TIN);
+  const int offr = off2 + RB * w2 * (int)sizeof(TIN);
+
+  for (int i = threadIdx.x; i < width; i += blockDim.x) {
+    s_gamma[i] = gamma[i];
+    s_beta[i] = beta[i];
+  }
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < LN_STAGES; ++k) {
+      mbar_init(&full[k], 1);
+      mbar_init(&empty[k], 32);
+    }
+    abort_flag_s = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int b = 0; b < nblk; ++b) {
+        const int st = b % LN_STAGES, use = b / LN_STAGES;
+        if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1, status, abort_flag)) break;
+        const long long row = r0 + (long long)b * RB;
+        const int nr = (int)(r1 - row < RB ? r1 - row : RB);
+        uint8_t* sb = ring + st * LN_STAGE_BYTES;
+        const uint32_t b1 = (uint32_t)(nr * w1 * sizeof(TIN)), b2 = (uint32_t)(nr * w2 * sizeof(TIN)),
+                       br = R != nullptr ? (uint32_t)(nr * width * sizeof(TRES)) : 0u;
+        mbar_arrive_expect_tx(&full[st], b1 + b2 + br);
+        bulk_load(sb, X1 + row * w1, b1, &full[st]);
+        if (b2) bulk_load(sb + off2, X2 + row * w2, b2, &full[st]);
+        if (br) bulk_load(sb + offr, R + row * width, br, &full[st]);
+        issued = b + 1;
+      }
+      for (int b = issued - LN_STAGES < 0 ? 0 : issued - LN_STAGES; b < issued; ++b)
+        mbar_wait(&full[b % LN_STAGES], (b / LN_STAGES) & 1, status, nullptr);
+    }
+    return;
+  }
+
+  const int cw = warp - 1;
+  for (int b = cw; b < nblk; b += LN_CONSUMERS) {
+    const int st = b % LN_STAGES;
+    if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (b / LN_STAGES) & 1, status, abort_flag))) break;
+    const uint8_t* sb = ring + st * LN_STAGE_BYTES;
+    const long long row0 = r0 + (long long)b * RB;
+    const int nr = (int)(r1 - row0 < RB ? r1 - row0 : RB);
+    for (int k = 0; k < nr; ++k) {
+      float v[NV][4];
+      float s = 0.f;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const int col = (i * 32 + lane) * 4;
+        if (col < w1) ld4<TIN>(reinterpret_cast<const TIN*>(sb) + k * w1 + col, v[i]);
+        else ld4<TIN>(reinterpret_cast<const TIN*>(sb + off2) + k * w2 + (col - w1), v[i]);
+        if (R != nullptr) {
+          float rr[4];
+          ld4<TRES>(reinterpret_cast<const TRES*>(sb + offr) + k * width + col, rr);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) v[i][j] += rr[j];
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) s += v[i][j];
+      }
+      if (k == nr - 1) mbar_arrive(&empty[st]);   // every read of this stage is done
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      const float mean = s * (1.0f / (float)width);
+      float q = 0.f;
+#pragma unroll
+      for (int i = 0; i < NV; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float d = v[i][j] - mean;
+          q += d * d;
+        }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+      const float rstd = rsqrtf(q * (1.0f / (float)width) + eps);
+      const long long row = row0 + k;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const int col = (i * 32 + lane) * 4;
+        const float4 gm = *reinterpret_cast<const float4*>(s_gamma + col);
+        const float4 bt = *reinterpret_cast<const float4*>(s_beta + col);
+        float o[4] = {(v[i][0] - mean) * rstd * gm.x + bt.x, (v[i][1] - mean) * rstd * gm.y + bt.y,
+                      (v[i][2] - mean) * rstd * gm.z + bt.z, (v[i][3] - mean) * rstd * gm.w + bt.w};
+        store_vec<TOUT, 4>(Y + row * width + col, o);
+        if (Y2 != nullptr) store_vec<__nv_bfloat16, 4>(Y2 + row * ldy2 + col, o);
+      }
+    }
+  }
+}
+
+template <typename TIN, typename TRES, typename TOUT, int NV>
+rocs_status run_ring(rocs_context* ctx, const void* X1, int w1, const void* X2, const void* R, long long rows,
+                     const float* g, const float* b, float eps, void* Y, void* Y2, long long ldy2, cudaStream_t s) {
+  constexpr int width = NV * 128;
+  const int row_bytes = (int)(width * sizeof(TIN) + (R != nullptr ? width * sizeof(TRES) : 0));
+  const int RB = LN_STAGE_BYTES / row_bytes;
+  const size_t smem = 2 * width * sizeof(float) + (size_t)LN_STAGES * LN_STAGE_BYTES;
+  static bool attr[64] = {false};
+  if (ctx->device < 64 && !attr[ctx->device]) {
+    rocs_status st = cuda_check(cudaFuncSetAttribute(layernorm_ring_kernel<TIN, TRES, TOUT, NV>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
+                                "cudaFuncSetAttribute(layernorm_ring)");
+    if (st != ROCS_OK) return st;
+    attr[ctx->device] = true;
+  }
+  const long long blocks = ctx->num_sms;
+  long long per_block = (rows + blocks - 1) / blocks;
+  per_block = (per_block + RB - 1) / RB * RB;
+  LaunchTimer lt_("layernorm", s);
+  layernorm_ring_kernel<TIN, TRES, TOUT, NV><<<(unsigned)blocks, 32 * (1 + LN_CONSUMERS), smem, s>>>(
+      (const TIN*)X1, w1, (const TIN*)X2, (const TRES*)R, rows, per_block, RB, g, b, eps, (TOUT*)Y,
+      (__nv_bfloat16*)Y2, ldy2, ctx->d_status);
+  return cuda_check(cudaGetLastError(), "layernorm_ring_kernel");
+}
+
+template <typename TIN, typename TRES, typename TOUT>
+rocs_status dispatch_ring(rocs_context* ctx, const void* X1, int w1, const void* X2, const void* R, long long rows,
+                          int width, const float* g, const float* b, float eps, void* Y, void* Y2, long long ldy2,
+                          cudaStream_t s) {
+  switch (width) {
+    case 256: return run_ring<TIN, TRES, TOUT, 2>(ctx, X1, w1, X2, R, rows, g, b, eps, Y, Y2, ldy2, s);
+    case 512: return run_ring<TIN, TRES, TOUT, 4>(ctx, X1, w1, X2, R, rows, g, b, eps, Y, Y2, ldy2, s);
+    case 1024: return run_ring<TIN, TRES, TOUT, 8>(ctx, X1, w1, X2, R, rows, g, b, eps, Y, Y2, ldy2, s);
+    case 2048: return run_ring<TIN, TRES, TOUT, 16>(ctx, X1, w1, X2, R, rows, g, b, eps, Y, Y2, ldy2, s);
+    default: return ROCS_ERR_UNSUPPORTED;
+  }
+}
+
 __global__ void convert_kernel(const __nv_bfloat16* __restrict__ src, long long ld_src, float* __restrict__ dst,
                                long long ld_dst, long long rows, int cols) {
   const long long total = rows * cols;
@@ -238,13 +415,27 @@ rocs_status launch_layernorm(rocs_context* ctx, const void* X1, int w1, long lon
                              long long ld2, const void* res, long long ldr, long long rows, const float* gamma,
                              const float* beta, float eps, void* Y, long long ldy, int in_f32, int res_f32,
                              int y_bf16, void* Y2, long long ldy2, cudaStream_t s) {
-  (void)ctx;
   if (rows == 0) return ROCS_OK;
   const int width = w1 + w2;
   auto al = [](const void* p) { return p == nullptr || ((uintptr_t)p & 15) == 0; };
   const bool vec = (w1 % 8 == 0) && (width % 8 == 0) && ld1 % 8 == 0 && (X2 == nullptr || ld2 % 8 == 0) &&
                    (res == nullptr || ldr % 8 == 0) && ldy % 8 == 0 && (Y2 == nullptr || ldy2 % 8 == 0) && al(X1) &&
                    al(X2) && al(res) && al(Y) && al(Y2);
+  // long runs of contiguous rows: the streaming (bulk-copy ring) variant
+  const bool ring = vec && ctx != nullptr && rows >= 16384 && w1 % 128 == 0 && ld1 == w1 &&
+                    (X2 == nullptr ? w2 == 0 : ld2 == w2) && (res == nullptr || ldr == width) && ldy == width;
+  if (ring) {
+    rocs_status st = ROCS_ERR_UNSUPPORTED;
+    if (in_f32 && !y_bf16 && (res_f32 || res == nullptr))
+      st = dispatch_ring<float, float, float>(ctx, X1, w1, X2, res, rows, width, gamma, beta, eps, Y, Y2, ldy2, s);
+    else if (in_f32 && !y_bf16)
+      st = dispatch_ring<float, __nv_bfloat16, float>(ctx, X1, w1, X2, res, rows, width, gamma, beta, eps, Y, Y2,
+                                                      ldy2, s);
+    else if (!in_f32 && y_bf16 && !(res != nullptr && res_f32))
+      st = dispatch_ring<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(ctx, X1, w1, X2, res, rows, width, gamma, beta,
+                                                                      eps, Y, Y2, ldy2, s);
+    if (st != ROCS_ERR_UNSUPPORTED) return st;
+  }
   if (in_f32 && y_bf16) {
     set_error("layernorm: fp32 inputs with a bf16 primary output are not instantiated");
     return ROCS_ERR_UNSUPPORTED;

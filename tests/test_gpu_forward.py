@@ -107,3 +107,22 @@ def test_forward_end_to_end_scoring(R):
     for l in range(case.dca.layers):
         check_bf16(host(out["A_R"][l]), ref["A_R"][l], what=f"A_R_{l}")
         check_bf16(host(out["A_C"][l]), ref["A_C"][l], what=f"A_C_{l}")
+
+
+def test_forward_glm_stack_many_candidates(R):
+    """More than 16384 candidates: the candidate LayerNorm takes its streaming (bulk-copy ring)
+    path, layer 0 with an fp32 input and a bf16 residual, and each CTA of the fused candidate
+    pass walks thousands of candidates across request boundaries.  Sampled candidates (first and
+    last of every request among them) against the oracle."""
+    from tests.gpu_util import sample_candidates
+    counts = [6000, 1, 5000, 0, 7000, 2999]
+    case = synth.model_cfg3(B_R=len(counts), counts=counts, seed=11)
+    x, W = synth.model_inputs(case), synth.model_weights(case)
+    out = run_forward(R, case, x, W)
+    _, m = O.segments(case.counts)
+    rows = sample_candidates(case.counts, 6)
+    xs = dict(x)
+    xs["E_C"] = x["E_C"][rows]
+    ref = O.forward_cfg3(case, xs, W, m[rows])
+    check_bf16(host(out["E_R"]), ref["E_R"], what="E_R")
+    check_bf16(host(out["E_C"][torch.from_numpy(rows).cuda()]), ref["E_C"], what="E_C sample")

@@ -191,7 +191,11 @@ def test_linear_cfg2_sampled_full_size(R):
 # ---------------------------------------------------------------------------------------------
 @pytest.mark.parametrize("io", [0, 1])
 @pytest.mark.parametrize("w1,w2,res,rows", [(2048, 2048, True, 37), (1024, 1024, True, 300), (256, 0, True, 1000),
-                                            (100, 28, False, 9), (4096, 0, False, 3)])
+                                            (100, 28, False, 9), (4096, 0, False, 3),
+                                            # >= 16384 contiguous rows: the streaming (bulk-copy ring) path,
+                                            # ragged against its row blocks and CTA ranges
+                                            (1024, 1024, True, 20011), (256, 0, True, 40001),
+                                            (512, 0, False, 16384)])
 def test_group_layernorm(R, io, w1, w2, res, rows):
     g = np.random.default_rng(w1 + w2 + rows)
     tdt = torch.bfloat16 if io == 1 else torch.float32
