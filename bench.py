@@ -70,6 +70,9 @@ def make_case(name: str, rank: int, requests: int = 0):
 # ---------------------------------------------------------------------------------------------
 # algorithmic work per launch (for the roofline of the dominant kernel)
 # ---------------------------------------------------------------------------------------------
+ATTN_MUFU_SHARE = 5.0 / 8.0   # share of the attention softmax's exponentials evaluated on MUFU
+
+
 def algo_work(case, label: str):
     """(bound, amount per launch, unit) for a timing-report label "<site>:<kernel>", or None.
     GEMMs: mathematical flops 2*M*N*K (a split hi/lo operand counts once).  Bandwidth-bound
@@ -145,9 +148,11 @@ def roofline_entry(case, label, launches, total_ms, peaks, sustained: bool):
         peak = peaks["hbm"]
         unit = "GB/s"
     else:
-        # MUFU ex2: 16 per clock per SM (4 per SM sub-partition) x 148 SMs at the max SM clock
+        # exp2 throughput: MUFU does 16 per clock per SM at the max SM clock and takes 5/8 of the
+        # softmax's exponentials (the other 3/8 run as a polynomial on the FMA pipe), so MUFU
+        # caps the rate at 16 / (5/8) = 25.6 exponentials per clock per SM
         achieved = amount / per_launch_s / 1e9
-        peak = 16 * 148 * peaks["sm_mhz"] * 1e6 / 1e9
+        peak = 16 / ATTN_MUFU_SHARE * 148 * peaks["sm_mhz"] * 1e6 / 1e9
         unit = "Gexp2/s"
     return {"kernel": label, "bound": bound, "achieved": round(achieved, 3), "peak": round(peak, 1), "unit": unit,
             "frac": round(achieved / peak, 4), "per_launch_ms": round(total_ms / launches, 4), "launches": launches,
