@@ -36,18 +36,21 @@ constexpr int B_STAGE = BN_MAX * BK * 2;   // 32 KiB
 constexpr int THREADS = 320;
 constexpr int EPI_THREADS = 256;
 constexpr int TMEM_COLS = 512;
-constexpr int SMEM_BYTES = 1024 + STAGES * (A_STAGE + B_STAGE) + 256;
+constexpr int EPI_BUF = 4096;              // per epilogue warp: one 32x32 output chunk (fp32, or bf16 hi + lo)
+constexpr int SMEM_BYTES = 1024 + STAGES * (A_STAGE + B_STAGE) + (EPI_THREADS / 32) * EPI_BUF + 256;
 
 struct Problem {
   CUtensorMap tmA;
   CUtensorMap tmB;
+  CUtensorMap tmO;     // output [M, N] (out_mode 2: the hi half), box 32 x 32, stored by TMA
+  CUtensorMap tmOlo;   // out_mode 2: the lo half at column offset lo_off
   const float* bias;
   const float* Z;
   const int32_t* gidx;
   void* out;
   long long ldo, ldz;
   int M, N, K, BN;
-  int out_mode, act, gidx_bound, vec_ok;
+  int out_mode, act, gidx_bound, vec_ok, tma_out;
   int m_tiles, n_tiles, k_blocks, b_kblocks, tile_start, n_start;
   long long lo_off;   // out_mode 2: column offset of the low half
 };
@@ -127,12 +130,105 @@ __device__ __forceinline__ void store_chunk(const Problem& pr, long long grow, i
   }
 }
 
+// bias, the request contribution Z[gidx[row]] and the activation on one thread's 32 values
+__device__ __forceinline__ void epilogue_math(const Problem& pr, const float* zrow, int col0, float (&v)[32]) {
+  const bool full32 = (col0 + 32 <= pr.N) && pr.vec_ok;
+  if (pr.bias != nullptr) {
+    if (full32) {
+      const float4* b4 = reinterpret_cast<const float4*>(pr.bias + col0);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float4 b = __ldg(b4 + j);
+        v[4 * j] += b.x; v[4 * j + 1] += b.y; v[4 * j + 2] += b.z; v[4 * j + 3] += b.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (col0 + j < pr.N) v[j] += pr.bias[col0 + j];
+    }
+  }
+  if (zrow != nullptr) {
+    if (full32) {
+      const float4* z4 = reinterpret_cast<const float4*>(zrow + col0);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float4 z = __ldg(z4 + j);
+        v[4 * j] += z.x; v[4 * j + 1] += z.y; v[4 * j + 2] += z.z; v[4 * j + 3] += z.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (col0 + j < pr.N) v[j] += zrow[col0 + j];
+    }
+  }
+  switch (pr.act) {
+    case ROCS_ACT_RELU:
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = fmaxf(v[j], 0.f);
+      break;
+    case ROCS_ACT_GELU:
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
+      break;
+    case ROCS_ACT_SIGMOID:
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = sigmoid_fast(v[j]);
+      break;
+    default:
+      break;
+  }
+}
+
+// One warp's 32 x 32 output chunk (lane = row) through shared memory and one TMA store: rows are
+// written into `buf` in the layout of the output map's swizzle (128-byte rows for fp32, 64-byte
+// rows for bf16: the 16-byte unit j of row r sits at j ^ (r & 7), resp. j ^ ((r >> 1) & 3)),
+// so the shared-memory writes are free of bank conflicts and the global write is whole lines.
+__device__ __forceinline__ void store_chunk_tma(const Problem& pr, uint8_t* buf, int row0, int col0,
+                                                const float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+  if (lane == 0) bulk_wait_read_all();   // the previous chunk's copy has read the buffer
+  __syncwarp();
+  if (pr.out_mode == 0) {
+    uint8_t* rowp = buf + lane * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      *reinterpret_cast<float4*>(rowp + ((j ^ (lane & 7)) << 4)) =
+          make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  } else {
+    uint8_t* rowp = buf + lane * 64;
+    const int sw = (lane >> 1) & 3;
+    uint32_t hi[16], lo[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      hi[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+      if (pr.out_mode == 2) lo[j] = pack_bf16x2(v[2 * j] - bf16_lo(hi[j]), v[2 * j + 1] - bf16_hi(hi[j]));
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      *reinterpret_cast<uint4*>(rowp + ((j ^ sw) << 4)) = make_uint4(hi[4 * j], hi[4 * j + 1], hi[4 * j + 2], hi[4 * j + 3]);
+    if (pr.out_mode == 2) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<uint4*>(rowp + 2048 + ((j ^ sw) << 4)) =
+            make_uint4(lo[4 * j], lo[4 * j + 1], lo[4 * j + 2], lo[4 * j + 3]);
+    }
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(&pr.tmO, buf, col0, row0);
+    if (pr.out_mode == 2) tma_store_2d(&pr.tmOlo, buf + 2048, col0, row0);
+    bulk_commit_group();
+  }
+}
+
 __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_constant__ Params P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = base;
   uint8_t* sB = base + STAGES * A_STAGE;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE);
+  uint8_t* sEpi = sB + STAGES * B_STAGE;   // 1024-B aligned
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + (EPI_THREADS / 32) * EPI_BUF);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* tfull = bars + 2 * STAGES;
@@ -260,6 +356,8 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
           zrow = pr.Z + (long long)zi * pr.ldz;
         }
       }
+      // a row with a bad request index is skipped, not written: such a warp stores element-wise
+      const bool use_tma = pr.tma_out && !__any_sync(0xffffffffu, grow < pr.M && !rvalid);
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MAX);
       const int nchunks = pr.BN / 32;
       // this warp takes chunks half, half + 2, ...; it releases the accumulator after its last load
@@ -277,7 +375,14 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
           mbar_arrive(&tempty[acc]);
         }
         const int col0 = nb * pr.BN + c * 32;
-        if (rvalid && col0 < pr.N) {
+        if (use_tma && col0 < pr.N && mb * BM + q * 32 < pr.M) {
+          // every lane takes part in the staged store; rows past M are clipped by the copy
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          if (rvalid) epilogue_math(pr, zrow, col0, v);
+          store_chunk_tma(pr, sEpi + (warp - 2) * EPI_BUF, mb * BM + q * 32, col0, v);
+        } else if (!use_tma && rvalid && col0 < pr.N) {
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
@@ -332,6 +437,9 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
+    // this warp's output stores have landed before the CTA (and its staging memory) goes away
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -356,6 +464,21 @@ bool encode_bf16_kmajor(rocs_context* ctx, CUtensorMap* map, const void* ptr, lo
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Output map for the TMA-store epilogue: [rows, cols] with row stride ld elements, box 32 x 32,
+// swizzled to match store_chunk_tma's shared-memory layout.
+bool encode_out(rocs_context* ctx, CUtensorMap* map, void* ptr, long long rows, int cols, long long ld, bool f32) {
+  EncodeTiledFn fn = reinterpret_cast<EncodeTiledFn>(ctx->encode_fn);
+  const int es = f32 ? 4 : 2;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * es};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -414,6 +537,17 @@ rocs_status launch_gemm_bf16(rocs_context* ctx, const GemmDesc* probs, int nprob
     const int ve = g.out_mode == 0 ? 4 : 8;
     p.vec_ok = (g.ldo % ve == 0) && (((uintptr_t)g.out & 15) == 0) && (!g.bias || ((uintptr_t)g.bias & 15) == 0) &&
                (!g.Z || (((uintptr_t)g.Z & 15) == 0 && g.ldz % 4 == 0)) && (g.out_mode != 2 || g.N % 8 == 0);
+    // TMA-store epilogue when the output rows are 16-byte aligned (and, for hi/lo pairs, the
+    // low half starts on a 16-byte boundary); element stores otherwise
+    {
+      const bool f32 = g.out_mode == 0;
+      const int es = f32 ? 4 : 2;
+      bool ok = ((uintptr_t)g.out & 15) == 0 && (g.ldo * es) % 16 == 0 && (g.out_mode != 2 || (g.N * 2) % 16 == 0);
+      ok = ok && encode_out(ctx, &p.tmO, g.out, g.M, g.N, g.ldo, f32);
+      if (ok && g.out_mode == 2)
+        ok = encode_out(ctx, &p.tmOlo, reinterpret_cast<__nv_bfloat16*>(g.out) + g.N, g.M, g.N, g.ldo, false);
+      p.tma_out = ok ? 1 : 0;
+    }
     p.m_tiles = (g.M + BM - 1) / BM;
     p.n_tiles = (g.N + p.BN - 1) / p.BN;
     p.b_kblocks = (g.K + BK - 1) / BK;
