@@ -443,7 +443,9 @@ def run_librocs(args, rank, world, local):
                        "description": WORKLOADS[args.workload], "B_R": case.B_R,
                        "B_C_per_rank": B_C, "l2": "inputs larger than L2 (E_C alone is "
                        f"{(xd['E_C'].numel() * 2 / 1e9) if 'E_C' in xd else 0:.2f} GB)",
-                       "parallelism": f"replicas x{world}"},
+                       "parallelism": f"replicas x{world}",
+                       "launch": "value: direct launches with per-launch CUDA events (the per-kernel report); "
+                                 "e2e: the forward's captured CUDA graph replayed"},
             "roofline": top,
             "e2e": {"value": round(e2e_value, 1), "unit": "candidates/s", "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": int(d2h)},

@@ -257,6 +257,15 @@ rocs_status rocs_dca_encode(rocs_handle_t handle, const rocs_dca_desc* desc, con
  * stream, MLP and LCB outputs, attention outputs) stay fp32, so rounding of intermediates does
  * not accumulate across the stacked layers.  Split operands need widths that are multiples of
  * 64 (n_R^2, n_C(n_R+n_C), hidden, q_dim, d).
+ * Graph replay (a11): the handle records each distinct call (the bytes of the descriptor, the
+ * weight/input/output pointer structs and the workspace pointer and size).  The first call
+ * with a given record launches the kernels directly; the second captures the same launch
+ * sequence into a CUDA graph (on a stream the handle owns) and launches it on `stream`; later
+ * calls replay it.  The graph reads the caller's buffers at replay time, so new contents of
+ * the same buffers are picked up; different pointers or sizes make a new record (the handle
+ * keeps the 8 most recent).  rocs_set_graph_replay(h, 0) turns replay off (every call then
+ * launches directly), as does per-launch timing while it runs.  Not callable while `stream`
+ * itself is being captured by the caller when replay is on.
  * ---------------------------------------------------------------------------------------- */
 typedef struct {
   const void *W_RR, *W_CR, *W_CC;  /* bf16 [out, in] */
@@ -318,6 +327,9 @@ rocs_status rocs_forward_workspace(rocs_handle_t handle, const rocs_model_desc* 
 rocs_status rocs_forward(rocs_handle_t handle, const rocs_model_desc* model,
                          const rocs_model_weights* weights, const rocs_inputs* inputs,
                          rocs_outputs* outputs, void* workspace, size_t workspace_bytes, void* stream);
+/* Turns rocs_forward's graph replay on (enable = 1, the default) or off (0) for this handle.
+ * Errors: ROCS_ERR_INVALID_ARG for a NULL handle or another value of enable. */
+rocs_status rocs_set_graph_replay(rocs_handle_t handle, int32_t enable);
 
 /* ------------------------------------------------------------------------------------------
  * Per-launch timing (tracing).  After rocs_timing_start(h, max_launches), every kernel the

@@ -249,6 +249,9 @@ extern "C" rocs_status rocs_create(rocs_handle_t* handle, int device) {
 extern "C" rocs_status rocs_destroy(rocs_handle_t h) {
   if (!h) return ROCS_OK;
   cudaDeviceSynchronize();
+  for (ForwardGraph& g : h->graphs)
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+  if (h->capture_stream) cudaStreamDestroy(h->capture_stream);
   if (h->d_status) cudaFree(h->d_status);
   delete h;
   return ROCS_OK;
@@ -699,47 +702,12 @@ extern "C" rocs_status rocs_forward_workspace(rocs_handle_t h, const rocs_model_
   return ROCS_OK;
 }
 
-extern "C" rocs_status rocs_forward(rocs_handle_t h, const rocs_model_desc* m, const rocs_model_weights* W,
-                                    const rocs_inputs* in, rocs_outputs* out, void* ws, size_t ws_bytes,
-                                    void* stream) {
-  CtxGuard ctx_guard_(h);
-  ROCS_REQUIRE(h, "rocs_forward: handle is NULL");
-  ROCS_TRY(check_model(m));
-  ROCS_REQUIRE(W && in && out && in->counts, "rocs_forward: NULL argument");
-  if (m->glm_layers > 0) ROCS_REQUIRE(in->E_R && (m->B_C == 0 || in->E_C), "rocs_forward: GLM inputs NULL");
-  if (m->dca_layers > 0) {
-    ROCS_REQUIRE(in->Hist, "rocs_forward: Hist NULL");
-    if (m->dca_query_source == 0) ROCS_REQUIRE(in->Y_R && (m->B_C == 0 || in->Y_C), "rocs_forward: Y_R/Y_C NULL");
-  }
-  for (int l = 0; l < m->glm_layers; ++l) {
-    const rocs_glm_layer_weights& g = W->glm[l];
-    ROCS_REQUIRE(g.mlp1.W_RR && g.mlp1.W_CR && g.mlp1.W_CC && g.mlp1.b_R && g.mlp1.b_C && g.mlp2.W_RR &&
-                     g.mlp2.W_CR && g.mlp2.W_CC && g.mlp2.b_R && g.mlp2.b_C && g.P_RR && g.P_CR && g.P_CC &&
-                     g.lnR_gamma && g.lnR_beta && g.lnC_gamma && g.lnC_beta,
-                 "rocs_forward: GLM layer %d has a NULL weight", l);
-  }
-  for (int l = 0; l < m->dca_layers; ++l) {
-    const rocs_dca_layer_weights& x = W->dca[l];
-    const rocs_qgen_weights& q = W->qgen[l];
-    ROCS_REQUIRE(x.Wq && x.Wk && x.Wv && x.Wo && x.ln_gamma && x.ln_beta && x.WK_R && x.WV_R && x.WK_C && x.WV_C &&
-                     q.p_RR && q.p_CR && q.p_CC && q.mlp1.W_RR && q.mlp1.W_CR && q.mlp1.W_CC && q.mlp1.b_R &&
-                     q.mlp1.b_C && q.mlp2.W_RR && q.mlp2.W_CR && q.mlp2.W_CC && q.mlp2.b_R && q.mlp2.b_C,
-                 "rocs_forward: DCA layer %d has a NULL weight", l);
-  }
-  if (m->score_h1 > 0) {
-    const rocs_score_weights& sc = W->score;
-    ROCS_REQUIRE(sc.s1.W_CR && sc.s1.W_CC && sc.s1.b_C && sc.W2 && sc.b2 && sc.w3 && sc.b3,
-                 "rocs_forward: scoring head has a NULL weight");
-  }
-  const bool own_off = out->offsets == nullptr, own_req = out->req_idx == nullptr;
-  FwdPlan need = plan_forward(m, nullptr, own_off, own_req);
-  if (!ws || ws_bytes < need.bytes) {
-    set_error("rocs_forward: workspace %zu B < required %zu B", ws_bytes, need.bytes);
-    return ROCS_ERR_WORKSPACE;
-  }
-  ROCS_REQUIRE(aligned16(ws), "rocs_forward: workspace must be 16-byte aligned");
-  FwdPlan p = plan_forward(m, ws, own_off, own_req);
-  cudaStream_t s = (cudaStream_t)stream;
+namespace {
+
+// The forward's launch sequence (a0 .. a10) on stream s, after validation and planning.
+rocs_status forward_launches(rocs_handle_t h, const rocs_model_desc* m, const rocs_model_weights* W,
+                             const rocs_inputs* in, rocs_outputs* out, const FwdPlan& p, bool own_off, bool own_req,
+                             cudaStream_t s) {
   const int BR = m->B_R;
   const long long BC = m->B_C;
   int32_t* offsets = own_off ? p.offsets : out->offsets;
@@ -949,9 +917,116 @@ extern "C" rocs_status rocs_forward(rocs_handle_t h, const rocs_model_desc* m, c
   return ROCS_OK;
 }
 
+// Key of one rocs_forward call: every byte that the launch sequence depends on.
+std::vector<uint8_t> forward_key(const rocs_model_desc* m, const rocs_model_weights* W, const rocs_inputs* in,
+                                 const rocs_outputs* out, const void* ws, size_t ws_bytes) {
+  std::vector<uint8_t> k;
+  auto put = [&](const void* p, size_t n) {
+    const uint8_t* b = static_cast<const uint8_t*>(p);
+    k.insert(k.end(), b, b + n);
+  };
+  put(m, sizeof(*m));
+  put(W, sizeof(*W));
+  put(in, sizeof(*in));
+  put(out, sizeof(*out));
+  put(&ws, sizeof(ws));
+  put(&ws_bytes, sizeof(ws_bytes));
+  return k;
+}
+
+}  // namespace
+
+extern "C" rocs_status rocs_forward(rocs_handle_t h, const rocs_model_desc* m, const rocs_model_weights* W,
+                                    const rocs_inputs* in, rocs_outputs* out, void* ws, size_t ws_bytes,
+                                    void* stream) {
+  CtxGuard ctx_guard_(h);
+  ROCS_REQUIRE(h, "rocs_forward: handle is NULL");
+  ROCS_TRY(check_model(m));
+  ROCS_REQUIRE(W && in && out && in->counts, "rocs_forward: NULL argument");
+  if (m->glm_layers > 0) ROCS_REQUIRE(in->E_R && (m->B_C == 0 || in->E_C), "rocs_forward: GLM inputs NULL");
+  if (m->dca_layers > 0) {
+    ROCS_REQUIRE(in->Hist, "rocs_forward: Hist NULL");
+    if (m->dca_query_source == 0) ROCS_REQUIRE(in->Y_R && (m->B_C == 0 || in->Y_C), "rocs_forward: Y_R/Y_C NULL");
+  }
+  for (int l = 0; l < m->glm_layers; ++l) {
+    const rocs_glm_layer_weights& g = W->glm[l];
+    ROCS_REQUIRE(g.mlp1.W_RR && g.mlp1.W_CR && g.mlp1.W_CC && g.mlp1.b_R && g.mlp1.b_C && g.mlp2.W_RR &&
+                     g.mlp2.W_CR && g.mlp2.W_CC && g.mlp2.b_R && g.mlp2.b_C && g.P_RR && g.P_CR && g.P_CC &&
+                     g.lnR_gamma && g.lnR_beta && g.lnC_gamma && g.lnC_beta,
+                 "rocs_forward: GLM layer %d has a NULL weight", l);
+  }
+  for (int l = 0; l < m->dca_layers; ++l) {
+    const rocs_dca_layer_weights& x = W->dca[l];
+    const rocs_qgen_weights& q = W->qgen[l];
+    ROCS_REQUIRE(x.Wq && x.Wk && x.Wv && x.Wo && x.ln_gamma && x.ln_beta && x.WK_R && x.WV_R && x.WK_C && x.WV_C &&
+                     q.p_RR && q.p_CR && q.p_CC && q.mlp1.W_RR && q.mlp1.W_CR && q.mlp1.W_CC && q.mlp1.b_R &&
+                     q.mlp1.b_C && q.mlp2.W_RR && q.mlp2.W_CR && q.mlp2.W_CC && q.mlp2.b_R && q.mlp2.b_C,
+                 "rocs_forward: DCA layer %d has a NULL weight", l);
+  }
+  if (m->score_h1 > 0) {
+    const rocs_score_weights& sc = W->score;
+    ROCS_REQUIRE(sc.s1.W_CR && sc.s1.W_CC && sc.s1.b_C && sc.W2 && sc.b2 && sc.w3 && sc.b3,
+                 "rocs_forward: scoring head has a NULL weight");
+  }
+  const bool own_off = out->offsets == nullptr, own_req = out->req_idx == nullptr;
+  FwdPlan need = plan_forward(m, nullptr, own_off, own_req);
+  if (!ws || ws_bytes < need.bytes) {
+    set_error("rocs_forward: workspace %zu B < required %zu B", ws_bytes, need.bytes);
+    return ROCS_ERR_WORKSPACE;
+  }
+  ROCS_REQUIRE(aligned16(ws), "rocs_forward: workspace must be 16-byte aligned");
+  FwdPlan p = plan_forward(m, ws, own_off, own_req);
+  cudaStream_t s = (cudaStream_t)stream;
+  // a11: the launch sequence is replayed as a CUDA graph once the same call has been seen
+  // before (the first call runs it eagerly); per-launch timing always runs eagerly
+  if (!h->graph_replay || h->timer.enabled) return forward_launches(h, m, W, in, out, p, own_off, own_req, s);
+  std::vector<uint8_t> key = forward_key(m, W, in, out, ws, ws_bytes);
+  ForwardGraph* fg = nullptr;
+  for (ForwardGraph& g : h->graphs)
+    if (g.key == key) fg = &g;
+  if (fg == nullptr) {
+    if (h->graphs.size() >= kMaxForwardGraphs) {
+      if (h->graphs.front().exec) cudaGraphExecDestroy(h->graphs.front().exec);
+      h->graphs.erase(h->graphs.begin());
+    }
+    h->graphs.push_back(ForwardGraph());
+    fg = &h->graphs.back();
+    fg->key = std::move(key);
+  }
+  if (fg->exec == nullptr && fg->calls++ == 0) return forward_launches(h, m, W, in, out, p, own_off, own_req, s);
+  if (fg->exec == nullptr) {
+    if (h->capture_stream == nullptr)
+      ROCS_TRY(cuda_check(cudaStreamCreateWithFlags(&h->capture_stream, cudaStreamNonBlocking), "cudaStreamCreate"));
+    ROCS_TRY(cuda_check(cudaStreamBeginCapture(h->capture_stream, cudaStreamCaptureModeThreadLocal),
+                        "cudaStreamBeginCapture"));
+    const rocs_status st = forward_launches(h, m, W, in, out, p, own_off, own_req, h->capture_stream);
+    cudaGraph_t graph = nullptr;
+    const cudaError_t ce = cudaStreamEndCapture(h->capture_stream, &graph);
+    if (st != ROCS_OK || ce != cudaSuccess) {
+      if (graph) cudaGraphDestroy(graph);
+      if (st != ROCS_OK) return st;
+      return cuda_check(ce, "cudaStreamEndCapture");
+    }
+    const cudaError_t ie = cudaGraphInstantiate(&fg->exec, graph, 0);
+    cudaGraphDestroy(graph);
+    if (ie != cudaSuccess) {
+      fg->exec = nullptr;
+      return cuda_check(ie, "cudaGraphInstantiate");
+    }
+  }
+  return cuda_check(cudaGraphLaunch(fg->exec, s), "cudaGraphLaunch");
+}
+
 // =============================================================================================
 // per-launch timing
 // =============================================================================================
+extern "C" rocs_status rocs_set_graph_replay(rocs_handle_t h, int32_t enable) {
+  ROCS_REQUIRE(h, "rocs_set_graph_replay: handle is NULL");
+  ROCS_REQUIRE(enable == 0 || enable == 1, "rocs_set_graph_replay: enable must be 0 or 1");
+  h->graph_replay = enable;
+  return ROCS_OK;
+}
+
 extern "C" rocs_status rocs_timing_start(rocs_handle_t h, int32_t max_launches) {
   ROCS_REQUIRE(h, "rocs_timing_start: handle is NULL");
   ROCS_REQUIRE(max_launches >= 1 && max_launches <= (1 << 20), "rocs_timing_start: max_launches out of range");

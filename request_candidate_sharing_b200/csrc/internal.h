@@ -18,13 +18,26 @@ struct RocsTimer {
   long long dropped = 0;           // launches beyond the pool size
 };
 
+// One recorded rocs_forward: the call's argument bytes (model, weights, inputs, outputs,
+// workspace) and, from the second identical call on, its launch sequence as a CUDA graph.
+struct ForwardGraph {
+  std::vector<uint8_t> key;
+  int calls = 0;
+  cudaGraphExec_t exec = nullptr;
+};
+
 struct rocs_context {
   int device = 0;
   int num_sms = 148;
   int* d_status = nullptr;   // sticky device status word
   void* encode_fn = nullptr; // cuTensorMapEncodeTiled
   RocsTimer timer;
+  int graph_replay = 1;                 // rocs_set_graph_replay
+  cudaStream_t capture_stream = nullptr;   // forward graphs are captured here (never the legacy stream)
+  std::vector<ForwardGraph> graphs;     // at most kMaxForwardGraphs, most recent last
 };
+
+constexpr size_t kMaxForwardGraphs = 8;
 
 namespace rocs {
 

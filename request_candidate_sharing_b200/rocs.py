@@ -123,13 +123,15 @@ _lib_fwd = _proto("rocs_forward", P, C.POINTER(ModelDesc), C.POINTER(ModelWeight
                   C.POINTER(Outputs), P, C.c_size_t, P)
 
 _lib_ikbo_na = _proto("rocs_linear_ikbo_noalloc", P, C.POINTER(IkboDesc), P, P, P, P, P, P, P, P, P, P, P)
+_lib_graph = _proto("rocs_set_graph_replay", P, I32)
 _lib_tstart = _proto("rocs_timing_start", P, I32)
 _lib_tstop = _proto("rocs_timing_stop", P, C.c_char_p, C.c_size_t)
 
 EXPORTED = ["rocs_linear_ikbo_noalloc", "rocs_timing_start", "rocs_timing_stop", "rocs_create", "rocs_destroy", "rocs_last_error", "rocs_get_device_status", "rocs_num_sms",
             "rocs_segments_from_counts", "rocs_linear_ikbo_workspace", "rocs_linear_ikbo", "rocs_group_layernorm",
             "rocs_fm_masked", "rocs_token_lcb_workspace", "rocs_token_lcb", "rocs_dca_cross_attn",
-            "rocs_dca_encode_workspace", "rocs_dca_encode", "rocs_forward_workspace", "rocs_forward"]
+            "rocs_dca_encode_workspace", "rocs_dca_encode", "rocs_forward_workspace", "rocs_forward",
+            "rocs_set_graph_replay"]
 
 
 def ptr(x) -> Optional[int]:
@@ -271,6 +273,9 @@ class Rocs:
                      workspace_bytes: int, stream=None):
         _check(_lib_fwd(self.h, C.byref(model), C.byref(weights), C.byref(inputs), C.byref(outputs), ptr(workspace),
                         int(workspace_bytes), stream))
+
+    def rocs_set_graph_replay(self, enable: int):
+        _check(_lib_graph(self.h, int(enable)))
 
 
 # ---- marshalling helpers for the model structs (names follow the synth weight dictionaries) ----

@@ -126,3 +126,48 @@ def test_forward_glm_stack_many_candidates(R):
     ref = O.forward_cfg3(case, xs, W, m[rows])
     check_bf16(host(out["E_R"]), ref["E_R"], what="E_R")
     check_bf16(host(out["E_C"][torch.from_numpy(rows).cuda()]), ref["E_C"], what="E_C sample")
+
+
+def test_forward_graph_replay(R):
+    """a11: the second identical rocs_forward call captures the launch sequence into a CUDA graph
+    and later calls replay it.  On the same buffers every call must equal the eager run bit for
+    bit, and new contents of an input buffer must show in the next replay (the graph reads the
+    caller's buffers, it does not snapshot them)."""
+    from request_candidate_sharing_b200 import rocs
+    case = synth.model_cfg5(B_R=3, counts=[4, 1, 20], L=256)
+    x, W = synth.model_inputs(case), synth.model_weights(case)
+    md = rocs.model_desc(case)
+    Wd = {k: dev(v, torch.float32 if k.endswith(FP32_KEYS) else torch.bfloat16) for k, v in W.items()}
+    g, a = case.glm, case.dca
+    mw = rocs.model_weights(Wd, g.layers, a.layers, True)
+    xin = {k: dev(v) for k, v in x.items()}
+    counts = dev_i32(case.counts)
+    inp = rocs.Inputs(counts.data_ptr(), rocs.ptr(xin.get("E_R")), rocs.ptr(xin.get("E_C")), rocs.ptr(xin.get("H")),
+                      rocs.ptr(xin.get("Y_R")), rocs.ptr(xin.get("Y_C")))
+    score = torch.empty(case.B_C, dtype=torch.float32, device="cuda")
+    EC = torch.empty((case.B_C, g.n_C, g.D), dtype=torch.float32, device="cuda")
+    o = rocs.Outputs(None, None, None, EC.data_ptr(), None, None, None, score.data_ptr())
+    nb = R.rocs_forward_workspace(md)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+
+    def call():
+        R.rocs_forward(md, mw, inp, o, ws, nb, stream())
+        assert R.rocs_get_device_status(stream()) == 0
+        return score.clone(), EC.clone()
+
+    try:
+        R.rocs_set_graph_replay(0)
+        s_eager, e_eager = call()
+        R.rocs_set_graph_replay(1)
+        for _ in range(4):   # eager, capture + launch, replay, replay
+            s_g, e_g = call()
+            assert torch.equal(s_g, s_eager) and torch.equal(e_g, e_eager)
+        # new input contents in the same buffer
+        xin["E_C"].copy_(dev(synth.bf16_round(x["E_C"] * 0.5 + 0.25)))
+        s_new, e_new = call()
+        R.rocs_set_graph_replay(0)
+        s_ref, e_ref = call()
+        assert torch.equal(s_new, s_ref) and torch.equal(e_new, e_ref)
+        assert not torch.equal(s_new, s_eager)
+    finally:
+        R.rocs_set_graph_replay(1)
