@@ -483,15 +483,19 @@ rocs_status encoder_layer(rocs_context* ctx, const EncScratch& e, int B_R, int L
   ROCS_TRY(launch_layernorm(ctx, e.tmp, d, d, nullptr, 0, 0, S_in, d, M, w.ln_gamma, w.ln_beta, 1e-5f, S_out, d, 0, 0,
                             1, nullptr, 0, s));
   SiteLabel sl4("enc.kv");
-  const void* Wk[4] = {w.WK_R, w.WV_R, w.WK_C, w.WV_C};
-  void* kv[4] = {KR, VR, KC, VC};
-  for (int i = 0; i < 4; ++i) {
+  // KR/VR NULL: only the candidate group's K/V (the request query's attention absorbs its
+  // projections, see attn_req.cu)
+  const bool req_kv = KR != nullptr && VR != nullptr;
+  const void* Wk[4] = {w.WK_C, w.WV_C, w.WK_R, w.WV_R};
+  void* kv[4] = {KC, VC, KR, VR};
+  const int nkv = req_kv ? 4 : 2;
+  for (int i = 0; i < nkv; ++i) {
     g[i] = GemmDesc();
     g[i].A = S_out; g[i].lda = d; g[i].M = (int)M; g[i].K = d;
     g[i].B = Wk[i]; g[i].ldb = d; g[i].N = d;
     g[i].out = kv[i]; g[i].ldo = d; g[i].out_mode = 1;
   }
-  return launch_gemm_bf16(ctx, g, 4, s);
+  return launch_gemm_bf16(ctx, g, nkv, s);
 }
 
 rocs_status check_dca_desc(const rocs_dca_desc* d) {
@@ -574,7 +578,7 @@ struct FwdPlan {
   float *Z1, *Z2, *ZL;
   // DCA
   EncScratch enc;
-  void *S[2], *KR, *VR, *KC, *VC;
+  void *S[2], *KR = nullptr, *VR = nullptr, *KC, *VC;   // KR/VR only when the request attention is not absorbed
   float *YR, *YC;            // own-query token streams (fp32)
   void *tR, *tC, *qhR, *qhC, *QR, *QC;   // hi/lo pairs
   float *AR, *AC;            // attention outputs when no caller buffer takes them
@@ -616,8 +620,10 @@ FwdPlan plan_forward(const rocs_model_desc* m, void* ws, bool own_offsets, bool 
     p.enc = carve_encoder(c, rowsL, m->d, m->B_R);
     p.S[0] = c.take(rowsL * m->d * 2);
     p.S[1] = c.take(rowsL * m->d * 2);
-    p.KR = c.take(rowsL * m->d * 2);
-    p.VR = c.take(rowsL * m->d * 2);
+    if (!attention_req_absorbed_supported(m->d, m->H, m->L)) {
+      p.KR = c.take(rowsL * m->d * 2);
+      p.VR = c.take(rowsL * m->d * 2);
+    }
     p.KC = c.take(rowsL * m->d * 2);
     p.VC = c.take(rowsL * m->d * 2);
     if (m->dca_query_source == 0) {
@@ -827,11 +833,14 @@ rocs_status forward_launches(rocs_handle_t h, const rocs_model_desc* m, const ro
       void* xC2 = m->score_h1 > 0 ? (char*)p.xC + (size_t)(wc + (long long)l * m->d) * 2 : nullptr;
       const int dh = m->d / m->H;
       const float scale = 1.0f / std::sqrt((float)dh);
-      const long long kvs = (long long)m->L * m->d;
       {
         SiteLabel s_xa("xattn.req");
-        ROCS_TRY(launch_attention_single(h, p.QR, d2, 1, p.KR, p.VR, m->d, kvs, p.iota1, BR, BR, m->L, m->H, dh,
-                                         scale, dR, ldR, 0, xR2, xr, s));
+        if (p.KR == nullptr)
+          ROCS_TRY(launch_attention_req_absorbed(h, p.QR, d2, S_l, dw.WK_R, dw.WV_R, BR, m->L, m->d, m->H, scale, dR,
+                                                 ldR, xR2, xr, s));
+        else
+          ROCS_TRY(launch_attention_single(h, p.QR, d2, 1, p.KR, p.VR, m->d, (long long)m->L * m->d, p.iota1, BR, BR,
+                                           m->L, m->H, dh, scale, dR, ldR, 0, xR2, xr, s));
       }
       {
         SiteLabel s_xc("xattn.cand");

@@ -163,6 +163,12 @@ rocs_status launch_attention_single(rocs_context* ctx, const void* Q, long long 
 // tcgen05/TMEM attention (one CTA per (request, head), K/V resident in shared memory): d_h 32
 // (L <= 1024) or 64 (L <= 256 with hi/lo queries, 512 without).  kv_rows = rows of K/V (B_R * L).
 // Returns ROCS_ERR_UNSUPPORTED, launching nothing, for shapes outside that range.
+// Request query's cross-attention with K^R = S W_K^R and V^R = S W_V^R absorbed into the query and
+// the output (one query per request; Q rows are bf16 hi/lo pairs [hi (d) | lo (d)]).
+bool attention_req_absorbed_supported(int d, int H, int L);
+rocs_status launch_attention_req_absorbed(rocs_context* ctx, const void* Q, long long ldq, const void* S,
+                                          const void* WK, const void* WV, int B_R, int L, int d, int H, float scale,
+                                          float* O, long long ldo, void* O2, long long ldo2, cudaStream_t s);
 rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq, int q_split, const void* K,
                                 const void* V, long long ldkv, long long kv_rows, const int32_t* offsets, int B_R,
                                 long long rows, int L, int H, int d_h, float scale, void* O, long long ldo,
