@@ -171,3 +171,18 @@ def test_forward_graph_replay(R):
         assert not torch.equal(s_new, s_eager)
     finally:
         R.rocs_set_graph_replay(1)
+
+
+def test_forward_end_to_end_long_history(R):
+    """The bench's history length L = 1024: each warp of the request-query attention walks four
+    32-row chunks (online softmax across chunks, then the warps' merge), and the tcgen05
+    attention runs eight 128-key blocks per tile with the lazy rescale between them."""
+    case = synth.model_cfg5(B_R=2, counts=[3, 130], L=1024, seed=5)
+    x, W = synth.model_inputs(case), synth.model_weights(case)
+    out = run_forward(R, case, x, W)
+    _, m = O.segments(case.counts)
+    ref = O.forward_cfg5(case, x, W, m)
+    check_bf16(host(out["score"][:case.B_C]), ref["score"], what="score")
+    for l in range(case.dca.layers):
+        check_bf16(host(out["A_R"][l]), ref["A_R"][l], what=f"A_R_{l}")
+        check_bf16(host(out["A_C"][l]), ref["A_C"][l], what=f"A_C_{l}")
