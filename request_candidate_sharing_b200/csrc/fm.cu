@@ -137,6 +137,10 @@ __device__ __forceinline__ void gram_tile(uint32_t sbase, int pitch, int a0, int
 // its loads are already in flight while it computes.
 constexpr int FC_CONSUMERS = 7;   // 8 warps in all: the whole register file (255 per thread) is available
 constexpr int FC_STAGES = 12;
+// A consumer's next candidate (i + consumers) reuses the stage of candidate i + consumers - stages,
+// which must already have been loaded (it is <= i) for the parity of its mbarrier wait to be
+// unambiguous.
+static_assert(FC_STAGES >= FC_CONSUMERS, "ring stages must cover the consumer warps");
 
 template <typename TIN>
 __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_kernel(

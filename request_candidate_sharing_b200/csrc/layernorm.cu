@@ -230,6 +230,9 @@ rocs_status dispatch(const void* X1, int w1, long long ld1, const void* X2, long
 // ---------------------------------------------------------------------------------------------
 constexpr int LN_CONSUMERS = 8;
 constexpr int LN_STAGES = 8;
+// a consumer's next block (b + consumers) reuses the stage of block b + consumers - stages, which
+// must already have been loaded for the parity of its mbarrier wait to be unambiguous
+static_assert(LN_STAGES >= LN_CONSUMERS, "ring stages must cover the consumer warps");
 constexpr int LN_STAGE_BYTES = 16384;
 
 template <typename T>
