@@ -48,6 +48,9 @@ WORKLOADS = {
                         "candidates ~ clipped lognormal (median 300, 16..2000), seed 1",
     "glm_stack": "Wukong-style GLM stack, 3 layers; 64 requests, candidates ~ U[100,1000], seed 0",
     "dca": "DCA path: L=200, d=256, 4 heads, 2 layers; 32 requests x 500 candidates, seed 0",
+    "ikbo_sweep": "IKBO linear sweep: B_R=256, N in {64, 256, 1024} candidates per request, d_in = d_out = d in "
+                  "{512, 1024, 4096}, bf16 in/out, fp32 accumulate, ReLU; against two materialised-broadcast "
+                  "GPU baselines (B1: Z[m] materialised and added; B2: gathered [X^R[m], X^C] with one K=2d GEMM)",
 }
 
 
@@ -499,6 +502,103 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------------------------
+# IKBO linear sweep with materialised-broadcast baselines
+# ---------------------------------------------------------------------------------------------
+def run_ikbo_sweep(args, rank, world, local):
+    """Each (N, d) point: rocs_linear_ikbo (bf16 in/out, ReLU), B1 = Z = X^R W_CR^T, Z[m] written
+    out and added to X^C W_CC^T (torch/cuBLAS), B2 = [X^R[m], X^C] gathered and one K=2d GEMM
+    (torch/cuBLAS).  Each repetition is timed alone with CUDA events after an L2 flush (a 256 MB
+    write); the median is reported.  Inputs: seeded torch normal draws on the device (X ~ N(0,1),
+    W ~ N(0, 1/fan_in), b ~ U(-0.1, 0.1)), bf16."""
+    import torch
+    from request_candidate_sharing_b200 import rocs
+    dev = torch.device("cuda", local)
+    R = rocs.Rocs(local)
+    peaks = load_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    B_R = 256
+    reps = max(args.steps, 3)
+    points = []
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            ts.append(e0.elapsed_time(e1))
+        ts.sort()
+        return ts[len(ts) // 2]
+
+    for N in (64, 256, 1024):
+        for d in (512, 1024, 4096):
+            g = torch.Generator(device=dev).manual_seed(1000 * N + d + 1000003 * rank)
+            B_C = B_R * N
+            bf = torch.bfloat16
+            XR = torch.randn(B_R, d, device=dev, generator=g).to(bf)
+            XC = torch.randn(B_C, d, device=dev, generator=g).to(bf)
+            W_RR, W_CR, W_CC = (torch.randn(d, d, device=dev, generator=g).mul_(d ** -0.5).to(bf) for _ in range(3))
+            bR = (torch.rand(d, device=dev, generator=g) * 0.2 - 0.1)
+            bC = (torch.rand(d, device=dev, generator=g) * 0.2 - 0.1)
+            m = torch.arange(B_R, device=dev, dtype=torch.int32).repeat_interleave(N)
+            YR = torch.empty(B_R, d, dtype=bf, device=dev)
+            YC = torch.empty(B_C, d, dtype=bf, device=dev)
+            desc = rocs.IkboDesc(B_R, B_C, d, d, d, d, rocs.ROCS_BF16, rocs.ROCS_BF16, rocs.ACT["relu"])
+            nb = R.rocs_linear_ikbo_workspace(desc)
+            ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
+            sh = torch.cuda.current_stream(dev).cuda_stream
+
+            def ikbo():
+                R.rocs_linear_ikbo(desc, XR, XC, m, W_RR, W_CR, W_CC, bR, bC, YR, YC, ws, nb, sh)
+
+            mi = m.long()
+
+            def b1():
+                z = torch.addmm(bC, XR.float(), W_CR.float().t()).to(bf)   # request partial (bias folded)
+                zm = z.index_select(0, mi)                                  # materialised broadcast [B_C, d]
+                torch.relu_(torch.addmm(zm, XC, W_CC.t()))
+                torch.relu_(torch.addmm(bR.to(bf), XR, W_RR.t()))
+
+            W2 = torch.cat([W_CR, W_CC], 1)                                 # [d, 2d]
+
+            def b2():
+                xg = torch.cat([XR.index_select(0, mi), XC], 1)            # gathered rows [B_C, 2d]
+                torch.relu_(torch.addmm(bC.to(bf), xg, W2.t()))
+                torch.relu_(torch.addmm(bR.to(bf), XR, W_RR.t()))
+
+            ms_i, ms_1, ms_2 = timed(ikbo), timed(b1), timed(b2)
+            st = R.rocs_get_device_status(sh)
+            if st != 0:
+                raise RuntimeError(f"device status {st} at N={N} d={d}")
+            flops = 2.0 * B_C * d * d + 2.0 * B_R * d * d * 2
+            tf = flops / (ms_i / 1e3) / 1e12
+            points.append({"N": N, "d": d, "B_C": B_C, "ikbo_ms": round(ms_i, 4),
+                           "ikbo_cands_per_s": round(B_C / (ms_i / 1e3), 1),
+                           "ikbo_tflops": round(tf, 2), "ikbo_frac_of_bf16_peak": round(tf / peaks["tensor"], 4),
+                           "b1_materialised_Zm_ms": round(ms_1, 4), "b2_gathered_2d_gemm_ms": round(ms_2, 4),
+                           "speedup_vs_b1": round(ms_1 / ms_i, 3), "speedup_vs_b2": round(ms_2 / ms_i, 3)})
+            del XR, XC, W_RR, W_CR, W_CC, YR, YC, ws, W2
+            torch.cuda.empty_cache()
+    head = next(p for p in points if p["N"] == 1024 and p["d"] == 1024)
+    if rank == 0:
+        line = {"metric": METRIC, "value": head["ikbo_cands_per_s"], "unit": "candidates/s", "n_gpus": world,
+                "steps": reps, "warmup": args.warmup, "ms_per_step": head["ikbo_ms"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded torch normal draws on the device)",
+                "config": {"workload": "ikbo_sweep", "description": WORKLOADS["ikbo_sweep"],
+                           "headline_point": "N=1024, d=1024", "l2": "flushed (256 MB write) before every repetition",
+                           "peak_source": peaks["source"] + " (of measured, burst: each GEMM timed alone)"},
+                "points": points}
+        print(json.dumps(line), flush=True)
+    R.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -519,7 +619,10 @@ def main():
         run_reference(args, rank, world)
         return
     rank, world, local = dist_setup(args.gpus)
-    run_librocs(args, rank, world, local)
+    if args.workload == "ikbo_sweep":
+        run_ikbo_sweep(args, rank, world, local)
+    else:
+        run_librocs(args, rank, world, local)
 
 
 if __name__ == "__main__":
