@@ -536,8 +536,11 @@ def run_ikbo_sweep(args, rank, world, local):
         ts.sort()
         return ts[len(ts) // 2]
 
+    only = tuple(int(v) for v in args.sweep_point.split(",")) if args.sweep_point else None
     for N in (64, 256, 1024):
         for d in (512, 1024, 4096):
+            if only is not None and (N, d) != only:
+                continue
             g = torch.Generator(device=dev).manual_seed(1000 * N + d + 1000003 * rank)
             B_C = B_R * N
             bf = torch.bfloat16
@@ -585,14 +588,15 @@ def run_ikbo_sweep(args, rank, world, local):
                            "speedup_vs_b1": round(ms_1 / ms_i, 3), "speedup_vs_b2": round(ms_2 / ms_i, 3)})
             del XR, XC, W_RR, W_CR, W_CC, YR, YC, ws, W2
             torch.cuda.empty_cache()
-    head = next(p for p in points if p["N"] == 1024 and p["d"] == 1024)
+    head = next((p for p in points if p["N"] == 1024 and p["d"] == 1024), points[-1])
     if rank == 0:
         line = {"metric": METRIC, "value": head["ikbo_cands_per_s"], "unit": "candidates/s", "n_gpus": world,
                 "steps": reps, "warmup": args.warmup, "ms_per_step": head["ikbo_ms"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
                 "data": "synthetic (seeded torch normal draws on the device)",
                 "config": {"workload": "ikbo_sweep", "description": WORKLOADS["ikbo_sweep"],
-                           "headline_point": "N=1024, d=1024", "l2": "flushed (256 MB write) before every repetition",
+                           "headline_point": f"N={head['N']}, d={head['d']}",
+                           "l2": "flushed (256 MB write) before every repetition",
                            "peak_source": peaks["source"] + " (of measured, burst: each GEMM timed alone)"},
                 "points": points}
         print(json.dumps(line), flush=True)
@@ -610,6 +614,7 @@ def main():
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--requests", type=int, default=0, help="keep only the first N requests (profiling runs)")
+    ap.add_argument("--sweep-point", default="", help="ikbo_sweep: run only the point 'N,d' (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "librocs":
         raise SystemExit("--warmup must be >= 3")
