@@ -186,3 +186,34 @@ def test_forward_end_to_end_long_history(R):
     for l in range(case.dca.layers):
         check_bf16(host(out["A_R"][l]), ref["A_R"][l], what=f"A_R_{l}")
         check_bf16(host(out["A_C"][l]), ref["A_C"][l], what=f"A_C_{l}")
+
+
+def test_forward_end_to_end_full_size_sampled(R):
+    """The benchmarked configuration at full size (512 requests, ~242k candidates, L = 1024): the
+    GPU runs the whole forward, the oracle only the sampled requests (the first, the one with the
+    most candidates and the last) with four of their candidates each.  Requests are independent,
+    so the oracle's sub-batch has the same outputs; its inputs are the same rows of the seeded
+    full-case generator."""
+    case = synth.model_cfg5()
+    x, W = synth.model_inputs(case), synth.model_weights(case)
+    out = run_forward(R, case, x, W)
+    off, m = O.segments(case.counts)
+    counts = np.asarray(case.counts)
+    reqs = sorted({0, int(np.argmax(counts)), case.B_R - 1})
+    g = np.random.default_rng(7)
+    rows, m_sub = [], []
+    for k, r in enumerate(reqs):
+        lo, n = int(off[r]), int(counts[r])
+        pick = sorted({lo, lo + n - 1} | {lo + int(v) for v in g.integers(0, n, 2)})
+        rows += pick
+        m_sub += [k] * len(pick)
+    rows, reqs_a = np.asarray(rows), np.asarray(reqs)
+    xs = synth.model_inputs(case, cand_rows=rows, req_rows=reqs_a)
+    ref = O.forward_cfg5(case, xs, W, np.asarray(m_sub, np.int32))
+    rt, qt = torch.from_numpy(rows).cuda(), torch.from_numpy(reqs_a).cuda()
+    check_bf16(host(out["score"][rt]), ref["score"], what="score (sampled)")
+    check_bf16(host(out["E_R"][qt]), ref["E_R"], what="E_R (sampled requests)")
+    check_bf16(host(out["E_C"][rt]), ref["E_C"], what="E_C (sampled)")
+    for l in range(case.dca.layers):
+        check_bf16(host(out["A_R"][l][qt]), ref["A_R"][l], what=f"A_R_{l} (sampled requests)")
+        check_bf16(host(out["A_C"][l][rt]), ref["A_C"][l], what=f"A_C_{l} (sampled)")
