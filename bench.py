@@ -365,7 +365,6 @@ def run_librocs(args, rank, world, local):
     clocks = ClockSampler(("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else (uuid or str(local)))
     clocks.start()
     time.sleep(0.3)
-    R.rocs_timing_start(200 * args.steps + 64)
     barrier(world)
     torch.cuda.synchronize(dev)
     # inputs smaller than twice the L2: each step is timed alone after an L2 flush (outside its
@@ -393,6 +392,14 @@ def run_librocs(args, rank, world, local):
         torch.cuda.synchronize(dev)
         barrier(world)
         ms = e0.elapsed_time(e1)
+    # per-kernel report: the same steps again with per-launch CUDA events (direct launches; the
+    # timed region above replays the forward's CUDA graph)
+    R.rocs_timing_start(200 * args.steps + 64)
+    for _ in range(args.steps):
+        if small:
+            flush.fill_(1)
+        step()
+    torch.cuda.synchronize(dev)
     report = R.rocs_timing_stop()
     clk = clocks.stop()
     st = R.rocs_get_device_status(sh)
@@ -466,8 +473,8 @@ def run_librocs(args, rank, world, local):
                               "L2 flush" if small else f"inputs larger than L2 ({in_bytes / 1e9:.2f} GB), "
                               "steps back to back"),
                        "parallelism": f"replicas x{world}",
-                       "launch": "value: direct launches with per-launch CUDA events (the per-kernel report); "
-                                 "e2e: the forward's captured CUDA graph replayed"},
+                       "launch": "value and e2e: the forward's captured CUDA graph replayed; per-kernel report "
+                                 "(roofline): the same steps again with direct launches and per-launch CUDA events"},
             "roofline": top,
             "e2e": {"value": round(e2e_value, 1), "unit": "candidates/s", "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": int(d2h)},
