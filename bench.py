@@ -418,20 +418,48 @@ def run_librocs(args, rank, world, local):
     res_h = torch.empty_like(res, device="cpu").pin_memory()
     d2h = res.numel() * res.element_size()
 
-    def e2e_step():
-        for k, v in host.items():
-            xd[k].copy_(v, non_blocking=True)
-        counts_d.copy_(counts_h, non_blocking=True)
-        step()
+    # two device input sets: step k+1's inputs are copied (copy stream) while step k computes;
+    # every step's inputs still cross PCIe inside the timed region, and each set has its own
+    # captured forward graph
+    sets = [(xd, counts_d, inp)]
+    xd2 = {k: torch.empty_like(v) for k, v in xd.items()}
+    counts_d2 = torch.empty_like(counts_d)
+    inp2 = rocs.Inputs(counts_d2.data_ptr(), rocs.ptr(xd2.get("E_R")), rocs.ptr(xd2.get("E_C")),
+                       rocs.ptr(xd2.get("H")), rocs.ptr(xd2.get("Y_R")), rocs.ptr(xd2.get("Y_C")))
+    sets.append((xd2, counts_d2, inp2))
+    copy_stream = torch.cuda.Stream(dev)
+    copied = [torch.cuda.Event(), torch.cuda.Event()]
+    done = [torch.cuda.Event(), torch.cuda.Event()]
+
+    def h2d_into(k):
+        xs, cs, _ = sets[k % 2]
+        with torch.cuda.stream(copy_stream):
+            copy_stream.wait_event(done[k % 2])     # the forward that last read this set is finished
+            for name, v in host.items():
+                xs[name].copy_(v, non_blocking=True)
+            cs.copy_(counts_h, non_blocking=True)
+            copied[k % 2].record(copy_stream)
+
+    def forward_on(k):
+        stream.wait_event(copied[k % 2])
+        R.rocs_forward(md, mw, sets[k % 2][2], out, ws, nb, sh)
+        done[k % 2].record(stream)
         res_h.copy_(res, non_blocking=True)
 
-    e2e_step()
+    def e2e_run(nsteps):
+        h2d_into(0)
+        for k in range(nsteps):
+            if k + 1 < nsteps:
+                h2d_into(k + 1)
+            forward_on(k)
+
+    e2e_run(4)   # each set's forward: a direct run, then its graph capture, before the timed region
     torch.cuda.synchronize(dev)
     barrier(world)
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     f0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    copy_stream.wait_event(f0)   # the first copy starts inside the timed region
+    e2e_run(args.steps)
     f1.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
@@ -474,7 +502,10 @@ def run_librocs(args, rank, world, local):
                               "steps back to back"),
                        "parallelism": f"replicas x{world}",
                        "launch": "value and e2e: the forward's captured CUDA graph replayed; per-kernel report "
-                                 "(roofline): the same steps again with direct launches and per-launch CUDA events"},
+                                 "(roofline): the same steps again with direct launches and per-launch CUDA events",
+                       "e2e_pipelining": "two device input sets: step k+1's host-to-device copy (pinned, copy "
+                                         "stream) overlaps step k's forward; every step's inputs are copied and "
+                                         "its scores read back inside the timed region"},
             "roofline": top,
             "e2e": {"value": round(e2e_value, 1), "unit": "candidates/s", "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": int(d2h)},
