@@ -9,10 +9,10 @@
 // weights from L2.  Same function; the scores and outputs are fp32 sums of exact bf16 x bf16
 // products (K^R and V^R are not rounded to bf16 on the way).
 //
-// One CTA per request, 8 warps, d = 256; each warp takes 32-row chunks of S in turn:
+// One CTA per request, 8 warps, d = 256; each warp takes 16-row chunks of S in turn:
 //   1. q = hi + lo of the request's query; k'_h (scale and log2(e) folded in) into shared memory.
-//   2. per chunk: the 32 rows are copied into the warp's shared tile (coalesced, rows padded to
-//      528 bytes); scores (32 rows x 8 heads) = S_chunk . k' and the weighted sums
+//   2. per warp, 16-row chunks of S double-buffered in shared memory (cp.async; rows padded to
+//      528 bytes): scores (16 rows x 8 heads) = S_chunk . k' and the weighted sums
 //      s^T += S_chunk^T P run as m16n8k16 MMAs (k' as a bf16 hi/lo pair, P in bf16), with a
 //      per-head online softmax (running max m, sum l) between them.
 //   3. the eight warps' (m, l, s) states are merged in shared memory.
@@ -43,11 +43,11 @@ __global__ void __launch_bounds__(AR_WARPS * 32) attn_req_absorbed_kernel(
   constexpr int D = AR_D;
   __shared__ float q[D];
   __shared__ __align__(16) float kp[AR_MAX_H][D];
-  __shared__ __align__(16) uint32_t pbuf[AR_WARPS][32][AR_MAX_H / 2];   // P as bf16 pairs [row][head pair]
+  __shared__ __align__(16) uint32_t pbuf[AR_WARPS][16][AR_MAX_H / 2];   // P as bf16 pairs [row][head pair]
   __shared__ __align__(16) __nv_bfloat16 kbh[AR_MAX_H * AR_KPITCH], kbl[AR_MAX_H * AR_KPITCH];
   __shared__ float wm[AR_WARPS][AR_MAX_H], wl[AR_WARPS][AR_MAX_H];
   __shared__ float inv_l[AR_MAX_H];
-  // dynamic: the warps' row tiles [AR_WARPS][32][AR_PITCH]; after the pass, the warps' weighted
+  // dynamic: the warps' row tiles [AR_WARPS][2 buffers][16][AR_PITCH]; after the pass, the warps' weighted
   // row sums [AR_WARPS][AR_MAX_H][D] fp32 (merged into warp 0's slot)
   extern __shared__ __align__(16) uint8_t ar_dyn[];
   auto ws = reinterpret_cast<float (*)[AR_MAX_H][D]>(ar_dyn);
@@ -86,9 +86,9 @@ __global__ void __launch_bounds__(AR_WARPS * 32) attn_req_absorbed_kernel(
     reinterpret_cast<uint4*>(ar_dyn)[k] = make_uint4(0, 0, 0, 0);
   __syncthreads();
 
-  // 2. 32-row chunks on the tensor cores (m16n8k16, fp32 accumulate) with a per-head online softmax:
-  //    scores (32 rows x 8 heads) = S_chunk (32 x D) . k' (D x 8, hi + lo);
-  //    s^T (D x 8 heads) += S_chunk^T (D x 32) . P (32 x 8, bf16).
+  // 2. 16-row chunks on the tensor cores (m16n8k16, fp32 accumulate) with a per-head online softmax:
+  //    scores (16 rows x 8 heads) = S_chunk (16 x D) . k' (D x 8, hi + lo);
+  //    s^T (D x 8 heads) += S_chunk^T (D x 16) . P (16 x 8, bf16).
   //    Lane (g, t) holds heads 2t, 2t+1 in both fragments, so each head's rescale stays in-lane.
   const int g8 = lane >> 2, t4 = lane & 3;
   uint32_t bh[D / 16][2], bl[D / 16][2];
@@ -105,69 +105,71 @@ __global__ void __launch_bounds__(AR_WARPS * 32) attn_req_absorbed_kernel(
   float accO[D / 16][4];
 #pragma unroll
   for (int mt = 0; mt < D / 16; ++mt) accO[mt][0] = accO[mt][1] = accO[mt][2] = accO[mt][3] = 0.f;
-  const uint32_t tbase = smem_u32(tile);
   const uint32_t pbase = smem_u32(&pbuf[warp][0][0]);
-  for (int t0 = warp * 32; t0 < L; t0 += AR_WARPS * 32) {
-    const int nrows = L - t0 < 32 ? L - t0 : 32;
-    // the chunk into the tile: row k, 16-byte column group lane
-    __syncwarp();
-#pragma unroll 8
-    for (int k = 0; k < 32; ++k)
+  // 16-row chunks, double-buffered per warp: chunk c + 1 streams in (cp.async) while chunk c runs
+  auto issue_chunk = [&](int t0, int buf) {
+    const int nrows = L - t0 < 16 ? L - t0 : 16;
+    const uint32_t dst = smem_u32(tile + buf * 16 * AR_PITCH) + lane * 16;
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
       if (k < nrows)
-        *reinterpret_cast<uint4*>(tile + k * AR_PITCH + lane * 16) =
-            __ldg(reinterpret_cast<const uint4*>(Sr + (long long)(t0 + k) * D) + lane);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + k * AR_PITCH),
+                     "l"(Sr + (long long)(t0 + k) * D + lane * 8)
+                     : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  const int stride = AR_WARPS * 16;
+  int buf = 0;
+  if (warp * 16 < L) issue_chunk(warp * 16, 0);
+  for (int t0 = warp * 16; t0 < L; t0 += stride, buf ^= 1) {
+    const int nrows = L - t0 < 16 ? L - t0 : 16;
+    if (t0 + stride < L) {
+      issue_chunk(t0 + stride, buf ^ 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
     __syncwarp();
-    // scores
-    float sc[2][4];
+    const uint32_t tbase = smem_u32(tile + buf * 16 * AR_PITCH);
+    // scores (16 rows x 8 heads)
+    float sc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-      sc[mt][0] = sc[mt][1] = sc[mt][2] = sc[mt][3] = 0.f;
-#pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        uint32_t a[4];
-        load_a_frag(tbase, AR_PITCH, mt * 16, ks * 16, a);
-        mma_bf16_16816(sc[mt], a, bh[ks][0], bh[ks][1]);
-        mma_bf16_16816(sc[mt], a, bl[ks][0], bl[ks][1]);
-      }
+    for (int ks = 0; ks < D / 16; ++ks) {
+      uint32_t a4[4];
+      load_a_frag(tbase, AR_PITCH, 0, ks * 16, a4);
+      mma_bf16_16816(sc, a4, bh[ks][0], bh[ks][1]);
+      mma_bf16_16816(sc, a4, bl[ks][0], bl[ks][1]);
     }
     // rows past the chunk's end do not exist
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-      if (mt * 16 + g8 >= nrows) sc[mt][0] = sc[mt][1] = -INFINITY;
-      if (mt * 16 + g8 + 8 >= nrows) sc[mt][2] = sc[mt][3] = -INFINITY;
-    }
+    if (g8 >= nrows) sc[0] = sc[1] = -INFINITY;
+    if (g8 + 8 >= nrows) sc[2] = sc[3] = -INFINITY;
     // online softmax for heads 2t (c = 0) and 2t + 1 (c = 1)
     float corr[2];
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
-      float mx = fmaxf(fmaxf(sc[0][c], sc[0][c + 2]), fmaxf(sc[1][c], sc[1][c + 2]));
+      float mx = fmaxf(sc[c], sc[c + 2]);
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
       const float m_new = fmaxf(m[c], mx);
       corr[c] = m[c] == -INFINITY ? 0.f : exp2f(m[c] - m_new);
-      float sum = 0.f;
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-        sc[mt][c] = exp2f(sc[mt][c] - m_new);
-        sc[mt][c + 2] = exp2f(sc[mt][c + 2] - m_new);
-        sum += sc[mt][c] + sc[mt][c + 2];
-      }
+      sc[c] = exp2f(sc[c] - m_new);
+      sc[c + 2] = exp2f(sc[c + 2] - m_new);
+      float sum = sc[c] + sc[c + 2];
       sum += __shfl_xor_sync(0xffffffffu, sum, 4);
       sum += __shfl_xor_sync(0xffffffffu, sum, 8);
       sum += __shfl_xor_sync(0xffffffffu, sum, 16);
       l[c] = fmaf(l[c], corr[c], sum);
       m[c] = m_new;
     }
-    // P (32 rows x 8 heads, bf16) into the warp's buffer, then back as B fragments
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-      pbuf[warp][mt * 16 + g8][t4] = pack_bf16x2(sc[mt][0], sc[mt][1]);
-      pbuf[warp][mt * 16 + g8 + 8][t4] = pack_bf16x2(sc[mt][2], sc[mt][3]);
-    }
+    // P (16 rows x 8 heads, bf16) through the warp's buffer, back as the B fragment
+    pbuf[warp][g8][t4] = pack_bf16x2(sc[0], sc[1]);
+    pbuf[warp][g8 + 8][t4] = pack_bf16x2(sc[2], sc[3]);
     __syncwarp();
-    uint32_t pb[2][2];
-    ldsm_x4_trans(pbase + lane * 16, pb[0][0], pb[0][1], pb[1][0], pb[1][1]);
+    uint32_t pb0, pb1;
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+                 : "=r"(pb0), "=r"(pb1)
+                 : "r"(pbase + (lane & 15) * 16));
     // s^T += S_chunk^T P, after the rescale of the old sums
 #pragma unroll
     for (int mt = 0; mt < D / 16; ++mt) {
@@ -175,16 +177,13 @@ __global__ void __launch_bounds__(AR_WARPS * 32) attn_req_absorbed_kernel(
       accO[mt][1] *= corr[1];
       accO[mt][2] *= corr[0];
       accO[mt][3] *= corr[1];
-#pragma unroll
-      for (int ks = 0; ks < 2; ++ks) {
-        uint32_t a[4];
-        const int j = lane >> 3;
-        const uint32_t addr = tbase + (uint32_t)((ks * 16 + ((j >> 1) << 3) + (lane & 7)) * AR_PITCH +
-                                                 (mt * 16 + ((j & 1) << 3)) * 2);
-        ldsm_x4_trans(addr, a[0], a[1], a[2], a[3]);
-        mma_bf16_16816(accO[mt], a, pb[ks][0], pb[ks][1]);
-      }
+      uint32_t a4[4];
+      const int j = lane >> 3;
+      const uint32_t addr = tbase + (uint32_t)((((j >> 1) << 3) + (lane & 7)) * AR_PITCH + (mt * 16 + ((j & 1) << 3)) * 2);
+      ldsm_x4_trans(addr, a4[0], a4[1], a4[2], a4[3]);
+      mma_bf16_16816(accO[mt], a4, pb0, pb1);
     }
+    __syncwarp();   // this buffer is read before the chunk after next streams into it
   }
   __syncthreads();   // every warp is done with its tile: the region now holds the weighted sums
 

@@ -316,48 +316,72 @@ __global__ void __launch_bounds__(32 * (1 + LN_CONSUMERS), 1) layernorm_ring_ker
     const uint8_t* sb = ring + st * LN_STAGE_BYTES;
     const long long row0 = r0 + (long long)b * RB;
     const int nr = (int)(r1 - row0 < RB ? r1 - row0 : RB);
-    for (int k = 0; k < nr; ++k) {
-      float v[NV][4];
-      float s = 0.f;
+    // narrow rows: MR rows at a time, so their reductions overlap
+    constexpr int MR = NV <= 4 ? 4 : 1;
+    for (int k0 = 0; k0 < nr; k0 += MR) {
+      float v[MR][NV][4];
+      float s[MR];
 #pragma unroll
-      for (int i = 0; i < NV; ++i) {
-        const int col = (i * 32 + lane) * 4;
-        if (col < w1) ld4<TIN>(reinterpret_cast<const TIN*>(sb) + k * w1 + col, v[i]);
-        else ld4<TIN>(reinterpret_cast<const TIN*>(sb + off2) + k * w2 + (col - w1), v[i]);
-        if (R != nullptr) {
-          float rr[4];
-          ld4<TRES>(reinterpret_cast<const TRES*>(sb + offr) + k * width + col, rr);
+      for (int m = 0; m < MR; ++m) {
+        s[m] = 0.f;
+        const int k = k0 + m;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) v[i][j] += rr[j];
+        for (int i = 0; i < NV; ++i) {
+          const int col = (i * 32 + lane) * 4;
+          if (k < nr) {
+            if (col < w1) ld4<TIN>(reinterpret_cast<const TIN*>(sb) + k * w1 + col, v[m][i]);
+            else ld4<TIN>(reinterpret_cast<const TIN*>(sb + off2) + k * w2 + (col - w1), v[m][i]);
+            if (R != nullptr) {
+              float rr[4];
+              ld4<TRES>(reinterpret_cast<const TRES*>(sb + offr) + k * width + col, rr);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) v[m][i][j] += rr[j];
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) v[m][i][j] = 0.f;
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) s[m] += v[m][i][j];
         }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) s += v[i][j];
       }
-      if (k == nr - 1) mbar_arrive(&empty[st]);   // every read of this stage is done
+      if (k0 + MR >= nr) mbar_arrive(&empty[st]);   // every read of this stage is done
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      const float mean = s * (1.0f / (float)width);
-      float q = 0.f;
+      for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-      for (int i = 0; i < NV; ++i)
+        for (int m = 0; m < MR; ++m) s[m] += __shfl_xor_sync(0xffffffffu, s[m], o);
+      float mean[MR], q[MR];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float d = v[i][j] - mean;
-          q += d * d;
+      for (int m = 0; m < MR; ++m) {
+        mean[m] = s[m] * (1.0f / (float)width);
+        q[m] = 0.f;
+#pragma unroll
+        for (int i = 0; i < NV; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float d = v[m][i][j] - mean[m];
+            q[m] += d * d;
+          }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int m = 0; m < MR; ++m) q[m] += __shfl_xor_sync(0xffffffffu, q[m], o);
+#pragma unroll
+      for (int m = 0; m < MR; ++m) {
+        if (k0 + m >= nr) break;
+        const float rstd = rsqrtf(q[m] * (1.0f / (float)width) + eps);
+        const long long row = row0 + k0 + m;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+          const int col = (i * 32 + lane) * 4;
+          const float4 gm = *reinterpret_cast<const float4*>(s_gamma + col);
+          const float4 bt = *reinterpret_cast<const float4*>(s_beta + col);
+          float o[4] = {(v[m][i][0] - mean[m]) * rstd * gm.x + bt.x, (v[m][i][1] - mean[m]) * rstd * gm.y + bt.y,
+                        (v[m][i][2] - mean[m]) * rstd * gm.z + bt.z, (v[m][i][3] - mean[m]) * rstd * gm.w + bt.w};
+          store_vec<TOUT, 4>(Y + row * width + col, o);
+          if (Y2 != nullptr) store_vec<__nv_bfloat16, 4>(Y2 + row * ldy2 + col, o);
         }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
-      const float rstd = rsqrtf(q * (1.0f / (float)width) + eps);
-      const long long row = row0 + k;
-#pragma unroll
-      for (int i = 0; i < NV; ++i) {
-        const int col = (i * 32 + lane) * 4;
-        const float4 gm = *reinterpret_cast<const float4*>(s_gamma + col);
-        const float4 bt = *reinterpret_cast<const float4*>(s_beta + col);
-        float o[4] = {(v[i][0] - mean) * rstd * gm.x + bt.x, (v[i][1] - mean) * rstd * gm.y + bt.y,
-                      (v[i][2] - mean) * rstd * gm.z + bt.z, (v[i][3] - mean) * rstd * gm.w + bt.w};
-        store_vec<TOUT, 4>(Y + row * width + col, o);
-        if (Y2 != nullptr) store_vec<__nv_bfloat16, 4>(Y2 + row * ldy2 + col, o);
       }
     }
   }
