@@ -110,9 +110,14 @@ def algo_work(case, label: str):
             "xattn.cand:attn_stream": ("alu", float(B_C) * H * L),
             "xattn.cand:attn_tc": ("alu", float(B_C) * H * L),
             "enc.qkv:gemm_tc": ("tensor", 2.0 * B_R * L * d * d * 3),
-            "enc.kv:gemm_tc": ("tensor", 2.0 * B_R * L * d * d * 4),
+            # the candidate group's K/V only when the request query's attention absorbs its
+            # projections (d = 256, up to 8 heads of a multiple of 16), else all four
+            "enc.kv:gemm_tc": ("tensor", 2.0 * B_R * L * d * d * (2 if (d == 256 and H <= 8 and (d // H) % 16 == 0) else 4)),
             "enc.wo:gemm_tc": ("tensor", 2.0 * B_R * L * d * d),
             "enc.ln:layernorm": ("hbm", B_R * L * d * 2 * 3.0),
+            # the request query's attention with its projections absorbed reads the final
+            # encoder output S once (bf16); weights and queries are L2-resident and negligible
+            "xattn.req:attn_req": ("hbm", float(B_R) * L * d * 2),
         }
         if label in table:
             return table[label]

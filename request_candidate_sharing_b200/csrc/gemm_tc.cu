@@ -338,24 +338,40 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
     const int row = q * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
+    // this row's request index in a tile, read one tile ahead of its use
+    auto load_gidx = [&](int tt) -> int {
+      if (tt >= P.total_tiles) return -1;
+      int pn, mn, nn;
+      decode_tile(P, tt, pn, mn, nn);
+      const Problem& q2 = P.p[pn];
+      const long long gn = (long long)mn * BM + row;
+      return (q2.Z != nullptr && gn < q2.M) ? __ldg(q2.gidx + gn) : -1;
+    };
+    int zi_next = load_gidx(blockIdx.x);
     for (int t = blockIdx.x; t < P.total_tiles; t += gridDim.x) {
       int pi, mb, nb;
       decode_tile(P, t, pi, mb, nb);
       const Problem& pr = P.p[pi];
-      if (!mbar_wait(&tfull[acc], acc_phase, P.status, abort_flag)) break;
-      tc_fence_after();
       const long long grow = (long long)mb * BM + row;
       bool rvalid = grow < pr.M;
       const float* zrow = nullptr;
+      const int zi = zi_next;
+      zi_next = load_gidx(t + gridDim.x);
       if (rvalid && pr.Z != nullptr) {
-        const int zi = pr.gidx[grow];
         if (zi < 0 || zi >= pr.gidx_bound) {
           set_status(P.status, ROCS_ERR_INDEX);
           rvalid = false;
         } else {
           zrow = pr.Z + (long long)zi * pr.ldz;
+          // this warp's chunks of the row's Z into L1 before the wait for the accumulator (the
+          // gathered rows were the epilogue's longest latency at short K)
+          for (int c = half; c < pr.BN / 32; c += 2)
+            if (nb * pr.BN + c * 32 < pr.N)
+              asm volatile("prefetch.global.L1 [%0];" ::"l"(zrow + nb * pr.BN + c * 32));
         }
       }
+      if (!mbar_wait(&tfull[acc], acc_phase, P.status, abort_flag)) break;
+      tc_fence_after();
       // a row with a bad request index is skipped, not written: such a warp stores element-wise
       const bool use_tma = pr.tma_out && !__any_sync(0xffffffffu, grow < pr.M && !rvalid);
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MAX);

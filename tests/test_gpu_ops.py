@@ -186,6 +186,27 @@ def test_linear_cfg2_sampled_full_size(R):
     check_bf16(host(YC[torch.from_numpy(rows).cuda()]), rC, out_bf16=True, what="Y_C sample")
 
 
+def test_linear_short_k_many_candidates(R):
+    """d = 256 with 159,840 candidates (K = 256: four k blocks per tile, so the gather epilogue and
+    its prefetch of the next chunk's Z row dominate); ragged last tile.  Oracle on a sample, every
+    row against a float32 torch evaluation of the same formula."""
+    from request_candidate_sharing_b200 import rocs
+    case = synth.linear_cfg2(999, 256, B_R=160)
+    x = synth.linear_inputs(case)
+    _, m = O.segments(case.counts)
+    YR, YC = _run_linear(R, case, x, m, rocs.ROCS_BF16, rocs.ROCS_F32)
+    rows = sample_candidates(case.counts, 2)
+    rR, rC = O.glm_linear(x["X_R"], x["X_C"][rows], m[rows], x["W_RR"], x["W_CR"], x["W_CC"], x["b_R"], x["b_C"],
+                          "relu")
+    check_bf16(host(YR), rR, out_bf16=False, what="Y_R")
+    check_fp32(host(YC[torch.from_numpy(rows).cuda()]), rC, rel=1e-4, what="Y_C sample")
+    t = {k: torch.from_numpy(np.asarray(v, np.float32)).cuda() for k, v in x.items()}
+    z = t["X_R"] @ t["W_CR"].T + t["b_C"]
+    ref = torch.relu(t["X_C"] @ t["W_CC"].T + z[torch.from_numpy(m.astype(np.int64)).cuda()])
+    err = (YC - ref).abs().max().item()
+    assert err <= 1e-3 * ref.abs().max().item(), err
+
+
 # ---------------------------------------------------------------------------------------------
 # a6 group LayerNorm
 # ---------------------------------------------------------------------------------------------
