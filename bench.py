@@ -94,6 +94,9 @@ def algo_work(case, label: str):
             "glm.mlp1.req:gemm_tc": ("tensor", 2.0 * B_R * g.hidden * fR * 2),
             "glm.mlp2.cand:gemm_tc": ("tensor", 2.0 * B_C * oCw * g.hidden),
             "glm.mlp2.req:gemm_tc": ("tensor", 2.0 * B_R * (oRw + oCw) * g.hidden),
+            # one fused launch (request and candidate tiles): the sum of the two
+            "glm.mlp1.ikbo:gemm_tc": ("tensor", 2.0 * B_C * g.hidden * fC + 2.0 * B_R * g.hidden * fR * 2),
+            "glm.mlp2.ikbo:gemm_tc": ("tensor", 2.0 * B_C * oCw * g.hidden + 2.0 * B_R * (oRw + oCw) * g.hidden),
             # fused candidate pass: reads E^C (bf16 at layer 0, fp32 after), writes F^C (hi/lo),
             # L^C (fp32) and, when DCA queries come from the GLM stack, t^C (hi/lo)
             "glm.fm:glm_cand_fused": ("hbm", B_C * (wc * (2 + 4 * (g.layers - 1)) / g.layers + fC * 4 + lCw * 4
@@ -115,6 +118,9 @@ def algo_work(case, label: str):
             "enc.kv:gemm_tc": ("tensor", 2.0 * B_R * L * d * d * (2 if (d == 256 and H <= 8 and (d // H) % 16 == 0) else 4)),
             "enc.wo:gemm_tc": ("tensor", 2.0 * B_R * L * d * d),
             "enc.ln:layernorm": ("hbm", B_R * L * d * 2 * 3.0),
+            # query generator, two IKBO linears q_dim -> d -> d (fused launches: request + candidate)
+            "qgen.mlp1.ikbo:gemm_tc": ("tensor", 2.0 * (B_C + 2 * B_R) * d * a.q_dim),
+            "qgen.mlp2.ikbo:gemm_tc": ("tensor", 2.0 * (B_C + 2 * B_R) * d * d),
             # the request query's attention with its projections absorbed reads the final
             # encoder output S once (bf16); weights and queries are L2-resident and negligible
             "xattn.req:attn_req": ("hbm", float(B_R) * L * d * 2),
@@ -124,7 +130,9 @@ def algo_work(case, label: str):
     if case.scoring is not None:
         h1, h2 = case.scoring
         xc = g.n_C * g.D + a.layers * a.d
+        xr = g.n_R * g.D + a.layers * a.d
         table = {"score.l1.cand:gemm_tc": ("tensor", 2.0 * B_C * h1 * xc),
+                 "score.l1.ikbo:gemm_tc": ("tensor", 2.0 * B_C * h1 * xc + 2.0 * B_R * h1 * xr),
                  "score.l2:gemm_tc": ("tensor", 2.0 * B_C * h2 * h1)}
         if label in table:
             return table[label]
@@ -327,6 +335,7 @@ def run_librocs(args, rank, world, local):
     counts_d = torch.from_numpy(case.counts).to(dev)
     g, a = case.glm, case.dca
     R = rocs.Rocs(local)
+    R.rocs_set_ikbo_fused(args.ikbo_fused)
     md = rocs.model_desc(case)
     mw = rocs.model_weights(Wd, g.layers if g else 0, a.layers if a else 0, case.scoring is not None)
     B_C = case.B_C
@@ -506,6 +515,8 @@ def run_librocs(args, rank, world, local):
                               "L2 flush" if small else f"inputs larger than L2 ({in_bytes / 1e9:.2f} GB), "
                               "steps back to back"),
                        "parallelism": f"replicas x{world}",
+                       "ikbo_launch": "fused (request + candidate tiles, completion flags)" if args.ikbo_fused
+                                      else "two launches (request GEMM, then candidate GEMM)",
                        "launch": "value and e2e: the forward's captured CUDA graph replayed; per-kernel report "
                                  "(roofline): the same steps again with direct launches and per-launch CUDA events",
                        "e2e_pipelining": "two device input sets: step k+1's host-to-device copy (pinned, copy "
@@ -577,6 +588,7 @@ def run_ikbo_sweep(args, rank, world, local):
     from request_candidate_sharing_b200 import rocs
     dev = torch.device("cuda", local)
     R = rocs.Rocs(local)
+    R.rocs_set_ikbo_fused(args.ikbo_fused)
     peaks = load_peaks()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     B_R = 256
@@ -677,6 +689,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--requests", type=int, default=0, help="keep only the first N requests (profiling runs)")
     ap.add_argument("--sweep-point", default="", help="ikbo_sweep: run only the point 'N,d' (profiling runs)")
+    ap.add_argument("--ikbo-fused", type=int, default=1, choices=[0, 1],
+                    help="IKBO linears as one fused launch (1, the library default) or two launches (0)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "librocs":
         raise SystemExit("--warmup must be >= 3")

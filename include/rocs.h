@@ -331,6 +331,19 @@ rocs_status rocs_forward(rocs_handle_t handle, const rocs_model_desc* model,
  * Errors: ROCS_ERR_INVALID_ARG for a NULL handle or another value of enable. */
 rocs_status rocs_set_graph_replay(rocs_handle_t handle, int32_t enable);
 
+/* Fused IKBO launch ([REV] §2.4: the request and candidate GEMMs in one persistent kernel) on
+ * (enable = 1, the default) or off (0) for this handle.  It applies to the bf16 path of
+ * rocs_linear_ikbo and to every IKBO linear inside rocs_forward, where the candidate GEMM has
+ * K >= 1024 (a hi/lo split input counting twice) or at most 32768 candidates; other shapes keep
+ * the two launches, which measured faster there.  Fused, the request GEMM's tiles
+ * come first in every CTA's order and publish completion flags (kept in the workspace, zeroed by
+ * each call); a candidate tile's epilogue waits (bounded) for the flags of the request tiles whose
+ * Z rows it gathers, and the launch is cooperative, so every CTA is resident.  Results are
+ * identical to the two-launch form.  A wait that runs out sets ROCS_ERR_DEVICE_TIMEOUT in the
+ * device status and leaves the affected rows unwritten.
+ * Errors: ROCS_ERR_INVALID_ARG for a NULL handle or another value of enable. */
+rocs_status rocs_set_ikbo_fused(rocs_handle_t handle, int32_t enable);
+
 /* ------------------------------------------------------------------------------------------
  * Per-launch timing (tracing).  After rocs_timing_start(h, max_launches), every kernel the
  * library launches for handle h records a CUDA event before and after itself on the stream it

@@ -3,6 +3,7 @@
 // carves the caller's workspace and enqueues launches on the caller's stream.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -86,10 +87,15 @@ struct IkboArgs {
   int out_mode; int act;     // 0 fp32, 1 bf16, 2 bf16 hi/lo pair
   int split_in = 0;          // X_R / X_C rows hold [hi (d_in) | lo (d_in)]
   float* Z;   // [B_R, dCo] fp32 scratch
+  int* flags = nullptr;      // ikbo_flag_ints(B_R, dCo) ints: request and candidate GEMMs in one launch
 };
 
+// Completion flags of one fused IKBO launch: one int per (128-request block, 32-column block), an
+// upper bound on the request GEMM's tiles for any tile width.
+long long ikbo_flag_ints(long long B_R, long long dCo) { return ((B_R + 127) / 128) * ((dCo + 31) / 32); }
+
 rocs_status ikbo_bf16(rocs_context* ctx, const IkboArgs& a, cudaStream_t s) {
-  GemmDesc req[2];
+  GemmDesc req[3];
   int nreq = 0;
   if (a.dRo > 0) {
     GemmDesc& g = req[nreq++];
@@ -102,6 +108,28 @@ rocs_status ikbo_bf16(rocs_context* ctx, const IkboArgs& a, cudaStream_t s) {
     g.A = a.X_R; g.lda = a.ldxr; g.M = a.B_R; g.K = a.dRi; g.split_a = a.split_in;
     g.B = a.W_CR; g.ldb = a.dRi; g.N = a.dCo;
     g.bias = a.b_C; g.out = a.Z; g.ldo = a.dCo; g.out_mode = 0; g.act = ROCS_ACT_NONE;
+  }
+  // [REV] §2.4's single launch where it pays: the candidate GEMM's tiles are long (K >= 1024, a
+  // split operand counting twice), or there are few of them (a separate request launch is then a
+  // large share).  At short K with many candidates the candidate epilogue is the bottleneck, and
+  // the fused form's wait for the first Z tiles costs more than the launch it saves.
+  const long long keff = (long long)a.dCi * (a.split_in ? 2 : 1);
+  const bool fuse = a.B_C > 0 && a.flags != nullptr && ctx->ikbo_fused && (keff >= 1024 || a.B_C <= 32768);
+  if (fuse) {
+    // request GEMMs' tiles first, then the candidate tiles, whose epilogues wait for the Z tiles
+    // they gather (completion flags, zeroed here)
+    GemmDesc& z = req[nreq - 1];
+    z.flags = a.flags; z.flag_role = 1;
+    GemmDesc& g = req[nreq++];
+    g.A = a.X_C; g.lda = a.ldxc; g.M = (int)a.B_C; g.K = a.dCi; g.split_a = a.split_in;
+    g.B = a.W_CC; g.ldb = a.dCi; g.N = a.dCo;
+    g.Z = a.Z; g.ldz = a.dCo; g.gidx = a.req_idx; g.gidx_bound = a.B_R;
+    g.out = a.Y_C; g.ldo = a.ldyc; g.out_mode = a.out_mode; g.act = a.act;
+    g.flags = a.flags; g.flag_role = 2;
+    std::string site = std::string(g_site ? g_site : "ikbo") + ".ikbo";
+    SiteLabel sl(site.c_str());
+    ROCS_TRY(cuda_check(cudaMemsetAsync(a.flags, 0, (size_t)ikbo_flag_ints(a.B_R, a.dCo) * 4, s), "zero IKBO flags"));
+    return launch_gemm_bf16(ctx, req, nreq, s);
   }
   {
     std::string site = std::string(g_site ? g_site : "ikbo") + ".req";
@@ -151,6 +179,7 @@ rocs_status attention_best(rocs_context* ctx, bool streaming_fallback, const voi
 // Workspace of rocs_linear_ikbo: Z, then (only if a row is not 16-B aligned) padded operands.
 struct IkboPlan {
   float* Z = nullptr;
+  int* flags = nullptr;
   void *XR = nullptr, *XC = nullptr, *WRR = nullptr, *WCR = nullptr, *WCC = nullptr;
   int kR = 0, kC = 0;   // padded K
   bool padR = false, padC = false;
@@ -161,6 +190,7 @@ IkboPlan plan_ikbo(const rocs_ikbo_desc* d, void* ws) {
   IkboPlan p;
   Carver c(ws);
   p.Z = (float*)c.take((size_t)d->B_R * d->d_C_out * 4);
+  if (d->dtype_in == ROCS_BF16 && d->B_C > 0) p.flags = (int*)c.take((size_t)ikbo_flag_ints(d->B_R, d->d_C_out) * 4);
   if (d->dtype_in == ROCS_BF16) {
     p.padR = (d->d_R_in % 8) != 0;
     p.padC = (d->d_C_in % 8) != 0;
@@ -331,7 +361,7 @@ extern "C" rocs_status rocs_linear_ikbo(rocs_handle_t h, const rocs_ikbo_desc* d
   a.X_R = X_R; a.ldxr = d->d_R_in; a.X_C = X_C; a.ldxc = d->d_C_in; a.req_idx = req_idx;
   a.W_RR = W_RR; a.W_CR = W_CR; a.W_CC = W_CC; a.b_R = b_R; a.b_C = b_C;
   a.Y_R = Y_R; a.ldyr = d->d_R_out; a.Y_C = Y_C; a.ldyc = d->d_C_out;
-  a.out_mode = d->dtype_out == ROCS_BF16 ? 1 : 0; a.act = d->act; a.Z = p.Z;
+  a.out_mode = d->dtype_out == ROCS_BF16 ? 1 : 0; a.act = d->act; a.Z = p.Z; a.flags = p.flags;
   // a1: alignment fix -- zero-pad K of any operand pair whose rows are not 16-byte multiples.
   if (p.padR) {
     ROCS_TRY(launch_pad_rows(X_R, d->d_R_in, p.XR, p.kR, d->B_R, d->d_R_in, 2, s));
@@ -586,6 +616,7 @@ struct FwdPlan {
   // scoring
   void *xR, *xC, *h1, *h2;
   float* Zs;
+  int* ikbo_flags;   // completion flags of the fused IKBO launches (reused, zeroed by each)
   size_t bytes;
 };
 
@@ -597,6 +628,11 @@ FwdPlan plan_forward(const rocs_model_desc* m, void* ws, bool own_offsets, bool 
   p.offsets = own_offsets ? (int32_t*)c.take((BR + 1) * 4) : nullptr;
   p.req_idx = own_req ? (int32_t*)c.take((size_t)BC * 4 + 4) : nullptr;
   p.iota1 = (int32_t*)c.take((BR + 1) * 4);
+  {
+    long long maxN = std::max<long long>({(long long)m->hidden, (long long)m->fm_out_C * m->D, (long long)m->d,
+                                          (long long)m->score_h1, 1LL});
+    p.ikbo_flags = (int*)c.take((size_t)ikbo_flag_ints(BR, maxN) * 4);
+  }
   if (m->glm_layers > 0) {
     const long long wr = (long long)m->n_R * m->D, wc = (long long)m->n_C * m->D;
     for (int i = 0; i < 2; ++i) {
@@ -804,7 +840,7 @@ rocs_status forward_launches(rocs_handle_t h, const rocs_model_desc* m, const ro
       a1.X_R = p.tR; a1.ldxr = q2; a1.X_C = p.tC; a1.ldxc = q2; a1.req_idx = req_idx; a1.split_in = 1;
       a1.W_RR = qw.mlp1.W_RR; a1.W_CR = qw.mlp1.W_CR; a1.W_CC = qw.mlp1.W_CC; a1.b_R = qw.mlp1.b_R; a1.b_C = qw.mlp1.b_C;
       a1.Y_R = p.qhR; a1.ldyr = d2; a1.Y_C = p.qhC; a1.ldyc = d2; a1.out_mode = 2; a1.act = ROCS_ACT_GELU;
-      a1.Z = p.Zq1;
+      a1.Z = p.Zq1; a1.flags = p.ikbo_flags;
       {
         SiteLabel sl("qgen.mlp1");
         ROCS_TRY(ikbo_bf16(h, a1, s));
@@ -867,7 +903,7 @@ rocs_status forward_launches(rocs_handle_t h, const rocs_model_desc* m, const ro
       a.X_R = p.FR; a.ldxr = 2LL * fR; a.X_C = p.FC; a.ldxc = 2LL * fC; a.req_idx = req_idx; a.split_in = 1;
       a.W_RR = gw.mlp1.W_RR; a.W_CR = gw.mlp1.W_CR; a.W_CC = gw.mlp1.W_CC; a.b_R = gw.mlp1.b_R; a.b_C = gw.mlp1.b_C;
       a.Y_R = p.hR; a.ldyr = 2LL * m->hidden; a.Y_C = p.hC; a.ldyc = 2LL * m->hidden; a.out_mode = 2;
-      a.act = ROCS_ACT_GELU; a.Z = p.Z1;
+      a.act = ROCS_ACT_GELU; a.Z = p.Z1; a.flags = p.ikbo_flags;
       {
         SiteLabel sl("glm.mlp1");
         ROCS_TRY(ikbo_bf16(h, a, s));
@@ -912,7 +948,7 @@ rocs_status forward_launches(rocs_handle_t h, const rocs_model_desc* m, const ro
     a.X_R = p.xR; a.ldxr = xr; a.X_C = p.xC; a.ldxc = xc; a.req_idx = req_idx;
     a.W_RR = nullptr; a.W_CR = sw.s1.W_CR; a.W_CC = sw.s1.W_CC; a.b_R = nullptr; a.b_C = sw.s1.b_C;
     a.Y_R = nullptr; a.ldyr = 0; a.Y_C = p.h1; a.ldyc = m->score_h1; a.out_mode = 1; a.act = ROCS_ACT_RELU;
-    a.Z = p.Zs;
+    a.Z = p.Zs; a.flags = p.ikbo_flags;
     {
       SiteLabel sl("score.l1");
       ROCS_TRY(ikbo_bf16(h, a, s));
@@ -1024,6 +1060,13 @@ extern "C" rocs_status rocs_forward(rocs_handle_t h, const rocs_model_desc* m, c
     }
   }
   return cuda_check(cudaGraphLaunch(fg->exec, s), "cudaGraphLaunch");
+}
+
+extern "C" rocs_status rocs_set_ikbo_fused(rocs_handle_t h, int32_t enable) {
+  ROCS_REQUIRE(h, "rocs_set_ikbo_fused: handle is NULL");
+  ROCS_REQUIRE(enable == 0 || enable == 1, "rocs_set_ikbo_fused: enable must be 0 or 1");
+  h->ikbo_fused = enable;
+  return ROCS_OK;
 }
 
 // =============================================================================================

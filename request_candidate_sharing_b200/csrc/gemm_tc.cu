@@ -53,6 +53,12 @@ struct Problem {
   int out_mode, act, gidx_bound, vec_ok, tma_out;
   int m_tiles, n_tiles, k_blocks, b_kblocks, tile_start, n_start;
   long long lo_off;   // out_mode 2: column offset of the low half
+  // Request/candidate tiles in one launch (the IKBO mega-kernel): flag_role 1 = this problem
+  // publishes each finished tile in flags[mb * n_tiles + nb] (one increment per epilogue warp);
+  // flag_role 2 = this problem's Z rows come from such a problem in the same launch, whose tile
+  // (zi / BM, nb) must have published before they are read (flag_ntiles = its n_tiles).
+  int* flags;
+  int flag_role, flag_ntiles;
 };
 
 struct Params {
@@ -77,6 +83,23 @@ __device__ __forceinline__ void decode_tile(const Params& P, int t, int& pi, int
     int local = t - P.p[pi].tile_start;
     mb = local / P.p[pi].n_tiles;
     nb = local - mb * P.p[pi].n_tiles;
+  }
+}
+
+// Spin (bounded) until *flag >= target, with acquire ordering for the reads that follow.
+__device__ __forceinline__ bool wait_flag(const int* flag, int target, int* status, volatile int* abort_flag) {
+  const long long t0 = clock64();
+  while (true) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v >= target) return true;
+    if (abort_flag && *abort_flag) return false;
+    if (clock64() - t0 > kWaitBudgetCycles) {
+      set_status(status, ROCS_ERR_DEVICE_TIMEOUT);
+      if (abort_flag) *abort_flag = 1;
+      return false;
+    }
+    __nanosleep(64);
   }
 }
 
@@ -130,7 +153,9 @@ __device__ __forceinline__ void store_chunk(const Problem& pr, long long grow, i
   }
 }
 
-// bias, the request contribution Z[gidx[row]] and the activation on one thread's 32 values
+// bias, the request contribution Z[gidx[row]] and the activation on one thread's 32 values.  Z
+// written by the same launch (flag_role 2) is read with ordinary loads, ordered after the flag's
+// acquire, never through the non-coherent read-only path.
 __device__ __forceinline__ void epilogue_math(const Problem& pr, const float* zrow, int col0, float (&v)[32]) {
   const bool full32 = (col0 + 32 <= pr.N) && pr.vec_ok;
   if (pr.bias != nullptr) {
@@ -152,7 +177,7 @@ __device__ __forceinline__ void epilogue_math(const Problem& pr, const float* zr
       const float4* z4 = reinterpret_cast<const float4*>(zrow + col0);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        float4 z = __ldg(z4 + j);
+        const float4 z = pr.flag_role == 2 ? z4[j] : __ldg(z4 + j);
         v[4 * j] += z.x; v[4 * j + 1] += z.y; v[4 * j + 2] += z.z; v[4 * j + 3] += z.w;
       }
     } else {
@@ -348,6 +373,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
       return (q2.Z != nullptr && gn < q2.M) ? __ldg(q2.gidx + gn) : -1;
     };
     int zi_next = load_gidx(blockIdx.x);
+    unsigned long long seen = 0;   // request tiles this warp has seen published (fused launches)
     for (int t = blockIdx.x; t < P.total_tiles; t += gridDim.x) {
       int pi, mb, nb;
       decode_tile(P, t, pi, mb, nb);
@@ -364,7 +390,32 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
         } else {
           zrow = pr.Z + (long long)zi * pr.ldz;
           // this warp's chunks of the row's Z into L1 before the wait for the accumulator (the
-          // gathered rows were the epilogue's longest latency at short K)
+          // gathered rows were the epilogue's longest latency at short K); Z that this launch
+          // writes only once it is published (below)
+          if (pr.flag_role != 2)
+            for (int c = half; c < pr.BN / 32; c += 2)
+              if (nb * pr.BN + c * 32 < pr.N)
+                asm volatile("prefetch.global.L1 [%0];" ::"l"(zrow + nb * pr.BN + c * 32));
+        }
+      }
+      if (pr.flag_role == 2) {
+        // the request tiles holding this warp's rows' Z must have published (their tiles precede
+        // every candidate tile in each CTA's order, so they never wait on this one)
+        const int lo = __reduce_min_sync(0xffffffffu, zrow != nullptr ? zi : 0x7fffffff);
+        const int hi = __reduce_max_sync(0xffffffffu, zrow != nullptr ? zi : -1);
+        bool ok = true;
+        for (int mbr = hi >= 0 ? lo / BM : 1, mend = hi >= 0 ? hi / BM : 0; mbr <= mend && ok; ++mbr) {
+          // a tile seen published stays published: later tiles skip its flag (the first 64)
+          const int fi = mbr * pr.flag_ntiles + nb;
+          if (fi < 64 && ((seen >> fi) & 1ull)) continue;
+          if (lane == 0) ok = wait_flag(pr.flags + fi, EPI_THREADS / 32, P.status, abort_flag);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (ok && fi < 64) seen |= 1ull << fi;
+        }
+        if (!ok) {
+          rvalid = false;   // timed out: the status says so; this row is not written
+          zrow = nullptr;
+        } else if (zrow != nullptr) {
           for (int c = half; c < pr.BN / 32; c += 2)
             if (nb * pr.BN + c * 32 < pr.N)
               asm volatile("prefetch.global.L1 [%0];" ::"l"(zrow + nb * pr.BN + c * 32));
@@ -449,6 +500,12 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
           }
           store_chunk(pr, grow, col0, v);
         }
+      }
+      if (pr.flag_role == 1) {
+        // this warp's part of the tile is stored (plain stores): publish it device-wide
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(pr.flags + mb * pr.n_tiles + nb, 1);
       }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
@@ -550,6 +607,8 @@ rocs_status launch_gemm_bf16(rocs_context* ctx, const GemmDesc* probs, int nprob
     p.out_mode = g.out_mode;
     p.act = g.act;
     p.lo_off = g.N;
+    p.flags = g.flags;
+    p.flag_role = g.flag_role;
     const int ve = g.out_mode == 0 ? 4 : 8;
     p.vec_ok = (g.ldo % ve == 0) && (((uintptr_t)g.out & 15) == 0) && (!g.bias || ((uintptr_t)g.bias & 15) == 0) &&
                (!g.Z || (((uintptr_t)g.Z & 15) == 0 && g.ldz % 4 == 0)) && (g.out_mode != 2 || g.N % 8 == 0);
@@ -562,7 +621,8 @@ rocs_status launch_gemm_bf16(rocs_context* ctx, const GemmDesc* probs, int nprob
       ok = ok && encode_out(ctx, &p.tmO, g.out, g.M, g.N, g.ldo, f32);
       if (ok && g.out_mode == 2)
         ok = encode_out(ctx, &p.tmOlo, reinterpret_cast<__nv_bfloat16*>(g.out) + g.N, g.M, g.N, g.ldo, false);
-      p.tma_out = ok ? 1 : 0;
+      // a publishing problem stores with plain stores, so that a fence orders them before its flag
+      p.tma_out = ok && g.flag_role != 1 ? 1 : 0;
     }
     p.m_tiles = (g.M + BM - 1) / BM;
     p.n_tiles = (g.N + p.BN - 1) / p.BN;
@@ -575,12 +635,51 @@ rocs_status launch_gemm_bf16(rocs_context* ctx, const GemmDesc* probs, int nprob
     if (g.M != probs[0].M) same_m = false;
   }
   P.total_tiles = tiles;
-  P.interleave = same_m ? 1 : 0;
+  bool any_flags = false;
+  for (int i = 0; i < nprob; ++i) any_flags = any_flags || probs[i].flag_role != 0;
+  // with completion flags the order stays problem-major: every publishing tile first
+  P.interleave = same_m && !any_flags ? 1 : 0;
   P.n_per_m = nstart;
+  // completion flags: one publishing problem, its readers with the same N; publishing tiles
+  // must come before every reading tile (problem-major order with the publisher first)
+  int producer = -1;
+  bool flagged = false;
+  for (int i = 0; i < nprob; ++i)
+    if (probs[i].flag_role == 1) {
+      if (producer >= 0 || probs[i].flags == nullptr) {
+        set_error("gemm: one publishing problem with a flags array expected");
+        return ROCS_ERR_INVALID_ARG;
+      }
+      producer = i;
+    }
+  for (int i = 0; i < nprob; ++i)
+    if (probs[i].flag_role == 2) {
+      if (producer < 0 || producer > i || probs[i].flags != probs[producer].flags || probs[i].N != probs[producer].N) {
+        set_error("gemm problem %d: reads flags of no earlier publishing problem of the same N", i);
+        return ROCS_ERR_INVALID_ARG;
+      }
+      P.p[i].flag_ntiles = P.p[producer].n_tiles;
+      flagged = true;
+    }
   const int grid = std::min(tiles, ctx->num_sms);
   LaunchTimer lt_("gemm_tc", s);
-  gemm_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(P);
-  return cuda_check(cudaGetLastError(), "gemm_tc_kernel launch");
+  if (!flagged) {
+    gemm_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(P);
+    return cuda_check(cudaGetLastError(), "gemm_tc_kernel launch");
+  }
+  // readers spin on tiles other CTAs publish: launch cooperatively (all CTAs resident)
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_check(cudaLaunchKernelEx(&cfg, gemm_tc_kernel, P), "gemm_tc_kernel cooperative launch");
 }
 
 }  // namespace rocs

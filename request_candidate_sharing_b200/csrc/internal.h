@@ -33,6 +33,7 @@ struct rocs_context {
   void* encode_fn = nullptr; // cuTensorMapEncodeTiled
   RocsTimer timer;
   int graph_replay = 1;                 // rocs_set_graph_replay
+  int ikbo_fused = 1;                   // rocs_set_ikbo_fused
   cudaStream_t capture_stream = nullptr;   // forward graphs are captured here (never the legacy stream)
   std::vector<ForwardGraph> graphs;     // at most kMaxForwardGraphs, most recent last
 };
@@ -88,6 +89,13 @@ struct GemmDesc {
   const float* bias = nullptr;
   const float* Z = nullptr; long long ldz = 0; const int32_t* gidx = nullptr; int gidx_bound = 0;
   void* out = nullptr; long long ldo = 0; int out_mode = 1; int act = ROCS_ACT_NONE;
+  // One launch for a request GEMM and the candidate GEMM that gathers its output (the IKBO
+  // mega-kernel): flag_role 1 marks the problem writing Z (it publishes each finished tile in
+  // `flags`, zeroed by the caller before the launch, ceil(M / 128) * ceil(N / BN) ints); flag_role 2
+  // marks the problem reading that Z through gidx (same flags, same N).  The launch is then
+  // cooperative, so every CTA is resident and the request tiles, first in every CTA's order,
+  // always finish.
+  int* flags = nullptr; int flag_role = 0;
 };
 
 constexpr int kMaxGemmProblems = 4;

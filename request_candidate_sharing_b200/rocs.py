@@ -124,6 +124,7 @@ _lib_fwd = _proto("rocs_forward", P, C.POINTER(ModelDesc), C.POINTER(ModelWeight
 
 _lib_ikbo_na = _proto("rocs_linear_ikbo_noalloc", P, C.POINTER(IkboDesc), P, P, P, P, P, P, P, P, P, P, P)
 _lib_graph = _proto("rocs_set_graph_replay", P, I32)
+_lib_fused = _proto("rocs_set_ikbo_fused", P, I32)
 _lib_tstart = _proto("rocs_timing_start", P, I32)
 _lib_tstop = _proto("rocs_timing_stop", P, C.c_char_p, C.c_size_t)
 
@@ -131,7 +132,7 @@ EXPORTED = ["rocs_linear_ikbo_noalloc", "rocs_timing_start", "rocs_timing_stop",
             "rocs_segments_from_counts", "rocs_linear_ikbo_workspace", "rocs_linear_ikbo", "rocs_group_layernorm",
             "rocs_fm_masked", "rocs_token_lcb_workspace", "rocs_token_lcb", "rocs_dca_cross_attn",
             "rocs_dca_encode_workspace", "rocs_dca_encode", "rocs_forward_workspace", "rocs_forward",
-            "rocs_set_graph_replay"]
+            "rocs_set_graph_replay", "rocs_set_ikbo_fused"]
 
 
 def ptr(x) -> Optional[int]:
@@ -276,6 +277,9 @@ class Rocs:
 
     def rocs_set_graph_replay(self, enable: int):
         _check(_lib_graph(self.h, int(enable)))
+
+    def rocs_set_ikbo_fused(self, enable: int):
+        _check(_lib_fused(self.h, int(enable)))
 
 
 # ---- marshalling helpers for the model structs (names follow the synth weight dictionaries) ----

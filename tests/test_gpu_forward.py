@@ -173,6 +173,25 @@ def test_forward_graph_replay(R):
         R.rocs_set_graph_replay(1)
 
 
+def test_forward_fused_ikbo_matches_two_launches(R):
+    """Every IKBO linear of the forward (GLM MLPs, query generator, scoring layer 1) as one fused
+    launch gives the same bits as the request and candidate launches; 160 requests span two
+    request row blocks, with empty and one-candidate requests among them."""
+    counts = [int(c) for c in np.random.default_rng(5).integers(0, 40, size=160)]
+    counts[7], counts[100] = 1, 0
+    case = synth.model_cfg5(B_R=len(counts), counts=counts, L=256)
+    x, W = synth.model_inputs(case), synth.model_weights(case)
+    try:
+        R.rocs_set_ikbo_fused(0)
+        out0 = run_forward(R, case, x, W)
+        R.rocs_set_ikbo_fused(1)
+        out1 = run_forward(R, case, x, W)
+    finally:
+        R.rocs_set_ikbo_fused(1)
+    for k in ("score", "E_R", "E_C", "A_R", "A_C"):
+        assert torch.equal(out0[k], out1[k]), k
+
+
 def test_forward_end_to_end_long_history(R):
     """The bench's history length L = 1024: each warp of the request-query attention walks four
     32-row chunks (online softmax across chunks, then the warps' merge), and the tcgen05

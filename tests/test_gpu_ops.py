@@ -186,6 +186,39 @@ def test_linear_cfg2_sampled_full_size(R):
     check_bf16(host(YC[torch.from_numpy(rows).cuda()]), rC, out_bf16=True, what="Y_C sample")
 
 
+@pytest.mark.parametrize("counts,dRo,dCo,act,perm", [
+    ([70, 0, 190, 33] * 80, 136, 384, "relu", False),    # 320 requests: three request row blocks, two N tiles
+    ([300] * 6, 0, 256, "gelu", False),                   # no request output; one request block
+    ([5, 1, 0, 200, 64] * 60, 64, 96, "none", True),      # candidates not grouped by request
+])
+def test_linear_fused_launch_matches_two_launches(R, counts, dRo, dCo, act, perm):
+    """The one-launch IKBO form (request tiles publish completion flags, candidate epilogues wait
+    for the Z tiles they gather) gives the same bits as the request and candidate launches."""
+    from request_candidate_sharing_b200 import rocs
+    case = synth.LinearCase("fused", np.asarray(counts, np.int32), 192, 128, dRo, dCo, act, True, 11)
+    x = synth.linear_inputs(case)
+    _, m = O.segments(case.counts)
+    if perm:   # the ABI takes any candidate order: shuffle rows and their request indices together
+        order = np.random.default_rng(3).permutation(case.B_C)
+        m = m[order].copy()
+        x = dict(x)
+        x["X_C"] = x["X_C"][order].copy()
+    try:
+        R.rocs_set_ikbo_fused(0)
+        YR0, YC0 = _run_linear(R, case, x, m, rocs.ROCS_BF16, rocs.ROCS_BF16)
+        R.rocs_set_ikbo_fused(1)
+        YR1, YC1 = _run_linear(R, case, x, m, rocs.ROCS_BF16, rocs.ROCS_BF16)
+    finally:
+        R.rocs_set_ikbo_fused(1)
+    if dRo:
+        assert torch.equal(YR0, YR1)
+    assert torch.equal(YC0, YC1)
+    rows = sample_candidates(case.counts, 2) if not perm else np.arange(0, case.B_C, 97)
+    _, rC = O.glm_linear(x["X_R"], x["X_C"][rows], m[rows], x["W_RR"] if dRo else None, x["W_CR"], x["W_CC"],
+                         x["b_R"] if dRo else None, x["b_C"], act)
+    check_bf16(host(YC1[torch.from_numpy(rows).cuda()]), rC, out_bf16=True, what="Y_C fused")
+
+
 def test_linear_short_k_many_candidates(R):
     """d = 256 with 159,840 candidates (K = 256: four k blocks per tile, so the gather epilogue and
     its prefetch of the next chunk's Z row dominate); ragged last tile.  Oracle on a sample, every
