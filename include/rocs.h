@@ -211,6 +211,43 @@ rocs_status rocs_dca_cross_attn(rocs_handle_t handle, const void* Q, const void*
                                 rocs_dtype out, void* stream);
 
 /* ------------------------------------------------------------------------------------------
+ * Candidates in any order ([REV] §2.4 notes that IKBO-DCA depends on how candidates are laid out
+ * around their request; the segment path above takes them grouped).
+ *
+ * rocs_sort_by_request: stable counting sort of B_C candidates by their request index.
+ *   req_idx [B_C] int32, device, any order; a value outside [0, B_R) is an error.
+ *   perm    [B_C] int32, device, written: perm[k] = the candidate at position k of the grouped
+ *           order.  Candidates of one request keep their relative order; candidates with a bad
+ *           index come after every valid one (in their order) and set ROCS_ERR_INDEX in the
+ *           device status.
+ *   offsets [B_R+1] int32, device, written: offsets[r] = first position of request r in perm,
+ *           offsets[B_R] = the number of candidates with a valid index.
+ *   workspace: rocs_sort_by_request_workspace bytes, 16-byte aligned (an int histogram of
+ *           (B_R + 1) x ceil(B_C / chunk) entries, chunk >= 2048).
+ *   Limits: 1 <= B_R <= 2^24, 0 <= B_C < 2^31.  Errors: ROCS_ERR_INVALID_ARG, ROCS_ERR_WORKSPACE.
+ *
+ * rocs_dca_cross_attn_unsorted: rocs_dca_cross_attn for query rows in any order, each with its
+ *   request index req_idx [rows] instead of grouped offsets.  The call sorts the rows (as
+ *   rocs_sort_by_request), gathers Q into that order, runs the segment path and writes each valid
+ *   row of O at its original position; rows with a bad index are left unwritten (and the device
+ *   status says ROCS_ERR_INDEX).  Results equal rocs_dca_cross_attn on the grouped rows.
+ *   Q, K, V, O, L, H, d_h, scale, ld_O, out and limits: as rocs_dca_cross_attn.
+ *   workspace: rocs_dca_cross_attn_unsorted_workspace bytes, 16-byte aligned (the permutation,
+ *   offsets, the sort histogram, Q and O in grouped order).
+ * ---------------------------------------------------------------------------------------- */
+rocs_status rocs_sort_by_request_workspace(rocs_handle_t handle, int32_t B_R, int64_t B_C, size_t* bytes);
+rocs_status rocs_sort_by_request(rocs_handle_t handle, const int32_t* req_idx, int32_t B_R, int64_t B_C,
+                                 int32_t* perm, int32_t* offsets, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+rocs_status rocs_dca_cross_attn_unsorted_workspace(rocs_handle_t handle, int32_t B_R, int64_t rows, int32_t H,
+                                                   int32_t d_h, rocs_dtype out, size_t* bytes);
+rocs_status rocs_dca_cross_attn_unsorted(rocs_handle_t handle, const void* Q, const void* K, const void* V,
+                                         const int32_t* req_idx, int32_t B_R, int64_t rows, int32_t L,
+                                         int32_t H, int32_t d_h, float scale, void* O, int64_t ld_O,
+                                         rocs_dtype out, void* workspace, size_t workspace_bytes,
+                                         void* stream);
+
+/* ------------------------------------------------------------------------------------------
  * a7. DCA shared sequence encoder and its K/V projections, request-only ([REV] §2.2:
  * S_i = Enc_i(S_{i-1}); S_i and its K/V computed once per request).
  *   Enc(S) = LN(S + MHSA(S) W_O^T), MHSA non-causal with Q = S W_Q^T, K = S W_K^T,

@@ -59,6 +59,21 @@ def segments(counts: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
     return offsets.astype(np.int32), m.astype(np.int32)
 
 
+def sort_by_request(m: np.ndarray, B_R: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Candidates given in any order with their request index m[c] ([REV] §2.4's map), put in
+    the grouped layout that `segments` describes: perm[k] is the candidate at grouped position k,
+    candidates of one request keep their given order, and offsets[r] is the first position of
+    request r.  An index outside [0, B_R) is not a request: such candidates follow every valid
+    one, in their given order, and offsets[B_R] counts only the valid ones."""
+    m = np.asarray(m, np.int64)
+    key = np.where((m >= 0) & (m < B_R), m, B_R)
+    perm = np.argsort(key, kind="stable")
+    counts = np.bincount(key, minlength=B_R + 1)
+    offsets = np.zeros(B_R + 1, np.int64)
+    offsets[1:] = np.cumsum(counts[:B_R])
+    return perm.astype(np.int32), offsets.astype(np.int32)
+
+
 # =============================================================================================
 # activations
 # =============================================================================================

@@ -466,6 +466,109 @@ extern "C" rocs_status rocs_dca_cross_attn(rocs_handle_t h, const void* Q, const
 }
 
 // =============================================================================================
+// candidates in any order: stable sort by request, and the cross-attention over it
+// =============================================================================================
+namespace rocs {
+namespace {
+
+struct UnsortedPlan {
+  int32_t *perm = nullptr, *offsets = nullptr, *H = nullptr;
+  void *Qs = nullptr, *Os = nullptr;
+  size_t bytes = 0;
+};
+
+UnsortedPlan plan_unsorted(int B_R, long long rows, long long qrow_bytes, long long orow_bytes, void* ws) {
+  UnsortedPlan p;
+  Carver c(ws);
+  p.perm = (int32_t*)c.take((size_t)rows * 4 + 4);
+  p.offsets = (int32_t*)c.take((size_t)(B_R + 1) * 4);
+  p.H = (int32_t*)c.take((size_t)plan_sort(B_R, rows).h_ints * 4 + 4);
+  if (qrow_bytes > 0) {
+    p.Qs = c.take((size_t)(rows * qrow_bytes) + 16);
+    p.Os = c.take((size_t)(rows * orow_bytes) + 16);
+  }
+  p.bytes = c.used;
+  return p;
+}
+
+}  // namespace
+}  // namespace rocs
+
+extern "C" rocs_status rocs_sort_by_request_workspace(rocs_handle_t h, int32_t B_R, int64_t B_C, size_t* bytes) {
+  ROCS_REQUIRE(h && bytes, "rocs_sort_by_request_workspace: NULL argument");
+  ROCS_REQUIRE(B_R >= 1 && B_R <= (1 << 24) && B_C >= 0 && B_C < 2147483647LL,
+               "rocs_sort_by_request_workspace: B_R=%d B_C=%lld out of range", B_R, (long long)B_C);
+  Carver c(nullptr);
+  c.take((size_t)plan_sort(B_R, B_C).h_ints * 4 + 4);
+  *bytes = c.used;
+  return ROCS_OK;
+}
+
+extern "C" rocs_status rocs_sort_by_request(rocs_handle_t h, const int32_t* req_idx, int32_t B_R, int64_t B_C,
+                                            int32_t* perm, int32_t* offsets, void* ws, size_t ws_bytes,
+                                            void* stream) {
+  CtxGuard ctx_guard_(h);
+  ROCS_REQUIRE(h, "rocs_sort_by_request: handle is NULL");
+  ROCS_REQUIRE(B_R >= 1 && B_R <= (1 << 24) && B_C >= 0 && B_C < 2147483647LL,
+               "rocs_sort_by_request: B_R=%d B_C=%lld out of range", B_R, (long long)B_C);
+  ROCS_REQUIRE(offsets && (B_C == 0 || (req_idx && perm && ws)), "rocs_sort_by_request: NULL argument");
+  size_t need = 0;
+  ROCS_TRY(rocs_sort_by_request_workspace(h, B_R, B_C, &need));
+  if (B_C > 0 && ws_bytes < need) {
+    set_error("rocs_sort_by_request: workspace %zu B < required %zu B", ws_bytes, need);
+    return ROCS_ERR_WORKSPACE;
+  }
+  return launch_sort_by_request(h, req_idx, B_R, B_C, perm, offsets, (int32_t*)ws, (cudaStream_t)stream);
+}
+
+extern "C" rocs_status rocs_dca_cross_attn_unsorted_workspace(rocs_handle_t h, int32_t B_R, int64_t rows, int32_t H,
+                                                              int32_t d_h, rocs_dtype out, size_t* bytes) {
+  ROCS_REQUIRE(h && bytes, "rocs_dca_cross_attn_unsorted_workspace: NULL argument");
+  ROCS_REQUIRE(B_R >= 1 && B_R <= (1 << 24) && rows >= 0 && rows < 2147483647LL && H >= 1 && d_h >= 1,
+               "rocs_dca_cross_attn_unsorted_workspace: bad sizes");
+  ROCS_REQUIRE(out == ROCS_F32 || out == ROCS_BF16, "rocs_dca_cross_attn_unsorted_workspace: bad dtype");
+  const long long dm = (long long)H * d_h;
+  *bytes = plan_unsorted(B_R, rows, dm * 2, dm * (out == ROCS_BF16 ? 2 : 4), nullptr).bytes;
+  return ROCS_OK;
+}
+
+extern "C" rocs_status rocs_dca_cross_attn_unsorted(rocs_handle_t h, const void* Q, const void* K, const void* V,
+                                                    const int32_t* req_idx, int32_t B_R, int64_t rows, int32_t L,
+                                                    int32_t H, int32_t d_h, float scale, void* O, int64_t ld_O,
+                                                    rocs_dtype out, void* ws, size_t ws_bytes, void* stream) {
+  CtxGuard ctx_guard_(h);
+  ROCS_REQUIRE(h, "rocs_dca_cross_attn_unsorted: handle is NULL");
+  ROCS_REQUIRE(Q && K && V && O && (rows == 0 || (req_idx && ws)), "rocs_dca_cross_attn_unsorted: NULL argument");
+  ROCS_REQUIRE(B_R >= 1 && B_R <= (1 << 24) && rows >= 0 && rows < 2147483647LL && L >= 1 && H >= 1,
+               "rocs_dca_cross_attn_unsorted: bad sizes");
+  ROCS_REQUIRE(d_h == 32 || d_h == 64, "rocs_dca_cross_attn_unsorted: d_h=%d (32 or 64 supported)", d_h);
+  ROCS_REQUIRE((long long)L * d_h <= 32768, "rocs_dca_cross_attn_unsorted: L*d_h=%lld exceeds 32768",
+               (long long)L * d_h);
+  ROCS_REQUIRE(ld_O >= (int64_t)H * d_h && ld_O % 2 == 0, "rocs_dca_cross_attn_unsorted: ld_O too small or odd");
+  ROCS_REQUIRE(aligned16(Q) && aligned16(K) && aligned16(V) && aligned16(O) && aligned16(ws),
+               "rocs_dca_cross_attn_unsorted: misaligned");
+  ROCS_REQUIRE(out == ROCS_F32 || out == ROCS_BF16, "rocs_dca_cross_attn_unsorted: bad dtype");
+  ROCS_REQUIRE(std::isfinite(scale), "rocs_dca_cross_attn_unsorted: scale not finite");
+  if (rows == 0) return ROCS_OK;
+  const long long dm = (long long)H * d_h;
+  const int es = out == ROCS_BF16 ? 2 : 4;
+  const UnsortedPlan need = plan_unsorted(B_R, rows, dm * 2, dm * es, nullptr);
+  if (ws_bytes < need.bytes) {
+    set_error("rocs_dca_cross_attn_unsorted: workspace %zu B < required %zu B", ws_bytes, need.bytes);
+    return ROCS_ERR_WORKSPACE;
+  }
+  const UnsortedPlan p = plan_unsorted(B_R, rows, dm * 2, dm * es, ws);
+  cudaStream_t s = (cudaStream_t)stream;
+  // sort by request (stable), gather the query rows into that order, attend on the segment path,
+  // and write every valid row back to the caller's position
+  ROCS_TRY(launch_sort_by_request(h, req_idx, B_R, rows, p.perm, p.offsets, p.H, s));
+  ROCS_TRY(launch_gather_rows(Q, dm * 2, p.perm, rows, (int)(dm * 2), p.Qs, dm * 2, s));
+  ROCS_TRY(attention_best(h, true, p.Qs, dm, 0, K, V, dm, p.offsets, B_R, rows, L, H, d_h, scale, p.Os, dm,
+                          out == ROCS_BF16, nullptr, 0, s));
+  return launch_scatter_rows(p.Os, dm * es, p.perm, p.offsets + B_R, rows, (int)(dm * es), O, ld_O * es, s);
+}
+
+// =============================================================================================
 // a7
 // =============================================================================================
 namespace rocs {

@@ -110,6 +110,23 @@ rocs_status launch_gemm_f32(rocs_context* ctx, const float* A, long long lda, in
                             const int32_t* gidx, int gidx_bound, float* out, long long ldo, int act,
                             cudaStream_t s);
 
+// Stable counting sort of candidates by request index (sort.cu).  perm[k] = the candidate at
+// sorted position k; offsets[r] = first position of request r, offsets[B_R] = valid candidates
+// (an index outside [0, B_R) sorts last and sets ROCS_ERR_INDEX).  H: plan_sort(...).h_ints ints.
+struct SortPlan {
+  int chunk = 0, nchunks = 0;
+  long long h_ints = 0;
+};
+SortPlan plan_sort(int B_R, long long B_C);
+rocs_status launch_sort_by_request(rocs_context* ctx, const int32_t* req_idx, int B_R, long long B_C, int32_t* perm,
+                                   int32_t* offsets, int32_t* H, cudaStream_t s);
+// dst[k] = src[perm[k]] for k < n (rows of row_bytes, a multiple of 16; 16-byte aligned rows)
+rocs_status launch_gather_rows(const void* src, long long ld_src_bytes, const int32_t* perm, long long n,
+                               int row_bytes, void* dst, long long ld_dst_bytes, cudaStream_t s);
+// dst[perm[k]] = src[k] for k < min(n, *count) (rows of row_bytes, a multiple of 4)
+rocs_status launch_scatter_rows(const void* src, long long ld_src_bytes, const int32_t* perm, const int32_t* count,
+                                long long n, int row_bytes, void* dst, long long ld_dst_bytes, cudaStream_t s);
+
 rocs_status launch_segments(rocs_context* ctx, const int32_t* counts, int B_R, int32_t* offsets,
                             int32_t* req_idx, long long B_C, cudaStream_t s);
 

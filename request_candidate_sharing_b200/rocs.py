@@ -125,6 +125,11 @@ _lib_fwd = _proto("rocs_forward", P, C.POINTER(ModelDesc), C.POINTER(ModelWeight
 _lib_ikbo_na = _proto("rocs_linear_ikbo_noalloc", P, C.POINTER(IkboDesc), P, P, P, P, P, P, P, P, P, P, P)
 _lib_graph = _proto("rocs_set_graph_replay", P, I32)
 _lib_fused = _proto("rocs_set_ikbo_fused", P, I32)
+_lib_sort_ws = _proto("rocs_sort_by_request_workspace", P, I32, I64, C.POINTER(C.c_size_t))
+_lib_sort = _proto("rocs_sort_by_request", P, P, I32, I64, P, P, P, C.c_size_t, P)
+_lib_xu_ws = _proto("rocs_dca_cross_attn_unsorted_workspace", P, I32, I64, I32, I32, C.c_int, C.POINTER(C.c_size_t))
+_lib_xu = _proto("rocs_dca_cross_attn_unsorted", P, P, P, P, P, I32, I64, I32, I32, I32, C.c_float, P, I64, C.c_int, P,
+                 C.c_size_t, P)
 _lib_tstart = _proto("rocs_timing_start", P, I32)
 _lib_tstop = _proto("rocs_timing_stop", P, C.c_char_p, C.c_size_t)
 
@@ -132,7 +137,8 @@ EXPORTED = ["rocs_linear_ikbo_noalloc", "rocs_timing_start", "rocs_timing_stop",
             "rocs_segments_from_counts", "rocs_linear_ikbo_workspace", "rocs_linear_ikbo", "rocs_group_layernorm",
             "rocs_fm_masked", "rocs_token_lcb_workspace", "rocs_token_lcb", "rocs_dca_cross_attn",
             "rocs_dca_encode_workspace", "rocs_dca_encode", "rocs_forward_workspace", "rocs_forward",
-            "rocs_set_graph_replay", "rocs_set_ikbo_fused"]
+            "rocs_set_graph_replay", "rocs_set_ikbo_fused", "rocs_sort_by_request_workspace",
+            "rocs_sort_by_request", "rocs_dca_cross_attn_unsorted_workspace", "rocs_dca_cross_attn_unsorted"]
 
 
 def ptr(x) -> Optional[int]:
@@ -280,6 +286,28 @@ class Rocs:
 
     def rocs_set_ikbo_fused(self, enable: int):
         _check(_lib_fused(self.h, int(enable)))
+
+    # -- candidates in any order --
+    def rocs_sort_by_request_workspace(self, B_R: int, B_C: int) -> int:
+        n = C.c_size_t(0)
+        _check(_lib_sort_ws(self.h, int(B_R), int(B_C), C.byref(n)))
+        return int(n.value)
+
+    def rocs_sort_by_request(self, req_idx, B_R: int, B_C: int, perm, offsets, workspace, workspace_bytes: int,
+                             stream=None):
+        _check(_lib_sort(self.h, ptr(req_idx), int(B_R), int(B_C), ptr(perm), ptr(offsets), ptr(workspace),
+                         int(workspace_bytes), stream))
+
+    def rocs_dca_cross_attn_unsorted_workspace(self, B_R: int, rows: int, H: int, d_h: int, out: int) -> int:
+        n = C.c_size_t(0)
+        _check(_lib_xu_ws(self.h, int(B_R), int(rows), int(H), int(d_h), int(out), C.byref(n)))
+        return int(n.value)
+
+    def rocs_dca_cross_attn_unsorted(self, Q, K, V, req_idx, B_R: int, rows: int, L: int, H: int, d_h: int,
+                                     scale: float, O, ld_O: int, out: int, workspace, workspace_bytes: int,
+                                     stream=None):
+        _check(_lib_xu(self.h, ptr(Q), ptr(K), ptr(V), ptr(req_idx), int(B_R), int(rows), int(L), int(H), int(d_h),
+                       float(scale), ptr(O), int(ld_O), int(out), ptr(workspace), int(workspace_bytes), stream))
 
 
 # ---- marshalling helpers for the model structs (names follow the synth weight dictionaries) ----

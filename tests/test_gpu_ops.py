@@ -351,6 +351,113 @@ def test_cross_attention(R, L, H, dh, counts):
 
 
 # ---------------------------------------------------------------------------------------------
+# candidates in any order: stable sort by request, and the cross-attention over it
+# ---------------------------------------------------------------------------------------------
+def _sort_case(kind, B_R, B_C, seed=0):
+    g = np.random.default_rng(seed)
+    if kind == "random":
+        return g.integers(0, B_R, B_C).astype(np.int32)
+    if kind == "grouped":
+        return np.sort(g.integers(0, B_R, B_C)).astype(np.int32)
+    if kind == "reversed":
+        return np.sort(g.integers(0, B_R, B_C))[::-1].astype(np.int32).copy()
+    if kind == "one_request":
+        return np.full(B_C, B_R - 1, np.int32)
+    if kind == "runs":   # grouped runs that revisit requests, crossing chunk boundaries
+        return np.repeat(g.integers(0, B_R, B_C // 700 + 1), 700)[:B_C].astype(np.int32)
+    raise ValueError(kind)
+
+
+@pytest.mark.parametrize("kind,B_R,B_C", [("random", 512, 242464), ("grouped", 512, 100000), ("reversed", 37, 5000),
+                                          ("one_request", 3, 4099), ("runs", 64, 50001), ("random", 1, 33),
+                                          ("random", 5, 1), ("random", 70000, 300000)])
+def test_sort_by_request_bit_exact(R, kind, B_R, B_C):
+    """The device counting sort gives the oracle's stable permutation and offsets exactly."""
+    m = _sort_case(kind, B_R, B_C)
+    perm_ref, off_ref = O.sort_by_request(m, B_R)
+    nb = R.rocs_sort_by_request_workspace(B_R, B_C)
+    ws = torch.empty(max(nb, 16), dtype=torch.uint8, device="cuda")
+    perm = torch.full((B_C,), -7, dtype=torch.int32, device="cuda")
+    off = torch.full((B_R + 1,), -7, dtype=torch.int32, device="cuda")
+    R.rocs_sort_by_request(dev_i32(m), B_R, B_C, perm, off, ws, nb, stream())
+    _status_ok(R)
+    assert np.array_equal(perm.cpu().numpy(), perm_ref)
+    assert np.array_equal(off.cpu().numpy(), off_ref)
+
+
+def test_sort_by_request_bad_indices(R):
+    """Indices outside [0, B_R) sort last in their given order, are not counted in offsets[B_R],
+    and set ROCS_ERR_INDEX."""
+    from request_candidate_sharing_b200 import rocs
+    B_R, B_C = 40, 9000
+    m = _sort_case("random", B_R, B_C, seed=4)
+    m[[0, 17, 4500, 8999]] = [-1, 40, 1 << 30, -5]
+    perm_ref, off_ref = O.sort_by_request(m, B_R)
+    nb = R.rocs_sort_by_request_workspace(B_R, B_C)
+    ws = torch.empty(max(nb, 16), dtype=torch.uint8, device="cuda")
+    perm = torch.empty(B_C, dtype=torch.int32, device="cuda")
+    off = torch.empty(B_R + 1, dtype=torch.int32, device="cuda")
+    R.rocs_sort_by_request(dev_i32(m), B_R, B_C, perm, off, ws, nb, stream())
+    assert R.rocs_get_device_status(stream()) == rocs.ROCS_ERR_INDEX
+    assert np.array_equal(perm.cpu().numpy(), perm_ref) and np.array_equal(off.cpu().numpy(), off_ref)
+    assert off_ref[-1] == B_C - 4
+
+
+@pytest.mark.parametrize("L,H,dh,counts,out", [(1024, 8, 32, [33, 1, 0, 300, 129], 0), (200, 4, 64, [3, 0, 40, 17], 1),
+                                               (1024, 8, 32, [2000, 16, 700], 1)])
+def test_cross_attention_unsorted(R, L, H, dh, counts, out):
+    """Query rows in a shuffled order, each with its request index: the result equals the grouped
+    call on the same rows bit for bit (after un-shuffling) and the oracle within the bf16 bound."""
+    from request_candidate_sharing_b200 import rocs
+    counts = np.asarray(counts, np.int32)
+    off, m = O.segments(counts)
+    B_R, n, d = len(counts), int(counts.sum()), H * dh
+    g = np.random.default_rng(L + n + 1)
+    K = synth.bf16_round(g.standard_normal((B_R, L, d)).astype(np.float32))
+    V = synth.bf16_round(g.standard_normal((B_R, L, d)).astype(np.float32))
+    Q = synth.bf16_round(g.standard_normal((n, d)).astype(np.float32))
+    order = g.permutation(n)                 # shuffled position i holds grouped row order[i]
+    Qs, ms = Q[order], m[order]
+    odt = torch.bfloat16 if out == 1 else torch.float32
+    scale = 1.0 / math.sqrt(dh)
+    Og = torch.full((n, d), float("nan"), dtype=odt, device="cuda")
+    R.rocs_dca_cross_attn(dev(Q), dev(K), dev(V), dev_i32(off), B_R, n, L, H, dh, scale, Og, d, out, stream())
+    _status_ok(R)
+    nb = R.rocs_dca_cross_attn_unsorted_workspace(B_R, n, H, dh, out)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    Ou = torch.full((n, d + 8), float("nan"), dtype=odt, device="cuda")   # wider rows: ld_O > H d_h
+    R.rocs_dca_cross_attn_unsorted(dev(Qs), dev(K), dev(V), dev_i32(ms), B_R, n, L, H, dh, scale, Ou, d + 8, out, ws,
+                                   nb, stream())
+    _status_ok(R)
+    assert torch.equal(Ou[:, :d], Og[torch.from_numpy(order).cuda()])
+    assert torch.isnan(Ou[:, d:].float()).all()          # columns past H d_h untouched
+    ref = O.cross_attn(Qs, K, V, ms, H)
+    check_bf16(host(Ou[:, :d].float()), ref, out_bf16=out == 1, what="unsorted cross-attention")
+
+
+def test_cross_attention_unsorted_bad_index_rows_untouched(R):
+    from request_candidate_sharing_b200 import rocs
+    B_R, L, H, dh, n = 3, 256, 8, 32, 500
+    d = H * dh
+    g = np.random.default_rng(9)
+    K = synth.bf16_round(g.standard_normal((B_R, L, d)).astype(np.float32))
+    V = synth.bf16_round(g.standard_normal((B_R, L, d)).astype(np.float32))
+    Q = synth.bf16_round(g.standard_normal((n, d)).astype(np.float32))
+    m = g.integers(0, B_R, n).astype(np.int32)
+    m[[5, 77]] = [3, -2]
+    nb = R.rocs_dca_cross_attn_unsorted_workspace(B_R, n, H, dh, 0)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    Ou = torch.full((n, d), -3.0, device="cuda")
+    R.rocs_dca_cross_attn_unsorted(dev(Q), dev(K), dev(V), dev_i32(m), B_R, n, L, H, dh, 1.0 / math.sqrt(dh), Ou, d, 0,
+                                   ws, nb, stream())
+    assert R.rocs_get_device_status(stream()) == rocs.ROCS_ERR_INDEX
+    assert torch.all(Ou[5] == -3.0) and torch.all(Ou[77] == -3.0)
+    ok = np.setdiff1d(np.arange(n), [5, 77])
+    ref = O.cross_attn(Q[ok], K, V, m[ok], H)
+    check_bf16(host(Ou[torch.from_numpy(ok).cuda()]), ref, what="valid rows")
+
+
+# ---------------------------------------------------------------------------------------------
 # a7 DCA encoder
 # ---------------------------------------------------------------------------------------------
 def test_dca_encode(R):

@@ -36,6 +36,33 @@ def test_segments_definition(counts):
     assert np.all(np.diff(m) >= 0)
 
 
+@pytest.mark.parametrize("m,B_R", [
+    ([2, 0, 2, 1, 0, 2], 3),
+    ([4, 4, 4], 5),                 # requests without candidates
+    ([1, -1, 0, 7, 1, 0], 3),       # bad indices (negative, too large) go last
+    ([], 2),
+])
+def test_sort_by_request_brute_force(m, B_R):
+    """Pinned against the definition written out by hand: list request 0's candidates in their
+    given order, then request 1's, ..., then the candidates whose index is not a request."""
+    perm, offsets = O.sort_by_request(np.asarray(m, np.int32), B_R)
+    expect, bounds = [], [0]
+    for r in range(B_R):
+        expect += [c for c in range(len(m)) if m[c] == r]
+        bounds.append(len(expect))
+    expect += [c for c in range(len(m)) if not 0 <= m[c] < B_R]
+    assert perm.tolist() == expect
+    assert offsets.tolist() == bounds
+
+
+def test_sort_by_request_matches_segments_on_grouped_input():
+    """Already grouped candidates: the identity permutation and exactly `segments`' offsets."""
+    counts = np.asarray([3, 0, 5, 1, 0, 2], np.int32)
+    off, m = O.segments(counts)
+    perm, offsets = O.sort_by_request(m, len(counts))
+    assert perm.tolist() == list(range(len(m))) and offsets.tolist() == off.tolist()
+
+
 def test_segments_config_counts():
     c3 = synth.model_cfg3().counts
     assert c3.min() >= 100 and c3.max() <= 1000 and len(c3) == 64
