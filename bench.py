@@ -51,6 +51,9 @@ WORKLOADS = {
     "ikbo_sweep": "IKBO linear sweep: B_R=256, N in {64, 256, 1024} candidates per request, d_in = d_out = d in "
                   "{512, 1024, 4096}, bf16 in/out, fp32 accumulate, ReLU; against two materialised-broadcast "
                   "GPU baselines (B1: Z[m] materialised and added; B2: gathered [X^R[m], X^C] with one K=2d GEMM)",
+    "xattn_unsorted": "candidate cross-attention with candidates in shuffled order (each with its request index): "
+                      "512 requests, candidates ~ clipped lognormal (median 300, 16..2000), L=1024, d=256, 8 heads; "
+                      "stable sort by request + gather + segment-path attention + scatter, against the grouped call",
 }
 
 
@@ -677,6 +680,87 @@ def run_ikbo_sweep(args, rank, world, local):
     R.close()
 
 
+def run_xattn_unsorted(args, rank, world, local):
+    """The grouped cross-attention (rocs_dca_cross_attn) and the same rows shuffled, each with its
+    request index (rocs_dca_cross_attn_unsorted: sort, gather, attention, scatter), plus the sort
+    alone (rocs_sort_by_request).  Each repetition is timed alone with CUDA events after an L2
+    flush; medians.  Inputs: the forward workload's counts (seed 1 + 1000 x rank), bf16 normal Q,
+    K, V drawn on the device, fp32 output."""
+    import torch
+    from request_candidate_sharing_b200 import rocs
+    import synth
+    dev = torch.device("cuda", local)
+    R = rocs.Rocs(local)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    reps = max(args.steps, 3)
+    counts = synth.counts_lognormal(1 + 1000 * rank, 512, 300.0, 1.0, 16, 2000)
+    B_R, L, H, dh = len(counts), 1024, 8, 32
+    d = H * dh
+    B_C = int(counts.sum())
+    g = torch.Generator(device=dev).manual_seed(7 + rank)
+    bf = torch.bfloat16
+    Q = torch.randn(B_C, d, device=dev, generator=g).to(bf)
+    K = torch.randn(B_R * L, d, device=dev, generator=g).to(bf)
+    V = torch.randn(B_R * L, d, device=dev, generator=g).to(bf)
+    off = torch.zeros(B_R + 1, dtype=torch.int32, device=dev)
+    off[1:] = torch.from_numpy(counts).to(dev).cumsum(0)
+    m = torch.repeat_interleave(torch.arange(B_R, device=dev, dtype=torch.int32), torch.from_numpy(counts).to(dev).long())
+    order = torch.randperm(B_C, device=dev, generator=g)
+    Qs, ms = Q[order].contiguous(), m[order].contiguous()
+    O = torch.empty(B_C, d, device=dev)
+    Ou = torch.empty(B_C, d, device=dev)
+    scale = 1.0 / math.sqrt(dh)
+    sh = torch.cuda.current_stream(dev).cuda_stream
+    nb = R.rocs_dca_cross_attn_unsorted_workspace(B_R, B_C, H, dh, rocs.ROCS_F32)
+    ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+    nbs = R.rocs_sort_by_request_workspace(B_R, B_C)
+    wss = torch.empty(max(nbs, 16), dtype=torch.uint8, device=dev)
+    perm = torch.empty(B_C, dtype=torch.int32, device=dev)
+    offs = torch.empty(B_R + 1, dtype=torch.int32, device=dev)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            ts.append(e0.elapsed_time(e1))
+        ts.sort()
+        return ts[len(ts) // 2]
+
+    ms_g = timed(lambda: R.rocs_dca_cross_attn(Q, K, V, off, B_R, B_C, L, H, dh, scale, O, d, rocs.ROCS_F32, sh))
+    ms_u = timed(lambda: R.rocs_dca_cross_attn_unsorted(Qs, K, V, ms, B_R, B_C, L, H, dh, scale, Ou, d, rocs.ROCS_F32,
+                                                        ws, nb, sh))
+    ms_s = timed(lambda: R.rocs_sort_by_request(ms, B_R, B_C, perm, offs, wss, nbs, sh))
+    if R.rocs_get_device_status(sh) != 0:
+        raise RuntimeError("device status set")
+    same = bool(torch.equal(Ou, O[order]))
+    # per-kernel times of the unsorted call (direct launches, per-launch CUDA events)
+    R.rocs_timing_start(64)
+    for _ in range(reps):
+        flush.fill_(1)
+        R.rocs_dca_cross_attn_unsorted(Qs, K, V, ms, B_R, B_C, L, H, dh, scale, Ou, d, rocs.ROCS_F32, ws, nb, sh)
+    kern = {k: round(t / reps, 4) for k, (n, t) in R.rocs_timing_stop().items()}
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(B_C / (ms_u / 1e3), 1), "unit": "candidates/s", "n_gpus": world,
+                "steps": reps, "warmup": args.warmup, "ms_per_step": round(ms_u, 4), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded counts; torch normal Q/K/V drawn on the device)",
+                "config": {"workload": "xattn_unsorted", "description": WORKLOADS["xattn_unsorted"], "B_R": B_R,
+                           "B_C": B_C, "l2": "flushed (256 MB write) before every repetition"},
+                "grouped_ms": round(ms_g, 4), "unsorted_ms": round(ms_u, 4), "sort_ms": round(ms_s, 4),
+                "unsorted_overhead": round(ms_u / ms_g - 1.0, 4),
+                "sort_cands_per_s": round(B_C / (ms_s / 1e3), 1),
+                "unsorted_equals_grouped": same, "unsorted_kernel_ms": kern}
+        print(json.dumps(line), flush=True)
+    R.close()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -702,6 +786,8 @@ def main():
     rank, world, local = dist_setup(args.gpus)
     if args.workload == "ikbo_sweep":
         run_ikbo_sweep(args, rank, world, local)
+    elif args.workload == "xattn_unsorted":
+        run_xattn_unsorted(args, rank, world, local)
     else:
         run_librocs(args, rank, world, local)
 

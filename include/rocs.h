@@ -223,7 +223,7 @@ rocs_status rocs_dca_cross_attn(rocs_handle_t handle, const void* Q, const void*
  *   offsets [B_R+1] int32, device, written: offsets[r] = first position of request r in perm,
  *           offsets[B_R] = the number of candidates with a valid index.
  *   workspace: rocs_sort_by_request_workspace bytes, 16-byte aligned (an int histogram of
- *           (B_R + 1) x ceil(B_C / chunk) entries, chunk >= 2048).
+ *           (B_R + 1) x ceil(B_C / chunk) entries, chunk >= 512).
  *   Limits: 1 <= B_R <= 2^24, 0 <= B_C < 2^31.  Errors: ROCS_ERR_INVALID_ARG, ROCS_ERR_WORKSPACE.
  *
  * rocs_dca_cross_attn_unsorted: rocs_dca_cross_attn for query rows in any order, each with its

@@ -560,9 +560,14 @@ extern "C" rocs_status rocs_dca_cross_attn_unsorted(rocs_handle_t h, const void*
   const UnsortedPlan p = plan_unsorted(B_R, rows, dm * 2, dm * es, ws);
   cudaStream_t s = (cudaStream_t)stream;
   // sort by request (stable), gather the query rows into that order, attend on the segment path,
-  // and write every valid row back to the caller's position
+  // and write every valid row at the caller's position
   ROCS_TRY(launch_sort_by_request(h, req_idx, B_R, rows, p.perm, p.offsets, p.H, s));
   ROCS_TRY(launch_gather_rows(Q, dm * 2, p.perm, rows, (int)(dm * 2), p.Qs, dm * 2, s));
+  // the tcgen05 kernel writes each row straight to its caller position (out_rows = perm); the
+  // other kernels write the grouped order, which is then scattered
+  const rocs_status st = launch_attention_tc(h, p.Qs, dm, 0, K, V, dm, (long long)B_R * L, p.offsets, B_R, rows, L,
+                                             H, d_h, scale, O, ld_O, out == ROCS_BF16, nullptr, 0, s, p.perm);
+  if (st != ROCS_ERR_UNSUPPORTED) return st;
   ROCS_TRY(attention_best(h, true, p.Qs, dm, 0, K, V, dm, p.offsets, B_R, rows, L, H, d_h, scale, p.Os, dm,
                           out == ROCS_BF16, nullptr, 0, s));
   return launch_scatter_rows(p.Os, dm * es, p.perm, p.offsets + B_R, rows, (int)(dm * es), O, ld_O * es, s);

@@ -49,6 +49,7 @@ struct AttnTcParams {
   int out_bf16;
   __nv_bfloat16* O2;
   long long ldo2;
+  const int32_t* out_rows;   // optional: query row q is written to output row out_rows[q]
   int* status;
 };
 
@@ -367,8 +368,9 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
         tmem_ld_wait();
         l_final = __uint_as_float(lw);
       }
-      const long long qrow = q0 + (long long)(g + GROUPS * k_tile) * TQ + row;
-      if (qrow >= q1) return;
+      const long long qrow0 = q0 + (long long)(g + GROUPS * k_tile) * TQ + row;
+      if (qrow0 >= q1) return;
+      const long long qrow = P.out_rows != nullptr ? (long long)P.out_rows[qrow0] : qrow0;
       const float inv = 1.0f / l_final;
 #pragma unroll
       for (int e = 0; e < DH; ++e) out[e] *= inv;
@@ -584,7 +586,7 @@ rocs_status at_launch(rocs_context* ctx, AttnTcParams& P, int B_R, int H, cudaSt
 rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq, int q_split, const void* K,
                                 const void* V, long long ldkv, long long kv_rows, const int32_t* offsets, int B_R,
                                 long long rows, int L, int H, int d_h, float scale, void* O, long long ldo,
-                                int out_bf16, void* O2, long long ldo2, cudaStream_t s) {
+                                int out_bf16, void* O2, long long ldo2, cudaStream_t s, const int32_t* out_rows) {
   if (B_R == 0 || rows == 0) return ROCS_OK;
   if ((d_h != 32 && d_h != 64) || L < 1 || (long long)L * d_h > 32768 || (L + TK - 1) / TK > AT_MAX_KB ||
       ((uintptr_t)Q & 15) || ((uintptr_t)K & 15) || ((uintptr_t)V & 15) || ldq % 8 || ldkv % 8 ||
@@ -614,6 +616,7 @@ rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq,
   P.out_bf16 = out_bf16;
   P.O2 = (__nv_bfloat16*)O2;
   P.ldo2 = ldo2;
+  P.out_rows = out_rows;
   P.status = ctx->d_status;
   LaunchTimer lt_("attn_tc", s);
   if (d_h == 32) return q_split ? at_launch<32, true>(ctx, P, B_R, H, s) : at_launch<32, false>(ctx, P, B_R, H, s);

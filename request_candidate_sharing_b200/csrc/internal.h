@@ -197,7 +197,8 @@ rocs_status launch_attention_req_absorbed(rocs_context* ctx, const void* Q, long
 rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq, int q_split, const void* K,
                                 const void* V, long long ldkv, long long kv_rows, const int32_t* offsets, int B_R,
                                 long long rows, int L, int H, int d_h, float scale, void* O, long long ldo,
-                                int out_bf16, void* O2, long long ldo2, cudaStream_t s);
+                                int out_bf16, void* O2, long long ldo2, cudaStream_t s,
+                                const int32_t* out_rows = nullptr);
 
 rocs_status launch_score_head(const void* X, long long ldx, long long rows, int K, const void* w,
                               const float* b, float* out, cudaStream_t s);

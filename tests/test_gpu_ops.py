@@ -403,11 +403,14 @@ def test_sort_by_request_bad_indices(R):
     assert off_ref[-1] == B_C - 4
 
 
-@pytest.mark.parametrize("L,H,dh,counts,out", [(1024, 8, 32, [33, 1, 0, 300, 129], 0), (200, 4, 64, [3, 0, 40, 17], 1),
-                                               (1024, 8, 32, [2000, 16, 700], 1)])
-def test_cross_attention_unsorted(R, L, H, dh, counts, out):
+@pytest.mark.parametrize("L,H,dh,counts,out,extra", [(1024, 8, 32, [33, 1, 0, 300, 129], 0, 8),
+                                                     (200, 4, 64, [3, 0, 40, 17], 1, 8),
+                                                     (1024, 8, 32, [2000, 16, 700], 1, 2)])
+def test_cross_attention_unsorted(R, L, H, dh, counts, out, extra):
     """Query rows in a shuffled order, each with its request index: the result equals the grouped
-    call on the same rows bit for bit (after un-shuffling) and the oracle within the bf16 bound."""
+    call on the same rows bit for bit (after un-shuffling) and the oracle within the bf16 bound.
+    Output rows wider than H d_h by `extra`: 8 keeps rows 16-byte aligned (the attention writes
+    each row at its caller position), 2 does not (grouped output, then a row scatter)."""
     from request_candidate_sharing_b200 import rocs
     counts = np.asarray(counts, np.int32)
     off, m = O.segments(counts)
@@ -425,9 +428,9 @@ def test_cross_attention_unsorted(R, L, H, dh, counts, out):
     _status_ok(R)
     nb = R.rocs_dca_cross_attn_unsorted_workspace(B_R, n, H, dh, out)
     ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
-    Ou = torch.full((n, d + 8), float("nan"), dtype=odt, device="cuda")   # wider rows: ld_O > H d_h
-    R.rocs_dca_cross_attn_unsorted(dev(Qs), dev(K), dev(V), dev_i32(ms), B_R, n, L, H, dh, scale, Ou, d + 8, out, ws,
-                                   nb, stream())
+    Ou = torch.full((n, d + extra), float("nan"), dtype=odt, device="cuda")   # wider rows: ld_O > H d_h
+    R.rocs_dca_cross_attn_unsorted(dev(Qs), dev(K), dev(V), dev_i32(ms), B_R, n, L, H, dh, scale, Ou, d + extra, out,
+                                   ws, nb, stream())
     _status_ok(R)
     assert torch.equal(Ou[:, :d], Og[torch.from_numpy(order).cuda()])
     assert torch.isnan(Ou[:, d:].float()).all()          # columns past H d_h untouched
