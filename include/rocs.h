@@ -200,15 +200,20 @@ rocs_status rocs_token_lcb(rocs_handle_t handle, const void* E_R, const void* E_
  *     attend to request r.  offsets int32 [B_R+1], device.
  *   K, V [B_R, L, H*d_h] bf16 (each request's K/V stored once).
  *   O [rows, ld_O] in `out` dtype (bf16 or fp32), head h at columns [h*d_h, (h+1)*d_h).
- *   O_q = softmax(q k^T * scale) v per head, no masking; fp32 softmax statistics.
- *   Each (request, head)'s K/V is streamed through shared memory once per 128 queries of that
- *   request and shared by those queries (no per-candidate copy of K/V exists).
- *   Limits: d_h in {32, 64}; L * d_h <= 32768.
+ *   O_q = softmax(q k^T * scale) v per head; fp32 softmax statistics.
+ *   kv_len int32 [B_R], device, or NULL: request r's keys are the first kv_len[r] of its L rows
+ *     (a ragged history, 1 <= kv_len[r] <= L); later rows are padding and never attended.  A
+ *     length outside [1, L] sets ROCS_ERR_COUNTS and that request's rows are not written.
+ *     NULL: every request has L keys.
+ *   Each (request, head)'s K/V is staged in shared memory once and shared by that request's
+ *   queries (no per-candidate copy of K/V exists) when L * d_h <= 32768; longer histories are
+ *   streamed through a shared-memory ring of 64-key blocks.
+ *   Limits: d_h in {32, 64}; B_R * L < 2^31.
  * ---------------------------------------------------------------------------------------- */
 rocs_status rocs_dca_cross_attn(rocs_handle_t handle, const void* Q, const void* K, const void* V,
                                 const int32_t* offsets, int32_t B_R, int64_t rows, int32_t L,
                                 int32_t H, int32_t d_h, float scale, void* O, int64_t ld_O,
-                                rocs_dtype out, void* stream);
+                                rocs_dtype out, const int32_t* kv_len, void* stream);
 
 /* ------------------------------------------------------------------------------------------
  * Candidates in any order ([REV] §2.4 notes that IKBO-DCA depends on how candidates are laid out
@@ -244,8 +249,8 @@ rocs_status rocs_dca_cross_attn_unsorted_workspace(rocs_handle_t handle, int32_t
 rocs_status rocs_dca_cross_attn_unsorted(rocs_handle_t handle, const void* Q, const void* K, const void* V,
                                          const int32_t* req_idx, int32_t B_R, int64_t rows, int32_t L,
                                          int32_t H, int32_t d_h, float scale, void* O, int64_t ld_O,
-                                         rocs_dtype out, void* workspace, size_t workspace_bytes,
-                                         void* stream);
+                                         rocs_dtype out, const int32_t* kv_len, void* workspace,
+                                         size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------------
  * a7. DCA shared sequence encoder and its K/V projections, request-only ([REV] §2.2:
@@ -256,6 +261,12 @@ rocs_status rocs_dca_cross_attn_unsorted(rocs_handle_t handle, const void* Q, co
  *   V^C_i = S_i W_V^C^T.
  *   Hist [B_R, L, d] bf16.  S [layers, B_R, L, d] bf16 written.
  *   KV [layers, 4, B_R, L, d] bf16 written, order (K^R, V^R, K^C, V^C).
+ *   lengths int32 [B_R], device, or NULL: request r's history is its first lengths[r] rows
+ *     (1 <= lengths[r] <= L); the self-attention takes only those rows as keys.  Rows after them
+ *     are padding: they are computed like the others (every per-row step is row-independent) and
+ *     their S and K/V rows are unspecified, but they never reach a history row.  NULL: every
+ *     history has L rows.  Histories longer than the staged kernels hold (L * d_h > 32768) are
+ *     streamed through shared memory.
  * ---------------------------------------------------------------------------------------- */
 typedef struct {
   const void *Wq, *Wk, *Wv, *Wo;       /* [d, d] bf16 */
@@ -271,6 +282,7 @@ typedef struct {
 
 rocs_status rocs_dca_encode_workspace(rocs_handle_t handle, const rocs_dca_desc* desc, size_t* bytes);
 rocs_status rocs_dca_encode(rocs_handle_t handle, const rocs_dca_desc* desc, const void* Hist,
+                            const int32_t* lengths /* [B_R] or NULL */,
                             const rocs_dca_layer_weights* weights /* [layers] */, void* S, void* KV,
                             void* workspace, size_t workspace_bytes, void* stream);
 
@@ -349,6 +361,9 @@ typedef struct {
   const void *E_R, *E_C;            /* GLM inputs */
   const void* Hist;                 /* DCA history */
   const void *Y_R, *Y_C;            /* DCA own query embeddings (source 0) */
+  const int32_t* hist_len;          /* [B_R] or NULL: request r's history is its first hist_len[r] of
+                                       the L rows of Hist (1 <= hist_len[r] <= L; the rest is padding,
+                                       never a key).  NULL: every history has L rows. */
 } rocs_inputs;
 
 typedef struct {

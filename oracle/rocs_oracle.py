@@ -257,11 +257,21 @@ def mha_rows(Q: np.ndarray, K: np.ndarray, V: np.ndarray, H: int) -> np.ndarray:
 
 
 def cross_attn(Q: np.ndarray, K: np.ndarray, V: np.ndarray, owner: np.ndarray, H: int,
-               chunk: int = 64) -> np.ndarray:
+               chunk: int = 64, kv_len: Optional[np.ndarray] = None) -> np.ndarray:
     """Each query row c attends to a materialised copy of K[owner[c]], V[owner[c]]
-    (K/V [B_R, L, d], Q [n, d]) -> [n, d]."""
+    (K/V [B_R, L, d], Q [n, d]) -> [n, d].  With kv_len, request r's history is its first
+    kv_len[r] rows: its queries attend to those keys only (the rows after them are padding)."""
     Q = np.asarray(Q, F64)
     out = np.empty_like(Q)
+    if kv_len is not None:
+        owner = np.asarray(owner)
+        for r in np.unique(owner):
+            idx = np.flatnonzero(owner == r)
+            Lr = int(kv_len[r])
+            Kr = np.asarray(K[r:r + 1, :Lr], F64)
+            Vr = np.asarray(V[r:r + 1, :Lr], F64)
+            out[idx] = mha_rows(Q[idx][None], Kr, Vr, H)[0]
+        return out
     for s0 in range(0, len(Q), chunk):
         idx = np.asarray(owner[s0:s0 + chunk])
         Kc = np.asarray(K, F64)[idx]          # broadcast copy, [c, L, d]
@@ -273,28 +283,33 @@ def cross_attn(Q: np.ndarray, K: np.ndarray, V: np.ndarray, owner: np.ndarray, H
 # =============================================================================================
 # A8: DCA shared sequence encoder (request-only) -- [REV] §2.2, S_i = Enc_i(S_{i-1})
 # =============================================================================================
-def encoder_layer(S: np.ndarray, Wq, Wk, Wv, Wo, gamma, beta, H: int) -> np.ndarray:
+def encoder_layer(S: np.ndarray, Wq, Wk, Wv, Wo, gamma, beta, H: int,
+                  lengths: Optional[np.ndarray] = None) -> np.ndarray:
     """Enc(S) = LN(S + MHSA(S) W_O^T) per request, MHSA with Q = S W_Q^T, K = S W_K^T,
-    V = S W_V^T, non-causal, LN per token over d."""
+    V = S W_V^T, non-causal, LN per token over d.  With lengths, request r's sequence is its
+    first lengths[r] rows; the rows after them are not part of it and come out as NaN."""
     S = np.asarray(S, F64)
     Q = S @ np.asarray(Wq, F64).T
     K = S @ np.asarray(Wk, F64).T
     V = S @ np.asarray(Wv, F64).T
-    A = np.empty_like(S)
+    A = np.full_like(S, np.nan)
     for r in range(S.shape[0]):
-        A[r] = mha_rows(Q[r:r + 1], K[r:r + 1], V[r:r + 1], H)[0]
+        Lr = S.shape[1] if lengths is None else int(lengths[r])
+        A[r, :Lr] = mha_rows(Q[r:r + 1, :Lr], K[r:r + 1, :Lr], V[r:r + 1, :Lr], H)[0]
     return group_layernorm(S + A @ np.asarray(Wo, F64).T, gamma, beta)
 
 
-def dca_encode(Hist: np.ndarray, W: Dict[str, np.ndarray], layers: int, H: int):
+def dca_encode(Hist: np.ndarray, W: Dict[str, np.ndarray], layers: int, H: int,
+               lengths: Optional[np.ndarray] = None):
     """Runs the request-only encoder and the per-depth K/V projections once per request.
-    Returns lists S[l] [B_R, L, d] and KV[l] = (K_R, V_R, K_C, V_C) each [B_R, L, d]."""
+    Returns lists S[l] [B_R, L, d] and KV[l] = (K_R, V_R, K_C, V_C) each [B_R, L, d].  With
+    lengths (a ragged history), rows past lengths[r] are NaN in every output."""
     S = np.asarray(Hist, F64)
     Ss, KVs = [], []
     for l in range(layers):
         p = f"enc{l}."
         S = encoder_layer(S, W[p + "Wq"], W[p + "Wk"], W[p + "Wv"], W[p + "Wo"],
-                          W[p + "ln.gamma"], W[p + "ln.beta"], H)
+                          W[p + "ln.gamma"], W[p + "ln.beta"], H, lengths)
         Ss.append(S)
         p = f"kv{l}."
         KVs.append(tuple(S @ np.asarray(W[p + k], F64).T for k in ("WK_R", "WV_R", "WK_C", "WV_C")))
@@ -372,8 +387,9 @@ def _dca_depths(case, inputs, W, db: DenseBatch, query_rows, Ss, KVs):
         QR, QC = query_gen_rows(YR, YC, W, f"qg{l}.")
         db.check_request_copies(QR, f"query generator {l}", rtol=1e-12)
         K_R, V_R, K_C, V_C = KVs[l]
-        aR = cross_attn(QR, K_R, V_R, db.owner, a.H)      # request queries, request K/V
-        aC = cross_attn(QC, K_C, V_C, db.owner, a.H)      # candidate queries, shared K/V copy
+        lengths = inputs.get("hist_len")                  # a ragged history, or None
+        aR = cross_attn(QR, K_R, V_R, db.owner, a.H, kv_len=lengths)      # request queries, request K/V
+        aC = cross_attn(QC, K_C, V_C, db.owner, a.H, kv_len=lengths)      # candidate queries, shared K/V
         db.check_request_copies(aR, f"request cross-attention {l}", rtol=1e-12)
         A_R.append(aR)
         A_C.append(aC)
@@ -386,7 +402,7 @@ def forward_cfg4(case, inputs, W, m):
     A_C[l] [n, d]."""
     a = case.dca
     db = DenseBatch(m, len(inputs["H"]))
-    Ss, KVs = dca_encode(inputs["H"], W, a.layers, a.H)
+    Ss, KVs = dca_encode(inputs["H"], W, a.layers, a.H, inputs.get("hist_len"))
     state = {"YR": db.broadcast(inputs["Y_R"]), "YC": db.with_probe(inputs["Y_C"])}
 
     def query_rows(l, appended):
@@ -405,7 +421,7 @@ def forward_cfg5(case, inputs, W, m):
     the candidate scoring MLP [Y^R_m, A^R_m | Y^C, A^C] -> 512 -> 256 -> 1 (sigmoid)."""
     g, a = case.glm, case.dca
     outs, rows, db = glm_stack(inputs["E_R"], inputs["E_C"], m, W, g)
-    Ss, KVs = dca_encode(inputs["H"], W, a.layers, a.H)
+    Ss, KVs = dca_encode(inputs["H"], W, a.layers, a.H, inputs.get("hist_len"))
 
     def query_rows(l, appended):
         return rows[l]

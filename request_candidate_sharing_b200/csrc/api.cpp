@@ -162,18 +162,22 @@ rocs_status linear_bf16(rocs_context* ctx, const void* X, long long ldx, long lo
 
 // Attention against per-request K/V: the tcgen05 kernel where its shared memory holds the
 // request's K/V, else the streaming (cross) or resident (self) mma.sync kernels.
+// kv_len (nullable): request r's keys are the first kv_len[r] of its L rows (a ragged history).
+// Histories too long to stage in shared memory take the streaming kernel.
 rocs_status attention_best(rocs_context* ctx, bool streaming_fallback, const void* Q, long long ldq, int q_split,
                            const void* K, const void* V, long long ldkv, const int32_t* offsets, int B_R,
                            long long rows, int L, int H, int d_h, float scale, void* O, long long ldo, int out_bf16,
-                           void* O2, long long ldo2, cudaStream_t s) {
+                           void* O2, long long ldo2, cudaStream_t s, const int32_t* kv_len = nullptr) {
   rocs_status st = launch_attention_tc(ctx, Q, ldq, q_split, K, V, ldkv, (long long)B_R * L, offsets, B_R, rows, L, H,
-                                       d_h, scale, O, ldo, out_bf16, O2, ldo2, s);
+                                       d_h, scale, O, ldo, out_bf16, O2, ldo2, s, nullptr, kv_len);
   if (st != ROCS_ERR_UNSUPPORTED) return st;
-  if (streaming_fallback)
-    return launch_attention_stream(ctx, Q, ldq, q_split, K, V, ldkv, (long long)L * ldkv, offsets, B_R, rows, L, H,
-                                   d_h, scale, O, ldo, out_bf16, O2, ldo2, s);
-  return launch_attention(ctx, Q, ldq, q_split, K, V, ldkv, (long long)L * ldkv, offsets, B_R, rows, L, H, d_h, scale,
-                          O, ldo, out_bf16, O2, ldo2, s);
+  if (!streaming_fallback) {
+    st = launch_attention(ctx, Q, ldq, q_split, K, V, ldkv, (long long)L * ldkv, offsets, B_R, rows, L, H, d_h, scale,
+                          O, ldo, out_bf16, O2, ldo2, s, kv_len);
+    if (st != ROCS_ERR_UNSUPPORTED) return st;
+  }
+  return launch_attention_stream(ctx, Q, ldq, q_split, K, V, ldkv, (long long)L * ldkv, offsets, B_R, rows, L, H,
+                                 d_h, scale, O, ldo, out_bf16, O2, ldo2, s, kv_len);
 }
 
 // Workspace of rocs_linear_ikbo: Z, then (only if a row is not 16-B aligned) padded operands.
@@ -449,20 +453,20 @@ extern "C" rocs_status rocs_token_lcb(rocs_handle_t h, const void* E_R, const vo
 extern "C" rocs_status rocs_dca_cross_attn(rocs_handle_t h, const void* Q, const void* K, const void* V,
                                            const int32_t* offsets, int32_t B_R, int64_t rows, int32_t L, int32_t H,
                                            int32_t d_h, float scale, void* O, int64_t ld_O, rocs_dtype out,
-                                           void* stream) {
+                                           const int32_t* kv_len, void* stream) {
   CtxGuard ctx_guard_(h);
   ROCS_REQUIRE(h, "rocs_dca_cross_attn: handle is NULL");
   ROCS_REQUIRE(Q && K && V && offsets && O, "rocs_dca_cross_attn: NULL argument");
   ROCS_REQUIRE(B_R >= 1 && rows >= 0 && L >= 1 && H >= 1, "rocs_dca_cross_attn: bad sizes");
   ROCS_REQUIRE(d_h == 32 || d_h == 64, "rocs_dca_cross_attn: d_h=%d (32 or 64 supported)", d_h);
-  ROCS_REQUIRE((long long)L * d_h <= 32768, "rocs_dca_cross_attn: L*d_h=%lld exceeds 32768", (long long)L * d_h);
+  ROCS_REQUIRE((long long)B_R * L < 2147483647LL, "rocs_dca_cross_attn: B_R*L too large");
   ROCS_REQUIRE(ld_O >= (int64_t)H * d_h && ld_O % 2 == 0, "rocs_dca_cross_attn: ld_O too small or odd");
   ROCS_REQUIRE(aligned16(Q) && aligned16(K) && aligned16(V) && aligned16(O), "rocs_dca_cross_attn: misaligned");
   ROCS_REQUIRE(out == ROCS_F32 || out == ROCS_BF16, "rocs_dca_cross_attn: bad dtype");
   ROCS_REQUIRE(std::isfinite(scale), "rocs_dca_cross_attn: scale not finite");
   const long long dm = (long long)H * d_h;
   return attention_best(h, true, Q, dm, 0, K, V, dm, offsets, B_R, rows, L, H, d_h, scale, O, ld_O, out == ROCS_BF16,
-                        nullptr, 0, (cudaStream_t)stream);
+                        nullptr, 0, (cudaStream_t)stream, kv_len);
 }
 
 // =============================================================================================
@@ -535,15 +539,15 @@ extern "C" rocs_status rocs_dca_cross_attn_unsorted_workspace(rocs_handle_t h, i
 extern "C" rocs_status rocs_dca_cross_attn_unsorted(rocs_handle_t h, const void* Q, const void* K, const void* V,
                                                     const int32_t* req_idx, int32_t B_R, int64_t rows, int32_t L,
                                                     int32_t H, int32_t d_h, float scale, void* O, int64_t ld_O,
-                                                    rocs_dtype out, void* ws, size_t ws_bytes, void* stream) {
+                                                    rocs_dtype out, const int32_t* kv_len, void* ws, size_t ws_bytes,
+                                                    void* stream) {
   CtxGuard ctx_guard_(h);
   ROCS_REQUIRE(h, "rocs_dca_cross_attn_unsorted: handle is NULL");
   ROCS_REQUIRE(Q && K && V && O && (rows == 0 || (req_idx && ws)), "rocs_dca_cross_attn_unsorted: NULL argument");
   ROCS_REQUIRE(B_R >= 1 && B_R <= (1 << 24) && rows >= 0 && rows < 2147483647LL && L >= 1 && H >= 1,
                "rocs_dca_cross_attn_unsorted: bad sizes");
   ROCS_REQUIRE(d_h == 32 || d_h == 64, "rocs_dca_cross_attn_unsorted: d_h=%d (32 or 64 supported)", d_h);
-  ROCS_REQUIRE((long long)L * d_h <= 32768, "rocs_dca_cross_attn_unsorted: L*d_h=%lld exceeds 32768",
-               (long long)L * d_h);
+  ROCS_REQUIRE((long long)B_R * L < 2147483647LL, "rocs_dca_cross_attn_unsorted: B_R*L too large");
   ROCS_REQUIRE(ld_O >= (int64_t)H * d_h && ld_O % 2 == 0, "rocs_dca_cross_attn_unsorted: ld_O too small or odd");
   ROCS_REQUIRE(aligned16(Q) && aligned16(K) && aligned16(V) && aligned16(O) && aligned16(ws),
                "rocs_dca_cross_attn_unsorted: misaligned");
@@ -566,10 +570,10 @@ extern "C" rocs_status rocs_dca_cross_attn_unsorted(rocs_handle_t h, const void*
   // the tcgen05 kernel writes each row straight to its caller position (out_rows = perm); the
   // other kernels write the grouped order, which is then scattered
   const rocs_status st = launch_attention_tc(h, p.Qs, dm, 0, K, V, dm, (long long)B_R * L, p.offsets, B_R, rows, L,
-                                             H, d_h, scale, O, ld_O, out == ROCS_BF16, nullptr, 0, s, p.perm);
+                                             H, d_h, scale, O, ld_O, out == ROCS_BF16, nullptr, 0, s, p.perm, kv_len);
   if (st != ROCS_ERR_UNSUPPORTED) return st;
   ROCS_TRY(attention_best(h, true, p.Qs, dm, 0, K, V, dm, p.offsets, B_R, rows, L, H, d_h, scale, p.Os, dm,
-                          out == ROCS_BF16, nullptr, 0, s));
+                          out == ROCS_BF16, nullptr, 0, s, kv_len));
   return launch_scatter_rows(p.Os, dm * es, p.perm, p.offsets + B_R, rows, (int)(dm * es), O, ld_O * es, s);
 }
 
@@ -597,9 +601,12 @@ EncScratch carve_encoder(Carver& c, long long rowsL, int d, int B_R) {
 }
 
 // One encoder layer S_out = LN(S_in + MHSA(S_in) W_O^T) and the four K/V projections of S_out.
+// lengths (nullable): request r's history is its first lengths[r] rows; the rows after them are
+// padding, computed like any row (each row's LayerNorm and projections are independent) but never
+// used as keys, so nothing in them reaches a valid row.
 rocs_status encoder_layer(rocs_context* ctx, const EncScratch& e, int B_R, int L, int d, int H,
                           const rocs_dca_layer_weights& w, const void* S_in, void* S_out, void* KR, void* VR, void* KC,
-                          void* VC, cudaStream_t s) {
+                          void* VC, cudaStream_t s, const int32_t* lengths = nullptr) {
   const long long M = (long long)B_R * L;
   GemmDesc g[4];
   const void* Ws[3] = {w.Wq, w.Wk, w.Wv};
@@ -614,7 +621,7 @@ rocs_status encoder_layer(rocs_context* ctx, const EncScratch& e, int B_R, int L
   ROCS_TRY(launch_gemm_bf16(ctx, g, 3, s));
   SiteLabel sl1("enc.attn");
   ROCS_TRY(attention_best(ctx, false, e.q, d, 0, e.k, e.v, d, e.self_off, B_R, M, L, H, d / H,
-                          1.0f / std::sqrt((float)(d / H)), e.att, d, 1, nullptr, 0, s));
+                          1.0f / std::sqrt((float)(d / H)), e.att, d, 1, nullptr, 0, s, lengths));
   SiteLabel sl2("enc.wo");
   ROCS_TRY(linear_bf16(ctx, e.att, d, M, d, w.Wo, d, nullptr, e.tmp, d, 1, ROCS_ACT_NONE, s));
   SiteLabel sl3("enc.ln");
@@ -643,7 +650,6 @@ rocs_status check_dca_desc(const rocs_dca_desc* d) {
   ROCS_REQUIRE(d->layers >= 1 && d->layers <= ROCS_MAX_LAYERS, "dca: layers=%d out of range", d->layers);
   const int dh = d->d / d->H;
   ROCS_REQUIRE(dh == 32 || dh == 64, "dca: head width %d (32 or 64 supported)", dh);
-  ROCS_REQUIRE((long long)d->L * dh <= 32768, "dca: L*d_h exceeds 32768");
   ROCS_REQUIRE(d->d % 8 == 0 && d->d <= 8192, "dca: d must be a multiple of 8");
   ROCS_REQUIRE((long long)d->B_R * d->L < 2147483647LL, "dca: B_R*L too large");
   return ROCS_OK;
@@ -662,8 +668,8 @@ extern "C" rocs_status rocs_dca_encode_workspace(rocs_handle_t h, const rocs_dca
 }
 
 extern "C" rocs_status rocs_dca_encode(rocs_handle_t h, const rocs_dca_desc* d, const void* Hist,
-                                       const rocs_dca_layer_weights* w, void* S, void* KV, void* ws, size_t ws_bytes,
-                                       void* stream) {
+                                       const int32_t* lengths, const rocs_dca_layer_weights* w, void* S, void* KV,
+                                       void* ws, size_t ws_bytes, void* stream) {
   CtxGuard ctx_guard_(h);
   ROCS_REQUIRE(h, "rocs_dca_encode: handle is NULL");
   ROCS_TRY(check_dca_desc(d));
@@ -688,7 +694,8 @@ extern "C" rocs_status rocs_dca_encode(rocs_handle_t h, const rocs_dca_desc* d, 
   for (int l = 0; l < d->layers; ++l) {
     char* Sl = (char*)S + per * l;
     char* kv = (char*)KV + per * 4 * l;
-    ROCS_TRY(encoder_layer(h, e, d->B_R, d->L, d->d, d->H, w[l], cur, Sl, kv, kv + per, kv + 2 * per, kv + 3 * per, s));
+    ROCS_TRY(encoder_layer(h, e, d->B_R, d->L, d->d, d->H, w[l], cur, Sl, kv, kv + per, kv + 2 * per, kv + 3 * per, s,
+                           lengths));
     cur = Sl;
   }
   return ROCS_OK;
@@ -926,7 +933,8 @@ rocs_status forward_launches(rocs_handle_t h, const rocs_model_desc* m, const ro
     if (dca_l) {
       const rocs_dca_layer_weights& dw = W->dca[l];
       void* S_l = out->S ? (void*)((char*)out->S + S_plane * l) : p.S[l & 1];
-      ROCS_TRY(encoder_layer(h, p.enc, BR, m->L, m->d, m->H, dw, S_prev, S_l, p.KR, p.VR, p.KC, p.VC, s));
+      ROCS_TRY(encoder_layer(h, p.enc, BR, m->L, m->d, m->H, dw, S_prev, S_l, p.KR, p.VR, p.KC, p.VC, s,
+                             in->hist_len));
       S_prev = S_l;
       // query generator: token LCB to one token per group (hi/lo), then the GLM-MLP
       const rocs_qgen_weights& qw = W->qgen[l];
@@ -981,15 +989,15 @@ rocs_status forward_launches(rocs_handle_t h, const rocs_model_desc* m, const ro
         SiteLabel s_xa("xattn.req");
         if (p.KR == nullptr)
           ROCS_TRY(launch_attention_req_absorbed(h, p.QR, d2, S_l, dw.WK_R, dw.WV_R, BR, m->L, m->d, m->H, scale, dR,
-                                                 ldR, xR2, xr, s));
+                                                 ldR, xR2, xr, s, in->hist_len));
         else
           ROCS_TRY(launch_attention_single(h, p.QR, d2, 1, p.KR, p.VR, m->d, (long long)m->L * m->d, p.iota1, BR, BR,
-                                           m->L, m->H, dh, scale, dR, ldR, 0, xR2, xr, s));
+                                           m->L, m->H, dh, scale, dR, ldR, 0, xR2, xr, s, in->hist_len));
       }
       {
         SiteLabel s_xc("xattn.cand");
         ROCS_TRY(attention_best(h, true, p.QC, d2, 1, p.KC, p.VC, m->d, offsets, BR, BC, m->L, m->H, dh, scale, dC,
-                                ldC, 0, xC2, xc, s));
+                                ldC, 0, xC2, xc, s, in->hist_len));
       }
       if (m->dca_query_source == 0) {
         if (out->A_R)

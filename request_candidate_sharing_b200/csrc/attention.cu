@@ -39,11 +39,11 @@ template <int DH, bool QSPLIT>
 __global__ void __launch_bounds__(ATT_THREADS, 1) attn_kernel(
     const __nv_bfloat16* __restrict__ Q, long long ldq, const __nv_bfloat16* __restrict__ K,
     const __nv_bfloat16* __restrict__ V, long long ldkv, long long kv_req_stride, const int32_t* __restrict__ offsets,
-    int B_R, long long rows, int L, int H, float scale_log2, void* O, long long ldo, int out_bf16,
-    __nv_bfloat16* __restrict__ O2, long long ldo2, int splits, int* status) {
+    int B_R, long long rows, int L_all, int H, float scale_log2, void* O, long long ldo, int out_bf16,
+    __nv_bfloat16* __restrict__ O2, long long ldo2, int splits, const int32_t* __restrict__ kv_len, int* status) {
   extern __shared__ __align__(16) uint8_t att_smem[];
   constexpr int PITCH = DH * 2 + 16;
-  const int Ls = (L + KB - 1) / KB * KB;
+  const int Ls = (L_all + KB - 1) / KB * KB;
   uint8_t* sK = att_smem;
   uint8_t* sV = att_smem + Ls * PITCH;
 
@@ -61,6 +61,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 1) attn_kernel(
   const long long ntiles = (q1 - q0 + 15) / 16;
   const long long t_begin = ntiles * sp / splits, t_end = ntiles * (sp + 1) / splits;
   if (t_begin >= t_end) return;
+  // this request's keys: the first L of its L_all K/V rows (a ragged history), L in [1, L_all]
+  const int L = kv_len != nullptr ? kv_len[r] : L_all;
+  if (L < 1 || L > L_all) {
+    if (threadIdx.x == 0) set_status(status, ROCS_ERR_COUNTS);
+    return;
+  }
 
   // ---- stage K and V of (r, h) once ----
   {
@@ -226,7 +232,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1) attn_kernel(
 rocs_status launch_attention(rocs_context* ctx, const void* Q, long long ldq, int q_split, const void* K,
                              const void* V, long long ldkv, long long kv_req_stride, const int32_t* offsets, int B_R,
                              long long rows, int L, int H, int d_h, float scale, void* O, long long ldo, int out_bf16,
-                             void* O2, long long ldo2, cudaStream_t s) {
+                             void* O2, long long ldo2, cudaStream_t s, const int32_t* kv_len) {
   if (B_R == 0 || rows == 0) return ROCS_OK;
   const int Ls = (L + KB - 1) / KB * KB;
   const int pitch = d_h * 2 + 16;
@@ -261,7 +267,7 @@ rocs_status launch_attention(rocs_context* ctx, const void* Q, long long ldq, in
 #define ROCS_ATT(DH, SPLIT)                                                                                         \
   attn_kernel<DH, SPLIT><<<(unsigned)grid, ATT_THREADS, smem, s>>>(                                                 \
       (const __nv_bfloat16*)Q, ldq, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, ldkv, kv_req_stride, offsets, \
-      B_R, rows, L, H, scale_log2, O, ldo, out_bf16, (__nv_bfloat16*)O2, ldo2, splits, ctx->d_status)
+      B_R, rows, L, H, scale_log2, O, ldo, out_bf16, (__nv_bfloat16*)O2, ldo2, splits, kv_len, ctx->d_status)
   LaunchTimer lt_("attn", s);
   switch (which) {
     case 0: ROCS_ATT(32, false); break;

@@ -38,8 +38,9 @@ constexpr int AR_KPITCH = AR_D + 8;        // bf16 elements per k' row (16-byte 
 
 __global__ void __launch_bounds__(AR_WARPS * 32) attn_req_absorbed_kernel(
     const __nv_bfloat16* __restrict__ Q, long long ldq, const __nv_bfloat16* __restrict__ S,
-    const __nv_bfloat16* __restrict__ WK, const __nv_bfloat16* __restrict__ WV, int L, int H, float scale_log2,
-    float* __restrict__ O, long long ldo, __nv_bfloat16* __restrict__ O2, long long ldo2) {
+    const __nv_bfloat16* __restrict__ WK, const __nv_bfloat16* __restrict__ WV, int L_all, int H, float scale_log2,
+    float* __restrict__ O, long long ldo, __nv_bfloat16* __restrict__ O2, long long ldo2,
+    const int32_t* __restrict__ kv_len, int* status) {
   constexpr int D = AR_D;
   __shared__ float q[D];
   __shared__ __align__(16) float kp[AR_MAX_H][D];
@@ -54,7 +55,13 @@ __global__ void __launch_bounds__(AR_WARPS * 32) attn_req_absorbed_kernel(
   const int r = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int dh = D / H;
-  const __nv_bfloat16* Sr = S + (long long)r * L * D;
+  const __nv_bfloat16* Sr = S + (long long)r * L_all * D;
+  // this request's rows: the first L of its L_all (a ragged history), L in [1, L_all]
+  const int L = kv_len != nullptr ? kv_len[r] : L_all;
+  if (L < 1 || L > L_all) {
+    if (tid == 0) set_status(status, ROCS_ERR_COUNTS);
+    return;
+  }
   uint8_t* tile = ar_dyn + warp * 32 * AR_PITCH;
 
   // 1. query (hi + lo) and k'_h[i] = sum_j q[h dh + j] W_K^R[h dh + j][i]
@@ -254,7 +261,8 @@ bool attention_req_absorbed_supported(int d, int H, int L) {
 
 rocs_status launch_attention_req_absorbed(rocs_context* ctx, const void* Q, long long ldq, const void* S,
                                           const void* WK, const void* WV, int B_R, int L, int d, int H, float scale,
-                                          float* O, long long ldo, void* O2, long long ldo2, cudaStream_t s) {
+                                          float* O, long long ldo, void* O2, long long ldo2, cudaStream_t s,
+                                          const int32_t* kv_len) {
   if (B_R == 0) return ROCS_OK;
   if (!attention_req_absorbed_supported(d, H, L) || ((uintptr_t)S & 15) || ((uintptr_t)WV & 15)) {
     set_error("request attention: unsupported d=%d H=%d L=%d", d, H, L);
@@ -273,7 +281,8 @@ rocs_status launch_attention_req_absorbed(rocs_context* ctx, const void* Q, long
   LaunchTimer lt_("attn_req", s);
   attn_req_absorbed_kernel<<<B_R, AR_WARPS * 32, smem, s>>>((const __nv_bfloat16*)Q, ldq, (const __nv_bfloat16*)S,
                                                          (const __nv_bfloat16*)WK, (const __nv_bfloat16*)WV, L, H,
-                                                         scale * 1.4426950408889634f, O, ldo, (__nv_bfloat16*)O2, ldo2);
+                                                         scale * 1.4426950408889634f, O, ldo, (__nv_bfloat16*)O2, ldo2,
+                                                         kv_len, ctx->d_status);
   return cuda_check(cudaGetLastError(), "attn_req_absorbed_kernel");
 }
 

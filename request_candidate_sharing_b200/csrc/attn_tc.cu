@@ -50,6 +50,7 @@ struct AttnTcParams {
   __nv_bfloat16* O2;
   long long ldo2;
   const int32_t* out_rows;   // optional: query row q is written to output row out_rows[q]
+  const int32_t* kv_len;     // optional: request r has kv_len[r] keys (1..L), the rest are padding
   int* status;
 };
 
@@ -182,7 +183,7 @@ struct AtCfg {
   static_assert(L_COL + (SUM_MMA ? GROUPS * 16 : 0) <= 512, "tensor memory columns");
 };
 
-template <int DH, bool SPLIT>
+template <int DH, bool SPLIT, bool RAGGED>
 __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __grid_constant__ AttnTcParams P) {
   using C = AtCfg<DH>;
   constexpr int GROUPS = C::GROUPS;
@@ -206,13 +207,21 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
   }
   const int ntiles = (int)((q1 - q0 + TQ - 1) / TQ);
   if (ntiles == 0) return;
-  const int nkb = P.nkb;
+  // this request's keys: the first Lr rows of its L-row K/V (a ragged history), Lr in [1, L];
+  // without per-request lengths (RAGGED false) every request has L keys
+  const int Lr = RAGGED ? P.kv_len[r] : P.L;
+  if (RAGGED && (Lr < 1 || Lr > P.L)) {
+    if (threadIdx.x == 0) set_status(P.status, ROCS_ERR_COUNTS);
+    return;
+  }
+  const int nkb = RAGGED ? (Lr + TK - 1) / TK : P.nkb;
+  const int tail_keys = nkb * TK - Lr;   // padding rows in the last staged key block
 
   extern __shared__ uint8_t at_smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(at_smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = base;
-  uint8_t* sV = sK + nkb * KV_BLOCK;
-  uint8_t* sQ = sV + nkb * KV_BLOCK;                  // [GROUPS][NQ][Q_TILE]
+  uint8_t* sV = sK + P.nkb * KV_BLOCK;
+  uint8_t* sQ = sV + P.nkb * KV_BLOCK;                // [GROUPS][NQ][Q_TILE]
   uint8_t* sOnes = sQ + GROUPS * NQ * Q_TILE;         // 1024-B aligned (Q tiles are 8 KiB multiples)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sOnes + ONES_BYTES);
   uint64_t* kv_full = bars;                           // [AT_MAX_KB]
@@ -223,8 +232,12 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
   uint64_t* p_full = s_free + GROUPS;                 // [GROUPS][2]: P half h of the block written
   uint64_t* o_full = p_full + 2 * GROUPS;             // [GROUPS][2]: P half h times V consumed
   uint64_t* drain = o_full + 2 * GROUPS;              // [GROUPS]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + GROUPS);
+  uint64_t* vtail = drain + GROUPS;                   // the last V block's rows past Lr are zeroed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(vtail + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // ragged: the request's key blocks and keys, re-read by the softmax warps where they need them
+  // (kept out of their registers; otherwise they read the launch parameters)
+  int* at_geom = reinterpret_cast<int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -240,6 +253,9 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
       }
       mbar_init(&drain[g], 1);
     }
+    mbar_init(vtail, 1);
+    at_geom[0] = nkb;
+    at_geom[1] = Lr;
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -285,6 +301,20 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
       for (int j = 0; j < nkb; ++j) mbar_wait(&kv_full[j], 0, P.status, nullptr);
       for (int t = last_t - GROUPS + 1 < 0 ? 0 : last_t - GROUPS + 1; t <= last_t; ++t)
         mbar_wait(&q_full[t % GROUPS], (t / GROUPS) & 1, P.status, nullptr);
+    } else if (warp == 3 && tail_keys > 0) {
+      // ---------------- the last key block's padding rows ----------------
+      // Keys past Lr have P = 0, but their V rows still enter the P V product, where any
+      // non-finite padding would give 0 * inf = NaN.  Once the block has landed, this warp zeroes
+      // those rows (whole rows: the swizzle permutes 16-byte units within a row) and releases the
+      // block for P V.
+      if (__all_sync(0xffffffffu, mbar_wait(&kv_full[nkb - 1], 0, P.status, abort_flag))) {
+        uint8_t* vb = sV + (nkb - 1) * KV_BLOCK + (TK - tail_keys) * ROWB;
+        for (int i = lane; i < tail_keys * ROWB / 16; i += 32)
+          reinterpret_cast<uint4*>(vb)[i] = make_uint4(0, 0, 0, 0);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
+        __syncwarp();
+        if (lane == 0) mbar_arrive(vtail);
+      }
     } else if (warp >= 1 && warp <= GROUPS && lane == 0) {
       // ---------------- MMA issuer of query-tile group g = warp - 1 ----------------
       // Per key block i:  S_i = Q K_j^T once the softmax has read S_{i-1} (s_free); then, for the
@@ -294,8 +324,9 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
       const int T = tiles_g(g) * nkb;
       auto issue_pv = [&](int ib, int hh) -> bool {
         if (!mbar_wait(&p_full[2 * g + hh], ib & 1, P.status, abort_flag)) return false;
-        tc_fence_after();
         const int j = ib % nkb;
+        if (j == nkb - 1 && tail_keys > 0 && !mbar_wait(vtail, 0, P.status, abort_flag)) return false;
+        tc_fence_after();
         const uint32_t va = smem_u32(sV + j * KV_BLOCK);
 #pragma unroll
         for (int kq = 0; kq < TK / 32; ++kq) {
@@ -346,7 +377,8 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
     const uint32_t paddr = lane_addr + C::P_COL + g * 64;
     const uint32_t oaddr = lane_addr + C::O_COL + g * DH;
     const uint32_t laddr = lane_addr + C::L_COL + g * 16;
-    const int Tg = tiles_g(g) * nkb;
+    volatile int* geom = at_geom;
+    const int Tg = tiles_g(g) * (RAGGED ? geom[0] : P.nkb);
     const float sl2 = P.scale_log2;
     float m_cur = -INFINITY, l_reg = 0.f;
 
@@ -396,7 +428,8 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
 
     bool ok = true;
     for (int i = 0; i < Tg; ++i) {
-      const int k_tile = i / nkb, j = i - k_tile * nkb;
+      const int nkb_i = RAGGED ? geom[0] : P.nkb;
+      const int k_tile = i / nkb_i, j = i - k_tile * nkb_i;
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[g], i & 1, P.status, abort_flag))) { ok = false; break; }
       tc_fence_after();
       // the whole S row into registers with one wait, then the S accumulator is released
@@ -406,7 +439,7 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&s_free[g]);
-      const int valid = P.L - j * TK;   // keys of this block that exist (>= 1)
+      const int valid = (RAGGED ? geom[1] : P.L) - j * TK;   // keys of this block that exist (>= 1)
       if (valid < TK) {
 #pragma unroll
         for (int c = 0; c < TK / 32; ++c)
@@ -515,7 +548,7 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
     if (ok && Tg > 0 && __all_sync(0xffffffffu, mbar_wait(&o_full[2 * g], (Tg - 1) & 1, P.status, abort_flag) &&
                                                mbar_wait(&o_full[2 * g + 1], (Tg - 1) & 1, P.status, abort_flag))) {
       tc_fence_after();
-      emit_row(Tg / nkb - 1);
+      emit_row(Tg / (RAGGED ? geom[0] : P.nkb) - 1);
     }
   }
 
@@ -532,7 +565,7 @@ template <int DH, bool SPLIT>
 size_t at_smem_bytes(int nkb) {
   constexpr int G = AtCfg<DH>::GROUPS;
   return 1024 + (size_t)2 * nkb * TK * DH * 2 + (size_t)G * (SPLIT ? 2 : 1) * TQ * DH * 2 + 2048 +
-         (AT_MAX_KB + 9 * G) * 8 + 16;
+         (AT_MAX_KB + 9 * G + 1) * 8 + 32;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -551,7 +584,7 @@ bool encode_rows(rocs_context* ctx, CUtensorMap* map, const void* ptr, long long
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int DH, bool SPLIT>
+template <int DH, bool SPLIT, bool RAGGED>
 rocs_status at_launch(rocs_context* ctx, AttnTcParams& P, int B_R, int H, cudaStream_t s) {
   const size_t smem = at_smem_bytes<DH, SPLIT>(P.nkb);
   if (smem > 232448) {
@@ -561,13 +594,13 @@ rocs_status at_launch(rocs_context* ctx, AttnTcParams& P, int B_R, int H, cudaSt
   static bool attr[64] = {false};
   if (ctx->device < 64 && !attr[ctx->device]) {
     rocs_status st = cuda_check(
-        cudaFuncSetAttribute(attn_tc_kernel<DH, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448),
+        cudaFuncSetAttribute(attn_tc_kernel<DH, SPLIT, RAGGED>, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448),
         "cudaFuncSetAttribute(attn_tc)");
     if (st != ROCS_OK) return st;
     // the softmax warpgroups raise their register limit out of the block's launch allocation;
     // refuse to launch if the compiled kernel was given fewer registers than that split needs
     cudaFuncAttributes fa;
-    st = cuda_check(cudaFuncGetAttributes(&fa, attn_tc_kernel<DH, SPLIT>), "cudaFuncGetAttributes(attn_tc)");
+    st = cuda_check(cudaFuncGetAttributes(&fa, attn_tc_kernel<DH, SPLIT, RAGGED>), "cudaFuncGetAttributes(attn_tc)");
     if (st != ROCS_OK) return st;
     using C = AtCfg<DH>;
     if (fa.numRegs < C::REG_LAUNCH) {
@@ -577,7 +610,7 @@ rocs_status at_launch(rocs_context* ctx, AttnTcParams& P, int B_R, int H, cudaSt
     }
     attr[ctx->device] = true;
   }
-  attn_tc_kernel<DH, SPLIT><<<(unsigned)((long long)B_R * H), AtCfg<DH>::THREADS, smem, s>>>(P);
+  attn_tc_kernel<DH, SPLIT, RAGGED><<<(unsigned)((long long)B_R * H), AtCfg<DH>::THREADS, smem, s>>>(P);
   return cuda_check(cudaGetLastError(), "attn_tc_kernel");
 }
 
@@ -586,7 +619,8 @@ rocs_status at_launch(rocs_context* ctx, AttnTcParams& P, int B_R, int H, cudaSt
 rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq, int q_split, const void* K,
                                 const void* V, long long ldkv, long long kv_rows, const int32_t* offsets, int B_R,
                                 long long rows, int L, int H, int d_h, float scale, void* O, long long ldo,
-                                int out_bf16, void* O2, long long ldo2, cudaStream_t s, const int32_t* out_rows) {
+                                int out_bf16, void* O2, long long ldo2, cudaStream_t s, const int32_t* out_rows,
+                                const int32_t* kv_len) {
   if (B_R == 0 || rows == 0) return ROCS_OK;
   if ((d_h != 32 && d_h != 64) || L < 1 || (long long)L * d_h > 32768 || (L + TK - 1) / TK > AT_MAX_KB ||
       ((uintptr_t)Q & 15) || ((uintptr_t)K & 15) || ((uintptr_t)V & 15) || ldq % 8 || ldkv % 8 ||
@@ -617,10 +651,16 @@ rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq,
   P.O2 = (__nv_bfloat16*)O2;
   P.ldo2 = ldo2;
   P.out_rows = out_rows;
+  P.kv_len = kv_len;
   P.status = ctx->d_status;
   LaunchTimer lt_("attn_tc", s);
-  if (d_h == 32) return q_split ? at_launch<32, true>(ctx, P, B_R, H, s) : at_launch<32, false>(ctx, P, B_R, H, s);
-  return q_split ? at_launch<64, true>(ctx, P, B_R, H, s) : at_launch<64, false>(ctx, P, B_R, H, s);
+  const bool rag = kv_len != nullptr;
+  if (d_h == 32) {
+    if (q_split) return rag ? at_launch<32, true, true>(ctx, P, B_R, H, s) : at_launch<32, true, false>(ctx, P, B_R, H, s);
+    return rag ? at_launch<32, false, true>(ctx, P, B_R, H, s) : at_launch<32, false, false>(ctx, P, B_R, H, s);
+  }
+  if (q_split) return rag ? at_launch<64, true, true>(ctx, P, B_R, H, s) : at_launch<64, true, false>(ctx, P, B_R, H, s);
+  return rag ? at_launch<64, false, true>(ctx, P, B_R, H, s) : at_launch<64, false, false>(ctx, P, B_R, H, s);
 }
 
 }  // namespace rocs

@@ -171,7 +171,7 @@ rocs_status launch_token_lcb(rocs_context* ctx, const void* E_R, long long ld_ER
 rocs_status launch_attention(rocs_context* ctx, const void* Q, long long ldq, int q_split, const void* K,
                              const void* V, long long ldkv, long long kv_req_stride, const int32_t* offsets, int B_R,
                              long long rows, int L, int H, int d_h, float scale, void* O, long long ldo,
-                             int out_bf16, void* O2, long long ldo2, cudaStream_t s);
+                             int out_bf16, void* O2, long long ldo2, cudaStream_t s, const int32_t* kv_len = nullptr);
 
 // Same contract as launch_attention.  _stream: K/V streamed through a small shared-memory ring
 // (any number of query rows per request); _single: one query row per request (a few at most),
@@ -179,11 +179,13 @@ rocs_status launch_attention(rocs_context* ctx, const void* Q, long long ldq, in
 rocs_status launch_attention_stream(rocs_context* ctx, const void* Q, long long ldq, int q_split, const void* K,
                                     const void* V, long long ldkv, long long kv_req_stride, const int32_t* offsets,
                                     int B_R, long long rows, int L, int H, int d_h, float scale, void* O,
-                                    long long ldo, int out_bf16, void* O2, long long ldo2, cudaStream_t s);
+                                    long long ldo, int out_bf16, void* O2, long long ldo2, cudaStream_t s,
+                                    const int32_t* kv_len = nullptr);
 rocs_status launch_attention_single(rocs_context* ctx, const void* Q, long long ldq, int q_split, const void* K,
                                     const void* V, long long ldkv, long long kv_req_stride, const int32_t* offsets,
                                     int B_R, long long rows, int L, int H, int d_h, float scale, void* O,
-                                    long long ldo, int out_bf16, void* O2, long long ldo2, cudaStream_t s);
+                                    long long ldo, int out_bf16, void* O2, long long ldo2, cudaStream_t s,
+                                    const int32_t* kv_len = nullptr);
 
 // tcgen05/TMEM attention (one CTA per (request, head), K/V resident in shared memory): d_h 32
 // (L <= 1024) or 64 (L <= 256 with hi/lo queries, 512 without).  kv_rows = rows of K/V (B_R * L).
@@ -193,12 +195,13 @@ rocs_status launch_attention_single(rocs_context* ctx, const void* Q, long long 
 bool attention_req_absorbed_supported(int d, int H, int L);
 rocs_status launch_attention_req_absorbed(rocs_context* ctx, const void* Q, long long ldq, const void* S,
                                           const void* WK, const void* WV, int B_R, int L, int d, int H, float scale,
-                                          float* O, long long ldo, void* O2, long long ldo2, cudaStream_t s);
+                                          float* O, long long ldo, void* O2, long long ldo2, cudaStream_t s,
+                                          const int32_t* kv_len = nullptr);
 rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq, int q_split, const void* K,
                                 const void* V, long long ldkv, long long kv_rows, const int32_t* offsets, int B_R,
                                 long long rows, int L, int H, int d_h, float scale, void* O, long long ldo,
                                 int out_bf16, void* O2, long long ldo2, cudaStream_t s,
-                                const int32_t* out_rows = nullptr);
+                                const int32_t* out_rows = nullptr, const int32_t* kv_len = nullptr);
 
 rocs_status launch_score_head(const void* X, long long ldx, long long rows, int K, const void* w,
                               const float* b, float* out, cudaStream_t s);

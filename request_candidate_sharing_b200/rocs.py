@@ -86,7 +86,7 @@ class ModelDesc(C.Structure):
 
 
 class Inputs(C.Structure):
-    _fields_ = [("counts", P), ("E_R", P), ("E_C", P), ("Hist", P), ("Y_R", P), ("Y_C", P)]
+    _fields_ = [("counts", P), ("E_R", P), ("E_C", P), ("Hist", P), ("Y_R", P), ("Y_C", P), ("hist_len", P)]
 
 
 class Outputs(C.Structure):
@@ -115,9 +115,9 @@ _lib_fm = _proto("rocs_fm_masked", P, P, P, P, I32, I64, I32, I32, I32, P, P, C.
 _lib_lcb_ws = _proto("rocs_token_lcb_workspace", P, I32, I32, I32, C.POINTER(C.c_size_t))
 _lib_lcb = _proto("rocs_token_lcb", P, P, P, P, I32, I64, I32, I32, I32, P, P, P, I32, I32, P, I64, P, I64, C.c_int,
                   P, C.c_size_t, P)
-_lib_attn = _proto("rocs_dca_cross_attn", P, P, P, P, P, I32, I64, I32, I32, I32, C.c_float, P, I64, C.c_int, P)
+_lib_attn = _proto("rocs_dca_cross_attn", P, P, P, P, P, I32, I64, I32, I32, I32, C.c_float, P, I64, C.c_int, P, P)
 _lib_enc_ws = _proto("rocs_dca_encode_workspace", P, C.POINTER(DcaDesc), C.POINTER(C.c_size_t))
-_lib_enc = _proto("rocs_dca_encode", P, C.POINTER(DcaDesc), P, C.POINTER(DcaLayerWeights), P, P, P, C.c_size_t, P)
+_lib_enc = _proto("rocs_dca_encode", P, C.POINTER(DcaDesc), P, P, C.POINTER(DcaLayerWeights), P, P, P, C.c_size_t, P)
 _lib_fwd_ws = _proto("rocs_forward_workspace", P, C.POINTER(ModelDesc), C.POINTER(C.c_size_t))
 _lib_fwd = _proto("rocs_forward", P, C.POINTER(ModelDesc), C.POINTER(ModelWeights), C.POINTER(Inputs),
                   C.POINTER(Outputs), P, C.c_size_t, P)
@@ -129,7 +129,7 @@ _lib_sort_ws = _proto("rocs_sort_by_request_workspace", P, I32, I64, C.POINTER(C
 _lib_sort = _proto("rocs_sort_by_request", P, P, I32, I64, P, P, P, C.c_size_t, P)
 _lib_xu_ws = _proto("rocs_dca_cross_attn_unsorted_workspace", P, I32, I64, I32, I32, C.c_int, C.POINTER(C.c_size_t))
 _lib_xu = _proto("rocs_dca_cross_attn_unsorted", P, P, P, P, P, I32, I64, I32, I32, I32, C.c_float, P, I64, C.c_int, P,
-                 C.c_size_t, P)
+                 P, C.c_size_t, P)
 _lib_tstart = _proto("rocs_timing_start", P, I32)
 _lib_tstop = _proto("rocs_timing_stop", P, C.c_char_p, C.c_size_t)
 
@@ -241,9 +241,11 @@ class Rocs:
                         int(workspace_bytes), stream))
 
     # -- a9 --
-    def rocs_dca_cross_attn(self, Q, K, V, offsets, B_R, rows, L, H, d_h, scale, O, ld_O, out, stream=None):
+    def rocs_dca_cross_attn(self, Q, K, V, offsets, B_R, rows, L, H, d_h, scale, O, ld_O, out, stream=None,
+                            kv_len=None):
+        """kv_len: per-request key counts (device int32 [B_R]) for ragged histories, or None."""
         _check(_lib_attn(self.h, ptr(Q), ptr(K), ptr(V), ptr(offsets), B_R, rows, L, H, d_h, float(scale), ptr(O),
-                         ld_O, out, stream))
+                         ld_O, out, ptr(kv_len), stream))
 
     # -- a7 --
     def rocs_dca_encode_workspace(self, desc: DcaDesc) -> int:
@@ -251,10 +253,12 @@ class Rocs:
         _check(_lib_enc_ws(self.h, C.byref(desc), C.byref(n)))
         return int(n.value)
 
-    def rocs_dca_encode(self, desc: DcaDesc, Hist, layer_weights, S, KV, workspace, workspace_bytes, stream=None):
+    def rocs_dca_encode(self, desc: DcaDesc, Hist, layer_weights, S, KV, workspace, workspace_bytes, stream=None,
+                        lengths=None):
+        """lengths: per-request history lengths (device int32 [B_R]) for ragged histories, or None."""
         arr = (DcaLayerWeights * len(layer_weights))(*layer_weights)
-        _check(_lib_enc(self.h, C.byref(desc), ptr(Hist), arr, ptr(S), ptr(KV), ptr(workspace), int(workspace_bytes),
-                        stream))
+        _check(_lib_enc(self.h, C.byref(desc), ptr(Hist), ptr(lengths), arr, ptr(S), ptr(KV), ptr(workspace),
+                        int(workspace_bytes), stream))
 
     # -- tracing --
     def rocs_timing_start(self, max_launches: int = 4096):
@@ -305,9 +309,10 @@ class Rocs:
 
     def rocs_dca_cross_attn_unsorted(self, Q, K, V, req_idx, B_R: int, rows: int, L: int, H: int, d_h: int,
                                      scale: float, O, ld_O: int, out: int, workspace, workspace_bytes: int,
-                                     stream=None):
+                                     stream=None, kv_len=None):
         _check(_lib_xu(self.h, ptr(Q), ptr(K), ptr(V), ptr(req_idx), int(B_R), int(rows), int(L), int(H), int(d_h),
-                       float(scale), ptr(O), int(ld_O), int(out), ptr(workspace), int(workspace_bytes), stream))
+                       float(scale), ptr(O), int(ld_O), int(out), ptr(kv_len), ptr(workspace), int(workspace_bytes),
+                       stream))
 
 
 # ---- marshalling helpers for the model structs (names follow the synth weight dictionaries) ----

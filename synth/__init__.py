@@ -111,6 +111,17 @@ def counts_uniform(seed: int, B_R: int, lo: int, hi: int) -> np.ndarray:
     return stream(seed, "counts", 0).integers(lo, hi + 1, size=B_R).astype(np.int32)
 
 
+def hist_lengths(seed: int, B_R: int, L: int, lo: int = 1) -> np.ndarray:
+    """Ragged history lengths: request r keeps its first lengths[r] of the L rows, uniform on
+    [lo, L] (both ends included), with the first request at L and the second at lo when there are
+    two or more, so both extremes always occur."""
+    g = stream(seed, "hist_len")
+    out = g.integers(lo, L + 1, size=B_R).astype(np.int32)
+    if B_R >= 2:
+        out[0], out[1] = L, lo
+    return out
+
+
 def counts_lognormal(seed: int, B_R: int, median: float, sigma: float, lo: int, hi: int) -> np.ndarray:
     """round(exp(N(ln median, sigma^2))) clipped to [lo, hi]; rounding is floor(x + 0.5)."""
     z = stream(seed, "counts", 0).standard_normal(B_R)

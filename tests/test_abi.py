@@ -94,10 +94,10 @@ def test_validation_errors_without_gpu(rocs):
     n2 = ctypes.c_size_t(0)
     assert rocs._lib_ikbo_ws(h, ctypes.byref(odd), ctypes.byref(n2)) == rocs.ROCS_OK
     assert n2.value > n.value
-    # attention limits
-    st = rocs._lib_attn(h, 16, 16, 16, 16, 1, 1, 4096, 1, 64, 0.125, 16, 64, 1, None)
-    assert st == rocs.ROCS_ERR_INVALID_ARG and "32768" in rocs.rocs_last_error()
-    st = rocs._lib_attn(h, 16, 16, 16, 16, 1, 1, 16, 1, 48, 0.125, 16, 64, 1, None)
+    # attention limits (long histories are accepted: they stream through shared memory)
+    st = rocs._lib_attn(h, 16, 16, 16, 16, 1 << 20, 1, 4096, 1, 64, 0.125, 16, 64, 1, None, None)
+    assert st == rocs.ROCS_ERR_INVALID_ARG and "too large" in rocs.rocs_last_error()
+    st = rocs._lib_attn(h, 16, 16, 16, 16, 1, 1, 16, 1, 48, 0.125, 16, 64, 1, None, None)
     assert st == rocs.ROCS_ERR_INVALID_ARG
     # FM limits
     st = rocs._lib_fm(h, 16, 16, 16, 1, 1, 60, 16, 128, 16, 16, 1, None)

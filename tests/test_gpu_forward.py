@@ -30,11 +30,13 @@ def run_forward(R, case, x, W):
     g, a = case.glm, case.dca
     mw = rocs.model_weights(Wd, g.layers if g else 0, a.layers if a else 0, case.scoring is not None)
     keep = dict(W=Wd)
-    xin = {k: dev(v) for k, v in x.items()}
+    xin = {k: dev(v) for k, v in x.items() if k != "hist_len"}
     keep["x"] = xin
     counts = dev_i32(case.counts)
+    hl = dev_i32(x["hist_len"]) if "hist_len" in x else None
+    keep["hist_len"] = hl
     inp = rocs.Inputs(counts.data_ptr(), rocs.ptr(xin.get("E_R")), rocs.ptr(xin.get("E_C")),
-                      rocs.ptr(xin.get("H")), rocs.ptr(xin.get("Y_R")), rocs.ptr(xin.get("Y_C")))
+                      rocs.ptr(xin.get("H")), rocs.ptr(xin.get("Y_R")), rocs.ptr(xin.get("Y_C")), rocs.ptr(hl))
     B_R, B_C = case.B_R, case.B_C
     out = {"offsets": torch.empty(B_R + 1, dtype=torch.int32, device="cuda"),
            "req_idx": torch.empty(max(B_C, 1), dtype=torch.int32, device="cuda")}
@@ -190,6 +192,26 @@ def test_forward_fused_ikbo_matches_two_launches(R):
         R.rocs_set_ikbo_fused(1)
     for k in ("score", "E_R", "E_C", "A_R", "A_C"):
         assert torch.equal(out0[k], out1[k]), k
+
+
+def test_forward_end_to_end_ragged_history(R):
+    """Histories of different lengths inside the padded [B_R, L, d] input (hist_len): the encoder,
+    the request and candidate cross-attention all stop at each request's length; padding rows
+    hold NaN, so a leak would show in the scores."""
+    case = synth.model_cfg5(B_R=4, counts=[4, 1, 20, 7], L=512)
+    x, W = synth.model_inputs(case), synth.model_weights(case)
+    x = dict(x, hist_len=np.asarray([512, 1, 300, 129], np.int32))
+    xn = dict(x)
+    xn["H"] = x["H"].copy()
+    for r, Lr in enumerate(x["hist_len"]):
+        xn["H"][r, Lr:] = np.nan
+    out = run_forward(R, case, xn, W)
+    _, m = O.segments(case.counts)
+    ref = O.forward_cfg5(case, x, W, m)
+    check_bf16(host(out["score"][:case.B_C]), ref["score"], what="score")
+    for l in range(case.dca.layers):
+        check_bf16(host(out["A_R"][l]), ref["A_R"][l], what=f"A_R_{l}")
+        check_bf16(host(out["A_C"][l]), ref["A_C"][l], what=f"A_C_{l}")
 
 
 def test_forward_end_to_end_long_history(R):

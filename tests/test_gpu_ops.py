@@ -350,6 +350,49 @@ def test_cross_attention(R, L, H, dh, counts):
     check_bf16(host(Ot[:n]), ref, what="cross-attention")
 
 
+@pytest.mark.parametrize("L,H,dh,counts,ragged", [
+    (1024, 8, 32, [33, 1, 0, 300, 129], True),     # staged K/V (tcgen05), ragged key counts
+    (200, 4, 64, [3, 0, 40, 17], True),            # staged, d_h 64
+    (1536, 8, 32, [70, 5, 200], True),             # L d_h = 49152: streamed through shared memory
+    (2048, 4, 64, [9, 130], False),                # long history, every key valid
+])
+def test_cross_attention_ragged_and_long(R, L, H, dh, counts, ragged):
+    """Per-request key counts (a ragged history: keys past kv_len[r] are padding, here filled with
+    large values that would dominate any softmax they entered) and histories longer than the
+    staged kernel holds, against the oracle on the truncated histories."""
+    counts = np.asarray(counts, np.int32)
+    off, m = O.segments(counts)
+    B_R, n, d = len(counts), int(counts.sum()), H * dh
+    g = np.random.default_rng(L + n + 7)
+    K = synth.bf16_round(g.standard_normal((B_R, L, d)).astype(np.float32))
+    V = synth.bf16_round(g.standard_normal((B_R, L, d)).astype(np.float32))
+    Q = synth.bf16_round(g.standard_normal((n, d)).astype(np.float32))
+    kv_len = synth.hist_lengths(L, B_R, L, 1) if ragged else None
+    if ragged:
+        for r in range(B_R):
+            K[r, kv_len[r]:] = 64.0
+            V[r, kv_len[r]:] = 1e4
+    Ot = torch.full((max(n, 1), d), float("nan"), device="cuda")
+    R.rocs_dca_cross_attn(dev(Q), dev(K), dev(V), dev_i32(off), B_R, n, L, H, dh, 1.0 / math.sqrt(dh), Ot, d, 0,
+                          stream(), kv_len=dev_i32(kv_len) if ragged else None)
+    _status_ok(R)
+    ref = O.cross_attn(Q, K, V, m, H, kv_len=kv_len)
+    check_bf16(host(Ot[:n]), ref, what="ragged/long cross-attention")
+
+
+def test_cross_attention_bad_length_sets_status(R):
+    from request_candidate_sharing_b200 import rocs
+    B_R, L, H, dh = 2, 256, 8, 32
+    d = H * dh
+    off = np.asarray([0, 4, 9], np.int32)
+    z = dev(np.zeros((B_R, L, d), np.float32))
+    Ot = torch.full((9, d), -2.0, device="cuda")
+    R.rocs_dca_cross_attn(dev(np.ones((9, d), np.float32)), z, z, dev_i32(off), B_R, 9, L, H, dh, 0.1, Ot, d, 0,
+                          stream(), kv_len=dev_i32(np.asarray([L + 1, 5], np.int32)))
+    assert R.rocs_get_device_status(stream()) == rocs.ROCS_ERR_COUNTS
+    assert torch.all(Ot[:4] == -2.0) and not torch.all(Ot[4:] == -2.0)
+
+
 # ---------------------------------------------------------------------------------------------
 # candidates in any order: stable sort by request, and the cross-attention over it
 # ---------------------------------------------------------------------------------------------
@@ -463,6 +506,38 @@ def test_cross_attention_unsorted_bad_index_rows_untouched(R):
 # ---------------------------------------------------------------------------------------------
 # a7 DCA encoder
 # ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("L,lengths", [(256, [256, 1, 100]), (1536, [1536, 700])])
+def test_dca_encode_ragged_and_long(R, L, lengths):
+    """Ragged histories (each request keeps its first lengths[r] rows; the padding rows hold NaN,
+    so a leak into any history row would show) and a history longer than the staged attention
+    kernels hold (streamed).  History rows of S and K/V against the oracle."""
+    from request_candidate_sharing_b200 import rocs
+    lengths = np.asarray(lengths, np.int32)
+    case = synth.model_cfg4(B_R=len(lengths), counts=[1] * len(lengths))
+    case.dca.L = L
+    a = case.dca
+    W = synth.model_weights(case)
+    x = synth.model_inputs(case)
+    Hn = x["H"].copy()
+    for r, Lr in enumerate(lengths):
+        Hn[r, Lr:] = np.nan
+    Wd = {k: dev(v, torch.float32 if ("ln." in k) else torch.bfloat16) for k, v in W.items()}
+    desc = rocs.DcaDesc(case.B_R, a.L, a.d, a.H, a.layers)
+    nb = R.rocs_dca_encode_workspace(desc)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    S = torch.empty((a.layers, case.B_R, a.L, a.d), dtype=torch.bfloat16, device="cuda")
+    KV = torch.empty((a.layers, 4, case.B_R, a.L, a.d), dtype=torch.bfloat16, device="cuda")
+    R.rocs_dca_encode(desc, dev(Hn), [rocs.dca_layer_weights(Wd, l) for l in range(a.layers)], S, KV, ws, nb,
+                      stream(), lengths=dev_i32(lengths))
+    _status_ok(R)
+    Ss, KVs = O.dca_encode(x["H"], W, a.layers, a.H, lengths)
+    for l in range(a.layers):
+        for r, Lr in enumerate(lengths):
+            check_bf16(host(S[l, r, :Lr]), Ss[l][r, :Lr], out_bf16=True, what=f"S_{l} request {r}")
+            for i in range(4):
+                check_bf16(host(KV[l, i, r, :Lr]), KVs[l][i][r, :Lr], out_bf16=True, what=f"KV_{l}_{i} request {r}")
+
+
 def test_dca_encode(R):
     from request_candidate_sharing_b200 import rocs
     case = synth.model_cfg4(B_R=3, counts=[1, 1, 1])

@@ -295,6 +295,49 @@ def test_encoder_layer_matches_torch_mha():
     np.testing.assert_allclose(out, ref, rtol=1e-11, atol=1e-11)
 
 
+def test_ragged_history_is_the_truncated_history():
+    """A ragged history (request r keeps its first lengths[r] rows) pinned three ways, each a
+    statement the padded layout must satisfy: (1) lengths = L gives the unragged result; (2) the
+    padding rows' contents never reach a history row or a query; (3) each request equals that
+    request encoded and attended on its own, on a history cut to its length."""
+    case = synth.model_cfg4(B_R=3, counts=[2, 3, 1])
+    case.dca.L = 10
+    a = case.dca
+    W = synth.model_weights(case)
+    x = synth.model_inputs(case)
+    lengths = np.asarray([10, 4, 1], np.int32)
+    _, m = O.segments(case.counts)
+    # (1)
+    full = O.forward_cfg4(case, x, W, m)
+    same = O.forward_cfg4(case, dict(x, hist_len=np.full(3, 10, np.int32)), W, m)
+    for k in ("A_R", "A_C", "S"):
+        for u, v in zip(full[k], same[k]):
+            np.testing.assert_allclose(u, v, rtol=1e-12, atol=1e-12)
+    # (2)
+    rag = O.forward_cfg4(case, dict(x, hist_len=lengths), W, m)
+    H2 = x["H"].copy()
+    for r, Lr in enumerate(lengths):
+        H2[r, Lr:] = 1e3
+    rag2 = O.forward_cfg4(case, dict(x, H=H2, hist_len=lengths), W, m)
+    for k in ("A_R", "A_C"):
+        for u, v in zip(rag[k], rag2[k]):
+            assert np.array_equal(u, v)
+    for l in range(a.layers):
+        for r, Lr in enumerate(lengths):
+            assert np.array_equal(rag["S"][l][r, :Lr], rag2["S"][l][r, :Lr])
+            assert np.isnan(rag["S"][l][r, Lr:]).all()
+    # (3) request 1 alone, on a history of 4 rows
+    Ss, KVs = O.dca_encode(x["H"][1:2, :4], W, a.layers, a.H)
+    for l in range(a.layers):
+        np.testing.assert_allclose(rag["S"][l][1, :4], Ss[l][0], rtol=1e-12, atol=1e-12)
+    q = np.random.default_rng(2).standard_normal((5, a.d))
+    owner = np.ones(5, np.int64)
+    K_C, V_C = KVs[0][2], KVs[0][3]
+    Sf, KVf = O.dca_encode(x["H"], W, a.layers, a.H, lengths)
+    np.testing.assert_allclose(O.cross_attn(q, KVf[0][2], KVf[0][3], owner, a.H, kv_len=lengths),
+                               O.cross_attn(q, K_C, V_C, np.zeros(5, np.int64), a.H), rtol=1e-12, atol=1e-12)
+
+
 # ---------------------------------------------------------------------------------------------
 # composition closure and invariants on the model configs (reduced sizes)
 # ---------------------------------------------------------------------------------------------
