@@ -46,6 +46,8 @@ WORKLOADS = {
     "rocs_forward_e2e": "end-to-end ranking forward: GLM stack (3 layers, 32|16 embeddings of 128) + DCA "
                         "(L=1024, d=256, 8 heads, 3 depths) + scoring MLP 512-256-1; 512 requests, "
                         "candidates ~ clipped lognormal (median 300, 16..2000), seed 1",
+    "rocs_forward_ragged": "the end-to-end ranking forward with ragged histories: request r's history is its first "
+                           "hist_len[r] of the L=1024 rows, hist_len ~ U[256, 1024] (seed 1), padding rows hold zeros",
     "glm_stack": "Wukong-style GLM stack, 3 layers; 64 requests, candidates ~ U[100,1000], seed 0",
     "dca": "DCA path: L=200, d=256, 4 heads, 2 layers; 32 requests x 500 candidates, seed 0",
     "ikbo_sweep": "IKBO linear sweep: B_R=256, N in {64, 256, 1024} candidates per request, d_in = d_out = d in "
@@ -62,6 +64,8 @@ def make_case(name: str, rank: int, requests: int = 0):
     seed_shift = 1000 * rank
     if name == "rocs_forward_e2e":
         case = synth.model_cfg5(seed=1 + seed_shift)
+    elif name == "rocs_forward_ragged":
+        case = dataclasses.replace(synth.model_cfg5(seed=1 + seed_shift), name="cfg5_ragged")
     elif name == "glm_stack":
         case = synth.model_cfg3(seed=0 + seed_shift)
     elif name == "dca":
@@ -110,23 +114,31 @@ def algo_work(case, label: str):
             return table[label]
     if a is not None:
         L, d, H = a.L, a.d, a.H
+        # history rows that exist (a ragged workload counts each request's own length: the rows
+        # the row-wise kernels spend on padding are no algorithmic work)
+        hl = hist_len_of(case)
+        hl = np.full(B_R, L, np.int64) if hl is None else np.asarray(hl[:B_R], np.int64)
+        rows_h = float(hl.sum())                                   # history tokens
+        pairs = float((hl * hl).sum())                             # self-attention (query, key) pairs
+        cand_keys = float((np.asarray(case.counts, np.int64) * hl).sum())   # candidate (query, key) pairs
         table = {
-            "enc.attn:attn": ("alu", float(B_R) * H * L * L),
-            "enc.attn:attn_tc": ("alu", float(B_R) * H * L * L),
-            "xattn.cand:attn_stream": ("alu", float(B_C) * H * L),
-            "xattn.cand:attn_tc": ("alu", float(B_C) * H * L),
-            "enc.qkv:gemm_tc": ("tensor", 2.0 * B_R * L * d * d * 3),
+            "enc.attn:attn": ("alu", H * pairs),
+            "enc.attn:attn_tc": ("alu", H * pairs),
+            "enc.attn:attn_stream": ("alu", H * pairs),
+            "xattn.cand:attn_stream": ("alu", H * cand_keys),
+            "xattn.cand:attn_tc": ("alu", H * cand_keys),
+            "enc.qkv:gemm_tc": ("tensor", 2.0 * rows_h * d * d * 3),
             # the candidate group's K/V only when the request query's attention absorbs its
             # projections (d = 256, up to 8 heads of a multiple of 16), else all four
-            "enc.kv:gemm_tc": ("tensor", 2.0 * B_R * L * d * d * (2 if (d == 256 and H <= 8 and (d // H) % 16 == 0) else 4)),
-            "enc.wo:gemm_tc": ("tensor", 2.0 * B_R * L * d * d),
-            "enc.ln:layernorm": ("hbm", B_R * L * d * 2 * 3.0),
+            "enc.kv:gemm_tc": ("tensor", 2.0 * rows_h * d * d * (2 if (d == 256 and H <= 8 and (d // H) % 16 == 0) else 4)),
+            "enc.wo:gemm_tc": ("tensor", 2.0 * rows_h * d * d),
+            "enc.ln:layernorm": ("hbm", rows_h * d * 2 * 3.0),
             # query generator, two IKBO linears q_dim -> d -> d (fused launches: request + candidate)
             "qgen.mlp1.ikbo:gemm_tc": ("tensor", 2.0 * (B_C + 2 * B_R) * d * a.q_dim),
             "qgen.mlp2.ikbo:gemm_tc": ("tensor", 2.0 * (B_C + 2 * B_R) * d * d),
             # the request query's attention with its projections absorbed reads the final
             # encoder output S once (bf16); weights and queries are L2-resident and negligible
-            "xattn.req:attn_req": ("hbm", float(B_R) * L * d * 2),
+            "xattn.req:attn_req": ("hbm", rows_h * d * 2),
         }
         if label in table:
             return table[label]
@@ -236,6 +248,28 @@ def blas_threads() -> int:
     return len(os.sched_getaffinity(0))
 
 
+def hist_len_of(case):
+    """Per-request history lengths of a ragged workload (None otherwise)."""
+    if not case.name.endswith("_ragged"):
+        return None
+    return synth.hist_lengths(case.seed, case.B_R, case.dca.L, case.dca.L // 4)
+
+
+def ragged_inputs(case, x, req_ids=None):
+    """Adds the ragged workload's lengths to the inputs and zeroes the padding rows of H."""
+    hl = hist_len_of(case)
+    if hl is None:
+        return x
+    if req_ids is not None:
+        hl = hl[np.asarray(req_ids, np.int64)]
+    x = dict(x, hist_len=hl)
+    H = x["H"].copy()
+    for r, Lr in enumerate(hl):
+        H[r, Lr:] = 0.0
+    x["H"] = H
+    return x
+
+
 def oracle_requests(case, req_ids):
     """Runs the oracle on whole requests `req_ids` of the workload; returns candidates processed."""
     from oracle import rocs_oracle as O
@@ -245,7 +279,7 @@ def oracle_requests(case, req_ids):
     cand_rows = np.concatenate([np.arange(offsets[r], offsets[r + 1]) for r in req_ids]) if len(req_ids) else \
         np.zeros(0, np.int64)
     sub = dataclasses.replace(case, counts=counts[req_ids])
-    x = synth.model_inputs(case, cand_rows=cand_rows, req_rows=req_ids)
+    x = ragged_inputs(case, synth.model_inputs(case, cand_rows=cand_rows, req_rows=req_ids), req_ids)
     W = synth.model_weights(case)
     _, m = O.segments(sub.counts)
     if case.scoring is not None:
@@ -327,7 +361,8 @@ def run_librocs(args, rank, world, local):
     dev = torch.device("cuda", local)
     t_gen = time.perf_counter()
     W = synth.model_weights(case)
-    x = synth.model_inputs(case)
+    x = ragged_inputs(case, synth.model_inputs(case))
+    hist_len = x.pop("hist_len", None)
     gen_s = time.perf_counter() - t_gen
 
     def to_dev(v, dt):
@@ -336,6 +371,7 @@ def run_librocs(args, rank, world, local):
     Wd = {k: to_dev(v, torch.float32 if k.endswith(FP32_KEYS) else torch.bfloat16) for k, v in W.items()}
     xd = {k: to_dev(v, torch.bfloat16) for k, v in x.items()}
     counts_d = torch.from_numpy(case.counts).to(dev)
+    hl_d = torch.from_numpy(np.ascontiguousarray(hist_len, np.int32)).to(dev) if hist_len is not None else None
     g, a = case.glm, case.dca
     R = rocs.Rocs(local)
     R.rocs_set_ikbo_fused(args.ikbo_fused)
@@ -362,7 +398,7 @@ def run_librocs(args, rank, world, local):
         return rocs.Outputs(None, None, None, None, None, outE[0].data_ptr(), outE[1].data_ptr(), None)
 
     inp = rocs.Inputs(counts_d.data_ptr(), rocs.ptr(xd.get("E_R")), rocs.ptr(xd.get("E_C")), rocs.ptr(xd.get("H")),
-                      rocs.ptr(xd.get("Y_R")), rocs.ptr(xd.get("Y_C")))
+                      rocs.ptr(xd.get("Y_R")), rocs.ptr(xd.get("Y_C")), rocs.ptr(hl_d))
     out = outputs()
     stream = torch.cuda.current_stream(dev)
     sh = stream.cuda_stream
@@ -429,8 +465,10 @@ def run_librocs(args, rank, world, local):
     # ---- end-to-end through the same call with host buffers ----
     host = {k: v.cpu().pin_memory() for k, v in xd.items()}
     counts_h = counts_d.cpu().pin_memory()
+    hl_h = hl_d.cpu().pin_memory() if hl_d is not None else None
     score_h = torch.empty_like(score, device="cpu").pin_memory()
-    h2d = sum(v.numel() * v.element_size() for v in host.values()) + counts_h.numel() * 4
+    h2d = sum(v.numel() * v.element_size() for v in host.values()) + counts_h.numel() * 4 + \
+        (hl_h.numel() * 4 if hl_h is not None else 0)
     res = score if case.scoring is not None else outE[1]
     res_h = torch.empty_like(res, device="cpu").pin_memory()
     d2h = res.numel() * res.element_size()
@@ -438,23 +476,26 @@ def run_librocs(args, rank, world, local):
     # two device input sets: step k+1's inputs are copied (copy stream) while step k computes;
     # every step's inputs still cross PCIe inside the timed region, and each set has its own
     # captured forward graph
-    sets = [(xd, counts_d, inp)]
+    sets = [(xd, counts_d, inp, hl_d)]
     xd2 = {k: torch.empty_like(v) for k, v in xd.items()}
     counts_d2 = torch.empty_like(counts_d)
+    hl_d2 = torch.empty_like(hl_d) if hl_d is not None else None
     inp2 = rocs.Inputs(counts_d2.data_ptr(), rocs.ptr(xd2.get("E_R")), rocs.ptr(xd2.get("E_C")),
-                       rocs.ptr(xd2.get("H")), rocs.ptr(xd2.get("Y_R")), rocs.ptr(xd2.get("Y_C")))
-    sets.append((xd2, counts_d2, inp2))
+                       rocs.ptr(xd2.get("H")), rocs.ptr(xd2.get("Y_R")), rocs.ptr(xd2.get("Y_C")), rocs.ptr(hl_d2))
+    sets.append((xd2, counts_d2, inp2, hl_d2))
     copy_stream = torch.cuda.Stream(dev)
     copied = [torch.cuda.Event(), torch.cuda.Event()]
     done = [torch.cuda.Event(), torch.cuda.Event()]
 
     def h2d_into(k):
-        xs, cs, _ = sets[k % 2]
+        xs, cs, _, hs = sets[k % 2]
         with torch.cuda.stream(copy_stream):
             copy_stream.wait_event(done[k % 2])     # the forward that last read this set is finished
             for name, v in host.items():
                 xs[name].copy_(v, non_blocking=True)
             cs.copy_(counts_h, non_blocking=True)
+            if hs is not None:
+                hs.copy_(hl_h, non_blocking=True)
             copied[k % 2].record(copy_stream)
 
     def forward_on(k):

@@ -162,22 +162,24 @@ rocs_status linear_bf16(rocs_context* ctx, const void* X, long long ldx, long lo
 
 // Attention against per-request K/V: the tcgen05 kernel where its shared memory holds the
 // request's K/V, else the streaming (cross) or resident (self) mma.sync kernels.
-// kv_len (nullable): request r's keys are the first kv_len[r] of its L rows (a ragged history).
-// Histories too long to stage in shared memory take the streaming kernel.
+// kv_len (nullable): request r's keys are the first kv_len[r] of its L rows (a ragged history);
+// q_by_kv: its query rows too (a self-attention over the ragged history).  Histories too long to
+// stage in shared memory take the streaming kernel.
 rocs_status attention_best(rocs_context* ctx, bool streaming_fallback, const void* Q, long long ldq, int q_split,
                            const void* K, const void* V, long long ldkv, const int32_t* offsets, int B_R,
                            long long rows, int L, int H, int d_h, float scale, void* O, long long ldo, int out_bf16,
-                           void* O2, long long ldo2, cudaStream_t s, const int32_t* kv_len = nullptr) {
+                           void* O2, long long ldo2, cudaStream_t s, const int32_t* kv_len = nullptr,
+                           int q_by_kv = 0) {
   rocs_status st = launch_attention_tc(ctx, Q, ldq, q_split, K, V, ldkv, (long long)B_R * L, offsets, B_R, rows, L, H,
-                                       d_h, scale, O, ldo, out_bf16, O2, ldo2, s, nullptr, kv_len);
+                                       d_h, scale, O, ldo, out_bf16, O2, ldo2, s, nullptr, kv_len, q_by_kv);
   if (st != ROCS_ERR_UNSUPPORTED) return st;
   if (!streaming_fallback) {
     st = launch_attention(ctx, Q, ldq, q_split, K, V, ldkv, (long long)L * ldkv, offsets, B_R, rows, L, H, d_h, scale,
-                          O, ldo, out_bf16, O2, ldo2, s, kv_len);
+                          O, ldo, out_bf16, O2, ldo2, s, kv_len, q_by_kv);
     if (st != ROCS_ERR_UNSUPPORTED) return st;
   }
   return launch_attention_stream(ctx, Q, ldq, q_split, K, V, ldkv, (long long)L * ldkv, offsets, B_R, rows, L, H,
-                                 d_h, scale, O, ldo, out_bf16, O2, ldo2, s, kv_len);
+                                 d_h, scale, O, ldo, out_bf16, O2, ldo2, s, kv_len, q_by_kv);
 }
 
 // Workspace of rocs_linear_ikbo: Z, then (only if a row is not 16-B aligned) padded operands.
@@ -602,8 +604,9 @@ EncScratch carve_encoder(Carver& c, long long rowsL, int d, int B_R) {
 
 // One encoder layer S_out = LN(S_in + MHSA(S_in) W_O^T) and the four K/V projections of S_out.
 // lengths (nullable): request r's history is its first lengths[r] rows; the rows after them are
-// padding, computed like any row (each row's LayerNorm and projections are independent) but never
-// used as keys, so nothing in them reaches a valid row.
+// padding, computed like any row by the row-wise steps (each row's LayerNorm and projections are
+// independent) but neither keys nor queries of the self-attention, so nothing in them reaches a
+// history row.  Their attention output is left as the workspace holds it.
 rocs_status encoder_layer(rocs_context* ctx, const EncScratch& e, int B_R, int L, int d, int H,
                           const rocs_dca_layer_weights& w, const void* S_in, void* S_out, void* KR, void* VR, void* KC,
                           void* VC, cudaStream_t s, const int32_t* lengths = nullptr) {
@@ -621,7 +624,7 @@ rocs_status encoder_layer(rocs_context* ctx, const EncScratch& e, int B_R, int L
   ROCS_TRY(launch_gemm_bf16(ctx, g, 3, s));
   SiteLabel sl1("enc.attn");
   ROCS_TRY(attention_best(ctx, false, e.q, d, 0, e.k, e.v, d, e.self_off, B_R, M, L, H, d / H,
-                          1.0f / std::sqrt((float)(d / H)), e.att, d, 1, nullptr, 0, s, lengths));
+                          1.0f / std::sqrt((float)(d / H)), e.att, d, 1, nullptr, 0, s, lengths, 1));
   SiteLabel sl2("enc.wo");
   ROCS_TRY(linear_bf16(ctx, e.att, d, M, d, w.Wo, d, nullptr, e.tmp, d, 1, ROCS_ACT_NONE, s));
   SiteLabel sl3("enc.ln");

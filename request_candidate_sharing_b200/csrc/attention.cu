@@ -40,7 +40,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1) attn_kernel(
     const __nv_bfloat16* __restrict__ Q, long long ldq, const __nv_bfloat16* __restrict__ K,
     const __nv_bfloat16* __restrict__ V, long long ldkv, long long kv_req_stride, const int32_t* __restrict__ offsets,
     int B_R, long long rows, int L_all, int H, float scale_log2, void* O, long long ldo, int out_bf16,
-    __nv_bfloat16* __restrict__ O2, long long ldo2, int splits, const int32_t* __restrict__ kv_len, int* status) {
+    __nv_bfloat16* __restrict__ O2, long long ldo2, int splits, const int32_t* __restrict__ kv_len, int q_by_kv,
+    int* status) {
   extern __shared__ __align__(16) uint8_t att_smem[];
   constexpr int PITCH = DH * 2 + 16;
   const int Ls = (L_all + KB - 1) / KB * KB;
@@ -53,20 +54,22 @@ __global__ void __launch_bounds__(ATT_THREADS, 1) attn_kernel(
   const int h = rem / splits;
   const int sp = rem - h * splits;
   if (r >= B_R) return;
-  const long long q0 = offsets[r], q1 = offsets[r + 1];
+  const long long q0 = offsets[r];
+  long long q1 = offsets[r + 1];
   if (q0 < 0 || q1 < q0 || q1 > rows) {
     if (threadIdx.x == 0) set_status(status, ROCS_ERR_INDEX);
     return;
   }
-  const long long ntiles = (q1 - q0 + 15) / 16;
-  const long long t_begin = ntiles * sp / splits, t_end = ntiles * (sp + 1) / splits;
-  if (t_begin >= t_end) return;
   // this request's keys: the first L of its L_all K/V rows (a ragged history), L in [1, L_all]
   const int L = kv_len != nullptr ? kv_len[r] : L_all;
   if (L < 1 || L > L_all) {
     if (threadIdx.x == 0) set_status(status, ROCS_ERR_COUNTS);
     return;
   }
+  if (kv_len != nullptr && q_by_kv) q1 = min(q1, q0 + L);   // ragged self-attention: padding rows ask nothing
+  const long long ntiles = (q1 - q0 + 15) / 16;
+  const long long t_begin = ntiles * sp / splits, t_end = ntiles * (sp + 1) / splits;
+  if (t_begin >= t_end) return;
 
   // ---- stage K and V of (r, h) once ----
   {
@@ -232,7 +235,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1) attn_kernel(
 rocs_status launch_attention(rocs_context* ctx, const void* Q, long long ldq, int q_split, const void* K,
                              const void* V, long long ldkv, long long kv_req_stride, const int32_t* offsets, int B_R,
                              long long rows, int L, int H, int d_h, float scale, void* O, long long ldo, int out_bf16,
-                             void* O2, long long ldo2, cudaStream_t s, const int32_t* kv_len) {
+                             void* O2, long long ldo2, cudaStream_t s, const int32_t* kv_len, int q_by_kv) {
   if (B_R == 0 || rows == 0) return ROCS_OK;
   const int Ls = (L + KB - 1) / KB * KB;
   const int pitch = d_h * 2 + 16;
@@ -267,7 +270,8 @@ rocs_status launch_attention(rocs_context* ctx, const void* Q, long long ldq, in
 #define ROCS_ATT(DH, SPLIT)                                                                                         \
   attn_kernel<DH, SPLIT><<<(unsigned)grid, ATT_THREADS, smem, s>>>(                                                 \
       (const __nv_bfloat16*)Q, ldq, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, ldkv, kv_req_stride, offsets, \
-      B_R, rows, L, H, scale_log2, O, ldo, out_bf16, (__nv_bfloat16*)O2, ldo2, splits, kv_len, ctx->d_status)
+      B_R, rows, L, H, scale_log2, O, ldo, out_bf16, (__nv_bfloat16*)O2, ldo2, splits, kv_len, q_by_kv,         \
+      ctx->d_status)
   LaunchTimer lt_("attn", s);
   switch (which) {
     case 0: ROCS_ATT(32, false); break;

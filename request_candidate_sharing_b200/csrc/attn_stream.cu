@@ -35,7 +35,8 @@ __global__ void __launch_bounds__(ST_WARPS * 32, 3) attn_stream_kernel(
     const __nv_bfloat16* __restrict__ Q, long long ldq, const __nv_bfloat16* __restrict__ K,
     const __nv_bfloat16* __restrict__ V, long long ldkv, long long kv_req_stride, const int32_t* __restrict__ offsets,
     int B_R, long long rows, int L_all, int H, float scale_log2, void* O, long long ldo, int out_bf16,
-    __nv_bfloat16* __restrict__ O2, long long ldo2, int S, const int32_t* __restrict__ kv_len, int* status) {
+    __nv_bfloat16* __restrict__ O2, long long ldo2, int S, const int32_t* __restrict__ kv_len, int q_by_kv,
+    int* status) {
   constexpr int PITCH = DH * 2 + 16;
   constexpr int KV_BYTES = KB * PITCH;   // one 64-key block of K (or V)
   constexpr int VPR = DH * 2 / 16;
@@ -46,19 +47,21 @@ __global__ void __launch_bounds__(ST_WARPS * 32, 3) attn_stream_kernel(
   const int h = rem / S;
   const int sidx = rem - h * S;
   if (r >= B_R) return;
-  const long long q0 = offsets[r], q1 = offsets[r + 1];
+  const long long q0 = offsets[r];
+  long long q1 = offsets[r + 1];
   if (q0 < 0 || q1 < q0 || q1 > rows) {
     if (threadIdx.x == 0) set_status(status, ROCS_ERR_INDEX);
     return;
   }
-  const long long nch = (q1 - q0 + ST_ROWS - 1) / ST_ROWS;
-  if (sidx >= nch) return;
   // this request's keys: the first L of its L_all K/V rows (a ragged history), L in [1, L_all]
   const int L = kv_len != nullptr ? kv_len[r] : L_all;
   if (L < 1 || L > L_all) {
     if (threadIdx.x == 0) set_status(status, ROCS_ERR_COUNTS);
     return;
   }
+  if (kv_len != nullptr && q_by_kv) q1 = min(q1, q0 + L);   // ragged self-attention: padding rows ask nothing
+  const long long nch = (q1 - q0 + ST_ROWS - 1) / ST_ROWS;
+  if (sidx >= nch) return;
   const int nkb = (L + KB - 1) / KB;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -381,7 +384,7 @@ rocs_status launch_attention_stream(rocs_context* ctx, const void* Q, long long 
                                     const void* V, long long ldkv, long long kv_req_stride, const int32_t* offsets,
                                     int B_R, long long rows, int L, int H, int d_h, float scale, void* O,
                                     long long ldo, int out_bf16, void* O2, long long ldo2, cudaStream_t s,
-                                    const int32_t* kv_len) {
+                                    const int32_t* kv_len, int q_by_kv) {
   if (B_R == 0 || rows == 0) return ROCS_OK;
   // chunks of one request spread over S CTAs: about twice the mean number of chunks per request
   const long long mean_chunks = (rows + (long long)B_R * ST_ROWS - 1) / ((long long)B_R * ST_ROWS);
@@ -396,7 +399,7 @@ rocs_status launch_attention_stream(rocs_context* ctx, const void* Q, long long 
 #define ROCS_ST(DH, SPLIT)                                                                                         \
   attn_stream_kernel<DH, SPLIT><<<(unsigned)grid, ST_WARPS * 32, 0, s>>>(                                          \
       (const __nv_bfloat16*)Q, ldq, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, ldkv, kv_req_stride, offsets, \
-      B_R, rows, L, H, scale_log2, O, ldo, out_bf16, (__nv_bfloat16*)O2, ldo2, S, kv_len, ctx->d_status)
+      B_R, rows, L, H, scale_log2, O, ldo, out_bf16, (__nv_bfloat16*)O2, ldo2, S, kv_len, q_by_kv, ctx->d_status)
   if (d_h == 32) {
     if (q_split) ROCS_ST(32, true); else ROCS_ST(32, false);
   } else {

@@ -51,6 +51,7 @@ struct AttnTcParams {
   long long ldo2;
   const int32_t* out_rows;   // optional: query row q is written to output row out_rows[q]
   const int32_t* kv_len;     // optional: request r has kv_len[r] keys (1..L), the rest are padding
+  int q_by_kv;               // with kv_len: request r's queries are also only its first kv_len[r] rows
   int* status;
 };
 
@@ -200,13 +201,12 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
 
   const int r = blockIdx.x / P.H;
   const int h = blockIdx.x - r * P.H;
-  const long long q0 = P.offsets[r], q1 = P.offsets[r + 1];
+  const long long q0 = P.offsets[r];
+  long long q1 = P.offsets[r + 1];
   if (q0 < 0 || q1 < q0 || q1 > P.rows) {
     if (threadIdx.x == 0) set_status(P.status, ROCS_ERR_INDEX);
     return;
   }
-  const int ntiles = (int)((q1 - q0 + TQ - 1) / TQ);
-  if (ntiles == 0) return;
   // this request's keys: the first Lr rows of its L-row K/V (a ragged history), Lr in [1, L];
   // without per-request lengths (RAGGED false) every request has L keys
   const int Lr = RAGGED ? P.kv_len[r] : P.L;
@@ -214,6 +214,10 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
     if (threadIdx.x == 0) set_status(P.status, ROCS_ERR_COUNTS);
     return;
   }
+  // a ragged self-attention: the padding rows are no queries either
+  if (RAGGED && P.q_by_kv) q1 = q1 < q0 + Lr ? q1 : q0 + Lr;
+  const int ntiles = (int)((q1 - q0 + TQ - 1) / TQ);
+  if (ntiles == 0) return;
   const int nkb = RAGGED ? (Lr + TK - 1) / TK : P.nkb;
   const int tail_keys = nkb * TK - Lr;   // padding rows in the last staged key block
 
@@ -620,7 +624,7 @@ rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq,
                                 const void* V, long long ldkv, long long kv_rows, const int32_t* offsets, int B_R,
                                 long long rows, int L, int H, int d_h, float scale, void* O, long long ldo,
                                 int out_bf16, void* O2, long long ldo2, cudaStream_t s, const int32_t* out_rows,
-                                const int32_t* kv_len) {
+                                const int32_t* kv_len, int q_by_kv) {
   if (B_R == 0 || rows == 0) return ROCS_OK;
   if ((d_h != 32 && d_h != 64) || L < 1 || (long long)L * d_h > 32768 || (L + TK - 1) / TK > AT_MAX_KB ||
       ((uintptr_t)Q & 15) || ((uintptr_t)K & 15) || ((uintptr_t)V & 15) || ldq % 8 || ldkv % 8 ||
@@ -652,6 +656,7 @@ rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq,
   P.ldo2 = ldo2;
   P.out_rows = out_rows;
   P.kv_len = kv_len;
+  P.q_by_kv = kv_len != nullptr && q_by_kv ? 1 : 0;
   P.status = ctx->d_status;
   LaunchTimer lt_("attn_tc", s);
   const bool rag = kv_len != nullptr;

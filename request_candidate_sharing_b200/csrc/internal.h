@@ -171,7 +171,8 @@ rocs_status launch_token_lcb(rocs_context* ctx, const void* E_R, long long ld_ER
 rocs_status launch_attention(rocs_context* ctx, const void* Q, long long ldq, int q_split, const void* K,
                              const void* V, long long ldkv, long long kv_req_stride, const int32_t* offsets, int B_R,
                              long long rows, int L, int H, int d_h, float scale, void* O, long long ldo,
-                             int out_bf16, void* O2, long long ldo2, cudaStream_t s, const int32_t* kv_len = nullptr);
+                             int out_bf16, void* O2, long long ldo2, cudaStream_t s, const int32_t* kv_len = nullptr,
+                             int q_by_kv = 0);
 
 // Same contract as launch_attention.  _stream: K/V streamed through a small shared-memory ring
 // (any number of query rows per request); _single: one query row per request (a few at most),
@@ -180,7 +181,7 @@ rocs_status launch_attention_stream(rocs_context* ctx, const void* Q, long long 
                                     const void* V, long long ldkv, long long kv_req_stride, const int32_t* offsets,
                                     int B_R, long long rows, int L, int H, int d_h, float scale, void* O,
                                     long long ldo, int out_bf16, void* O2, long long ldo2, cudaStream_t s,
-                                    const int32_t* kv_len = nullptr);
+                                    const int32_t* kv_len = nullptr, int q_by_kv = 0);
 rocs_status launch_attention_single(rocs_context* ctx, const void* Q, long long ldq, int q_split, const void* K,
                                     const void* V, long long ldkv, long long kv_req_stride, const int32_t* offsets,
                                     int B_R, long long rows, int L, int H, int d_h, float scale, void* O,
@@ -201,7 +202,8 @@ rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq,
                                 const void* V, long long ldkv, long long kv_rows, const int32_t* offsets, int B_R,
                                 long long rows, int L, int H, int d_h, float scale, void* O, long long ldo,
                                 int out_bf16, void* O2, long long ldo2, cudaStream_t s,
-                                const int32_t* out_rows = nullptr, const int32_t* kv_len = nullptr);
+                                const int32_t* out_rows = nullptr, const int32_t* kv_len = nullptr,
+                                int q_by_kv = 0);
 
 rocs_status launch_score_head(const void* X, long long ldx, long long rows, int K, const void* w,
                               const float* b, float* out, cudaStream_t s);
