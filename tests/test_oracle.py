@@ -423,3 +423,79 @@ def test_bf16_rounding_of_inputs():
     np.testing.assert_array_equal(r, t)
     big = np.random.default_rng(0).standard_normal(100000).astype(np.float32)
     np.testing.assert_array_equal(synth.bf16_round(big), torch.tensor(big).to(torch.bfloat16).float().numpy())
+
+
+# ---------------------------------------------------------------------------------------------
+# FP8 (E4M3) weights: the encoding written out from the format, pinned by exhaustive checks
+# ---------------------------------------------------------------------------------------------
+def test_e4m3_known_patterns():
+    from oracle import fp8
+    vals = [448.0, -448.0, 1.0, 0.5, 2.0 ** -6, 2.0 ** -9, 0.0, 1.75, 3.25, -2.0 ** -7]
+    pats = [0x7E, 0xFE, 0x38, 0x30, 0x08, 0x01, 0x00, 0x3E, 0x45, 0x84]
+    assert fp8.e4m3_encode(np.asarray(vals)).tolist() == pats
+    assert np.array_equal(fp8.e4m3_decode(np.asarray(pats, np.uint8)), np.asarray(vals))
+
+
+def test_e4m3_every_pattern_round_trips():
+    from oracle import fp8
+    b = np.arange(256, dtype=np.uint8)
+    v = fp8.e4m3_decode(b)
+    nan = np.isnan(v)
+    assert sorted(b[nan].tolist()) == [0x7F, 0xFF]
+    assert np.array_equal(fp8.e4m3_encode(v[~nan]), b[~nan])
+    assert np.nanmax(np.abs(v)) == 448.0
+
+
+def test_e4m3_round_is_nearest_with_ties_to_even():
+    """Against a brute-force search over all finite E4M3 values: the nearest one, a tie going to
+    the value whose pattern is even, magnitudes past 448 saturating."""
+    from oracle import fp8
+    b = np.arange(256, dtype=np.uint8)
+    v = fp8.e4m3_decode(b)
+    fin = ~np.isnan(v)
+    vals, pats = v[fin], b[fin]
+    rng = np.random.default_rng(0)
+    xs = np.concatenate([rng.standard_normal(3000) * 30, rng.standard_normal(2000) * 1e-2,
+                         (vals[:, None] + vals[None, :]).ravel()[::37] / 2,      # midpoints: ties
+                         [500.0, -1e9, 464.0, 465.0, 2.0 ** -10, 3 * 2.0 ** -11]])
+    got = fp8.e4m3_round(xs)
+    for x, g in zip(xs, got):
+        xc = np.clip(x, -448.0, 448.0)
+        d = np.abs(vals - xc)
+        best = np.flatnonzero(d == d.min())
+        if len(best) > 1:
+            best = [i for i in best if pats[i] % 2 == 0 and not (vals[i] == 0 and np.signbit(vals[i]) != np.signbit(xc))]
+        want = vals[best[0]]
+        assert g == want or (g == 0 and want == 0), (x, g, want)
+
+
+def test_quantize_rows_bounds():
+    """Per-channel scales put every row's largest magnitude at the top of the format, and each
+    weight is within half a step (relative 2^-4) of its quantised value."""
+    from oracle import fp8
+    rng = np.random.default_rng(1)
+    W = (rng.standard_normal((33, 70)) * np.exp(rng.standard_normal((33, 1)))).astype(np.float32)
+    W[5] = 0.0
+    Q, s = fp8.quantize_rows(W)
+    q = fp8.e4m3_decode(Q)
+    assert np.all(np.abs(q) <= 448) and s[5] == 1.0 and np.all(q[5] == 0)
+    assert np.allclose(np.abs(q[np.arange(33) != 5]).max(axis=1), 448.0)
+    Wd = fp8.dequantize_rows(Q, s)
+    rel = np.abs(Wd - W) / np.maximum(np.abs(W), s[:, None] * 2.0 ** -6)
+    assert rel.max() <= 2.0 ** -4 + 1e-7
+
+
+def test_w8_linear_by_hand():
+    from oracle import fp8
+    rng = np.random.default_rng(2)
+    X = rng.standard_normal((3, 5))
+    Q = rng.integers(0, 256, (4, 5)).astype(np.uint8)
+    Q[(Q & 0x7F) == 0x7F] = 0x10                       # no NaN patterns
+    s = rng.uniform(0.1, 2.0, 4)
+    b = rng.uniform(-1, 1, 4)
+    y = fp8.w8_linear(X, Q, s, b, "relu")
+    q = fp8.e4m3_decode(Q)
+    for r in range(3):
+        for o in range(4):
+            acc = sum(q[o, i] * X[r, i] for i in range(5))
+            assert abs(y[r, o] - max(s[o] * acc + b[o], 0.0)) < 1e-12
