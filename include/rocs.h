@@ -124,6 +124,36 @@ rocs_status rocs_linear_ikbo(rocs_handle_t handle, const rocs_ikbo_desc* desc,
                              void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------------
+ * FP8-weight (W8A16) IKBO linear ("Compute Only Once: UG-Separation for Efficient Large
+ * Recommendation Models", §三 Stage 4 and the W8A16 table of §六: 8-bit floating-point weights,
+ * bf16 activations).  Weights are E4M3 bytes ("finite" E4M3: bias 7, no infinities, largest
+ * magnitude 448) with one float32 scale per output channel: the effective weight is q_oi * s_o,
+ * and the scale multiplies the accumulated dot product before the bias, Z[m] and activation.
+ *
+ * rocs_quantize_weights_fp8: per-output-channel quantisation of W [rows, cols] (ROCS_F32 or
+ *   ROCS_BF16, device): s_r = max_c |W_rc| / 448 in float32 (1 for an all-zero row), Q_rc =
+ *   E4M3(W_rc / s_r) with the division in float32, rounded to nearest even and saturated.
+ *   Q [rows, cols] uint8 and scale [rows] float32 written.
+ *
+ * rocs_linear_ikbo_w8: rocs_linear_ikbo (dtype_in = ROCS_BF16) with the three weight blocks as
+ *   (Q_RR, s_RR), (Q_CR, s_CR), (Q_CC, s_CC).  Shapes as rocs_linear_ikbo; Q_* [out, in] uint8,
+ *   8-byte aligned; s_* [out] float32.  A GEMM side with at most 64 rows (B_R, resp. B_C) and
+ *   d_in % 32 == 0 streams the FP8 weights directly (each byte read once, expanded to bf16 in
+ *   registers for the tensor cores); a larger side expands its weights to bf16 in the workspace
+ *   once (exactly: every E4M3 value is a bf16 value) and runs the tcgen05 GEMM.  Requires
+ *   d_R_in % 8 == 0 and d_C_in % 8 == 0.  Workspace: rocs_linear_ikbo_w8_workspace.
+ * ---------------------------------------------------------------------------------------- */
+rocs_status rocs_quantize_weights_fp8(rocs_handle_t handle, const void* W, rocs_dtype w_dtype, int32_t rows,
+                                      int32_t cols, uint8_t* Q, float* scale, void* stream);
+rocs_status rocs_linear_ikbo_w8_workspace(rocs_handle_t handle, const rocs_ikbo_desc* desc, size_t* bytes);
+rocs_status rocs_linear_ikbo_w8(rocs_handle_t handle, const rocs_ikbo_desc* desc, const void* X_R,
+                                const void* X_C, const int32_t* req_idx, const uint8_t* Q_RR,
+                                const uint8_t* Q_CR, const uint8_t* Q_CC, const float* s_RR,
+                                const float* s_CR, const float* s_CC, const float* b_R, const float* b_C,
+                                void* Y_R, void* Y_C, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
+/* ------------------------------------------------------------------------------------------
  * rocs_linear_ikbo_noalloc: the same operation as rocs_linear_ikbo for callers that cannot
  * allocate device memory at all, not even a workspace to hand over -- for example plugin hosts
  * and serving loops that plan every device buffer up front and forbid allocation while

@@ -88,6 +88,7 @@ struct IkboArgs {
   int split_in = 0;          // X_R / X_C rows hold [hi (d_in) | lo (d_in)]
   float* Z;   // [B_R, dCo] fp32 scratch
   int* flags = nullptr;      // ikbo_flag_ints(B_R, dCo) ints: request and candidate GEMMs in one launch
+  const float *s_RR = nullptr, *s_CR = nullptr, *s_CC = nullptr;   // per-output-channel accumulator scales
 };
 
 // Completion flags of one fused IKBO launch: one int per (128-request block, 32-column block), an
@@ -101,13 +102,13 @@ rocs_status ikbo_bf16(rocs_context* ctx, const IkboArgs& a, cudaStream_t s) {
     GemmDesc& g = req[nreq++];
     g.A = a.X_R; g.lda = a.ldxr; g.M = a.B_R; g.K = a.dRi; g.split_a = a.split_in;
     g.B = a.W_RR; g.ldb = a.dRi; g.N = a.dRo;
-    g.bias = a.b_R; g.out = a.Y_R; g.ldo = a.ldyr; g.out_mode = a.out_mode; g.act = a.act;
+    g.bias = a.b_R; g.scale = a.s_RR; g.out = a.Y_R; g.ldo = a.ldyr; g.out_mode = a.out_mode; g.act = a.act;
   }
   {
     GemmDesc& g = req[nreq++];
     g.A = a.X_R; g.lda = a.ldxr; g.M = a.B_R; g.K = a.dRi; g.split_a = a.split_in;
     g.B = a.W_CR; g.ldb = a.dRi; g.N = a.dCo;
-    g.bias = a.b_C; g.out = a.Z; g.ldo = a.dCo; g.out_mode = 0; g.act = ROCS_ACT_NONE;
+    g.bias = a.b_C; g.scale = a.s_CR; g.out = a.Z; g.ldo = a.dCo; g.out_mode = 0; g.act = ROCS_ACT_NONE;
   }
   // [REV] §2.4's single launch where it pays: the candidate GEMM's tiles are long (K >= 1024, a
   // split operand counting twice), or there are few of them (a separate request launch is then a
@@ -123,7 +124,7 @@ rocs_status ikbo_bf16(rocs_context* ctx, const IkboArgs& a, cudaStream_t s) {
     GemmDesc& g = req[nreq++];
     g.A = a.X_C; g.lda = a.ldxc; g.M = (int)a.B_C; g.K = a.dCi; g.split_a = a.split_in;
     g.B = a.W_CC; g.ldb = a.dCi; g.N = a.dCo;
-    g.Z = a.Z; g.ldz = a.dCo; g.gidx = a.req_idx; g.gidx_bound = a.B_R;
+    g.Z = a.Z; g.ldz = a.dCo; g.gidx = a.req_idx; g.gidx_bound = a.B_R; g.scale = a.s_CC;
     g.out = a.Y_C; g.ldo = a.ldyc; g.out_mode = a.out_mode; g.act = a.act;
     g.flags = a.flags; g.flag_role = 2;
     std::string site = std::string(g_site ? g_site : "ikbo") + ".ikbo";
@@ -142,7 +143,7 @@ rocs_status ikbo_bf16(rocs_context* ctx, const IkboArgs& a, cudaStream_t s) {
     GemmDesc g;
     g.A = a.X_C; g.lda = a.ldxc; g.M = (int)a.B_C; g.K = a.dCi; g.split_a = a.split_in;
     g.B = a.W_CC; g.ldb = a.dCi; g.N = a.dCo;
-    g.Z = a.Z; g.ldz = a.dCo; g.gidx = a.req_idx; g.gidx_bound = a.B_R;
+    g.Z = a.Z; g.ldz = a.dCo; g.gidx = a.req_idx; g.gidx_bound = a.B_R; g.scale = a.s_CC;
     g.out = a.Y_C; g.ldo = a.ldyc; g.out_mode = a.out_mode; g.act = a.act;
     ROCS_TRY(launch_gemm_bf16(ctx, &g, 1, s));
   }
@@ -380,6 +381,134 @@ extern "C" rocs_status rocs_linear_ikbo(rocs_handle_t h, const rocs_ikbo_desc* d
     ROCS_TRY(launch_pad_rows(W_CC, d->d_C_in, p.WCC, p.kC, d->d_C_out, d->d_C_in, 2, s));
     a.X_C = p.XC; a.ldxc = p.kC; a.W_CC = p.WCC; a.dCi = p.kC;
   }
+  return ikbo_bf16(h, a, s);
+}
+
+// =============================================================================================
+// FP8-weight (W8A16) IKBO linear
+// =============================================================================================
+namespace rocs {
+namespace {
+
+struct W8Plan {
+  float* Z = nullptr;
+  int* flags = nullptr;
+  void *WRR = nullptr, *WCR = nullptr, *WCC = nullptr;   // bf16 expansions (large-M paths only)
+  bool req_skinny = false, cand_skinny = false;
+  size_t bytes = 0;
+};
+
+W8Plan plan_w8(const rocs_ikbo_desc* d, void* ws) {
+  W8Plan p;
+  Carver c(ws);
+  p.req_skinny = w8_skinny_supported(d->B_R, d->d_R_in);
+  p.cand_skinny = d->B_C == 0 || w8_skinny_supported((int)d->B_C, d->d_C_in);
+  p.Z = (float*)c.take((size_t)d->B_R * d->d_C_out * 4);
+  if (!p.cand_skinny) p.flags = (int*)c.take((size_t)ikbo_flag_ints(d->B_R, d->d_C_out) * 4);
+  if (!p.req_skinny) {
+    if (d->d_R_out > 0) p.WRR = c.take((size_t)d->d_R_out * d->d_R_in * 2);
+    p.WCR = c.take((size_t)d->d_C_out * d->d_R_in * 2);
+  }
+  if (!p.cand_skinny) p.WCC = c.take((size_t)d->d_C_out * d->d_C_in * 2);
+  p.bytes = c.used;
+  return p;
+}
+
+rocs_status check_w8_desc(const rocs_ikbo_desc* d) {
+  ROCS_TRY(check_ikbo_desc(d));
+  ROCS_REQUIRE(d->dtype_in == ROCS_BF16, "rocs_linear_ikbo_w8: activations must be bf16");
+  ROCS_REQUIRE(d->d_R_in % 8 == 0 && d->d_C_in % 8 == 0, "rocs_linear_ikbo_w8: d_R_in and d_C_in must be multiples of 8");
+  return ROCS_OK;
+}
+
+}  // namespace
+}  // namespace rocs
+
+extern "C" rocs_status rocs_quantize_weights_fp8(rocs_handle_t h, const void* W, rocs_dtype w_dtype, int32_t rows,
+                                                 int32_t cols, uint8_t* Q, float* scale, void* stream) {
+  CtxGuard ctx_guard_(h);
+  ROCS_REQUIRE(h, "rocs_quantize_weights_fp8: handle is NULL");
+  ROCS_REQUIRE(rows >= 0 && cols >= 0, "rocs_quantize_weights_fp8: negative size");
+  ROCS_REQUIRE(w_dtype == ROCS_F32 || w_dtype == ROCS_BF16, "rocs_quantize_weights_fp8: bad dtype");
+  ROCS_REQUIRE(rows == 0 || cols == 0 || (W && Q && scale), "rocs_quantize_weights_fp8: NULL argument");
+  return launch_w8_quantize(W, w_dtype == ROCS_BF16, rows, cols, Q, scale, (cudaStream_t)stream);
+}
+
+extern "C" rocs_status rocs_linear_ikbo_w8_workspace(rocs_handle_t h, const rocs_ikbo_desc* d, size_t* bytes) {
+  ROCS_REQUIRE(h && bytes, "rocs_linear_ikbo_w8_workspace: NULL argument");
+  ROCS_TRY(check_w8_desc(d));
+  *bytes = plan_w8(d, nullptr).bytes;
+  return ROCS_OK;
+}
+
+extern "C" rocs_status rocs_linear_ikbo_w8(rocs_handle_t h, const rocs_ikbo_desc* d, const void* X_R,
+                                           const void* X_C, const int32_t* req_idx, const uint8_t* Q_RR,
+                                           const uint8_t* Q_CR, const uint8_t* Q_CC, const float* s_RR,
+                                           const float* s_CR, const float* s_CC, const float* b_R, const float* b_C,
+                                           void* Y_R, void* Y_C, void* ws, size_t ws_bytes, void* stream) {
+  CtxGuard ctx_guard_(h);
+  ROCS_REQUIRE(h, "rocs_linear_ikbo_w8: handle is NULL");
+  ROCS_TRY(check_w8_desc(d));
+  ROCS_REQUIRE(X_R && Q_CR && s_CR && b_C, "rocs_linear_ikbo_w8: X_R, Q_CR, s_CR, b_C must be non-NULL");
+  ROCS_REQUIRE(d->d_R_out == 0 || (Q_RR && s_RR && b_R && Y_R),
+               "rocs_linear_ikbo_w8: Q_RR, s_RR, b_R, Y_R needed when d_R_out > 0");
+  ROCS_REQUIRE(d->B_C == 0 || (X_C && Q_CC && s_CC && req_idx && Y_C), "rocs_linear_ikbo_w8: candidate pointers NULL");
+  const void* ptrs[] = {X_R, X_C, Y_R, Y_C, ws};
+  for (const void* p : ptrs) ROCS_REQUIRE(aligned16(p), "rocs_linear_ikbo_w8: X, Y and workspace must be 16-byte aligned");
+  const void* wq[] = {Q_RR, Q_CR, Q_CC};
+  for (const void* p : wq) ROCS_REQUIRE(((uintptr_t)p & 7) == 0, "rocs_linear_ikbo_w8: weights must be 8-byte aligned");
+  const W8Plan need = plan_w8(d, nullptr);
+  if (ws_bytes < need.bytes) {
+    set_error("rocs_linear_ikbo_w8: workspace %zu B < required %zu B", ws_bytes, need.bytes);
+    return ROCS_ERR_WORKSPACE;
+  }
+  const W8Plan p = plan_w8(d, ws);
+  cudaStream_t s = (cudaStream_t)stream;
+  const int out_bf16 = d->dtype_out == ROCS_BF16;
+  // request side: weight-streaming kernel at small B_R, else the bf16 expansion and the tcgen05
+  // GEMM (both with the channel scales on the accumulator)
+  IkboArgs a;
+  a.B_R = d->B_R; a.B_C = d->B_C; a.dRi = d->d_R_in; a.dCi = d->d_C_in; a.dRo = d->d_R_out; a.dCo = d->d_C_out;
+  a.X_R = X_R; a.ldxr = d->d_R_in; a.X_C = X_C; a.ldxc = d->d_C_in; a.req_idx = req_idx;
+  a.b_R = b_R; a.b_C = b_C; a.Y_R = Y_R; a.ldyr = d->d_R_out; a.Y_C = Y_C; a.ldyc = d->d_C_out;
+  a.out_mode = out_bf16 ? 1 : 0; a.act = d->act; a.Z = p.Z; a.flags = p.flags;
+  a.s_RR = s_RR; a.s_CR = s_CR; a.s_CC = s_CC;
+  if (p.req_skinny) {
+    SiteLabel sl("ikbo_w8.req");
+    if (d->d_R_out > 0)
+      ROCS_TRY(launch_w8_skinny(h, X_R, d->d_R_in, d->B_R, d->d_R_in, Q_RR, d->d_R_out, s_RR, b_R, nullptr, 0, nullptr,
+                                0, Y_R, d->d_R_out, out_bf16, d->act, s));
+    ROCS_TRY(launch_w8_skinny(h, X_R, d->d_R_in, d->B_R, d->d_R_in, Q_CR, d->d_C_out, s_CR, b_C, nullptr, 0, nullptr, 0,
+                              p.Z, d->d_C_out, 0, ROCS_ACT_NONE, s));
+  } else {
+    if (d->d_R_out > 0) ROCS_TRY(launch_w8_expand(Q_RR, (long long)d->d_R_out * d->d_R_in, p.WRR, s));
+    ROCS_TRY(launch_w8_expand(Q_CR, (long long)d->d_C_out * d->d_R_in, p.WCR, s));
+  }
+  if (d->B_C > 0 && p.cand_skinny) {
+    if (!p.req_skinny) {   // the request GEMMs alone (the candidate side does not run on tcgen05)
+      IkboArgs r = a;
+      r.B_C = 0; r.W_RR = p.WRR; r.W_CR = p.WCR;
+      SiteLabel sl("ikbo_w8");
+      ROCS_TRY(ikbo_bf16(h, r, s));
+    }
+    SiteLabel sl("ikbo_w8.cand");
+    return launch_w8_skinny(h, X_C, d->d_C_in, (int)d->B_C, d->d_C_in, Q_CC, d->d_C_out, s_CC, nullptr, p.Z,
+                            d->d_C_out, req_idx, d->B_R, Y_C, d->d_C_out, out_bf16, d->act, s);
+  }
+  if (d->B_C > 0) ROCS_TRY(launch_w8_expand(Q_CC, (long long)d->d_C_out * d->d_C_in, p.WCC, s));
+  if (p.req_skinny) {
+    if (d->B_C == 0) return ROCS_OK;
+    // request outputs exist; the candidate GEMM alone on tcgen05 (no request problems in it)
+    GemmDesc g;
+    g.A = X_C; g.lda = d->d_C_in; g.M = (int)d->B_C; g.K = d->d_C_in;
+    g.B = p.WCC; g.ldb = d->d_C_in; g.N = d->d_C_out;
+    g.Z = p.Z; g.ldz = d->d_C_out; g.gidx = req_idx; g.gidx_bound = d->B_R; g.scale = s_CC;
+    g.out = Y_C; g.ldo = d->d_C_out; g.out_mode = out_bf16 ? 1 : 0; g.act = d->act;
+    SiteLabel sl("ikbo_w8.cand");
+    return launch_gemm_bf16(h, &g, 1, s);
+  }
+  a.W_RR = p.WRR; a.W_CR = p.WCR; a.W_CC = p.WCC;
+  SiteLabel sl("ikbo_w8");
   return ikbo_bf16(h, a, s);
 }
 

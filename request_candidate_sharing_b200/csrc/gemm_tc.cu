@@ -45,6 +45,7 @@ struct Problem {
   CUtensorMap tmO;     // output [M, N] (out_mode 2: the hi half), box 32 x 32, stored by TMA
   CUtensorMap tmOlo;   // out_mode 2: the lo half at column offset lo_off
   const float* bias;
+  const float* scale;   // optional per-column factor on the accumulator (FP8 weights' channel scales)
   const float* Z;
   const int32_t* gidx;
   void* out;
@@ -158,6 +159,10 @@ __device__ __forceinline__ void store_chunk(const Problem& pr, long long grow, i
 // acquire, never through the non-coherent read-only path.
 __device__ __forceinline__ void epilogue_math(const Problem& pr, const float* zrow, int col0, float (&v)[32]) {
   const bool full32 = (col0 + 32 <= pr.N) && pr.vec_ok;
+  if (pr.scale != nullptr) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] *= col0 + j < pr.N ? __ldg(pr.scale + col0 + j) : 0.f;
+  }
   if (pr.bias != nullptr) {
     if (full32) {
       const float4* b4 = reinterpret_cast<const float4*>(pr.bias + col0);
@@ -454,6 +459,10 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
           const bool full32 = (col0 + 32 <= pr.N) && pr.vec_ok;
+          if (pr.scale != nullptr) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] *= col0 + j < pr.N ? __ldg(pr.scale + col0 + j) : 0.f;
+          }
           if (pr.bias != nullptr) {
             if (full32) {
               const float4* b4 = reinterpret_cast<const float4*>(pr.bias + col0);
@@ -595,6 +604,7 @@ rocs_status launch_gemm_bf16(rocs_context* ctx, const GemmDesc* probs, int nprob
       return ROCS_ERR_CUDA;
     }
     p.bias = g.bias;
+    p.scale = g.scale;
     p.Z = g.Z;
     p.gidx = g.gidx;
     p.gidx_bound = g.gidx_bound;

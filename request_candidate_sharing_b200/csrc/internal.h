@@ -78,7 +78,7 @@ void set_error(const char* fmt, ...);
 rocs_status cuda_check(cudaError_t e, const char* what);
 
 // One GEMM problem for the tcgen05 kernel:
-//   out[r, c] = act( sum_k A[r, k] * B[c, k] + bias[c] + Z[gidx[r], c] )
+//   out[r, c] = act( scale[c] * sum_k A[r, k] * B[c, k] + bias[c] + Z[gidx[r], c] )
 // A [M, K] bf16 (row stride lda), B [N, K] bf16 (row stride ldb); bias, Z, gidx optional.
 // split_a: A rows hold a hi/lo pair [hi (K) | lo (K)] of one fp32-precise activation
 //   (K % 64 == 0); the kernel accumulates hi*B + lo*B.
@@ -87,6 +87,7 @@ struct GemmDesc {
   const void* A = nullptr; long long lda = 0; int M = 0; int K = 0; int split_a = 0;
   const void* B = nullptr; long long ldb = 0; int N = 0;
   const float* bias = nullptr;
+  const float* scale = nullptr;   // per-column factor on the accumulator, before bias and Z
   const float* Z = nullptr; long long ldz = 0; const int32_t* gidx = nullptr; int gidx_bound = 0;
   void* out = nullptr; long long ldo = 0; int out_mode = 1; int act = ROCS_ACT_NONE;
   // One launch for a request GEMM and the candidate GEMM that gathers its output (the IKBO
@@ -109,6 +110,18 @@ rocs_status launch_gemm_f32(rocs_context* ctx, const float* A, long long lda, in
                             long long ldb, int N, const float* bias, const float* Z, long long ldz,
                             const int32_t* gidx, int gidx_bound, float* out, long long ldo, int act,
                             cudaStream_t s);
+
+// FP8-weight (W8A16) linears (w8.cu).  Q: E4M3 bytes [rows, cols]; scale: one float per row.
+rocs_status launch_w8_quantize(const void* W, int w_bf16, int rows, int cols, uint8_t* Q, float* scale,
+                               cudaStream_t s);
+// E4M3 -> bf16, exact (count even)
+rocs_status launch_w8_expand(const uint8_t* Q, long long count, void* out, cudaStream_t s);
+bool w8_skinny_supported(int M, int K);
+// out[r, c] = act(scale[c] * sum_k X[r, k] q[c, k] + bias[c] + Z[gidx[r], c]) for M <= 64 rows
+rocs_status launch_w8_skinny(rocs_context* ctx, const void* X, long long ldx, int M, int K, const uint8_t* W8, int N,
+                             const float* scale, const float* bias, const float* Z, long long ldz,
+                             const int32_t* gidx, int gidx_bound, void* out, long long ldo, int out_bf16, int act,
+                             cudaStream_t s);
 
 // Stable counting sort of candidates by request index (sort.cu).  perm[k] = the candidate at
 // sorted position k; offsets[r] = first position of request r, offsets[B_R] = valid candidates

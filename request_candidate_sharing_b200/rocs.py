@@ -125,6 +125,9 @@ _lib_fwd = _proto("rocs_forward", P, C.POINTER(ModelDesc), C.POINTER(ModelWeight
 _lib_ikbo_na = _proto("rocs_linear_ikbo_noalloc", P, C.POINTER(IkboDesc), P, P, P, P, P, P, P, P, P, P, P)
 _lib_graph = _proto("rocs_set_graph_replay", P, I32)
 _lib_fused = _proto("rocs_set_ikbo_fused", P, I32)
+_lib_q8 = _proto("rocs_quantize_weights_fp8", P, P, C.c_int, I32, I32, P, P, P)
+_lib_w8_ws = _proto("rocs_linear_ikbo_w8_workspace", P, C.POINTER(IkboDesc), C.POINTER(C.c_size_t))
+_lib_w8 = _proto("rocs_linear_ikbo_w8", P, C.POINTER(IkboDesc), P, P, P, P, P, P, P, P, P, P, P, P, P, P, C.c_size_t, P)
 _lib_sort_ws = _proto("rocs_sort_by_request_workspace", P, I32, I64, C.POINTER(C.c_size_t))
 _lib_sort = _proto("rocs_sort_by_request", P, P, I32, I64, P, P, P, C.c_size_t, P)
 _lib_xu_ws = _proto("rocs_dca_cross_attn_unsorted_workspace", P, I32, I64, I32, I32, C.c_int, C.POINTER(C.c_size_t))
@@ -138,7 +141,8 @@ EXPORTED = ["rocs_linear_ikbo_noalloc", "rocs_timing_start", "rocs_timing_stop",
             "rocs_fm_masked", "rocs_token_lcb_workspace", "rocs_token_lcb", "rocs_dca_cross_attn",
             "rocs_dca_encode_workspace", "rocs_dca_encode", "rocs_forward_workspace", "rocs_forward",
             "rocs_set_graph_replay", "rocs_set_ikbo_fused", "rocs_sort_by_request_workspace",
-            "rocs_sort_by_request", "rocs_dca_cross_attn_unsorted_workspace", "rocs_dca_cross_attn_unsorted"]
+            "rocs_sort_by_request", "rocs_dca_cross_attn_unsorted_workspace", "rocs_dca_cross_attn_unsorted",
+            "rocs_quantize_weights_fp8", "rocs_linear_ikbo_w8_workspace", "rocs_linear_ikbo_w8"]
 
 
 def ptr(x) -> Optional[int]:
@@ -290,6 +294,21 @@ class Rocs:
 
     def rocs_set_ikbo_fused(self, enable: int):
         _check(_lib_fused(self.h, int(enable)))
+
+    # -- FP8-weight (W8A16) IKBO linear --
+    def rocs_quantize_weights_fp8(self, W, w_dtype: int, rows: int, cols: int, Q, scale, stream=None):
+        _check(_lib_q8(self.h, ptr(W), int(w_dtype), int(rows), int(cols), ptr(Q), ptr(scale), stream))
+
+    def rocs_linear_ikbo_w8_workspace(self, desc: IkboDesc) -> int:
+        n = C.c_size_t(0)
+        _check(_lib_w8_ws(self.h, C.byref(desc), C.byref(n)))
+        return int(n.value)
+
+    def rocs_linear_ikbo_w8(self, desc: IkboDesc, X_R, X_C, req_idx, Q_RR, Q_CR, Q_CC, s_RR, s_CR, s_CC, b_R, b_C,
+                            Y_R, Y_C, workspace, workspace_bytes: int, stream=None):
+        _check(_lib_w8(self.h, C.byref(desc), ptr(X_R), ptr(X_C), ptr(req_idx), ptr(Q_RR), ptr(Q_CR), ptr(Q_CC),
+                       ptr(s_RR), ptr(s_CR), ptr(s_CC), ptr(b_R), ptr(b_C), ptr(Y_R), ptr(Y_C), ptr(workspace),
+                       int(workspace_bytes), stream))
 
     # -- candidates in any order --
     def rocs_sort_by_request_workspace(self, B_R: int, B_C: int) -> int:

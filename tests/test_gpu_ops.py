@@ -241,6 +241,75 @@ def test_linear_short_k_many_candidates(R):
 
 
 # ---------------------------------------------------------------------------------------------
+# FP8-weight (W8A16) IKBO linear
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("w_bf16", [0, 1])
+def test_quantize_weights_fp8_bit_exact(R, w_bf16):
+    """Per-channel E4M3 quantisation: bytes and scales equal the oracle's exactly."""
+    from oracle import fp8
+    from request_candidate_sharing_b200 import rocs
+    g = np.random.default_rng(5)
+    W = (g.standard_normal((300, 1000)) * np.exp(2 * g.standard_normal((300, 1)))).astype(np.float32)
+    W[3] = 0.0
+    W[7, ::3] = 1e-30
+    W[9, 5] = 3e30
+    if w_bf16:
+        W = synth.bf16_round(W)
+    Q_ref, s_ref = fp8.quantize_rows(W)
+    Q = torch.empty((300, 1000), dtype=torch.uint8, device="cuda")
+    sc = torch.empty(300, dtype=torch.float32, device="cuda")
+    R.rocs_quantize_weights_fp8(dev(W, torch.bfloat16 if w_bf16 else torch.float32),
+                                rocs.ROCS_BF16 if w_bf16 else rocs.ROCS_F32, 300, 1000, Q, sc, stream())
+    _status_ok(R)
+    assert np.array_equal(sc.cpu().numpy(), s_ref)
+    assert np.array_equal(Q.cpu().numpy(), Q_ref)
+
+
+def _run_w8(R, case, x, q, m, out_dtype):
+    from request_candidate_sharing_b200 import rocs
+    d = rocs.IkboDesc(case.B_R, case.B_C, case.d_R_in, case.d_C_in, case.d_R_out, case.d_C_out, rocs.ROCS_BF16,
+                      out_dtype, rocs.ACT[case.act])
+    nb = R.rocs_linear_ikbo_w8_workspace(d)
+    ws = torch.empty(max(nb, 16), dtype=torch.uint8, device="cuda")
+    odt = torch.bfloat16 if out_dtype == rocs.ROCS_BF16 else torch.float32
+    YR = torch.full((case.B_R, max(case.d_R_out, 1)), float("nan"), dtype=odt, device="cuda")
+    YC = torch.full((max(case.B_C, 1), case.d_C_out), float("nan"), dtype=odt, device="cuda")
+    t = {k: torch.from_numpy(np.ascontiguousarray(v)).cuda() for k, v in q.items()}
+    R.rocs_linear_ikbo_w8(d, dev(x["X_R"], torch.bfloat16), dev(x["X_C"], torch.bfloat16), dev_i32(m),
+                          t.get("Q_RR"), t["Q_CR"], t["Q_CC"], t.get("s_RR"), t["s_CR"], t["s_CC"],
+                          dev(x["b_R"], torch.float32), dev(x["b_C"], torch.float32), YR, YC, ws, nb, stream())
+    _status_ok(R)
+    return YR[:, :case.d_R_out], YC[:case.B_C]
+
+
+@pytest.mark.parametrize("counts,dRi,dCi,dRo,dCo,out", [
+    ([16], 1280, 1280, 2560, 2560, 1),               # the pages' (1, 16, 1280, 2560): small M on both sides
+    ([8], 1280, 1280, 640, 640, 0),                  # (1, 8, 1280, 640), fp32 out
+    ([40, 0, 23], 96, 200, 64, 136, 1),              # small M, candidate K not a multiple of 32 (expanded)
+    ([300] * 5 + [7], 256, 512, 128, 384, 1),        # B_C > 64: expanded weights on the tcgen05 GEMM
+    ([1] * 60 + [0] * 30, 512, 256, 0, 256, 0),     # B_R > 64 (expanded) with a small candidate side
+])
+def test_linear_ikbo_w8(R, counts, dRi, dCi, dRo, dCo, out):
+    """W8A16 IKBO linear against the oracle's early-broadcast evaluation with the effective weights
+    q * s, on the weight-streaming kernel, the expanded-weight GEMM, and mixes of the two."""
+    from oracle import fp8
+    case = synth.LinearCase("w8", np.asarray(counts, np.int32), dRi, dCi, dRo, dCo, "gelu", True, 13)
+    x = synth.linear_inputs(case)
+    _, m = O.segments(case.counts)
+    q = {}
+    for k in ("RR", "CR", "CC"):
+        if k == "RR" and dRo == 0:
+            continue
+        q["Q_" + k], q["s_" + k] = fp8.quantize_rows(x["W_" + k])
+    YR, YC = _run_w8(R, case, x, q, m, out)
+    rR, rC = fp8.w8_glm_linear(x["X_R"], x["X_C"], m, q.get("Q_RR"), q.get("s_RR"), q["Q_CR"], q["s_CR"], q["Q_CC"],
+                               q["s_CC"], x["b_R"] if dRo else None, x["b_C"], "gelu")
+    if dRo:
+        check_bf16(host(YR.float()), rR, out_bf16=out == 1, what="Y_R")
+    check_bf16(host(YC.float()), rC, out_bf16=out == 1, what="Y_C")
+
+
+# ---------------------------------------------------------------------------------------------
 # a6 group LayerNorm
 # ---------------------------------------------------------------------------------------------
 @pytest.mark.parametrize("io", [0, 1])
