@@ -53,6 +53,9 @@ WORKLOADS = {
     "ikbo_sweep": "IKBO linear sweep: B_R=256, N in {64, 256, 1024} candidates per request, d_in = d_out = d in "
                   "{512, 1024, 4096}, bf16 in/out, fp32 accumulate, ReLU; against two materialised-broadcast "
                   "GPU baselines (B1: Z[m] materialised and added; B2: gathered [X^R[m], X^C] with one K=2d GEMM)",
+    "w8a16": "FP8-weight (W8A16) IKBO linear against the same linear with bf16 weights, weights read from HBM "
+             "(L2 flushed): the UG-Separation review's four configurations (1, N, d_in, d_out) = (1, 16|8, 1280, "
+             "2560|640) read as one request with N candidates, plus two larger weight-bound shapes",
     "xattn_unsorted": "candidate cross-attention with candidates in shuffled order (each with its request index): "
                       "512 requests, candidates ~ clipped lognormal (median 300, 16..2000), L=1024, d=256, 8 heads; "
                       "stable sort by request + gather + segment-path attention + scatter, against the grouped call",
@@ -721,6 +724,100 @@ def run_ikbo_sweep(args, rank, world, local):
     R.close()
 
 
+def run_w8a16(args, rank, world, local):
+    """Per configuration (B_R, N, d_in, d_out): rocs_linear_ikbo with bf16 weights and
+    rocs_linear_ikbo_w8 with per-channel E4M3 weights (quantised by rocs_quantize_weights_fp8),
+    bf16 activations and outputs, GELU.  Each repetition is timed alone with CUDA events after an L2
+    flush (a 256 MB write), so the weights come from HBM as in a model whose other layers evict
+    them; medians.  Inputs: torch normal draws on the device."""
+    import torch
+    from request_candidate_sharing_b200 import rocs
+    dev = torch.device("cuda", local)
+    R = rocs.Rocs(local)
+    peaks = load_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    reps = max(args.steps, 3)
+    sh = torch.cuda.current_stream(dev).cuda_stream
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            ts.append(e0.elapsed_time(e1))
+        ts.sort()
+        return ts[len(ts) // 2]
+
+    points = []
+    for (B_R, N, di, do) in ((1, 16, 1280, 2560), (1, 16, 1280, 640), (1, 8, 1280, 2560), (1, 8, 1280, 640),
+                             (1, 16, 8192, 8192), (4, 16, 4096, 16384)):
+        B_C = B_R * N
+        g = torch.Generator(device=dev).manual_seed(di + do + N)
+        bf = torch.bfloat16
+        XR = torch.randn(B_R, di, device=dev, generator=g).to(bf)
+        XC = torch.randn(B_C, di, device=dev, generator=g).to(bf)
+        Ws = [torch.randn(do, di, device=dev, generator=g).mul_(di ** -0.5).to(bf) for _ in range(3)]
+        bR = torch.rand(do, device=dev, generator=g) * 0.2 - 0.1
+        bC = torch.rand(do, device=dev, generator=g) * 0.2 - 0.1
+        m = torch.arange(B_R, device=dev, dtype=torch.int32).repeat_interleave(N)
+        Q = [torch.empty(do, di, dtype=torch.uint8, device=dev) for _ in range(3)]
+        S = [torch.empty(do, dtype=torch.float32, device=dev) for _ in range(3)]
+        for i in range(3):
+            R.rocs_quantize_weights_fp8(Ws[i], rocs.ROCS_BF16, do, di, Q[i], S[i], sh)
+        desc = rocs.IkboDesc(B_R, B_C, di, di, do, do, rocs.ROCS_BF16, rocs.ROCS_BF16, rocs.ACT["gelu"])
+        nb = R.rocs_linear_ikbo_workspace(desc)
+        nb8 = R.rocs_linear_ikbo_w8_workspace(desc)
+        ws = torch.empty(max(nb, nb8, 16), dtype=torch.uint8, device=dev)
+        YR = torch.empty(B_R, do, dtype=bf, device=dev)
+        YC = torch.empty(B_C, do, dtype=bf, device=dev)
+        ms_b = timed(lambda: R.rocs_linear_ikbo(desc, XR, XC, m, Ws[0], Ws[1], Ws[2], bR, bC, YR, YC, ws, nb, sh))
+        YC_b = YC.float().clone()
+        ms_8 = timed(lambda: R.rocs_linear_ikbo_w8(desc, XR, XC, m, Q[0], Q[1], Q[2], S[0], S[1], S[2], bR, bC, YR, YC,
+                                                    ws, nb8, sh))
+        if R.rocs_get_device_status(sh) != 0:
+            raise RuntimeError("device status set")
+        # per-kernel times of both calls (direct launches, per-launch CUDA events, L2 flushed)
+        kern = {}
+        for name, fn in (("bf16", lambda: R.rocs_linear_ikbo(desc, XR, XC, m, Ws[0], Ws[1], Ws[2], bR, bC, YR, YC, ws, nb,
+                                                            sh)),
+                         ("fp8", lambda: R.rocs_linear_ikbo_w8(desc, XR, XC, m, Q[0], Q[1], Q[2], S[0], S[1], S[2], bR,
+                                                               bC, YR, YC, ws, nb8, sh))):
+            R.rocs_timing_start(256)
+            for _ in range(reps):
+                flush.fill_(1)
+                fn()
+            kern[name] = {k: round(t / reps, 4) for k, (n_, t) in R.rocs_timing_stop().items()}
+        rel = float((YC.float() - YC_b).norm() / YC_b.norm())
+        wbytes8 = 3.0 * do * di + 3 * do * 4
+        act_bytes = (B_R + B_C) * di * 2.0 + (B_R + B_C) * do * 2.0
+        gbs = (wbytes8 + act_bytes) / (ms_8 / 1e3) / 1e9
+        points.append({"B_R": B_R, "N": N, "d_in": di, "d_out": do, "bf16_weights_ms": round(ms_b, 4),
+                       "fp8_weights_ms": round(ms_8, 4), "latency_change": round(ms_8 / ms_b - 1.0, 4),
+                       "fp8_GBps": round(gbs, 1), "fp8_frac_of_hbm": round(gbs / peaks["hbm"], 4),
+                       "rel_l2_vs_bf16_weights": round(rel, 5), "kernel_ms": kern})
+        del XR, XC, Ws, Q, S, ws, YR, YC
+        torch.cuda.empty_cache()
+    if rank == 0:
+        head = points[0]
+        line = {"metric": METRIC, "value": round(head["N"] * head["B_R"] / (head["fp8_weights_ms"] / 1e3), 1),
+                "unit": "candidates/s", "n_gpus": world, "steps": reps, "warmup": args.warmup,
+                "ms_per_step": head["fp8_weights_ms"], "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16 activations, e4m3 weights",
+                "data": "synthetic (torch normal draws on the device)",
+                "config": {"workload": "w8a16", "description": WORKLOADS["w8a16"],
+                           "l2": "flushed (256 MB write) before every repetition",
+                           "peak_source": peaks["source"] + " (of measured)"},
+                "points": points}
+        print(json.dumps(line), flush=True)
+    R.close()
+
+
 def run_xattn_unsorted(args, rank, world, local):
     """The grouped cross-attention (rocs_dca_cross_attn) and the same rows shuffled, each with its
     request index (rocs_dca_cross_attn_unsorted: sort, gather, attention, scatter), plus the sort
@@ -829,6 +926,8 @@ def main():
         run_ikbo_sweep(args, rank, world, local)
     elif args.workload == "xattn_unsorted":
         run_xattn_unsorted(args, rank, world, local)
+    elif args.workload == "w8a16":
+        run_w8a16(args, rank, world, local)
     else:
         run_librocs(args, rank, world, local)
 

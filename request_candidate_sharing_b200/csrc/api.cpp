@@ -394,6 +394,8 @@ struct W8Plan {
   float* Z = nullptr;
   int* flags = nullptr;
   void *WRR = nullptr, *WCR = nullptr, *WCC = nullptr;   // bf16 expansions (large-M paths only)
+  void *XhR = nullptr, *XhC = nullptr;                    // f16 activations (weight-streaming paths only)
+  int *shR = nullptr, *shC = nullptr;
   bool req_skinny = false, cand_skinny = false;
   size_t bytes = 0;
 };
@@ -410,6 +412,14 @@ W8Plan plan_w8(const rocs_ikbo_desc* d, void* ws) {
     p.WCR = c.take((size_t)d->d_C_out * d->d_R_in * 2);
   }
   if (!p.cand_skinny) p.WCC = c.take((size_t)d->d_C_out * d->d_C_in * 2);
+  if (p.req_skinny) {
+    p.XhR = c.take((size_t)d->B_R * d->d_R_in * 2);
+    p.shR = (int*)c.take((size_t)d->B_R * 4);
+  }
+  if (p.cand_skinny && d->B_C > 0) {
+    p.XhC = c.take((size_t)d->B_C * d->d_C_in * 2);
+    p.shC = (int*)c.take((size_t)d->B_C * 4);
+  }
   p.bytes = c.used;
   return p;
 }
@@ -473,12 +483,25 @@ extern "C" rocs_status rocs_linear_ikbo_w8(rocs_handle_t h, const rocs_ikbo_desc
   a.b_R = b_R; a.b_C = b_C; a.Y_R = Y_R; a.ldyr = d->d_R_out; a.Y_C = Y_C; a.ldyc = d->d_C_out;
   a.out_mode = out_bf16 ? 1 : 0; a.act = d->act; a.Z = p.Z; a.flags = p.flags;
   a.s_RR = s_RR; a.s_CR = s_CR; a.s_CC = s_CC;
+  {
+    // both sides' activations as f16 operands of the weight-streaming kernel, in one launch
+    const bool prepR = p.req_skinny, prepC = p.cand_skinny && d->B_C > 0;
+    SiteLabel sl("ikbo_w8");
+    if (prepR && prepC)
+      ROCS_TRY(launch_w8_xprep(X_R, d->d_R_in, d->B_R, d->d_R_in, p.XhR, p.shR, X_C, d->d_C_in, (int)d->B_C,
+                               d->d_C_in, p.XhC, p.shC, s));
+    else if (prepR)
+      ROCS_TRY(launch_w8_xprep(X_R, d->d_R_in, d->B_R, d->d_R_in, p.XhR, p.shR, nullptr, 0, 0, 0, nullptr, nullptr, s));
+    else if (prepC)
+      ROCS_TRY(launch_w8_xprep(X_C, d->d_C_in, (int)d->B_C, d->d_C_in, p.XhC, p.shC, nullptr, 0, 0, 0, nullptr, nullptr,
+                               s));
+  }
   if (p.req_skinny) {
     SiteLabel sl("ikbo_w8.req");
     if (d->d_R_out > 0)
-      ROCS_TRY(launch_w8_skinny(h, X_R, d->d_R_in, d->B_R, d->d_R_in, Q_RR, d->d_R_out, s_RR, b_R, nullptr, 0, nullptr,
+      ROCS_TRY(launch_w8_skinny(h, p.XhR, p.shR, d->B_R, d->d_R_in, Q_RR, d->d_R_out, s_RR, b_R, nullptr, 0, nullptr,
                                 0, Y_R, d->d_R_out, out_bf16, d->act, s));
-    ROCS_TRY(launch_w8_skinny(h, X_R, d->d_R_in, d->B_R, d->d_R_in, Q_CR, d->d_C_out, s_CR, b_C, nullptr, 0, nullptr, 0,
+    ROCS_TRY(launch_w8_skinny(h, p.XhR, p.shR, d->B_R, d->d_R_in, Q_CR, d->d_C_out, s_CR, b_C, nullptr, 0, nullptr, 0,
                               p.Z, d->d_C_out, 0, ROCS_ACT_NONE, s));
   } else {
     if (d->d_R_out > 0) ROCS_TRY(launch_w8_expand(Q_RR, (long long)d->d_R_out * d->d_R_in, p.WRR, s));
@@ -492,7 +515,7 @@ extern "C" rocs_status rocs_linear_ikbo_w8(rocs_handle_t h, const rocs_ikbo_desc
       ROCS_TRY(ikbo_bf16(h, r, s));
     }
     SiteLabel sl("ikbo_w8.cand");
-    return launch_w8_skinny(h, X_C, d->d_C_in, (int)d->B_C, d->d_C_in, Q_CC, d->d_C_out, s_CC, nullptr, p.Z,
+    return launch_w8_skinny(h, p.XhC, p.shC, (int)d->B_C, d->d_C_in, Q_CC, d->d_C_out, s_CC, nullptr, p.Z,
                             d->d_C_out, req_idx, d->B_R, Y_C, d->d_C_out, out_bf16, d->act, s);
   }
   if (d->B_C > 0) ROCS_TRY(launch_w8_expand(Q_CC, (long long)d->d_C_out * d->d_C_in, p.WCC, s));

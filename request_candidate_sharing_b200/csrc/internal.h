@@ -117,9 +117,14 @@ rocs_status launch_w8_quantize(const void* W, int w_bf16, int rows, int cols, ui
 // E4M3 -> bf16, exact (count even)
 rocs_status launch_w8_expand(const uint8_t* Q, long long count, void* out, cudaStream_t s);
 bool w8_skinny_supported(int M, int K);
-// out[r, c] = act(scale[c] * sum_k X[r, k] q[c, k] + bias[c] + Z[gidx[r], c]) for M <= 64 rows
-rocs_status launch_w8_skinny(rocs_context* ctx, const void* X, long long ldx, int M, int K, const uint8_t* W8, int N,
-                             const float* scale, const float* bias, const float* Z, long long ldz,
+// X [M, K] bf16 (row stride ldx) -> Xh [M, K] f16 times 2^-shift[m], the operand of launch_w8_skinny;
+// two activation sets in one launch (M1 may be 0)
+rocs_status launch_w8_xprep(const void* X0, long long ldx0, int M0, int K0, void* Xh0, int* sh0, const void* X1,
+                            long long ldx1, int M1, int K1, void* Xh1, int* sh1, cudaStream_t s);
+// out[r, c] = act(scale[c] * sum_k X[r, k] q[c, k] + bias[c] + Z[gidx[r], c]) for M <= 64 rows, from
+// the prepared Xh and shift
+rocs_status launch_w8_skinny(rocs_context* ctx, const void* Xh, const int* shift, int M, int K, const uint8_t* W8,
+                             int N, const float* scale, const float* bias, const float* Z, long long ldz,
                              const int32_t* gidx, int gidx_bound, void* out, long long ldo, int out_bf16, int act,
                              cudaStream_t s);
 
