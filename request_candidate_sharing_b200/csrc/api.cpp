@@ -879,6 +879,7 @@ struct FwdPlan {
   // DCA
   EncScratch enc;
   void *S[2], *KR = nullptr, *VR = nullptr, *KC, *VC;   // KR/VR only when the request attention is not absorbed
+  void* ar_scratch = nullptr;                             // the absorbed request attention's k' and split states
   float *YR, *YC;            // own-query token streams (fp32)
   void *tR, *tC, *qhR, *qhC, *QR, *QC;   // hi/lo pairs
   float *AR, *AC;            // attention outputs when no caller buffer takes them
@@ -929,6 +930,8 @@ FwdPlan plan_forward(const rocs_model_desc* m, void* ws, bool own_offsets, bool 
     if (!attention_req_absorbed_supported(m->d, m->H, m->L)) {
       p.KR = c.take(rowsL * m->d * 2);
       p.VR = c.take(rowsL * m->d * 2);
+    } else {
+      p.ar_scratch = c.take(attention_req_absorbed_scratch(m->B_R, m->L));
     }
     p.KC = c.take(rowsL * m->d * 2);
     p.VC = c.take(rowsL * m->d * 2);
@@ -1144,7 +1147,7 @@ rocs_status forward_launches(rocs_handle_t h, const rocs_model_desc* m, const ro
         SiteLabel s_xa("xattn.req");
         if (p.KR == nullptr)
           ROCS_TRY(launch_attention_req_absorbed(h, p.QR, d2, S_l, dw.WK_R, dw.WV_R, BR, m->L, m->d, m->H, scale, dR,
-                                                 ldR, xR2, xr, s, in->hist_len));
+                                                 ldR, xR2, xr, s, in->hist_len, p.ar_scratch));
         else
           ROCS_TRY(launch_attention_single(h, p.QR, d2, 1, p.KR, p.VR, m->d, (long long)m->L * m->d, p.iota1, BR, BR,
                                            m->L, m->H, dh, scale, dR, ldR, 0, xR2, xr, s, in->hist_len));

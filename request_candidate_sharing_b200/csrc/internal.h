@@ -215,7 +215,10 @@ bool attention_req_absorbed_supported(int d, int H, int L);
 rocs_status launch_attention_req_absorbed(rocs_context* ctx, const void* Q, long long ldq, const void* S,
                                           const void* WK, const void* WV, int B_R, int L, int d, int H, float scale,
                                           float* O, long long ldo, void* O2, long long ldo2, cudaStream_t s,
-                                          const int32_t* kv_len = nullptr);
+                                          const int32_t* kv_len, void* scratch);
+// bytes of device scratch (256-byte aligned) the absorbed request attention needs for B_R requests
+// of up to L history rows: the k' pairs and the per-split softmax states
+size_t attention_req_absorbed_scratch(int B_R, int L);
 rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq, int q_split, const void* K,
                                 const void* V, long long ldkv, long long kv_rows, const int32_t* offsets, int B_R,
                                 long long rows, int L, int H, int d_h, float scale, void* O, long long ldo,
