@@ -133,14 +133,29 @@ __device__ __forceinline__ void gram_tile(uint32_t sbase, int pitch, int a0, int
 // ---------------------------------------------------------------------------------------------
 // One CTA per SM walks a contiguous range of candidates.  Warp 0 streams each candidate's E^C rows
 // (contiguous, n_C x D) into a ring of shared-memory stages with bulk async copies, FC_STAGES
-// candidates ahead; consumer warp w takes the candidates w, w + FC_CONSUMERS, ... of the range, so
-// its loads are already in flight while it computes.
-constexpr int FC_CONSUMERS = 7;   // 8 warps in all: the whole register file (255 per thread) is available
+// candidates ahead; consumer pair p (two warps sharing one tile) takes the candidates p,
+// p + FC_PAIRS, ... of the range, so its loads are already in flight while it computes.  Splitting
+// each candidate over two warps halves the registers a warp needs (its half of the features and of
+// the Gram k-range) and doubles the warps that hide each other's latencies.
+constexpr int FC_PAIRS = 7;                    // consumer warp pairs, one candidate tile each
+constexpr int FC_CONSUMERS = 2 * FC_PAIRS;     // 15 warps in all: 136 registers per thread
 constexpr int FC_STAGES = 12;
-// A consumer's next candidate (i + consumers) reuses the stage of candidate i + consumers - stages,
-// which must already have been loaded (it is <= i) for the parity of its mbarrier wait to be
-// unambiguous.
-static_assert(FC_STAGES >= FC_CONSUMERS, "ring stages must cover the consumer warps");
+// A pair's next candidate (i + pairs) reuses the stage of candidate i + pairs - stages, which must
+// already have been loaded (it is <= i) for the parity of its mbarrier wait to be unambiguous.
+static_assert(FC_STAGES >= FC_PAIRS, "ring stages must cover the consumer pairs");
+
+// Barrier `id` over the 64 threads of a consumer pair.
+__device__ __forceinline__ void pair_sync(int id) { asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory"); }
+// The same barrier, returning the AND of v over the pair's threads (so both warps take one branch).
+__device__ __forceinline__ bool pair_and(int id, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, 64, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id)
+      : "memory");
+  return r != 0;
+}
 
 template <typename TIN>
 __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_kernel(
@@ -171,7 +186,7 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
   if (threadIdx.x == 0) {
     for (int k = 0; k < FC_STAGES; ++k) {
       mbar_init(&full[k], 1);
-      mbar_init(&empty[k], 32);
+      mbar_init(&empty[k], 64);   // both warps of a pair
     }
     abort_flag_s = 0;
     fence_barrier_init();
@@ -199,14 +214,22 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
     return;
   }
 
-  // ---------------- consumers ----------------
-  const int cw = warp - 1;
-  uint8_t* T = tiles + cw * (trows + NC_MAX) * pitch;   // [E^R rows ; E^C hi rows ; 0 pad] then E^C lo rows
+  // ---------------- consumers: warp pairs ----------------
+  // Pair pr takes candidates pr, pr + FC_PAIRS, ... of the range; warp hf of the pair owns features
+  // [64 hf, 64 hf + 64) of the token LCB and the k-half [64 hf, 64 hf + 64) of the Gram products,
+  // whose partial sums the two warps exchange through the pair's lo-row tile (free once the LCB
+  // has read it).  Named barrier 1 + pr synchronises the pair.
+  const int cw = warp - 1, pr = cw >> 1, hf = cw & 1;
+  const int bar_id = 1 + pr;
+  uint8_t* T = tiles + pr * (trows + NC_MAX) * pitch;   // [E^R rows ; E^C hi rows ; 0 pad] then E^C lo rows
   uint8_t* TL = T + trows * pitch;
+  float4* xb = reinterpret_cast<float4*>(TL);           // exchange: [warp][4 n-tile slots][32 lanes]
   const uint32_t sbase = smem_u32(T);
   const int ncols = n_R + n_C;
+  const int nt2 = (ncols + 15) / 16;                    // pairs of 8-wide Gram n-tiles
   const long long fsz = (long long)n_C * ncols;
   const int g8 = lane >> 2, t4 = lane & 3;
+  const int f0 = hf * (D / 2);                          // this warp's first feature
   // A operand of the token LCB (16 x 16 tokens): rows 0..o_C-1 hold P_CC, row 8 the query
   // generator's one-token weights, every other entry zero.  Constant for the whole kernel.
   uint32_t pa[4];
@@ -222,24 +245,25 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
     pa[2] = pack_bf16x2(A(g8, 2 * t4 + 8), A(g8, 2 * t4 + 9));
     pa[3] = pack_bf16x2(A(g8 + 8, 2 * t4 + 8), A(g8 + 8, 2 * t4 + 9));
   }
-  // Z^L row g8 and Z^Q (lanes with g8 == 0) of the current request, in the C-fragment layout:
-  // n-tile nt, columns nt*8 + 2*t4 and +1
-  float zl[D / 8][2], zq[D / 8][2];
+  // Z^L row g8 and Z^Q (lanes with g8 == 0) of the current request for this warp's features, in
+  // the C-fragment layout: n-tile nt, columns f0 + nt*8 + 2*t4 and +1
+  float zl[D / 16][2], zq[D / 16][2];
 #pragma unroll
-  for (int nt = 0; nt < D / 8; ++nt) zl[nt][0] = zl[nt][1] = zq[nt][0] = zq[nt][1] = 0.f;
+  for (int nt = 0; nt < D / 16; ++nt) zl[nt][0] = zl[nt][1] = zq[nt][0] = zq[nt][1] = 0.f;
   int staged = -1;
-  zero_rows(T + (n_R + n_C) * pitch, pitch, trows - (n_R + n_C), D);
-  zero_rows(TL + n_C * pitch, pitch, NC_MAX - n_C, D);
-  for (int i = cw; i < n; i += FC_CONSUMERS) {
+  if (hf == 0) zero_rows(T + (n_R + n_C) * pitch, pitch, trows - (n_R + n_C), D);
+  for (int i = pr; i < n; i += FC_PAIRS) {
     const int st = i % FC_STAGES;
-    if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (i / FC_STAGES) & 1, status, abort_flag))) break;
+    // both warps agree (and synchronise: the pair's reads of the previous candidate's tile and
+    // exchange buffer are done)
+    if (!pair_and(bar_id, mbar_wait(&full[st], (i / FC_STAGES) & 1, status, abort_flag))) break;
     const long long c = c0 + i;
     // this candidate's rows from the stage into the tile as bf16 (hi, and lo = E - hi for fp32
-    // inputs); lane j converts features 4j..4j+3, then the stage goes back to the producer
+    // inputs); warp hf converts rows hf, hf + 2, ...; lane j features 4j..4j+3
     const TIN* ec = reinterpret_cast<const TIN*>(ring + st * NC_MAX * D * sizeof(TIN));
-    __syncwarp();   // the previous candidate's tile reads are done
 #pragma unroll
-    for (int t = 0; t < NC_MAX; ++t) {
+    for (int k = 0; k < NC_MAX / 2; ++k) {
+      const int t = 2 * k + hf;
       if (t < n_C) {
         if constexpr (sizeof(TIN) == 4) {
           const float4 v = reinterpret_cast<const float4*>(ec + t * D)[lane];
@@ -251,70 +275,114 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
         } else {
           *reinterpret_cast<uint2*>(T + (n_R + t) * pitch + lane * 8) = reinterpret_cast<const uint2*>(ec + t * D)[lane];
         }
+      } else if constexpr (sizeof(TIN) == 4) {
+        // padding token rows of the lo tile meet zero LCB weights but must be finite: the exchange
+        // buffer of the previous candidate overwrote them
+        *reinterpret_cast<uint2*>(TL + t * pitch + lane * 8) = make_uint2(0, 0);
       }
     }
     const int r = stage_r[st];
     mbar_arrive(&empty[st]);
-    if (r < 0 || r >= B_R) {
-      if (lane == 0) set_status(status, ROCS_ERR_INDEX);
+    if (r < 0 || r >= B_R) {   // the same r for both warps: both skip
+      if (lane == 0 && hf == 0) set_status(status, ROCS_ERR_INDEX);
       continue;
     }
     if (r != staged) {
-      // a new request run: its rows into the tile, its Z^L and Z^Q rows into registers
-      __syncwarp();
-      stage_rows(T, pitch, E_R + (long long)r * n_R * D, n_R, D);
+      // a new request run: its rows into the tile (warp hf rows hf, hf + 2, ...), this warp's
+      // Z^L and Z^Q columns into registers
+      const int nrw = (n_R - hf + 1) / 2;
+      for (int k = lane; k < nrw * (D / 8); k += 32) {
+        const int rr = hf + 2 * (k / (D / 8)), v = k % (D / 8);
+        *reinterpret_cast<uint4*>(T + rr * pitch + v * 16) = load8_as_bf16(E_R + ((long long)r * n_R + rr) * D + v * 8);
+      }
 #pragma unroll
-      for (int nt = 0; nt < D / 8; ++nt) {
+      for (int nt = 0; nt < D / 16; ++nt) {
         if (g8 < o_C) {
-          const float2 z = __ldg(reinterpret_cast<const float2*>(ZL + ((long long)r * o_C + g8) * D + nt * 8 + 2 * t4));
+          const float2 z = __ldg(reinterpret_cast<const float2*>(ZL + ((long long)r * o_C + g8) * D + f0 + nt * 8 + 2 * t4));
           zl[nt][0] = z.x;
           zl[nt][1] = z.y;
         }
         if (tC != nullptr && g8 == 0) {
-          const float2 z = __ldg(reinterpret_cast<const float2*>(ZQ + (long long)r * D + nt * 8 + 2 * t4));
+          const float2 z = __ldg(reinterpret_cast<const float2*>(ZQ + (long long)r * D + f0 + nt * 8 + 2 * t4));
           zq[nt][0] = z.x;
           zq[nt][1] = z.y;
         }
       }
       staged = r;
     }
-    __syncwarp();
-    // token LCB on the tensor cores: [P_CC ; p_CC] (16 x 16) times E^C (16 tokens x 128), the
-    // fp32 embeddings as hi + lo bf16 parts
-    float acc[D / 8][4];
+    pair_sync(bar_id);   // the tile is complete
+    {
+      // token LCB on the tensor cores for this warp's 64 features: [P_CC ; p_CC] (16 x 16) times
+      // E^C (16 tokens x 64), the fp32 embeddings as hi + lo bf16 parts
+      float acc[D / 16][4];
 #pragma unroll
-    for (int nt = 0; nt < D / 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+      for (int nt = 0; nt < D / 16; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
 #pragma unroll
-    for (int p = 0; p < D / 16; ++p) {
-      uint32_t b[4];
-      load_b_frag_kmajor_x2(sbase, pitch, n_R, p * 16, b);
-      mma_bf16_16816(acc[2 * p], pa, b[0], b[1]);
-      mma_bf16_16816(acc[2 * p + 1], pa, b[2], b[3]);
-      if constexpr (sizeof(TIN) == 4) {
-        load_b_frag_kmajor_x2(smem_u32(TL), pitch, 0, p * 16, b);
+      for (int p = 0; p < D / 32; ++p) {
+        uint32_t b[4];
+        load_b_frag_kmajor_x2(sbase, pitch, n_R, f0 + p * 16, b);
         mma_bf16_16816(acc[2 * p], pa, b[0], b[1]);
         mma_bf16_16816(acc[2 * p + 1], pa, b[2], b[3]);
+        if constexpr (sizeof(TIN) == 4) {
+          load_b_frag_kmajor_x2(smem_u32(TL), pitch, 0, f0 + p * 16, b);
+          mma_bf16_16816(acc[2 * p], pa, b[0], b[1]);
+          mma_bf16_16816(acc[2 * p + 1], pa, b[2], b[3]);
+        }
+      }
+      // L^C = Z^L + P_CC E^C (fp32), row g8 of every n-tile
+      if (g8 < o_C) {
+        float* lp = L_C + (c * o_C + g8) * (long long)D + f0 + 2 * t4;
+#pragma unroll
+        for (int nt = 0; nt < D / 16; ++nt)
+          *reinterpret_cast<float2*>(lp + nt * 8) = make_float2(acc[nt][0] + zl[nt][0], acc[nt][1] + zl[nt][1]);
+      }
+      // t^C = Z^Q + p_CC E^C as a bf16 hi/lo pair (row 8 of the fragment: lanes with g8 == 0)
+      if (tC != nullptr && g8 == 0) {
+        __nv_bfloat16* tp = tC + c * 2LL * D + f0 + 2 * t4;
+#pragma unroll
+        for (int nt = 0; nt < D / 16; ++nt) {
+          const float v0 = acc[nt][2] + zq[nt][0], v1 = acc[nt][3] + zq[nt][1];
+          const uint32_t h = pack_bf16x2(v0, v1);
+          *reinterpret_cast<uint32_t*>(tp + nt * 8) = h;
+          *reinterpret_cast<uint32_t*>(tp + D + nt * 8) = pack_bf16x2(v0 - bf16_lo(h), v1 - bf16_hi(h));
+        }
       }
     }
-    // L^C = Z^L + P_CC E^C (fp32), row g8 of every n-tile
-    if (g8 < o_C) {
-      float* lp = L_C + (c * o_C + g8) * (long long)D + 2 * t4;
+    // F^C = E^C [E^R ; E^C]^T: this warp's k-half for every n-tile, then the pair exchange; warp hf
+    // finishes the n-tiles nt with nt % 2 == hf
+    float acc[8][4];
 #pragma unroll
-      for (int nt = 0; nt < D / 8; ++nt)
-        *reinterpret_cast<float2*>(lp + nt * 8) = make_float2(acc[nt][0] + zl[nt][0], acc[nt][1] + zl[nt][1]);
-    }
-    // t^C = Z^Q + p_CC E^C as a bf16 hi/lo pair (row 8 of the fragment: lanes with g8 == 0)
-    if (tC != nullptr && g8 == 0) {
-      __nv_bfloat16* tp = tC + c * 2LL * D + 2 * t4;
+    for (int q = 0; q < 8; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.f;
 #pragma unroll
-      for (int nt = 0; nt < D / 8; ++nt) {
-        const float v0 = acc[nt][2] + zq[nt][0], v1 = acc[nt][3] + zq[nt][1];
-        const uint32_t h = pack_bf16x2(v0, v1);
-        *reinterpret_cast<uint32_t*>(tp + nt * 8) = h;
-        *reinterpret_cast<uint32_t*>(tp + D + nt * 8) = pack_bf16x2(v0 - bf16_lo(h), v1 - bf16_hi(h));
+    for (int k0 = 0; k0 < D / 2; k0 += 16) {
+      uint32_t a[4];
+      load_a_frag(sbase, pitch, n_R, f0 + k0, a);
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        if (p < nt2) {
+          uint32_t b[4];
+          load_b_frag_nmajor_x2(sbase, pitch, p * 16, f0 + k0, b);
+          mma_bf16_16816(acc[2 * p], a, b[0], b[1]);
+          mma_bf16_16816(acc[2 * p + 1], a, b[2], b[3]);
+        }
       }
     }
-    gram_tile(sbase, pitch, n_R, n_C, ncols, D, F_C, 2, c * fsz * 2, ncols, fsz);
+    if constexpr (sizeof(TIN) == 4) pair_sync(bar_id);   // both warps are done reading the lo rows
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (q < 2 * nt2 && (q & 1) != hf) xb[(hf * 4 + (q >> 1)) * 32 + lane] = make_float4(acc[q][0], acc[q][1], acc[q][2], acc[q][3]);
+    pair_sync(bar_id);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (q < 2 * nt2 && (q & 1) == hf && q * 8 < ncols) {
+        const float4 o = xb[((1 - hf) * 4 + (q >> 1)) * 32 + lane];
+        acc[q][0] += o.x;
+        acc[q][1] += o.y;
+        acc[q][2] += o.z;
+        acc[q][3] += o.w;
+        store_c_frag(F_C, 2, c * fsz * 2, ncols, 0, q * 8, n_C, ncols, acc[q], fsz);
+      }
+    }
   }
 }
 
@@ -539,7 +607,7 @@ rocs_status fused_launch(rocs_context* ctx, const TIN* E_R, const TIN* E_C, cons
   const int D = 128;
   const int pitch = D * 2 + 16;
   const int trows = fm_trows(n_R, n_C);
-  const size_t smem = (size_t)FC_STAGES * NC_MAX * D * sizeof(TIN) + (size_t)FC_CONSUMERS * (trows + NC_MAX) * pitch;
+  const size_t smem = (size_t)FC_STAGES * NC_MAX * D * sizeof(TIN) + (size_t)FC_PAIRS * (trows + NC_MAX) * pitch;
   if (n_C > NC_MAX || o_C > LCB_OMAX_F || smem > 220 * 1024) {
     set_error("fused candidate pass: unsupported n_C=%d o_C=%d", n_C, o_C);
     return ROCS_ERR_UNSUPPORTED;

@@ -69,6 +69,19 @@ def test_forward_glm_stack(R):
     check_bf16(host(out["E_C"][:case.B_C]), ref["E_C"], what="E_C")
 
 
+def test_forward_glm_stack_narrow_candidates(R):
+    """8 candidate and 24 request embeddings: the fused candidate pass then has padding token rows
+    (n_C < 16) and four 8-wide Gram column tiles; two GLM layers, fp32 then bf16 stream."""
+    g = synth.GLMShape(n_R=24, n_C=8, hidden=256, fm_out_R=12, lcb_out_R=12, fm_out_C=4, lcb_out_C=4, layers=2)
+    case = synth.ModelCase("cfg3", np.asarray([5, 0, 37, 120], np.int32), 3, g, None, None)
+    x, W = synth.model_inputs(case), synth.model_weights(case)
+    out = run_forward(R, case, x, W)
+    _, m = O.segments(case.counts)
+    ref = O.forward_cfg3(case, x, W, m)
+    check_bf16(host(out["E_R"]), ref["E_R"], what="E_R")
+    check_bf16(host(out["E_C"][:case.B_C]), ref["E_C"], what="E_C")
+
+
 def test_forward_glm_invariant_on_gpu(R):
     case = synth.model_cfg3(B_R=2, counts=[9, 4])
     x, W = synth.model_inputs(case), synth.model_weights(case)
