@@ -170,6 +170,7 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
   __shared__ float sQ[64];
   __shared__ __align__(8) uint64_t full[FC_STAGES], empty[FC_STAGES];
   __shared__ int stage_r[FC_STAGES];   // request index of the candidate in each stage
+  __shared__ int stage_c[FC_STAGES];   // the candidate (index in the range) each stage was last loaded for
   __shared__ int abort_flag_s;
   volatile int* abort_flag = &abort_flag_s;
 
@@ -203,6 +204,7 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
         const int r = req_idx[c0 + i];   // loaded ahead of the consumers
         if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1, status, abort_flag)) break;
         stage_r[st] = r;
+        stage_c[st] = i;
         mbar_arrive_expect_tx(&full[st], stage_bytes);
         bulk_load(ring + st * NC_MAX * D * sizeof(TIN), E_C + (c0 + i) * (long long)n_C * D, stage_bytes, &full[st]);
         issued = i + 1;
@@ -254,9 +256,33 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
   if (hf == 0) zero_rows(T + (n_R + n_C) * pitch, pitch, trows - (n_R + n_C), D);
   for (int i = pr; i < n; i += FC_PAIRS) {
     const int st = i % FC_STAGES;
+    // Candidate i's rows in stage st.  A pair waits only on every FC_PAIRS-th candidate, so the
+    // phase parity alone is ambiguous if the stage's previous load (candidate i - FC_STAGES) were
+    // still landing: then the completed phase before it has the same parity.  The stage's tag is
+    // set to i only once that previous phase has completed and been consumed; after it reads i,
+    // a second wait on the same parity can only mean candidate i's own phase.
+    bool got = true;
+    {
+      volatile int* tag = stage_c;
+      const long long t0 = clock64();
+      while (true) {
+        got = mbar_wait(&full[st], (i / FC_STAGES) & 1, status, abort_flag);
+        if (!got) break;
+        if (tag[st] == i) {
+          got = mbar_wait(&full[st], (i / FC_STAGES) & 1, status, abort_flag);
+          break;
+        }
+        if (clock64() - t0 > kWaitBudgetCycles) {
+          set_status(status, ROCS_ERR_DEVICE_TIMEOUT);
+          *abort_flag = 1;
+          got = false;
+          break;
+        }
+      }
+    }
     // both warps agree (and synchronise: the pair's reads of the previous candidate's tile and
     // exchange buffer are done)
-    if (!pair_and(bar_id, mbar_wait(&full[st], (i / FC_STAGES) & 1, status, abort_flag))) break;
+    if (!pair_and(bar_id, got)) break;
     const long long c = c0 + i;
     // this candidate's rows from the stage into the tile as bf16 (hi, and lo = E - hi for fp32
     // inputs); warp hf converts rows hf, hf + 2, ...; lane j features 4j..4j+3

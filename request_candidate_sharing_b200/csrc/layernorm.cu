@@ -230,9 +230,10 @@ rocs_status dispatch(const void* X1, int w1, long long ld1, const void* X2, long
 // ---------------------------------------------------------------------------------------------
 constexpr int LN_CONSUMERS = 8;
 constexpr int LN_STAGES = 8;
-// a consumer's next block (b + consumers) reuses the stage of block b + consumers - stages, which
-// must already have been loaded for the parity of its mbarrier wait to be unambiguous
-static_assert(LN_STAGES >= LN_CONSUMERS, "ring stages must cover the consumer warps");
+// Consumer warp w takes blocks w, w + LN_CONSUMERS, ...; with as many stages as consumers every
+// one of them lands in stage w, so each warp waits on every phase of its own stage's barrier in
+// order and the phase parity is never ambiguous.
+static_assert(LN_STAGES == LN_CONSUMERS, "each consumer warp owns one ring stage");
 constexpr int LN_STAGE_BYTES = 16384;
 
 template <typename T>
