@@ -170,9 +170,9 @@ rocs_status attention_best(rocs_context* ctx, bool streaming_fallback, const voi
                            const void* K, const void* V, long long ldkv, const int32_t* offsets, int B_R,
                            long long rows, int L, int H, int d_h, float scale, void* O, long long ldo, int out_bf16,
                            void* O2, long long ldo2, cudaStream_t s, const int32_t* kv_len = nullptr,
-                           int q_by_kv = 0) {
+                           int q_by_kv = 0, const int32_t* order = nullptr) {
   rocs_status st = launch_attention_tc(ctx, Q, ldq, q_split, K, V, ldkv, (long long)B_R * L, offsets, B_R, rows, L, H,
-                                       d_h, scale, O, ldo, out_bf16, O2, ldo2, s, nullptr, kv_len, q_by_kv);
+                                       d_h, scale, O, ldo, out_bf16, O2, ldo2, s, nullptr, kv_len, q_by_kv, order);
   if (st != ROCS_ERR_UNSUPPORTED) return st;
   if (!streaming_fallback) {
     st = launch_attention(ctx, Q, ldq, q_split, K, V, ldkv, (long long)L * ldkv, offsets, B_R, rows, L, H, d_h, scale,
@@ -630,7 +630,7 @@ namespace rocs {
 namespace {
 
 struct UnsortedPlan {
-  int32_t *perm = nullptr, *offsets = nullptr, *H = nullptr;
+  int32_t *perm = nullptr, *offsets = nullptr, *H = nullptr, *order = nullptr;
   void *Qs = nullptr, *Os = nullptr;
   size_t bytes = 0;
 };
@@ -641,6 +641,7 @@ UnsortedPlan plan_unsorted(int B_R, long long rows, long long qrow_bytes, long l
   p.perm = (int32_t*)c.take((size_t)rows * 4 + 4);
   p.offsets = (int32_t*)c.take((size_t)(B_R + 1) * 4);
   p.H = (int32_t*)c.take((size_t)plan_sort(B_R, rows).h_ints * 4 + 4);
+  if (B_R <= kRequestOrderMax) p.order = (int32_t*)c.take((size_t)B_R * 4);
   if (qrow_bytes > 0) {
     p.Qs = c.take((size_t)(rows * qrow_bytes) + 16);
     p.Os = c.take((size_t)(rows * orow_bytes) + 16);
@@ -720,14 +721,16 @@ extern "C" rocs_status rocs_dca_cross_attn_unsorted(rocs_handle_t h, const void*
   // sort by request (stable), gather the query rows into that order, attend on the segment path,
   // and write every valid row at the caller's position
   ROCS_TRY(launch_sort_by_request(h, req_idx, B_R, rows, p.perm, p.offsets, p.H, s));
+  if (p.order != nullptr) ROCS_TRY(launch_request_order(p.offsets, B_R, p.order, s));
   ROCS_TRY(launch_gather_rows(Q, dm * 2, p.perm, rows, (int)(dm * 2), p.Qs, dm * 2, s));
   // the tcgen05 kernel writes each row straight to its caller position (out_rows = perm); the
   // other kernels write the grouped order, which is then scattered
   const rocs_status st = launch_attention_tc(h, p.Qs, dm, 0, K, V, dm, (long long)B_R * L, p.offsets, B_R, rows, L,
-                                             H, d_h, scale, O, ld_O, out == ROCS_BF16, nullptr, 0, s, p.perm, kv_len);
+                                             H, d_h, scale, O, ld_O, out == ROCS_BF16, nullptr, 0, s, p.perm, kv_len, 0,
+                                             p.order);
   if (st != ROCS_ERR_UNSUPPORTED) return st;
   ROCS_TRY(attention_best(h, true, p.Qs, dm, 0, K, V, dm, p.offsets, B_R, rows, L, H, d_h, scale, p.Os, dm,
-                          out == ROCS_BF16, nullptr, 0, s, kv_len));
+                          out == ROCS_BF16, nullptr, 0, s, kv_len, 0, p.order));
   return launch_scatter_rows(p.Os, dm * es, p.perm, p.offsets + B_R, rows, (int)(dm * es), O, ld_O * es, s);
 }
 
@@ -888,6 +891,7 @@ struct FwdPlan {
   void *xR, *xC, *h1, *h2;
   float* Zs;
   int* ikbo_flags;   // completion flags of the fused IKBO launches (reused, zeroed by each)
+  int32_t* order = nullptr;   // requests by descending candidate count (the candidate attention's CTA order)
   size_t bytes;
 };
 
@@ -933,6 +937,7 @@ FwdPlan plan_forward(const rocs_model_desc* m, void* ws, bool own_offsets, bool 
     } else {
       p.ar_scratch = c.take(attention_req_absorbed_scratch(m->B_R, m->L));
     }
+    if (m->B_R <= kRequestOrderMax) p.order = (int32_t*)c.take((size_t)m->B_R * 4);
     p.KC = c.take(rowsL * m->d * 2);
     p.VC = c.take(rowsL * m->d * 2);
     if (m->dca_query_source == 0) {
@@ -1031,6 +1036,7 @@ rocs_status forward_launches(rocs_handle_t h, const rocs_model_desc* m, const ro
   // a0: segment bookkeeping
   SiteLabel site_fwd("fwd");
   ROCS_TRY(launch_segments(h, in->counts, BR, offsets, req_idx, BC, s));
+  if (p.order != nullptr) ROCS_TRY(launch_request_order(offsets, BR, p.order, s));
   ROCS_TRY(launch_iota(p.iota1, BR + 1, 1, s));
 
   const long long wr = (long long)m->n_R * m->D, wc = (long long)m->n_C * m->D;
@@ -1155,7 +1161,7 @@ rocs_status forward_launches(rocs_handle_t h, const rocs_model_desc* m, const ro
       {
         SiteLabel s_xc("xattn.cand");
         ROCS_TRY(attention_best(h, true, p.QC, d2, 1, p.KC, p.VC, m->d, offsets, BR, BC, m->L, m->H, dh, scale, dC,
-                                ldC, 0, xC2, xc, s, in->hist_len));
+                                ldC, 0, xC2, xc, s, in->hist_len, 0, p.order));
       }
       if (m->dca_query_source == 0) {
         if (out->A_R)

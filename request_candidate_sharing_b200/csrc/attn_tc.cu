@@ -52,6 +52,7 @@ struct AttnTcParams {
   const int32_t* out_rows;   // optional: query row q is written to output row out_rows[q]
   const int32_t* kv_len;     // optional: request r has kv_len[r] keys (1..L), the rest are padding
   int q_by_kv;               // with kv_len: request r's queries are also only its first kv_len[r] rows
+  const int32_t* order;      // optional: CTA group b serves request order[b] (a permutation; heaviest first)
   int* status;
 };
 
@@ -199,8 +200,9 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
   constexpr uint32_t IDESC_O = idesc_bf16(TQ, DH, true);
   constexpr uint32_t IDESC_L = idesc_bf16(TQ, 16, false);
 
-  const int r = blockIdx.x / P.H;
-  const int h = blockIdx.x - r * P.H;
+  const int rb = blockIdx.x / P.H;
+  const int h = blockIdx.x - rb * P.H;
+  const int r = P.order != nullptr ? P.order[rb] : rb;
   const long long q0 = P.offsets[r];
   long long q1 = P.offsets[r + 1];
   if (q0 < 0 || q1 < q0 || q1 > P.rows) {
@@ -624,7 +626,7 @@ rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq,
                                 const void* V, long long ldkv, long long kv_rows, const int32_t* offsets, int B_R,
                                 long long rows, int L, int H, int d_h, float scale, void* O, long long ldo,
                                 int out_bf16, void* O2, long long ldo2, cudaStream_t s, const int32_t* out_rows,
-                                const int32_t* kv_len, int q_by_kv) {
+                                const int32_t* kv_len, int q_by_kv, const int32_t* order) {
   if (B_R == 0 || rows == 0) return ROCS_OK;
   if ((d_h != 32 && d_h != 64) || L < 1 || (long long)L * d_h > 32768 || (L + TK - 1) / TK > AT_MAX_KB ||
       ((uintptr_t)Q & 15) || ((uintptr_t)K & 15) || ((uintptr_t)V & 15) || ldq % 8 || ldkv % 8 ||
@@ -657,6 +659,7 @@ rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq,
   P.out_rows = out_rows;
   P.kv_len = kv_len;
   P.q_by_kv = kv_len != nullptr && q_by_kv ? 1 : 0;
+  P.order = order;
   P.status = ctx->d_status;
   LaunchTimer lt_("attn_tc", s);
   const bool rag = kv_len != nullptr;

@@ -138,6 +138,11 @@ struct SortPlan {
 SortPlan plan_sort(int B_R, long long B_C);
 rocs_status launch_sort_by_request(rocs_context* ctx, const int32_t* req_idx, int B_R, long long B_C, int32_t* perm,
                                    int32_t* offsets, int32_t* H, cudaStream_t s);
+// order[k] = the request of rank k by descending query count offsets[r+1] - offsets[r] (ties by
+// index), for B_R <= kRequestOrderMax.  Launching a request-per-CTA kernel in this order puts the
+// longest CTAs first, so the shortest ones fill the last wave.
+constexpr int kRequestOrderMax = 2048;
+rocs_status launch_request_order(const int32_t* offsets, int B_R, int32_t* order, cudaStream_t s);
 // dst[k] = src[perm[k]] for k < n (rows of row_bytes, a multiple of 16; 16-byte aligned rows)
 rocs_status launch_gather_rows(const void* src, long long ld_src_bytes, const int32_t* perm, long long n,
                                int row_bytes, void* dst, long long ld_dst_bytes, cudaStream_t s);
@@ -224,7 +229,7 @@ rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq,
                                 long long rows, int L, int H, int d_h, float scale, void* O, long long ldo,
                                 int out_bf16, void* O2, long long ldo2, cudaStream_t s,
                                 const int32_t* out_rows = nullptr, const int32_t* kv_len = nullptr,
-                                int q_by_kv = 0);
+                                int q_by_kv = 0, const int32_t* order = nullptr);
 
 rocs_status launch_score_head(const void* X, long long ldx, long long rows, int K, const void* w,
                               const float* b, float* out, cudaStream_t s);

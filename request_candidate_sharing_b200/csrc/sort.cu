@@ -306,4 +306,40 @@ rocs_status launch_scatter_rows(const void* src, long long ld_src_bytes, const i
   return cuda_check(cudaGetLastError(), "scatter_rows_kernel");
 }
 
+// Requests by descending query count, ties by index: order[k] is the request of rank k.  The rank of
+// request r counts the requests that precede it in that strict total order, so order is a
+// permutation of [0, B_R) whatever the offsets hold.  One thread per request, the counts staged
+// 256 at a time in shared memory: O(B_R^2) comparisons, for up to kRequestOrderMax requests.
+static __global__ void __launch_bounds__(256) request_order_kernel(const int32_t* __restrict__ offsets, int B_R,
+                                                                   int32_t* __restrict__ order) {
+  __shared__ int keys[256];
+  const int r = blockIdx.x * 256 + threadIdx.x;
+  const int mine = r < B_R ? offsets[r + 1] - offsets[r] : 0;
+  int rank = 0;
+  for (int s0 = 0; s0 < B_R; s0 += 256) {
+    const int j = s0 + threadIdx.x;
+    keys[threadIdx.x] = j < B_R ? offsets[j + 1] - offsets[j] : 0;
+    __syncthreads();
+    const int n = B_R - s0 < 256 ? B_R - s0 : 256;
+    if (r < B_R)
+      for (int k = 0; k < n; ++k) {
+        const int key = keys[k];
+        rank += (key > mine) || (key == mine && s0 + k < r);
+      }
+    __syncthreads();
+  }
+  if (r < B_R) order[rank] = r;
+}
+
+rocs_status launch_request_order(const int32_t* offsets, int B_R, int32_t* order, cudaStream_t s) {
+  if (B_R <= 0) return ROCS_OK;
+  if (B_R > kRequestOrderMax) {
+    set_error("request order: %d requests (at most %d)", B_R, kRequestOrderMax);
+    return ROCS_ERR_UNSUPPORTED;
+  }
+  LaunchTimer lt_("request_order", s);
+  request_order_kernel<<<(B_R + 255) / 256, 256, 0, s>>>(offsets, B_R, order);
+  return cuda_check(cudaGetLastError(), "request_order_kernel");
+}
+
 }  // namespace rocs
