@@ -157,6 +157,27 @@ def algo_work(case, label: str):
     return None
 
 
+def gpu_local_cpus(dev) -> set:
+    """The CPUs of the GPU's own NUMA node (sysfs local_cpulist of its PCI function) that this
+    process may run on; empty when unknown."""
+    import torch
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        bdf = f"{p.pci_domain_id:04x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+        with open(f"/sys/bus/pci/devices/{bdf}/local_cpulist") as f:
+            text = f.read().strip()
+        cpus = set()
+        for part in text.split(","):
+            if "-" in part:
+                a, b = part.split("-")
+                cpus.update(range(int(a), int(b) + 1))
+            elif part:
+                cpus.add(int(part))
+        return cpus & os.sched_getaffinity(0)
+    except (OSError, ValueError, AttributeError, RuntimeError):
+        return set()
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -466,6 +487,12 @@ def run_librocs(args, rank, world, local):
     value = cands / (ms_max / 1e3)
 
     # ---- end-to-end through the same call with host buffers ----
+    # the pinned buffers are allocated (and their pages first touched) by a thread bound to the
+    # GPU's local CPUs, so the copy engine reads memory of the GPU's own NUMA node
+    old_aff = os.sched_getaffinity(0)
+    local = gpu_local_cpus(dev)
+    if local:
+        os.sched_setaffinity(0, local)
     host = {k: v.cpu().pin_memory() for k, v in xd.items()}
     counts_h = counts_d.cpu().pin_memory()
     hl_h = hl_d.cpu().pin_memory() if hl_d is not None else None
@@ -474,6 +501,8 @@ def run_librocs(args, rank, world, local):
         (hl_h.numel() * 4 if hl_h is not None else 0)
     res = score if case.scoring is not None else outE[1]
     res_h = torch.empty_like(res, device="cpu").pin_memory()
+    if local:
+        os.sched_setaffinity(0, old_aff)
     d2h = res.numel() * res.element_size()
 
     # two device input sets: step k+1's inputs are copied (copy stream) while step k computes;
@@ -568,7 +597,9 @@ def run_librocs(args, rank, world, local):
                                  "(roofline): the same steps again with direct launches and per-launch CUDA events",
                        "e2e_pipelining": "two device input sets: step k+1's host-to-device copy (pinned, copy "
                                          "stream) overlaps step k's forward; every step's inputs are copied and "
-                                         "its scores read back inside the timed region"},
+                                         "its scores read back inside the timed region",
+                       "e2e_host_buffers": (f"pinned, allocated from the GPU's NUMA node ({len(local)} local CPUs)"
+                                            if local else "pinned (the GPU's NUMA node is unknown)")},
             "roofline": top,
             "e2e": {"value": round(e2e_value, 1), "unit": "candidates/s", "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": int(d2h)},
