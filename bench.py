@@ -450,7 +450,7 @@ def run_librocs(args, rank, world, local):
     small = in_bytes < (256 << 20)
     if small:
         flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-        ms = 0.0
+        step_ms = []
         for _ in range(args.steps):
             flush.fill_(1)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -458,17 +458,20 @@ def run_librocs(args, rank, world, local):
             step()
             e1.record(stream)
             torch.cuda.synchronize(dev)
-            ms += e0.elapsed_time(e1)
+            step_ms.append(e0.elapsed_time(e1))
+        ms = sum(step_ms)
         barrier(world)
     else:
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
+        # an event after every step: the region is first to last, each step the gap between two
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+        evs[0].record(stream)
+        for i in range(args.steps):
             step()
-        e1.record(stream)
+            evs[i + 1].record(stream)
         torch.cuda.synchronize(dev)
         barrier(world)
-        ms = e0.elapsed_time(e1)
+        ms = evs[0].elapsed_time(evs[-1])
+        step_ms = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
     # per-kernel report: the same steps again with per-launch CUDA events (direct launches; the
     # timed region above replays the forward's CUDA graph)
     R.rocs_timing_start(200 * args.steps + 64)
@@ -601,6 +604,9 @@ def run_librocs(args, rank, world, local):
                        "e2e_host_buffers": (f"pinned, allocated from the GPU's NUMA node ({len(local)} local CPUs)"
                                             if local else "pinned (the GPU's NUMA node is unknown)")},
             "roofline": top,
+            "step_ms": {"median": round(statistics.median(step_ms), 4),
+                        "p90": round(sorted(step_ms)[min(len(step_ms) - 1, int(math.ceil(0.9 * len(step_ms))) - 1)], 4),
+                        "n": len(step_ms), "rank": 0},
             "e2e": {"value": round(e2e_value, 1), "unit": "candidates/s", "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": int(d2h)},
             "gpu_launches": int(launches),
