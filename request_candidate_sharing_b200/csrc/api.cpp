@@ -896,8 +896,7 @@ struct FwdPlan {
 };
 
 FwdPlan plan_forward(const rocs_model_desc* m, void* ws, bool own_offsets, bool own_req) {
-  FwdPlan p;
-  memset(&p, 0, sizeof(p));
+  FwdPlan p{};
   Carver c(ws);
   const long long BR = m->B_R, BC = m->B_C;
   p.offsets = own_offsets ? (int32_t*)c.take((BR + 1) * 4) : nullptr;

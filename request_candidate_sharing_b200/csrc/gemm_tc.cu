@@ -678,8 +678,7 @@ rocs_status launch_gemm_bf16(rocs_context* ctx, const GemmDesc* probs, int nprob
     return cuda_check(cudaGetLastError(), "gemm_tc_kernel launch");
   }
   // readers spin on tiles other CTAs publish: launch cooperatively (all CTAs resident)
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(THREADS);
   cfg.dynamicSmemBytes = SMEM_BYTES;
