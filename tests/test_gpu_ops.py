@@ -103,19 +103,28 @@ def test_linear_fp32_cfg1(R):
     ([129], 100, 36, 40, 300),        # K not a multiple of 8 -> alignment fix on the bf16 path
     ([5, 300], 512, 512, 0, 512),     # no request output (scoring-head form)
 ])
-def test_linear_integer_inputs_bit_exact(R, dtype_in, shape):
-    """Small integers: every product and partial sum is exact in fp32, so GPU == oracle bit for bit."""
+@pytest.mark.parametrize("out_dtype", [0, 1])
+def test_linear_integer_inputs_bit_exact(R, dtype_in, shape, out_dtype):
+    """Small integers: every product and partial sum is exact in fp32, so GPU == oracle bit for bit;
+    a bf16 output is then the oracle's value rounded to nearest even.  The output widths give the
+    bf16 store path odd chunk counts (136 -> 5 chunks of 32, 32 -> 1), boxes clipped at N (264, 40)
+    and rows that are not 16-byte multiples (300: element stores)."""
     from request_candidate_sharing_b200 import rocs
     counts, dRi, dCi, dRo, dCo = shape
     case = synth.LinearCase("int", np.asarray(counts, np.int32), dRi, dCi, dRo, dCo, "relu", dtype_in == 1, 7)
     x = synth.linear_inputs(case, integer=3)
     _, m = O.segments(case.counts)
-    YR, YC = _run_linear(R, case, x, m, dtype_in, rocs.ROCS_F32)
+    if dtype_in == rocs.ROCS_F32 and out_dtype == rocs.ROCS_BF16:
+        with pytest.raises(rocs.RocsError, match="fp32 path writes fp32 outputs"):   # host-checked
+            _run_linear(R, case, x, m, dtype_in, out_dtype)
+        return
+    YR, YC = _run_linear(R, case, x, m, dtype_in, out_dtype)
     rR, rC = O.glm_linear(x["X_R"], x["X_C"], m, x["W_RR"] if dRo else None, x["W_CR"], x["W_CC"],
                           x["b_R"] if dRo else None, x["b_C"], "relu")
+    expect = (lambda a: synth.bf16_round(a.astype(np.float32))) if out_dtype == 1 else (lambda a: a)
     if dRo:
-        assert np.array_equal(host(YR), rR)
-    assert np.array_equal(host(YC), rC)
+        assert np.array_equal(host(YR), expect(rR))
+    assert np.array_equal(host(YC), expect(rC))
 
 
 @pytest.mark.parametrize("out_dtype", [0, 1])
