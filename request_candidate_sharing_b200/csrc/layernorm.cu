@@ -224,16 +224,19 @@ rocs_status dispatch(const void* X1, int w1, long long ld1, const void* X2, long
 // ---------------------------------------------------------------------------------------------
 // Streaming variant for long row counts with contiguous rows (ld == width of every operand):
 // one CTA per SM walks a contiguous row range; one thread bulk-copies blocks of RB rows of the two
-// segments and the residual into a ring of shared-memory stages, LN_CONSUMERS warps normalise
+// segments and the residual into a ring of shared-memory stages, LnRing<NV>::DEPTH warps normalise
 // them (one row at a time per warp, lane j holding the float4 groups j, j + 32, ...) and write the
 // outputs straight from registers.  gamma/beta live in shared memory.
 // ---------------------------------------------------------------------------------------------
-constexpr int LN_CONSUMERS = 8;
-constexpr int LN_STAGES = 8;
-// Consumer warp w takes blocks w, w + LN_CONSUMERS, ...; with as many stages as consumers every
-// one of them lands in stage w, so each warp waits on every phase of its own stage's barrier in
-// order and the phase parity is never ambiguous.
-static_assert(LN_STAGES == LN_CONSUMERS, "each consumer warp owns one ring stage");
+// Ring depth = consumer warps = stages.  Consumer warp w takes blocks w, w + DEPTH, ...; with as
+// many stages as consumers every one of them lands in stage w, so each warp waits on every phase of
+// its own stage's barrier in order and the phase parity is never ambiguous.  Narrow rows (width
+// <= 256: 16 encoder rows per stage) run 12 deep, wide rows (a candidate row per stage) 8 deep:
+// 12 measured 16% faster for the former and 3% slower for the latter.
+template <int NV>
+struct LnRing {
+  static constexpr int DEPTH = NV <= 2 ? 12 : 8;
+};
 constexpr int LN_STAGE_BYTES = 16384;
 
 template <typename T>
@@ -250,7 +253,7 @@ __device__ __forceinline__ void ld4<__nv_bfloat16>(const __nv_bfloat16* p, float
 }
 
 template <typename TIN, typename TRES, typename TOUT, int NV>
-__global__ void __launch_bounds__(32 * (1 + LN_CONSUMERS), 1) layernorm_ring_kernel(
+__global__ void __launch_bounds__(32 * (1 + LnRing<NV>::DEPTH), 1) layernorm_ring_kernel(
     const TIN* __restrict__ X1, int w1, const TIN* __restrict__ X2, const TRES* __restrict__ R, long long rows,
     long long rows_per_block, int RB, const float* __restrict__ gamma, const float* __restrict__ beta, float eps,
     TOUT* __restrict__ Y, __nv_bfloat16* __restrict__ Y2, long long ldy2, int* status) {
@@ -260,7 +263,7 @@ __global__ void __launch_bounds__(32 * (1 + LN_CONSUMERS), 1) layernorm_ring_ker
   float* s_gamma = reinterpret_cast<float*>(ln_smem);
   float* s_beta = s_gamma + width;
   uint8_t* ring = ln_smem + 2 * width * sizeof(float);
-  __shared__ __align__(8) uint64_t full[LN_STAGES], empty[LN_STAGES];
+  __shared__ __align__(8) uint64_t full[LnRing<NV>::DEPTH], empty[LnRing<NV>::DEPTH];
   __shared__ int abort_flag_s;
   volatile int* abort_flag = &abort_flag_s;
 
@@ -277,7 +280,7 @@ __global__ void __launch_bounds__(32 * (1 + LN_CONSUMERS), 1) layernorm_ring_ker
     s_beta[i] = beta[i];
   }
   if (threadIdx.x == 0) {
-    for (int k = 0; k < LN_STAGES; ++k) {
+    for (int k = 0; k < LnRing<NV>::DEPTH; ++k) {
       mbar_init(&full[k], 1);
       mbar_init(&empty[k], 32);
     }
@@ -291,7 +294,7 @@ __global__ void __launch_bounds__(32 * (1 + LN_CONSUMERS), 1) layernorm_ring_ker
     if (lane == 0) {
       int issued = 0;
       for (int b = 0; b < nblk; ++b) {
-        const int st = b % LN_STAGES, use = b / LN_STAGES;
+        const int st = b % LnRing<NV>::DEPTH, use = b / LnRing<NV>::DEPTH;
         if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1, status, abort_flag)) break;
         const long long row = r0 + (long long)b * RB;
         const int nr = (int)(r1 - row < RB ? r1 - row : RB);
@@ -304,16 +307,16 @@ __global__ void __launch_bounds__(32 * (1 + LN_CONSUMERS), 1) layernorm_ring_ker
         if (br) bulk_load(sb + offr, R + row * width, br, &full[st]);
         issued = b + 1;
       }
-      for (int b = issued - LN_STAGES < 0 ? 0 : issued - LN_STAGES; b < issued; ++b)
-        mbar_wait(&full[b % LN_STAGES], (b / LN_STAGES) & 1, status, nullptr);
+      for (int b = issued - LnRing<NV>::DEPTH < 0 ? 0 : issued - LnRing<NV>::DEPTH; b < issued; ++b)
+        mbar_wait(&full[b % LnRing<NV>::DEPTH], (b / LnRing<NV>::DEPTH) & 1, status, nullptr);
     }
     return;
   }
 
   const int cw = warp - 1;
-  for (int b = cw; b < nblk; b += LN_CONSUMERS) {
-    const int st = b % LN_STAGES;
-    if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (b / LN_STAGES) & 1, status, abort_flag))) break;
+  for (int b = cw; b < nblk; b += LnRing<NV>::DEPTH) {
+    const int st = b % LnRing<NV>::DEPTH;
+    if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (b / LnRing<NV>::DEPTH) & 1, status, abort_flag))) break;
     const uint8_t* sb = ring + st * LN_STAGE_BYTES;
     const long long row0 = r0 + (long long)b * RB;
     const int nr = (int)(r1 - row0 < RB ? r1 - row0 : RB);
@@ -394,7 +397,7 @@ rocs_status run_ring(rocs_context* ctx, const void* X1, int w1, const void* X2, 
   constexpr int width = NV * 128;
   const int row_bytes = (int)(width * sizeof(TIN) + (R != nullptr ? width * sizeof(TRES) : 0));
   const int RB = LN_STAGE_BYTES / row_bytes;
-  const size_t smem = 2 * width * sizeof(float) + (size_t)LN_STAGES * LN_STAGE_BYTES;
+  const size_t smem = 2 * width * sizeof(float) + (size_t)LnRing<NV>::DEPTH * LN_STAGE_BYTES;
   static bool attr[64] = {false};
   if (ctx->device < 64 && !attr[ctx->device]) {
     rocs_status st = cuda_check(cudaFuncSetAttribute(layernorm_ring_kernel<TIN, TRES, TOUT, NV>,
@@ -407,7 +410,7 @@ rocs_status run_ring(rocs_context* ctx, const void* X1, int w1, const void* X2, 
   long long per_block = (rows + blocks - 1) / blocks;
   per_block = (per_block + RB - 1) / RB * RB;
   LaunchTimer lt_("layernorm", s);
-  layernorm_ring_kernel<TIN, TRES, TOUT, NV><<<(unsigned)blocks, 32 * (1 + LN_CONSUMERS), smem, s>>>(
+  layernorm_ring_kernel<TIN, TRES, TOUT, NV><<<(unsigned)blocks, 32 * (1 + LnRing<NV>::DEPTH), smem, s>>>(
       (const TIN*)X1, w1, (const TIN*)X2, (const TRES*)R, rows, per_block, RB, g, b, eps, (TOUT*)Y,
       (__nv_bfloat16*)Y2, ldy2, ctx->d_status);
   return cuda_check(cudaGetLastError(), "layernorm_ring_kernel");
