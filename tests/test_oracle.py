@@ -55,6 +55,19 @@ def test_sort_by_request_brute_force(m, B_R):
     assert offsets.tolist() == bounds
 
 
+def test_sort_by_request_is_a_stable_argsort():
+    """On random maps (invalid indices included) the oracle's counting sort equals a library stable
+    sort of the keys, with every index outside [0, B_R) keyed as B_R; the offsets are the keys'
+    left insertion points."""
+    g = np.random.default_rng(5)
+    for B_R, n in [(1, 50), (7, 1000), (300, 5000)]:
+        m = g.integers(-2, B_R + 2, size=n).astype(np.int32)
+        perm, offsets = O.sort_by_request(m, B_R)
+        keys = np.where((m >= 0) & (m < B_R), m, B_R)
+        assert np.array_equal(perm, np.argsort(keys, kind="stable"))
+        assert np.array_equal(offsets, np.searchsorted(np.sort(keys), np.arange(B_R + 1), side="left"))
+
+
 def test_sort_by_request_matches_segments_on_grouped_input():
     """Already grouped candidates: the identity permutation and exactly `segments`' offsets."""
     counts = np.asarray([3, 0, 5, 1, 0, 2], np.int32)
