@@ -33,28 +33,30 @@ def stream(seed: int, name: str, block: int = 0) -> np.random.Generator:
     return np.random.default_rng(np.random.SeedSequence([int(seed), _tensor_id(name), int(block)]))
 
 
+def _block(seed, name, shape, kind, a, b, bi) -> np.ndarray:
+    """Row block `bi` (rows bi*ROW_BLOCK ... up to ROW_BLOCK of them) of a drawn tensor."""
+    n0, inner = shape[0], shape[1:]
+    per_row = int(np.prod(inner)) if inner else 1
+    r0 = bi * ROW_BLOCK
+    nr = min(ROW_BLOCK, n0 - r0)
+    g = stream(seed, name, bi)
+    if kind == "normal":
+        v = g.standard_normal(nr * per_row, dtype=np.float64) * a
+    else:
+        v = g.uniform(a, b, nr * per_row)
+    return v.astype(np.float32).reshape((nr,) + inner)
+
+
 def _draw(seed, name, shape, kind, a, b, rows=None) -> np.ndarray:
     shape = tuple(int(s) for s in shape)
     n0 = shape[0]
     inner = shape[1:]
-    per_row = int(np.prod(inner)) if inner else 1
     nblocks = (n0 + ROW_BLOCK - 1) // ROW_BLOCK
-
-    def block(bi):
-        r0 = bi * ROW_BLOCK
-        nr = min(ROW_BLOCK, n0 - r0)
-        g = stream(seed, name, bi)
-        if kind == "normal":
-            v = g.standard_normal(nr * per_row, dtype=np.float64) * a
-        else:
-            v = g.uniform(a, b, nr * per_row)
-        return v.astype(np.float32).reshape((nr,) + inner)
-
     if rows is None:
         out = np.empty(shape, dtype=np.float32)
         for bi in range(nblocks):
             r0 = bi * ROW_BLOCK
-            out[r0:r0 + ROW_BLOCK] = block(bi)
+            out[r0:r0 + ROW_BLOCK] = _block(seed, name, shape, kind, a, b, bi)
         return out
     rows = np.asarray(rows, dtype=np.int64)
     out = np.empty((len(rows),) + inner, dtype=np.float32)
@@ -62,9 +64,17 @@ def _draw(seed, name, shape, kind, a, b, rows=None) -> np.ndarray:
     for i, r in enumerate(rows):
         bi = int(r) // ROW_BLOCK
         if bi not in cache:
-            cache[bi] = block(bi)
+            cache[bi] = _block(seed, name, shape, kind, a, b, bi)
         out[i] = cache[bi][int(r) - bi * ROW_BLOCK]
     return out
+
+
+def normal_blocks(seed: int, name: str, shape: Sequence[int], std: float = 1.0):
+    """Yields (first_row, rows) over the row blocks of `normal(seed, name, shape, std)`, in order,
+    so a tensor too large to hold twice on the host can be filled block by block."""
+    shape = tuple(int(s) for s in shape)
+    for bi in range((shape[0] + ROW_BLOCK - 1) // ROW_BLOCK):
+        yield bi * ROW_BLOCK, _block(seed, name, shape, "normal", float(std), None, bi)
 
 
 def normal(seed: int, name: str, shape: Sequence[int], std: float = 1.0, rows=None) -> np.ndarray:

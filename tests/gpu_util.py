@@ -76,3 +76,21 @@ def sample_candidates(counts, per_request: int, seed: int = 123) -> np.ndarray:
             idx.update(g.choice(n, size=min(n, extra + 2), replace=False).tolist())
         picks.extend(base + i for i in sorted(idx)[:max(per_request, 2)])
     return np.asarray(sorted(set(picks)), dtype=np.int64)
+
+
+def dev_normal_bf16(seed: int, name: str, shape, std: float = 1.0, keep_rows=None):
+    """The seeded N(0, std^2) tensor `synth.normal(seed, name, shape, std)` rounded to bf16, built
+    on cuda:0 one row block at a time (the full-size candidate batches are several GB).  With
+    `keep_rows` (sorted row indices) it also returns those rows' host values, taken from the same
+    blocks as they pass."""
+    import synth
+    out = torch.empty(tuple(shape), dtype=torch.bfloat16, device="cuda")
+    keep = None if keep_rows is None else np.asarray(keep_rows, np.int64)
+    kept = None if keep is None else np.empty((len(keep),) + tuple(shape[1:]), np.float32)
+    for r0, blk in synth.normal_blocks(seed, name, shape, std):
+        blk = synth.bf16_round(blk)
+        out[r0:r0 + len(blk)].copy_(torch.from_numpy(blk).to(torch.bfloat16))
+        if keep is not None:
+            sel = np.flatnonzero((keep >= r0) & (keep < r0 + len(blk)))
+            kept[sel] = blk[keep[sel] - r0]
+    return out if keep is None else (out, kept)

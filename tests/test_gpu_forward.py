@@ -271,3 +271,43 @@ def test_forward_end_to_end_full_size_sampled(R):
     for l in range(case.dca.layers):
         check_bf16(host(out["A_R"][l][qt]), ref["A_R"][l], what=f"A_R_{l} (sampled requests)")
         check_bf16(host(out["A_C"][l][rt]), ref["A_C"][l], what=f"A_C_{l} (sampled)")
+
+
+def test_forward_glm_stack_stated_size(R):
+    """The GLM-stack configuration at its stated size: 64 requests with U[100, 1000] candidates
+    each (seed 0), three layers of 32 | 16 embeddings of 128.  The GPU runs every candidate; the
+    oracle checks every request and four candidates of each request (its first and last among
+    them)."""
+    from tests.gpu_util import sample_candidates
+    case = synth.model_cfg3()
+    assert case.B_R == 64 and case.counts.min() >= 100 and case.counts.max() <= 1000
+    x, W = synth.model_inputs(case), synth.model_weights(case)
+    out = run_forward(R, case, x, W)
+    off, m = O.segments(case.counts)
+    assert np.array_equal(out["offsets"].cpu().numpy(), off)
+    rows = sample_candidates(case.counts, 4)
+    xs = dict(x, E_C=x["E_C"][rows])
+    ref = O.forward_cfg3(case, xs, W, m[rows])
+    rt = torch.from_numpy(rows).cuda()
+    check_bf16(host(out["E_R"]), ref["E_R"], what="E_R (every request)")
+    check_bf16(host(out["E_C"][rt]), ref["E_C"], what="E_C (sampled)")
+
+
+def test_forward_dca_stated_size(R):
+    """The DCA configuration at its stated size: 32 requests x 500 candidates, history L = 200,
+    d = 256, 4 heads, 2 encoder layers, 16 + 8 query embeddings of 256 (seed 0).  Every encoder
+    output and request attention output is checked, and four candidates of each request."""
+    from tests.gpu_util import sample_candidates
+    case = synth.model_cfg4()
+    assert (case.B_R, case.B_C, case.dca.L, case.dca.H) == (32, 16000, 200, 4)
+    x, W = synth.model_inputs(case), synth.model_weights(case)
+    out = run_forward(R, case, x, W)
+    _, m = O.segments(case.counts)
+    rows = sample_candidates(case.counts, 4)
+    xs = dict(x, Y_C=x["Y_C"][rows])
+    ref = O.forward_cfg4(case, xs, W, m[rows])
+    rt = torch.from_numpy(rows).cuda()
+    for l in range(case.dca.layers):
+        check_bf16(host(out["S"][l]), ref["S"][l], out_bf16=True, what=f"S_{l}")
+        check_bf16(host(out["A_R"][l]), ref["A_R"][l], what=f"A_R_{l}")
+        check_bf16(host(out["A_C"][l][rt]), ref["A_C"][l], what=f"A_C_{l} (sampled)")

@@ -181,18 +181,35 @@ def test_linear_bad_request_index_sets_status(R):
     assert not torch.all(YC[4] == -5.0)
 
 
-def test_linear_cfg2_sampled_full_size(R):
-    """IKBO sweep point N=256, d=1024 at full size (65536 candidates); oracle on a sample."""
+@pytest.mark.parametrize("N,d", [(N, d) for N in synth.CFG2_N for d in synth.CFG2_D])
+def test_linear_cfg2_every_point_sampled(R, N, d):
+    """Every IKBO sweep point at full size: 256 requests x N candidates, d_in = d_out = d, bf16 in
+    and out, ReLU.  The GPU runs the whole batch (up to 262,144 candidates at K = 4096); the oracle
+    checks every request output and four candidates of each request, its first and last among
+    them.  The candidate batch is the seeded draw the sweep in bench.py times."""
     from request_candidate_sharing_b200 import rocs
-    case = synth.linear_cfg2(256, 1024)
-    x = synth.linear_inputs(case)
-    _, m = O.segments(case.counts)
-    YR, YC = _run_linear(R, case, x, m, rocs.ROCS_BF16, rocs.ROCS_BF16)
+    from tests.gpu_util import dev_normal_bf16
+    case = synth.linear_cfg2(N, d)
     rows = sample_candidates(case.counts, 4)
-    rR, rC = O.glm_linear(x["X_R"], x["X_C"][rows], m[rows], x["W_RR"], x["W_CR"], x["W_CC"], x["b_R"], x["b_C"],
-                          "relu")
+    x = synth.linear_inputs(case, cand_rows=rows[:1])
+    _, m = O.segments(case.counts)
+    XC, x_rows = dev_normal_bf16(case.seed, "X_C", (case.B_C, d), keep_rows=rows)
+    assert np.array_equal(x_rows[:1], x["X_C"])        # the same seeded draw as the oracle's generator
+    x["X_C"] = x_rows
+    rt = torch.from_numpy(rows).cuda()
+    desc = rocs.IkboDesc(case.B_R, case.B_C, d, d, d, d, rocs.ROCS_BF16, rocs.ROCS_BF16, rocs.ACT[case.act])
+    nb = R.rocs_linear_ikbo_workspace(desc)
+    ws = torch.empty(max(nb, 16), dtype=torch.uint8, device="cuda")
+    t = {k: dev(x[k]) for k in ("X_R", "W_RR", "W_CR", "W_CC")}
+    YR = torch.full((case.B_R, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    YC = torch.full((case.B_C, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    R.rocs_linear_ikbo(desc, t["X_R"], XC, dev_i32(m), t["W_RR"], t["W_CR"], t["W_CC"],
+                       dev(x["b_R"], torch.float32), dev(x["b_C"], torch.float32), YR, YC, ws, nb, stream())
+    _status_ok(R)
+    assert not torch.isnan(YC).any(), "candidate rows left unwritten"
+    rR, rC = O.glm_linear(x["X_R"], x["X_C"], m[rows], x["W_RR"], x["W_CR"], x["W_CC"], x["b_R"], x["b_C"], "relu")
     check_bf16(host(YR), rR, out_bf16=True, what="Y_R")
-    check_bf16(host(YC[torch.from_numpy(rows).cuda()]), rC, out_bf16=True, what="Y_C sample")
+    check_bf16(host(YC[rt]), rC, out_bf16=True, what="Y_C sample")
 
 
 @pytest.mark.parametrize("counts,dRo,dCo,act,perm", [
