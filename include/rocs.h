@@ -162,10 +162,15 @@ rocs_status rocs_linear_ikbo_w8(rocs_handle_t handle, const rocs_ikbo_desc* desc
  *     (4 MiB) that every GPU loading the library keeps until the process exits.  Requests with
  *     B_R * d_C_out above that limit, or bf16 rows that would need the alignment fix
  *     (d_R_in or d_C_in not a multiple of 8), return ROCS_ERR_UNSUPPORTED with a message
- *     pointing to rocs_linear_ikbo.  The call never allocates or frees device memory.
+ *     pointing to rocs_linear_ikbo.  The call never calls an allocation or free routine.
  *   - Set-up: the first call on each device (with that device current, as for every call on
- *     the handle) looks up the array's device address once and caches it; make that first call
- *     before any stream capture.
+ *     the handle) looks up the array's device address once and caches it.  Under lazy module
+ *     loading (the CUDA 12 default) the driver loads the library's device code, and commits the
+ *     4 MiB array, at that first call: make it once per device as a warm-up, before serving and
+ *     before any stream capture; later calls allocate nothing.  A call from a context other than
+ *     the one of the first call looks the address up again in its own context.  Resetting the
+ *     device (cudaDeviceReset) while the library stays loaded is not supported: the cached
+ *     address may then no longer be the array's.
  *   - Sharing: all calls on a device use the same array, and it keeps the last call's Z.
  *     Z is fully rewritten before it is read, so nothing has to be cleared, but calls whose
  *     work overlaps on the GPU (different streams, or different host threads) race on it:
@@ -425,6 +430,32 @@ rocs_status rocs_set_graph_replay(rocs_handle_t handle, int32_t enable);
  * device status and leaves the affected rows unwritten.
  * Errors: ROCS_ERR_INVALID_ARG for a NULL handle or another value of enable. */
 rocs_status rocs_set_ikbo_fused(rocs_handle_t handle, int32_t enable);
+
+/* Test hook for the failure-detection path; off by default and not for production use.  The
+ * pages have no counterpart: it exists so that a test can make the fused IKBO launch's bounded
+ * completion-flag wait run out on purpose, without faulting or hanging the GPU.
+ * With flag_index >= 0, every later fused IKBO launch on this handle skips publishing completion
+ * flag `flag_index` (the request GEMM's tile in row block b and output column tile n has index
+ * b * n_tiles + n; with d_C_out <= 256 there is one column tile, so the index is the request
+ * block) and bounds each completion-flag wait by wait_budget_cycles SM clock cycles (clock64)
+ * instead of about 1 s.  The candidate tiles that gather Z rows from that request block then give
+ * up after the budget: ROCS_ERR_DEVICE_TIMEOUT is set in the device status, those candidate rows
+ * are left unwritten, and the kernel returns normally (its CTAs drain their copies and MMAs and
+ * release tensor memory), so the next call on the stream runs as usual.  flag_index = -1 turns the
+ * hook off and restores the default budget (wait_budget_cycles is then ignored).
+ * Errors: ROCS_ERR_INVALID_ARG for a NULL handle, flag_index < -1, or, with flag_index >= 0, a
+ * budget outside [1e3, 1e10] cycles. */
+rocs_status rocs_test_withhold_ikbo_flag(rocs_handle_t handle, int32_t flag_index, int64_t wait_budget_cycles);
+
+/* Measurement: the exponential throughput that bounds the DCA attention kernels (one exponential
+ * per score, [REV] §2.2 grouped cross-attention and the shared encoder).  The pages give no such
+ * rate.  Every thread of a grid that fills all SMs carries eight independent pairs of scores
+ * through the attention softmax's per-score steps: scale and shift on the packed FMA path, 2^x,
+ * packing to bf16 pairs; n_poly of every eight pairs (0..8) take the FMA-pipe polynomial, the rest
+ * MUFU ex2 (the attention kernels use n_poly = 3).  Writes the best of five timed launches as
+ * exponentials per second to *exp2_per_second.  Synchronises `stream`; allocates nothing.
+ * Errors: ROCS_ERR_INVALID_ARG (NULL handle or output, n_poly outside [0, 8]); ROCS_ERR_CUDA. */
+rocs_status rocs_probe_exp2_rate(rocs_handle_t handle, int32_t n_poly, double* exp2_per_second, void* stream);
 
 /* ------------------------------------------------------------------------------------------
  * Per-launch timing (tracing).  After rocs_timing_start(h, max_launches), every kernel the

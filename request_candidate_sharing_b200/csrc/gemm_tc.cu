@@ -69,6 +69,8 @@ struct Params {
   int interleave;     // 1: tile order (m block, problem, n block); 0: problem-major
   int n_per_m;        // sum of n_tiles over problems (interleave mode)
   int* status;
+  long long flag_budget;   // clock64 cycles a completion-flag wait may take
+  int withhold_flag;       // test hook: this completion flag is never published (-1: none)
 };
 
 __device__ __forceinline__ void decode_tile(const Params& P, int t, int& pi, int& mb, int& nb) {
@@ -87,15 +89,17 @@ __device__ __forceinline__ void decode_tile(const Params& P, int t, int& pi, int
   }
 }
 
-// Spin (bounded) until *flag >= target, with acquire ordering for the reads that follow.
-__device__ __forceinline__ bool wait_flag(const int* flag, int target, int* status, volatile int* abort_flag) {
+// Spin (bounded by `budget` cycles) until *flag >= target, with acquire ordering for the reads
+// that follow.
+__device__ __forceinline__ bool wait_flag(const int* flag, int target, long long budget, int* status,
+                                          volatile int* abort_flag) {
   const long long t0 = clock64();
   while (true) {
     int v;
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
     if (v >= target) return true;
     if (abort_flag && *abort_flag) return false;
-    if (clock64() - t0 > kWaitBudgetCycles) {
+    if (clock64() - t0 > budget) {
       set_status(status, ROCS_ERR_DEVICE_TIMEOUT);
       if (abort_flag) *abort_flag = 1;
       return false;
@@ -417,7 +421,7 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
           // a tile seen published stays published: later tiles skip its flag (the first 64)
           const int fi = mbr * pr.flag_ntiles + nb;
           if (fi < 64 && ((seen >> fi) & 1ull)) continue;
-          if (lane == 0) ok = wait_flag(pr.flags + fi, EPI_THREADS / 32, P.status, abort_flag);
+          if (lane == 0) ok = wait_flag(pr.flags + fi, EPI_THREADS / 32, P.flag_budget, P.status, abort_flag);
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (ok && fi < 64) seen |= 1ull << fi;
         }
@@ -561,7 +565,8 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
         // this warp's part of the tile is stored (plain stores): publish it device-wide
         __threadfence();
         __syncwarp();
-        if (lane == 0) atomicAdd(pr.flags + mb * pr.n_tiles + nb, 1);
+        const int fi = mb * pr.n_tiles + nb;
+        if (lane == 0 && fi != P.withhold_flag) atomicAdd(pr.flags + fi, 1);
       }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
@@ -632,6 +637,8 @@ rocs_status launch_gemm_bf16(rocs_context* ctx, const GemmDesc* probs, int nprob
   memset(&P, 0, sizeof(P));
   P.nprob = nprob;
   P.status = ctx->d_status;
+  P.flag_budget = ctx->test_flag_budget > 0 ? ctx->test_flag_budget : kWaitBudgetCycles;
+  P.withhold_flag = ctx->test_withhold_flag;
   int tiles = 0;
   bool same_m = true;
   int nstart = 0;
