@@ -56,6 +56,9 @@ WORKLOADS = {
     "w8a16": "FP8-weight (W8A16) IKBO linear against the same linear with bf16 weights, weights read from HBM "
              "(L2 flushed): the UG-Separation review's four configurations (1, N, d_in, d_out) = (1, 16|8, 1280, "
              "2560|640) read as one request with N candidates, plus two larger weight-bound shapes",
+    "ex2_rate": "throughput of the attention softmax's exponentials (scale and shift on the packed FMA path, 2^x, "
+                "bf16 packing) with n_poly of every eight pairs on the FMA-pipe polynomial and the rest on MUFU ex2, "
+                "n_poly = 0..8; every SM filled (2048 threads each)",
     "xattn_unsorted": "candidate cross-attention with candidates in shuffled order (each with its request index): "
                       "512 requests, candidates ~ clipped lognormal (median 300, 16..2000), L=1024, d=256, 8 heads; "
                       "stable sort by request + gather + segment-path attention + scatter, against the grouped call",
@@ -203,15 +206,22 @@ def roofline_entry(case, label, launches, total_ms, peaks, sustained: bool):
         peak = peaks["hbm"]
         unit = "GB/s"
     else:
-        # exp2 throughput: MUFU does 16 per clock per SM at the max SM clock and takes 5/8 of the
-        # softmax's exponentials (the other 3/8 run as a polynomial on the FMA pipe), so MUFU
-        # caps the rate at 16 / (5/8) = 25.6 exponentials per clock per SM
         achieved = amount / per_launch_s / 1e9
-        peak = 16 / ATTN_MUFU_SHARE * 148 * peaks["sm_mhz"] * 1e6 / 1e9
         unit = "Gexp2/s"
+        if peaks.get("exp2_gps"):
+            # measured in this run by rocs_probe_exp2_rate: the softmax's per-score steps with the
+            # attention kernels' split (3 of 8 exponential pairs on the FMA-pipe polynomial)
+            peak = peaks["exp2_gps"]
+            return {"kernel": label, "bound": bound, "achieved": round(achieved, 3), "peak": round(peak, 1),
+                    "unit": unit, "frac": round(achieved / peak, 4), "per_launch_ms": round(total_ms / launches, 4),
+                    "launches": launches, "peak_source": "measured in this run (rocs_probe_exp2_rate, 3-in-8 split)"}
+        # without the probe: MUFU does 16 per clock per SM at the max SM clock and takes 5/8 of
+        # the softmax's exponentials, so it caps the rate at 16 / (5/8) = 25.6 per clock per SM
+        peak = 16 / ATTN_MUFU_SHARE * 148 * peaks["sm_mhz"] * 1e6 / 1e9
     return {"kernel": label, "bound": bound, "achieved": round(achieved, 3), "peak": round(peak, 1), "unit": unit,
             "frac": round(achieved / peak, 4), "per_launch_ms": round(total_ms / launches, 4), "launches": launches,
-            "peak_source": f"{peaks['source']}{' sustained' if sustained and bound == 'tensor' else ''}"}
+            "peak_source": (f"{peaks['source']}{' sustained' if sustained and bound == 'tensor' else ''}"
+                            if bound != "alu" else "derived: 16 ex2/clk/SM / (5/8) x 148 SMs x max SM clock")}
 
 
 # ---------------------------------------------------------------------------------------------
@@ -485,6 +495,8 @@ def run_librocs(args, rank, world, local):
     st = R.rocs_get_device_status(sh)
     if st != 0:
         raise RuntimeError(f"device status {rocs.STATUS_NAMES.get(st, st)} in the timed region")
+    # the exponential ceiling of the attention kernels, measured on this GPU now (B-16 probe)
+    exp2_probe = {f"n_poly={n}": round(R.rocs_probe_exp2_rate(n, sh) / 1e9, 1) for n in (0, 3, 8)}
     _, total_c, ms_max = shard_totals(args.workload, rank, world, args.requests, ms)
     cands = total_c * args.steps
     value = cands / (ms_max / 1e3)
@@ -561,6 +573,7 @@ def run_librocs(args, rank, world, local):
 
     # ---- per-kernel breakdown and the dominant kernel's roofline ----
     peaks = load_peaks()
+    peaks["exp2_gps"] = exp2_probe["n_poly=3"]
     kernels = sorted(report.items(), key=lambda kv: -kv[1][1])
     launches = sum(n for name, (n, _) in report.items() if name != "dropped")
     total_k = sum(t for _, (_, t) in report.items())
@@ -614,7 +627,12 @@ def run_librocs(args, rank, world, local):
             "kernels": [{k: v for k, v in e.items() if k in ("kernel", "bound", "achieved", "unit", "frac", "share",
                                                              "per_launch_ms", "launches")} for e in rooflines[:8]],
             "kernel_ms": {name: round(t / args.steps, 4) for name, (n, t) in kernels[:16]},
-            "input_generation_s": round(gen_s, 1)}
+            "input_generation_s": round(gen_s, 1),
+            "exp2_probe_Gexp2_per_s": exp2_probe}
+    if a is not None and g is not None and not args.no_baselines:
+        del ws, sets, xd2
+        torch.cuda.empty_cache()
+        line["baselines"] = gpu_baselines(R, dev, sh, case, peaks, rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, n, reqs, dt = oracle_rate(case, args.cpu_seconds)
         line["cpu_baseline"] = {"value": round(rate, 2), "unit": "candidates/s", "cores": blas_threads(),
@@ -628,6 +646,123 @@ def run_librocs(args, rank, world, local):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------------------------
+# GPU materialised-broadcast baselines (torch / cuBLAS / SDPA), beside the headline
+# ---------------------------------------------------------------------------------------------
+def _timed_median(fn, reps, warmup, flush, dev):
+    import torch
+    for _ in range(warmup):
+        fn()
+    ts = []
+    for _ in range(reps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        ts.append(e0.elapsed_time(e1))
+    ts.sort()
+    return ts[len(ts) // 2]
+
+
+def gpu_baselines(R, dev, sh, case, peaks, rank):
+    """B1 and B2 against rocs_linear_ikbo at the IKBO sweep point N = 1024, d = 1024 (256 requests,
+    262,144 candidates, bf16, ReLU), and B3 against rocs_dca_cross_attn on the forward's depth-0
+    candidate cross-attention shapes (its counts, L, heads).  Each repetition is timed alone after
+    an L2 flush (256 MB write); medians.  Inputs: seeded torch normal draws on the device.
+      B1  Z = X^R W_CR^T + b^C written out as Z[m] [B_C, d] and added to X^C W_CC^T ("Fig. 3(a)")
+      B2  [X^R[m], X^C] gathered and one K = 2d GEMM (the early broadcast)
+      B3  K/V copied per candidate ([c, L, d], chunks of 2048 candidates), then SDPA (the pages'
+          "explicit K/V broadcast" attention arms)"""
+    import torch
+    import torch.nn.functional as F
+    from request_candidate_sharing_b200 import rocs
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    bf = torch.bfloat16
+    out = {}
+    # ---- B1 / B2: the IKBO linear ----
+    B_R, N, d = 256, 1024, 1024
+    B_C = B_R * N
+    gen = torch.Generator(device=dev).manual_seed(20 + rank)
+    XR = torch.randn(B_R, d, device=dev, generator=gen).to(bf)
+    XC = torch.randn(B_C, d, device=dev, generator=gen).to(bf)
+    W_RR, W_CR, W_CC = (torch.randn(d, d, device=dev, generator=gen).mul_(d ** -0.5).to(bf) for _ in range(3))
+    bR = torch.rand(d, device=dev, generator=gen) * 0.2 - 0.1
+    bC = torch.rand(d, device=dev, generator=gen) * 0.2 - 0.1
+    m = torch.arange(B_R, device=dev, dtype=torch.int32).repeat_interleave(N)
+    mi = m.long()
+    YR = torch.empty(B_R, d, dtype=bf, device=dev)
+    YC = torch.empty(B_C, d, dtype=bf, device=dev)
+    desc = rocs.IkboDesc(B_R, B_C, d, d, d, d, rocs.ROCS_BF16, rocs.ROCS_BF16, rocs.ACT["relu"])
+    nb = R.rocs_linear_ikbo_workspace(desc)
+    ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
+    W2 = torch.cat([W_CR, W_CC], 1)
+    res = {}
+
+    def ikbo():
+        R.rocs_linear_ikbo(desc, XR, XC, m, W_RR, W_CR, W_CC, bR, bC, YR, YC, ws, nb, sh)
+
+    def b1():
+        z = torch.addmm(bC, XR.float(), W_CR.float().t()).to(bf)
+        res["b1"] = torch.relu_(torch.addmm(z.index_select(0, mi), XC, W_CC.t()))
+        torch.relu_(torch.addmm(bR.to(bf), XR, W_RR.t()))
+
+    def b2():
+        xg = torch.cat([XR.index_select(0, mi), XC], 1)
+        res["b2"] = torch.relu_(torch.addmm(bC.to(bf), xg, W2.t()))
+        torch.relu_(torch.addmm(bR.to(bf), XR, W_RR.t()))
+
+    t_i, t_1, t_2 = (_timed_median(f, 5, 3, flush, dev) for f in (ikbo, b1, b2))
+    flops = 2.0 * B_C * d * d + 2.0 * B_R * d * d * 2
+    out["linear_N1024_d1024"] = {
+        "rocs_linear_ikbo_ms": round(t_i, 4), "B1_materialised_Zm_ms": round(t_1, 4),
+        "B2_gathered_2d_gemm_ms": round(t_2, 4), "speedup_vs_B1": round(t_1 / t_i, 3),
+        "speedup_vs_B2": round(t_2 / t_i, 3),
+        "ikbo_tflops": round(flops / (t_i / 1e3) / 1e12, 1),
+        "max_abs_diff_vs_B2": round(float((YC.float() - res["b2"].float()).abs().max()), 4)}
+    del XR, XC, W_RR, W_CR, W_CC, YR, YC, ws, W2, res, m, mi
+    torch.cuda.empty_cache()
+    # ---- B3: candidate cross-attention with K/V copied per candidate ----
+    a = case.dca
+    L, H, dh = a.L, a.H, a.d // a.H
+    counts = torch.from_numpy(np.asarray(case.counts, np.int64)).to(dev)
+    Bc = int(counts.sum())
+    Q = torch.randn(Bc, a.d, device=dev, generator=gen).to(bf)
+    K = torch.randn(case.B_R, L, a.d, device=dev, generator=gen).to(bf)
+    V = torch.randn(case.B_R, L, a.d, device=dev, generator=gen).to(bf)
+    off = torch.zeros(case.B_R + 1, dtype=torch.int32, device=dev)
+    off[1:] = counts.cumsum(0).to(torch.int32)
+    mq = torch.repeat_interleave(torch.arange(case.B_R, device=dev), counts)
+    O = torch.empty(Bc, a.d, device=dev)
+    O3 = torch.empty(Bc, a.d, device=dev, dtype=bf)
+    scale = 1.0 / math.sqrt(dh)
+    chunk = 2048
+
+    def rocs_x():
+        R.rocs_dca_cross_attn(Q, K, V, off, case.B_R, Bc, L, H, dh, scale, O, a.d, rocs.ROCS_F32, sh)
+
+    def b3():
+        for c0 in range(0, Bc, chunk):
+            idx = mq[c0:c0 + chunk]
+            kc = K.index_select(0, idx).view(-1, L, H, dh).transpose(1, 2)     # [c, H, L, dh] copy per candidate
+            vc = V.index_select(0, idx).view(-1, L, H, dh).transpose(1, 2)
+            q = Q[c0:c0 + chunk].view(-1, H, 1, dh)
+            O3[c0:c0 + chunk] = F.scaled_dot_product_attention(q, kc, vc).reshape(-1, a.d)
+
+    t_x = _timed_median(rocs_x, 5, 3, flush, dev)
+    t_3 = _timed_median(b3, 2, 1, flush, dev)
+    out["dca_cross_attn_depth0"] = {
+        "candidates": Bc, "L": L, "heads": H, "rocs_dca_cross_attn_ms": round(t_x, 4),
+        "B3_kv_copied_per_candidate_sdpa_ms": round(t_3, 3), "speedup_vs_B3": round(t_3 / t_x, 1),
+        "B3_chunk": chunk, "max_abs_diff_vs_B3": round(float((O - O3.float()).abs().max()), 4)}
+    if R.rocs_get_device_status(sh) != 0:
+        raise RuntimeError("device status set in the baselines")
+    del Q, K, V, O, O3
+    torch.cuda.empty_cache()
+    return out
 
 
 # ---------------------------------------------------------------------------------------------
@@ -666,8 +801,9 @@ def run_ikbo_sweep(args, rank, world, local):
     """Each (N, d) point: rocs_linear_ikbo (bf16 in/out, ReLU), B1 = Z = X^R W_CR^T, Z[m] written
     out and added to X^C W_CC^T (torch/cuBLAS), B2 = [X^R[m], X^C] gathered and one K=2d GEMM
     (torch/cuBLAS).  Each repetition is timed alone with CUDA events after an L2 flush (a 256 MB
-    write); the median is reported.  Inputs: seeded torch normal draws on the device (X ~ N(0,1),
-    W ~ N(0, 1/fan_in), b ~ U(-0.1, 0.1)), bf16."""
+    write); the median is reported.  Inputs: the seeded synth draws of each point (X ~ N(0,1),
+    W ~ N(0, 1/fan_in), b ~ U(-0.1, 0.1), bf16), the same values tests/test_gpu_ops.py checks
+    against the oracle at every point (rank r > 0 shifts the seed by 1000 r)."""
     import torch
     from request_candidate_sharing_b200 import rocs
     dev = torch.device("cuda", local)
@@ -699,14 +835,17 @@ def run_ikbo_sweep(args, rank, world, local):
         for d in (512, 1024, 4096):
             if only is not None and (N, d) != only:
                 continue
-            g = torch.Generator(device=dev).manual_seed(1000 * N + d + 1000003 * rank)
+            # the seeded inputs the parity test checks against the oracle at this point
+            case = dataclasses.replace(synth.linear_cfg2(N, d, B_R), seed=synth.linear_cfg2(N, d, B_R).seed + 1000 * rank)
+            x = synth.linear_inputs(case, cand_rows=np.zeros(0, np.int64))
             B_C = B_R * N
             bf = torch.bfloat16
-            XR = torch.randn(B_R, d, device=dev, generator=g).to(bf)
-            XC = torch.randn(B_C, d, device=dev, generator=g).to(bf)
-            W_RR, W_CR, W_CC = (torch.randn(d, d, device=dev, generator=g).mul_(d ** -0.5).to(bf) for _ in range(3))
-            bR = (torch.rand(d, device=dev, generator=g) * 0.2 - 0.1)
-            bC = (torch.rand(d, device=dev, generator=g) * 0.2 - 0.1)
+            up = lambda v, dt=bf: torch.from_numpy(np.ascontiguousarray(v, np.float32)).to(dev).to(dt)
+            XR, W_RR, W_CR, W_CC = (up(x[k]) for k in ("X_R", "W_RR", "W_CR", "W_CC"))
+            bR, bC = up(x["b_R"], torch.float32), up(x["b_C"], torch.float32)
+            XC = torch.empty(B_C, d, dtype=bf, device=dev)
+            for r0, blk in synth.normal_blocks(case.seed, "X_C", (B_C, d)):
+                XC[r0:r0 + len(blk)].copy_(torch.from_numpy(synth.bf16_round(blk)).to(bf))
             m = torch.arange(B_R, device=dev, dtype=torch.int32).repeat_interleave(N)
             YR = torch.empty(B_R, d, dtype=bf, device=dev)
             YC = torch.empty(B_C, d, dtype=bf, device=dev)
@@ -751,7 +890,7 @@ def run_ikbo_sweep(args, rank, world, local):
         line = {"metric": METRIC, "value": head["ikbo_cands_per_s"], "unit": "candidates/s", "n_gpus": world,
                 "steps": reps, "warmup": args.warmup, "ms_per_step": head["ikbo_ms"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-                "data": "synthetic (seeded torch normal draws on the device)",
+                "data": "synthetic (seeded synth draws, the inputs of the per-point parity test)",
                 "config": {"workload": "ikbo_sweep", "description": WORKLOADS["ikbo_sweep"],
                            "headline_point": f"N={head['N']}, d={head['d']}",
                            "l2": "flushed (256 MB write) before every repetition",
@@ -936,6 +1075,42 @@ def run_xattn_unsorted(args, rank, world, local):
     R.close()
 
 
+def run_ex2_rate(args, rank, world, local):
+    """The attention softmax's exponential throughput on this GPU (rocs_probe_exp2_rate) for every
+    split of the exponentials between MUFU ex2 and the FMA-pipe polynomial (n_poly of every eight
+    pairs on the polynomial), with the SM clock sampled during the measurement."""
+    import torch
+    from request_candidate_sharing_b200 import rocs
+    torch.cuda.set_device(local)
+    R = rocs.Rocs(local)
+    sh = torch.cuda.current_stream(local).cuda_stream
+    uuid = str(getattr(torch.cuda.get_device_properties(local), "uuid", "") or "")
+    clocks = ClockSampler(("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else (uuid or str(local)))
+    for n in range(9):       # warm-up: clocks up
+        R.rocs_probe_exp2_rate(n, sh)
+    clocks.start()
+    time.sleep(0.3)
+    rates = {}
+    for _ in range(max(1, args.steps // 3)):
+        for n in range(9):
+            rates[n] = max(rates.get(n, 0.0), R.rocs_probe_exp2_rate(n, sh))
+    clk = clocks.stop()
+    R.close()
+    sms = torch.cuda.get_device_properties(local).multi_processor_count
+    mhz = (clk or {}).get("sm_mhz") or 1965.0
+    per_clk = {f"n_poly={n}": round(r / (sms * mhz * 1e6), 2) for n, r in rates.items()}
+    best = max(rates, key=rates.get)
+    if rank == 0:
+        print(json.dumps({"metric": "exponentials/s of the attention softmax's per-score steps", "value": round(rates[3], 1),
+                          "unit": "exp2/s", "n_gpus": 1, "steps": args.steps, "warmup": 9, "higher_is_better": True,
+                          "dtype": "f32", "data": "synthetic", "impl": "librocs",
+                          "config": {"workload": "ex2_rate", "description": WORKLOADS["ex2_rate"],
+                                     "headline": "n_poly=3, the attention kernels' split"},
+                          "rates_exp2_per_s": {f"n_poly={n}": round(r, 1) for n, r in rates.items()},
+                          "per_clock_per_sm": per_clk, "best_split": f"n_poly={best}", "sms": sms,
+                          "clocks": clk}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -946,6 +1121,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-baselines", action="store_true", help="skip the GPU materialised-broadcast baselines")
     ap.add_argument("--requests", type=int, default=0, help="keep only the first N requests (profiling runs)")
     ap.add_argument("--sweep-point", default="", help="ikbo_sweep: run only the point 'N,d' (profiling runs)")
     ap.add_argument("--ikbo-fused", type=int, default=1, choices=[0, 1],
@@ -965,6 +1141,8 @@ def main():
         run_xattn_unsorted(args, rank, world, local)
     elif args.workload == "w8a16":
         run_w8a16(args, rank, world, local)
+    elif args.workload == "ex2_rate":
+        run_ex2_rate(args, rank, world, local)
     else:
         run_librocs(args, rank, world, local)
 

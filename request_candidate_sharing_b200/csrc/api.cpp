@@ -217,21 +217,23 @@ IkboPlan plan_ikbo(const rocs_ikbo_desc* d, void* ws) {
   return p;
 }
 
-rocs_status check_ikbo_desc(const rocs_ikbo_desc* d) {
-  ROCS_REQUIRE(d != nullptr, "rocs_linear_ikbo: desc is NULL");
-  ROCS_REQUIRE(d->B_R >= 1, "rocs_linear_ikbo: B_R=%d must be >= 1", d->B_R);
-  ROCS_REQUIRE(d->B_C >= 0 && d->B_C < 2147483647LL, "rocs_linear_ikbo: B_C=%lld out of range", (long long)d->B_C);
+rocs_status check_ikbo_desc(const rocs_ikbo_desc* d) { return rocs::check_ikbo_desc(d, "rocs_linear_ikbo"); }
+
+}  // namespace
+
+rocs_status check_ikbo_desc(const rocs_ikbo_desc* d, const char* who) {
+  ROCS_REQUIRE(d != nullptr, "%s: desc is NULL", who);
+  ROCS_REQUIRE(d->B_R >= 1, "%s: B_R=%d must be >= 1", who, d->B_R);
+  ROCS_REQUIRE(d->B_C >= 0 && d->B_C < 2147483647LL, "%s: B_C=%lld out of range", who, (long long)d->B_C);
   ROCS_REQUIRE(d->d_R_in >= 1 && d->d_C_in >= 1 && d->d_C_out >= 1 && d->d_R_out >= 0,
-               "rocs_linear_ikbo: dims must be positive (d_R_out may be 0)");
-  ROCS_REQUIRE(d->dtype_in == ROCS_F32 || d->dtype_in == ROCS_BF16, "rocs_linear_ikbo: bad dtype_in");
-  ROCS_REQUIRE(d->dtype_out == ROCS_F32 || d->dtype_out == ROCS_BF16, "rocs_linear_ikbo: bad dtype_out");
-  ROCS_REQUIRE(!(d->dtype_in == ROCS_F32 && d->dtype_out != ROCS_F32),
-               "rocs_linear_ikbo: the fp32 path writes fp32 outputs");
-  ROCS_REQUIRE(d->act >= ROCS_ACT_NONE && d->act <= ROCS_ACT_SIGMOID, "rocs_linear_ikbo: bad act");
+               "%s: dims must be positive (d_R_out may be 0)", who);
+  ROCS_REQUIRE(d->dtype_in == ROCS_F32 || d->dtype_in == ROCS_BF16, "%s: bad dtype_in", who);
+  ROCS_REQUIRE(d->dtype_out == ROCS_F32 || d->dtype_out == ROCS_BF16, "%s: bad dtype_out", who);
+  ROCS_REQUIRE(!(d->dtype_in == ROCS_F32 && d->dtype_out != ROCS_F32), "%s: the fp32 path writes fp32 outputs", who);
+  ROCS_REQUIRE(d->act >= ROCS_ACT_NONE && d->act <= ROCS_ACT_SIGMOID, "%s: bad act", who);
   return ROCS_OK;
 }
 
-}  // namespace
 }  // namespace rocs
 
 using namespace rocs;
@@ -1345,6 +1347,30 @@ extern "C" rocs_status rocs_set_ikbo_fused(rocs_handle_t h, int32_t enable) {
   ROCS_REQUIRE(h, "rocs_set_ikbo_fused: handle is NULL");
   ROCS_REQUIRE(enable == 0 || enable == 1, "rocs_set_ikbo_fused: enable must be 0 or 1");
   h->ikbo_fused = enable;
+  return ROCS_OK;
+}
+
+extern "C" rocs_status rocs_probe_exp2_rate(rocs_handle_t h, int32_t n_poly, double* exp2_per_second, void* stream) {
+  CtxGuard ctx_guard_(h);
+  ROCS_REQUIRE(h, "rocs_probe_exp2_rate: handle is NULL");
+  ROCS_REQUIRE(exp2_per_second, "rocs_probe_exp2_rate: exp2_per_second is NULL");
+  ROCS_REQUIRE(n_poly >= 0 && n_poly <= 8, "rocs_probe_exp2_rate: n_poly=%d outside [0, 8]", n_poly);
+  return probe_exp2_rate(h, n_poly, exp2_per_second, (cudaStream_t)stream);
+}
+
+extern "C" rocs_status rocs_test_withhold_ikbo_flag(rocs_handle_t h, int32_t flag_index, int64_t wait_budget_cycles) {
+  ROCS_REQUIRE(h, "rocs_test_withhold_ikbo_flag: handle is NULL");
+  ROCS_REQUIRE(flag_index >= -1, "rocs_test_withhold_ikbo_flag: flag_index=%d must be >= -1", flag_index);
+  if (flag_index < 0) {
+    h->test_withhold_flag = -1;
+    h->test_flag_budget = 0;
+    return ROCS_OK;
+  }
+  ROCS_REQUIRE(wait_budget_cycles >= 1000 && wait_budget_cycles <= 10000000000LL,
+               "rocs_test_withhold_ikbo_flag: wait_budget_cycles=%lld outside [1e3, 1e10]",
+               (long long)wait_budget_cycles);
+  h->test_withhold_flag = flag_index;
+  h->test_flag_budget = wait_budget_cycles;
   return ROCS_OK;
 }
 

@@ -34,6 +34,8 @@ struct rocs_context {
   RocsTimer timer;
   int graph_replay = 1;                 // rocs_set_graph_replay
   int ikbo_fused = 1;                   // rocs_set_ikbo_fused
+  int test_withhold_flag = -1;          // rocs_test_withhold_ikbo_flag: flag never published (-1: none)
+  long long test_flag_budget = 0;       // ... and the flag-wait budget in SM cycles (0: the default ~1 s)
   cudaStream_t capture_stream = nullptr;   // forward graphs are captured here (never the legacy stream)
   std::vector<ForwardGraph> graphs;     // at most kMaxForwardGraphs, most recent last
 };
@@ -76,6 +78,9 @@ struct LaunchTimer {
 
 void set_error(const char* fmt, ...);
 rocs_status cuda_check(cudaError_t e, const char* what);
+// Host validation of an IKBO linear's descriptor (dims, dtypes, activation); error messages are
+// prefixed with `who`, the entry point's name.
+rocs_status check_ikbo_desc(const rocs_ikbo_desc* d, const char* who);
 
 // One GEMM problem for the tcgen05 kernel:
 //   out[r, c] = act( scale[c] * sum_k A[r, k] * B[c, k] + bias[c] + Z[gidx[r], c] )
@@ -230,6 +235,10 @@ rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq,
                                 int out_bf16, void* O2, long long ldo2, cudaStream_t s,
                                 const int32_t* out_rows = nullptr, const int32_t* kv_len = nullptr,
                                 int q_by_kv = 0, const int32_t* order = nullptr);
+
+// Exponentials per second of the attention softmax's per-score steps with n_poly of every eight
+// pairs on the FMA-pipe polynomial (probe.cu); synchronises s.
+rocs_status probe_exp2_rate(rocs_context* ctx, int n_poly, double* rate, cudaStream_t s);
 
 rocs_status launch_score_head(const void* X, long long ldx, long long rows, int K, const void* w,
                               const float* b, float* out, cudaStream_t s);

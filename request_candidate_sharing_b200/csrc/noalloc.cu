@@ -11,7 +11,9 @@
 // Host code must not pass the array's name to a kernel: on the host that name is only a
 // stand-in for the symbol, not a device address.  The first call on each device (with that
 // device current) asks the runtime for the real address with cudaGetSymbolAddress and caches
-// it; kernels then receive that pointer.
+// it, with the context it belongs to; kernels then receive that pointer.  Under lazy module
+// loading (the CUDA 12 default) that first call is also when the driver loads this module and
+// commits the array's 4 MiB.
 #include <mutex>
 
 #include "common.cuh"
@@ -27,16 +29,39 @@ static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
+// Per device: the address of the scratch array and the CUDA context it was looked up in.  The
+// array belongs to the module loaded into that context; a call from another context (a context
+// the caller created, not the device's primary one) looks the address up again in its own.
 float* g_scratch_addr[kMaxDevices] = {nullptr};
+CUcontext g_scratch_ctx[kMaxDevices] = {nullptr};
 
-// Resolves (once per device) the device address of the scratch array for the current device.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+
+// Resolves the device address of the scratch array for the current device and context: once per
+// (device, context), on the first call there.
 rocs_status scratch_address(int device, float** out) {
   if (device < 0 || device >= kMaxDevices) {
     set_error("rocs_linear_ikbo_noalloc: device %d out of range", device);
     return ROCS_ERR_UNSUPPORTED;
   }
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (g_scratch_addr[device] == nullptr) {
+  if (g_ctx_get_current == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || fn == nullptr) {
+      set_error("rocs_linear_ikbo_noalloc: cuCtxGetCurrent not available");
+      return ROCS_ERR_CUDA;
+    }
+    g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+  }
+  CUcontext cur = nullptr;
+  if (g_ctx_get_current(&cur) != CUDA_SUCCESS || cur == nullptr) {
+    set_error("rocs_linear_ikbo_noalloc: no current CUDA context");
+    return ROCS_ERR_CUDA;
+  }
+  if (g_scratch_addr[device] == nullptr || g_scratch_ctx[device] != cur) {
     void* p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || p == nullptr) {
@@ -44,6 +69,7 @@ rocs_status scratch_address(int device, float** out) {
       return ROCS_ERR_CUDA;
     }
     g_scratch_addr[device] = static_cast<float*>(p);
+    g_scratch_ctx[device] = cur;
   }
   *out = g_scratch_addr[device];
   return ROCS_OK;
@@ -58,17 +84,12 @@ extern "C" rocs_status rocs_linear_ikbo_noalloc(rocs_handle_t h, const rocs_ikbo
                                                 const void* X_C, const int32_t* req_idx, const void* W_RR,
                                                 const void* W_CR, const void* W_CC, const float* b_R,
                                                 const float* b_C, void* Y_R, void* Y_C, void* stream) {
-  if (h == nullptr || d == nullptr) {
-    set_error("rocs_linear_ikbo_noalloc: handle or desc is NULL");
+  if (h == nullptr) {
+    set_error("rocs_linear_ikbo_noalloc: handle is NULL");
     return ROCS_ERR_INVALID_ARG;
   }
-  if (d->B_R < 1 || d->B_C < 0 || d->B_C >= 2147483647LL || d->d_R_in < 1 || d->d_C_in < 1 || d->d_C_out < 1 ||
-      d->d_R_out < 0 || (d->dtype_in != ROCS_F32 && d->dtype_in != ROCS_BF16) ||
-      (d->dtype_out != ROCS_F32 && d->dtype_out != ROCS_BF16) || (d->dtype_in == ROCS_F32 && d->dtype_out != ROCS_F32) ||
-      d->act < ROCS_ACT_NONE || d->act > ROCS_ACT_SIGMOID) {
-    set_error("rocs_linear_ikbo_noalloc: invalid descriptor");
-    return ROCS_ERR_INVALID_ARG;
-  }
+  rocs_status st = check_ikbo_desc(d, "rocs_linear_ikbo_noalloc");
+  if (st != ROCS_OK) return st;
   const long long need = (long long)d->B_R * d->d_C_out;
   if (need > kNoAllocScratchFloats) {
     set_error("rocs_linear_ikbo_noalloc: B_R * d_C_out = %lld exceeds the built-in scratch of %lld floats; "
@@ -93,7 +114,7 @@ extern "C" rocs_status rocs_linear_ikbo_noalloc(rocs_handle_t h, const rocs_ikbo
       return ROCS_ERR_INVALID_ARG;
     }
   int cur = -1;
-  rocs_status st = cuda_check(cudaGetDevice(&cur), "cudaGetDevice");
+  st = cuda_check(cudaGetDevice(&cur), "cudaGetDevice");
   if (st != ROCS_OK) return st;
   if (cur != h->device) {
     set_error("rocs_linear_ikbo_noalloc: device %d is current but the handle is bound to device %d", cur, h->device);

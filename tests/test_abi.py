@@ -120,3 +120,33 @@ def test_create_without_gpu_fails_cleanly(rocs):
         pytest.skip("a GPU is present")
     with pytest.raises(rocs.RocsError):
         rocs.Rocs(0)
+
+
+def _function_body(src: str, signature: str) -> str:
+    """The text of the function whose definition starts with `signature`, through its closing
+    brace (brace matching; the sources have no braces inside string literals there)."""
+    i = src.index(signature)
+    j = src.index("{", i)
+    depth = 0
+    for k in range(j, len(src)):
+        depth += {"{": 1, "}": -1}.get(src[k], 0)
+        if depth == 0:
+            return src[i:k + 1]
+    raise AssertionError(f"unbalanced braces after {signature}")
+
+
+def test_noalloc_path_calls_no_allocation_routine():
+    """rocs_linear_ikbo_noalloc and the launchers it calls name no routine that allocates, frees
+    or clears device memory (a memset on the shared scratch would also be a hidden dependency)."""
+    import re
+    csrc = os.path.join(ROOT, "request_candidate_sharing_b200", "csrc")
+    read = lambda f: open(os.path.join(csrc, f)).read()
+    code = lambda t: re.sub(r"//[^\n]*", "", t)          # comments may name them
+    bodies = [code(read("noalloc.cu")),
+              code(_function_body(read("misc.cu"), "rocs_status launch_gemm_f32(")),
+              code(_function_body(read("gemm_tc.cu"), "rocs_status launch_gemm_bf16("))]
+    banned = re.compile(r"\b(cudaMalloc\w*|cudaFree\w*|cudaMemset\w*|cuMemAlloc\w*|cuMemFree\w*|cuMemCreate|"
+                        r"cudaMallocAsync|malloc|free|new|delete)\b")
+    for b in bodies:
+        assert not banned.search(b), banned.search(b).group(0)
+    assert "launch_gemm_f32" in bodies[0] and "launch_gemm_bf16" in bodies[0]

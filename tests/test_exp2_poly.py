@@ -17,10 +17,10 @@ CSRC = os.path.join(ROOT, "request_candidate_sharing_b200", "csrc")
 
 
 def _kernel_coeffs():
-    src = open(os.path.join(CSRC, "attn_tc.cu")).read()
+    src = open(os.path.join(CSRC, "softmax_math.cuh")).read()
     m = re.search(r"c3 = dup2\(([0-9.e+-]+)f\), c2 = dup2\(([0-9.e+-]+)f\), c1 = dup2\(([0-9.e+-]+)f\), "
                   r"c0 = dup2\(([0-9.e+-]+)f\)", src)
-    assert m, "polynomial coefficients not found in attn_tc.cu"
+    assert m, "polynomial coefficients not found in softmax_math.cuh"
     c3, c2, c1, c0 = (np.float32(float(v)) for v in m.groups())
     return c0, c1, c2, c3
 
