@@ -191,6 +191,11 @@ def load_peaks():
     return dict(hbm=6650.0, tensor=1590.0, tensor_sustained=1400.0, sm_mhz=1965.0, source="fallback")
 
 
+# GEMM sites whose A operand is a bf16 hi/lo pair (the GLM MLPs and the DCA query generator): the
+# tensor cores execute twice the algorithmic flops there
+SPLIT_A_SITES = ("glm.mlp1.", "glm.mlp2.", "qgen.mlp1.", "qgen.mlp2.")
+
+
 def roofline_entry(case, label, launches, total_ms, peaks, sustained: bool):
     w = algo_work(case, label)
     if w is None or launches == 0:
@@ -218,10 +223,13 @@ def roofline_entry(case, label, launches, total_ms, peaks, sustained: bool):
         # without the probe: MUFU does 16 per clock per SM at the max SM clock and takes 5/8 of
         # the softmax's exponentials, so it caps the rate at 16 / (5/8) = 25.6 per clock per SM
         peak = 16 / ATTN_MUFU_SHARE * 148 * peaks["sm_mhz"] * 1e6 / 1e9
-    return {"kernel": label, "bound": bound, "achieved": round(achieved, 3), "peak": round(peak, 1), "unit": unit,
-            "frac": round(achieved / peak, 4), "per_launch_ms": round(total_ms / launches, 4), "launches": launches,
-            "peak_source": (f"{peaks['source']}{' sustained' if sustained and bound == 'tensor' else ''}"
-                            if bound != "alu" else "derived: 16 ex2/clk/SM / (5/8) x 148 SMs x max SM clock")}
+    e = {"kernel": label, "bound": bound, "achieved": round(achieved, 3), "peak": round(peak, 1), "unit": unit,
+         "frac": round(achieved / peak, 4), "per_launch_ms": round(total_ms / launches, 4), "launches": launches,
+         "peak_source": (f"{peaks['source']}{' sustained' if sustained and bound == 'tensor' else ''}"
+                         if bound != "alu" else "derived: 16 ex2/clk/SM / (5/8) x 148 SMs x max SM clock")}
+    if bound == "tensor" and label.startswith(SPLIT_A_SITES):
+        e["executed_frac"] = round(2.0 * achieved / peak, 4)   # hi and lo halves of A both multiplied
+    return e
 
 
 # ---------------------------------------------------------------------------------------------
@@ -625,7 +633,8 @@ def run_librocs(args, rank, world, local):
             "gpu_launches": int(launches),
             "clocks": clk,
             "kernels": [{k: v for k, v in e.items() if k in ("kernel", "bound", "achieved", "unit", "frac", "share",
-                                                             "per_launch_ms", "launches")} for e in rooflines[:8]],
+                                                             "per_launch_ms", "launches", "executed_frac")}
+                        for e in rooflines[:8]],
             "kernel_ms": {name: round(t / args.steps, 4) for name, (n, t) in kernels[:16]},
             "input_generation_s": round(gen_s, 1),
             "exp2_probe_Gexp2_per_s": exp2_probe}
