@@ -392,9 +392,10 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
     };
 
     bool ok = true;
+    const int nkb_g = RAGGED ? geom[0] : P.nkb;
+    int k_tile = 0, j = -1;
     for (int i = 0; i < Tg; ++i) {
-      const int nkb_i = RAGGED ? geom[0] : P.nkb;
-      const int k_tile = i / nkb_i, j = i - k_tile * nkb_i;
+      if (++j == nkb_g) { j = 0; ++k_tile; }
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[g], i & 1, P.status, abort_flag))) { ok = false; break; }
       tc_fence_after();
       // the whole S row into registers with one wait, then the S accumulator is released
@@ -434,12 +435,14 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
         m_new = fmaxf(m_cur, mx);
         corr = ex2_approx(m_cur - m_new);
       }
-      // the previous block's P V, first half, has completed: that half of P may be overwritten;
-      // O is read (finished tile) or rescaled only once both halves have completed
+      // O is read (finished tile) or rescaled only once both halves of the previous block's P V
+      // have completed.  Otherwise those waits come later, just before each half of P is
+      // overwritten, so that the exponentials of the half are computed while the tensor core is
+      // still reading it.
       const bool need_o = i > 0 && (j == 0 || rescale);
-      if (i > 0) {
+      if (need_o) {
         if (!__all_sync(0xffffffffu, mbar_wait(&o_full[2 * g], (i - 1) & 1, P.status, abort_flag) &&
-                                         (!need_o || mbar_wait(&o_full[2 * g + 1], (i - 1) & 1, P.status, abort_flag)))) {
+                                         mbar_wait(&o_full[2 * g + 1], (i - 1) & 1, P.status, abort_flag))) {
           ok = false;
           break;
         }
@@ -465,43 +468,49 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
         }
       }
       // exponentials: three pairs in eight on the FMA pipe (polynomial), the rest on MUFU; P_i
-      // as bf16 pairs into TMEM, 32 keys per store
+      // as bf16 pairs into TMEM, one 64-key half at a time (32 keys per store), each half handed
+      // to the tensor core as soon as it is written
       const float neg_m = -m_new;
       float rs = 0.f;
 #pragma unroll
-      for (int c = 0; c < TK / 32; ++c) {
-        if (c == TK / 64) {
-          // first half of P_i is written: hand it to the tensor core, then wait for the
-          // previous block's second-half P V before overwriting that half
-          tmem_st_wait();
-          tc_fence_before();
-          mbar_arrive(&p_full[2 * g]);
-          if (i > 0 && !need_o &&
-              !__all_sync(0xffffffffu, mbar_wait(&o_full[2 * g + 1], (i - 1) & 1, P.status, abort_flag))) {
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t pk[2][16];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = 2 * hh + cc;
+#pragma unroll
+          for (int k = 0; k < 32; k += 2) {
+            float x0, x1, p0, p1;
+            ffma2(__uint_as_float(v[c][k]), __uint_as_float(v[c][k + 1]), sl2, neg_m, x0, x1);
+            if (((k >> 1) & 7) >= 5) {
+              exp2_poly2(x0, x1, p0, p1);
+              if (valid < TK) {   // masked keys (x = -inf) must give exactly zero
+                p0 = x0 == -INFINITY ? 0.f : p0;
+                p1 = x1 == -INFINITY ? 0.f : p1;
+              }
+            } else {
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+            if (!C::SUM_MMA) rs += p0 + p1;
+            pk[cc][k >> 1] = pack_bf16x2(p0, p1);
+          }
+        }
+        // this half of P may be overwritten once the previous block's P V of it has completed
+        if (i > 0 && !need_o) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&o_full[2 * g + hh], (i - 1) & 1, P.status, abort_flag))) {
             ok = false;
             break;
           }
           tc_fence_after();
         }
-        uint32_t pk[16];
-#pragma unroll
-        for (int k = 0; k < 32; k += 2) {
-          float x0, x1, p0, p1;
-          ffma2(__uint_as_float(v[c][k]), __uint_as_float(v[c][k + 1]), sl2, neg_m, x0, x1);
-          if (((k >> 1) & 7) >= 5) {
-            exp2_poly2(x0, x1, p0, p1);
-            if (valid < TK) {   // masked keys (x = -inf) must give exactly zero
-              p0 = x0 == -INFINITY ? 0.f : p0;
-              p1 = x1 == -INFINITY ? 0.f : p1;
-            }
-          } else {
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
-          }
-          if (!C::SUM_MMA) rs += p0 + p1;
-          pk[k >> 1] = pack_bf16x2(p0, p1);
+        tmem_st_32x32b_x16(paddr + (2 * hh) * 16, pk[0]);
+        tmem_st_32x32b_x16(paddr + (2 * hh + 1) * 16, pk[1]);
+        if (hh == 0) {
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&p_full[2 * g]);
         }
-        tmem_st_32x32b_x16(paddr + c * 16, pk);
       }
       if (!ok) break;
       tmem_st_wait();
