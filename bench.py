@@ -55,7 +55,8 @@ WORKLOADS = {
                   "GPU baselines (B1: Z[m] materialised and added; B2: gathered [X^R[m], X^C] with one K=2d GEMM)",
     "w8a16": "FP8-weight (W8A16) IKBO linear against the same linear with bf16 weights, weights read from HBM "
              "(L2 flushed): the UG-Separation review's four configurations (1, N, d_in, d_out) = (1, 16|8, 1280, "
-             "2560|640) read as one request with N candidates, plus two larger weight-bound shapes",
+             "2560|640) read as one request with N candidates, plus two larger weight-bound shapes; the default "
+             "FP8 path and the opt-in tensor-core path (FP8 operands converted in shared memory)",
     "ex2_rate": "throughput of the attention softmax's exponentials (scale and shift on the packed FMA path, 2^x, "
                 "bf16 packing) with n_poly of every eight pairs on the FMA-pipe polynomial and the rest on MUFU ex2, "
                 "n_poly = 0..8; every SM filled (2048 threads each)",
@@ -965,6 +966,14 @@ def run_w8a16(args, rank, world, local):
         YC_b = YC.float().clone()
         ms_8 = timed(lambda: R.rocs_linear_ikbo_w8(desc, XR, XC, m, Q[0], Q[1], Q[2], S[0], S[1], S[2], bR, bC, YR, YC,
                                                     ws, nb8, sh))
+        # the opt-in path: FP8 operands converted in shared memory for the tcgen05 MMAs
+        R.rocs_set_w8_tensor_cores(1)
+        nbt = R.rocs_linear_ikbo_w8_workspace(desc)
+        wst = torch.empty(max(nbt, 16), dtype=torch.uint8, device=dev)
+        YC_t = torch.empty_like(YC)
+        ms_t = timed(lambda: R.rocs_linear_ikbo_w8(desc, XR, XC, m, Q[0], Q[1], Q[2], S[0], S[1], S[2], bR, bC, YR, YC_t,
+                                                    wst, nbt, sh))
+        R.rocs_set_w8_tensor_cores(0)
         if R.rocs_get_device_status(sh) != 0:
             raise RuntimeError("device status set")
         # per-kernel times of both calls (direct launches, per-launch CUDA events, L2 flushed)
@@ -984,9 +993,11 @@ def run_w8a16(args, rank, world, local):
         gbs = (wbytes8 + act_bytes) / (ms_8 / 1e3) / 1e9
         points.append({"B_R": B_R, "N": N, "d_in": di, "d_out": do, "bf16_weights_ms": round(ms_b, 4),
                        "fp8_weights_ms": round(ms_8, 4), "latency_change": round(ms_8 / ms_b - 1.0, 4),
+                       "fp8_tensor_core_path_ms": round(ms_t, 4),
+                       "tensor_core_path_max_abs_diff": round(float((YC_t.float() - YC.float()).abs().max()), 5),
                        "fp8_GBps": round(gbs, 1), "fp8_frac_of_hbm": round(gbs / peaks["hbm"], 4),
                        "rel_l2_vs_bf16_weights": round(rel, 5), "kernel_ms": kern})
-        del XR, XC, Ws, Q, S, ws, YR, YC
+        del XR, XC, Ws, Q, S, ws, YR, YC, wst, YC_t
         torch.cuda.empty_cache()
     if rank == 0:
         head = points[0]

@@ -136,12 +136,18 @@ rocs_status rocs_linear_ikbo(rocs_handle_t handle, const rocs_ikbo_desc* desc,
  *   Q [rows, cols] uint8 and scale [rows] float32 written.
  *
  * rocs_linear_ikbo_w8: rocs_linear_ikbo (dtype_in = ROCS_BF16) with the three weight blocks as
- *   (Q_RR, s_RR), (Q_CR, s_CR), (Q_CC, s_CC).  Shapes as rocs_linear_ikbo; Q_* [out, in] uint8,
- *   8-byte aligned; s_* [out] float32.  A GEMM side with at most 64 rows (B_R, resp. B_C) and
- *   d_in % 32 == 0 streams the FP8 weights directly (each byte read once, expanded to bf16 in
- *   registers for the tensor cores); a larger side expands its weights to bf16 in the workspace
- *   once (exactly: every E4M3 value is a bf16 value) and runs the tcgen05 GEMM.  Requires
- *   d_R_in % 8 == 0 and d_C_in % 8 == 0.  Workspace: rocs_linear_ikbo_w8_workspace.
+ *   (Q_RR, s_RR), (Q_CR, s_CR), (Q_CC, s_CC).  Shapes as rocs_linear_ikbo; Q_* [out, in] uint8;
+ *   s_* [out] float32.  By default a GEMM side with at most 64 rows streams the weights through
+ *   a register-tiled kernel (each byte read once, converted to f16 operands in registers), and a
+ *   larger side expands its weights to bf16 in the workspace once (exactly) and runs the tcgen05
+ *   GEMM.  With rocs_set_w8_tensor_cores(handle, 1) and d_R_in, d_C_in multiples of 128, the FP8
+ *   weights go to the tcgen05 tensor cores directly instead: TMA brings each weight tile into
+ *   shared memory as bytes, where it is converted to f16 exactly (every E4M3 value is an f16
+ *   value) and multiplied with the activations, brought to f16 once per call with a per-row
+ *   power-of-two shift that the epilogue undoes; the weights then must be 16-byte aligned.  Both
+ *   give the same results up to fp32 summation order.  Requires d_R_in % 8 == 0 and
+ *   d_C_in % 8 == 0; weights at least 8-byte aligned.  Workspace: rocs_linear_ikbo_w8_workspace
+ *   (query it after choosing the path: the two paths need different amounts).
  * ---------------------------------------------------------------------------------------- */
 rocs_status rocs_quantize_weights_fp8(rocs_handle_t handle, const void* W, rocs_dtype w_dtype, int32_t rows,
                                       int32_t cols, uint8_t* Q, float* scale, void* stream);
@@ -456,6 +462,13 @@ rocs_status rocs_test_withhold_ikbo_flag(rocs_handle_t handle, int32_t flag_inde
  * exponentials per second to *exp2_per_second.  Synchronises `stream`; allocates nothing.
  * Errors: ROCS_ERR_INVALID_ARG (NULL handle or output, n_poly outside [0, 8]); ROCS_ERR_CUDA. */
 rocs_status rocs_probe_exp2_rate(rocs_handle_t handle, int32_t n_poly, double* exp2_per_second, void* stream);
+
+/* FP8-weight linears on the tensor cores ([UGS] §三 Stage 4): with enable = 1, rocs_linear_ikbo_w8
+ * on this handle feeds the E4M3 weights to tcgen05 MMAs through a shared-memory conversion to f16
+ * (when both input widths are multiples of 128); with enable = 0, the default, it uses the
+ * register-tiled weight-streaming kernel and the bf16 expansion, which measured faster on most
+ * shapes.  Errors: ROCS_ERR_INVALID_ARG for a NULL handle or another value of enable. */
+rocs_status rocs_set_w8_tensor_cores(rocs_handle_t handle, int32_t enable);
 
 /* ------------------------------------------------------------------------------------------
  * Per-launch timing (tracing).  After rocs_timing_start(h, max_launches), every kernel the

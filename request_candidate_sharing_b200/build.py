@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "librocs.so")
 
-SOURCES = ["api.cpp", "gemm_tc.cu", "misc.cu", "layernorm.cu", "fm.cu", "attention.cu", "attn_stream.cu", "attn_tc.cu", "attn_req.cu", "noalloc.cu", "sort.cu", "w8.cu", "probe.cu"]
+SOURCES = ["api.cpp", "gemm_tc.cu", "misc.cu", "layernorm.cu", "fm.cu", "attention.cu", "attn_stream.cu", "attn_tc.cu", "attn_req.cu", "noalloc.cu", "sort.cu", "w8.cu", "w8_tc.cu", "probe.cu"]
 HEADERS = ["common.cuh", "internal.h", "mma_frag.cuh", "softmax_math.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",

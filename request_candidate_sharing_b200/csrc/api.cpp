@@ -399,12 +399,25 @@ struct W8Plan {
   void *XhR = nullptr, *XhC = nullptr;                    // f16 activations (weight-streaming paths only)
   int *shR = nullptr, *shC = nullptr;
   bool req_skinny = false, cand_skinny = false;
+  bool tc = false;   // the FP8-weight tcgen05 GEMM on both sides (input widths multiples of 64)
   size_t bytes = 0;
 };
 
-W8Plan plan_w8(const rocs_ikbo_desc* d, void* ws) {
+W8Plan plan_w8(const rocs_context* h, const rocs_ikbo_desc* d, void* ws) {
   W8Plan p;
   Carver c(ws);
+  p.tc = h->w8_tensor_cores && w8_tc_supported(d->d_R_in, d->d_C_out) && w8_tc_supported(d->d_C_in, d->d_C_out);
+  if (p.tc) {
+    p.Z = (float*)c.take((size_t)d->B_R * d->d_C_out * 4);
+    p.XhR = c.take((size_t)d->B_R * d->d_R_in * 2);
+    p.shR = (int*)c.take((size_t)d->B_R * 4);
+    if (d->B_C > 0) {
+      p.XhC = c.take((size_t)d->B_C * d->d_C_in * 2);
+      p.shC = (int*)c.take((size_t)d->B_C * 4);
+    }
+    p.bytes = c.used;
+    return p;
+  }
   p.req_skinny = w8_skinny_supported(d->B_R, d->d_R_in);
   p.cand_skinny = d->B_C == 0 || w8_skinny_supported((int)d->B_C, d->d_C_in);
   p.Z = (float*)c.take((size_t)d->B_R * d->d_C_out * 4);
@@ -449,7 +462,7 @@ extern "C" rocs_status rocs_quantize_weights_fp8(rocs_handle_t h, const void* W,
 extern "C" rocs_status rocs_linear_ikbo_w8_workspace(rocs_handle_t h, const rocs_ikbo_desc* d, size_t* bytes) {
   ROCS_REQUIRE(h && bytes, "rocs_linear_ikbo_w8_workspace: NULL argument");
   ROCS_TRY(check_w8_desc(d));
-  *bytes = plan_w8(d, nullptr).bytes;
+  *bytes = plan_w8(h, d, nullptr).bytes;
   return ROCS_OK;
 }
 
@@ -469,14 +482,51 @@ extern "C" rocs_status rocs_linear_ikbo_w8(rocs_handle_t h, const rocs_ikbo_desc
   for (const void* p : ptrs) ROCS_REQUIRE(aligned16(p), "rocs_linear_ikbo_w8: X, Y and workspace must be 16-byte aligned");
   const void* wq[] = {Q_RR, Q_CR, Q_CC};
   for (const void* p : wq) ROCS_REQUIRE(((uintptr_t)p & 7) == 0, "rocs_linear_ikbo_w8: weights must be 8-byte aligned");
-  const W8Plan need = plan_w8(d, nullptr);
+  const W8Plan need = plan_w8(h, d, nullptr);
   if (ws_bytes < need.bytes) {
     set_error("rocs_linear_ikbo_w8: workspace %zu B < required %zu B", ws_bytes, need.bytes);
     return ROCS_ERR_WORKSPACE;
   }
-  const W8Plan p = plan_w8(d, ws);
+  const W8Plan p = plan_w8(h, d, ws);
   cudaStream_t s = (cudaStream_t)stream;
   const int out_bf16 = d->dtype_out == ROCS_BF16;
+  if (p.tc) {
+    // FP8 weights straight to the tensor cores: activations to f16 once (both sides, one launch),
+    // then [Y^R | Z] in one launch and the candidate GEMM with the Z[m] gather in a second
+    for (const void* q : wq)
+      ROCS_REQUIRE(((uintptr_t)q & 15) == 0, "rocs_linear_ikbo_w8: weights must be 16-byte aligned");
+    {
+      SiteLabel sl("ikbo_w8");
+      ROCS_TRY(launch_w8_xprep(X_R, d->d_R_in, d->B_R, d->d_R_in, p.XhR, p.shR, X_C, d->d_C_in, (int)d->B_C,
+                               d->d_C_in, p.XhC, p.shC, s));
+    }
+    W8GemmDesc req[2];
+    int nreq = 0;
+    if (d->d_R_out > 0) {
+      W8GemmDesc& g = req[nreq++];
+      g.Xh = p.XhR; g.ldx = d->d_R_in; g.shift = p.shR; g.M = d->B_R; g.K = d->d_R_in;
+      g.W8 = Q_RR; g.N = d->d_R_out; g.scale = s_RR; g.bias = b_R;
+      g.out = Y_R; g.ldo = d->d_R_out; g.out_bf16 = out_bf16; g.act = d->act;
+    }
+    {
+      W8GemmDesc& g = req[nreq++];
+      g.Xh = p.XhR; g.ldx = d->d_R_in; g.shift = p.shR; g.M = d->B_R; g.K = d->d_R_in;
+      g.W8 = Q_CR; g.N = d->d_C_out; g.scale = s_CR; g.bias = b_C;
+      g.out = p.Z; g.ldo = d->d_C_out; g.out_bf16 = 0; g.act = ROCS_ACT_NONE;
+    }
+    {
+      SiteLabel sl("ikbo_w8.req");
+      ROCS_TRY(launch_gemm_w8(h, req, nreq, s));
+    }
+    if (d->B_C == 0) return ROCS_OK;
+    W8GemmDesc g;
+    g.Xh = p.XhC; g.ldx = d->d_C_in; g.shift = p.shC; g.M = (int)d->B_C; g.K = d->d_C_in;
+    g.W8 = Q_CC; g.N = d->d_C_out; g.scale = s_CC;
+    g.Z = p.Z; g.ldz = d->d_C_out; g.gidx = req_idx; g.gidx_bound = d->B_R;
+    g.out = Y_C; g.ldo = d->d_C_out; g.out_bf16 = out_bf16; g.act = d->act;
+    SiteLabel sl("ikbo_w8.cand");
+    return launch_gemm_w8(h, &g, 1, s);
+  }
   // request side: weight-streaming kernel at small B_R, else the bf16 expansion and the tcgen05
   // GEMM (both with the channel scales on the accumulator)
   IkboArgs a;
@@ -1347,6 +1397,13 @@ extern "C" rocs_status rocs_set_ikbo_fused(rocs_handle_t h, int32_t enable) {
   ROCS_REQUIRE(h, "rocs_set_ikbo_fused: handle is NULL");
   ROCS_REQUIRE(enable == 0 || enable == 1, "rocs_set_ikbo_fused: enable must be 0 or 1");
   h->ikbo_fused = enable;
+  return ROCS_OK;
+}
+
+extern "C" rocs_status rocs_set_w8_tensor_cores(rocs_handle_t h, int32_t enable) {
+  ROCS_REQUIRE(h, "rocs_set_w8_tensor_cores: handle is NULL");
+  ROCS_REQUIRE(enable == 0 || enable == 1, "rocs_set_w8_tensor_cores: enable must be 0 or 1");
+  h->w8_tensor_cores = enable;
   return ROCS_OK;
 }
 

@@ -34,6 +34,7 @@ struct rocs_context {
   RocsTimer timer;
   int graph_replay = 1;                 // rocs_set_graph_replay
   int ikbo_fused = 1;                   // rocs_set_ikbo_fused
+  int w8_tensor_cores = 0;              // rocs_set_w8_tensor_cores: FP8 operands on tcgen05 (opt-in)
   int test_withhold_flag = -1;          // rocs_test_withhold_ikbo_flag: flag never published (-1: none)
   long long test_flag_budget = 0;       // ... and the flag-wait budget in SM cycles (0: the default ~1 s)
   cudaStream_t capture_stream = nullptr;   // forward graphs are captured here (never the legacy stream)
@@ -122,6 +123,19 @@ rocs_status launch_w8_quantize(const void* W, int w_bf16, int rows, int cols, ui
 // E4M3 -> bf16, exact (count even)
 rocs_status launch_w8_expand(const uint8_t* Q, long long count, void* out, cudaStream_t s);
 bool w8_skinny_supported(int M, int K);
+// FP8-weight GEMM on the tensor cores (w8_tc.cu):
+//   out[r, c] = act(2^shift[r] * scale[c] * sum_k Xh[r, k] q[c, k] + bias[c] + Z[gidx[r], c])
+// Xh [M, K] f16 with row shifts from launch_w8_xprep, q [N, K] E4M3 bytes (16-byte aligned),
+// K % 64 == 0.  Up to three problems share one persistent launch (problem-major tile order).
+struct W8GemmDesc {
+  const void* Xh = nullptr; long long ldx = 0; const int* shift = nullptr; int M = 0; int K = 0;
+  const uint8_t* W8 = nullptr; int N = 0;
+  const float* scale = nullptr; const float* bias = nullptr;
+  const float* Z = nullptr; long long ldz = 0; const int32_t* gidx = nullptr; int gidx_bound = 0;
+  void* out = nullptr; long long ldo = 0; int out_bf16 = 1; int act = ROCS_ACT_NONE;
+};
+bool w8_tc_supported(int K, int N);
+rocs_status launch_gemm_w8(rocs_context* ctx, const W8GemmDesc* probs, int nprob, cudaStream_t s);
 // X [M, K] bf16 (row stride ldx) -> Xh [M, K] f16 times 2^-shift[m], the operand of launch_w8_skinny;
 // two activation sets in one launch (M1 may be 0)
 rocs_status launch_w8_xprep(const void* X0, long long ldx0, int M0, int K0, void* Xh0, int* sh0, const void* X1,

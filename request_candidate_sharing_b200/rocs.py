@@ -127,6 +127,7 @@ _lib_graph = _proto("rocs_set_graph_replay", P, I32)
 _lib_fused = _proto("rocs_set_ikbo_fused", P, I32)
 _lib_withhold = _proto("rocs_test_withhold_ikbo_flag", P, I32, I64)
 _lib_probe = _proto("rocs_probe_exp2_rate", P, I32, C.POINTER(C.c_double), P)
+_lib_w8tc = _proto("rocs_set_w8_tensor_cores", P, I32)
 _lib_q8 = _proto("rocs_quantize_weights_fp8", P, P, C.c_int, I32, I32, P, P, P)
 _lib_w8_ws = _proto("rocs_linear_ikbo_w8_workspace", P, C.POINTER(IkboDesc), C.POINTER(C.c_size_t))
 _lib_w8 = _proto("rocs_linear_ikbo_w8", P, C.POINTER(IkboDesc), P, P, P, P, P, P, P, P, P, P, P, P, P, P, C.c_size_t, P)
@@ -142,7 +143,7 @@ EXPORTED = ["rocs_linear_ikbo_noalloc", "rocs_timing_start", "rocs_timing_stop",
             "rocs_segments_from_counts", "rocs_linear_ikbo_workspace", "rocs_linear_ikbo", "rocs_group_layernorm",
             "rocs_fm_masked", "rocs_token_lcb_workspace", "rocs_token_lcb", "rocs_dca_cross_attn",
             "rocs_dca_encode_workspace", "rocs_dca_encode", "rocs_forward_workspace", "rocs_forward",
-            "rocs_set_graph_replay", "rocs_set_ikbo_fused", "rocs_test_withhold_ikbo_flag", "rocs_probe_exp2_rate", "rocs_sort_by_request_workspace",
+            "rocs_set_graph_replay", "rocs_set_ikbo_fused", "rocs_test_withhold_ikbo_flag", "rocs_probe_exp2_rate", "rocs_set_w8_tensor_cores", "rocs_sort_by_request_workspace",
             "rocs_sort_by_request", "rocs_dca_cross_attn_unsorted_workspace", "rocs_dca_cross_attn_unsorted",
             "rocs_quantize_weights_fp8", "rocs_linear_ikbo_w8_workspace", "rocs_linear_ikbo_w8"]
 
@@ -299,6 +300,9 @@ class Rocs:
 
     def rocs_test_withhold_ikbo_flag(self, flag_index: int, wait_budget_cycles: int = 0):
         _check(_lib_withhold(self.h, int(flag_index), int(wait_budget_cycles)))
+
+    def rocs_set_w8_tensor_cores(self, enable: int):
+        _check(_lib_w8tc(self.h, int(enable)))
 
     def rocs_probe_exp2_rate(self, n_poly: int, stream=None) -> float:
         r = C.c_double(0.0)

@@ -314,10 +314,17 @@ def _run_w8(R, case, x, q, m, out_dtype):
     ([40, 0, 23], 96, 200, 64, 136, 1),              # small M, candidate K not a multiple of 32 (expanded)
     ([300] * 5 + [7], 256, 512, 128, 384, 1),        # B_C > 64: expanded weights on the tcgen05 GEMM
     ([1] * 60 + [0] * 30, 512, 256, 0, 256, 0),     # B_R > 64 (expanded) with a small candidate side
+    ([130, 5, 300] * 50, 256, 384, 72, 200, 1),      # 150 requests, 21,750 candidates: several M tiles, a ragged
+                                                     # N tile, two and three weight tiles of 128 k bytes on the
+                                                     # FP8 tensor-core path
+    ([3] * 7, 4096, 4096, 1024, 384, 0),             # long K (64 k blocks), fp32 out
 ])
-def test_linear_ikbo_w8(R, counts, dRi, dCi, dRo, dCo, out):
+@pytest.mark.parametrize("tc", [0, 1])
+def test_linear_ikbo_w8(R, counts, dRi, dCi, dRo, dCo, out, tc):
     """W8A16 IKBO linear against the oracle's early-broadcast evaluation with the effective weights
-    q * s, on the weight-streaming kernel, the expanded-weight GEMM, and mixes of the two."""
+    q * s, on both paths: the default one (the weight-streaming kernel for sides of at most 64 rows,
+    the expanded-weight GEMM otherwise) and, with tc = 1, the FP8-operand tensor-core GEMM wherever
+    both input widths are multiples of 128."""
     from oracle import fp8
     case = synth.LinearCase("w8", np.asarray(counts, np.int32), dRi, dCi, dRo, dCo, "gelu", True, 13)
     x = synth.linear_inputs(case)
@@ -327,7 +334,11 @@ def test_linear_ikbo_w8(R, counts, dRi, dCi, dRo, dCo, out):
         if k == "RR" and dRo == 0:
             continue
         q["Q_" + k], q["s_" + k] = fp8.quantize_rows(x["W_" + k])
-    YR, YC = _run_w8(R, case, x, q, m, out)
+    try:
+        R.rocs_set_w8_tensor_cores(tc)
+        YR, YC = _run_w8(R, case, x, q, m, out)
+    finally:
+        R.rocs_set_w8_tensor_cores(0)
     rR, rC = fp8.w8_glm_linear(x["X_R"], x["X_C"], m, q.get("Q_RR"), q.get("s_RR"), q["Q_CR"], q["s_CR"], q["Q_CC"],
                                q["s_CC"], x["b_R"] if dRo else None, x["b_C"], "gelu")
     if dRo:
