@@ -941,8 +941,11 @@ def run_w8a16(args, rank, world, local):
         return ts[len(ts) // 2]
 
     points = []
+    only = tuple(int(v) for v in args.sweep_point.split(",")) if args.sweep_point else None
     for (B_R, N, di, do) in ((1, 16, 1280, 2560), (1, 16, 1280, 640), (1, 8, 1280, 2560), (1, 8, 1280, 640),
                              (1, 16, 8192, 8192), (4, 16, 4096, 16384)):
+        if only is not None and (B_R, N, di, do) != only:
+            continue
         B_C = B_R * N
         g = torch.Generator(device=dev).manual_seed(di + do + N)
         bf = torch.bfloat16
@@ -1143,7 +1146,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-baselines", action="store_true", help="skip the GPU materialised-broadcast baselines")
     ap.add_argument("--requests", type=int, default=0, help="keep only the first N requests (profiling runs)")
-    ap.add_argument("--sweep-point", default="", help="ikbo_sweep: run only the point 'N,d' (profiling runs)")
+    ap.add_argument("--sweep-point", default="", help="ikbo_sweep: run only the point 'N,d'; w8a16: only "
+                                                      "'B_R,N,d_in,d_out' (profiling runs)")
     ap.add_argument("--ikbo-fused", type=int, default=1, choices=[0, 1],
                     help="IKBO linears as one fused launch (1, the library default) or two launches (0)")
     args = ap.parse_args()
