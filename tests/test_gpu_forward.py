@@ -82,6 +82,26 @@ def test_forward_glm_stack_narrow_candidates(R):
     check_bf16(host(out["E_C"][:case.B_C]), ref["E_C"], what="E_C")
 
 
+@pytest.mark.parametrize("cfg", ["cfg3", "cfg4", "cfg5"])
+def test_forward_without_candidates(R, cfg):
+    """A batch whose requests have no candidates at all (B_C = 0): the request-side results still
+    match the oracle, and no candidate pointer is needed."""
+    kw = dict(L=256) if cfg == "cfg5" else {}
+    case = getattr(synth, "model_" + cfg)(B_R=3, counts=[0, 0, 0], **kw)
+    assert case.B_C == 0
+    x, W = synth.model_inputs(case), synth.model_weights(case)
+    out = run_forward(R, case, x, W)
+    off, m = O.segments(case.counts)
+    assert np.array_equal(out["offsets"].cpu().numpy(), off)
+    ref = getattr(O, "forward_" + cfg)(case, x, W, m)
+    if case.glm is not None:
+        check_bf16(host(out["E_R"]), ref["E_R"], what="E_R")
+    if case.dca is not None:
+        for l in range(case.dca.layers):
+            check_bf16(host(out["S"][l]), ref["S"][l], out_bf16=True, what=f"S_{l}")
+            check_bf16(host(out["A_R"][l]), ref["A_R"][l], what=f"A_R_{l}")
+
+
 def test_forward_glm_invariant_on_gpu(R):
     case = synth.model_cfg3(B_R=2, counts=[9, 4])
     x, W = synth.model_inputs(case), synth.model_weights(case)
