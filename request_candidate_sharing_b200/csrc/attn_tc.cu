@@ -5,17 +5,22 @@
 // cross-attention) reads the same K/V; [REV] §2.4 (IKBO-DCA): the kernel consumes request-batch
 // K/V directly, never a per-candidate copy.
 //
-// One CTA per (request, head), three warpgroups (384 threads):
-//   warp 0      TMA: the head's K and V (L x d_h bf16) into shared memory ONCE, in 128-key blocks
-//               with one mbarrier each (compute starts when block 0 lands); 128-row query tiles
-//               (bf16, or a hi/lo pair), one per softmax warpgroup.
-//   warp 1      allocates TMEM; one thread issues, for both query tiles in flight and each
-//               128-key block j,
-//                 S_j = Q K_j^T       (tcgen05.mma M=128, N=128, K=d_h; one S buffer per tile)
+// Persistent: one CTA per SM, each over its share of the (request, head) items, dealt out in
+// alternating directions.  Three warpgroups (384 threads):
+//   warp 0      TMA: the item's K and V (L x d_h bf16) into shared memory ONCE, in 128-key blocks
+//               with one mbarrier each.  Block j of the next item is loaded as soon as the groups
+//               that read block j of the current one are done with it, so items follow each other
+//               without a pipeline drain, and the CTA's startup (TMEM, barriers, first loads) is
+//               paid once per SM instead of once per item.
+//   warp 3      the query tiles (bf16, or a hi/lo pair) of all the CTA's items, alternating between
+//               the two softmax warpgroups (an odd tile count of one item no longer leaves a group
+//               idle), each with a small descriptor (rows, head, keys) in shared memory.
+//   warps 1, 2  one MMA issuer per group; one thread issues, for each 128-key block j,
+//                 S_j = Q K_j^T       (tcgen05.mma M=128, N=128, K=d_h; one S buffer per group)
 //                 O  += P_j V_j       (M=128, N=d_h, K=128; V read as an MN-major operand; O
 //                                      accumulates in TMEM across the key blocks)
-//               issuing both tiles' S blocks before it waits on either tile's P, so one tile's
-//               exponentials overlap the other tile's tensor-core work.
+//               issuing the next S block before it waits on the current P, so the group's
+//               exponentials overlap the other group's tensor-core work.
 //   warps 4..11 two softmax warpgroups, one thread per query row (TMEM lane): the S row is read
 //               from TMEM in one batch, its maximum and exp2 taken in registers (no shuffles; part
 //               of the exponentials on the FMA pipe as a polynomial), P_j written back to TMEM as
@@ -144,10 +149,77 @@ struct AtCfg {
   static_assert(L_COL + (SUM_MMA ? GROUPS * 16 : 0) <= 512, "tensor memory columns");
 };
 
+constexpr int AT_DESC = 4;   // tile descriptors in flight per softmax warpgroup
+
+// One query tile of a softmax warpgroup, published by the query producer.  The MMA issuer and
+// the softmax warpgroup of that group read it; the softmax reads it again when it writes the
+// tile's output, one tile later.
+struct AtTile {
+  long long q0;      // first query row of the tile's request
+  long long q1;      // end of the request's query rows
+  int tile;          // tile index within the request; -1 closes the group's tile stream
+  int h;             // head
+  int Lr;            // keys of the request
+  int nkb;           // key blocks of the request
+  uint32_t kv_par;   // bit j: phase parity of kv_full[j] for this request's load
+  uint32_t flags;    // AT_LAST | AT_TAIL | AT_TAIL_PAR
+};
+constexpr uint32_t AT_LAST = 1;       // the group's last tile of this request
+constexpr uint32_t AT_TAIL = 2;       // the last key block has padding rows (zeroed before P V)
+constexpr uint32_t AT_TAIL_PAR = 4;   // phase parity of vtail[nkb - 1] for this request
+
+// Work item n of the list (request rb in processing order, head h), its query rows and keys.
+struct AtItem {
+  long long q0, q1;
+  int r, h, Lr, nkb, ntiles;
+};
+
+// Geometry of item idx = rb * H + h.  An item whose offsets or key count are invalid gets
+// ntiles = 0 and `bad` the status to report.
+template <bool RAGGED>
+__device__ __forceinline__ void at_item(const AttnTcParams& P, int idx, AtItem& it, int& bad) {
+  const int rb = idx / P.H;
+  it.h = idx - rb * P.H;
+  it.r = P.order != nullptr ? P.order[rb] : rb;
+  it.ntiles = 0;
+  it.nkb = 0;
+  bad = 0;
+  if (it.r < 0 || it.r >= P.B_R) {
+    bad = ROCS_ERR_INDEX;
+    return;
+  }
+  it.q0 = P.offsets[it.r];
+  it.q1 = P.offsets[it.r + 1];
+  if (it.q0 < 0 || it.q1 < it.q0 || it.q1 > P.rows) {
+    bad = ROCS_ERR_INDEX;
+    return;
+  }
+  // the request's keys: the first Lr rows of its L-row K/V (a ragged history), Lr in [1, L]
+  it.Lr = RAGGED ? P.kv_len[it.r] : P.L;
+  if (RAGGED && (it.Lr < 1 || it.Lr > P.L)) {
+    bad = ROCS_ERR_COUNTS;
+    return;
+  }
+  // a ragged self-attention: the padding rows are no queries either
+  if (RAGGED && P.q_by_kv && it.q1 > it.q0 + it.Lr) it.q1 = it.q0 + it.Lr;
+  it.ntiles = (int)((it.q1 - it.q0 + TQ - 1) / TQ);
+  it.nkb = RAGGED ? (it.Lr + TK - 1) / TK : P.nkb;
+}
+
+// Item index of pass `pass` for this CTA: the list is dealt out in alternating directions
+// (CTA c takes items c, 2G - 1 - c, 2G + c, ...), so that a list sorted heaviest first spreads
+// evenly over the CTAs.  Returns -1 past the end of the list.
+__device__ __forceinline__ int at_item_index(int pass, int n_items) {
+  const int G = (int)gridDim.x, c = (int)blockIdx.x;
+  const long long idx = (long long)pass * G + ((pass & 1) ? G - 1 - c : c);
+  return idx < n_items ? (int)idx : -1;
+}
+
 template <int DH, bool SPLIT, bool RAGGED>
 __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __grid_constant__ AttnTcParams P) {
   using C = AtCfg<DH>;
   constexpr int GROUPS = C::GROUPS;
+  static_assert(GROUPS == 2, "query tiles alternate between two softmax warpgroups");
   constexpr int ROWB = DH * 2;                        // bytes per K/V/Q row
   constexpr uint32_t SW = DH == 32 ? 4u : 2u;         // 64-B or 128-B swizzle for K/V/Q
   constexpr uint32_t SBO = 8 * ROWB;                  // 8-row group stride
@@ -158,29 +230,7 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
   constexpr uint32_t IDESC_S = idesc_bf16(TQ, TK, false);
   constexpr uint32_t IDESC_O = idesc_bf16(TQ, DH, true);
   constexpr uint32_t IDESC_L = idesc_bf16(TQ, 16, false);
-
-  const int rb = blockIdx.x / P.H;
-  const int h = blockIdx.x - rb * P.H;
-  const int r = P.order != nullptr ? P.order[rb] : rb;
-  const long long q0 = P.offsets[r];
-  long long q1 = P.offsets[r + 1];
-  if (q0 < 0 || q1 < q0 || q1 > P.rows) {
-    if (threadIdx.x == 0) set_status(P.status, ROCS_ERR_INDEX);
-    return;
-  }
-  // this request's keys: the first Lr rows of its L-row K/V (a ragged history), Lr in [1, L];
-  // without per-request lengths (RAGGED false) every request has L keys
-  const int Lr = RAGGED ? P.kv_len[r] : P.L;
-  if (RAGGED && (Lr < 1 || Lr > P.L)) {
-    if (threadIdx.x == 0) set_status(P.status, ROCS_ERR_COUNTS);
-    return;
-  }
-  // a ragged self-attention: the padding rows are no queries either
-  if (RAGGED && P.q_by_kv) q1 = q1 < q0 + Lr ? q1 : q0 + Lr;
-  const int ntiles = (int)((q1 - q0 + TQ - 1) / TQ);
-  if (ntiles == 0) return;
-  const int nkb = RAGGED ? (Lr + TK - 1) / TK : P.nkb;
-  const int tail_keys = nkb * TK - Lr;   // padding rows in the last staged key block
+  const int n_items = P.B_R * P.H;
 
   extern __shared__ uint8_t at_smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(at_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -188,25 +238,29 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
   uint8_t* sV = sK + P.nkb * KV_BLOCK;
   uint8_t* sQ = sV + P.nkb * KV_BLOCK;                // [GROUPS][NQ][Q_TILE]
   uint8_t* sOnes = sQ + GROUPS * NQ * Q_TILE;         // 1024-B aligned (Q tiles are 8 KiB multiples)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sOnes + ONES_BYTES);
-  uint64_t* kv_full = bars;                           // [AT_MAX_KB]
-  uint64_t* q_full = kv_full + AT_MAX_KB;             // [GROUPS] each
+  AtTile* descs = reinterpret_cast<AtTile*>(sOnes + ONES_BYTES);   // [GROUPS][AT_DESC]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(descs + GROUPS * AT_DESC);
+  uint64_t* kv_full = bars;                           // [AT_MAX_KB]: block j of the current request landed
+  uint64_t* kv_empty = kv_full + AT_MAX_KB;           // [AT_MAX_KB][GROUPS]: group g done with block j
+  uint64_t* vtail = kv_empty + AT_MAX_KB * GROUPS;    // [AT_MAX_KB]: block j's padding rows zeroed
+  uint64_t* q_full = vtail + AT_MAX_KB;               // [GROUPS] each
   uint64_t* q_free = q_full + GROUPS;
   uint64_t* s_full = q_free + GROUPS;
   uint64_t* s_free = s_full + GROUPS;
   uint64_t* p_full = s_free + GROUPS;                 // [GROUPS][2]: P half h of the block written
   uint64_t* o_full = p_full + 2 * GROUPS;             // [GROUPS][2]: P half h times V consumed
   uint64_t* drain = o_full + 2 * GROUPS;              // [GROUPS]
-  uint64_t* vtail = drain + GROUPS;                   // the last V block's rows past Lr are zeroed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(vtail + 1);
+  uint64_t* d_full = drain + GROUPS;                  // [GROUPS][AT_DESC]: tile descriptor written
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(d_full + GROUPS * AT_DESC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  // ragged: the request's key blocks and keys, re-read by the softmax warps where they need them
-  // (kept out of their registers; otherwise they read the launch parameters)
-  int* at_geom = reinterpret_cast<int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < AT_MAX_KB; ++i) mbar_init(&kv_full[i], 1);
+    for (int i = 0; i < AT_MAX_KB; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&vtail[i], 1);
+      for (int g = 0; g < GROUPS; ++g) mbar_init(&kv_empty[i * GROUPS + g], 1);
+    }
     for (int g = 0; g < GROUPS; ++g) {
       mbar_init(&q_full[g], 1);
       mbar_init(&q_free[g], 1);
@@ -217,10 +271,8 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
         mbar_init(&o_full[2 * g + hh], 1);
       }
       mbar_init(&drain[g], 1);
+      for (int s = 0; s < AT_DESC; ++s) mbar_init(&d_full[g * AT_DESC + s], 1);
     }
-    mbar_init(vtail, 1);
-    at_geom[0] = nkb;
-    at_geom[1] = Lr;
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -236,61 +288,160 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // group G takes tiles G, G + GROUPS, ...; its sequence has tiles_g(G) * nkb key blocks
-  auto tiles_g = [&](int g) { return ntiles > g ? (ntiles - g + GROUPS - 1) / GROUPS : 0; };
 
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REG_CTRL));
-    if (warp == 0 && lane == 0) {
-      // ---------------- TMA producer ----------------
-      prefetch_tensormap(&P.tmQ);
-      prefetch_tensormap(&P.tmK);
-      prefetch_tensormap(&P.tmV);
-      const int kv_row0 = r * P.L;
-      for (int j = 0; j < nkb; ++j) {
-        mbar_arrive_expect_tx(&kv_full[j], 2 * KV_BLOCK);
-        tma_load_2d(sK + j * KV_BLOCK, &P.tmK, &kv_full[j], h * DH, kv_row0 + j * TK);
-        tma_load_2d(sV + j * KV_BLOCK, &P.tmV, &kv_full[j], h * DH, kv_row0 + j * TK);
+    if (warp == 0) {
+      // ---------------- K/V producer (the whole warp; lane 0 issues the copies) ----------------
+      // Block j of the next request is loaded as soon as every group that read block j of the
+      // previous one has finished with it (kv_empty), so a group that runs out of tiles of one
+      // request starts the next request one block behind the other group instead of waiting
+      // for it.  Keys past Lr have P = 0, but their V rows still enter the P V product, where
+      // non-finite padding would give 0 * inf = NaN: once the last block has landed, the warp
+      // zeroes those rows (whole rows: the swizzle permutes 16-byte units within a row) and
+      // releases the block for P V (vtail).
+      if (lane == 0) {
+        prefetch_tensormap(&P.tmK);
+        prefetch_tensormap(&P.tmV);
       }
-      int last_t = -1;
-      for (int t = 0; t < ntiles; ++t) {
-        const int g = t % GROUPS, k = t / GROUPS;
-        if (k > 0 && !mbar_wait(&q_free[g], (k - 1) & 1, P.status, abort_flag)) break;
-        mbar_arrive_expect_tx(&q_full[g], NQ * Q_TILE);
-        const int qrow = (int)(q0 + (long long)t * TQ);
-        tma_load_2d(sQ + (g * NQ) * Q_TILE, &P.tmQ, &q_full[g], h * DH, qrow);
-        if (SPLIT) tma_load_2d(sQ + (g * NQ + 1) * Q_TILE, &P.tmQ, &q_full[g], (int)P.q_lo_col + h * DH, qrow);
-        last_t = t;
+      uint32_t kv_par = 0;     // bit j: parity of block j's next load
+      uint32_t last_par = 0;   // bit j: parity of block j's last load
+      uint32_t loaded = 0;     // bit j: block j has been loaded
+      uint32_t pend = 0;       // bit GROUPS j + g: group g reads block j's last load
+      uint32_t e_par = 0;      // bit GROUPS j + g: parity of kv_empty[j][g]'s next completion
+      int tcount = 0;          // query tiles of the items so far (tile t goes to group t % 2)
+      bool ok = true;
+      for (int pass = 0; ok && pass * (long long)gridDim.x < n_items; ++pass) {
+        const int idx = at_item_index(pass, n_items);
+        if (idx < 0) continue;
+        AtItem it;
+        int bad;
+        at_item<RAGGED>(P, idx, it, bad);
+        if (it.ntiles == 0) continue;
+        const uint32_t used = it.ntiles >= 2 ? 3u : (1u << (tcount & 1));
+        const int kv_row0 = it.r * P.L;
+        for (int j = 0; j < it.nkb && ok; ++j) {
+#pragma unroll
+          for (int g = 0; g < GROUPS; ++g) {
+            const int b = GROUPS * j + g;
+            if (ok && ((pend >> b) & 1u)) {
+              ok = __all_sync(0xffffffffu, mbar_wait(&kv_empty[b], (e_par >> b) & 1u, P.status, abort_flag));
+              e_par ^= 1u << b;
+            }
+          }
+          if (!ok) break;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&kv_full[j], 2 * KV_BLOCK);
+            tma_load_2d(sK + j * KV_BLOCK, &P.tmK, &kv_full[j], it.h * DH, kv_row0 + j * TK);
+            tma_load_2d(sV + j * KV_BLOCK, &P.tmV, &kv_full[j], it.h * DH, kv_row0 + j * TK);
+          }
+          loaded |= 1u << j;
+          last_par = (last_par & ~(1u << j)) | (kv_par & (1u << j));
+          pend = (pend & ~(3u << (GROUPS * j))) | (used << (GROUPS * j));
+        }
+        if (!ok) break;
+        const int tail_keys = it.nkb * TK - it.Lr;   // padding rows in the last staged key block
+        if (tail_keys > 0) {
+          const int jb = it.nkb - 1;
+          if (!__all_sync(0xffffffffu, mbar_wait(&kv_full[jb], (kv_par >> jb) & 1u, P.status, abort_flag))) {
+            ok = false;
+            break;
+          }
+          uint8_t* vb = sV + jb * KV_BLOCK + (TK - tail_keys) * ROWB;
+          for (int i = lane; i < tail_keys * ROWB / 16; i += 32) reinterpret_cast<uint4*>(vb)[i] = make_uint4(0, 0, 0, 0);
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&vtail[jb]);
+        }
+        kv_par ^= (1u << it.nkb) - 1u;
+        tcount += it.ntiles;
       }
       // no copy of this CTA may still be landing when it exits
-      for (int j = 0; j < nkb; ++j) mbar_wait(&kv_full[j], 0, P.status, nullptr);
-      for (int t = last_t - GROUPS + 1 < 0 ? 0 : last_t - GROUPS + 1; t <= last_t; ++t)
-        mbar_wait(&q_full[t % GROUPS], (t / GROUPS) & 1, P.status, nullptr);
-    } else if (warp == 3 && tail_keys > 0) {
-      // ---------------- the last key block's padding rows ----------------
-      // Keys past Lr have P = 0, but their V rows still enter the P V product, where any
-      // non-finite padding would give 0 * inf = NaN.  Once the block has landed, this warp zeroes
-      // those rows (whole rows: the swizzle permutes 16-byte units within a row) and releases the
-      // block for P V.
-      if (__all_sync(0xffffffffu, mbar_wait(&kv_full[nkb - 1], 0, P.status, abort_flag))) {
-        uint8_t* vb = sV + (nkb - 1) * KV_BLOCK + (TK - tail_keys) * ROWB;
-        for (int i = lane; i < tail_keys * ROWB / 16; i += 32)
-          reinterpret_cast<uint4*>(vb)[i] = make_uint4(0, 0, 0, 0);
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
-        __syncwarp();
-        if (lane == 0) mbar_arrive(vtail);
+      if (lane == 0)
+        for (int j = 0; j < AT_MAX_KB; ++j)
+          if ((loaded >> j) & 1u) mbar_wait(&kv_full[j], (last_par >> j) & 1u, P.status, nullptr);
+    } else if (warp == 3 && lane == 0) {
+      // ---------------- query producer: tile descriptors and query tiles ----------------
+      // The query tiles of the CTA's requests alternate between the two groups; each group has
+      // one query buffer and AT_DESC descriptor slots.  A slot is rewritten only after the
+      // group's query buffer has been released three tiles later, by which time the softmax
+      // has written that tile's output (it does so while it works on the following tile).
+      prefetch_tensormap(&P.tmQ);
+      uint32_t kv_par = 0, vt_par = 0;
+      int tcount = 0, kq0 = 0, kq1 = 0;
+      bool ok = true;
+      for (int pass = 0; ok && pass * (long long)gridDim.x < n_items; ++pass) {
+        const int idx = at_item_index(pass, n_items);
+        if (idx < 0) continue;
+        AtItem it;
+        int bad;
+        at_item<RAGGED>(P, idx, it, bad);
+        if (bad != 0) set_status(P.status, bad);
+        if (it.ntiles == 0) continue;
+        const uint32_t item_par = kv_par;
+        kv_par ^= (1u << it.nkb) - 1u;
+        uint32_t tail_flags = 0;
+        if (it.nkb * TK > it.Lr) {
+          const int jb = it.nkb - 1;
+          tail_flags = AT_TAIL | (((vt_par >> jb) & 1u) ? AT_TAIL_PAR : 0u);
+          vt_par ^= 1u << jb;
+        }
+        for (int t = 0; t < it.ntiles; ++t) {
+          const int g = tcount & 1;
+          const int k = g ? kq1 : kq0;
+          if (k > 0 && !mbar_wait(&q_free[g], (k - 1) & 1, P.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int slot = g * AT_DESC + (k % AT_DESC);
+          AtTile& d = descs[slot];
+          d.q0 = it.q0;
+          d.q1 = it.q1;
+          d.tile = t;
+          d.h = it.h;
+          d.Lr = it.Lr;
+          d.nkb = it.nkb;
+          d.kv_par = item_par;
+          d.flags = tail_flags | (t + GROUPS >= it.ntiles ? AT_LAST : 0u);
+          mbar_arrive(&d_full[slot]);
+          mbar_arrive_expect_tx(&q_full[g], NQ * Q_TILE);
+          const int qrow = (int)(it.q0 + (long long)t * TQ);
+          tma_load_2d(sQ + (g * NQ) * Q_TILE, &P.tmQ, &q_full[g], it.h * DH, qrow);
+          if (SPLIT) tma_load_2d(sQ + (g * NQ + 1) * Q_TILE, &P.tmQ, &q_full[g], (int)P.q_lo_col + it.h * DH, qrow);
+          if (g) ++kq1; else ++kq0;
+          ++tcount;
+        }
+      }
+      // close each group's tile stream; by then its last query tile has been read
+#pragma unroll
+      for (int g = 0; g < GROUPS; ++g) {
+        const int k = g ? kq1 : kq0;
+        if (ok && k > 0 && !mbar_wait(&q_free[g], (k - 1) & 1, P.status, abort_flag)) ok = false;
+        if (ok) {
+          const int slot = g * AT_DESC + (k % AT_DESC);
+          descs[slot].tile = -1;
+          mbar_arrive(&d_full[slot]);
+        }
+      }
+      // no copy of this CTA may still be landing when it exits
+#pragma unroll
+      for (int g = 0; g < GROUPS; ++g) {
+        const int k = g ? kq1 : kq0;
+        if (k > 0) mbar_wait(&q_full[g], (k - 1) & 1, P.status, nullptr);
       }
     } else if (warp >= 1 && warp <= GROUPS && lane == 0) {
       // ---------------- MMA issuer of query-tile group g = warp - 1 ----------------
-      // Per key block i:  S_i = Q K_j^T once the softmax has read S_{i-1} (s_free); then, for the
-      // previous block, O += P V_j and l += P 1 in two 64-key halves, each once the softmax has
-      // written that half of P (p_full).  Each group's MMAs touch only its own TMEM columns.
+      // Per key block i of the group's tile stream:  S_i = Q K_j^T once the softmax has read
+      // S_{i-1} (s_free); then, for the previous block, O += P V_j and l += P 1 in two 64-key
+      // halves, each once the softmax has written that half of P (p_full).  After the group's
+      // last tile of a request, each block's P V is followed by a commit that hands the block
+      // back to the K/V producer (kv_empty).  Each group's MMAs touch only its own TMEM columns.
       const int g = warp - 1;
-      const int T = tiles_g(g) * nkb;
-      auto issue_pv = [&](int ib, int hh) -> bool {
+      auto issue_pv = [&](int ib, int hh, int j, uint32_t fl, int nkb) -> bool {
         if (!mbar_wait(&p_full[2 * g + hh], ib & 1, P.status, abort_flag)) return false;
-        const int j = ib % nkb;
-        if (j == nkb - 1 && tail_keys > 0 && !mbar_wait(vtail, 0, P.status, abort_flag)) return false;
+        if (hh == 0 && j == nkb - 1 && (fl & AT_TAIL) &&
+            !mbar_wait(&vtail[j], (fl & AT_TAIL_PAR) ? 1u : 0u, P.status, abort_flag))
+          return false;
         tc_fence_after();
         const uint32_t va = smem_u32(sV + j * KV_BLOCK);
 #pragma unroll
@@ -304,30 +455,70 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
                       (ks > 0 || j > 0) ? 1u : 0u);
         }
         tc_commit(&o_full[2 * g + hh]);
+        if (hh == 1 && (fl & AT_LAST)) tc_commit(&kv_empty[GROUPS * j + g]);
         return true;
       };
       bool ok = true;
-      for (int i = 0; i < T && ok; ++i) {
-        const int k = i / nkb, j = i - k * nkb;
-        if (j == 0 && !mbar_wait(&q_full[g], k & 1, P.status, abort_flag)) { ok = false; break; }
-        if (!mbar_wait(&kv_full[j], 0, P.status, abort_flag)) { ok = false; break; }
-        if (i > 0 && !mbar_wait(&s_free[g], (i - 1) & 1, P.status, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t qa = smem_u32(sQ + (g * NQ) * Q_TILE);
-        const uint32_t ka = smem_u32(sK + j * KV_BLOCK);
-#pragma unroll
-        for (int ks = 0; ks < DH / 16; ++ks) {
-          tc_mma_ss(tmem_base + C::S_COL + g * TK, sdesc(qa + ks * 32, SBO, SW), sdesc(ka + ks * 32, SBO, SW),
-                    IDESC_S, ks > 0 ? 1u : 0u);
-          if (SPLIT)
-            tc_mma_ss(tmem_base + C::S_COL + g * TK, sdesc(qa + Q_TILE + ks * 32, SBO, SW),
-                      sdesc(ka + ks * 32, SBO, SW), IDESC_S, 1u);
+      int k = 0, i = 0;
+      bool pend_pv = false;   // block i - 1's P V is not issued yet
+      int pj = 0, pnkb = 0;   // that block's index and its request's block count
+      uint32_t pfl = 0;       // and its tile's flags
+      for (;;) {
+        const int slot = g * AT_DESC + (k % AT_DESC);
+        if (!mbar_wait(&d_full[slot], (k / AT_DESC) & 1, P.status, abort_flag)) {
+          ok = false;
+          break;
         }
-        tc_commit(&s_full[g]);
-        if (j == nkb - 1) tc_commit(&q_free[g]);   // this tile's queries are no longer read
-        if (i > 0) ok = issue_pv(i - 1, 0) && issue_pv(i - 1, 1);
+        const int tile = descs[slot].tile;
+        if (tile < 0) break;
+        const int nkb = descs[slot].nkb;
+        const uint32_t kvp = descs[slot].kv_par, fl = descs[slot].flags;
+        if (!mbar_wait(&q_full[g], k & 1, P.status, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint32_t qa = smem_u32(sQ + (g * NQ) * Q_TILE);
+        for (int j = 0; j < nkb; ++j, ++i) {
+          if (!mbar_wait(&kv_full[j], (kvp >> j) & 1u, P.status, abort_flag) ||
+              (i > 0 && !mbar_wait(&s_free[g], (i - 1) & 1, P.status, abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t ka = smem_u32(sK + j * KV_BLOCK);
+#pragma unroll
+          for (int ks = 0; ks < DH / 16; ++ks) {
+            tc_mma_ss(tmem_base + C::S_COL + g * TK, sdesc(qa + ks * 32, SBO, SW), sdesc(ka + ks * 32, SBO, SW),
+                      IDESC_S, ks > 0 ? 1u : 0u);
+            if (SPLIT)
+              tc_mma_ss(tmem_base + C::S_COL + g * TK, sdesc(qa + Q_TILE + ks * 32, SBO, SW),
+                        sdesc(ka + ks * 32, SBO, SW), IDESC_S, 1u);
+          }
+          tc_commit(&s_full[g]);
+          if (j == nkb - 1) tc_commit(&q_free[g]);   // this tile's queries are no longer read
+          if (pend_pv && !(issue_pv(i - 1, 0, pj, pfl, pnkb) && issue_pv(i - 1, 1, pj, pfl, pnkb))) {
+            ok = false;
+            break;
+          }
+          pj = j;
+          pfl = fl;
+          pnkb = nkb;
+          pend_pv = true;
+        }
+        if (!ok) break;
+        // The group's last tile of a request: its last P V (and the hand-back of the last block)
+        // is issued now, not after the next tile's first S, which may need the next request's
+        // K/V, whose load waits for this hand-back.
+        if (fl & AT_LAST) {
+          if (!(issue_pv(i - 1, 0, pj, pfl, pnkb) && issue_pv(i - 1, 1, pj, pfl, pnkb))) {
+            ok = false;
+            break;
+          }
+          pend_pv = false;
+        }
+        ++k;
       }
-      if (ok && T > 0) ok = issue_pv(T - 1, 0) && issue_pv(T - 1, 1);
+      if (ok && pend_pv) ok = issue_pv(i - 1, 0, pj, pfl, pnkb) && issue_pv(i - 1, 1, pj, pfl, pnkb);
       tc_commit(&drain[g]);
       mbar_wait(&drain[g], 0, P.status, nullptr);
     }
@@ -342,13 +533,13 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
     const uint32_t paddr = lane_addr + C::P_COL + g * 64;
     const uint32_t oaddr = lane_addr + C::O_COL + g * DH;
     const uint32_t laddr = lane_addr + C::L_COL + g * 16;
-    volatile int* geom = at_geom;
-    const int Tg = tiles_g(g) * (RAGGED ? geom[0] : P.nkb);
+    // the group's tile descriptors, re-read where needed (kept out of the registers)
+    volatile AtTile* dq = descs + g * AT_DESC;
     const float sl2 = P.scale_log2;
     float m_cur = -INFINITY, l_reg = 0.f;
 
-    // O of the finished tile k_tile, divided by its row sum, to global memory
-    auto emit_row = [&](int k_tile) {
+    // O of the group's finished tile kt, divided by its row sum, to global memory
+    auto emit_row = [&](int kt) {
       float out[DH];
 #pragma unroll
       for (int c = 0; c < DH / 32; ++c) {
@@ -365,8 +556,10 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
         tmem_ld_wait();
         l_final = __uint_as_float(lw);
       }
-      const long long qrow0 = q0 + (long long)(g + GROUPS * k_tile) * TQ + row;
-      if (qrow0 >= q1) return;
+      volatile AtTile& d = dq[kt % AT_DESC];
+      const long long qrow0 = d.q0 + (long long)d.tile * TQ + row;
+      if (qrow0 >= d.q1) return;
+      const int h = d.h;
       const long long qrow = P.out_rows != nullptr ? (long long)P.out_rows[qrow0] : qrow0;
       const float inv = 1.0f / l_final;
 #pragma unroll
@@ -392,137 +585,146 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
     };
 
     bool ok = true;
-    const int nkb_g = RAGGED ? geom[0] : P.nkb;
-    int k_tile = 0, j = -1;
-    for (int i = 0; i < Tg; ++i) {
-      if (++j == nkb_g) { j = 0; ++k_tile; }
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[g], i & 1, P.status, abort_flag))) { ok = false; break; }
-      tc_fence_after();
-      // the whole S row into registers with one wait, then the S accumulator is released
-      uint32_t v[TK / 32][32];
-#pragma unroll
-      for (int c = 0; c < TK / 32; ++c) tmem_ld_32x32b_x32(saddr + c * 32, v[c]);
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&s_free[g]);
-      const int valid = (RAGGED ? geom[1] : P.L) - j * TK;   // keys of this block that exist (>= 1)
-      if (valid < TK) {
-#pragma unroll
-        for (int c = 0; c < TK / 32; ++c)
-#pragma unroll
-          for (int k = 0; k < 32; ++k)
-            if (c * 32 + k >= valid) v[c][k] = __float_as_uint(-INFINITY);
+    int k = 0, i = 0;
+    for (;;) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&d_full[g * AT_DESC + (k % AT_DESC)], (k / AT_DESC) & 1, P.status,
+                                             abort_flag))) {
+        ok = false;
+        break;
       }
-      // row maximum: eight chains of three-input max
-      float mt[8];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) mt[t] = fmaxf(__uint_as_float(v[0][t]), __uint_as_float(v[0][t + 8]));
-#pragma unroll
-      for (int e = 16; e < TK; e += 16)
-#pragma unroll
-        for (int t = 0; t < 8; ++t)
-          mt[t] = fmax3(mt[t], __uint_as_float(v[(e + t) >> 5][(e + t) & 31]),
-                        __uint_as_float(v[(e + 8 + t) >> 5][(e + 8 + t) & 31]));
-      const float mx = fmax3(fmax3(mt[0], mt[1], mt[2]), fmax3(mt[3], mt[4], mt[5]), fmaxf(mt[6], mt[7])) * sl2;
-      // the first block sets the row's reference maximum; later blocks move it only when some
-      // row of the warp would otherwise produce exponentials above 2^8 (warp-uniform, since the
-      // rescale is a warp-wide TMEM access)
-      float m_new = m_cur, corr = 1.0f;
-      const bool rescale = j != 0 && __any_sync(0xffffffffu, mx > m_cur + kLazyRescaleLog2);
-      if (j == 0) {
-        m_new = mx;
-      } else if (rescale) {
-        m_new = fmaxf(m_cur, mx);
-        corr = ex2_approx(m_cur - m_new);
-      }
-      // O is read (finished tile) or rescaled only once both halves of the previous block's P V
-      // have completed.  Otherwise those waits come later, just before each half of P is
-      // overwritten, so that the exponentials of the half are computed while the tensor core is
-      // still reading it.
-      const bool need_o = i > 0 && (j == 0 || rescale);
-      if (need_o) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&o_full[2 * g], (i - 1) & 1, P.status, abort_flag) &&
-                                         mbar_wait(&o_full[2 * g + 1], (i - 1) & 1, P.status, abort_flag))) {
-          ok = false;
-          break;
-        }
+      if (dq[k % AT_DESC].tile < 0) break;
+      const int nkb = dq[k % AT_DESC].nkb;
+      for (int j = 0; j < nkb; ++j, ++i) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&s_full[g], i & 1, P.status, abort_flag))) { ok = false; break; }
         tc_fence_after();
+        // the whole S row into registers with one wait, then the S accumulator is released
+        uint32_t v[TK / 32][32];
+#pragma unroll
+        for (int c = 0; c < TK / 32; ++c) tmem_ld_32x32b_x32(saddr + c * 32, v[c]);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&s_free[g]);
+        const int valid = dq[k % AT_DESC].Lr - j * TK;   // keys of this block that exist (>= 1)
+        if (valid < TK) {
+#pragma unroll
+          for (int c = 0; c < TK / 32; ++c)
+#pragma unroll
+            for (int kk = 0; kk < 32; ++kk)
+              if (c * 32 + kk >= valid) v[c][kk] = __float_as_uint(-INFINITY);
+        }
+        // row maximum: eight chains of three-input max
+        float mt[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) mt[t] = fmaxf(__uint_as_float(v[0][t]), __uint_as_float(v[0][t + 8]));
+#pragma unroll
+        for (int e = 16; e < TK; e += 16)
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+            mt[t] = fmax3(mt[t], __uint_as_float(v[(e + t) >> 5][(e + t) & 31]),
+                          __uint_as_float(v[(e + 8 + t) >> 5][(e + 8 + t) & 31]));
+        const float mx = fmax3(fmax3(mt[0], mt[1], mt[2]), fmax3(mt[3], mt[4], mt[5]), fmaxf(mt[6], mt[7])) * sl2;
+        // the first block sets the row's reference maximum; later blocks move it only when some
+        // row of the warp would otherwise produce exponentials above 2^8 (warp-uniform, since the
+        // rescale is a warp-wide TMEM access)
+        float m_new = m_cur, corr = 1.0f;
+        const bool rescale = j != 0 && __any_sync(0xffffffffu, mx > m_cur + kLazyRescaleLog2);
         if (j == 0) {
-          emit_row(k_tile - 1);
+          m_new = mx;
         } else if (rescale) {
-#pragma unroll
-          for (int c = 0; c < DH / 32; ++c) {
-            uint32_t w[32];
-            tmem_ld_32x32b_x32(oaddr + c * 32, w);
-            tmem_ld_wait();
-#pragma unroll
-            for (int k = 0; k < 32; ++k) w[k] = __float_as_uint(__uint_as_float(w[k]) * corr);
-            tmem_st_32x32b_x32(oaddr + c * 32, w);
-          }
-          if (C::SUM_MMA) {
-            uint32_t lw;
-            tmem_ld_32x32b_x1(laddr, lw);
-            tmem_ld_wait();
-            tmem_st_32x32b_x1(laddr, __float_as_uint(__uint_as_float(lw) * corr));
-          }
+          m_new = fmaxf(m_cur, mx);
+          corr = ex2_approx(m_cur - m_new);
         }
-      }
-      // exponentials: three pairs in eight on the FMA pipe (polynomial), the rest on MUFU; P_i
-      // as bf16 pairs into TMEM, one 64-key half at a time (32 keys per store), each half handed
-      // to the tensor core as soon as it is written
-      const float neg_m = -m_new;
-      float rs = 0.f;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t pk[2][16];
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int c = 2 * hh + cc;
-#pragma unroll
-          for (int k = 0; k < 32; k += 2) {
-            float x0, x1, p0, p1;
-            ffma2(__uint_as_float(v[c][k]), __uint_as_float(v[c][k + 1]), sl2, neg_m, x0, x1);
-            if (((k >> 1) & 7) >= 5) {
-              exp2_poly2(x0, x1, p0, p1);
-              if (valid < TK) {   // masked keys (x = -inf) must give exactly zero
-                p0 = x0 == -INFINITY ? 0.f : p0;
-                p1 = x1 == -INFINITY ? 0.f : p1;
-              }
-            } else {
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
-            }
-            if (!C::SUM_MMA) rs += p0 + p1;
-            pk[cc][k >> 1] = pack_bf16x2(p0, p1);
-          }
-        }
-        // this half of P may be overwritten once the previous block's P V of it has completed
-        if (i > 0 && !need_o) {
-          if (!__all_sync(0xffffffffu, mbar_wait(&o_full[2 * g + hh], (i - 1) & 1, P.status, abort_flag))) {
+        // O is read (finished tile) or rescaled only once both halves of the previous block's P V
+        // have completed.  Otherwise those waits come later, just before each half of P is
+        // overwritten, so that the exponentials of the half are computed while the tensor core is
+        // still reading it.
+        const bool need_o = i > 0 && (j == 0 || rescale);
+        if (need_o) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&o_full[2 * g], (i - 1) & 1, P.status, abort_flag) &&
+                                           mbar_wait(&o_full[2 * g + 1], (i - 1) & 1, P.status, abort_flag))) {
             ok = false;
             break;
           }
           tc_fence_after();
+          if (j == 0) {
+            emit_row(k - 1);
+          } else if (rescale) {
+#pragma unroll
+            for (int c = 0; c < DH / 32; ++c) {
+              uint32_t w[32];
+              tmem_ld_32x32b_x32(oaddr + c * 32, w);
+              tmem_ld_wait();
+#pragma unroll
+              for (int kk = 0; kk < 32; ++kk) w[kk] = __float_as_uint(__uint_as_float(w[kk]) * corr);
+              tmem_st_32x32b_x32(oaddr + c * 32, w);
+            }
+            if (C::SUM_MMA) {
+              uint32_t lw;
+              tmem_ld_32x32b_x1(laddr, lw);
+              tmem_ld_wait();
+              tmem_st_32x32b_x1(laddr, __float_as_uint(__uint_as_float(lw) * corr));
+            }
+          }
         }
-        tmem_st_32x32b_x16(paddr + (2 * hh) * 16, pk[0]);
-        tmem_st_32x32b_x16(paddr + (2 * hh + 1) * 16, pk[1]);
-        if (hh == 0) {
-          tmem_st_wait();
-          tc_fence_before();
-          mbar_arrive(&p_full[2 * g]);
+        // exponentials: three pairs in eight on the FMA pipe (polynomial), the rest on MUFU; P_i
+        // as bf16 pairs into TMEM, one 64-key half at a time (32 keys per store), each half handed
+        // to the tensor core as soon as it is written
+        const float neg_m = -m_new;
+        float rs = 0.f;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t pk[2][16];
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * hh + cc;
+#pragma unroll
+            for (int kk = 0; kk < 32; kk += 2) {
+              float x0, x1, p0, p1;
+              ffma2(__uint_as_float(v[c][kk]), __uint_as_float(v[c][kk + 1]), sl2, neg_m, x0, x1);
+              if (((kk >> 1) & 7) >= 5) {
+                exp2_poly2(x0, x1, p0, p1);
+                if (valid < TK) {   // masked keys (x = -inf) must give exactly zero
+                  p0 = x0 == -INFINITY ? 0.f : p0;
+                  p1 = x1 == -INFINITY ? 0.f : p1;
+                }
+              } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+              }
+              if (!C::SUM_MMA) rs += p0 + p1;
+              pk[cc][kk >> 1] = pack_bf16x2(p0, p1);
+            }
+          }
+          // this half of P may be overwritten once the previous block's P V of it has completed
+          if (i > 0 && !need_o) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&o_full[2 * g + hh], (i - 1) & 1, P.status, abort_flag))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          tmem_st_32x32b_x16(paddr + (2 * hh) * 16, pk[0]);
+          tmem_st_32x32b_x16(paddr + (2 * hh + 1) * 16, pk[1]);
+          if (hh == 0) {
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&p_full[2 * g]);
+          }
         }
+        if (!ok) break;
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[2 * g + 1]);
+        if (!C::SUM_MMA) l_reg = j == 0 ? rs : fmaf(l_reg, corr, rs);
+        m_cur = m_new;
       }
       if (!ok) break;
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_full[2 * g + 1]);
-      if (!C::SUM_MMA) l_reg = j == 0 ? rs : fmaf(l_reg, corr, rs);
-      m_cur = m_new;
+      ++k;
     }
-    if (ok && Tg > 0 && __all_sync(0xffffffffu, mbar_wait(&o_full[2 * g], (Tg - 1) & 1, P.status, abort_flag) &&
-                                               mbar_wait(&o_full[2 * g + 1], (Tg - 1) & 1, P.status, abort_flag))) {
+    if (ok && i > 0 && __all_sync(0xffffffffu, mbar_wait(&o_full[2 * g], (i - 1) & 1, P.status, abort_flag) &&
+                                              mbar_wait(&o_full[2 * g + 1], (i - 1) & 1, P.status, abort_flag))) {
       tc_fence_after();
-      emit_row(Tg / (RAGGED ? geom[0] : P.nkb) - 1);
+      emit_row(k - 1);
     }
   }
 
@@ -539,7 +741,7 @@ template <int DH, bool SPLIT>
 size_t at_smem_bytes(int nkb) {
   constexpr int G = AtCfg<DH>::GROUPS;
   return 1024 + (size_t)2 * nkb * TK * DH * 2 + (size_t)G * (SPLIT ? 2 : 1) * TQ * DH * 2 + 2048 +
-         (AT_MAX_KB + 9 * G + 1) * 8 + 32;
+         G * AT_DESC * sizeof(AtTile) + (size_t)(AT_MAX_KB * (2 + G) + G * (9 + AT_DESC)) * 8 + 16;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -584,7 +786,11 @@ rocs_status at_launch(rocs_context* ctx, AttnTcParams& P, int B_R, int H, cudaSt
     }
     attr[ctx->device] = true;
   }
-  attn_tc_kernel<DH, SPLIT, RAGGED><<<(unsigned)((long long)B_R * H), AtCfg<DH>::THREADS, smem, s>>>(P);
+  // persistent: one CTA per SM (shared memory allows no second), each over its share of the
+  // (request, head) items
+  const long long items = (long long)B_R * H;
+  const unsigned grid = (unsigned)(items < ctx->num_sms ? items : ctx->num_sms);
+  attn_tc_kernel<DH, SPLIT, RAGGED><<<grid, AtCfg<DH>::THREADS, smem, s>>>(P);
   return cuda_check(cudaGetLastError(), "attn_tc_kernel");
 }
 
@@ -597,6 +803,7 @@ rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq,
                                 const int32_t* kv_len, int q_by_kv, const int32_t* order) {
   if (B_R == 0 || rows == 0) return ROCS_OK;
   if ((d_h != 32 && d_h != 64) || L < 1 || (long long)L * d_h > 32768 || (L + TK - 1) / TK > AT_MAX_KB ||
+      (long long)B_R * H > 2147483647LL ||
       ((uintptr_t)Q & 15) || ((uintptr_t)K & 15) || ((uintptr_t)V & 15) || ldq % 8 || ldkv % 8 ||
       (q_split && (ldq < 2LL * H * d_h)) || ldkv < (long long)H * d_h || ((uintptr_t)O & 15) ||
       (O2 && ((uintptr_t)O2 & 15)) || ldo % 8 || (O2 && ldo2 % 8)) {
