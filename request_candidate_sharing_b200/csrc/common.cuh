@@ -78,6 +78,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
   }
 }
 
+// The same bounded wait for roles that are not on the critical path (producers a long way ahead
+// of their consumers): between polls the thread sleeps about `ns` nanoseconds, which leaves the
+// issue slots of its sub-partition to the warps that compute.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, int* status,
+                                                volatile int* abort_flag, unsigned ns) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    __nanosleep(ns);
+    if (mbar_try_wait(a, parity)) return true;
+    if (abort_flag && *abort_flag) return false;
+    if (clock64() - t0 > kWaitBudgetCycles) {
+      set_status(status, ROCS_ERR_DEVICE_TIMEOUT);
+      if (abort_flag) *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
 // ------------------------------------------------------------------------------------------
 // TMA (bulk tensor copies, no multicast)
 // ------------------------------------------------------------------------------------------

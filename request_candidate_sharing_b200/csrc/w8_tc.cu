@@ -105,19 +105,7 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
 // thread that issues the MMAs.
 __device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, int* status,
                                                   volatile int* abort_flag) {
-  const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait(a, parity)) return true;
-  const long long t0 = clock64();
-  while (true) {
-    __nanosleep(64);
-    if (mbar_try_wait(a, parity)) return true;
-    if (abort_flag && *abort_flag) return false;
-    if (clock64() - t0 > kWaitBudgetCycles) {
-      set_status(status, ROCS_ERR_DEVICE_TIMEOUT);
-      if (abort_flag) *abort_flag = 1;
-      return false;
-    }
-  }
+  return mbar_wait_sleep(bar, parity, status, abort_flag, 64);
 }
 
 // A ring position: slot and the phase parity of its current use.
