@@ -150,6 +150,20 @@ struct AtCfg {
 };
 
 constexpr int AT_DESC = 4;   // tile descriptors in flight per softmax warpgroup
+constexpr unsigned kKvPollSleepNs = 32;   // the K/V producer's pause between polls that found nothing to do
+
+// Non-blocking check whether the phase with the given parity has completed.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 
 // One query tile of a softmax warpgroup, published by the query producer.  The MMA issuer and
 // the softmax warpgroup of that group read it; the softmax reads it again when it writes the
@@ -161,12 +175,9 @@ struct AtTile {
   int h;             // head
   int Lr;            // keys of the request
   int nkb;           // key blocks of the request
-  uint32_t kv_par;   // bit j: phase parity of kv_full[j] for this request's load
-  uint32_t flags;    // AT_LAST | AT_TAIL | AT_TAIL_PAR
+  uint32_t flags;    // AT_LAST
 };
-constexpr uint32_t AT_LAST = 1;       // the group's last tile of this request
-constexpr uint32_t AT_TAIL = 2;       // the last key block has padding rows (zeroed before P V)
-constexpr uint32_t AT_TAIL_PAR = 4;   // phase parity of vtail[nkb - 1] for this request
+constexpr uint32_t AT_LAST = 1;   // the group's last tile of this request
 
 // Work item n of the list (request rb in processing order, head h), its query rows and keys.
 struct AtItem {
@@ -240,10 +251,10 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
   uint8_t* sOnes = sQ + GROUPS * NQ * Q_TILE;         // 1024-B aligned (Q tiles are 8 KiB multiples)
   AtTile* descs = reinterpret_cast<AtTile*>(sOnes + ONES_BYTES);   // [GROUPS][AT_DESC]
   uint64_t* bars = reinterpret_cast<uint64_t*>(descs + GROUPS * AT_DESC);
-  uint64_t* kv_full = bars;                           // [AT_MAX_KB]: block j of the current request landed
-  uint64_t* kv_empty = kv_full + AT_MAX_KB;           // [AT_MAX_KB][GROUPS]: group g done with block j
-  uint64_t* vtail = kv_empty + AT_MAX_KB * GROUPS;    // [AT_MAX_KB]: block j's padding rows zeroed
-  uint64_t* q_full = vtail + AT_MAX_KB;               // [GROUPS] each
+  uint64_t* kv_full = bars;                           // [AT_MAX_KB]: block j's copy landed (K/V producer only)
+  uint64_t* kv_ready = kv_full + AT_MAX_KB;           // [AT_MAX_KB][GROUPS]: block j ready for group g
+  uint64_t* kv_empty = kv_ready + AT_MAX_KB * GROUPS; // [AT_MAX_KB][GROUPS]: group g done with block j
+  uint64_t* q_full = kv_empty + AT_MAX_KB * GROUPS;   // [GROUPS] each
   uint64_t* q_free = q_full + GROUPS;
   uint64_t* s_full = q_free + GROUPS;
   uint64_t* s_free = s_full + GROUPS;
@@ -258,8 +269,10 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
   if (threadIdx.x == 0) {
     for (int i = 0; i < AT_MAX_KB; ++i) {
       mbar_init(&kv_full[i], 1);
-      mbar_init(&vtail[i], 1);
-      for (int g = 0; g < GROUPS; ++g) mbar_init(&kv_empty[i * GROUPS + g], 1);
+      for (int g = 0; g < GROUPS; ++g) {
+        mbar_init(&kv_ready[i * GROUPS + g], 1);
+        mbar_init(&kv_empty[i * GROUPS + g], 1);
+      }
     }
     for (int g = 0; g < GROUPS; ++g) {
       mbar_init(&q_full[g], 1);
@@ -294,72 +307,126 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
     if (warp == 0) {
       // ---------------- K/V producer (the whole warp; lane 0 issues the copies) ----------------
       // Block j of the next request is loaded as soon as every group that read block j of the
-      // previous one has finished with it (kv_empty), so a group that runs out of tiles of one
-      // request starts the next request one block behind the other group instead of waiting
-      // for it.  Keys past Lr have P = 0, but their V rows still enter the P V product, where
-      // non-finite padding would give 0 * inf = NaN: once the last block has landed, the warp
-      // zeroes those rows (whole rows: the swizzle permutes 16-byte units within a row) and
-      // releases the block for P V (vtail).
+      // previous one has handed it back (kv_empty), so a group that runs out of tiles of one
+      // request starts the next one a block behind the other group instead of waiting for it.
+      // The warp observes every copy it issued, in order, and only then passes the block on to
+      // the groups that read it (kv_ready, one barrier per block and group): a group that
+      // skips a request (one-tile requests alternate between the groups) would otherwise wait on
+      // a copy barrier that may be two phases from the one it saw last, where parity alone is
+      // ambiguous.  Keys past Lr have P = 0, but their V rows still enter the P V product, where
+      // non-finite padding would give 0 * inf = NaN: the last block's padding rows are zeroed
+      // (whole rows: the swizzle permutes 16-byte units within a row) before it is passed on.
+      // The warp polls instead of blocking, so a copy waiting for its hand-back never holds up
+      // the forwarding of one that has landed.
       if (lane == 0) {
         prefetch_tensormap(&P.tmK);
         prefetch_tensormap(&P.tmV);
       }
-      uint32_t kv_par = 0;     // bit j: parity of block j's next load
-      uint32_t last_par = 0;   // bit j: parity of block j's last load
-      uint32_t loaded = 0;     // bit j: block j has been loaded
-      uint32_t pend = 0;       // bit GROUPS j + g: group g reads block j's last load
-      uint32_t e_par = 0;      // bit GROUPS j + g: parity of kv_empty[j][g]'s next completion
-      int tcount = 0;          // query tiles of the items so far (tile t goes to group t % 2)
+      uint32_t kv_par = 0;   // bit j: parity of kv_full[j] for block j's oldest copy not yet passed on
+      uint32_t pend = 0;     // bit GROUPS j + g: group g reads block j's last copy and has not handed it back
+      uint32_t e_par = 0;    // bit GROUPS j + g: parity of kv_empty[j][g]'s next completion
+      // copies issued and not yet passed on, oldest first, 16 bits each: block (3 bits), groups
+      // (2 bits), padding rows of the block (7 bits); a block is in the queue at most once
+      uint64_t fq_lo = 0, fq_hi = 0;
+      int fn = 0;
+      AtItem it;
+      int pass = 0, jn = 0, tcount = 0;
+      bool have = false, more = true;   // an item with blocks left to issue; items left in the list
+      uint32_t used = 0;                // the groups that read the current item
+      long long t_idle = clock64();
       bool ok = true;
-      for (int pass = 0; ok && pass * (long long)gridDim.x < n_items; ++pass) {
-        const int idx = at_item_index(pass, n_items);
-        if (idx < 0) continue;
-        AtItem it;
-        int bad;
-        at_item<RAGGED>(P, idx, it, bad);
-        if (it.ntiles == 0) continue;
-        const uint32_t used = it.ntiles >= 2 ? 3u : (1u << (tcount & 1));
-        const int kv_row0 = it.r * P.L;
-        for (int j = 0; j < it.nkb && ok; ++j) {
+      while (ok) {
+        bool progress = false;
+        while (!have && more) {
+          if ((long long)pass * gridDim.x >= n_items) {
+            more = false;
+            break;
+          }
+          const int idx = at_item_index(pass++, n_items);
+          if (idx < 0) continue;
+          int bad;
+          at_item<RAGGED>(P, idx, it, bad);
+          if (it.ntiles == 0) continue;
+          used = it.ntiles >= 2 ? 3u : (1u << (tcount & 1));
+          tcount += it.ntiles;
+          jn = 0;
+          have = true;
+        }
+        if (have && fn < AT_MAX_KB) {
+          const int j = jn;
+          bool free_blk = true;
 #pragma unroll
           for (int g = 0; g < GROUPS; ++g) {
             const int b = GROUPS * j + g;
-            if (ok && ((pend >> b) & 1u)) {
-              ok = __all_sync(0xffffffffu, mbar_wait(&kv_empty[b], (e_par >> b) & 1u, P.status, abort_flag));
-              e_par ^= 1u << b;
+            if ((pend >> b) & 1u) free_blk = free_blk && mbar_test(&kv_empty[b], (e_par >> b) & 1u);
+          }
+          free_blk = __shfl_sync(0xffffffffu, free_blk, 0);
+          if (free_blk) {
+            e_par ^= pend & (3u << (GROUPS * j));
+            if (lane == 0) {
+              const int kv_row = it.r * P.L + j * TK;
+              mbar_arrive_expect_tx(&kv_full[j], 2 * KV_BLOCK);
+              tma_load_2d(sK + j * KV_BLOCK, &P.tmK, &kv_full[j], it.h * DH, kv_row);
+              tma_load_2d(sV + j * KV_BLOCK, &P.tmV, &kv_full[j], it.h * DH, kv_row);
             }
+            pend = (pend & ~(3u << (GROUPS * j))) | (used << (GROUPS * j));
+            const uint32_t pad = j == it.nkb - 1 ? (uint32_t)(it.nkb * TK - it.Lr) : 0u;
+            const uint64_t e = (uint64_t)(j | (used << 3) | (pad << 5));
+            if (fn < 4) fq_lo |= e << (16 * fn);
+            else fq_hi |= e << (16 * (fn - 4));
+            ++fn;
+            if (++jn == it.nkb) have = false;
+            progress = true;
           }
-          if (!ok) break;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&kv_full[j], 2 * KV_BLOCK);
-            tma_load_2d(sK + j * KV_BLOCK, &P.tmK, &kv_full[j], it.h * DH, kv_row0 + j * TK);
-            tma_load_2d(sV + j * KV_BLOCK, &P.tmV, &kv_full[j], it.h * DH, kv_row0 + j * TK);
-          }
-          loaded |= 1u << j;
-          last_par = (last_par & ~(1u << j)) | (kv_par & (1u << j));
-          pend = (pend & ~(3u << (GROUPS * j))) | (used << (GROUPS * j));
         }
-        if (!ok) break;
-        const int tail_keys = it.nkb * TK - it.Lr;   // padding rows in the last staged key block
-        if (tail_keys > 0) {
-          const int jb = it.nkb - 1;
-          if (!__all_sync(0xffffffffu, mbar_wait(&kv_full[jb], (kv_par >> jb) & 1u, P.status, abort_flag))) {
-            ok = false;
-            break;
+        if (fn > 0) {
+          const uint32_t e = (uint32_t)(fq_lo & 0xFFFFu);
+          const int j = (int)(e & 7u);
+          const bool landed = __shfl_sync(0xffffffffu, mbar_test(&kv_full[j], (kv_par >> j) & 1u), 0);
+          if (landed) {
+            const int pad = (int)((e >> 5) & 127u);
+            if (pad > 0) {
+              uint8_t* vb = sV + j * KV_BLOCK + (TK - pad) * ROWB;
+              for (int i = lane; i < pad * ROWB / 16; i += 32) reinterpret_cast<uint4*>(vb)[i] = make_uint4(0, 0, 0, 0);
+              asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
+              __syncwarp();
+            }
+            if (lane == 0) {
+#pragma unroll
+              for (int g = 0; g < GROUPS; ++g)
+                if ((e >> (3 + g)) & 1u) mbar_arrive(&kv_ready[GROUPS * j + g]);
+            }
+            kv_par ^= 1u << j;
+            fq_lo = (fq_lo >> 16) | (fq_hi << 48);
+            fq_hi >>= 16;
+            --fn;
+            progress = true;
           }
-          uint8_t* vb = sV + jb * KV_BLOCK + (TK - tail_keys) * ROWB;
-          for (int i = lane; i < tail_keys * ROWB / 16; i += 32) reinterpret_cast<uint4*>(vb)[i] = make_uint4(0, 0, 0, 0);
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&vtail[jb]);
         }
-        kv_par ^= (1u << it.nkb) - 1u;
-        tcount += it.ntiles;
+        if (!have && !more && fn == 0) break;
+        if (progress) {
+          t_idle = clock64();
+        } else if (*abort_flag) {
+          ok = false;
+        } else if (clock64() - t_idle > kWaitBudgetCycles) {
+          if (lane == 0) set_status(P.status, ROCS_ERR_DEVICE_TIMEOUT);
+          *abort_flag = 1;
+          ok = false;
+        } else if (kKvPollSleepNs != 0) {
+          __nanosleep(kKvPollSleepNs);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
       }
-      // no copy of this CTA may still be landing when it exits
-      if (lane == 0)
-        for (int j = 0; j < AT_MAX_KB; ++j)
-          if ((loaded >> j) & 1u) mbar_wait(&kv_full[j], (last_par >> j) & 1u, P.status, nullptr);
+      // no copy of this CTA may still be landing when it exits (after an abort, the queue holds
+      // the copies issued and not passed on)
+      while (fn > 0) {
+        const int j = (int)(fq_lo & 7u);
+        if (lane == 0) mbar_wait(&kv_full[j], (kv_par >> j) & 1u, P.status, nullptr);
+        kv_par ^= 1u << j;
+        fq_lo = (fq_lo >> 16) | (fq_hi << 48);
+        fq_hi >>= 16;
+        --fn;
+      }
     } else if (warp == 3 && lane == 0) {
       // ---------------- query producer: tile descriptors and query tiles ----------------
       // The query tiles of the CTA's requests alternate between the two groups; each group has
@@ -367,7 +434,6 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
       // group's query buffer has been released three tiles later, by which time the softmax
       // has written that tile's output (it does so while it works on the following tile).
       prefetch_tensormap(&P.tmQ);
-      uint32_t kv_par = 0, vt_par = 0;
       int tcount = 0, kq0 = 0, kq1 = 0;
       bool ok = true;
       for (int pass = 0; ok && pass * (long long)gridDim.x < n_items; ++pass) {
@@ -378,14 +444,6 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
         at_item<RAGGED>(P, idx, it, bad);
         if (bad != 0) set_status(P.status, bad);
         if (it.ntiles == 0) continue;
-        const uint32_t item_par = kv_par;
-        kv_par ^= (1u << it.nkb) - 1u;
-        uint32_t tail_flags = 0;
-        if (it.nkb * TK > it.Lr) {
-          const int jb = it.nkb - 1;
-          tail_flags = AT_TAIL | (((vt_par >> jb) & 1u) ? AT_TAIL_PAR : 0u);
-          vt_par ^= 1u << jb;
-        }
         for (int t = 0; t < it.ntiles; ++t) {
           const int g = tcount & 1;
           const int k = g ? kq1 : kq0;
@@ -401,8 +459,7 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
           d.h = it.h;
           d.Lr = it.Lr;
           d.nkb = it.nkb;
-          d.kv_par = item_par;
-          d.flags = tail_flags | (t + GROUPS >= it.ntiles ? AT_LAST : 0u);
+          d.flags = t + GROUPS >= it.ntiles ? AT_LAST : 0u;
           mbar_arrive(&d_full[slot]);
           mbar_arrive_expect_tx(&q_full[g], NQ * Q_TILE);
           const int qrow = (int)(it.q0 + (long long)t * TQ);
@@ -439,9 +496,6 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
       const int g = warp - 1;
       auto issue_pv = [&](int ib, int hh, int j, uint32_t fl, int nkb) -> bool {
         if (!mbar_wait(&p_full[2 * g + hh], ib & 1, P.status, abort_flag)) return false;
-        if (hh == 0 && j == nkb - 1 && (fl & AT_TAIL) &&
-            !mbar_wait(&vtail[j], (fl & AT_TAIL_PAR) ? 1u : 0u, P.status, abort_flag))
-          return false;
         tc_fence_after();
         const uint32_t va = smem_u32(sV + j * KV_BLOCK);
 #pragma unroll
@@ -458,11 +512,31 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
         if (hh == 1 && (fl & AT_LAST)) tc_commit(&kv_empty[GROUPS * j + g]);
         return true;
       };
+      // S_i = Q K_j^T into the group's S buffer, once the softmax has read S_{i-1}
+      auto issue_s = [&](int ib, int j, uint32_t qa, int nkb) -> bool {
+        if (ib > 0 && !mbar_wait(&s_free[g], (ib - 1) & 1, P.status, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t ka = smem_u32(sK + j * KV_BLOCK);
+#pragma unroll
+        for (int ks = 0; ks < DH / 16; ++ks) {
+          tc_mma_ss(tmem_base + C::S_COL + g * TK, sdesc(qa + ks * 32, SBO, SW), sdesc(ka + ks * 32, SBO, SW),
+                    IDESC_S, ks > 0 ? 1u : 0u);
+          if (SPLIT)
+            tc_mma_ss(tmem_base + C::S_COL + g * TK, sdesc(qa + Q_TILE + ks * 32, SBO, SW),
+                      sdesc(ka + ks * 32, SBO, SW), IDESC_S, 1u);
+        }
+        tc_commit(&s_full[g]);
+        if (j == nkb - 1) tc_commit(&q_free[g]);   // this tile's queries are no longer read
+        return true;
+      };
+      const uint32_t qa = smem_u32(sQ + (g * NQ) * Q_TILE);
       bool ok = true;
       int k = 0, i = 0;
       bool pend_pv = false;   // block i - 1's P V is not issued yet
       int pj = 0, pnkb = 0;   // that block's index and its request's block count
       uint32_t pfl = 0;       // and its tile's flags
+      bool s0_done = false;   // tile k's first S was issued at the end of tile k - 1
+      uint32_t rpar = 0;      // bit j: parity of kv_ready[j][g] for the next request this group reads
       for (;;) {
         const int slot = g * AT_DESC + (k % AT_DESC);
         if (!mbar_wait(&d_full[slot], (k / AT_DESC) & 1, P.status, abort_flag)) {
@@ -472,31 +546,14 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
         const int tile = descs[slot].tile;
         if (tile < 0) break;
         const int nkb = descs[slot].nkb;
-        const uint32_t kvp = descs[slot].kv_par, fl = descs[slot].flags;
+        const uint32_t fl = descs[slot].flags;
         if (!mbar_wait(&q_full[g], k & 1, P.status, abort_flag)) {
           ok = false;
           break;
         }
-        const uint32_t qa = smem_u32(sQ + (g * NQ) * Q_TILE);
-        for (int j = 0; j < nkb; ++j, ++i) {
-          if (!mbar_wait(&kv_full[j], (kvp >> j) & 1u, P.status, abort_flag) ||
-              (i > 0 && !mbar_wait(&s_free[g], (i - 1) & 1, P.status, abort_flag))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t ka = smem_u32(sK + j * KV_BLOCK);
-#pragma unroll
-          for (int ks = 0; ks < DH / 16; ++ks) {
-            tc_mma_ss(tmem_base + C::S_COL + g * TK, sdesc(qa + ks * 32, SBO, SW), sdesc(ka + ks * 32, SBO, SW),
-                      IDESC_S, ks > 0 ? 1u : 0u);
-            if (SPLIT)
-              tc_mma_ss(tmem_base + C::S_COL + g * TK, sdesc(qa + Q_TILE + ks * 32, SBO, SW),
-                        sdesc(ka + ks * 32, SBO, SW), IDESC_S, 1u);
-          }
-          tc_commit(&s_full[g]);
-          if (j == nkb - 1) tc_commit(&q_free[g]);   // this tile's queries are no longer read
-          if (pend_pv && !(issue_pv(i - 1, 0, pj, pfl, pnkb) && issue_pv(i - 1, 1, pj, pfl, pnkb))) {
+        for (int j = s0_done ? 1 : 0; j < nkb; ++j) {
+          if (!mbar_wait(&kv_ready[GROUPS * j + g], (rpar >> j) & 1u, P.status, abort_flag) || !issue_s(i, j, qa, nkb) ||
+              (pend_pv && !(issue_pv(i - 1, 0, pj, pfl, pnkb) && issue_pv(i - 1, 1, pj, pfl, pnkb)))) {
             ok = false;
             break;
           }
@@ -504,17 +561,39 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
           pfl = fl;
           pnkb = nkb;
           pend_pv = true;
+          ++i;
         }
         if (!ok) break;
+        s0_done = false;
         // The group's last tile of a request: its last P V (and the hand-back of the last block)
-        // is issued now, not after the next tile's first S, which may need the next request's
-        // K/V, whose load waits for this hand-back.
+        // is issued now, not after a first S that would wait for the next request's K/V, whose
+        // load waits for this hand-back.  If the next tile can start at once (descriptor,
+        // queries and first key block already there, checked without waiting), its first S still
+        // goes first, so the softmax finds it ready.
         if (fl & AT_LAST) {
+          rpar ^= (1u << nkb) - 1u;   // the group is done with this request's blocks
+          const int ns = g * AT_DESC + ((k + 1) % AT_DESC);
+          if (mbar_test(&d_full[ns], ((k + 1) / AT_DESC) & 1) && descs[ns].tile >= 0 &&
+              mbar_test(&q_full[g], (k + 1) & 1) && mbar_test(&kv_ready[g], rpar & 1u)) {
+            const int nkb1 = descs[ns].nkb;
+            if (!issue_s(i, 0, qa, nkb1)) {
+              ok = false;
+              break;
+            }
+            s0_done = true;
+          }
           if (!(issue_pv(i - 1, 0, pj, pfl, pnkb) && issue_pv(i - 1, 1, pj, pfl, pnkb))) {
             ok = false;
             break;
           }
           pend_pv = false;
+          if (s0_done) {
+            pj = 0;
+            pfl = descs[ns].flags;
+            pnkb = descs[ns].nkb;
+            pend_pv = true;
+            ++i;
+          }
         }
         ++k;
       }
@@ -741,7 +820,7 @@ template <int DH, bool SPLIT>
 size_t at_smem_bytes(int nkb) {
   constexpr int G = AtCfg<DH>::GROUPS;
   return 1024 + (size_t)2 * nkb * TK * DH * 2 + (size_t)G * (SPLIT ? 2 : 1) * TQ * DH * 2 + 2048 +
-         G * AT_DESC * sizeof(AtTile) + (size_t)(AT_MAX_KB * (2 + G) + G * (9 + AT_DESC)) * 8 + 16;
+         G * AT_DESC * sizeof(AtTile) + (size_t)(AT_MAX_KB * (1 + 2 * G) + G * (9 + AT_DESC)) * 8 + 16;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
