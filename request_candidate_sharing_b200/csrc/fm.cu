@@ -500,6 +500,35 @@ __global__ void lcb_req_kernel(const TIN* __restrict__ E_R, long long ld_ER, int
   }
 }
 
+// The same with the request's rows and the weights staged in shared memory first (as floats),
+// so the token loop reads shared memory instead of re-reading global memory for every output
+// row.  Same accumulation order, so the same bits.
+template <typename TIN>
+__global__ void lcb_req_staged_kernel(const TIN* __restrict__ E_R, long long ld_ER, int n_R, int D,
+                                      const __nv_bfloat16* __restrict__ P_RR, const __nv_bfloat16* __restrict__ P_CR,
+                                      int o_R, int o_C, void* L_R, long long ld_LR, int out_mode, long long lo_off,
+                                      float* __restrict__ ZL) {
+  extern __shared__ float lcb_sm[];
+  float* sE = lcb_sm;              // [n_R][D]
+  float* sP = sE + n_R * D;        // [o_R + o_C][n_R]
+  const int r = blockIdx.x;
+  const TIN* e = E_R + (long long)r * ld_ER;
+  for (int i = threadIdx.x; i < n_R * D; i += blockDim.x) sE[i] = ld_f(e + i);
+  for (int i = threadIdx.x; i < (o_R + o_C) * n_R; i += blockDim.x) {
+    const int o = i / n_R, t = i - o * n_R;
+    sP[i] = __bfloat162float(o < o_R ? P_RR[(long long)o * n_R + t] : P_CR[(long long)(o - o_R) * n_R + t]);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < (o_R + o_C) * D; i += blockDim.x) {
+    const int o = i / D, d = i - o * D;
+    const float* p = sP + o * n_R;
+    float acc = 0.f;
+    for (int t = 0; t < n_R; ++t) acc = fmaf(p[t], sE[t * D + d], acc);
+    if (o < o_R) store_val(L_R, (long long)r * ld_LR + (long long)o * D + d, acc, out_mode, lo_off);
+    else ZL[((long long)r * o_C + (o - o_R)) * D + d] = acc;
+  }
+}
+
 // Candidate side: one warp per candidate; lane owns features d = lane + 32 j (j < DPL).
 constexpr int LCB_OMAX = 8;
 
@@ -605,8 +634,14 @@ rocs_status lcb_launch(rocs_context* ctx, const TIN* E_R, long long ld_ER, const
                        long long ld_LC, int out_mode, long long lo_R, long long lo_C, float* ws_Z, cudaStream_t s) {
   if (B_R > 0 && (o_R + o_C) > 0) {
     LaunchTimer lt_("lcb_req", s);
-    lcb_req_kernel<TIN><<<B_R, 256, 0, s>>>(E_R, ld_ER, n_R, D, (const __nv_bfloat16*)P_RR,
-                                            (const __nv_bfloat16*)P_CR, o_R, o_C, L_R, ld_LR, out_mode, lo_R, ws_Z);
+    const size_t sm_bytes = ((size_t)n_R * D + (size_t)(o_R + o_C) * n_R) * sizeof(float);
+    if (sm_bytes <= 48 * 1024)
+      lcb_req_staged_kernel<TIN><<<B_R, 256, sm_bytes, s>>>(E_R, ld_ER, n_R, D, (const __nv_bfloat16*)P_RR,
+                                                             (const __nv_bfloat16*)P_CR, o_R, o_C, L_R, ld_LR,
+                                                             out_mode, lo_R, ws_Z);
+    else
+      lcb_req_kernel<TIN><<<B_R, 256, 0, s>>>(E_R, ld_ER, n_R, D, (const __nv_bfloat16*)P_RR,
+                                              (const __nv_bfloat16*)P_CR, o_R, o_C, L_R, ld_LR, out_mode, lo_R, ws_Z);
     rocs_status st = cuda_check(cudaGetLastError(), "lcb_req_kernel");
     if (st != ROCS_OK) return st;
   }
