@@ -6,30 +6,31 @@
 // K/V directly, never a per-candidate copy.
 //
 // Persistent: one CTA per SM, each over its share of the (request, head) items, dealt out in
-// alternating directions.  Three warpgroups (384 threads):
-//   warp 0      TMA: the item's K and V (L x d_h bf16) into shared memory ONCE, in 128-key blocks.
-//               Block j of the next item is loaded as soon as the groups that read block j of the
-//               current one are done with it, so items follow each other without a pipeline
-//               drain, and the CTA's startup (TMEM, barriers, first loads) is paid once per SM
-//               instead of once per item.  The warp observes each copy land and passes the block
-//               on to the groups that read it, through one barrier per block and group.
-//   warp 3      the query tiles (bf16, or a hi/lo pair) of all the CTA's items, alternating between
-//               the two softmax warpgroups (an odd tile count of one item no longer leaves a group
-//               idle), each with a small descriptor (rows, head, keys) in shared memory.
-//   warps 1, 2  one MMA issuer per group; one thread issues, for each 128-key block j,
-//                 S_j = Q K_j^T       (tcgen05.mma M=128, N=128, K=d_h; one S buffer per group)
-//                 O  += P_j V_j       (M=128, N=d_h, K=128; V read as an MN-major operand; O
+// alternating directions.  G query-tile groups (2 or 3) of one softmax warpgroup each, blocks of
+// TK keys (128 or 64), one control warpgroup; 128 (G + 1) threads:
+//   warp 0      producer, one polling loop over three jobs: the item's K and V (L x d_h bf16)
+//               into shared memory ONCE, in blocks of TK keys, block j of the next item loaded
+//               as soon as the groups that read block j of the current one are done with it (so
+//               items follow each other without a pipeline drain, and the CTA's startup is paid
+//               once per SM); passing each block on to the groups that read it once it has
+//               landed (one barrier per block and group); and the query tiles (bf16, or a hi/lo
+//               pair) of the CTA's items, which go to the groups in turn, each with a small
+//               descriptor (rows, head, keys) in shared memory.
+//   warps 1..G  one MMA issuer per group; one thread issues, for each key block j,
+//                 S_j = Q K_j^T       (tcgen05.mma M=128, N=TK, K=d_h; one S buffer per group)
+//                 O  += P_j V_j       (M=128, N=d_h, K=TK; V read as an MN-major operand; O
 //                                      accumulates in TMEM across the key blocks)
 //               issuing the next S block before it waits on the current P, so the group's
-//               exponentials overlap the other group's tensor-core work.
-//   warps 4..11 two softmax warpgroups, one thread per query row (TMEM lane): the S row is read
+//               exponentials overlap the other groups' tensor-core work.
+//   warps 4..   the softmax warpgroups, one thread per query row (TMEM lane): the S row is read
 //               from TMEM in one batch, its maximum and exp2 taken in registers (no shuffles; part
 //               of the exponentials on the FMA pipe as a polynomial), P_j written back to TMEM as
 //               bf16 pairs (tcgen05.st), where it is the A operand of P_j V_j; the row sum is an MMA
 //               of the same P_j against a ones tile.  The row's reference maximum moves only when a
 //               block exceeds it by more than 2^8 (then the warp rescales its O and l rows in
 //               TMEM); at the end O is read once and divided by the row sum.
-//   setmaxnreg moves registers from the control warpgroup (72) to the softmax warpgroups (216).
+//   setmaxnreg moves registers from the control warpgroup (72) to the softmax warpgroups (216 for
+//   two groups, 144 for three).
 // All waits are bounded; a wait that runs out sets ROCS_ERR_DEVICE_TIMEOUT and the CTA unwinds
 // (in-flight copies and MMAs drained, TMEM released) instead of spinning.
 #include "common.cuh"
@@ -39,10 +40,17 @@
 namespace rocs {
 namespace {
 
-constexpr int TQ = 128;    // query rows per tile (MMA M)
-constexpr int TK = 128;    // keys per block
+constexpr int TQ = 128;         // query rows per tile (MMA M)
 constexpr int AT_TMEM_COLS = 512;
-constexpr int AT_MAX_KB = 8;   // L <= 1024
+constexpr int AT_MAX_L = 1024;  // keys staged in shared memory at most
+constexpr int AT_FIFO = 8;      // K/V copies issued and not yet passed on, at most
+// (query-tile groups, keys per block).  Three groups of 64-key blocks give each sub-partition a
+// third softmax warp and were 4.5% faster on the encoder (one bf16 query per row); with hi/lo
+// queries (twice the S MMAs per block, and twice the blocks) they were 1% slower, so those keep
+// two groups of 128-key blocks, as does d_h = 64 (whose registers would not fit three groups).
+constexpr int kAtGroups32 = 3, kAtKeys32 = 64;
+constexpr int kAtGroupsSplit = 2, kAtKeysSplit = 128;
+constexpr int kAtGroups64 = 2, kAtKeys64 = 128;
 
 struct AttnTcParams {
   CUtensorMap tmQ;   // queries [rows, cols] bf16: box {d_h, 128}
@@ -135,19 +143,22 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // (log2 units): exponentials stay <= 2^8, and the O accumulator in TMEM is rescaled rarely.
 constexpr float kLazyRescaleLog2 = 8.0f;
 
-template <int DH>
+// G query-tile groups (one softmax warpgroup and one MMA issuer each, one tile in flight each)
+// and TK keys per block.
+template <int DH, int G, int TK>
 struct AtCfg {
-  static constexpr int GROUPS = 2;                   // query tiles in flight
+  static constexpr int GROUPS = G;
+  static constexpr int MAX_KB = AT_MAX_L / TK;       // key blocks at most
   static constexpr bool SUM_MMA = DH == 32;          // row sums by an MMA of P against ones
-  static constexpr int THREADS = 128 + 128 * GROUPS;
-  static constexpr int REG_LAUNCH = 168;
+  static constexpr int THREADS = 128 + 128 * G;
+  static constexpr int REG_LAUNCH = 65536 / THREADS / 8 * 8;
   static constexpr int REG_CTRL = 72;                // producer / MMA warpgroup after setmaxnreg.dec
-  static constexpr int REG_SOFTMAX = 216;
-  static_assert(128 * REG_CTRL + 128 * GROUPS * REG_SOFTMAX <= THREADS * REG_LAUNCH, "register split");
-  // tensor memory: S (128 fp32 columns) | P (64 columns of bf16 pairs) | O (DH) | row sum (16)
-  static constexpr int S_COL = 0, P_COL = GROUPS * 128, O_COL = P_COL + GROUPS * 64,
-                       L_COL = O_COL + GROUPS * DH;
-  static_assert(L_COL + (SUM_MMA ? GROUPS * 16 : 0) <= 512, "tensor memory columns");
+  static constexpr int REG_SOFTMAX = (65536 - 128 * REG_CTRL) / (128 * G) / 8 * 8;
+  static_assert(128 * REG_CTRL + 128 * G * REG_SOFTMAX <= THREADS * REG_LAUNCH, "register split");
+  static_assert(G >= 2 && G <= 3 && TK % 64 == 0 && AT_MAX_L % TK == 0 && MAX_KB <= 16, "tile shape");
+  // tensor memory per group: S (TK fp32 columns) | P (TK / 2 columns of bf16 pairs) | O (DH) | row sum (16)
+  static constexpr int S_COL = 0, P_COL = G * TK, O_COL = P_COL + G * (TK / 2), L_COL = O_COL + G * DH;
+  static_assert(L_COL + (SUM_MMA ? G * 16 : 0) <= AT_TMEM_COLS, "tensor memory columns");
 };
 
 constexpr int AT_DESC = 4;   // tile descriptors in flight per softmax warpgroup
@@ -188,7 +199,7 @@ struct AtItem {
 
 // Geometry of item idx = rb * H + h.  An item whose offsets or key count are invalid gets
 // ntiles = 0 and `bad` the status to report.
-template <bool RAGGED>
+template <int TK, bool RAGGED>
 __device__ __forceinline__ void at_item(const AttnTcParams& P, int idx, AtItem& it, int& bad) {
   const int rb = idx / P.H;
   it.h = idx - rb * P.H;
@@ -227,18 +238,20 @@ __device__ __forceinline__ int at_item_index(int pass, int n_items) {
   return idx < n_items ? (int)idx : -1;
 }
 
-template <int DH, bool SPLIT, bool RAGGED>
-__global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __grid_constant__ AttnTcParams P) {
-  using C = AtCfg<DH>;
-  constexpr int GROUPS = C::GROUPS;
-  static_assert(GROUPS == 2, "query tiles alternate between two softmax warpgroups");
+template <int DH, bool SPLIT, bool RAGGED, int G, int TK>
+__global__ void __launch_bounds__(AtCfg<DH, G, TK>::THREADS, 1) attn_tc_kernel(const __grid_constant__ AttnTcParams P) {
+  using C = AtCfg<DH, G, TK>;
+  constexpr int GROUPS = G;
+  constexpr int MAX_KB = C::MAX_KB;
+  constexpr uint32_t GMASK = (1u << G) - 1u;
   constexpr int ROWB = DH * 2;                        // bytes per K/V/Q row
   constexpr uint32_t SW = DH == 32 ? 4u : 2u;         // 64-B or 128-B swizzle for K/V/Q
   constexpr uint32_t SBO = 8 * ROWB;                  // 8-row group stride
-  constexpr int KV_BLOCK = TK * ROWB;                 // bytes of one 128-key block
+  constexpr int KV_BLOCK = TK * ROWB;                 // bytes of one key block
   constexpr int Q_TILE = TQ * ROWB;
   constexpr int NQ = SPLIT ? 2 : 1;
   constexpr int ONES_BYTES = 2048;                    // 16 rows x 64 bf16 ones (128-byte rows)
+  constexpr int CH = TK / 64;                         // 32-key chunks per half block
   constexpr uint32_t IDESC_S = idesc_bf16(TQ, TK, false);
   constexpr uint32_t IDESC_O = idesc_bf16(TQ, DH, true);
   constexpr uint32_t IDESC_L = idesc_bf16(TQ, 16, false);
@@ -252,10 +265,10 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
   uint8_t* sOnes = sQ + GROUPS * NQ * Q_TILE;         // 1024-B aligned (Q tiles are 8 KiB multiples)
   AtTile* descs = reinterpret_cast<AtTile*>(sOnes + ONES_BYTES);   // [GROUPS][AT_DESC]
   uint64_t* bars = reinterpret_cast<uint64_t*>(descs + GROUPS * AT_DESC);
-  uint64_t* kv_full = bars;                           // [AT_MAX_KB]: block j's copy landed (K/V producer only)
-  uint64_t* kv_ready = kv_full + AT_MAX_KB;           // [AT_MAX_KB][GROUPS]: block j ready for group g
-  uint64_t* kv_empty = kv_ready + AT_MAX_KB * GROUPS; // [AT_MAX_KB][GROUPS]: group g done with block j
-  uint64_t* q_full = kv_empty + AT_MAX_KB * GROUPS;   // [GROUPS] each
+  uint64_t* kv_full = bars;                           // [MAX_KB]: block j's copy landed (producer only)
+  uint64_t* kv_ready = kv_full + MAX_KB;              // [MAX_KB][GROUPS]: block j ready for group g
+  uint64_t* kv_empty = kv_ready + MAX_KB * GROUPS;    // [MAX_KB][GROUPS]: group g done with block j
+  uint64_t* q_full = kv_empty + MAX_KB * GROUPS;      // [GROUPS] each
   uint64_t* q_free = q_full + GROUPS;
   uint64_t* s_full = q_free + GROUPS;
   uint64_t* s_free = s_full + GROUPS;
@@ -268,7 +281,7 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < AT_MAX_KB; ++i) {
+    for (int i = 0; i < MAX_KB; ++i) {
       mbar_init(&kv_full[i], 1);
       for (int g = 0; g < GROUPS; ++g) {
         mbar_init(&kv_ready[i * GROUPS + g], 1);
@@ -306,38 +319,52 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REG_CTRL));
     if (warp == 0) {
-      // ---------------- K/V producer (the whole warp; lane 0 issues the copies) ----------------
-      // Block j of the next request is loaded as soon as every group that read block j of the
-      // previous one has handed it back (kv_empty), so a group that runs out of tiles of one
-      // request starts the next one a block behind the other group instead of waiting for it.
-      // The warp observes every copy it issued, in order, and only then passes the block on to
-      // the groups that read it (kv_ready, one barrier per block and group): a group that
-      // skips a request (one-tile requests alternate between the groups) would otherwise wait on
-      // a copy barrier that may be two phases from the one it saw last, where parity alone is
-      // ambiguous.  Keys past Lr have P = 0, but their V rows still enter the P V product, where
-      // non-finite padding would give 0 * inf = NaN: the last block's padding rows are zeroed
-      // (whole rows: the swizzle permutes 16-byte units within a row) before it is passed on.
-      // The warp polls instead of blocking, so a copy waiting for its hand-back never holds up
-      // the forwarding of one that has landed.
+      // ---------------- producer (the whole warp; lane 0 issues copies and arrivals) ----------------
+      // One polling loop with three jobs, none of which may hold up the others:
+      //  * K/V copies: block j of the next item is loaded as soon as every group that read block
+      //    j of the previous copy has handed it back (kv_empty), so a group that runs out of
+      //    tiles of one item starts the next a block behind the others instead of waiting.
+      //  * passing blocks on: the warp observes every copy it issued, in order (kv_full), and
+      //    only then passes the block to the groups that read the item (kv_ready, one barrier
+      //    per block and group).  A group that skips an item would otherwise wait on a copy
+      //    barrier that may be two phases from the one it saw last, where parity alone is
+      //    ambiguous.  Keys past Lr have P = 0, but their V rows still enter the P V product,
+      //    where non-finite padding would give 0 * inf = NaN: the last block's padding rows are
+      //    zeroed (whole rows: the swizzle permutes 16-byte units within a row) before it is
+      //    passed on.
+      //  * query tiles: the tiles of the CTA's items go to the groups in turn; each gets a small
+      //    descriptor (rows, head, keys) in one of the group's AT_DESC slots and its queries in
+      //    the group's query buffer, once the group has released the previous tile's queries
+      //    (q_free).  A slot is rewritten only after that release three tiles later, by which
+      //    time the softmax has written that tile's output (it does so during the next tile).
       if (lane == 0) {
         prefetch_tensormap(&P.tmK);
         prefetch_tensormap(&P.tmV);
+        prefetch_tensormap(&P.tmQ);
       }
       uint32_t kv_par = 0;   // bit j: parity of kv_full[j] for block j's oldest copy not yet passed on
-      uint32_t pend = 0;     // bit GROUPS j + g: group g reads block j's last copy and has not handed it back
-      uint32_t e_par = 0;    // bit GROUPS j + g: parity of kv_empty[j][g]'s next completion
-      // copies issued and not yet passed on, oldest first, 16 bits each: block (3 bits), groups
-      // (2 bits), padding rows of the block (7 bits); a block is in the queue at most once
+      uint64_t pend = 0;     // bit GROUPS j + g: group g reads block j's last copy and has not handed it back
+      uint64_t e_par = 0;    // bit GROUPS j + g: parity of kv_empty[j][g]'s next completion
+      // copies issued and not yet passed on, oldest first, 16 bits each: block (4 bits), groups
+      // (3 bits), padding rows of the block (7 bits); at most AT_FIFO
       uint64_t fq_lo = 0, fq_hi = 0;
       int fn = 0;
       AtItem it;
       int pass = 0, jn = 0, tcount = 0;
       bool have = false, more = true;   // an item with blocks left to issue; items left in the list
       uint32_t used = 0;                // the groups that read the current item
+      // query side: its own walk over the same items
+      AtItem qi;
+      int qpass = 0, qt = 0, qcount = 0, closed = 0;
+      bool qhave = false, qmore = true;
+      int kq[GROUPS];
+#pragma unroll
+      for (int g = 0; g < GROUPS; ++g) kq[g] = 0;
       long long t_idle = clock64();
       bool ok = true;
       while (ok) {
         bool progress = false;
+        // ---- K/V copies
         while (!have && more) {
           if ((long long)pass * gridDim.x >= n_items) {
             more = false;
@@ -346,33 +373,34 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
           const int idx = at_item_index(pass++, n_items);
           if (idx < 0) continue;
           int bad;
-          at_item<RAGGED>(P, idx, it, bad);
+          at_item<TK, RAGGED>(P, idx, it, bad);
           if (it.ntiles == 0) continue;
-          used = it.ntiles >= 2 ? 3u : (1u << (tcount & 1));
+          used = 0;
+          for (int t = 0; t < it.ntiles && t < GROUPS; ++t) used |= 1u << ((tcount + t) % GROUPS);
           tcount += it.ntiles;
           jn = 0;
           have = true;
         }
-        if (have && fn < AT_MAX_KB) {
+        if (have && fn < AT_FIFO) {
           const int j = jn;
           bool free_blk = true;
 #pragma unroll
           for (int g = 0; g < GROUPS; ++g) {
             const int b = GROUPS * j + g;
-            if ((pend >> b) & 1u) free_blk = free_blk && mbar_test(&kv_empty[b], (e_par >> b) & 1u);
+            if ((pend >> b) & 1u) free_blk = free_blk && mbar_test(&kv_empty[b], (uint32_t)((e_par >> b) & 1u));
           }
           free_blk = __shfl_sync(0xffffffffu, free_blk, 0);
           if (free_blk) {
-            e_par ^= pend & (3u << (GROUPS * j));
+            e_par ^= pend & ((uint64_t)GMASK << (GROUPS * j));
             if (lane == 0) {
               const int kv_row = it.r * P.L + j * TK;
               mbar_arrive_expect_tx(&kv_full[j], 2 * KV_BLOCK);
               tma_load_2d(sK + j * KV_BLOCK, &P.tmK, &kv_full[j], it.h * DH, kv_row);
               tma_load_2d(sV + j * KV_BLOCK, &P.tmV, &kv_full[j], it.h * DH, kv_row);
             }
-            pend = (pend & ~(3u << (GROUPS * j))) | (used << (GROUPS * j));
+            pend = (pend & ~((uint64_t)GMASK << (GROUPS * j))) | ((uint64_t)used << (GROUPS * j));
             const uint32_t pad = j == it.nkb - 1 ? (uint32_t)(it.nkb * TK - it.Lr) : 0u;
-            const uint64_t e = (uint64_t)(j | (used << 3) | (pad << 5));
+            const uint64_t e = (uint64_t)(j | (used << 4) | (pad << 7));
             if (fn < 4) fq_lo |= e << (16 * fn);
             else fq_hi |= e << (16 * (fn - 4));
             ++fn;
@@ -380,12 +408,13 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
             progress = true;
           }
         }
+        // ---- passing landed blocks on
         if (fn > 0) {
           const uint32_t e = (uint32_t)(fq_lo & 0xFFFFu);
-          const int j = (int)(e & 7u);
+          const int j = (int)(e & 15u);
           const bool landed = __shfl_sync(0xffffffffu, mbar_test(&kv_full[j], (kv_par >> j) & 1u), 0);
           if (landed) {
-            const int pad = (int)((e >> 5) & 127u);
+            const int pad = (int)((e >> 7) & 127u);
             if (pad > 0) {
               uint8_t* vb = sV + j * KV_BLOCK + (TK - pad) * ROWB;
               for (int i = lane; i < pad * ROWB / 16; i += 32) reinterpret_cast<uint4*>(vb)[i] = make_uint4(0, 0, 0, 0);
@@ -395,7 +424,7 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
             if (lane == 0) {
 #pragma unroll
               for (int g = 0; g < GROUPS; ++g)
-                if ((e >> (3 + g)) & 1u) mbar_arrive(&kv_ready[GROUPS * j + g]);
+                if ((e >> (4 + g)) & 1u) mbar_arrive(&kv_ready[GROUPS * j + g]);
             }
             kv_par ^= 1u << j;
             fq_lo = (fq_lo >> 16) | (fq_hi << 48);
@@ -404,7 +433,58 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
             progress = true;
           }
         }
-        if (!have && !more && fn == 0) break;
+        // ---- query tiles
+        while (!qhave && qmore) {
+          if ((long long)qpass * gridDim.x >= n_items) {
+            qmore = false;
+            break;
+          }
+          const int idx = at_item_index(qpass++, n_items);
+          if (idx < 0) continue;
+          int bad;
+          at_item<TK, RAGGED>(P, idx, qi, bad);
+          if (bad != 0 && lane == 0) set_status(P.status, bad);
+          if (qi.ntiles == 0) continue;
+          qt = 0;
+          qhave = true;
+        }
+        if (qhave || closed < GROUPS) {
+          const int g = qhave ? qcount % GROUPS : closed;
+          const int k = kq[g];
+          const bool q_ok = __shfl_sync(0xffffffffu, k == 0 || mbar_test(&q_free[g], (k - 1) & 1), 0);
+          if (q_ok) {
+            const int slot = g * AT_DESC + (k % AT_DESC);
+            if (lane == 0) {
+              AtTile& d = descs[slot];
+              if (qhave) {
+                d.q0 = qi.q0;
+                d.q1 = qi.q1;
+                d.tile = qt;
+                d.h = qi.h;
+                d.Lr = qi.Lr;
+                d.nkb = qi.nkb;
+                d.flags = qt + GROUPS >= qi.ntiles ? AT_LAST : 0u;
+                mbar_arrive(&d_full[slot]);
+                mbar_arrive_expect_tx(&q_full[g], NQ * Q_TILE);
+                const int qrow = (int)(qi.q0 + (long long)qt * TQ);
+                tma_load_2d(sQ + (g * NQ) * Q_TILE, &P.tmQ, &q_full[g], qi.h * DH, qrow);
+                if (SPLIT) tma_load_2d(sQ + (g * NQ + 1) * Q_TILE, &P.tmQ, &q_full[g], (int)P.q_lo_col + qi.h * DH, qrow);
+              } else {
+                d.tile = -1;   // the group's tile stream is closed
+                mbar_arrive(&d_full[slot]);
+              }
+            }
+            if (qhave) {
+              kq[g] = k + 1;
+              ++qcount;
+              if (++qt == qi.ntiles) qhave = false;
+            } else {
+              ++closed;
+            }
+            progress = true;
+          }
+        }
+        if (!have && !more && fn == 0 && !qhave && !qmore && closed == GROUPS) break;
         if (progress) {
           t_idle = clock64();
         } else if (*abort_flag) {
@@ -419,90 +499,34 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
         ok = __shfl_sync(0xffffffffu, ok, 0);
       }
       // no copy of this CTA may still be landing when it exits (after an abort, the queue holds
-      // the copies issued and not passed on)
+      // the K/V copies issued and not passed on, and a group's last query copy may be in flight)
       while (fn > 0) {
-        const int j = (int)(fq_lo & 7u);
+        const int j = (int)(fq_lo & 15u);
         if (lane == 0) mbar_wait(&kv_full[j], (kv_par >> j) & 1u, P.status, nullptr);
         kv_par ^= 1u << j;
         fq_lo = (fq_lo >> 16) | (fq_hi << 48);
         fq_hi >>= 16;
         --fn;
       }
-    } else if (warp == 3 && lane == 0) {
-      // ---------------- query producer: tile descriptors and query tiles ----------------
-      // The query tiles of the CTA's requests alternate between the two groups; each group has
-      // one query buffer and AT_DESC descriptor slots.  A slot is rewritten only after the
-      // group's query buffer has been released three tiles later, by which time the softmax
-      // has written that tile's output (it does so while it works on the following tile).
-      prefetch_tensormap(&P.tmQ);
-      int tcount = 0, kq0 = 0, kq1 = 0;
-      bool ok = true;
-      for (int pass = 0; ok && pass * (long long)gridDim.x < n_items; ++pass) {
-        const int idx = at_item_index(pass, n_items);
-        if (idx < 0) continue;
-        AtItem it;
-        int bad;
-        at_item<RAGGED>(P, idx, it, bad);
-        if (bad != 0) set_status(P.status, bad);
-        if (it.ntiles == 0) continue;
-        for (int t = 0; t < it.ntiles; ++t) {
-          const int g = tcount & 1;
-          const int k = g ? kq1 : kq0;
-          if (k > 0 && !mbar_wait(&q_free[g], (k - 1) & 1, P.status, abort_flag)) {
-            ok = false;
-            break;
-          }
-          const int slot = g * AT_DESC + (k % AT_DESC);
-          AtTile& d = descs[slot];
-          d.q0 = it.q0;
-          d.q1 = it.q1;
-          d.tile = t;
-          d.h = it.h;
-          d.Lr = it.Lr;
-          d.nkb = it.nkb;
-          d.flags = t + GROUPS >= it.ntiles ? AT_LAST : 0u;
-          mbar_arrive(&d_full[slot]);
-          mbar_arrive_expect_tx(&q_full[g], NQ * Q_TILE);
-          const int qrow = (int)(it.q0 + (long long)t * TQ);
-          tma_load_2d(sQ + (g * NQ) * Q_TILE, &P.tmQ, &q_full[g], it.h * DH, qrow);
-          if (SPLIT) tma_load_2d(sQ + (g * NQ + 1) * Q_TILE, &P.tmQ, &q_full[g], (int)P.q_lo_col + it.h * DH, qrow);
-          if (g) ++kq1; else ++kq0;
-          ++tcount;
-        }
-      }
-      // close each group's tile stream; by then its last query tile has been read
-#pragma unroll
-      for (int g = 0; g < GROUPS; ++g) {
-        const int k = g ? kq1 : kq0;
-        if (ok && k > 0 && !mbar_wait(&q_free[g], (k - 1) & 1, P.status, abort_flag)) ok = false;
-        if (ok) {
-          const int slot = g * AT_DESC + (k % AT_DESC);
-          descs[slot].tile = -1;
-          mbar_arrive(&d_full[slot]);
-        }
-      }
-      // no copy of this CTA may still be landing when it exits
-#pragma unroll
-      for (int g = 0; g < GROUPS; ++g) {
-        const int k = g ? kq1 : kq0;
-        if (k > 0) mbar_wait(&q_full[g], (k - 1) & 1, P.status, nullptr);
-      }
-    } else if (warp >= 1 && warp <= GROUPS && lane == 0) {
+      if (lane == 0)
+        for (int g = 0; g < GROUPS; ++g)
+          if (kq[g] > 0) mbar_wait(&q_full[g], (kq[g] - 1) & 1, P.status, nullptr);
+    } else if (warp <= GROUPS && lane == 0) {
       // ---------------- MMA issuer of query-tile group g = warp - 1 ----------------
       // Per key block i of the group's tile stream:  S_i = Q K_j^T once the softmax has read
-      // S_{i-1} (s_free); then, for the previous block, O += P V_j and l += P 1 in two 64-key
-      // halves, each once the softmax has written that half of P (p_full).  After the group's
-      // last tile of a request, each block's P V is followed by a commit that hands the block
-      // back to the K/V producer (kv_empty).  Each group's MMAs touch only its own TMEM columns.
+      // S_{i-1} (s_free); then, for the previous block, O += P V_j and l += P 1 in two halves,
+      // each once the softmax has written that half of P (p_full).  After the group's last tile
+      // of an item, each block's P V is followed by a commit that hands the block back to the
+      // producer (kv_empty).  Each group's MMAs touch only its own TMEM columns.
       const int g = warp - 1;
       auto issue_pv = [&](int ib, int hh, int j, uint32_t fl, int nkb) -> bool {
         if (!mbar_wait(&p_full[2 * g + hh], ib & 1, P.status, abort_flag)) return false;
         tc_fence_after();
         const uint32_t va = smem_u32(sV + j * KV_BLOCK);
 #pragma unroll
-        for (int kq = 0; kq < TK / 32; ++kq) {
-          const int ks = hh * (TK / 32) + kq;
-          const uint32_t pa = tmem_base + C::P_COL + g * 64 + ks * 8;
+        for (int kq2 = 0; kq2 < TK / 32; ++kq2) {
+          const int ks = hh * (TK / 32) + kq2;
+          const uint32_t pa = tmem_base + C::P_COL + g * (TK / 2) + ks * 8;
           tc_mma_ts(tmem_base + C::O_COL + g * DH, pa, sdesc(va + ks * 16 * ROWB, SBO, SW), IDESC_O,
                     (ks > 0 || j > 0) ? 1u : 0u);
           if (C::SUM_MMA)
@@ -534,9 +558,9 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
       bool ok = true;
       int k = 0, i = 0;
       bool pend_pv = false;   // block i - 1's P V is not issued yet
-      int pj = 0, pnkb = 0;   // that block's index and its request's block count
+      int pj = 0, pnkb = 0;   // that block's index and its item's block count
       uint32_t pfl = 0;       // and its tile's flags
-      uint32_t rpar = 0;      // bit j: parity of kv_ready[j][g] for the next request this group reads
+      uint32_t rpar = 0;      // bit j: parity of kv_ready[j][g] for the next item this group reads
       for (;;) {
         const int slot = g * AT_DESC + (k % AT_DESC);
         if (!mbar_wait(&d_full[slot], (k / AT_DESC) & 1, P.status, abort_flag)) {
@@ -564,12 +588,11 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
           ++i;
         }
         if (!ok) break;
-        // The group's last tile of a request: its last P V (and the hand-back of the last block)
-        // is issued now, not after the next tile's first S, which may wait for the next request's
-        // K/V, whose load waits for this hand-back.  (Issuing that S first when it could start
-        // at once was measured 1% slower on the encoder.)
+        // The group's last tile of an item: its last P V (and the hand-back of the last block)
+        // is issued now, not after the next tile's first S, which may wait for the next item's
+        // K/V, whose load waits for this hand-back.
         if (fl & AT_LAST) {
-          rpar ^= (1u << nkb) - 1u;   // the group is done with this request's blocks
+          rpar ^= (1u << nkb) - 1u;   // the group is done with this item's blocks
           if (!(issue_pv(i - 1, 0, pj, pfl, pnkb) && issue_pv(i - 1, 1, pj, pfl, pnkb))) {
             ok = false;
             break;
@@ -590,7 +613,7 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
     const int row = quarter * 32 + lane;
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
     const uint32_t saddr = lane_addr + C::S_COL + g * TK;
-    const uint32_t paddr = lane_addr + C::P_COL + g * 64;
+    const uint32_t paddr = lane_addr + C::P_COL + g * (TK / 2);
     const uint32_t oaddr = lane_addr + C::O_COL + g * DH;
     const uint32_t laddr = lane_addr + C::L_COL + g * 16;
     // the group's tile descriptors, re-read where needed (kept out of the registers)
@@ -727,16 +750,16 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
           }
         }
         // exponentials: three pairs in eight on the FMA pipe (polynomial), the rest on MUFU; P_i
-        // as bf16 pairs into TMEM, one 64-key half at a time (32 keys per store), each half handed
+        // as bf16 pairs into TMEM, one half block at a time (32 keys per store), each half handed
         // to the tensor core as soon as it is written
         const float neg_m = -m_new;
         float rs = 0.f;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
-          uint32_t pk[2][16];
+          uint32_t pk[CH][16];
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            const int c = 2 * hh + cc;
+          for (int cc = 0; cc < CH; ++cc) {
+            const int c = CH * hh + cc;
 #pragma unroll
             for (int kk = 0; kk < 32; kk += 2) {
               float x0, x1, p0, p1;
@@ -763,8 +786,8 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
             }
             tc_fence_after();
           }
-          tmem_st_32x32b_x16(paddr + (2 * hh) * 16, pk[0]);
-          tmem_st_32x32b_x16(paddr + (2 * hh + 1) * 16, pk[1]);
+#pragma unroll
+          for (int cc = 0; cc < CH; ++cc) tmem_st_32x32b_x16(paddr + (CH * hh + cc) * 16, pk[cc]);
           if (hh == 0) {
             tmem_st_wait();
             tc_fence_before();
@@ -797,11 +820,11 @@ __global__ void __launch_bounds__(AtCfg<DH>::THREADS, 1) attn_tc_kernel(const __
   }
 }
 
-template <int DH, bool SPLIT>
+template <int DH, bool SPLIT, int G, int TK>
 size_t at_smem_bytes(int nkb) {
-  constexpr int G = AtCfg<DH>::GROUPS;
+  using C = AtCfg<DH, G, TK>;
   return 1024 + (size_t)2 * nkb * TK * DH * 2 + (size_t)G * (SPLIT ? 2 : 1) * TQ * DH * 2 + 2048 +
-         G * AT_DESC * sizeof(AtTile) + (size_t)(AT_MAX_KB * (1 + 2 * G) + G * (9 + AT_DESC)) * 8 + 16;
+         G * AT_DESC * sizeof(AtTile) + (size_t)(C::MAX_KB * (1 + 2 * G) + G * (9 + AT_DESC)) * 8 + 16;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -809,36 +832,44 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 bool encode_rows(rocs_context* ctx, CUtensorMap* map, const void* ptr, long long rows, long long cols, long long ld,
-                 int dh) {
+                 int dh, int box_rows) {
   EncodeTiledFn fn = reinterpret_cast<EncodeTiledFn>(ctx->encode_fn);
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
-  cuuint32_t box[2] = {(cuuint32_t)dh, 128};
+  cuuint32_t box[2] = {(cuuint32_t)dh, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, dh == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int DH, bool SPLIT, bool RAGGED>
-rocs_status at_launch(rocs_context* ctx, AttnTcParams& P, int B_R, int H, cudaStream_t s) {
-  const size_t smem = at_smem_bytes<DH, SPLIT>(P.nkb);
+template <int DH, bool SPLIT, bool RAGGED, int G, int TK>
+rocs_status at_launch(rocs_context* ctx, AttnTcParams& P, const void* K, const void* V, long long ldkv,
+                      long long kv_rows, int B_R, int H, cudaStream_t s) {
+  using C = AtCfg<DH, G, TK>;
+  P.nkb = (P.L + TK - 1) / TK;
+  const size_t smem = at_smem_bytes<DH, SPLIT, G, TK>(P.nkb);
   if (smem > 232448) {
     set_error("tcgen05 attention: L=%d needs %zu B of shared memory", P.L, smem);
     return ROCS_ERR_UNSUPPORTED;
   }
+  if (!encode_rows(ctx, &P.tmK, K, kv_rows, (long long)H * DH, ldkv, DH, TK) ||
+      !encode_rows(ctx, &P.tmV, V, kv_rows, (long long)H * DH, ldkv, DH, TK)) {
+    set_error("tcgen05 attention: cuTensorMapEncodeTiled failed");
+    return ROCS_ERR_CUDA;
+  }
   static bool attr[64] = {false};
   if (ctx->device < 64 && !attr[ctx->device]) {
-    rocs_status st = cuda_check(
-        cudaFuncSetAttribute(attn_tc_kernel<DH, SPLIT, RAGGED>, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448),
-        "cudaFuncSetAttribute(attn_tc)");
+    rocs_status st = cuda_check(cudaFuncSetAttribute(attn_tc_kernel<DH, SPLIT, RAGGED, G, TK>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, 232448),
+                                "cudaFuncSetAttribute(attn_tc)");
     if (st != ROCS_OK) return st;
     // the softmax warpgroups raise their register limit out of the block's launch allocation;
     // refuse to launch if the compiled kernel was given fewer registers than that split needs
     cudaFuncAttributes fa;
-    st = cuda_check(cudaFuncGetAttributes(&fa, attn_tc_kernel<DH, SPLIT, RAGGED>), "cudaFuncGetAttributes(attn_tc)");
+    st = cuda_check(cudaFuncGetAttributes(&fa, attn_tc_kernel<DH, SPLIT, RAGGED, G, TK>),
+                    "cudaFuncGetAttributes(attn_tc)");
     if (st != ROCS_OK) return st;
-    using C = AtCfg<DH>;
     if (fa.numRegs < C::REG_LAUNCH) {
       set_error("tcgen05 attention: kernel compiled with %d registers per thread, below the warpgroup split",
                 fa.numRegs);
@@ -850,8 +881,18 @@ rocs_status at_launch(rocs_context* ctx, AttnTcParams& P, int B_R, int H, cudaSt
   // (request, head) items
   const long long items = (long long)B_R * H;
   const unsigned grid = (unsigned)(items < ctx->num_sms ? items : ctx->num_sms);
-  attn_tc_kernel<DH, SPLIT, RAGGED><<<grid, AtCfg<DH>::THREADS, smem, s>>>(P);
+  attn_tc_kernel<DH, SPLIT, RAGGED, G, TK><<<grid, C::THREADS, smem, s>>>(P);
   return cuda_check(cudaGetLastError(), "attn_tc_kernel");
+}
+
+template <int DH, int G, int TK, int GS, int TKS>
+rocs_status at_dispatch(rocs_context* ctx, AttnTcParams& P, bool split, bool rag, const void* K, const void* V,
+                        long long ldkv, long long kv_rows, int B_R, int H, cudaStream_t s) {
+  if (split)
+    return rag ? at_launch<DH, true, true, GS, TKS>(ctx, P, K, V, ldkv, kv_rows, B_R, H, s)
+               : at_launch<DH, true, false, GS, TKS>(ctx, P, K, V, ldkv, kv_rows, B_R, H, s);
+  return rag ? at_launch<DH, false, true, G, TK>(ctx, P, K, V, ldkv, kv_rows, B_R, H, s)
+             : at_launch<DH, false, false, G, TK>(ctx, P, K, V, ldkv, kv_rows, B_R, H, s);
 }
 
 }  // namespace
@@ -862,7 +903,7 @@ rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq,
                                 int out_bf16, void* O2, long long ldo2, cudaStream_t s, const int32_t* out_rows,
                                 const int32_t* kv_len, int q_by_kv, const int32_t* order) {
   if (B_R == 0 || rows == 0) return ROCS_OK;
-  if ((d_h != 32 && d_h != 64) || L < 1 || (long long)L * d_h > 32768 || (L + TK - 1) / TK > AT_MAX_KB ||
+  if ((d_h != 32 && d_h != 64) || L < 1 || (long long)L * d_h > 32768 || L > AT_MAX_L ||
       (long long)B_R * H > 2147483647LL ||
       ((uintptr_t)Q & 15) || ((uintptr_t)K & 15) || ((uintptr_t)V & 15) || ldq % 8 || ldkv % 8 ||
       (q_split && (ldq < 2LL * H * d_h)) || ldkv < (long long)H * d_h || ((uintptr_t)O & 15) ||
@@ -873,8 +914,7 @@ rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq,
   AttnTcParams P;
   memset(&P, 0, sizeof(P));
   const long long qcols = q_split ? 2LL * H * d_h : (long long)H * d_h;
-  if (!encode_rows(ctx, &P.tmQ, Q, rows, qcols, ldq, d_h) || !encode_rows(ctx, &P.tmK, K, kv_rows, (long long)H * d_h, ldkv, d_h) ||
-      !encode_rows(ctx, &P.tmV, V, kv_rows, (long long)H * d_h, ldkv, d_h)) {
+  if (!encode_rows(ctx, &P.tmQ, Q, rows, qcols, ldq, d_h, TQ)) {
     set_error("tcgen05 attention: cuTensorMapEncodeTiled failed");
     return ROCS_ERR_CUDA;
   }
@@ -883,7 +923,6 @@ rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq,
   P.B_R = B_R;
   P.H = H;
   P.L = L;
-  P.nkb = (L + TK - 1) / TK;
   P.q_lo_col = (long long)H * d_h;
   P.scale_log2 = scale * 1.4426950408889634f;
   P.O = O;
@@ -898,12 +937,11 @@ rocs_status launch_attention_tc(rocs_context* ctx, const void* Q, long long ldq,
   P.status = ctx->d_status;
   LaunchTimer lt_("attn_tc", s);
   const bool rag = kv_len != nullptr;
-  if (d_h == 32) {
-    if (q_split) return rag ? at_launch<32, true, true>(ctx, P, B_R, H, s) : at_launch<32, true, false>(ctx, P, B_R, H, s);
-    return rag ? at_launch<32, false, true>(ctx, P, B_R, H, s) : at_launch<32, false, false>(ctx, P, B_R, H, s);
-  }
-  if (q_split) return rag ? at_launch<64, true, true>(ctx, P, B_R, H, s) : at_launch<64, true, false>(ctx, P, B_R, H, s);
-  return rag ? at_launch<64, false, true>(ctx, P, B_R, H, s) : at_launch<64, false, false>(ctx, P, B_R, H, s);
+  if (d_h == 32)
+    return at_dispatch<32, kAtGroups32, kAtKeys32, kAtGroupsSplit, kAtKeysSplit>(ctx, P, q_split != 0, rag, K, V, ldkv,
+                                                                               kv_rows, B_R, H, s);
+  return at_dispatch<64, kAtGroups64, kAtKeys64, kAtGroups64, kAtKeys64>(ctx, P, q_split != 0, rag, K, V, ldkv,
+                                                                         kv_rows, B_R, H, s);
 }
 
 }  // namespace rocs

@@ -4,8 +4,8 @@ mbarriers that, like the hardware's, are waited on by phase parity only.
 Roles, as in csrc/attn_tc.cu: the K/V producer issues block j of an item once every group that
 read block j of the previous copy has handed it back (kv_empty[j][g]); the copy lands after a
 random delay (kv_full[j], waited on by the producer alone, in issue order); the producer then
-passes the block to the groups that read the item (kv_ready[j][g]).  Query tiles alternate
-between two groups across items; a group reads the blocks of its tiles in order and hands each
+passes the block to the groups that read the item (kv_ready[j][g]).  Query tiles go to the
+groups (two or three) in turn across items; a group reads the blocks of its tiles in order and hands each
 block back after its last tile of the item.
 
 The model checks that every block a group reads holds its own item's data and that the run
@@ -32,17 +32,16 @@ class Barrier:
         return (self.phase & 1) != parity
 
 
-def simulate(seed, items, per_group_ready=True, nkb_max=8, steps=200000):
+def simulate(seed, items, per_group_ready=True, nkb_max=8, steps=200000, groups=2):
     """items: (query tiles, key blocks) per item, in the CTA's processing order."""
     rng = random.Random(seed)
-    groups = 2
-    tiles = {0: [], 1: []}
+    tiles = {g: [] for g in range(groups)}
     users = []
     tcount = 0
     for x, (nt, nkb) in enumerate(items):
-        users.append(3 if nt >= 2 else 1 << (tcount & 1))
+        users.append(sum(1 << ((tcount + t) % groups) for t in range(min(nt, groups))))
         for t in range(nt):
-            tiles[(tcount + t) & 1].append((x, nkb, t + groups >= nt))
+            tiles[(tcount + t) % groups].append((x, nkb, t + groups >= nt))
         tcount += nt
     kv_full = [Barrier() for _ in range(nkb_max)]
     kv_ready = [[Barrier() for _ in range(groups)] for _ in range(nkb_max)]
@@ -67,10 +66,10 @@ def simulate(seed, items, per_group_ready=True, nkb_max=8, steps=200000):
                 if c[0] <= now:
                     kv_empty[c[1]][g].arrive()
                     grp[g]["commits"].remove(c)
-        order = [0, 1, 2]
+        order = list(range(groups + 1))
         rng.shuffle(order)
         for who in order:
-            if who == 2:
+            if who == groups:
                 # producer: issue the next copy once its block is handed back
                 if prod["x"] < len(items) and len(prod["queue"]) < nkb_max:
                     x, j = prod["x"], prod["j"]
@@ -132,8 +131,12 @@ def _cases(n):
         yield seed, items
 
 
-def test_per_group_handoff_never_reads_a_foreign_block():
-    bad = [(seed, r) for seed, items in _cases(1500) for r in [simulate(seed, items)] if r != "ok"]
+import pytest
+
+
+@pytest.mark.parametrize("groups", [2, 3])
+def test_per_group_handoff_never_reads_a_foreign_block(groups):
+    bad = [(seed, r) for seed, items in _cases(1000) for r in [simulate(seed, items, groups=groups)] if r != "ok"]
     assert not bad, bad[:5]
 
 
