@@ -147,7 +147,6 @@ constexpr float kLazyRescaleLog2 = 8.0f;
 // and TK keys per block.
 template <int DH, int G, int TK>
 struct AtCfg {
-  static constexpr int GROUPS = G;
   static constexpr int MAX_KB = AT_MAX_L / TK;       // key blocks at most
   static constexpr bool SUM_MMA = DH == 32;          // row sums by an MMA of P against ones
   static constexpr int THREADS = 128 + 128 * G;
