@@ -439,7 +439,10 @@ def test_token_lcb(R, o_R, o_C):
 # ---------------------------------------------------------------------------------------------
 @pytest.mark.parametrize("L,H,dh,counts", [(200, 4, 64, [3, 0, 40, 17]), (1024, 8, 32, [33, 1]),
                                            (5, 2, 32, [16, 2, 0]), (512, 1, 64, [70]),
-                                           (1024, 8, 32, [300, 129, 0, 1000]), (200, 4, 64, [517, 2])])
+                                           (1024, 8, 32, [300, 129, 0, 1000]), (200, 4, 64, [517, 2]),
+                                           # key blocks with a ragged last one; many one-tile items,
+                                           # which the query-tile groups take in turn
+                                           (100, 2, 32, [40, 1, 0, 130]), (700, 8, 32, [5] * 40 + [300, 0, 129])])
 def test_cross_attention(R, L, H, dh, counts):
     counts = np.asarray(counts, np.int32)
     off, m = O.segments(counts)
