@@ -442,7 +442,10 @@ def test_token_lcb(R, o_R, o_C):
                                            (1024, 8, 32, [300, 129, 0, 1000]), (200, 4, 64, [517, 2]),
                                            # key blocks with a ragged last one; many one-tile items,
                                            # which the query-tile groups take in turn
-                                           (100, 2, 32, [40, 1, 0, 130]), (700, 8, 32, [5] * 40 + [300, 0, 129])])
+                                           (100, 2, 32, [40, 1, 0, 130]), (700, 8, 32, [5] * 40 + [300, 0, 129]),
+                                           # one key block per item, hundreds of one-tile items: the
+                                           # tile descriptor slots are reused at the fastest pace
+                                           (50, 4, 32, [3] * 100 + [129, 1]), (64, 8, 64, [7] * 60)])
 def test_cross_attention(R, L, H, dh, counts):
     counts = np.asarray(counts, np.int32)
     off, m = O.segments(counts)
