@@ -146,3 +146,95 @@ def test_model_finds_the_copy_barrier_aliasing():
     results = [simulate(seed, items, per_group_ready=False) for seed, items in _cases(1500)]
     assert sum(r != "ok" for r in results) > 0
     assert "wrong block" in results
+
+
+def simulate_descriptors(seed, blocks_per_tile, slots=4, steps=200000):
+    """One group's tile descriptors.  The producer writes tile k's descriptor into slot
+    k % slots once tile k - 1's queries are released (q_free: its last S product completed).  The
+    issuer runs S_0, S_1, PV_0, S_2, PV_1, ..., PV_last, each S_i once the softmax has read S_{i-1}
+    and each PV_m once P_m is written.  The softmax reads a tile's descriptor at its first block,
+    and again when it writes the previous tile's output (during that first block, after PV of
+    the previous block completed).  Returns "ok", "overwritten" (the softmax found another tile's
+    descriptor in the slot) or "stuck"."""
+    rng = random.Random(seed)
+    n = len(blocks_per_tile)
+    tile_of, last_of = [], []
+    for k, nb in enumerate(blocks_per_tile):
+        for j in range(nb):
+            tile_of.append(k)
+            last_of.append(j == nb - 1)
+    total = len(tile_of)
+    actions = [("S", 0)]
+    for i in range(1, total):
+        actions += [("S", i), ("PV", i - 1)]
+    actions.append(("PV", total - 1))
+    slot = [None] * slots
+    published = q_free = s_done = s_read = p_written = pv_done = 0
+    pending = []                       # (time, kind, block)
+    a = 0                              # issuer's next action
+    i_sm, phase = 0, 0                 # softmax: block, phase within it
+    for now in range(1, steps):
+        progress = False
+        for ev in [e for e in pending if e[0] <= now]:
+            pending.remove(ev)
+            if ev[1] == "S":
+                s_done += 1
+                if last_of[ev[2]]:
+                    q_free += 1
+            else:
+                pv_done += 1
+            progress = True
+        order = [0, 1, 2]
+        rng.shuffle(order)
+        for who in order:
+            if who == 0:
+                if published < n and (published == 0 or q_free >= published):
+                    slot[published % slots] = published
+                    published += 1
+                    progress = True
+            elif who == 1 and a < len(actions):
+                kind, i = actions[a]
+                if kind == "S" and published > tile_of[i] and (i == 0 or s_read >= i):
+                    pending.append((now + rng.randint(1, 10), "S", i))
+                    a += 1
+                    progress = True
+                elif kind == "PV" and p_written > i:
+                    pending.append((now + rng.randint(1, 10), "PV", i))
+                    a += 1
+                    progress = True
+            elif who == 2 and i_sm < total:
+                k = tile_of[i_sm]
+                first = i_sm == 0 or tile_of[i_sm - 1] != k
+                if phase == 0 and s_done > i_sm:
+                    if first and slot[k % slots] != k:
+                        return "overwritten"
+                    s_read = i_sm + 1
+                    phase = 1
+                    progress = True
+                elif phase == 1 and (i_sm == 0 or pv_done >= i_sm):
+                    if first and i_sm > 0 and slot[(k - 1) % slots] != k - 1:
+                        return "overwritten"
+                    p_written = i_sm + 1
+                    i_sm, phase = i_sm + 1, 0
+                    progress = True
+        if i_sm == total and pv_done == total:
+            return "ok" if slot[(n - 1) % slots] == n - 1 else "overwritten"
+        if not progress and not pending:
+            return "stuck"
+    return "stuck"
+
+
+@pytest.mark.parametrize("slots,expect_safe", [(4, True), (3, False)])
+def test_descriptor_slots_outlive_the_output(slots, expect_safe):
+    """Four slots per group (AT_DESC): a slot is rewritten only after the softmax has written the
+    output of the tile it held.  Three would not be enough when a tile has one key block."""
+    results = []
+    for seed in range(400):
+        rng = random.Random(seed)
+        tiles = [rng.choice([1, 1, 1, 2, 8]) for _ in range(rng.randint(2, 20))]
+        results.append(simulate_descriptors(seed, tiles, slots=slots))
+    assert "stuck" not in results
+    if expect_safe:
+        assert all(r == "ok" for r in results)
+    else:
+        assert "overwritten" in results
