@@ -69,7 +69,8 @@ struct AttnTcParams {
   const int32_t* out_rows;   // optional: query row q is written to output row out_rows[q]
   const int32_t* kv_len;     // optional: request r has kv_len[r] keys (1..L), the rest are padding
   int q_by_kv;               // with kv_len: request r's queries are also only its first kv_len[r] rows
-  const int32_t* order;      // optional: CTA group b serves request order[b] (a permutation; heaviest first)
+  const int32_t* order;      // optional: the item list takes the requests in this order (a permutation;
+                             // heaviest first spreads them evenly over the CTAs)
   int* status;
 };
 
