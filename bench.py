@@ -66,8 +66,22 @@ WORKLOADS = {
 }
 
 
-def make_case(name: str, rank: int, requests: int = 0):
-    """The workload's case; `requests` > 0 keeps only the first requests (smaller profiling runs)."""
+# Work of one request and of one candidate in the end-to-end forward (microseconds on one B200,
+# from the bench's per-site split: the encoder, its projections and the request query scale with
+# requests, everything else with candidates); the weights of the LPT request partition.
+SHARD_COST_R, SHARD_COST_C = 14.8, 0.0586
+
+
+def make_case(name: str, rank: int, requests: int = 0, shard: str = "own", world: int = 1):
+    """The workload's case; `requests` > 0 keeps only the first requests (smaller profiling runs).
+    shard "own": every rank draws its own batch (seed + 1000 rank; weak scaling).  shard "lpt":
+    every rank builds the same batch and keeps its part of rocs_partition_requests over `world`
+    parts (whole requests, longest processing time first; strong scaling)."""
+    if shard == "lpt" and world > 1:
+        full = make_case(name, 0, requests)
+        from request_candidate_sharing_b200 import rocs
+        part = rocs.partition_requests(full.counts, world, SHARD_COST_R, SHARD_COST_C)
+        return dataclasses.replace(full, counts=full.counts[part == rank].copy())
     seed_shift = 1000 * rank
     if name == "rocs_forward_e2e":
         case = synth.model_cfg5(seed=1 + seed_shift)
@@ -377,10 +391,10 @@ def allreduce(x: float, op: str, world: int) -> float:
     return float(t.item())
 
 
-def shard_totals(workload: str, rank: int, world: int, requests: int, local_ms: float):
-    """Weak-scaling bookkeeping of one rank: its own request shard, the job-wide candidate total
-    and the max-over-ranks time that the throughput divides by."""
-    case = make_case(workload, rank, requests)
+def shard_totals(workload: str, rank: int, world: int, requests: int, local_ms: float, shard: str = "own"):
+    """Multi-rank bookkeeping of one rank: its request shard, the job-wide candidate total and the
+    max-over-ranks time that the throughput divides by."""
+    case = make_case(workload, rank, requests, shard, world)
     total = allreduce(float(case.B_C), "sum", world)
     ms_max = allreduce(local_ms, "max", world)
     return case.B_C, total, ms_max
@@ -400,7 +414,7 @@ def run_librocs(args, rank, world, local):
 
     from request_candidate_sharing_b200 import rocs
     torch.cuda.set_device(local)
-    case = make_case(args.workload, rank, args.requests)
+    case = make_case(args.workload, rank, args.requests, args.shard, world)
     dev = torch.device("cuda", local)
     t_gen = time.perf_counter()
     W = synth.model_weights(case)
@@ -506,7 +520,7 @@ def run_librocs(args, rank, world, local):
         raise RuntimeError(f"device status {rocs.STATUS_NAMES.get(st, st)} in the timed region")
     # the exponential ceiling of the attention kernels, measured on this GPU now (B-16 probe)
     exp2_probe = {f"n_poly={n}": round(R.rocs_probe_exp2_rate(n, sh) / 1e9, 1) for n in (0, 3, 8)}
-    _, total_c, ms_max = shard_totals(args.workload, rank, world, args.requests, ms)
+    _, total_c, ms_max = shard_totals(args.workload, rank, world, args.requests, ms, args.shard)
     cands = total_c * args.steps
     value = cands / (ms_max / 1e3)
 
@@ -607,7 +621,8 @@ def run_librocs(args, rank, world, local):
 
     line = {"metric": METRIC, "value": round(value, 1), "unit": "candidates/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "strong" if args.shard == "lpt" and world > 1 else "weak",
+            "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) inputs, N(0,1/fan_in) bf16 weights)",
             "config": {"workload": args.workload + (f"[first {case.B_R} requests]" if args.requests else ""),
                        "description": WORKLOADS[args.workload], "B_R": case.B_R,
@@ -1154,6 +1169,9 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="rocs_forward_e2e", choices=sorted(WORKLOADS))
+    ap.add_argument("--shard", default="own", choices=["own", "lpt"],
+                    help="N > 1: each rank its own batch (weak scaling, the default) or the LPT "
+                         "partition of one batch (strong scaling)")
     ap.add_argument("--impl", default="librocs", choices=["librocs", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=4.0)

@@ -89,6 +89,22 @@ rocs_status rocs_segments_from_counts(rocs_handle_t handle, const int32_t* count
                                       int32_t* offsets, int32_t* req_idx, int64_t B_C, void* stream);
 
 /* ------------------------------------------------------------------------------------------
+ * Multi-GPU sharding (host only, no handle).  Requests are independent ([REV] §1: a request's
+ * inputs are constant across its candidates, and requests share only the weights), so a batch
+ * shards by whole requests with no exchange step.  rocs_partition_requests assigns each request
+ * of one batch to one of n_parts parts (GPUs), balancing the work cost_R + counts[r] * cost_C
+ * by longest-processing-time-first greedy: requests in decreasing work (ties: lower index
+ * first) each go to the part with the least work so far (ties: lower part).  The largest part is
+ * then within 4/3 of the best possible.  Deterministic.
+ *   counts  [B_R] int32, host: candidates of each request (>= 0).
+ *   part_of [B_R] int32, host, written: the part of request r, in [0, n_parts).
+ *   cost_R, cost_C >= 0 and finite, not both 0; 1 <= B_R <= 2^24; 1 <= n_parts <= 4096.
+ *   Returns ROCS_ERR_INVALID_ARG (nothing written) otherwise.
+ * ---------------------------------------------------------------------------------------- */
+rocs_status rocs_partition_requests(const int32_t* counts, int32_t B_R, int32_t n_parts, double cost_R,
+                                    double cost_C, int32_t* part_of);
+
+/* ------------------------------------------------------------------------------------------
  * a1-a3. Two-group GLM linear with in-kernel broadcast ([REV] §2.1 two-group block matrix,
  * §2.4 equation Y_i^C = Z_{m_i} + W_CC X_i^C):
  *   Y^R = act(W_RR X^R + b^R)                    on the request batch (B_R rows), once;

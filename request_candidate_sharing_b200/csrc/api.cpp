@@ -8,6 +8,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <queue>
 #include <string>
 #include <vector>
 
@@ -307,6 +308,36 @@ extern "C" rocs_status rocs_get_device_status(rocs_handle_t h, void* stream, int
   ROCS_TRY(cuda_check(cudaMemcpy(&v, h->d_status, sizeof(int), cudaMemcpyDeviceToHost), "read status"));
   ROCS_TRY(cuda_check(cudaMemset(h->d_status, 0, sizeof(int)), "clear status"));
   *code = v;
+  return ROCS_OK;
+}
+
+// =============================================================================================
+// Multi-GPU sharding: whole requests per part, longest processing time first
+// =============================================================================================
+extern "C" rocs_status rocs_partition_requests(const int32_t* counts, int32_t B_R, int32_t n_parts, double cost_R,
+                                               double cost_C, int32_t* part_of) {
+  ROCS_REQUIRE(counts && part_of, "rocs_partition_requests: NULL argument");
+  ROCS_REQUIRE(B_R >= 1 && B_R <= (1 << 24), "rocs_partition_requests: B_R out of range");
+  ROCS_REQUIRE(n_parts >= 1 && n_parts <= 4096, "rocs_partition_requests: n_parts out of range");
+  ROCS_REQUIRE(std::isfinite(cost_R) && std::isfinite(cost_C) && cost_R >= 0 && cost_C >= 0 &&
+                   (cost_R > 0 || cost_C > 0),
+               "rocs_partition_requests: costs must be finite, >= 0 and not both 0");
+  for (int32_t r = 0; r < B_R; ++r) ROCS_REQUIRE(counts[r] >= 0, "rocs_partition_requests: negative count");
+  std::vector<int32_t> idx(B_R);
+  for (int32_t r = 0; r < B_R; ++r) idx[r] = r;
+  // decreasing work; equal work keeps index order
+  std::stable_sort(idx.begin(), idx.end(), [&](int32_t a, int32_t b) { return counts[a] > counts[b]; });
+  // least-loaded part first, ties to the lower part
+  using Slot = std::pair<double, int32_t>;
+  std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> parts;
+  for (int32_t p = 0; p < n_parts; ++p) parts.push({0.0, p});
+  for (int32_t r : idx) {
+    Slot s = parts.top();
+    parts.pop();
+    part_of[r] = s.second;
+    s.first += cost_R + cost_C * (double)counts[r];
+    parts.push(s);
+  }
   return ROCS_OK;
 }
 

@@ -136,6 +136,7 @@ _lib_sort = _proto("rocs_sort_by_request", P, P, I32, I64, P, P, P, C.c_size_t, 
 _lib_xu_ws = _proto("rocs_dca_cross_attn_unsorted_workspace", P, I32, I64, I32, I32, C.c_int, C.POINTER(C.c_size_t))
 _lib_xu = _proto("rocs_dca_cross_attn_unsorted", P, P, P, P, P, I32, I64, I32, I32, I32, C.c_float, P, I64, C.c_int, P,
                  P, C.c_size_t, P)
+_lib_partition = _proto("rocs_partition_requests", P, I32, I32, C.c_double, C.c_double, P)
 _lib_tstart = _proto("rocs_timing_start", P, I32)
 _lib_tstop = _proto("rocs_timing_stop", P, C.c_char_p, C.c_size_t)
 
@@ -145,7 +146,8 @@ EXPORTED = ["rocs_linear_ikbo_noalloc", "rocs_timing_start", "rocs_timing_stop",
             "rocs_dca_encode_workspace", "rocs_dca_encode", "rocs_forward_workspace", "rocs_forward",
             "rocs_set_graph_replay", "rocs_set_ikbo_fused", "rocs_test_withhold_ikbo_flag", "rocs_probe_exp2_rate", "rocs_set_w8_tensor_cores", "rocs_sort_by_request_workspace",
             "rocs_sort_by_request", "rocs_dca_cross_attn_unsorted_workspace", "rocs_dca_cross_attn_unsorted",
-            "rocs_quantize_weights_fp8", "rocs_linear_ikbo_w8_workspace", "rocs_linear_ikbo_w8"]
+            "rocs_quantize_weights_fp8", "rocs_linear_ikbo_w8_workspace", "rocs_linear_ikbo_w8",
+            "rocs_partition_requests"]
 
 
 def ptr(x) -> Optional[int]:
@@ -155,6 +157,15 @@ def ptr(x) -> Optional[int]:
     if isinstance(x, int):
         return x
     return x.data_ptr()
+
+
+def partition_requests(counts, n_parts: int, cost_R: float, cost_C: float):
+    """rocs_partition_requests on host arrays: the part (0 .. n_parts-1) of each request."""
+    import numpy as np
+    c = np.ascontiguousarray(counts, dtype=np.int32)
+    out = np.empty(len(c), dtype=np.int32)
+    _check(_lib_partition(c.ctypes.data, len(c), int(n_parts), float(cost_R), float(cost_C), out.ctypes.data))
+    return out
 
 
 def rocs_last_error() -> str:
