@@ -230,11 +230,11 @@ __device__ __forceinline__ void at_item(const AttnTcParams& P, int idx, AtItem& 
 }
 
 // Item index of pass `pass` for this CTA: the list is dealt out in alternating directions
-// (CTA c takes items c, 2G - 1 - c, 2G + c, ...), so that a list sorted heaviest first spreads
-// evenly over the CTAs.  Returns -1 past the end of the list.
+// (CTA c of n takes items c, 2n - 1 - c, 2n + c, ...), so that a list sorted heaviest first
+// spreads evenly over the CTAs.  Returns -1 past the end of the list.
 __device__ __forceinline__ int at_item_index(int pass, int n_items) {
-  const int G = (int)gridDim.x, c = (int)blockIdx.x;
-  const long long idx = (long long)pass * G + ((pass & 1) ? G - 1 - c : c);
+  const int n = (int)gridDim.x, c = (int)blockIdx.x;
+  const long long idx = (long long)pass * n + ((pass & 1) ? n - 1 - c : c);
   return idx < n_items ? (int)idx : -1;
 }
 
