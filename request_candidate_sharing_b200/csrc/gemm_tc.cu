@@ -260,6 +260,7 @@ __device__ __forceinline__ void store_chunk_tma(const Problem& pr, uint8_t* buf,
   }
 }
 
+template <bool PLAIN>
 __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_constant__ Params P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -370,115 +371,54 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
       mbar_wait(drain, 0, P.status, nullptr);
     }
   } else {
-    // ---------------- epilogue warps ----------------
-    const int q = warp & 3;            // TMEM lane quarter this warp may access
-    const int half = (warp - 2) >> 2;  // which of the two warps on this quarter
-    const int row = q * 32 + lane;
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    // this row's request index in a tile, read one tile ahead of its use
-    auto load_gidx = [&](int tt) -> int {
-      if (tt >= P.total_tiles) return -1;
-      int pn, mn, nn;
-      decode_tile(P, tt, pn, mn, nn);
-      const Problem& q2 = P.p[pn];
-      const long long gn = (long long)mn * BM + row;
-      return (q2.Z != nullptr && gn < q2.M) ? __ldg(q2.gidx + gn) : -1;
-    };
-    int zi_next = load_gidx(blockIdx.x);
-    unsigned long long seen = 0;   // request tiles this warp has seen published (fused launches)
-    for (int t = blockIdx.x; t < P.total_tiles; t += gridDim.x) {
-      int pi, mb, nb;
-      decode_tile(P, t, pi, mb, nb);
-      const Problem& pr = P.p[pi];
-      const long long grow = (long long)mb * BM + row;
-      bool rvalid = grow < pr.M;
-      const float* zrow = nullptr;
-      const int zi = zi_next;
-      zi_next = load_gidx(t + gridDim.x);
-      if (rvalid && pr.Z != nullptr) {
-        if (zi < 0 || zi >= pr.gidx_bound) {
-          set_status(P.status, ROCS_ERR_INDEX);
-          rvalid = false;
-        } else {
-          zrow = pr.Z + (long long)zi * pr.ldz;
-          // this warp's chunks of the row's Z into L1 before the wait for the accumulator (the
-          // gathered rows were the epilogue's longest latency at short K); Z that this launch
-          // writes only once it is published (below)
-          if (pr.flag_role != 2)
-            for (int c = half; c < pr.BN / 32; c += 2)
-              if (nb * pr.BN + c * 32 < pr.N)
-                asm volatile("prefetch.global.L1 [%0];" ::"l"(zrow + nb * pr.BN + c * 32));
-        }
-      }
-      if (pr.flag_role == 2) {
-        // the request tiles holding this warp's rows' Z must have published (their tiles precede
-        // every candidate tile in each CTA's order, so they never wait on this one)
-        const int lo = __reduce_min_sync(0xffffffffu, zrow != nullptr ? zi : 0x7fffffff);
-        const int hi = __reduce_max_sync(0xffffffffu, zrow != nullptr ? zi : -1);
-        bool ok = true;
-        for (int mbr = hi >= 0 ? lo / BM : 1, mend = hi >= 0 ? hi / BM : 0; mbr <= mend && ok; ++mbr) {
-          // a tile seen published stays published: later tiles skip its flag (the first 64)
-          const int fi = mbr * pr.flag_ntiles + nb;
-          if (fi < 64 && ((seen >> fi) & 1ull)) continue;
-          if (lane == 0) ok = wait_flag(pr.flags + fi, EPI_THREADS / 32, P.flag_budget, P.status, abort_flag);
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-          if (ok && fi < 64) seen |= 1ull << fi;
-        }
-        if (!ok) {
-          rvalid = false;   // timed out: the status says so; this row is not written
-          zrow = nullptr;
-        } else if (zrow != nullptr) {
-          for (int c = half; c < pr.BN / 32; c += 2)
-            if (nb * pr.BN + c * 32 < pr.N)
-              asm volatile("prefetch.global.L1 [%0];" ::"l"(zrow + nb * pr.BN + c * 32));
-        }
-      }
-      if (!mbar_wait(&tfull[acc], acc_phase, P.status, abort_flag)) break;
-      tc_fence_after();
-      // a row with a bad request index is skipped, not written: such a warp stores element-wise
-      const bool use_tma = pr.tma_out && !__any_sync(0xffffffffu, grow < pr.M && !rvalid);
-      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MAX);
-      const int nchunks = pr.BN / 32;
-      // this warp takes chunks half, half + 2, ... (bf16 output through TMA: adjacent pairs of
-      // chunks 2p, 2p + 1 for p = half, half + 2, ..., one 32 x 64 store per pair); it releases the
-      // accumulator after its last load
-      const bool pair_path = use_tma && pr.out_mode == 1;
-      const int npairs = (nchunks + 1) / 2;
-      const int lp = npairs - 1 - ((npairs - 1 - half) & 1);
-      const int last = pair_path ? (lp < 0 ? -1 : (2 * lp + 1 < nchunks ? 2 * lp + 1 : nchunks - 1))
-                                 : nchunks - 1 - ((nchunks - 1 - half) & 1);
-      if (last < 0) {
-        mbar_arrive(&tempty[acc]);
-      }
-      if (pair_path) {
-        uint8_t* buf = sEpi + (warp - 2) * EPI_BUF;
-        uint8_t* rowp = buf + lane * 128;
+    if constexpr (PLAIN) {
+      // ---------------- epilogue warps, bf16 output with nothing to add or apply ----------------
+      // (the encoder's projections): both chunks of a pair are loaded from TMEM before one wait
+      // and go straight to bf16.  A kernel of its own, so the general epilogue's state does not
+      // crowd its registers.
+      const int q = warp & 3, half = (warp - 2) >> 2;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      uint8_t* buf = sEpi + (warp - 2) * EPI_BUF;
+      uint8_t* rowp = buf + lane * 128;
+      for (int t = blockIdx.x; t < P.total_tiles; t += gridDim.x) {
+        int pi, mb, nb;
+        decode_tile(P, t, pi, mb, nb);
+        const Problem& pr = P.p[pi];
+        if (!mbar_wait(&tfull[acc], acc_phase, P.status, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MAX);
+        const int nchunks = pr.BN / 32, npairs = (nchunks + 1) / 2;
+        const int lp = npairs - 1 - ((npairs - 1 - half) & 1);   // this warp's last pair (< 0: none)
+        if (lp < 0) mbar_arrive(&tempty[acc]);
         for (int pp = half; pp < npairs; pp += 2) {
           if (lane == 0) bulk_wait_read_all();   // the previous copy has read the buffer
           __syncwarp();
-#pragma unroll 1
-          for (int hh = 0; hh < 2; ++hh) {
-            const int c = 2 * pp + hh;
-            if (c >= nchunks) break;
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(tbase + (uint32_t)(c * 32), r);
-            tmem_ld_wait();
-            if (c == last) {
-              tc_fence_before();
-              mbar_arrive(&tempty[acc]);
-            }
-            const int col0 = nb * pr.BN + c * 32;
-            float v[32];
+          const bool two = 2 * pp + 1 < nchunks;
+          uint32_t r0[32], r1[32];
+          tmem_ld_32x32b_x32(tbase + (uint32_t)(2 * pp * 32), r0);
+          if (two) tmem_ld_32x32b_x32(tbase + (uint32_t)((2 * pp + 1) * 32), r1);
+          tmem_ld_wait();
+          if (pp == lp) {
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+          }
+          // 128-byte rows, 128-byte swizzle: 16-byte unit j of row r at j ^ (r & 7)
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-            if (rvalid) epilogue_math(pr, zrow, col0, v);
-            // 128-byte rows, 128-byte swizzle: 16-byte unit j of row r at j ^ (r & 7)
+          for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<uint4*>(rowp + ((u ^ (lane & 7)) << 4)) =
+                make_uint4(pack_bf16x2(__uint_as_float(r0[8 * u]), __uint_as_float(r0[8 * u + 1])),
+                           pack_bf16x2(__uint_as_float(r0[8 * u + 2]), __uint_as_float(r0[8 * u + 3])),
+                           pack_bf16x2(__uint_as_float(r0[8 * u + 4]), __uint_as_float(r0[8 * u + 5])),
+                           pack_bf16x2(__uint_as_float(r0[8 * u + 6]), __uint_as_float(r0[8 * u + 7])));
+          if (two) {
 #pragma unroll
             for (int u = 0; u < 4; ++u)
-              *reinterpret_cast<uint4*>(rowp + (((4 * hh + u) ^ (lane & 7)) << 4)) =
-                  make_uint4(pack_bf16x2(v[8 * u], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
-                             pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
+              *reinterpret_cast<uint4*>(rowp + (((4 + u) ^ (lane & 7)) << 4)) =
+                  make_uint4(pack_bf16x2(__uint_as_float(r1[8 * u]), __uint_as_float(r1[8 * u + 1])),
+                             pack_bf16x2(__uint_as_float(r1[8 * u + 2]), __uint_as_float(r1[8 * u + 3])),
+                             pack_bf16x2(__uint_as_float(r1[8 * u + 4]), __uint_as_float(r1[8 * u + 5])),
+                             pack_bf16x2(__uint_as_float(r1[8 * u + 6]), __uint_as_float(r1[8 * u + 7])));
           }
           fence_proxy_async_smem();
           __syncwarp();
@@ -487,93 +427,218 @@ __global__ void __launch_bounds__(THREADS, 1) gemm_tc_kernel(const __grid_consta
             bulk_commit_group();
           }
         }
-      } else
-      for (int c = half; c < nchunks; c += 2) {
-        uint32_t r[32];
-        __syncwarp();
-        tmem_ld_32x32b_x32(tbase + (uint32_t)(c * 32), r);
-        tmem_ld_wait();
-        if (c == last) {
-          tc_fence_before();
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+      // this warp's output stores have landed before the CTA (and its staging memory) goes away
+      if (lane == 0) bulk_wait_all();
+      __syncwarp();
+    } else {
+      // ---------------- epilogue warps ----------------
+      const int q = warp & 3;            // TMEM lane quarter this warp may access
+      const int half = (warp - 2) >> 2;  // which of the two warps on this quarter
+      const int row = q * 32 + lane;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      // this row's request index in a tile, read one tile ahead of its use
+      auto load_gidx = [&](int tt) -> int {
+        if (tt >= P.total_tiles) return -1;
+        int pn, mn, nn;
+        decode_tile(P, tt, pn, mn, nn);
+        const Problem& q2 = P.p[pn];
+        const long long gn = (long long)mn * BM + row;
+        return (q2.Z != nullptr && gn < q2.M) ? __ldg(q2.gidx + gn) : -1;
+      };
+      int zi_next = load_gidx(blockIdx.x);
+      unsigned long long seen = 0;   // request tiles this warp has seen published (fused launches)
+      for (int t = blockIdx.x; t < P.total_tiles; t += gridDim.x) {
+        int pi, mb, nb;
+        decode_tile(P, t, pi, mb, nb);
+        const Problem& pr = P.p[pi];
+        const long long grow = (long long)mb * BM + row;
+        bool rvalid = grow < pr.M;
+        const float* zrow = nullptr;
+        const int zi = zi_next;
+        zi_next = load_gidx(t + gridDim.x);
+        if (rvalid && pr.Z != nullptr) {
+          if (zi < 0 || zi >= pr.gidx_bound) {
+            set_status(P.status, ROCS_ERR_INDEX);
+            rvalid = false;
+          } else {
+            zrow = pr.Z + (long long)zi * pr.ldz;
+            // this warp's chunks of the row's Z into L1 before the wait for the accumulator (the
+            // gathered rows were the epilogue's longest latency at short K); Z that this launch
+            // writes only once it is published (below)
+            if (pr.flag_role != 2)
+              for (int c = half; c < pr.BN / 32; c += 2)
+                if (nb * pr.BN + c * 32 < pr.N)
+                  asm volatile("prefetch.global.L1 [%0];" ::"l"(zrow + nb * pr.BN + c * 32));
+          }
+        }
+        if (pr.flag_role == 2) {
+          // the request tiles holding this warp's rows' Z must have published (their tiles precede
+          // every candidate tile in each CTA's order, so they never wait on this one)
+          const int lo = __reduce_min_sync(0xffffffffu, zrow != nullptr ? zi : 0x7fffffff);
+          const int hi = __reduce_max_sync(0xffffffffu, zrow != nullptr ? zi : -1);
+          bool ok = true;
+          for (int mbr = hi >= 0 ? lo / BM : 1, mend = hi >= 0 ? hi / BM : 0; mbr <= mend && ok; ++mbr) {
+            // a tile seen published stays published: later tiles skip its flag (the first 64)
+            const int fi = mbr * pr.flag_ntiles + nb;
+            if (fi < 64 && ((seen >> fi) & 1ull)) continue;
+            if (lane == 0) ok = wait_flag(pr.flags + fi, EPI_THREADS / 32, P.flag_budget, P.status, abort_flag);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (ok && fi < 64) seen |= 1ull << fi;
+          }
+          if (!ok) {
+            rvalid = false;   // timed out: the status says so; this row is not written
+            zrow = nullptr;
+          } else if (zrow != nullptr) {
+            for (int c = half; c < pr.BN / 32; c += 2)
+              if (nb * pr.BN + c * 32 < pr.N)
+                asm volatile("prefetch.global.L1 [%0];" ::"l"(zrow + nb * pr.BN + c * 32));
+          }
+        }
+        if (!mbar_wait(&tfull[acc], acc_phase, P.status, abort_flag)) break;
+        tc_fence_after();
+        // a row with a bad request index is skipped, not written: such a warp stores element-wise
+        const bool use_tma = pr.tma_out && !__any_sync(0xffffffffu, grow < pr.M && !rvalid);
+        const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN_MAX);
+        const int nchunks = pr.BN / 32;
+        // this warp takes chunks half, half + 2, ... (bf16 output through TMA: adjacent pairs of
+        // chunks 2p, 2p + 1 for p = half, half + 2, ..., one 32 x 64 store per pair); it releases the
+        // accumulator after its last load
+        const bool pair_path = use_tma && pr.out_mode == 1;
+        const int npairs = (nchunks + 1) / 2;
+        const int lp = npairs - 1 - ((npairs - 1 - half) & 1);
+        const int last = pair_path ? (lp < 0 ? -1 : (2 * lp + 1 < nchunks ? 2 * lp + 1 : nchunks - 1))
+                                   : nchunks - 1 - ((nchunks - 1 - half) & 1);
+        if (last < 0) {
           mbar_arrive(&tempty[acc]);
         }
-        const int col0 = nb * pr.BN + c * 32;
-        if (use_tma && col0 < pr.N && mb * BM + q * 32 < pr.M) {
-          // every lane takes part in the staged store; rows past M are clipped by the copy
-          float v[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          if (rvalid) epilogue_math(pr, zrow, col0, v);
-          store_chunk_tma(pr, sEpi + (warp - 2) * EPI_BUF, mb * BM + q * 32, col0, v);
-        } else if (!use_tma && rvalid && col0 < pr.N) {
-          float v[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          const bool full32 = (col0 + 32 <= pr.N) && pr.vec_ok;
-          if (pr.scale != nullptr) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] *= col0 + j < pr.N ? __ldg(pr.scale + col0 + j) : 0.f;
-          }
-          if (pr.bias != nullptr) {
-            if (full32) {
-              const float4* b4 = reinterpret_cast<const float4*>(pr.bias + col0);
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                float4 b = __ldg(b4 + j);
-                v[4 * j] += b.x; v[4 * j + 1] += b.y; v[4 * j + 2] += b.z; v[4 * j + 3] += b.w;
+        if (pair_path) {
+          uint8_t* buf = sEpi + (warp - 2) * EPI_BUF;
+          uint8_t* rowp = buf + lane * 128;
+          for (int pp = half; pp < npairs; pp += 2) {
+            if (lane == 0) bulk_wait_read_all();   // the previous copy has read the buffer
+            __syncwarp();
+  #pragma unroll 1
+            for (int hh = 0; hh < 2; ++hh) {
+              const int c = 2 * pp + hh;
+              if (c >= nchunks) break;
+              uint32_t r[32];
+              tmem_ld_32x32b_x32(tbase + (uint32_t)(c * 32), r);
+              tmem_ld_wait();
+              if (c == last) {
+                tc_fence_before();
+                mbar_arrive(&tempty[acc]);
               }
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (col0 + j < pr.N) v[j] += pr.bias[col0 + j];
+              const int col0 = nb * pr.BN + c * 32;
+              float v[32];
+  #pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+              if (rvalid) epilogue_math(pr, zrow, col0, v);
+              // 128-byte rows, 128-byte swizzle: 16-byte unit j of row r at j ^ (r & 7)
+  #pragma unroll
+              for (int u = 0; u < 4; ++u)
+                *reinterpret_cast<uint4*>(rowp + (((4 * hh + u) ^ (lane & 7)) << 4)) =
+                    make_uint4(pack_bf16x2(v[8 * u], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
+                               pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7]));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              if (mb * BM + q * 32 < pr.M) tma_store_2d(&pr.tmO, buf, nb * pr.BN + 64 * pp, mb * BM + q * 32);
+              bulk_commit_group();
             }
           }
-          if (zrow != nullptr) {
-            if (full32) {
-              const float4* z4 = reinterpret_cast<const float4*>(zrow + col0);
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                float4 z = __ldg(z4 + j);
-                v[4 * j] += z.x; v[4 * j + 1] += z.y; v[4 * j + 2] += z.z; v[4 * j + 3] += z.w;
-              }
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (col0 + j < pr.N) v[j] += zrow[col0 + j];
+        } else
+        for (int c = half; c < nchunks; c += 2) {
+          uint32_t r[32];
+          __syncwarp();
+          tmem_ld_32x32b_x32(tbase + (uint32_t)(c * 32), r);
+          tmem_ld_wait();
+          if (c == last) {
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+          }
+          const int col0 = nb * pr.BN + c * 32;
+          if (use_tma && col0 < pr.N && mb * BM + q * 32 < pr.M) {
+            // every lane takes part in the staged store; rows past M are clipped by the copy
+            float v[32];
+  #pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+            if (rvalid) epilogue_math(pr, zrow, col0, v);
+            store_chunk_tma(pr, sEpi + (warp - 2) * EPI_BUF, mb * BM + q * 32, col0, v);
+          } else if (!use_tma && rvalid && col0 < pr.N) {
+            float v[32];
+  #pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+            const bool full32 = (col0 + 32 <= pr.N) && pr.vec_ok;
+            if (pr.scale != nullptr) {
+  #pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] *= col0 + j < pr.N ? __ldg(pr.scale + col0 + j) : 0.f;
             }
+            if (pr.bias != nullptr) {
+              if (full32) {
+                const float4* b4 = reinterpret_cast<const float4*>(pr.bias + col0);
+  #pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  float4 b = __ldg(b4 + j);
+                  v[4 * j] += b.x; v[4 * j + 1] += b.y; v[4 * j + 2] += b.z; v[4 * j + 3] += b.w;
+                }
+              } else {
+  #pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (col0 + j < pr.N) v[j] += pr.bias[col0 + j];
+              }
+            }
+            if (zrow != nullptr) {
+              if (full32) {
+                const float4* z4 = reinterpret_cast<const float4*>(zrow + col0);
+  #pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  float4 z = __ldg(z4 + j);
+                  v[4 * j] += z.x; v[4 * j + 1] += z.y; v[4 * j + 2] += z.z; v[4 * j + 3] += z.w;
+                }
+              } else {
+  #pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (col0 + j < pr.N) v[j] += zrow[col0 + j];
+              }
+            }
+            switch (pr.act) {
+              case ROCS_ACT_RELU:
+  #pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = fmaxf(v[j], 0.f);
+                break;
+              case ROCS_ACT_GELU:
+  #pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
+                break;
+              case ROCS_ACT_SIGMOID:
+  #pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = sigmoid_fast(v[j]);
+                break;
+              default:
+                break;
+            }
+            store_chunk(pr, grow, col0, v);
           }
-          switch (pr.act) {
-            case ROCS_ACT_RELU:
-#pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] = fmaxf(v[j], 0.f);
-              break;
-            case ROCS_ACT_GELU:
-#pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] = gelu_erf(v[j]);
-              break;
-            case ROCS_ACT_SIGMOID:
-#pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] = sigmoid_fast(v[j]);
-              break;
-            default:
-              break;
-          }
-          store_chunk(pr, grow, col0, v);
         }
+        if (pr.flag_role == 1) {
+          // this warp's part of the tile is stored (plain stores): publish it device-wide
+          __threadfence();
+          __syncwarp();
+          const int fi = mb * pr.n_tiles + nb;
+          if (lane == 0 && fi != P.withhold_flag) atomicAdd(pr.flags + fi, 1);
+        }
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
       }
-      if (pr.flag_role == 1) {
-        // this warp's part of the tile is stored (plain stores): publish it device-wide
-        __threadfence();
-        __syncwarp();
-        const int fi = mb * pr.n_tiles + nb;
-        if (lane == 0 && fi != P.withhold_flag) atomicAdd(pr.flags + fi, 1);
-      }
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1;
+      // this warp's output stores have landed before the CTA (and its staging memory) goes away
+      if (lane == 0) bulk_wait_all();
+      __syncwarp();
     }
-    // this warp's output stores have landed before the CTA (and its staging memory) goes away
-    if (lane == 0) bulk_wait_all();
-    __syncwarp();
   }
 
   tc_fence_before();
@@ -628,8 +693,12 @@ rocs_status launch_gemm_bf16(rocs_context* ctx, const GemmDesc* probs, int nprob
   static bool attr_set[64] = {false};
   if (ctx->device < 64 && !attr_set[ctx->device]) {
     rocs_status st = cuda_check(
-        cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES),
+        cudaFuncSetAttribute(gemm_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES),
         "cudaFuncSetAttribute(gemm)");
+    if (st == ROCS_OK)
+      st = cuda_check(
+          cudaFuncSetAttribute(gemm_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES),
+          "cudaFuncSetAttribute(gemm)");
     if (st != ROCS_OK) return st;
     attr_set[ctx->device] = true;
   }
@@ -730,7 +799,17 @@ rocs_status launch_gemm_bf16(rocs_context* ctx, const GemmDesc* probs, int nprob
   const int grid = std::min(tiles, ctx->num_sms);
   LaunchTimer lt_("gemm_tc", s);
   if (!flagged) {
-    gemm_tc_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(P);
+    // bf16 outputs stored through TMA with nothing to add or apply take the lean epilogue
+    bool plain = true;
+    for (int i = 0; i < nprob; ++i) {
+      const Problem& p = P.p[i];
+      plain = plain && p.out_mode == 1 && p.tma_out && p.bias == nullptr && p.Z == nullptr && p.scale == nullptr &&
+              p.act == ROCS_ACT_NONE;
+    }
+    if (plain)
+      gemm_tc_kernel<true><<<grid, THREADS, SMEM_BYTES, s>>>(P);
+    else
+      gemm_tc_kernel<false><<<grid, THREADS, SMEM_BYTES, s>>>(P);
     return cuda_check(cudaGetLastError(), "gemm_tc_kernel launch");
   }
   // readers spin on tiles other CTAs publish: launch cooperatively (all CTAs resident)
@@ -744,7 +823,7 @@ rocs_status launch_gemm_bf16(rocs_context* ctx, const GemmDesc* probs, int nprob
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_check(cudaLaunchKernelEx(&cfg, gemm_tc_kernel, P), "gemm_tc_kernel cooperative launch");
+  return cuda_check(cudaLaunchKernelEx(&cfg, gemm_tc_kernel<false>, P), "gemm_tc_kernel cooperative launch");
 }
 
 }  // namespace rocs
