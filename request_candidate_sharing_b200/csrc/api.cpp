@@ -1142,7 +1142,6 @@ rocs_status forward_launches(rocs_handle_t h, const rocs_model_desc* m, const ro
   const void* S_prev = in->Hist;
   const int steps = m->glm_layers > m->dca_layers ? m->glm_layers : m->dca_layers;
   const long long d2 = 2LL * m->d, q2 = 2LL * m->q_dim;
-  const bool fused_ok = m->D == 128 && m->lcb_out_C <= 8 && m->n_C <= 16;
 
   for (int l = 0; l < steps; ++l) {
     const bool glm_l = l < m->glm_layers;
@@ -1163,7 +1162,7 @@ rocs_status forward_launches(rocs_handle_t h, const rocs_model_desc* m, const ro
       if (qw)
         ROCS_TRY(launch_token_lcb(h, ER, wr, EC, wc, req_idx, BR, 0, m->n_R, m->n_C, m->D, qw->p_RR, qw->p_CR,
                                   qw->p_CC, 1, 1, p.tR, q2, p.tC, q2, e_f32, 2, m->q_dim, m->q_dim, p.ZqL, s));
-      if (fused_ok) {
+      if (glm_cand_fused_fits(m->D, m->n_R, m->n_C, m->lcb_out_C, e_f32)) {
         // candidate side in one kernel: F^C (hi/lo), L^C and the depth-l query token t^C
         ROCS_TRY(launch_glm_cand_fused(h, ER, EC, req_idx, BR, BC, m->n_R, m->n_C, e_f32, p.FC, gw.P_CC, m->lcb_out_C,
                                        p.ZL, p.LC, qw ? qw->p_CC : nullptr, p.ZqL, qw ? p.tC : nullptr, s));

@@ -16,6 +16,8 @@
 #include "internal.h"
 #include "mma_frag.cuh"
 
+#include <cstring>
+
 namespace rocs {
 namespace {
 
@@ -128,8 +130,8 @@ __device__ __forceinline__ void gram_tile(uint32_t sbase, int pitch, int a0, int
 //   L^C_c  = Z^L_{m_c} + P_CC E^C_c                  (token LCB, fp32; Z^L = P_CR E^R per request)
 //   t^C_c  = Z^Q_{m_c} + p_CC E^C_c                  (optional: the DCA query generator's one-token
 //                                                      LCB of the same embeddings, bf16 hi/lo pairs)
-// Lane j owns features [DPL*j, DPL*j + DPL); the LCB sums use the full-precision embeddings, the
-// FM products their bf16 rounding (tensor-core operands).
+// The LCB sums take fp32 embeddings as a bf16 hi + lo pair (bf16 ones as they are), the FM
+// products their bf16 rounding; both run as m16n8k16 tensor-core fragments.
 // ---------------------------------------------------------------------------------------------
 // One CTA per SM walks a contiguous range of candidates.  Warp 0 streams each candidate's E^C rows
 // (contiguous, n_C x D) into a ring of shared-memory stages with bulk async copies, FC_STAGES
@@ -138,11 +140,38 @@ __device__ __forceinline__ void gram_tile(uint32_t sbase, int pitch, int a0, int
 // each candidate over two warps halves the registers a warp needs (its half of the features and of
 // the Gram k-range) and doubles the warps that hide each other's latencies.
 constexpr int FC_PAIRS = 7;                    // consumer warp pairs, one candidate tile each
-constexpr int FC_CONSUMERS = 2 * FC_PAIRS;     // 15 warps in all: 136 registers per thread
+constexpr int FC_CONSUMERS = 2 * FC_PAIRS;     // 15 warps in all: at most 128 registers per thread
 constexpr int FC_STAGES = 12;
 // A pair's next candidate (i + pairs) reuses the stage of candidate i + pairs - stages, which must
 // already have been loaded (it is <= i) for the parity of its mbarrier wait to be unambiguous.
 static_assert(FC_STAGES >= FC_PAIRS, "ring stages must cover the consumer pairs");
+// Each pair's block of shared memory starts with one region per warp (1024-byte aligned, so a
+// 128-byte-swizzled TMA box can start there).  Warp hf's region holds feature half hf of the
+// candidate's lo rows (fp32 inputs), read only by warp hf's token LCB; after that the same bytes
+// stage warp hf's L^C columns for a TMA store, and then its partial Gram sums for the exchange.
+// The pair's tile [E^R rows ; E^C hi rows ; 0 pad] follows the two regions.
+constexpr int FC_LO_PITCH = 144;                            // 64 bf16 + 16 bytes: conflict-free ldmatrix rows
+constexpr int FC_HALF = 3072;                               // one warp's region
+constexpr int FC_LO_BYTES = FC_HALF + NC_MAX * FC_LO_PITCH; // both regions (the second one ends early)
+static_assert(NC_MAX * FC_LO_PITCH <= FC_HALF && FC_HALF % 1024 == 0, "lo-row regions");
+static_assert(2 * 1024 <= NC_MAX * FC_LO_PITCH, "two 8 x 32 fp32 swizzled boxes per warp region");
+static_assert(4 * 32 * 16 <= NC_MAX * FC_LO_PITCH, "exchange slot per warp region");
+
+__host__ __device__ constexpr int fc_pair_bytes(int trows, int pitch) {
+  return (FC_LO_BYTES + trows * pitch + 1023) / 1024 * 1024;
+}
+
+__device__ __forceinline__ void st_shared_f32x2(uint32_t addr, float a, float b) {
+  asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
+}
+__device__ __forceinline__ void st_shared_f32x4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+__device__ __forceinline__ float4 ld_shared_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
+  return v;
+}
 
 // Barrier `id` over the 64 threads of a consumer pair.
 __device__ __forceinline__ void pair_sync(int id) { asm volatile("bar.sync %0, 64;" ::"r"(id) : "memory"); }
@@ -163,9 +192,10 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
     long long B_C, long long per_block, int n_R, int n_C, int trows, int pitch, __nv_bfloat16* __restrict__ F_C,
     const __nv_bfloat16* __restrict__ P_CC, int o_C, const float* __restrict__ ZL, float* __restrict__ L_C,
     const __nv_bfloat16* __restrict__ q_pCC, const float* __restrict__ ZQ, __nv_bfloat16* __restrict__ tC,
-    int* status) {
+    const __grid_constant__ CUtensorMap mapL, int l_tma, int* status) {
   constexpr int D = 128;
-  extern __shared__ __align__(128) uint8_t fc_smem[];
+  extern __shared__ __align__(128) uint8_t fc_smem_raw[];
+  uint8_t* fc_smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(fc_smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ float sP[LCB_OMAX_F * 64];
   __shared__ float sQ[64];
   __shared__ __align__(8) uint64_t full[FC_STAGES], empty[FC_STAGES];
@@ -180,6 +210,7 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
   const int n = (int)(c1 - c0);
   const uint32_t stage_bytes = (uint32_t)(n_C * D * sizeof(TIN));
   uint8_t* ring = fc_smem;
+  static_assert(FC_STAGES * NC_MAX * D * sizeof(TIN) % 1024 == 0, "pair blocks start 1024-byte aligned");
   uint8_t* tiles = fc_smem + FC_STAGES * NC_MAX * D * sizeof(TIN);
 
   for (int i = threadIdx.x; i < o_C * n_C; i += blockDim.x) sP[i] = __bfloat162float(P_CC[i]);
@@ -219,27 +250,30 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
   // ---------------- consumers: warp pairs ----------------
   // Pair pr takes candidates pr, pr + FC_PAIRS, ... of the range; warp hf of the pair owns features
   // [64 hf, 64 hf + 64) of the token LCB and the k-half [64 hf, 64 hf + 64) of the Gram products,
-  // whose partial sums the two warps exchange through the pair's lo-row tile (free once the LCB
-  // has read it).  Named barrier 1 + pr synchronises the pair.
+  // whose partial sums the two warps exchange through their lo-row regions (each free once its
+  // own warp's LCB has read it).  Named barrier 1 + pr synchronises the pair.
   const int cw = warp - 1, pr = cw >> 1, hf = cw & 1;
   const int bar_id = 1 + pr;
-  uint8_t* T = tiles + pr * (trows + NC_MAX) * pitch;   // [E^R rows ; E^C hi rows ; 0 pad] then E^C lo rows
-  uint8_t* TL = T + trows * pitch;
-  float4* xb = reinterpret_cast<float4*>(TL);           // exchange: [warp][4 n-tile slots][32 lanes]
+  uint8_t* TL = tiles + pr * fc_pair_bytes(trows, pitch);   // two warp regions, FC_HALF bytes apart
+  uint8_t* TLh = TL + hf * FC_HALF;                         // this warp's region
+  uint8_t* T = TL + FC_LO_BYTES;                            // [E^R rows ; E^C hi rows ; 0 pad]
+  // exchange slots: [4 n-tile slots][32 lanes] at the start of each warp's region
   const uint32_t sbase = smem_u32(T);
   const int ncols = n_R + n_C;
   const int nt2 = (ncols + 15) / 16;                    // pairs of 8-wide Gram n-tiles
   const long long fsz = (long long)n_C * ncols;
   const int g8 = lane >> 2, t4 = lane & 3;
   const int f0 = hf * (D / 2);                          // this warp's first feature
-  // A operand of the token LCB (16 x 16 tokens): rows 0..o_C-1 hold P_CC, row 8 the query
-  // generator's one-token weights, every other entry zero.  Constant for the whole kernel.
+  // A operand of the token LCB (16 x 16 tokens): rows 0..o_C-1 hold P_CC and rows 8..15 each the
+  // query generator's one-token weights, every other entry zero.  Constant for the whole kernel.
+  // The eight equal rows give every lane the query token for its n-tile g8, so the warp writes
+  // its 64 features of t^C with one 128-byte store per half (hi, lo).
   uint32_t pa[4];
   {
     auto A = [&](int row, int k) -> float {
       if (k >= n_C) return 0.f;
       if (row < o_C && row < 8) return sP[row * n_C + k];
-      if (row == 8) return sQ[k];
+      if (row >= 8) return sQ[k];
       return 0.f;
     };
     pa[0] = pack_bf16x2(A(g8, 2 * t4), A(g8, 2 * t4 + 1));
@@ -247,11 +281,12 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
     pa[2] = pack_bf16x2(A(g8, 2 * t4 + 8), A(g8, 2 * t4 + 9));
     pa[3] = pack_bf16x2(A(g8 + 8, 2 * t4 + 8), A(g8 + 8, 2 * t4 + 9));
   }
-  // Z^L row g8 and Z^Q (lanes with g8 == 0) of the current request for this warp's features, in
-  // the C-fragment layout: n-tile nt, columns f0 + nt*8 + 2*t4 and +1
-  float zl[D / 16][2], zq[D / 16][2];
+  // Z^L row g8 of the current request for this warp's features, in the C-fragment layout (n-tile
+  // nt, columns f0 + nt*8 + 2*t4 and +1), and the Z^Q pair at columns f0 + g8*8 + 2*t4 and +1
+  float zl[D / 16][2];
+  float2 zq = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int nt = 0; nt < D / 16; ++nt) zl[nt][0] = zl[nt][1] = zq[nt][0] = zq[nt][1] = 0.f;
+  for (int nt = 0; nt < D / 16; ++nt) zl[nt][0] = zl[nt][1] = 0.f;
   int staged = -1;
   if (hf == 0) zero_rows(T + (n_R + n_C) * pitch, pitch, trows - (n_R + n_C), D);
   for (int i = pr; i < n; i += FC_PAIRS) {
@@ -295,16 +330,16 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
           const float4 v = reinterpret_cast<const float4*>(ec + t * D)[lane];
           const uint32_t h01 = pack_bf16x2(v.x, v.y), h23 = pack_bf16x2(v.z, v.w);
           *reinterpret_cast<uint2*>(T + (n_R + t) * pitch + lane * 8) = make_uint2(h01, h23);
-          *reinterpret_cast<uint2*>(TL + t * pitch + lane * 8) =
+          *reinterpret_cast<uint2*>(TL + (lane >> 4) * FC_HALF + t * FC_LO_PITCH + (lane & 15) * 8) =
               make_uint2(pack_bf16x2(v.x - bf16_lo(h01), v.y - bf16_hi(h01)),
                          pack_bf16x2(v.z - bf16_lo(h23), v.w - bf16_hi(h23)));
         } else {
           *reinterpret_cast<uint2*>(T + (n_R + t) * pitch + lane * 8) = reinterpret_cast<const uint2*>(ec + t * D)[lane];
         }
       } else if constexpr (sizeof(TIN) == 4) {
-        // padding token rows of the lo tile meet zero LCB weights but must be finite: the exchange
-        // buffer of the previous candidate overwrote them
-        *reinterpret_cast<uint2*>(TL + t * pitch + lane * 8) = make_uint2(0, 0);
+        // padding token rows of the lo tile meet zero LCB weights but must be finite: the staged
+        // L^C and the exchange of the previous candidate overwrote them
+        *reinterpret_cast<uint2*>(TL + (lane >> 4) * FC_HALF + t * FC_LO_PITCH + (lane & 15) * 8) = make_uint2(0, 0);
       }
     }
     const int r = stage_r[st];
@@ -328,12 +363,8 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
           zl[nt][0] = z.x;
           zl[nt][1] = z.y;
         }
-        if (tC != nullptr && g8 == 0) {
-          const float2 z = __ldg(reinterpret_cast<const float2*>(ZQ + (long long)r * D + f0 + nt * 8 + 2 * t4));
-          zq[nt][0] = z.x;
-          zq[nt][1] = z.y;
-        }
       }
+      if (tC != nullptr) zq = __ldg(reinterpret_cast<const float2*>(ZQ + (long long)r * D + f0 + g8 * 8 + 2 * t4));
       staged = r;
     }
     pair_sync(bar_id);   // the tile is complete
@@ -350,28 +381,53 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
         mma_bf16_16816(acc[2 * p], pa, b[0], b[1]);
         mma_bf16_16816(acc[2 * p + 1], pa, b[2], b[3]);
         if constexpr (sizeof(TIN) == 4) {
-          load_b_frag_kmajor_x2(smem_u32(TL), pitch, 0, f0 + p * 16, b);
+          load_b_frag_kmajor_x2(smem_u32(TLh), FC_LO_PITCH, 0, p * 16, b);
           mma_bf16_16816(acc[2 * p], pa, b[0], b[1]);
           mma_bf16_16816(acc[2 * p + 1], pa, b[2], b[3]);
         }
       }
-      // L^C = Z^L + P_CC E^C (fp32), row g8 of every n-tile
-      if (g8 < o_C) {
+      // L^C = Z^L + P_CC E^C (fp32), row g8 of every n-tile.  With the TMA path, the warp's 64
+      // columns go to its region as two boxes of o_C rows x 32 floats in the 128-byte swizzle (the
+      // 16-byte unit u of row g8 at u ^ g8), which the stores of one instruction meet without bank
+      // conflicts, and one lane hands the boxes to the tensor-store engine.  The region's lo rows
+      // were this warp's alone, and its LCB products above have consumed them.
+      if (l_tma) {
+        if (g8 < o_C) {
+          const uint32_t sl = smem_u32(TLh) + (g8 << 7) + ((t4 & 1) << 3);
+          const uint32_t x = (uint32_t)((t4 >> 1) ^ g8);
+#pragma unroll
+          for (int nt = 0; nt < D / 16; ++nt)
+            st_shared_f32x2(sl + ((nt >> 2) << 10) + ((x ^ ((nt & 3) << 1)) << 4), acc[nt][0] + zl[nt][0],
+                            acc[nt][1] + zl[nt][1]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&mapL, TLh, f0, (int32_t)(c * o_C));
+          tma_store_2d(&mapL, TLh + 1024, f0 + 32, (int32_t)(c * o_C));
+          bulk_commit_group();
+        }
+      } else if (g8 < o_C) {
         float* lp = L_C + (c * o_C + g8) * (long long)D + f0 + 2 * t4;
 #pragma unroll
         for (int nt = 0; nt < D / 16; ++nt)
           *reinterpret_cast<float2*>(lp + nt * 8) = make_float2(acc[nt][0] + zl[nt][0], acc[nt][1] + zl[nt][1]);
       }
-      // t^C = Z^Q + p_CC E^C as a bf16 hi/lo pair (row 8 of the fragment: lanes with g8 == 0)
-      if (tC != nullptr && g8 == 0) {
-        __nv_bfloat16* tp = tC + c * 2LL * D + f0 + 2 * t4;
+      // t^C = Z^Q + p_CC E^C as a bf16 hi/lo pair: fragment row 8 + g8 holds it for every g8, and
+      // lane (g8, t4) writes n-tile g8's columns 2*t4 and +1
+      if (tC != nullptr) {
+        float a0 = acc[0][2], a1 = acc[0][3];
 #pragma unroll
-        for (int nt = 0; nt < D / 16; ++nt) {
-          const float v0 = acc[nt][2] + zq[nt][0], v1 = acc[nt][3] + zq[nt][1];
-          const uint32_t h = pack_bf16x2(v0, v1);
-          *reinterpret_cast<uint32_t*>(tp + nt * 8) = h;
-          *reinterpret_cast<uint32_t*>(tp + D + nt * 8) = pack_bf16x2(v0 - bf16_lo(h), v1 - bf16_hi(h));
-        }
+        for (int nt = 1; nt < D / 16; ++nt)
+          if (g8 == nt) {
+            a0 = acc[nt][2];
+            a1 = acc[nt][3];
+          }
+        const float v0 = a0 + zq.x, v1 = a1 + zq.y;
+        const uint32_t h = pack_bf16x2(v0, v1);
+        __nv_bfloat16* tp = tC + c * 2LL * D + f0 + g8 * 8 + 2 * t4;
+        *reinterpret_cast<uint32_t*>(tp) = h;
+        *reinterpret_cast<uint32_t*>(tp + D) = pack_bf16x2(v0 - bf16_lo(h), v1 - bf16_hi(h));
       }
     }
     // F^C = E^C [E^R ; E^C]^T: this warp's k-half for every n-tile, then the pair exchange; warp hf
@@ -393,15 +449,20 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
         }
       }
     }
-    if constexpr (sizeof(TIN) == 4) pair_sync(bar_id);   // both warps are done reading the lo rows
+    // the exchange slot is this warp's region: the tensor store must have read the staged L^C
+    if (l_tma) {
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
+    }
 #pragma unroll
     for (int q = 0; q < 8; ++q)
-      if (q < 2 * nt2 && (q & 1) != hf) xb[(hf * 4 + (q >> 1)) * 32 + lane] = make_float4(acc[q][0], acc[q][1], acc[q][2], acc[q][3]);
+      if (q < 2 * nt2 && (q & 1) != hf)
+        st_shared_f32x4(smem_u32(TLh) + (((q >> 1) * 32 + lane) << 4), acc[q][0], acc[q][1], acc[q][2], acc[q][3]);
     pair_sync(bar_id);
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       if (q < 2 * nt2 && (q & 1) == hf && q * 8 < ncols) {
-        const float4 o = xb[((1 - hf) * 4 + (q >> 1)) * 32 + lane];
+        const float4 o = ld_shared_f32x4(smem_u32(TL) + (1 - hf) * FC_HALF + (((q >> 1) * 32 + lane) << 4));
         acc[q][0] += o.x;
         acc[q][1] += o.y;
         acc[q][2] += o.z;
@@ -410,6 +471,8 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
       }
     }
   }
+  // the CTA's last tensor stores complete before it exits
+  if (l_tma && lane == 0) bulk_wait_all();
 }
 
 
@@ -661,6 +724,18 @@ rocs_status lcb_launch(rocs_context* ctx, const TIN* E_R, long long ld_ER, const
   return ROCS_OK;
 }
 
+// Dynamic shared memory of the fused pass: the ring, the pair blocks and 1 KB to align them.  The
+// cap leaves room under the 227 KB per block for the kernel's static arrays.
+constexpr size_t FC_SMEM_MAX = 223 * 1024;
+size_t fused_smem_bytes(int n_R, int n_C, int in_f32) {
+  const int D = 128, pitch = D * 2 + 16;
+  return 1024 + (size_t)FC_STAGES * NC_MAX * D * (in_f32 ? 4 : 2) + (size_t)FC_PAIRS * fc_pair_bytes(fm_trows(n_R, n_C), pitch);
+}
+
+typedef CUresult (*EncodeTiledFnFm)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
 template <typename TIN>
 rocs_status fused_launch(rocs_context* ctx, const TIN* E_R, const TIN* E_C, const int32_t* req_idx, int B_R,
                          long long B_C, int n_R, int n_C, void* F_C, const void* P_CC, int o_C, const float* ZL,
@@ -668,31 +743,51 @@ rocs_status fused_launch(rocs_context* ctx, const TIN* E_R, const TIN* E_C, cons
   const int D = 128;
   const int pitch = D * 2 + 16;
   const int trows = fm_trows(n_R, n_C);
-  const size_t smem = (size_t)FC_STAGES * NC_MAX * D * sizeof(TIN) + (size_t)FC_PAIRS * (trows + NC_MAX) * pitch;
-  if (n_C > NC_MAX || o_C > LCB_OMAX_F || smem > 220 * 1024) {
-    set_error("fused candidate pass: unsupported n_C=%d o_C=%d", n_C, o_C);
+  const size_t smem = fused_smem_bytes(n_R, n_C, sizeof(TIN) == 4);
+  if (n_C > NC_MAX || o_C < 1 || o_C > LCB_OMAX_F || smem > FC_SMEM_MAX) {
+    set_error("fused candidate pass: unsupported n_R=%d n_C=%d o_C=%d", n_R, n_C, o_C);
     return ROCS_ERR_UNSUPPORTED;
   }
   static bool attr[64] = {false};
   if (ctx->device < 64 && !attr[ctx->device]) {
     rocs_status st = cuda_check(cudaFuncSetAttribute(glm_cand_fused_kernel<TIN>,
-                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024),
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FC_SMEM_MAX),
                                 "cudaFuncSetAttribute(glm_cand_fused)");
     if (st != ROCS_OK) return st;
     attr[ctx->device] = true;
   }
   if (B_C == 0) return ROCS_OK;
+  // L^C [B_C * o_C, D] fp32 through TMA stores: boxes of o_C rows x 32 floats, 128-byte swizzle.
+  // A base address off the 16-byte grid takes the plain stores.
+  CUtensorMap mapL;
+  memset(&mapL, 0, sizeof(mapL));
+  int l_tma = 0;
+  if ((reinterpret_cast<uintptr_t>(L_C) & 15) == 0 && B_C * o_C < (1LL << 31)) {
+    EncodeTiledFnFm fn = reinterpret_cast<EncodeTiledFnFm>(ctx->encode_fn);
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)(B_C * o_C)};
+    cuuint64_t strides[1] = {(cuuint64_t)D * 4};
+    cuuint32_t box[2] = {32, (cuuint32_t)o_C};
+    cuuint32_t estr[2] = {1, 1};
+    l_tma = fn(&mapL, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, L_C, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  }
   // one CTA per SM, each over a contiguous candidate range (runs of a request stay together)
   const long long blocks = B_C < ctx->num_sms ? B_C : ctx->num_sms;
   const long long per_block = (B_C + blocks - 1) / blocks;
   LaunchTimer lt_("glm_cand_fused", s);
   glm_cand_fused_kernel<TIN><<<(unsigned)blocks, 32 * (1 + FC_CONSUMERS), smem, s>>>(
       E_R, E_C, req_idx, B_R, B_C, per_block, n_R, n_C, trows, pitch, (__nv_bfloat16*)F_C,
-      (const __nv_bfloat16*)P_CC, o_C, ZL, L_C, (const __nv_bfloat16*)q_pCC, ZQ, (__nv_bfloat16*)tC, ctx->d_status);
+      (const __nv_bfloat16*)P_CC, o_C, ZL, L_C, (const __nv_bfloat16*)q_pCC, ZQ, (__nv_bfloat16*)tC, mapL, l_tma,
+      ctx->d_status);
   return cuda_check(cudaGetLastError(), "glm_cand_fused_kernel");
 }
 
 }  // namespace
+
+bool glm_cand_fused_fits(int D, int n_R, int n_C, int o_C, int in_f32) {
+  return D == 128 && n_C <= NC_MAX && o_C >= 1 && o_C <= LCB_OMAX_F && fused_smem_bytes(n_R, n_C, in_f32) <= FC_SMEM_MAX;
+}
 
 rocs_status launch_glm_cand_fused(rocs_context* ctx, const void* E_R, const void* E_C, const int32_t* req_idx,
                                   int B_R, long long B_C, int n_R, int n_C, int in_f32, void* F_C, const void* P_CC,

@@ -197,6 +197,9 @@ rocs_status launch_fm(rocs_context* ctx, const void* E_R, const void* E_C, const
 // One pass over the candidates' embeddings (D = 128): masked-FM products as bf16 hi/lo pairs, the
 // token LCB output L_C (fp32, o_C tokens, Z^L from the request side) and, if tC is non-NULL, the
 // one-token query-generator LCB (hi/lo pairs, Z^Q from the request side).
+// Whether the fused pass takes this layer (D 128, n_C <= 16, 1 <= o_C <= 8, and its shared
+// memory, which grows with n_R and with fp32 embeddings, fits).
+bool glm_cand_fused_fits(int D, int n_R, int n_C, int o_C, int in_f32);
 rocs_status launch_glm_cand_fused(rocs_context* ctx, const void* E_R, const void* E_C, const int32_t* req_idx,
                                   int B_R, long long B_C, int n_R, int n_C, int in_f32, void* F_C, const void* P_CC,
                                   int o_C, const float* ZL, float* L_C, const void* q_pCC, const float* ZQ, void* tC,
