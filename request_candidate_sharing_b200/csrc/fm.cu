@@ -264,25 +264,30 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
   const long long fsz = (long long)n_C * ncols;
   const int g8 = lane >> 2, t4 = lane & 3;
   const int f0 = hf * (D / 2);                          // this warp's first feature
-  // A operand of the token LCB (16 x 16 tokens): rows 0..o_C-1 hold P_CC and rows 8..15 each the
-  // query generator's one-token weights, every other entry zero.  Constant for the whole kernel.
-  // The eight equal rows give every lane the query token for its n-tile g8, so the warp writes
-  // its 64 features of t^C with one 128-byte store per half (hi, lo).
+  // Fragment row g8 (< 8) carries LCB output o(g8) = 2 (g8 mod 4) + g8 / 4: the first half-warp
+  // holds the even outputs, the second the odd ones, so the swizzled staging of L^C below puts
+  // each half-warp's 16 stores on 16 different 8-byte bank pairs.
+  const int og = ((g8 & 3) << 1) | (g8 >> 2);
+  // A operand of the token LCB (16 x 16 tokens): row g8 < 8 holds P_CC row o(g8) (zero beyond
+  // o_C) and rows 8..15 each the query generator's one-token weights.  Constant for the whole
+  // kernel.  The eight equal rows give every lane the query token for its n-tile g8, so the warp
+  // writes its 64 features of t^C with one 128-byte store per half (hi, lo).
   uint32_t pa[4];
   {
     auto A = [&](int row, int k) -> float {
       if (k >= n_C) return 0.f;
-      if (row < o_C && row < 8) return sP[row * n_C + k];
       if (row >= 8) return sQ[k];
-      return 0.f;
+      const int o = ((row & 3) << 1) | (row >> 2);
+      return o < o_C ? sP[o * n_C + k] : 0.f;
     };
     pa[0] = pack_bf16x2(A(g8, 2 * t4), A(g8, 2 * t4 + 1));
     pa[1] = pack_bf16x2(A(g8 + 8, 2 * t4), A(g8 + 8, 2 * t4 + 1));
     pa[2] = pack_bf16x2(A(g8, 2 * t4 + 8), A(g8, 2 * t4 + 9));
     pa[3] = pack_bf16x2(A(g8 + 8, 2 * t4 + 8), A(g8 + 8, 2 * t4 + 9));
   }
-  // Z^L row g8 of the current request for this warp's features, in the C-fragment layout (n-tile
-  // nt, columns f0 + nt*8 + 2*t4 and +1), and the Z^Q pair at columns f0 + g8*8 + 2*t4 and +1
+  // Z^L row o(g8) of the current request for this warp's features, in the C-fragment layout
+  // (n-tile nt, columns f0 + nt*8 + 2*t4 and +1), and the Z^Q pair at columns f0 + g8*8 + 2*t4
+  // and +1
   float zl[D / 16][2];
   float2 zq = make_float2(0.f, 0.f);
 #pragma unroll
@@ -358,8 +363,8 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
       }
 #pragma unroll
       for (int nt = 0; nt < D / 16; ++nt) {
-        if (g8 < o_C) {
-          const float2 z = __ldg(reinterpret_cast<const float2*>(ZL + ((long long)r * o_C + g8) * D + f0 + nt * 8 + 2 * t4));
+        if (og < o_C) {
+          const float2 z = __ldg(reinterpret_cast<const float2*>(ZL + ((long long)r * o_C + og) * D + f0 + nt * 8 + 2 * t4));
           zl[nt][0] = z.x;
           zl[nt][1] = z.y;
         }
@@ -386,15 +391,15 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
           mma_bf16_16816(acc[2 * p + 1], pa, b[2], b[3]);
         }
       }
-      // L^C = Z^L + P_CC E^C (fp32), row g8 of every n-tile.  With the TMA path, the warp's 64
-      // columns go to its region as two boxes of o_C rows x 32 floats in the 128-byte swizzle (the
-      // 16-byte unit u of row g8 at u ^ g8), which the stores of one instruction meet without bank
-      // conflicts, and one lane hands the boxes to the tensor-store engine.  The region's lo rows
-      // were this warp's alone, and its LCB products above have consumed them.
+      // L^C = Z^L + P_CC E^C (fp32): output o(g8) in fragment row g8 of every n-tile.  With the
+      // TMA path, the warp's 64 columns go to its region as two boxes of o_C rows x 32 floats in
+      // the 128-byte swizzle (the 16-byte unit u of row o at u ^ o), and one lane hands the boxes
+      // to the tensor-store engine.  The region's lo rows were this warp's alone, and its LCB
+      // products above have consumed them.
       if (l_tma) {
-        if (g8 < o_C) {
-          const uint32_t sl = smem_u32(TLh) + (g8 << 7) + ((t4 & 1) << 3);
-          const uint32_t x = (uint32_t)((t4 >> 1) ^ g8);
+        if (og < o_C) {
+          const uint32_t sl = smem_u32(TLh) + (og << 7) + ((t4 & 1) << 3);
+          const uint32_t x = (uint32_t)((t4 >> 1) ^ og);
 #pragma unroll
           for (int nt = 0; nt < D / 16; ++nt)
             st_shared_f32x2(sl + ((nt >> 2) << 10) + ((x ^ ((nt & 3) << 1)) << 4), acc[nt][0] + zl[nt][0],
@@ -407,8 +412,8 @@ __global__ void __launch_bounds__(32 * (1 + FC_CONSUMERS), 1) glm_cand_fused_ker
           tma_store_2d(&mapL, TLh + 1024, f0 + 32, (int32_t)(c * o_C));
           bulk_commit_group();
         }
-      } else if (g8 < o_C) {
-        float* lp = L_C + (c * o_C + g8) * (long long)D + f0 + 2 * t4;
+      } else if (og < o_C) {
+        float* lp = L_C + (c * o_C + og) * (long long)D + f0 + 2 * t4;
 #pragma unroll
         for (int nt = 0; nt < D / 16; ++nt)
           *reinterpret_cast<float2*>(lp + nt * 8) = make_float2(acc[nt][0] + zl[nt][0], acc[nt][1] + zl[nt][1]);
