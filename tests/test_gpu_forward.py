@@ -82,6 +82,21 @@ def test_forward_glm_stack_narrow_candidates(R):
     check_bf16(host(out["E_C"][:case.B_C]), ref["E_C"], what="E_C")
 
 
+def test_forward_glm_stack_wide_requests(R):
+    """48 request and 16 candidate embeddings (n_R + n_C = 64, the widest group pair): the fused
+    candidate pass takes layer 0 (bf16 embeddings), and its shared memory would not hold the pair
+    tiles next to a ring of fp32 stages, so the later layers take the two-kernel path (masked FM,
+    then token LCB).  Three layers: bf16, then two fp32 stream layers."""
+    g = synth.GLMShape(n_R=48, n_C=16, hidden=256, fm_out_R=24, lcb_out_R=24, fm_out_C=8, lcb_out_C=8, layers=3)
+    case = synth.ModelCase("cfg3", np.asarray([5, 0, 37, 120, 1], np.int32), 11, g, None, None)
+    x, W = synth.model_inputs(case), synth.model_weights(case)
+    out = run_forward(R, case, x, W)
+    _, m = O.segments(case.counts)
+    ref = O.forward_cfg3(case, x, W, m)
+    check_bf16(host(out["E_R"]), ref["E_R"], what="E_R")
+    check_bf16(host(out["E_C"][:case.B_C]), ref["E_C"], what="E_C")
+
+
 @pytest.mark.parametrize("cfg", ["cfg3", "cfg4", "cfg5"])
 def test_forward_without_candidates(R, cfg):
     """A batch whose requests have no candidates at all (B_C = 0): the request-side results still
