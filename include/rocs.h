@@ -363,6 +363,12 @@ rocs_status rocs_dca_encode(rocs_handle_t handle, const rocs_dca_desc* desc, con
  * stream, MLP and LCB outputs, attention outputs) stay fp32, so rounding of intermediates does
  * not accumulate across the stacked layers.  Split operands need widths that are multiples of
  * 64 (n_R^2, n_C(n_R+n_C), hidden, q_dim, d).
+ * GLM limits (else ROCS_ERR_INVALID_ARG): n_R + n_C <= 64; D a multiple of 16, at most 256;
+ * n * D <= 8192 per group; fm_out + lcb_out = n per group (the residual); 1 <= lcb_out_C <= 8.
+ * With D = 128 and n_C <= 16 the candidate FM, token LCB and query token of a layer run as one
+ * pass over the embeddings where its shared memory fits (always for bf16 layer-0 inputs; for the
+ * fp32 stream of later layers while n_R + 16 <= 48), and as separate kernels otherwise, with the
+ * same results.
  * Graph replay (a11): the handle records each distinct call (the bytes of the descriptor, the
  * weight/input/output pointer structs and the workspace pointer and size).  The first call
  * with a given record launches the kernels directly; the second captures the same launch
