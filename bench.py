@@ -277,18 +277,26 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.p.kill()
         self.f.flush()
-        rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
+        text = open(self.f.name).read()
         os.unlink(self.f.name)
-        if not rows:
-            return None
-        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
-        mx = float(rows[0][2]) if rows[0][2].strip().replace(".", "").isdigit() else None
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 5 + i and "Active" in r[5 + i]
-                          and "Not" not in r[5 + i]})
-        under = sorted(sm)[len(sm) // 2:] if sm else []
-        return {"sm_mhz": statistics.median(under) if under else None, "sm_max_mhz": mx, "reasons": reasons,
-                "samples": len(rows)}
+        return summarize_clocks(text)
+
+
+def summarize_clocks(text: str):
+    """The clock record of a timed region from nvidia-smi's CSV rows (ClockSampler.FIELDS, no
+    header, no units): the median SM clock of the busier half of the samples (the GPU under
+    load), the maximum SM clock, and the throttle reasons that were active in any sample."""
+    rows = [r.split(",") for r in text.strip().splitlines() if r.strip()]
+    if not rows:
+        return None
+    sm = [float(r[1]) for r in rows if len(r) > 1 and r[1].strip().replace(".", "").isdigit()]
+    mx = float(rows[0][2]) if len(rows[0]) > 2 and rows[0][2].strip().replace(".", "").isdigit() else None
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = sorted({names[i] for r in rows for i in range(4) if len(r) > 5 + i and "Active" in r[5 + i]
+                      and "Not" not in r[5 + i]})
+    under = sorted(sm)[len(sm) // 2:] if sm else []
+    return {"sm_mhz": statistics.median(under) if under else None, "sm_max_mhz": mx, "reasons": reasons,
+            "samples": len(rows)}
 
 
 # ---------------------------------------------------------------------------------------------
