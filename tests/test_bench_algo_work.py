@@ -49,3 +49,25 @@ def test_gemm_flops():
 
 def test_unknown_site_has_no_roofline():
     assert work("fwd:iota") is None
+
+
+def test_roofline_entries_from_launch_times():
+    """The per-kernel entries of the bench line: achieved = work per launch / mean launch time,
+    against the measured peaks; the split-A GEMMs also report the executed fraction (twice the
+    flops).  Launch times as one bench line reported them."""
+    case = bench.make_case("rocs_forward_e2e", 0, 0)
+    peaks = dict(hbm=6540.0, tensor=1614.0, tensor_sustained=1366.0, sm_mhz=1965.0, source="measured",
+                 exp2_gps=5593.6)
+    e = bench.roofline_entry(case, "glm.mlp2.ikbo:gemm_tc", 30, 30 * 0.8231, peaks, sustained=True)
+    flops = 2.0 * 242_464 * 1024 * 1024 + 2.0 * 512 * 3072 * 1024
+    assert e["unit"] == "TFLOP/s" and e["peak"] == 1366.0
+    assert abs(e["achieved"] - flops / 0.8231e-3 / 1e12) < 1e-3
+    assert abs(e["frac"] - flops / 0.8231e-3 / 1e12 / 1366.0) < 1e-4
+    assert abs(e["executed_frac"] - 2 * e["frac"]) < 2e-4
+    e = bench.roofline_entry(case, "enc.attn:attn_tc", 30, 30 * 1.7256, peaks, sustained=True)
+    assert e["unit"] == "Gexp2/s" and e["peak"] == 5593.6
+    assert abs(e["frac"] - 8 * 512 * 1024 * 1024 / 1.7256e-3 / 1e9 / 5593.6) < 1e-4
+    e = bench.roofline_entry(case, "glm.lnC:layernorm", 30, 30 * 0.9548, peaks, sustained=True)
+    assert e["unit"] == "GB/s" and e["peak"] == 6540.0 and "executed_frac" not in e
+    assert abs(e["frac"] - 242_464 * 24_576 / 0.9548e-3 / 1e9 / 6540.0) < 1e-4
+    assert bench.roofline_entry(case, "glm.lnC:layernorm", 0, 0.0, peaks, sustained=True) is None
