@@ -54,7 +54,7 @@ constexpr int kAtGroups64 = 2, kAtKeys64 = 128;
 
 struct AttnTcParams {
   CUtensorMap tmQ;   // queries [rows, cols] bf16: box {d_h, 128}
-  CUtensorMap tmK;   // keys    [B_R * L, H * d_h]: box {d_h, 128}
+  CUtensorMap tmK;   // keys    [B_R * L, H * d_h]: box {d_h, TK}
   CUtensorMap tmV;   // values  same layout
   const int32_t* offsets;
   long long rows;
