@@ -154,9 +154,14 @@ def algo_work(case, label: str):
             "enc.kv:gemm_tc": ("tensor", 2.0 * rows_h * d * d * (2 if (d == 256 and H <= 8 and (d // H) % 16 == 0) else 4)),
             "enc.wo:gemm_tc": ("tensor", 2.0 * rows_h * d * d),
             "enc.ln:layernorm": ("hbm", rows_h * d * 2 * 3.0),
-            # query generator, two IKBO linears q_dim -> d -> d (fused launches: request + candidate)
+            # query generator, two IKBO linears q_dim -> d -> d: one fused launch (request and
+            # candidate tiles) or a request launch ([Y^R | Z], 2d outputs) and a candidate launch
             "qgen.mlp1.ikbo:gemm_tc": ("tensor", 2.0 * (B_C + 2 * B_R) * d * a.q_dim),
             "qgen.mlp2.ikbo:gemm_tc": ("tensor", 2.0 * (B_C + 2 * B_R) * d * d),
+            "qgen.mlp1.req:gemm_tc": ("tensor", 2.0 * 2 * B_R * d * a.q_dim),
+            "qgen.mlp1.cand:gemm_tc": ("tensor", 2.0 * B_C * d * a.q_dim),
+            "qgen.mlp2.req:gemm_tc": ("tensor", 2.0 * 2 * B_R * d * d),
+            "qgen.mlp2.cand:gemm_tc": ("tensor", 2.0 * B_C * d * d),
             # the request query's attention with its projections absorbed reads the final
             # encoder output S once (bf16); weights and queries are L2-resident and negligible
             "xattn.req:attn_req": ("hbm", rows_h * d * 2),
@@ -204,6 +209,29 @@ def load_peaks():
                     tensor_sustained=float(j["bf16_tflops_sustained"]), sm_mhz=float(j.get("sm_max_mhz", 1965.0)),
                     source="measured")
     return dict(hbm=6650.0, tensor=1590.0, tensor_sustained=1400.0, sm_mhz=1965.0, source="fallback")
+
+
+def forward_roofline(case, report, steps: int, ms_per_step: float, peaks):
+    """The whole forward against its roofline: the sum over the per-kernel report's sites of
+    (algorithmic work per launch / the site's roof) x launches per step, divided by the measured
+    step time.  Roofs: burst bf16 tensor, HBM copy bandwidth, and the exponential rate measured
+    in the same run.  Sites with no algorithmic-work entry (small request-side kernels,
+    bookkeeping) add nothing to the ideal time; their measured time is reported as uncovered."""
+    roof = {"tensor": peaks["tensor"] * 1e12, "hbm": peaks["hbm"] * 1e9,
+            "alu": (peaks.get("exp2_gps") or 16 / ATTN_MUFU_SHARE * 148 * peaks["sm_mhz"] * 1e-3) * 1e9}
+    ideal = covered = uncovered = 0.0
+    for name, (n, t) in report.items():
+        w = algo_work(case, name)
+        if w is None or n == 0:
+            uncovered += t / steps
+            continue
+        bound, amount = w
+        ideal += amount / roof[bound] * 1e3 * n / steps
+        covered += t / steps
+    return {"ideal_ms": round(ideal, 3), "measured_ms": round(ms_per_step, 4), "frac": round(ideal / ms_per_step, 4),
+            "covered_kernel_ms": round(covered, 3), "uncovered_kernel_ms": round(uncovered, 3),
+            "roofs": (f"bf16 {peaks['tensor']:.0f} TFLOP/s (burst), HBM {peaks['hbm']:.0f} GB/s, "
+                      f"exp2 {roof['alu'] / 1e9:.0f} G/s")}
 
 
 # GEMM sites whose A operand is a bf16 hi/lo pair (the GLM MLPs and the DCA query generator): the
@@ -649,6 +677,7 @@ def run_librocs(args, rank, world, local):
                        "e2e_host_buffers": (f"pinned, allocated from the GPU's NUMA node ({len(local)} local CPUs)"
                                             if local else "pinned (the GPU's NUMA node is unknown)")},
             "roofline": top,
+            "forward_roofline": forward_roofline(case, report, args.steps, ms_max / args.steps, peaks),
             "step_ms": {"median": round(statistics.median(step_ms), 4),
                         "p90": round(sorted(step_ms)[min(len(step_ms) - 1, int(math.ceil(0.9 * len(step_ms))) - 1)], 4),
                         "n": len(step_ms), "rank": 0},

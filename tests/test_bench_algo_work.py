@@ -71,3 +71,29 @@ def test_roofline_entries_from_launch_times():
     assert e["unit"] == "GB/s" and e["peak"] == 6540.0 and "executed_frac" not in e
     assert abs(e["frac"] - 242_464 * 24_576 / 0.9548e-3 / 1e9 / 6540.0) < 1e-4
     assert bench.roofline_entry(case, "glm.lnC:layernorm", 0, 0.0, peaks, sustained=True) is None
+
+
+def test_forward_roofline_sums_sites_against_their_roofs():
+    """The whole-forward roofline: per step, each site's launches times its work over its roof
+    (burst bf16, HBM, the measured exponential rate), summed and divided by the step time.
+    Sites with no work entry count as uncovered time."""
+    case = bench.make_case("rocs_forward_e2e", 0, 0)
+    peaks = dict(hbm=6540.0, tensor=1614.0, tensor_sustained=1366.0, sm_mhz=1965.0, source="measured",
+                 exp2_gps=5600.0)
+    steps = 2
+    report = {"enc.attn:attn_tc": (3 * steps, 5.2 * steps),        # 3 launches per step
+              "glm.lnC:layernorm": (3 * steps, 2.9 * steps),
+              "glm.mlp2.ikbo:gemm_tc": (3 * steps, 2.5 * steps),
+              "qgen.mlp1.cand:gemm_tc": (3 * steps, 0.4 * steps),
+              "fwd:iota": (2 * steps, 0.1 * steps),
+              "dropped": (0, 0.0)}
+    r = bench.forward_roofline(case, report, steps, 20.0, peaks)
+    ideal_ms = 1e3 * 3 * (8 * 512 * 1024 * 1024 / 5600e9
+                          + 242_464 * 24_576 / 6540e9
+                          + (2.0 * 242_464 * 1024 * 1024 + 2.0 * 512 * 3072 * 1024) / 1614e12
+                          + 2.0 * 242_464 * 256 * 128 / 1614e12)
+    assert abs(r["ideal_ms"] - ideal_ms) < 1e-3
+    assert abs(r["frac"] - ideal_ms / 20.0) < 1e-4
+    assert abs(r["covered_kernel_ms"] - (5.2 + 2.9 + 2.5 + 0.4)) < 1e-6
+    assert abs(r["uncovered_kernel_ms"] - 0.1) < 1e-6
+    assert r["measured_ms"] == 20.0
