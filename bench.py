@@ -554,7 +554,7 @@ def run_librocs(args, rank, world, local):
     st = R.rocs_get_device_status(sh)
     if st != 0:
         raise RuntimeError(f"device status {rocs.STATUS_NAMES.get(st, st)} in the timed region")
-    # the exponential ceiling of the attention kernels, measured on this GPU now (B-16 probe)
+    # the exponential ceiling of the attention kernels, measured on this GPU now (rocs_probe_exp2_rate)
     exp2_probe = {f"n_poly={n}": round(R.rocs_probe_exp2_rate(n, sh) / 1e9, 1) for n in (0, 3, 8)}
     _, total_c, ms_max = shard_totals(args.workload, rank, world, args.requests, ms, args.shard)
     cands = total_c * args.steps
